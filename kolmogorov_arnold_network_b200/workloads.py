@@ -1,0 +1,139 @@
+"""Named synthetic workloads and their seeded input generators.
+
+This module holds no arithmetic of the KAN layer: only shapes, grid
+parameters and the random draws of the inputs.  The tests, the oracle checks
+and the benchmark all take their inputs from here, so that the CUDA path and
+the fp64 oracle see the same values.
+
+Recipe (every tensor): a CPU ``torch.Generator`` seeded with
+``1000 * family + tensor_id`` (tensor ids: x=0, coef=1, w_base=2, dY=3,
+second-layer coef=4), drawn in fp32, then rounded once to the operand dtype.
+Distributions: ``N(0, s)`` takes ``s`` as the standard deviation, except the
+base weights, drawn with variance ``1/in`` (standard deviation ``1/sqrt(in)``).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Layer:
+    """One KAN layer's hyper-parameters (cubic B-splines on a uniform grid)."""
+    inp: int
+    out: int
+    G: int
+    lo: float
+    hi: float
+    base: bool = False
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    family: int                  # seed family
+    batch: int
+    layers: tuple                # tuple[Layer, ...]; >1 only for the FFN block
+    dtype: str                   # "f32" or "bf16" (operand dtype; accumulation is fp32)
+    x_dist: tuple                # ("uniform", a, b) or ("normal", std)
+    coef_std: float
+    mode: str = "fwd+bwd"        # "fwd" or "fwd+bwd"
+    note: str = ""
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def edges(self) -> int:
+        """Edge evaluations per step: batch * in * out summed over layers."""
+        return sum(self.batch * L.inp * L.out for L in self.layers)
+
+
+def _grid_sweep():
+    out = {}
+    for G in (8, 20, 50):
+        for dt in ("f32", "bf16"):
+            for mode in ("fwd", "fwd+bwd"):
+                nm = f"sweep512_g{G}_{dt}_{'fwd' if mode == 'fwd' else 'fwdbwd'}"
+                out[nm] = Workload(nm, 4, 65536, (Layer(512, 512, G, -1.0, 1.0),), dt, ("uniform", -1.0, 1.0), 0.1,
+                                   mode=mode, note="grid sweep 512x512, batch 65536")
+    return out
+
+
+WORKLOADS = {
+    "layer8x4": Workload("layer8x4", 1, 32, (Layer(8, 4, 8, -1.0, 1.0),), "f32", ("uniform", -1.0, 1.0), 0.1,
+                         note="KANLayer(8,4) on a [32,8] batch, G=8 on [-1,1]"),
+    "layer784x64_silu": Workload("layer784x64_silu", 2, 4096, (Layer(784, 64, 8, -1.0, 1.0, base=True),), "f32",
+                                 ("uniform", -1.0, 1.0), 0.1,
+                                 note="first layer of KANNetwork([784,64,10]) at batch 4096, SiLU base branch"),
+    "layer1024_g20_bf16": Workload("layer1024_g20_bf16", 3, 16384, (Layer(1024, 1024, 20, -1.0, 1.0),), "bf16",
+                                   ("uniform", -1.1, 1.1), 0.1,
+                                   note="1024x1024, G=20, inputs reach the extended knot intervals"),
+    **_grid_sweep(),
+    "ffn768_3072_bf16": Workload("ffn768_3072_bf16", 5, 8192,
+                                 (Layer(768, 3072, 5, -3.0, 3.0), Layer(3072, 768, 5, -3.0, 3.0)), "bf16",
+                                 ("normal", 1.0), 0.05, note="KAN FFN block 768->3072->768, 8192 tokens"),
+}
+
+#: the workload the benchmark times by default
+BENCH_DEFAULT = "layer784x64_silu"
+
+
+def _gen(family: int, tensor_id: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(1000 * family + tensor_id)
+    return g
+
+
+def draw_x(w: Workload, rows: int | None = None) -> torch.Tensor:
+    rows = w.batch if rows is None else rows
+    g = _gen(w.family, 0)
+    shape = (rows, w.layers[0].inp)
+    if w.x_dist[0] == "uniform":
+        a, b = w.x_dist[1], w.x_dist[2]
+        x = torch.rand(shape, generator=g, dtype=torch.float32) * (b - a) + a
+    else:
+        x = torch.randn(shape, generator=g, dtype=torch.float32) * w.x_dist[1]
+    return x.to(w.torch_dtype)
+
+
+def draw_coef(w: Workload, layer: int = 0) -> torch.Tensor:
+    L = w.layers[layer]
+    g = _gen(w.family, 1 if layer == 0 else 4)
+    c = torch.randn((L.out, L.inp, L.G + 3), generator=g, dtype=torch.float32) * w.coef_std
+    return c.to(w.torch_dtype)
+
+
+def draw_w_base(w: Workload, layer: int = 0):
+    L = w.layers[layer]
+    if not L.base:
+        return None
+    g = _gen(w.family, 2)
+    c = torch.randn((L.out, L.inp), generator=g, dtype=torch.float32) * (1.0 / L.inp) ** 0.5
+    return c.to(w.torch_dtype)
+
+
+def draw_dY(w: Workload, rows: int | None = None) -> torch.Tensor:
+    rows = w.batch if rows is None else rows
+    g = _gen(w.family, 3)
+    return torch.randn((rows, w.layers[-1].out), generator=g, dtype=torch.float32).to(w.torch_dtype)
+
+
+def draw_all(w: Workload, rows: int | None = None) -> dict:
+    """All inputs of a workload as CPU tensors in the operand dtype."""
+    d = {"x": draw_x(w, rows), "dY": draw_dY(w, rows)}
+    for li in range(len(w.layers)):
+        d[f"coef{li}"] = draw_coef(w, li)
+        d[f"w_base{li}"] = draw_w_base(w, li)
+    return d
+
+
+def custom(batch, inp, out, G, lo, hi, dtype="f32", base=False, x_range=None, coef_std=0.1, family=90):
+    """An ad-hoc single-layer workload (tests of ragged and edge shapes)."""
+    h = (hi - lo) / G
+    xr = x_range or (lo - 2 * h, hi + 2 * h)
+    return Workload(f"custom_{batch}x{inp}x{out}_g{G}_{dtype}", family, batch, (Layer(inp, out, G, lo, hi, base),),
+                    dtype, ("uniform", xr[0], xr[1]), coef_std)
