@@ -1,0 +1,146 @@
+/*
+ * kan_b200.h -- C ABI of libkan_b200.so: forward and backward pass of a
+ * B-spline Kolmogorov-Arnold (KAN) layer on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources):
+ *   y[b,j] = sum_i phi_ji(x[b,i])                  InKAN landing page, "What is a KAN?"
+ *   phi_ji(x) = sum_m coef[j,i,m] B_m(x)            cubic B-spline with local support
+ *                                                   (same page and section)
+ *             (+ w_base[j,i] silu(x) when has_base) optional SiLU base branch
+ *   B_m: uniform cubic B-splines on G intervals of [lo,hi], the grid extended
+ *   by 3 knots on each side, m = 0..G+2 ("predefined, bounded grids": UKAN
+ *   abstract, "Want to train KANS at scale? Now UKAN!").  Knots
+ *   t_k = lo + (k-3)(hi-lo)/G, k = 0..G+6; supp B_m = [t_m, t_{m+4}).
+ *   An input outside [t_0, t_{G+6}) (and any NaN or inf) has all B_m = 0.
+ *   Each input touches only 4 basis functions ("local 4-basis lookup":
+ *   InKAN landing page, "Why InKAN?"), which are evaluated in the stable
+ *   piecewise form with non-negative output (same page, "Numerically
+ *   Stable"); no Cox-de Boor recursion runs on the device.
+ *
+ * Gradients (backward):
+ *   dcoef[j,i,m]  = sum_b B_m(x[b,i]) dY[b,j]
+ *   dw_base[j,i]  = sum_b silu(x[b,i]) dY[b,j]
+ *   dx[b,i]       = sum_j dY[b,j] (sum_m coef[j,i,m] B'_m(x[b,i]) + w_base[j,i] silu'(x[b,i]))
+ *   Batch reductions are deterministic: fixed order, no atomic adds (the
+ *   FlashKAT abstract names atomic gradient accumulation as a bottleneck and
+ *   a source of rounding error).
+ *
+ * Layouts: every tensor is dense row-major (C order) in device memory.
+ *   x       [batch, in]          operand dtype
+ *   coef    [out, in, G+3]       operand dtype
+ *   w_base  [out, in]            operand dtype (only when has_base)
+ *   y       [batch, out]         operand dtype
+ *   dY      [batch, out]         operand dtype
+ *   dx      [batch, in]          operand dtype
+ *   dcoef   [out, in, G+3]       float32, overwritten
+ *   dw_base [out, in]            float32, overwritten
+ * The operand dtype is float32 or bfloat16; accumulation is always fp32.
+ * Pointers must be 16-byte aligned.
+ *
+ * Ownership: the caller owns every buffer, the workspace included.  The
+ * library keeps no allocation across calls; it allocates nothing itself.
+ *
+ * Streams: every compute call is asynchronous on `stream` (a cudaStream_t
+ * passed as void*, NULL = legacy default stream).  Errors found on the host
+ * are returned before anything is launched.  A device-side wait that gives up
+ * (every wait inside a kernel has a time limit of about one second) records
+ * KAN_ERR_TIMEOUT in a device status word, which kan_sync_status() reports.
+ *
+ * Threading: calls may come from several host threads; kan_last_error() is
+ * per thread.
+ */
+#ifndef KAN_B200_H
+#define KAN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KAN_API __attribute__((visibility("default")))
+#else
+#define KAN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KAN_ABI_VERSION 1
+
+typedef enum { KAN_F32 = 0, KAN_BF16 = 1 } kan_dtype;
+
+typedef enum {
+    KAN_OK = 0,
+    KAN_ERR_INVALID_ARG = 1,   /* a null pointer, a non-positive size, G < 1, hi <= lo, ... */
+    KAN_ERR_UNSUPPORTED = 2,   /* valid but not handled: misaligned pointer, G > 250, forced path not possible */
+    KAN_ERR_WORKSPACE = 3,     /* workspace smaller than kan_workspace_size() */
+    KAN_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed (detail in kan_last_error) */
+    KAN_ERR_TIMEOUT = 5,       /* a device-side wait gave up (reported by kan_sync_status) */
+    KAN_ERR_DEVICE_CHECK = 6   /* a device-side consistency check failed (reported by kan_sync_status) */
+} kan_status;
+
+/* Kernel family selection (kan_shape.path). */
+#define KAN_PATH_AUTO 0    /* tensor-core kernels when the shape allows them, else CUDA-core kernels */
+#define KAN_PATH_TENSOR 1  /* tcgen05/TMEM GEMM kernels with TMA-staged operands; KAN_ERR_UNSUPPORTED if not possible */
+#define KAN_PATH_SIMT 2    /* CUDA-core kernels (any shape) */
+
+typedef struct {
+    int64_t batch;     /* rows of x; 0 is allowed (nothing to compute, dcoef/dw_base zeroed) */
+    int64_t in;        /* input features, >= 1 */
+    int64_t out;       /* output features, >= 1 */
+    int32_t G;         /* grid intervals on [lo,hi], 1..250 */
+    float lo, hi;      /* grid range, hi > lo, both finite */
+    int32_t dtype;     /* kan_dtype of x, coef, w_base, y, dY, dx */
+    int32_t has_base;  /* 1: add the SiLU base branch w_base[j,i] silu(x[b,i]) */
+    int32_t path;      /* KAN_PATH_* */
+} kan_shape;
+
+/* ABI version of the loaded library (KAN_ABI_VERSION it was built with). */
+KAN_API int kan_abi_version(void);
+
+/* Bytes of device workspace that kan_forward (for_backward = 0) or
+ * kan_backward (for_backward = 1) needs for this shape on the current
+ * device.  *bytes may be 0.  Pure host computation. */
+KAN_API kan_status kan_workspace_size(const kan_shape* s, int for_backward, size_t* bytes);
+
+/* Forward pass: y = sum_i sum_m coef[j,i,m] B_m(x[b,i]) (+ w_base silu).
+ * w_base must be NULL when has_base = 0 and non-NULL otherwise.
+ * workspace may be NULL when the required size is 0. */
+KAN_API kan_status kan_forward(const kan_shape* s, const void* x, const void* coef, const void* w_base, void* y,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward pass for upstream gradient dY.  dx, dcoef, dw_base may each be
+ * NULL to skip that output (dw_base must be NULL when has_base = 0).
+ * dcoef and dw_base are float32 and overwritten (not accumulated). */
+KAN_API kan_status kan_backward(const kan_shape* s, const void* x, const void* coef, const void* w_base, const void* dY,
+                        void* dx, float* dcoef, float* dw_base, void* workspace, size_t ws_bytes, void* stream);
+
+/* The basis step alone, for inspection and tests: for each x[b,i] (batch*in
+ * values) the span s (int32; the 4 non-zero functions are B_s..B_{s+3}, some
+ * of which may fall outside 0..G+2 and are then absent; s = INT32_MIN when
+ * the input is outside the extended knots), the 4 weights w[.,4] = B_{s+r}(x)
+ * and the 4 derivatives dw[.,4] = B'_{s+r}(x).  Any output may be NULL. */
+KAN_API kan_status kan_basis(const kan_shape* s, const void* x, int32_t* span, float* w, float* dw, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word that
+ * kernels of this library set when a wait gives up (KAN_ERR_TIMEOUT) or a
+ * device check fails (KAN_ERR_DEVICE_CHECK).  KAN_OK if none did. */
+KAN_API kan_status kan_sync_status(void* stream);
+
+/* Failure-path self test: launches one kernel whose thread waits on an
+ * mbarrier that nothing completes, with a limit of limit_ns nanoseconds
+ * (1 .. 2e9).  The wait gives up and records KAN_ERR_TIMEOUT, which the next
+ * kan_sync_status() returns.  Faults and hangs nothing. */
+KAN_API kan_status kan_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
+/* Static description of a status code. */
+KAN_API const char* kan_status_string(kan_status st);
+
+/* Detail of the last non-OK status returned on this host thread ("" if none). */
+KAN_API const char* kan_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KAN_B200_H */

@@ -1,0 +1,123 @@
+"""ctypes binding of libkan_b200.so (declared in include/kan_b200.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  The library must exist (``python -m kolmogorov_arnold_network_b200.build``);
+there is no fallback of any kind when it does not.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkan_b200.so")
+
+KAN_F32, KAN_BF16 = 0, 1
+KAN_PATH_AUTO, KAN_PATH_TENSOR, KAN_PATH_SIMT = 0, 1, 2
+STATUS = {0: "KAN_OK", 1: "KAN_ERR_INVALID_ARG", 2: "KAN_ERR_UNSUPPORTED", 3: "KAN_ERR_WORKSPACE",
+          4: "KAN_ERR_CUDA", 5: "KAN_ERR_TIMEOUT", 6: "KAN_ERR_DEVICE_CHECK"}
+
+#: every symbol the header declares
+EXPORTS = ("kan_abi_version", "kan_workspace_size", "kan_forward", "kan_backward", "kan_basis", "kan_sync_status",
+           "kan_selftest_wait_timeout", "kan_status_string", "kan_last_error")
+
+
+class kan_shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("in_", ctypes.c_int64), ("out", ctypes.c_int64),
+                ("G", ctypes.c_int32), ("lo", ctypes.c_float), ("hi", ctypes.c_float),
+                ("dtype", ctypes.c_int32), ("has_base", ctypes.c_int32), ("path", ctypes.c_int32)]
+
+
+class KanError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {detail}")
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def load(path: str | None = None):
+    """Load libkan_b200.so; raises if it is missing (no fallback)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"{p} is missing: build it with `python -m kolmogorov_arnold_network_b200.build`")
+    lib = ctypes.CDLL(p)
+    sp = ctypes.POINTER(kan_shape)
+    lib.kan_abi_version.restype = ctypes.c_int
+    lib.kan_abi_version.argtypes = []
+    lib.kan_workspace_size.restype = ctypes.c_int
+    lib.kan_workspace_size.argtypes = [sp, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kan_forward.restype = ctypes.c_int
+    lib.kan_forward.argtypes = [sp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.kan_backward.restype = ctypes.c_int
+    lib.kan_backward.argtypes = [sp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.kan_basis.restype = ctypes.c_int
+    lib.kan_basis.argtypes = [sp, _vp, _vp, _vp, _vp, _vp]
+    lib.kan_sync_status.restype = ctypes.c_int
+    lib.kan_sync_status.argtypes = [_vp]
+    lib.kan_selftest_wait_timeout.restype = ctypes.c_int
+    lib.kan_selftest_wait_timeout.argtypes = [ctypes.c_int64, _vp]
+    lib.kan_status_string.restype = ctypes.c_char_p
+    lib.kan_status_string.argtypes = [ctypes.c_int]
+    lib.kan_last_error.restype = ctypes.c_char_p
+    lib.kan_last_error.argtypes = []
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def check(status: int, where: str):
+    if status != 0:
+        raise KanError(status, where, load().kan_last_error().decode())
+
+
+def make_shape(batch, n_in, n_out, G, lo, hi, dtype, has_base, path=KAN_PATH_AUTO) -> kan_shape:
+    return kan_shape(int(batch), int(n_in), int(n_out), int(G), float(lo), float(hi), int(dtype), int(bool(has_base)),
+                     int(path))
+
+
+# ---- the C-ABI calls, same names, raw pointers (ints) and sizes ----
+def kan_abi_version() -> int:
+    return load().kan_abi_version()
+
+
+def kan_workspace_size(shape: kan_shape, for_backward: bool) -> int:
+    n = ctypes.c_size_t(0)
+    check(load().kan_workspace_size(ctypes.byref(shape), int(bool(for_backward)), ctypes.byref(n)),
+          "kan_workspace_size")
+    return n.value
+
+
+def kan_forward(shape, x, coef, w_base, y, workspace, ws_bytes, stream):
+    check(load().kan_forward(ctypes.byref(shape), x, coef, w_base, y, workspace, ws_bytes, stream), "kan_forward")
+
+
+def kan_backward(shape, x, coef, w_base, dY, dx, dcoef, dw_base, workspace, ws_bytes, stream):
+    check(load().kan_backward(ctypes.byref(shape), x, coef, w_base, dY, dx, dcoef, dw_base, workspace, ws_bytes,
+                              stream), "kan_backward")
+
+
+def kan_basis(shape, x, span, w, dw, stream):
+    check(load().kan_basis(ctypes.byref(shape), x, span, w, dw, stream), "kan_basis")
+
+
+def kan_sync_status(stream) -> int:
+    """Returns the status code (does not raise) so callers can test for timeouts."""
+    return load().kan_sync_status(stream)
+
+
+def kan_selftest_wait_timeout(limit_ns: int, stream):
+    check(load().kan_selftest_wait_timeout(int(limit_ns), stream), "kan_selftest_wait_timeout")
+
+
+def kan_status_string(st: int) -> str:
+    return load().kan_status_string(int(st)).decode()
+
+
+def kan_last_error() -> str:
+    return load().kan_last_error().decode()

@@ -1,0 +1,311 @@
+// kan_device.cuh -- device-side building blocks shared by the kernels:
+// the span/weight evaluation of uniform cubic B-splines, bounded waits, and
+// thin wrappers over the sm_100a PTX used by the tensor-core kernels
+// (mbarrier, TMA, tcgen05).  All PTX is written from the public PTX ISA.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kan_internal.h"
+
+namespace kan {
+
+// ---------------------------------------------------------------------------
+// Span and local weights (steps S1, S2)
+//
+// For the uniform grid t_k = lo + (k-3)h, h = (hi-lo)/G, an input x lies in
+// knot interval floor(u)+3 with u = (x-lo)/h.  With s = floor(u) and the
+// local coordinate t = u - s in [0,1), exactly B_s..B_{s+3} can be non-zero
+// (the "local 4-basis lookup" of the InKAN landing page, "Why InKAN?"), and
+// those with index outside 0..G+2 do not exist.  The input is inside the
+// extended knots iff -3 <= u < G+3; NaN and +-inf fail that test, so they
+// contribute nothing and never reach an index computation.
+//
+// The weights are the four pieces of the uniform cubic B-spline written in a
+// form without cancellation on the bounded coordinate t in [0,1) (the
+// "stable piecewise polynomial evaluation" with non-negative output of the
+// InKAN page, "Numerically Stable"; the clamp to a bounded coordinate is the
+// FlashKAN abstract's stabilisation):
+//   w0 = (1-t)^3/6            w3 = t^3/6
+//   w1 = 2/3 - t^2 (2-t)/2    w2 = 2/3 - (1-t)^2 (1+t)/2     (w2(t) = w1(1-t))
+// and their derivatives with respect to x (factor 1/h):
+//   w0' = -(1-t)^2/2   w1' = (3t^2-4t)/2   w2' = -(3(1-t)^2-4(1-t))/2   w3' = t^2/2
+// ---------------------------------------------------------------------------
+struct Span {
+    int s;       // first of the 4 basis indices
+    float t;     // local coordinate in [0,1)
+    bool valid;  // inside the extended knots
+};
+
+__device__ __forceinline__ Span span_of(float x, float lo, float inv_h, int G)
+{
+    Span r;
+    float u = (x - lo) * inv_h;
+    r.valid = (u >= -3.0f) && (u < (float)(G + 3));
+    float f = floorf(r.valid ? u : 0.0f);
+    r.s = (int)f;
+    r.t = r.valid ? (u - f) : 0.0f;
+    return r;
+}
+
+__device__ __forceinline__ void weights(float t, float w[4])
+{
+    const float s = 1.0f - t;
+    const float t2 = t * t, s2 = s * s;
+    w[0] = s2 * s * (1.0f / 6.0f);
+    w[1] = (2.0f / 3.0f) - 0.5f * t2 * (1.0f + s);
+    w[2] = (2.0f / 3.0f) - 0.5f * s2 * (1.0f + t);
+    w[3] = t2 * t * (1.0f / 6.0f);
+}
+
+__device__ __forceinline__ void dweights(float t, float inv_h, float d[4])
+{
+    const float s = 1.0f - t;
+    d[0] = -0.5f * s * s * inv_h;
+    d[1] = (1.5f * t - 2.0f) * t * inv_h;
+    d[2] = -(1.5f * s - 2.0f) * s * inv_h;
+    d[3] = 0.5f * t * t * inv_h;
+}
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+
+__device__ __forceinline__ float dsilu_f(float x)
+{
+    float sg = 1.0f / (1.0f + __expf(-x));
+    return sg * (1.0f + x * (1.0f - sg));
+}
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// ---------------------------------------------------------------------------
+// Device status word and bounded waits
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Record an error code (any writer wins; every writer writes a non-zero code).
+__device__ __forceinline__ void record_status(unsigned int* status, unsigned int code)
+{
+    if (status) *(volatile unsigned int*)status = code;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of the mbarrier to complete, giving up after
+// limit_ns nanoseconds: then records KAN_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int* status,
+                                          uint64_t limit_ns = KAN_WAIT_LIMIT_NS)
+{
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_test(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_status(status, KAN_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA (per-CTA tiled loads, no multicast)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            dst),
+        "l"(tmap), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* tmap)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05: TMEM allocation, MMA, commit, loads
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 operands, fp32 accumulation.
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Same with tf32 operands (32-bit containers; the unit reads the tf32 part).
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the mbarrier when every tcgen05 op issued so far by this
+// thread has completed.
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns: lane l of the warp gets row
+// (lane base + l), columns col..col+15.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// Operand descriptors
+// ---------------------------------------------------------------------------
+// Shared-memory matrix descriptor (tcgen05 "matrix descriptor"):
+//   bits  0-13  start address >> 4
+//   bits 16-29  leading-dimension byte offset >> 4
+//   bits 32-45  stride-dimension byte offset >> 4
+//   bits 46-47  descriptor version (1 on sm_100)
+//   bits 49-51  base offset (0: every swizzle atom here is 1024-byte aligned)
+//   bit  52     leading-dimension offset mode (0: relative)
+//   bits 61-63  swizzle mode (2 = 128-byte swizzle)
+// With the 128-byte swizzle, a K-major tile is a stack of 8-row x 128-byte
+// atoms (SBO = 1024, LBO unused); an MN-major tile is a set of
+// [K rows x 128 bytes] column blocks, LBO apart, whose 8-row groups are
+// SBO = 1024 apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation:
+//   bits 4-5 D format (1 = f32), bits 7-9 A format, bits 10-12 B format
+//   (bf16 = 1, tf32 = 2), bit 15 A major, bit 16 B major (0 = K, 1 = MN),
+//   bits 17-22 N >> 3, bits 24-28 M >> 4.
+__host__ __device__ constexpr uint32_t instr_desc(uint32_t ab_format, uint32_t a_mn_major, uint32_t b_mn_major,
+                                                  uint32_t M, uint32_t N)
+{
+    return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
+           ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` inside a 128-byte
+// swizzled tile (the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B).
+__device__ __forceinline__ uint32_t sw128_chunk(uint32_t row, uint32_t chunk)
+{
+    return row * 128u + (((chunk ^ (row & 7u)) & 7u) << 4);
+}
+
+// Byte offset of the element at byte column `colb` (0..127) of row `row`.
+__device__ __forceinline__ uint32_t sw128_byte(uint32_t row, uint32_t colb)
+{
+    return sw128_chunk(row, colb >> 4) | (colb & 15u);
+}
+
+// tf32 split: hi keeps the 10 explicit mantissa bits of x rounded to
+// nearest (cvt.rna.tf32.f32), lo = x - hi is exact in fp32 and is itself
+// read by the unit at tf32 precision; hi*hi' + hi*lo' + lo*hi' then carries
+// about 21 bits of each product.
+__device__ __forceinline__ float tf32_hi(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+}  // namespace kan

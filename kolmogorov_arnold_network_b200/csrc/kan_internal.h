@@ -1,0 +1,54 @@
+// kan_internal.h -- declarations shared by the library's translation units
+// (not part of the public ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kan_b200.h"
+
+#define KAN_WAIT_LIMIT_NS 1000000000ull  // every device-side wait gives up after ~1 s
+#define KAN_MAX_G 250
+
+namespace kan {
+
+// Validated problem description passed from the C-ABI layer to launchers.
+struct Problem {
+    int64_t batch, in, out;
+    int G;
+    int nb;          // G + 3 basis functions per edge
+    int64_t Kt;      // in * nb (spline columns of the dense expansion)
+    float lo, hi, inv_h;
+    int dtype;       // KAN_F32 / KAN_BF16
+    bool base;
+    int path;
+};
+
+// Device status word (defined in kan_api.cu).
+unsigned int* device_status_ptr();
+
+// ---- CUDA-core kernels (kan_simt.cu) ----
+cudaError_t simt_basis(const Problem& p, const void* x, int32_t* span, float* w, float* dw, cudaStream_t st);
+cudaError_t simt_forward(const Problem& p, const void* x, const void* coef, const void* w_base, void* y,
+                         cudaStream_t st);
+cudaError_t simt_backward(const Problem& p, const void* x, const void* coef, const void* w_base, const void* dY,
+                          void* dx, float* dcoef, float* dw_base, cudaStream_t st);
+cudaError_t simt_wait_selftest(int64_t limit_ns, unsigned int* status, cudaStream_t st);
+cudaError_t zero_f32(float* p, int64_t n, cudaStream_t st);
+
+// ---- tensor-core kernels (kan_tc.cu) ----
+// Returns true when the tensor-core path can run this problem (alignment of
+// the strides that TMA needs, sizes); `why` receives the reason otherwise.
+bool tc_supported(const Problem& p, bool backward, const char** why);
+size_t tc_workspace_forward(const Problem& p, int num_sms);
+size_t tc_workspace_backward(const Problem& p, int num_sms);
+// Return cudaSuccess or an error; a driver-level failure (tensor map encode)
+// is mapped to cudaErrorInvalidValue with detail in *detail.
+cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const void* w_base, void* y, void* ws,
+                       int num_sms, cudaStream_t st, const char** detail);
+cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const void* w_base, const void* dY,
+                        void* dx, float* dcoef, float* dw_base, void* ws, int num_sms, cudaStream_t st,
+                        const char** detail);
+
+}  // namespace kan

@@ -1,0 +1,267 @@
+// kan_simt.cu -- CUDA-core kernels of the KAN layer: the basis step on its
+// own, and a complete forward/backward for shapes the tensor-core path does
+// not take (tiny layers, strides TMA cannot address).  Each output element
+// is produced by one thread with a fixed summation order, so results are
+// deterministic; no atomics.
+#include "kan_device.cuh"
+
+namespace kan {
+namespace {
+
+constexpr int kFwdRows = 4;       // batch rows per forward block
+constexpr int kFwdChunk = 512;    // inputs staged per pass in the forward block
+constexpr int kMaxNb = KAN_MAX_G + 3;
+
+template <typename T>
+__global__ void basis_kernel(const T* __restrict__ x, int64_t n, float lo, float inv_h, int G, int32_t* span,
+                             float* w, float* dw)
+{
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        Span sp = span_of(to_f(x[e]), lo, inv_h, G);
+        float wv[4] = {0.f, 0.f, 0.f, 0.f}, dv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (sp.valid) {
+            weights(sp.t, wv);
+            dweights(sp.t, inv_h, dv);
+        }
+        if (span) span[e] = sp.valid ? sp.s : INT32_MIN;
+        if (w) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) w[e * 4 + r] = wv[r];
+        }
+        if (dw) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) dw[e * 4 + r] = dv[r];
+        }
+    }
+}
+
+// y[b, j]: block = kFwdRows rows, threads stride over j.  The rows' spans
+// and weights for a chunk of inputs are staged in shared memory.
+template <typename T>
+__global__ void forward_kernel(const T* __restrict__ x, const T* __restrict__ coef, const T* __restrict__ w_base,
+                               T* __restrict__ y, int64_t batch, int64_t in, int64_t out, int G, float lo,
+                               float inv_h)
+{
+    __shared__ int s_span[kFwdRows][kFwdChunk];
+    __shared__ float s_w[kFwdRows][kFwdChunk][4];
+    __shared__ float s_silu[kFwdRows][kFwdChunk];
+    const int nb = G + 3;
+    const int64_t b0 = (int64_t)blockIdx.x * kFwdRows;
+    const int nrows = (int)(batch - b0 < kFwdRows ? batch - b0 : kFwdRows);
+
+    for (int64_t jb = 0; jb < out; jb += blockDim.x) {
+        const int64_t j = jb + threadIdx.x;
+        float acc[kFwdRows], accb[kFwdRows];
+#pragma unroll
+        for (int r = 0; r < kFwdRows; ++r) acc[r] = accb[r] = 0.f;
+
+        for (int64_t i0 = 0; i0 < in; i0 += kFwdChunk) {
+            const int ni = (int)(in - i0 < kFwdChunk ? in - i0 : kFwdChunk);
+            __syncthreads();
+            for (int e = threadIdx.x; e < kFwdRows * ni; e += blockDim.x) {
+                int r = e / ni, ii = e % ni;
+                float xv = r < nrows ? to_f(x[(b0 + r) * in + i0 + ii]) : 0.f;
+                Span sp = span_of(xv, lo, inv_h, G);
+                float wv[4] = {0.f, 0.f, 0.f, 0.f};
+                if (sp.valid && r < nrows) weights(sp.t, wv);
+                s_span[r][ii] = (sp.valid && r < nrows) ? sp.s : -1000;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) s_w[r][ii][q] = wv[q];
+                s_silu[r][ii] = (w_base && r < nrows) ? silu_f(xv) : 0.f;
+            }
+            __syncthreads();
+            if (j < out) {
+                const T* cj = coef + (j * in + i0) * nb;
+                for (int ii = 0; ii < ni; ++ii) {
+                    const T* cji = cj + (int64_t)ii * nb;
+#pragma unroll
+                    for (int r = 0; r < kFwdRows; ++r) {
+                        int s = s_span[r][ii];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            int m = s + q;
+                            if (m >= 0 && m < nb) acc[r] += to_f(cji[m]) * s_w[r][ii][q];
+                        }
+                    }
+                    if (w_base) {
+                        float wb = to_f(w_base[j * in + i0 + ii]);
+#pragma unroll
+                        for (int r = 0; r < kFwdRows; ++r) accb[r] += wb * s_silu[r][ii];
+                    }
+                }
+            }
+        }
+        if (j < out)
+            for (int r = 0; r < nrows; ++r) y[(b0 + r) * out + j] = from_f<T>(acc[r] + accb[r]);
+    }
+}
+
+// dcoef[j, i, :], dw_base[j, i]: one thread per (j, i), batch summed in order.
+template <typename T>
+__global__ void dcoef_kernel(const T* __restrict__ x, const T* __restrict__ dY, float* __restrict__ dcoef,
+                             float* __restrict__ dw_base, int64_t batch, int64_t in, int64_t out, int G, float lo,
+                             float inv_h)
+{
+    const int nb = G + 3;
+    const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (e >= in * out) return;
+    const int64_t j = e / in, i = e % in;
+    float acc[kMaxNb];
+    for (int m = 0; m < nb; ++m) acc[m] = 0.f;
+    float accb = 0.f;
+    for (int64_t b = 0; b < batch; ++b) {
+        float xv = to_f(x[b * in + i]);
+        float g = to_f(dY[b * out + j]);
+        Span sp = span_of(xv, lo, inv_h, G);
+        if (sp.valid) {
+            float wv[4];
+            weights(sp.t, wv);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                int m = sp.s + q;
+                if (m >= 0 && m < nb) acc[m] += wv[q] * g;
+            }
+        }
+        if (dw_base) accb += silu_f(xv) * g;
+    }
+    if (dcoef)
+        for (int m = 0; m < nb; ++m) dcoef[e * nb + m] = acc[m];
+    if (dw_base) dw_base[e] = accb;
+}
+
+// dx[b, i]: one thread per (b, i), j summed in order.
+template <typename T>
+__global__ void dx_kernel(const T* __restrict__ x, const T* __restrict__ coef, const T* __restrict__ w_base,
+                          const T* __restrict__ dY, T* __restrict__ dx, int64_t batch, int64_t in, int64_t out,
+                          int G, float lo, float inv_h)
+{
+    const int nb = G + 3;
+    const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (e >= batch * in) return;
+    const int64_t b = e / in, i = e % in;
+    float xv = to_f(x[e]);
+    Span sp = span_of(xv, lo, inv_h, G);
+    float dv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (sp.valid) dweights(sp.t, inv_h, dv);
+    const float ds = w_base ? dsilu_f(xv) : 0.f;
+    float acc = 0.f;
+    for (int64_t j = 0; j < out; ++j) {
+        const T* cji = coef + (j * in + i) * nb;
+        float d = 0.f;
+        if (sp.valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                int m = sp.s + q;
+                if (m >= 0 && m < nb) d += to_f(cji[m]) * dv[q];
+            }
+        }
+        if (w_base) d += to_f(w_base[j * in + i]) * ds;
+        acc += to_f(dY[b * out + j]) * d;
+    }
+    dx[e] = from_f<T>(acc);
+}
+
+__global__ void zero_kernel(float* p, int64_t n)
+{
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+        p[e] = 0.f;
+}
+
+// One thread waits on an mbarrier that nothing arrives at; the bounded wait
+// gives up after limit_ns and records KAN_ERR_TIMEOUT.
+__global__ void wait_selftest_kernel(uint64_t limit_ns, unsigned int* status)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(smem_addr(&bar), 0, status, limit_ns);
+}
+
+inline int blocks_for(int64_t n, int threads)
+{
+    int64_t b = (n + threads - 1) / threads;
+    return (int)(b < 1 ? 1 : (b > 65535LL * 32 ? 65535LL * 32 : b));
+}
+
+}  // namespace
+
+cudaError_t simt_basis(const Problem& p, const void* x, int32_t* span, float* w, float* dw, cudaStream_t st)
+{
+    const int64_t n = p.batch * p.in;
+    if (n == 0) return cudaSuccess;
+    if (p.dtype == KAN_F32)
+        basis_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>((const float*)x, n, p.lo, p.inv_h, p.G, span, w, dw);
+    else
+        basis_kernel<__nv_bfloat16><<<blocks_for(n, 256), 256, 0, st>>>((const __nv_bfloat16*)x, n, p.lo, p.inv_h,
+                                                                         p.G, span, w, dw);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_forward(const Problem& p, const void* x, const void* coef, const void* w_base, void* y,
+                         cudaStream_t st)
+{
+    if (p.batch == 0) return cudaSuccess;
+    const int blocks = (int)((p.batch + kFwdRows - 1) / kFwdRows);
+    const int threads = p.out >= 128 ? 128 : (int)((p.out + 31) / 32 * 32);
+    if (p.dtype == KAN_F32)
+        forward_kernel<float><<<blocks, threads, 0, st>>>((const float*)x, (const float*)coef, (const float*)w_base,
+                                                          (float*)y, p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+    else
+        forward_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+            (const __nv_bfloat16*)x, (const __nv_bfloat16*)coef, (const __nv_bfloat16*)w_base, (__nv_bfloat16*)y,
+            p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_backward(const Problem& p, const void* x, const void* coef, const void* w_base, const void* dY,
+                          void* dx, float* dcoef, float* dw_base, cudaStream_t st)
+{
+    cudaError_t e;
+    if (p.batch == 0) {
+        if (dcoef && (e = zero_f32(dcoef, p.out * p.Kt, st)) != cudaSuccess) return e;
+        if (dw_base && (e = zero_f32(dw_base, p.out * p.in, st)) != cudaSuccess) return e;
+        return cudaSuccess;
+    }
+    if (dcoef || dw_base) {
+        const int64_t n = p.in * p.out;
+        if (p.dtype == KAN_F32)
+            dcoef_kernel<float><<<blocks_for(n, 128), 128, 0, st>>>((const float*)x, (const float*)dY, dcoef, dw_base,
+                                                                     p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+        else
+            dcoef_kernel<__nv_bfloat16><<<blocks_for(n, 128), 128, 0, st>>>(
+                (const __nv_bfloat16*)x, (const __nv_bfloat16*)dY, dcoef, dw_base, p.batch, p.in, p.out, p.G, p.lo,
+                p.inv_h);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (dx) {
+        const int64_t n = p.batch * p.in;
+        if (p.dtype == KAN_F32)
+            dx_kernel<float><<<blocks_for(n, 128), 128, 0, st>>>((const float*)x, (const float*)coef,
+                                                                  (const float*)w_base, (const float*)dY, (float*)dx,
+                                                                  p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+        else
+            dx_kernel<__nv_bfloat16><<<blocks_for(n, 128), 128, 0, st>>>(
+                (const __nv_bfloat16*)x, (const __nv_bfloat16*)coef, (const __nv_bfloat16*)w_base,
+                (const __nv_bfloat16*)dY, (__nv_bfloat16*)dx, p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t zero_f32(float* p, int64_t n, cudaStream_t st)
+{
+    if (n <= 0) return cudaSuccess;
+    zero_kernel<<<blocks_for(n, 256) > 4096 ? 4096 : blocks_for(n, 256), 256, 0, st>>>(p, n);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_wait_selftest(int64_t limit_ns, unsigned int* status, cudaStream_t st)
+{
+    wait_selftest_kernel<<<1, 32, 0, st>>>((uint64_t)limit_ns, status);
+    return cudaGetLastError();
+}
+
+}  // namespace kan

@@ -1,0 +1,160 @@
+"""Torch-facing calls over the C ABI, and the drop-in ``KANLayer`` module.
+
+``KANLayer(in, out)`` replaces ``nn.Linear(in, out)`` (InKAN landing page,
+"Drop-in Replacement" and "Quick Start"); ``KANNetwork([784, 64, 10])`` stacks
+layers.  PyTorch provides device memory, the stream and autograd; every step
+of the layer itself runs in libkan_b200.so.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _native as N
+
+_DT = {torch.float32: N.KAN_F32, torch.bfloat16: N.KAN_BF16}
+
+
+def _code(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"dtype {t.dtype} not supported (float32 or bfloat16)")
+    return _DT[t.dtype]
+
+
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check(t, name, dtype=None, shape=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def shape_of(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO) -> N.kan_shape:
+    batch, n_in = x.shape
+    return N.make_shape(batch, n_in, coef.shape[0], G, lo, hi, _code(x), w_base is not None, path)
+
+
+def _stream(t):
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def workspace(shape: N.kan_shape, for_backward: bool, device) -> torch.Tensor | None:
+    n = N.kan_workspace_size(shape, for_backward)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def forward(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, y=None, ws=None):
+    """y[b,j] = sum_i sum_m coef[j,i,m] B_m(x[b,i]) (+ sum_i w_base[j,i] silu(x[b,i]))."""
+    batch, n_in = x.shape
+    n_out = coef.shape[0]
+    _check(x, "x", None)
+    _check(coef, "coef", x.dtype, (n_out, n_in, G + 3))
+    _check(w_base, "w_base", x.dtype, (n_out, n_in))
+    s = shape_of(x, coef, G, lo, hi, w_base, path)
+    if y is None:
+        y = torch.empty((batch, n_out), dtype=x.dtype, device=x.device)
+    _check(y, "y", x.dtype, (batch, n_out))
+    if ws is None:
+        ws = workspace(s, False, x.device)
+    N.kan_forward(s, _p(x), _p(coef), _p(w_base), _p(y), _p(ws), 0 if ws is None else ws.numel(), _stream(x))
+    return y
+
+
+def backward(x, coef, dY, G, lo, hi, w_base=None, need_dx=True, need_dcoef=True, need_dw_base=True,
+             path=N.KAN_PATH_AUTO, out=None, ws=None):
+    """(dx, dcoef, dw_base) of the layer for upstream gradient dY; dcoef/dw_base are float32."""
+    batch, n_in = x.shape
+    n_out = coef.shape[0]
+    _check(x, "x", None)
+    _check(coef, "coef", x.dtype, (n_out, n_in, G + 3))
+    _check(w_base, "w_base", x.dtype, (n_out, n_in))
+    _check(dY, "dY", x.dtype, (batch, n_out))
+    s = shape_of(x, coef, G, lo, hi, w_base, path)
+    if out is not None:
+        dx, dcoef, dwb = out
+    else:
+        dx = torch.empty_like(x) if need_dx else None
+        dcoef = torch.empty(coef.shape, dtype=torch.float32, device=x.device) if need_dcoef else None
+        dwb = (torch.empty(w_base.shape, dtype=torch.float32, device=x.device)
+               if (need_dw_base and w_base is not None) else None)
+    if ws is None:
+        ws = workspace(s, True, x.device)
+    N.kan_backward(s, _p(x), _p(coef), _p(w_base), _p(dY), _p(dx), _p(dcoef), _p(dwb), _p(ws),
+                   0 if ws is None else ws.numel(), _stream(x))
+    return dx, dcoef, dwb
+
+
+def basis(x, G, lo, hi):
+    """(span int32 [.., in], w [.., in, 4], dw [.., in, 4]) of the basis step alone."""
+    _check(x, "x", None)
+    batch, n_in = x.shape
+    s = N.make_shape(batch, n_in, 1, G, lo, hi, _code(x), False)
+    span = torch.empty((batch, n_in), dtype=torch.int32, device=x.device)
+    w = torch.empty((batch, n_in, 4), dtype=torch.float32, device=x.device)
+    dw = torch.empty((batch, n_in, 4), dtype=torch.float32, device=x.device)
+    N.kan_basis(s, _p(x), _p(span), _p(w), _p(dw), _stream(x))
+    return span, w, dw
+
+
+class _KANFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, coef, w_base, G, lo, hi):
+        x = x.contiguous()
+        y = forward(x, coef, G, lo, hi, w_base)
+        ctx.save_for_backward(x, coef, w_base)
+        ctx.grid = (G, lo, hi)
+        return y
+
+    @staticmethod
+    def backward(ctx, dY):
+        x, coef, w_base = ctx.saved_tensors
+        G, lo, hi = ctx.grid
+        dx, dcoef, dwb = backward(x, coef, dY.contiguous().to(x.dtype), G, lo, hi, w_base,
+                                  need_dx=ctx.needs_input_grad[0], need_dcoef=ctx.needs_input_grad[1],
+                                  need_dw_base=w_base is not None and ctx.needs_input_grad[2])
+        return (dx, None if dcoef is None else dcoef.to(coef.dtype), None if dwb is None else dwb.to(w_base.dtype),
+                None, None, None)
+
+
+class KANLayer(torch.nn.Module):
+    """Cubic B-spline KAN layer, a drop-in for ``nn.Linear(in, out)``.
+
+    Parameters: ``coef`` [out, in, G+3] and, with ``base=True``, ``w_base``
+    [out, in] for the SiLU base branch.
+    """
+
+    def __init__(self, in_features, out_features, G=8, lo=-1.0, hi=1.0, base=False, coef_std=0.1,
+                 dtype=torch.float32, device=None):
+        super().__init__()
+        self.in_features, self.out_features = in_features, out_features
+        self.G, self.lo, self.hi = int(G), float(lo), float(hi)
+        self.coef = torch.nn.Parameter(
+            torch.randn(out_features, in_features, G + 3, dtype=torch.float32, device=device).mul_(coef_std).to(dtype))
+        self.w_base = (torch.nn.Parameter(torch.randn(out_features, in_features, dtype=torch.float32, device=device)
+                                          .mul_(in_features ** -0.5).to(dtype)) if base else None)
+
+    def forward(self, x):
+        lead = x.shape[:-1]
+        y = _KANFunction.apply(x.reshape(-1, self.in_features), self.coef, self.w_base, self.G, self.lo, self.hi)
+        return y.reshape(*lead, self.out_features)
+
+
+class KANNetwork(torch.nn.Module):
+    """Stack of KANLayer: ``KANNetwork([784, 64, 10])``."""
+
+    def __init__(self, widths, **kw):
+        super().__init__()
+        self.layers = torch.nn.ModuleList(KANLayer(a, b, **kw) for a, b in zip(widths[:-1], widths[1:]))
+
+    def forward(self, x):
+        for L in self.layers:
+            x = L(x)
+        return x
