@@ -1,0 +1,454 @@
+"""Benchmark: KAN layer forward+backward edge evaluations per second on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+the forward (y), then the backward (dx, and dcoef / dw_base), through the C ABI
+of libkan_b200.so.  Edge evaluations per step = batch * in * out (summed over
+the layers of the FFN block).  One JSON line is printed by rank 0.
+
+Timing: W untimed steps, then K timed steps between a barrier and a device
+synchronize on both sides.  Each step is bracketed by CUDA events on the
+launching stream; a 256 MiB buffer (larger than the 126 MB L2) is rewritten
+between steps, outside the events.  Each C-ABI call inside the step carries
+its own events too, which give the dominant kernel's launch time for the
+roofline.  With N > 1 (torchrun), every rank runs an independent replica of
+the workload (weak scaling, no collective on the data path) and the time is
+the maximum over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (the
+only reference this build has), each step a bounded row sample of the same
+workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from kolmogorov_arnold_network_b200 import workloads as W  # noqa: E402
+
+METRIC = "KAN layer fwd+bwd edge-evals/sec (batch*in*out) and % of roofline, 1xB200"
+UNIT = "edge-evals/s"
+TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor-core ratio on B200
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sus": d.get("bf16_tflops_sustained"),
+                "src": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sus": 1400.0, "src": "fallback"}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# FLOP / byte accounting (per call, algorithmic)
+def layer_dense_flops(batch, L):
+    """Dense-expanded FLOPs of one layer GEMM: 2 * batch * out * (in*(G+3) [+ in for SiLU])."""
+    k = L.inp * (L.G + 3) + (L.inp if L.base else 0)
+    return 2.0 * batch * L.out * k
+
+
+def layer_bytes(batch, L, esz, call):
+    """Algorithmic HBM bytes of one call: operands read once, outputs written once."""
+    x = batch * L.inp * esz
+    dy = batch * L.out * esz
+    coef = L.out * L.inp * (L.G + 3) * esz + (L.out * L.inp * esz if L.base else 0)
+    if call == "fwd":
+        return x + coef + batch * L.out * esz
+    if call == "dcoef":
+        return x + dy + (L.out * L.inp * (L.G + 3) + (L.out * L.inp if L.base else 0)) * 4
+    return x + dy + coef + batch * L.inp * esz          # dx
+
+
+# ---------------------------------------------------------------------------
+class Runner:
+    """Pre-allocated buffers and the step's C-ABI calls for one workload."""
+
+    def __init__(self, w: W.Workload, dev):
+        from kolmogorov_arnold_network_b200 import _native as N
+        from kolmogorov_arnold_network_b200 import layer as LY
+        self.N, self.LY, self.w, self.dev = N, LY, w, dev
+        d = W.draw_all(w)
+        self.host = d
+        dt = w.torch_dtype
+        self.x = d["x"].to(dev)
+        self.dY = d["dY"].to(dev)
+        self.layers = []
+        act = self.x
+        for li, L in enumerate(w.layers):
+            coef = d[f"coef{li}"].to(dev)
+            wb = None if d[f"w_base{li}"] is None else d[f"w_base{li}"].to(dev)
+            s = LY.shape_of(act, coef, L.G, L.lo, L.hi, wb)
+            ws_f = LY.workspace(s, False, dev)
+            ws_b = LY.workspace(s, True, dev)
+            y = torch.empty((w.batch, L.out), dtype=dt, device=dev)
+            dx = torch.empty((w.batch, L.inp), dtype=dt, device=dev)
+            dcoef = torch.empty(coef.shape, dtype=torch.float32, device=dev)
+            dwb = None if wb is None else torch.empty(wb.shape, dtype=torch.float32, device=dev)
+            self.layers.append(dict(L=L, s=s, x=act, coef=coef, wb=wb, y=y, dx=dx, dcoef=dcoef, dwb=dwb,
+                                    ws_f=ws_f, ws_b=ws_b))
+            act = y
+        # pinned host mirrors for the end-to-end variant
+        self.h_x = d["x"].pin_memory()
+        self.h_dY = d["dY"].pin_memory()
+        self.h_out = []
+        for l in self.layers:
+            self.h_out.append(dict(y=torch.empty_like(l["y"], device="cpu").pin_memory(),
+                                   dx=torch.empty_like(l["dx"], device="cpu").pin_memory(),
+                                   dcoef=torch.empty_like(l["dcoef"], device="cpu").pin_memory(),
+                                   dwb=None if l["dwb"] is None else
+                                   torch.empty_like(l["dwb"], device="cpu").pin_memory()))
+
+    def calls(self):
+        """The step as a list of (name, callable), in launch order."""
+        N, P = self.N, lambda t: None if t is None else t.data_ptr()
+        st = torch.cuda.current_stream(self.dev).cuda_stream
+        out = []
+        for li, l in enumerate(self.layers):
+            def fwd(l=l):
+                N.kan_forward(l["s"], P(l["x"]), P(l["coef"]), P(l["wb"]), P(l["y"]), P(l["ws_f"]),
+                              0 if l["ws_f"] is None else l["ws_f"].numel(), st)
+            out.append((f"fwd{li}", fwd))
+        for li in reversed(range(len(self.layers))):
+            l = self.layers[li]
+            dy = self.dY if li == len(self.layers) - 1 else self.layers[li + 1]["dx"]
+
+            def dcoef(l=l, dy=dy):
+                N.kan_backward(l["s"], P(l["x"]), P(l["coef"]), P(l["wb"]), P(dy), None, P(l["dcoef"]),
+                               P(l["dwb"]), P(l["ws_b"]), 0 if l["ws_b"] is None else l["ws_b"].numel(), st)
+
+            def dx(l=l, dy=dy):
+                N.kan_backward(l["s"], P(l["x"]), P(l["coef"]), P(l["wb"]), P(dy), P(l["dx"]), None, None,
+                               P(l["ws_b"]), 0 if l["ws_b"] is None else l["ws_b"].numel(), st)
+            out.append((f"dcoef{li}", dcoef))
+            out.append((f"dx{li}", dx))
+        return out
+
+    def h2d(self):
+        self.x.copy_(self.h_x, non_blocking=True)
+        self.dY.copy_(self.h_dY, non_blocking=True)
+        return self.h_x.numel() * self.h_x.element_size() + self.h_dY.numel() * self.h_dY.element_size()
+
+    def d2h(self):
+        n = 0
+        for l, h in zip(self.layers, self.h_out):
+            for k in ("y", "dx", "dcoef", "dwb"):
+                if h[k] is not None:
+                    h[k].copy_(l[k], non_blocking=True)
+                    n += h[k].numel() * h[k].element_size()
+        return n
+
+
+class ClockSampler:
+    def __init__(self, dev_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            uuid = None
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        cmd = ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if uuid:
+            cmd += ["-i", uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            f = [t.strip() for t in line.split(",")]
+            if len(f) >= 8:
+                try:
+                    rows.append((float(f[0]), float(f[1]), f[3:]))
+                except ValueError:
+                    pass
+        if not rows:
+            return None
+        sm = sorted(r[0] for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for nm, v in zip(names, r[2][1:]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+def cpu_baseline(w: W.Workload, target_s=12.0):
+    """The fp64 oracle, as it stands, on a row sample of the workload (host cores)."""
+    import oracle
+    o = oracle.get()
+    cores = oracle.default_threads()
+    d = W.draw_all(w)
+
+    def run(rows):
+        x = d["x"][:rows]
+        dY = d["dY"][:rows]
+        t0 = time.perf_counter()
+        act = x
+        acts = []
+        for li, L in enumerate(w.layers):
+            acts.append(act)
+            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], nthreads=cores)
+        g = dY
+        for li in reversed(range(len(w.layers))):
+            L = w.layers[li]
+            gx, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"],
+                                  nthreads=cores)
+            g = gx
+        return time.perf_counter() - t0
+
+    probe = max(cores, 8)
+    t = run(probe)
+    rows = int(min(w.batch, max(probe, probe * target_s / max(t, 1e-6))))
+    t = run(rows)
+    edges = sum(rows * L.inp * L.out for L in w.layers)
+    return {"value": edges / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{rows} of {w.batch} rows of {w.name}, fp64 Cox-de Boor forward+backward, {t:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    w = W.WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    import oracle
+    o = oracle.get()
+    cores = oracle.default_threads()
+    d = W.draw_all(w)
+
+    def step(rows):
+        x = d["x"][:rows]
+        act = x
+        acts = []
+        for li, L in enumerate(w.layers):
+            acts.append(act)
+            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], nthreads=cores)
+        g = d["dY"][:rows]
+        for li in reversed(range(len(w.layers))):
+            L = w.layers[li]
+            g, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"],
+                                 nthreads=cores)
+
+    # size the per-step sample so that warmup + steps end within ~2 minutes
+    probe = max(cores, 8)
+    t0 = time.perf_counter()
+    step(probe)
+    per_row = (time.perf_counter() - t0) / probe
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(w.batch, budget / max(per_row, 1e-9))))
+    for _ in range(args.warmup):
+        step(rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(rows)
+    dt = time.perf_counter() - t0
+    edges = sum(rows * L.inp * L.out for L in w.layers) * args.steps
+    value = edges / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} of {w.batch} rows per step of {w.name}"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w: W.Workload):
+    L0 = w.layers[0]
+    c = {"workload": w.name, "batch": w.batch, "layers": [[L.inp, L.out] for L in w.layers], "G": L0.G,
+         "grid": [L0.lo, L0.hi], "silu_base": L0.base, "mode": "fwd+bwd", "l2": "256 MiB flush between steps",
+         "note": w.note}
+    if w.dtype == "f32":
+        c["compute"] = "fp32 operands as 3 tf32 tensor-core products, fp32 accumulation"
+    else:
+        c["compute"] = "bf16 operands, fp32 accumulation"
+    return c
+
+
+def run_ours(args, world, rank, local):
+    from kolmogorov_arnold_network_b200 import _native as N
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = W.WORKLOADS[args.workload]
+    R = Runner(w, dev)
+    calls = R.calls()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        for _, c in calls:
+            c()
+    torch.cuda.synchronize(dev)
+    st = N.kan_sync_status(None)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {N.STATUS.get(st, st)}")
+
+    # ---- device-resident timed region ----
+    K = args.steps
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(K)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    n0 = N.kan_launch_count()
+    wall0 = time.perf_counter()
+    for k in range(K):
+        flush.zero_()
+        step_ev[k][0].record(stream)
+        for (a, b), (_, c) in zip(ev[k], calls):
+            a.record(stream)
+            c()
+            b.record(stream)
+        step_ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    wall = time.perf_counter() - wall0
+    launches = N.kan_launch_count() - n0
+    clocks = sampler.stop()
+    step_ms = sum(s.elapsed_time(e) for s, e in step_ev)
+    per_call = {}
+    for k in range(K):
+        for (a, b), (nm, _) in zip(ev[k], calls):
+            per_call[nm] = per_call.get(nm, 0.0) + a.elapsed_time(b)
+    t_max = step_ms
+    if world > 1:
+        t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_max = float(t.item())
+    edges = w.edges
+    value = world * edges * K / (t_max / 1000.0)
+
+    # ---- roofline of the dominant call ----
+    pk = peaks()
+    dom = max(per_call, key=per_call.get)
+    li = int(dom[-1])
+    L = w.layers[li]
+    kind = dom[:-1]
+    flops = layer_dense_flops(w.batch, L)
+    avg_s = per_call[dom] / K / 1000.0
+    if w.dtype == "bf16":
+        peak = pk["bf16"]
+        peak_note = f"bf16 dense, {pk['src']} burst"
+    else:
+        peak = pk["bf16"] * TF32_PER_BF16
+        peak_note = f"tf32 dense = {pk['src']} bf16 burst x nominal tf32/bf16 ratio {TF32_PER_BF16:.3f}"
+    achieved = flops / avg_s / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": None, "kernel": f"{kind} call of layer {li}", "peak_note": peak_note,
+            "algorithmic_flops_per_launch": flops,
+            "algorithmic_bytes_per_launch": layer_bytes(w.batch, L, 4 if w.dtype == "f32" else 2, kind),
+            "call_ms": {k: v / K for k, v in per_call.items()}}
+    if w.dtype == "f32":
+        roof["note"] = "3 tf32 products per term: the executed tensor FLOPs are 3x the algorithmic ones"
+
+    # ---- end to end: pinned host inputs in, results out, every step ----
+    e2e = None
+    if not args.no_e2e:
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        hb = db = 0
+        barrier()
+        torch.cuda.synchronize(dev)
+        for k in range(K):
+            flush.zero_()
+            e2e_ev[k][0].record(stream)
+            hb = R.h2d()
+            for _, c in calls:
+                c()
+            db = R.d2h()
+            e2e_ev[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * edges * K / (e_ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": hb,
+               "d2h_bytes_per_step": db}
+
+    st = N.kan_sync_status(None)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {N.STATUS.get(st, st)}")
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+                "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": w.dtype, "data": "synthetic", "config": config_of(w), "roofline": roof,
+                "e2e": e2e, "gpu_launches": launches, "clocks": clocks, "wall_s": wall}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=W.BENCH_DEFAULT, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup() if args.impl == "ours" else (int(os.environ.get("WORLD_SIZE", "1")),
+                                                                    int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if args.impl == "ours" and world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -133,6 +133,10 @@ KAN_API kan_status kan_sync_status(void* stream);
  * kan_sync_status() returns.  Faults and hangs nothing. */
 KAN_API kan_status kan_selftest_wait_timeout(int64_t limit_ns, void* stream);
 
+/* Number of kernels this library has launched in this process (all entry
+ * points, all devices), for accounting of the launches inside a timed region. */
+KAN_API uint64_t kan_launch_count(void);
+
 /* Static description of a status code. */
 KAN_API const char* kan_status_string(kan_status st);
 

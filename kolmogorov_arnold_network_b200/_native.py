@@ -19,6 +19,7 @@ STATUS = {0: "KAN_OK", 1: "KAN_ERR_INVALID_ARG", 2: "KAN_ERR_UNSUPPORTED", 3: "K
 
 #: every symbol the header declares
 EXPORTS = ("kan_abi_version", "kan_workspace_size", "kan_forward", "kan_backward", "kan_basis", "kan_sync_status",
+           "kan_launch_count",
            "kan_selftest_wait_timeout", "kan_status_string", "kan_last_error")
 
 
@@ -66,6 +67,8 @@ def load(path: str | None = None):
     lib.kan_status_string.argtypes = [ctypes.c_int]
     lib.kan_last_error.restype = ctypes.c_char_p
     lib.kan_last_error.argtypes = []
+    lib.kan_launch_count.restype = ctypes.c_uint64
+    lib.kan_launch_count.argtypes = []
     if path is None:
         _lib = lib
     return lib
@@ -121,3 +124,7 @@ def kan_status_string(st: int) -> str:
 
 def kan_last_error() -> str:
     return load().kan_last_error().decode()
+
+
+def kan_launch_count() -> int:
+    return int(load().kan_launch_count())

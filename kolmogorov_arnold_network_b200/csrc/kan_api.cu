@@ -5,11 +5,15 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "kan_internal.h"
 
 namespace kan {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 __device__ unsigned int g_device_status = 0;
 
@@ -248,5 +252,7 @@ const char* kan_status_string(kan_status st)
 }
 
 const char* kan_last_error(void) { return g_last_error; }
+
+uint64_t kan_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -28,6 +28,9 @@ struct Problem {
 // Device status word (defined in kan_api.cu).
 unsigned int* device_status_ptr();
 
+// Count one kernel launch (defined in kan_api.cu).
+void count_launch(int n = 1);
+
 // ---- CUDA-core kernels (kan_simt.cu) ----
 cudaError_t simt_basis(const Problem& p, const void* x, int32_t* span, float* w, float* dw, cudaStream_t st);
 cudaError_t simt_forward(const Problem& p, const void* x, const void* coef, const void* w_base, void* y,

@@ -192,11 +192,14 @@ cudaError_t simt_basis(const Problem& p, const void* x, int32_t* span, float* w,
 {
     const int64_t n = p.batch * p.in;
     if (n == 0) return cudaSuccess;
-    if (p.dtype == KAN_F32)
+    if (p.dtype == KAN_F32) {
         basis_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>((const float*)x, n, p.lo, p.inv_h, p.G, span, w, dw);
-    else
+        count_launch();
+    } else {
         basis_kernel<__nv_bfloat16><<<blocks_for(n, 256), 256, 0, st>>>((const __nv_bfloat16*)x, n, p.lo, p.inv_h,
                                                                          p.G, span, w, dw);
+        count_launch();
+    }
     return cudaGetLastError();
 }
 
@@ -206,13 +209,16 @@ cudaError_t simt_forward(const Problem& p, const void* x, const void* coef, cons
     if (p.batch == 0) return cudaSuccess;
     const int blocks = (int)((p.batch + kFwdRows - 1) / kFwdRows);
     const int threads = p.out >= 128 ? 128 : (int)((p.out + 31) / 32 * 32);
-    if (p.dtype == KAN_F32)
+    if (p.dtype == KAN_F32) {
         forward_kernel<float><<<blocks, threads, 0, st>>>((const float*)x, (const float*)coef, (const float*)w_base,
                                                           (float*)y, p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
-    else
+        count_launch();
+    } else {
         forward_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
             (const __nv_bfloat16*)x, (const __nv_bfloat16*)coef, (const __nv_bfloat16*)w_base, (__nv_bfloat16*)y,
             p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+        count_launch();
+    }
     return cudaGetLastError();
 }
 
@@ -227,25 +233,31 @@ cudaError_t simt_backward(const Problem& p, const void* x, const void* coef, con
     }
     if (dcoef || dw_base) {
         const int64_t n = p.in * p.out;
-        if (p.dtype == KAN_F32)
+        if (p.dtype == KAN_F32) {
             dcoef_kernel<float><<<blocks_for(n, 128), 128, 0, st>>>((const float*)x, (const float*)dY, dcoef, dw_base,
                                                                      p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
-        else
+            count_launch();
+        } else {
             dcoef_kernel<__nv_bfloat16><<<blocks_for(n, 128), 128, 0, st>>>(
                 (const __nv_bfloat16*)x, (const __nv_bfloat16*)dY, dcoef, dw_base, p.batch, p.in, p.out, p.G, p.lo,
                 p.inv_h);
+            count_launch();
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (dx) {
         const int64_t n = p.batch * p.in;
-        if (p.dtype == KAN_F32)
+        if (p.dtype == KAN_F32) {
             dx_kernel<float><<<blocks_for(n, 128), 128, 0, st>>>((const float*)x, (const float*)coef,
                                                                   (const float*)w_base, (const float*)dY, (float*)dx,
                                                                   p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
-        else
+            count_launch();
+        } else {
             dx_kernel<__nv_bfloat16><<<blocks_for(n, 128), 128, 0, st>>>(
                 (const __nv_bfloat16*)x, (const __nv_bfloat16*)coef, (const __nv_bfloat16*)w_base,
                 (const __nv_bfloat16*)dY, (__nv_bfloat16*)dx, p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+            count_launch();
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -253,14 +265,17 @@ cudaError_t simt_backward(const Problem& p, const void* x, const void* coef, con
 
 cudaError_t zero_f32(float* p, int64_t n, cudaStream_t st)
 {
-    if (n <= 0) return cudaSuccess;
+    if (n <= 0) return cudaSuccess; {
     zero_kernel<<<blocks_for(n, 256) > 4096 ? 4096 : blocks_for(n, 256), 256, 0, st>>>(p, n);
+    count_launch();
+    }
     return cudaGetLastError();
 }
 
 cudaError_t simt_wait_selftest(int64_t limit_ns, unsigned int* status, cudaStream_t st)
 {
     wait_selftest_kernel<<<1, 32, 0, st>>>((uint64_t)limit_ns, status);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -1,28 +1,43 @@
 // kan_tc.cu -- tensor-core (tcgen05 / TMEM / TMA) kernels of the KAN layer.
 //
 // The layer is a contraction over the dense basis expansion
-//   A[b, i*(G+3)+m] = B_m(x[b,i])            (4 non-zeros per (b,i))
+//   A[b, i*(G+3)+m] = B_m(x[b,i])            (at most 4 non-zeros per (b,i))
 // with coef viewed as a [out, in*(G+3)] matrix:
-//   y      = A . coef^T       (+ silu(x) . w_base^T)
-//   dcoef  = dY^T . A         (dw_base = dY^T . silu(x))
-//   dx     = gather of dY . coef at each input's 4 columns, times B'.
-// A never exists in global memory: producer warps evaluate the span and the
-// four weights of each input (the InKAN page's "local 4-basis lookup" and
-// stable piecewise form) and write the dense, mostly-zero A tile straight
-// into shared memory in the 128-byte-swizzled layout the tensor core reads.
-// The dense expansion is cheap on tensor cores; the per-input work stays
-// O(4) whatever G is.
+//   forward  y     = A . coef^T        (+ silu(x) . w_base^T)
+//   dcoef          = dY^T . A          (dw_base = dY^T . silu(x))
+//   dx             = sum over each input's 4 columns of (dY . coef) times B'
+//                    (+ silu'(x) * (dY . w_base))
+// A never exists in global memory: producer warps evaluate each input's span
+// and four weights (the InKAN page's "local 4-basis lookup" in its stable
+// piecewise form) and write the dense, mostly-zero A tile (or its transpose)
+// straight into shared memory in the 128-byte-swizzled layout the tensor core
+// reads.  The dense expansion costs little on tensor cores, and the per-input
+// work stays O(4) whatever G is.
 //
-// fp32 operands use three tf32 products (hi*hi + hi*lo + lo*hi) per term,
-// which keeps about 21 significant bits per product; bf16 operands use one
-// kind::f16 product.  Accumulation is fp32 in TMEM in both cases.
+// One kernel template serves the four GEMMs:
+//   FWD    A = basis rows (producers)  B = coef / w_base, K-major (TMA)
+//   DCOEF  A = basis^T (producers)     B = dY, MN-major (TMA)
+//   DX     A = dY, K-major (TMA)       B = coef, MN-major (TMA); B'-gather epilogue
+//   GEMM   A = dY, K-major (TMA)       B = w_base, MN-major (TMA); fp32 store
+// Warp roles (14 warps): 0 TMA, 1 MMA issue + TMEM allocation, 2-9 A
+// producers, 10-13 epilogue (and, for fp32, accumulator promotion).
 //
-// Deterministic by construction: every output element is reduced by one
-// CTA in a fixed order, and split-K partials are summed by a separate
-// kernel in split order.  No atomics.
+// fp32 operands: three tf32 products per term, hi*hi + hi*lo + lo*hi, which
+// keep about 21 significant bits of each product.  The tensor core's fp32
+// accumulation truncates, so long accumulations drift; the kernel therefore
+// (a) accumulates the small hi*lo + lo*hi products in their own TMEM
+// accumulator, and (b) accumulates hi*hi in short segments of `seg_kb`
+// k-blocks, alternating between two TMEM buffers, which the epilogue warps add
+// into a running fp32 total (round-to-nearest) while the next segment runs.
+// bf16 operands: one kind::f16 product, fp32 accumulation in TMEM.
+//
+// Deterministic by construction: every output element is reduced by one CTA
+// in a fixed order; split-K partials are summed by a separate kernel in
+// split order.  No atomics.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kan_device.cuh"
@@ -30,41 +45,50 @@
 namespace kan {
 namespace {
 
-constexpr int kBM = 128;                  // MMA M (rows of A / TMEM lanes)
-constexpr int kThreads = 320;             // warp 0: TMA, warp 1: MMA + TMEM, warps 2-9: producers/epilogue
-constexpr int kProducers = 256;
+constexpr int kBM = 128;          // MMA M: rows of A, TMEM lanes
+constexpr int kThreads = 448;     // 14 warps
+constexpr int kProducers = 256;   // warps 2-9
+constexpr int kEpi = 128;         // warps 10-13
 constexpr int kSmemBudget = 227 * 1024 - 2048;
+
+enum Mode { FWD = 0, DCOEF = 1, DX = 2, GEMM = 3 };
 
 template <int DT> struct Cfg;
 template <> struct Cfg<KAN_BF16> {
     using T = __nv_bfloat16;
-    static constexpr int BK = 64;         // elements per 128-byte row
+    static constexpr int BK = 64;          // K elements per 128-byte row
     static constexpr int ESZ = 2;
-    static constexpr int SPLIT = 1;       // operand copies per tile (1: plain)
-    static constexpr uint32_t FMT = 1;    // bf16
+    static constexpr int SPLIT = 1;        // operand copies (hi only)
+    static constexpr int UMMA_K = 16;
+    static constexpr uint32_t FMT = 1;     // bf16
 };
 template <> struct Cfg<KAN_F32> {
     using T = float;
     static constexpr int BK = 32;
     static constexpr int ESZ = 4;
-    static constexpr int SPLIT = 2;       // hi and lo tf32 parts
-    static constexpr uint32_t FMT = 2;    // tf32
+    static constexpr int SPLIT = 2;        // hi and lo tf32 parts
+    static constexpr int UMMA_K = 8;
+    static constexpr uint32_t FMT = 2;     // tf32
 };
 
-struct FwdArgs {
-    const void* x;
-    void* y;                   // [batch,out] operand dtype, or fp32 partials [splits,batch,out]
+struct TcArgs {
+    const void* x;             // [batch, in] operand dtype (FWD, DCOEF, DX epilogue)
+    void* out;                 // FWD: y or partials; DCOEF: dcoef or partials; DX: dx; GEMM: fp32 [batch, in]
+    float* out2;               // DCOEF: dw_base (non-partial); DX: Gb = dY.w_base (fp32 [batch,in]) or null
     unsigned int* status;
-    int64_t batch, in, out;
+    int64_t batch, in, out_f;
     int G, nb;
     float lo, inv_h;
     int Kt;                    // in * nb
-    int nkb_spline;            // k-blocks covering the spline columns
-    int nkb_total;             // + k-blocks of the SiLU columns
+    int BN, stages, seg_kb;
+    int nkb_main;              // FWD: spline k-blocks; others: k-blocks over K
+    int nkb_total;             // FWD: + SiLU k-blocks; others: = nkb_main
     int kb_per_split;
     int partial;
-    int BN;
-    int stages;
+    int n_kt_tiles;            // DCOEF: M tiles over spline rows (base tiles follow)
+    int64_t part_ld;           // DCOEF partial row length (Kt + in with base)
+    int n_in_tile;             // DX: inputs per N tile
+    int has_base;
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
@@ -99,8 +123,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Store one A element (row, column col of the k-block) into the swizzled
-// tile(s): bf16 value, or the tf32 hi/lo pair.
+// One A element at (row, col) of a K-major swizzled tile: bf16, or the tf32 hi/lo pair.
 template <int DT>
 __device__ __forceinline__ void put_a(uint32_t a_hi, uint32_t a_lo, uint32_t row, int col, float v)
 {
@@ -109,25 +132,55 @@ __device__ __forceinline__ void put_a(uint32_t a_hi, uint32_t a_lo, uint32_t row
         __nv_bfloat16 h = __float2bfloat16_rn(v);
         st_shared_u16(a_hi + off, *reinterpret_cast<uint16_t*>(&h));
     } else {
-        float hi = tf32_hi(v);
+        const float hi = tf32_hi(v);
         st_shared_f32(a_hi + off, hi);
         st_shared_f32(a_lo + off, v - hi);
     }
 }
 
-// ---------------------------------------------------------------------------
-// Forward: y[m0:m0+128, n0:n0+BN] over k-blocks [kb_begin, kb_end).
-// ---------------------------------------------------------------------------
+// 16 bytes of dense A values (8 bf16 or 4 fp32) at 16-byte chunk `chunk` of `row`.
 template <int DT>
+__device__ __forceinline__ void put_a_chunk(uint32_t a_hi, uint32_t a_lo, uint32_t row, uint32_t chunk, const float* v)
+{
+    const uint32_t off = sw128_chunk(row, chunk);
+    if constexpr (DT == KAN_BF16) {
+        st_shared_v4(a_hi + off, pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                     pack_bf16(v[6], v[7]));
+    } else {
+        float h[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            h[e] = tf32_hi(v[e]);
+            l[e] = v[e] - h[e];
+        }
+        st_shared_v4(a_hi + off, __float_as_uint(h[0]), __float_as_uint(h[1]), __float_as_uint(h[2]),
+                     __float_as_uint(h[3]));
+        st_shared_v4(a_lo + off, __float_as_uint(l[0]), __float_as_uint(l[1]), __float_as_uint(l[2]),
+                     __float_as_uint(l[3]));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+template <int MODE, int DT>
 __global__ void __launch_bounds__(kThreads, 1)
-    fwd_kernel(const __grid_constant__ CUtensorMap tm_c_hi, const __grid_constant__ CUtensorMap tm_c_lo,
-               const __grid_constant__ CUtensorMap tm_w_hi, const __grid_constant__ CUtensorMap tm_w_lo,
-               const FwdArgs a)
+    tc_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
+              const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
+              const __grid_constant__ CUtensorMap tB2_hi, const __grid_constant__ CUtensorMap tB2_lo,
+              const TcArgs a)
 {
     using C = Cfg<DT>;
     using T = typename C::T;
     constexpr int BK = C::BK;
-    constexpr int HALF = BK / 2;          // elements per producer thread per k-block (64 bytes)
+    constexpr int EPB = 128 / C::ESZ;               // elements per 128-byte row
+    constexpr bool F32 = DT == KAN_F32;
+    constexpr bool PRODUCE = MODE == FWD || MODE == DCOEF;
+    constexpr bool A_BY_TMA = MODE == DX || MODE == GEMM;
+    // B stored MN-major (dY for dcoef, coef / w_base for dx) for bf16; the
+    // fp32 path's split copies are transposed to K-major instead (tf32
+    // MN-major operands would need the 32-byte-atom swizzle).
+    constexpr bool B_MN = MODE != FWD && !F32;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
 
@@ -136,30 +189,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t stage_bytes = (a_bytes + b_bytes) * C::SPLIT;
     const uint32_t sbase = smem_addr(smem);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * stages + 1);
+    // barrier block: full_a[S] full_b[S] empty[S] zeroed[S] seg_full[2] seg_empty[2] accum
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * stages + 5);
     auto full_a = [&](int s) { return smem_addr(&bars[s]); };
     auto full_b = [&](int s) { return smem_addr(&bars[stages + s]); };
     auto empty = [&](int s) { return smem_addr(&bars[2 * stages + s]); };
-    const uint32_t accum_bar = smem_addr(&bars[3 * stages]);
+    auto zeroed = [&](int s) { return smem_addr(&bars[3 * stages + s]); };
+    auto seg_full = [&](int g) { return smem_addr(&bars[4 * stages + g]); };
+    auto seg_empty = [&](int g) { return smem_addr(&bars[4 * stages + 2 + g]); };
+    const uint32_t accum_bar = smem_addr(&bars[4 * stages + 4]);
     auto A_hi = [&](int s) { return sbase + s * stage_bytes; };
     auto A_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes; };
     auto B_hi = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT; };
     auto B_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT + b_bytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m0 = (int64_t)blockIdx.y * kBM;
-    const int n0 = blockIdx.x * BN;
     const int kb_begin = blockIdx.z * a.kb_per_split;
     const int kb_end = min(a.nkb_total, kb_begin + a.kb_per_split);
     const int nk = kb_end - kb_begin;
-    const uint32_t tmem_cols = BN < 32 ? 32 : BN;
+    const int nseg = F32 ? (nk + a.seg_kb - 1) / a.seg_kb : 1;
+    // TMEM columns: bf16 [acc]; fp32 [main0 | main1 | corr | total]
+    const uint32_t tmem_cols = F32 ? 512u : (BN <= 32 ? 32u : (BN <= 64 ? 64u : (BN <= 128 ? 128u : 256u)));
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(full_a(s), kProducers);
             mbar_init(full_b(s), 1);
             mbar_init(empty(s), 1);
+            mbar_init(zeroed(s), kProducers);
         }
+        mbar_init(seg_full(0), 1);
+        mbar_init(seg_full(1), 1);
+        mbar_init(seg_empty(0), kEpi);
+        mbar_init(seg_empty(1), kEpi);
         mbar_init(accum_bar, 1);
         fence_barrier_init();
     }
@@ -170,192 +232,375 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_main0 = tmem, t_main1 = tmem + (uint32_t)BN, t_corr = tmem + 2u * BN, t_total = tmem + 3u * BN;
+
+    // tile coordinates
+    const int64_t m0 = (int64_t)blockIdx.y * kBM;     // FWD/DX/GEMM: batch rows; DCOEF: see below
+    const int n0 = blockIdx.x * BN;                   // FWD/DCOEF/GEMM: output columns
 
     if (warp == 0) {
+        // ---------------- TMA producer ----------------
         if (lane == 0 && nk > 0) {
-            prefetch_tmap(&tm_c_hi);
-            if (C::SPLIT == 2) prefetch_tmap(&tm_c_lo);
+            prefetch_tmap(&tB_hi);
+            if (A_BY_TMA) prefetch_tmap(&tA_hi);
+            int dx_kt0 = 0;
+            if (MODE == DX) {
+                const int i0 = blockIdx.x * a.n_in_tile;
+                // a TMA column start must be 16-byte aligned; a row start need not
+                dx_kt0 = B_MN ? (i0 * a.nb) / (16 / C::ESZ) * (16 / C::ESZ) : i0 * a.nb;
+            }
             int issued = 0;
             for (int it = 0; it < nk; ++it) {
                 const int s = it % stages;
                 const uint32_t ph = (it / stages) & 1;
                 if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
                 const int kb = kb_begin + it;
-                mbar_arrive_expect_tx(full_b(s), b_bytes * C::SPLIT);
-                if (kb < a.nkb_spline) {
-                    tma_load_2d(B_hi(s), &tm_c_hi, full_b(s), kb * BK, n0);
-                    if (C::SPLIT == 2) tma_load_2d(B_lo(s), &tm_c_lo, full_b(s), kb * BK, n0);
+                const uint32_t bytes = (b_bytes + (A_BY_TMA ? a_bytes : 0u)) * C::SPLIT;
+                mbar_arrive_expect_tx(full_b(s), bytes);
+                if (MODE == FWD) {
+                    if (kb < a.nkb_main) {
+                        tma_load_2d(B_hi(s), &tB_hi, full_b(s), kb * BK, n0);
+                        if (F32) tma_load_2d(B_lo(s), &tB_lo, full_b(s), kb * BK, n0);
+                    } else {
+                        const int kc = (kb - a.nkb_main) * BK;
+                        tma_load_2d(B_hi(s), &tB2_hi, full_b(s), kc, n0);
+                        if (F32) tma_load_2d(B_lo(s), &tB2_lo, full_b(s), kc, n0);
+                    }
                 } else {
-                    const int kc = (kb - a.nkb_spline) * BK;
-                    tma_load_2d(B_hi(s), &tm_w_hi, full_b(s), kc, n0);
-                    if (C::SPLIT == 2) tma_load_2d(B_lo(s), &tm_w_lo, full_b(s), kc, n0);
+                    if (A_BY_TMA) {
+                        tma_load_2d(A_hi(s), &tA_hi, full_b(s), kb * BK, (int)m0);
+                        if (F32) tma_load_2d(A_lo(s), &tA_lo, full_b(s), kb * BK, (int)m0);
+                    }
+                    const int nbase = MODE == DX ? dx_kt0 : n0;
+                    if (B_MN) {
+                        for (int c = 0; c < BN / EPB; ++c) {
+                            const uint32_t off = (uint32_t)c * BK * 128;
+                            tma_load_2d(B_hi(s) + off, &tB_hi, full_b(s), nbase + c * EPB, kb * BK);
+                        }
+                    } else {
+                        tma_load_2d(B_hi(s), &tB_hi, full_b(s), kb * BK, nbase);
+                        if (F32) tma_load_2d(B_lo(s), &tB_lo, full_b(s), kb * BK, nbase);
+                    }
                 }
                 ++issued;
             }
-            // Drain: every load issued has landed before the CTA can exit.
+            // every load issued lands before the CTA can exit
             for (int it = max(0, issued - stages); it < issued; ++it)
                 mbar_wait(full_b(it % stages), (it / stages) & 1, a.status);
         }
     } else if (warp == 1) {
+        // ---------------- MMA issue ----------------
         if (lane == 0 && nk > 0) {
-            const uint32_t idesc = instr_desc(C::FMT, 0, 0, kBM, BN);
+            const uint32_t idesc = instr_desc(C::FMT, 0, B_MN ? 1u : 0u, kBM, BN);
+            const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
+            const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
             bool ok = true;
             for (int it = 0; it < nk && ok; ++it) {
                 const int s = it % stages;
                 const uint32_t ph = (it / stages) & 1;
-                if (!mbar_wait(full_a(s), ph, a.status) || !mbar_wait(full_b(s), ph, a.status)) {
+                if (PRODUCE && !mbar_wait(full_a(s), ph, a.status)) { ok = false; break; }
+                if (!mbar_wait(full_b(s), ph, a.status)) { ok = false; break; }
+                const int g = F32 ? it / a.seg_kb : 0;
+                const bool seg_start = F32 && (it % a.seg_kb == 0);
+                if (seg_start && g >= 2 && !mbar_wait(seg_empty(g & 1), ((g >> 1) - 1) & 1, a.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t t_main = (g & 1) ? t_main1 : t_main0;
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {   // 4 x 32 bytes of K per 128-byte row
+                for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t ad = smem_desc_sw128(A_hi(s) + ks * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(B_hi(s) + ks * 32, 16, 1024);
-                    const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
-                    if constexpr (DT == KAN_BF16) {
-                        mma_bf16_ss(tmem_base, ad, bd, idesc, acc);
+                    const uint64_t bd = smem_desc_sw128(B_hi(s) + ks * b_step, b_lbo, 1024);
+                    if constexpr (!F32) {
+                        mma_bf16_ss(t_main0, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                     } else {
                         const uint64_t adl = smem_desc_sw128(A_lo(s) + ks * 32, 16, 1024);
-                        const uint64_t bdl = smem_desc_sw128(B_lo(s) + ks * 32, 16, 1024);
-                        mma_tf32_ss(tmem_base, adl, bd, idesc, acc);
-                        mma_tf32_ss(tmem_base, ad, bdl, idesc, 1u);
-                        mma_tf32_ss(tmem_base, ad, bd, idesc, 1u);
+                        const uint64_t bdl = smem_desc_sw128(B_lo(s) + ks * b_step, b_lbo, 1024);
+                        mma_tf32_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+                        mma_tf32_ss(t_corr, ad, bdl, idesc, 1u);
+                        mma_tf32_ss(t_main, ad, bd, idesc, (!seg_start || ks > 0) ? 1u : 0u);
                     }
                 }
                 mma_commit(empty(s));
+                if (F32 && ((it + 1) % a.seg_kb == 0 || it + 1 == nk)) mma_commit(seg_full(g & 1));
             }
             if (ok) mma_commit(accum_bar);
         }
-    } else {
-        // ---------------- producers: the A tile ----------------
-        const int p = threadIdx.x - 64;
-        const uint32_t row = p & (kBM - 1);
-        const int half = p >> 7;
-        const int64_t b = m0 + row;
-        const bool row_ok = b < a.batch;
-        const T* xrow = reinterpret_cast<const T*>(a.x) + (row_ok ? b : 0) * a.in;
-        bool ok = true;
-        for (int it = 0; it < nk; ++it) {
-            const int s = it % stages;
-            const uint32_t ph = (it / stages) & 1;
-            if (!mbar_wait(empty(s), ph ^ 1, a.status)) {
-                ok = false;
-                break;
-            }
-            const int kb = kb_begin + it;
-            const uint32_t ahi = A_hi(s), alo = A_lo(s);
-            if (kb < a.nkb_spline) {
-                // zero this thread's 64 bytes, then place the non-zero weights
+    } else if (warp < 10) {
+        // ---------------- A producers ----------------
+        if constexpr (PRODUCE) {
+            const int p = threadIdx.x - 64;
+            for (int it = 0; it < nk; ++it) {
+                const int s = it % stages;
+                const uint32_t ph = (it / stages) & 1;
+                if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
+                const int kb = kb_begin + it;
+                const uint32_t ahi = A_hi(s), alo = A_lo(s);
+                if constexpr (MODE == FWD) {
+                    // rows = batch m0..m0+127, columns = spline or SiLU columns of k-block kb
+                    constexpr int HALF = BK / 2;
+                    const uint32_t row = p & (kBM - 1);
+                    const int half = p >> 7;
+                    const int64_t b = m0 + row;
+                    const bool row_ok = b < a.batch;
+                    const T* xrow = reinterpret_cast<const T*>(a.x) + (row_ok ? b : 0) * a.in;
+                    if (kb < a.nkb_main) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t off = sw128_chunk(row, half * 4 + c);
-                    st_shared_zero16(ahi + off);
-                    if (C::SPLIT == 2) st_shared_zero16(alo + off);
-                }
-                const int c_lo = kb * BK + half * HALF;       // first spline column of this thread
-                const int c_hi = min(c_lo + HALF, a.Kt);      // one past the last
-                if (row_ok && c_lo < c_hi) {
-                    const int i_first = c_lo / a.nb, i_last = (c_hi - 1) / a.nb;
-                    for (int i = i_first; i <= i_last; ++i) {
-                        const Span sp = span_of(to_f(xrow[i]), a.lo, a.inv_h, a.G);
-                        if (!sp.valid) continue;
-                        float w[4];
-                        weights(sp.t, w);
+                        for (int c = 0; c < 4; ++c) {
+                            const uint32_t off = sw128_chunk(row, half * 4 + c);
+                            st_shared_zero16(ahi + off);
+                            if (F32) st_shared_zero16(alo + off);
+                        }
+                        const int c_lo = kb * BK + half * HALF;
+                        const int c_hi = min(c_lo + HALF, a.Kt);
+                        if (row_ok && c_lo < c_hi) {
+                            const int i_first = c_lo / a.nb, i_last = (c_hi - 1) / a.nb;
+                            for (int i = i_first; i <= i_last; ++i) {
+                                const Span sp = span_of(to_f(xrow[i]), a.lo, a.inv_h, a.G);
+                                if (!sp.valid) continue;
+                                float w[4];
+                                weights(sp.t, w);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int m = sp.s + q;
-                            const int col = i * a.nb + m;
-                            if (m >= 0 && m < a.nb && col >= c_lo && col < c_hi)
-                                put_a<DT>(ahi, alo, row, col - kb * BK, w[q]);
+                                for (int q = 0; q < 4; ++q) {
+                                    const int m = sp.s + q;
+                                    const int col = i * a.nb + m;
+                                    if (m >= 0 && m < a.nb && col >= c_lo && col < c_hi)
+                                        put_a<DT>(ahi, alo, row, col - kb * BK, w[q]);
+                                }
+                            }
+                        }
+                    } else {
+                        const int i0 = (kb - a.nkb_main) * BK + half * HALF;
+                        constexpr int EPC = 16 / C::ESZ;   // elements per 16-byte chunk
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            float v[EPC];
+#pragma unroll
+                            for (int e = 0; e < EPC; ++e) {
+                                const int i = i0 + c * EPC + e;
+                                v[e] = (row_ok && i < a.in) ? silu_f(to_f(xrow[i])) : 0.0f;
+                            }
+                            put_a_chunk<DT>(ahi, alo, row, half * 4 + c, v);
                         }
                     }
-                }
-            } else {
-                // SiLU columns: dense
-                const int i0 = (kb - a.nkb_spline) * BK + half * HALF;
-                float v[HALF];
-#pragma unroll
-                for (int c = 0; c < HALF; ++c) {
-                    const int i = i0 + c;
-                    v[c] = (row_ok && i < a.in) ? silu_f(to_f(xrow[i])) : 0.0f;
-                }
-                if constexpr (DT == KAN_BF16) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        st_shared_v4(ahi + sw128_chunk(row, half * 4 + c), pack_bf16(v[8 * c], v[8 * c + 1]),
-                                     pack_bf16(v[8 * c + 2], v[8 * c + 3]), pack_bf16(v[8 * c + 4], v[8 * c + 5]),
-                                     pack_bf16(v[8 * c + 6], v[8 * c + 7]));
                 } else {
+                    // DCOEF: rows = spline columns kt0..kt0+127 (or inputs for SiLU tiles),
+                    // columns = batch rows b0..b0+BK-1
+                    const int64_t b0 = (int64_t)kb * BK;
+                    const int mt = blockIdx.y;
+                    if (mt < a.n_kt_tiles) {
+                        const int kt0 = mt * kBM;
+                        // zero the tile: 128 rows x 8 chunks, 4 chunks per thread
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float h[4], l[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            h[e] = tf32_hi(v[4 * c + e]);
-                            l[e] = v[4 * c + e] - h[e];
+                        for (int c = 0; c < 4; ++c) {
+                            const int e = p * 4 + c;
+                            const uint32_t off = sw128_chunk(e >> 3, e & 7);
+                            st_shared_zero16(ahi + off);
+                            if (F32) st_shared_zero16(alo + off);
                         }
-                        const uint32_t off = sw128_chunk(row, half * 4 + c);
-                        st_shared_v4(ahi + off, __float_as_uint(h[0]), __float_as_uint(h[1]), __float_as_uint(h[2]),
-                                     __float_as_uint(h[3]));
-                        st_shared_v4(alo + off, __float_as_uint(l[0]), __float_as_uint(l[1]), __float_as_uint(l[2]),
-                                     __float_as_uint(l[3]));
+                        // every producer's zeros are in place before anyone scatters
+                        mbar_arrive(zeroed(s));
+                        if (!mbar_wait(zeroed(s), ph, a.status)) break;
+                        const int i_first = kt0 / a.nb;
+                        const int i_last = min((int)a.in - 1, (kt0 + kBM - 1) / a.nb);
+                        const int n_pairs = BK * (i_last - i_first + 1);
+                        for (int e = p; e < n_pairs; e += kProducers) {
+                            const int c = e % BK;
+                            const int i = i_first + e / BK;
+                            const int64_t b = b0 + c;
+                            if (b >= a.batch) continue;
+                            const Span sp = span_of(to_f(reinterpret_cast<const T*>(a.x)[b * a.in + i]), a.lo,
+                                                    a.inv_h, a.G);
+                            if (!sp.valid) continue;
+                            float w[4];
+                            weights(sp.t, w);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const int m = sp.s + q;
+                                const int r = i * a.nb + m - kt0;
+                                if (m >= 0 && m < a.nb && r >= 0 && r < kBM) put_a<DT>(ahi, alo, (uint32_t)r, c, w[q]);
+                            }
+                        }
+                    } else {
+                        // SiLU rows: inputs i0..i0+127, dense
+                        const int i0 = (mt - a.n_kt_tiles) * kBM;
+                        constexpr int EPC = 16 / C::ESZ;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int e = p * 4 + c;
+                            const int r = e >> 3, ch = e & 7;
+                            const int64_t i = i0 + r;
+                            float v[EPC];
+#pragma unroll
+                            for (int q = 0; q < EPC; ++q) {
+                                const int64_t b = b0 + ch * EPC + q;
+                                v[q] = (i < a.in && b < a.batch)
+                                           ? silu_f(to_f(reinterpret_cast<const T*>(a.x)[b * a.in + i]))
+                                           : 0.0f;
+                            }
+                            put_a_chunk<DT>(ahi, alo, (uint32_t)r, (uint32_t)ch, v);
+                        }
                     }
                 }
+                fence_async_smem();
+                mbar_arrive(full_a(s));
             }
-            fence_async_smem();
-            mbar_arrive(full_a(s));
         }
-
-        // ---------------- epilogue: TMEM -> y ----------------
-        // tcgen05.ld is warp-collective: decide per warp, not per lane
-        bool go = __all_sync(0xffffffffu, ok && nk > 0);
+    } else {
+        // ---------------- epilogue warps 10-13 ----------------
+        const int q = warp & 3;                       // TMEM lane quarter
+        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+        const uint32_t r = 32 * q + lane;             // tile row of this thread
+        bool go = nk > 0;
+        if (F32 && go) {
+            // promotion: total (+)= main[g & 1] for every segment
+            for (int g = 0; g < nseg && go; ++g) {
+                go = __all_sync(0xffffffffu, mbar_wait(seg_full(g & 1), (g >> 1) & 1, a.status));
+                if (!go) break;
+                tc_fence_after();
+                const uint32_t tm = ((g & 1) ? t_main1 : t_main0) + lane_off;
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    uint32_t v[16], t[16];
+                    tmem_ld16(tm + c0, v);
+                    if (g > 0) tmem_ld16(t_total + lane_off + c0, t);
+                    tmem_ld_wait();
+                    if (g > 0) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(t[e]));
+                    }
+                    tmem_st16(t_total + lane_off + c0, v);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(seg_empty(g & 1));
+            }
+        }
         if (go) go = __all_sync(0xffffffffu, mbar_wait(accum_bar, 0, a.status));
         if (go) {
             tc_fence_after();
-            const int q = warp & 3;                 // TMEM lane quarter of this warp
-            const int chalf = (warp - 2) >> 2;      // which half of the columns
-            const uint32_t r = 32 * q + lane;
-            const int64_t bo = m0 + r;
-            const int cbeg = chalf * (BN / 2), cend = cbeg + BN / 2;
-            for (int c0 = cbeg; c0 < cend; c0 += 16) {
+            // value of accumulator column c0..c0+15 of this thread's row
+            auto load16 = [&](int c0, float (&out)[16]) {
                 uint32_t v[16];
-                tmem_ld16(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
-                tmem_ld_wait();
-                if (bo >= a.batch) continue;
-                const int64_t j0 = n0 + c0;
-                if (a.partial) {
-                    float* dst = reinterpret_cast<float*>(a.y) + ((int64_t)blockIdx.z * a.batch + bo) * a.out + j0;
-                    if (j0 + 16 <= a.out) {
+                if constexpr (F32) {
+                    uint32_t w[16];
+                    tmem_ld16(t_total + lane_off + c0, v);
+                    tmem_ld16(t_corr + lane_off + c0, w);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 16; e += 4)
-                            *reinterpret_cast<uint4*>(dst + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                    } else {
-                        for (int e = 0; e < 16 && j0 + e < a.out; ++e) dst[e] = __uint_as_float(v[e]);
-                    }
+                    for (int e = 0; e < 16; ++e) out[e] = __uint_as_float(v[e]) + __uint_as_float(w[e]);
                 } else {
-                    T* dst = reinterpret_cast<T*>(a.y) + bo * a.out + j0;
-                    if constexpr (DT == KAN_BF16) {
-                        if (j0 + 16 <= a.out) {
-                            uint32_t pk[8];
+                    tmem_ld16(t_main0 + lane_off + c0, v);
+                    tmem_ld_wait();
 #pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                pk[e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                            *reinterpret_cast<uint4*>(dst + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                        } else {
-                            for (int e = 0; e < 16 && j0 + e < a.out; ++e)
-                                dst[e] = __float2bfloat16_rn(__uint_as_float(v[e]));
-                        }
-                    } else {
-                        if (j0 + 16 <= a.out) {
+                    for (int e = 0; e < 16; ++e) out[e] = __uint_as_float(v[e]);
+                }
+            };
+
+            if constexpr (MODE == FWD || MODE == GEMM) {
+                const int64_t bo = m0 + r;
+                const int64_t ncols = MODE == FWD ? a.out_f : a.in;
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    float v[16];
+                    load16(c0, v);
+                    if (bo >= a.batch) continue;
+                    const int64_t j0 = n0 + c0;
+                    if (MODE == GEMM || a.partial) {
+                        float* dst = reinterpret_cast<float*>(a.out) +
+                                     ((MODE == FWD ? (int64_t)blockIdx.z * a.batch : 0) + bo) * ncols + j0;
+                        if (j0 + 16 <= ncols && (ncols & 3) == 0) {
 #pragma unroll
                             for (int e = 0; e < 16; e += 4)
-                                *reinterpret_cast<uint4*>(dst + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                                *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                         } else {
-                            for (int e = 0; e < 16 && j0 + e < a.out; ++e) dst[e] = __uint_as_float(v[e]);
+                            for (int e = 0; e < 16 && j0 + e < ncols; ++e) dst[e] = v[e];
                         }
+                    } else {
+                        T* dst = reinterpret_cast<T*>(a.out) + bo * ncols + j0;
+                        if constexpr (!F32) {
+                            if (j0 + 16 <= ncols) {
+                                uint32_t pk[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+                                *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                                *reinterpret_cast<uint4*>(dst + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                            } else {
+                                for (int e = 0; e < 16 && j0 + e < ncols; ++e) dst[e] = __float2bfloat16_rn(v[e]);
+                            }
+                        } else {
+                            if (j0 + 16 <= ncols) {
+#pragma unroll
+                                for (int e = 0; e < 16; e += 4)
+                                    *reinterpret_cast<float4*>(dst + e) =
+                                        make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                            } else {
+                                for (int e = 0; e < 16 && j0 + e < ncols; ++e) dst[e] = v[e];
+                            }
+                        }
+                    }
+                }
+            } else if constexpr (MODE == DCOEF) {
+                // rows are spline columns kt (or inputs of a SiLU tile); columns are outputs j
+                const int mt = blockIdx.y;
+                const bool base_tile = mt >= a.n_kt_tiles;
+                const int64_t rowg = base_tile ? (int64_t)(mt - a.n_kt_tiles) * kBM + r : (int64_t)mt * kBM + r;
+                const bool row_ok = base_tile ? rowg < a.in : rowg < a.Kt;
+                float* dst;
+                int64_t ld;
+                if (a.partial) {
+                    dst = reinterpret_cast<float*>(a.out) + (int64_t)blockIdx.z * a.out_f * a.part_ld +
+                          (base_tile ? a.Kt + rowg : rowg);
+                    ld = a.part_ld;
+                } else {
+                    float* basep = base_tile ? a.out2 : reinterpret_cast<float*>(a.out);
+                    dst = basep ? basep + rowg : nullptr;   // an output the caller skipped
+                    ld = base_tile ? a.in : a.Kt;
+                }
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    float v[16];
+                    load16(c0, v);
+                    if (!row_ok || !dst) continue;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int64_t j = n0 + c0 + e;
+                        if (j < a.out_f) dst[j * ld] = v[e];
+                    }
+                }
+            } else {
+                // DX: Gm row -> shared staging (the pipeline buffers are free now),
+                // then each input's 4 columns times B' (+ silu' * Gb).
+                const int ldst = BN + 1;
+                float* stage = reinterpret_cast<float*>(smem) + (size_t)(warp - 10) * 32 * ldst + (size_t)lane * ldst;
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    float v[16];
+                    load16(c0, v);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) stage[c0 + e] = v[e];
+                }
+                const int64_t b = m0 + r;
+                if (b < a.batch) {
+                    const int i0 = blockIdx.x * a.n_in_tile;
+                    const int kt_al = B_MN ? (i0 * a.nb) / (16 / C::ESZ) * (16 / C::ESZ) : i0 * a.nb;
+                    const int i1 = min((int)a.in, i0 + a.n_in_tile);
+                    const T* xr = reinterpret_cast<const T*>(a.x) + b * a.in;
+                    T* dxr = reinterpret_cast<T*>(a.out) + b * a.in;
+                    for (int i = i0; i < i1; ++i) {
+                        const float xv = to_f(xr[i]);
+                        const Span sp = span_of(xv, a.lo, a.inv_h, a.G);
+                        float acc = 0.0f;
+                        if (sp.valid) {
+                            float d[4];
+                            dweights(sp.t, a.inv_h, d);
+                            const int cb = i * a.nb - kt_al;
+#pragma unroll
+                            for (int qq = 0; qq < 4; ++qq) {
+                                const int m = sp.s + qq;
+                                if (m >= 0 && m < a.nb) acc += stage[cb + m] * d[qq];
+                            }
+                        }
+                        if (a.has_base) acc += dsilu_f(xv) * a.out2[b * a.in + i];
+                        dxr[i] = from_f<T>(acc);
                     }
                 }
             }
@@ -366,11 +611,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, tmem_cols);
+        tmem_dealloc(tmem, tmem_cols);
     }
 }
 
-// y[b, j] = sum over splits z (ascending) of part[z, b, j].
+// y[e] = sum over splits z (ascending) of part[z][e].
 template <typename T>
 __global__ void reduce_splits_kernel(const float* __restrict__ part, T* __restrict__ y, int64_t n, int splits)
 {
@@ -381,15 +626,56 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, T* __restri
     }
 }
 
+// dcoef[j, kt] and dw_base[j, i] from partials [splits][out][Kt (+ in)], split order.
+__global__ void reduce_dcoef_kernel(const float* __restrict__ part, float* __restrict__ dcoef,
+                                    float* __restrict__ dw_base, int64_t out, int64_t Kt, int64_t in, int64_t ld,
+                                    int splits)
+{
+    const int64_t n = out * ld;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t j = e / ld, c = e % ld;
+        float acc = 0.f;
+        for (int z = 0; z < splits; ++z) acc += part[(int64_t)z * n + e];
+        if (c < Kt) {
+            if (dcoef) dcoef[j * Kt + c] = acc;
+        } else if (dw_base) {
+            dw_base[j * in + (c - Kt)] = acc;
+        }
+    }
+}
+
 // hi/lo tf32 split of an fp32 array.
 __global__ void split_tf32_kernel(const float* __restrict__ src, float* __restrict__ hi, float* __restrict__ lo,
                                   int64_t n)
 {
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        float v = src[e];
-        float h = tf32_hi(v);
+        const float v = src[e];
+        const float h = tf32_hi(v);
         hi[e] = h;
         lo[e] = v - h;
+    }
+}
+
+// hi/lo tf32 split of a row-major fp32 [R, C] matrix, written transposed:
+// hi[c * ldo + r], lo[c * ldo + r] (ldo >= R), through a 32x32 shared tile.
+__global__ void split_tf32_t_kernel(const float* __restrict__ src, int64_t R, int64_t C, float* __restrict__ hi,
+                                    float* __restrict__ lo, int64_t ldo)
+{
+    __shared__ float tile[32][33];
+    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+    for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+        const int64_t r = r0 + k, c = c0 + threadIdx.x;
+        tile[k][threadIdx.x] = (r < R && c < C) ? src[r * C + c] : 0.0f;
+    }
+    __syncthreads();
+    for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+        const int64_t c = c0 + k, r = r0 + threadIdx.x;
+        if (c < C && r < R) {
+            const float v = tile[threadIdx.x][k];
+            const float h = tf32_hi(v);
+            hi[c * ldo + r] = h;
+            lo[c * ldo + r] = v - h;
+        }
     }
 }
 
@@ -410,10 +696,10 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
     return fn;
 }
 
-// 2-D tiled map over a row-major [rows, cols] matrix; box = [box_rows, box_cols],
-// 128-byte swizzle (box_cols * esize must be 128), zero fill out of bounds.
+// 2-D tiled map over a row-major [rows, cols] matrix; box = [box_rows, box_cols]
+// with box_cols * esize = 128 bytes, 128-byte swizzle, zero fill out of bounds.
 bool make_map_2d(CUtensorMap* m, const void* base, bool f32, int64_t rows, int64_t cols, int box_rows, int box_cols,
-                 const char** detail)
+                 const char** detail, int64_t ld = -1)
 {
     auto enc = get_encoder();
     if (!enc) {
@@ -422,7 +708,7 @@ bool make_map_2d(CUtensorMap* m, const void* base, bool f32, int64_t rows, int64
     }
     const int esz = f32 ? 4 : 2;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)(cols * esz)};
+    cuuint64_t strides[1] = {(cuuint64_t)((ld > 0 ? ld : cols) * esz)};
     cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
@@ -436,68 +722,225 @@ bool make_map_2d(CUtensorMap* m, const void* base, bool f32, int64_t rows, int64
 }
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
-inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-struct FwdPlan {
-    int BN, stages, n_tiles, m_tiles, splits, kb_per_split, nkb_spline, nkb_total;
-    size_t ws_split_coef;   // bytes of tf32 hi/lo copies of coef and w_base
-    size_t ws_partial;      // bytes of split partials
+// Split count minimising ceil(tiles*s / sms) / s (waves per unit of work), s <= cap.
+int pick_splits(int64_t tiles, int sms, int cap)
+{
+    int best = 1;
+    double best_cost = 1e30;
+    for (int s = 1; s <= std::max(1, cap); ++s) {
+        const double cost = (double)cdiv(tiles * s, sms) / s + 0.02 * (s - 1);  // small price per extra split
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
+}
+
+// Tile width over n output columns.  An MN-major bf16 B operand is loaded in
+// 64-column (128-byte) boxes, so its tile is at least one box wide.
+int bn_for(int64_t n, bool f32, bool mn_major = false)
+{
+    const int cap = f32 ? 128 : 256;
+    int bn = (mn_major && !f32) ? 64 : 32;
+    while (bn < n && bn < cap) bn *= 2;
+    return bn;
+}
+
+int stages_for(int BN, bool f32)
+{
+    const int stage_bytes = (kBM * 128 + BN * 128) * (f32 ? 2 : 1);
+    return std::min(8, (kSmemBudget - 1024 - 512) / stage_bytes);
+}
+
+// pipeline stages + 1024 alignment slack + 512 for the barrier block (4*stages+5 mbarriers) and the TMEM slot
+int smem_bytes(int BN, int stages, bool f32) { return stages * (kBM * 128 + BN * 128) * (f32 ? 2 : 1) + 1024 + 512; }
+
+constexpr int kSegKb = 2;   // fp32: k-blocks per promoted accumulation segment
+
+// Workspace layout, shared by the size query and the launches.
+struct Layout {
+    size_t coef_hl = 0, wb_hl = 0, dy_hl = 0;   // tf32 hi/lo copies (fp32 only)
+    size_t dyt_hl = 0;                           // tf32 hi/lo of dY^T [out][ldb] (fp32 backward)
+    size_t fwd_part = 0, dc_part = 0, gb = 0;   // split partials and dY.w_base
+    size_t total = 0;
 };
 
-int pick_bn(int64_t out)
-{
-    if (out <= 32) return 32;
-    if (out <= 64) return 64;
-    if (out <= 128) return 128;
-    return 256;
-}
+struct Plan {
+    // forward
+    int f_BN, f_stages, f_n, f_m, f_splits, f_kps, f_nkb_main, f_nkb_total;
+    // dcoef
+    int d_BN, d_stages, d_n, d_m, d_nkt, d_splits, d_kps, d_nkb;
+    int64_t d_ld;
+    int64_t ldb;   // padded row length of dY^T (fp32)
+    // dx
+    int x_BN, x_stages, x_n, x_m, x_nin, x_nkb;
+    // dY . w_base
+    int g_BN, g_stages, g_n, g_m;
+    Layout fwd, bwd;
+};
 
-FwdPlan plan_forward(const Problem& p, int num_sms)
+Plan make_plan(const Problem& p, int sms)
 {
-    FwdPlan f{};
+    Plan P{};
     const bool f32 = p.dtype == KAN_F32;
     const int BK = f32 ? 32 : 64;
-    const int split = f32 ? 2 : 1;
-    f.BN = pick_bn(p.out);
-    const int stage_bytes = (kBM * 128 + f.BN * 128) * split;
-    f.stages = std::min(8, (kSmemBudget - 1024 - 256) / stage_bytes);
-    f.n_tiles = (int)cdiv(p.out, f.BN);
-    f.m_tiles = (int)cdiv(p.batch, kBM);
-    f.nkb_spline = (int)cdiv(p.Kt, BK);
-    f.nkb_total = f.nkb_spline + (p.base ? (int)cdiv(p.in, BK) : 0);
-    const int64_t tiles = (int64_t)f.n_tiles * f.m_tiles;
-    int splits = 1;
-    if (tiles < num_sms) {
-        splits = (int)std::max<int64_t>(1, num_sms / std::max<int64_t>(1, tiles));
-        splits = std::min<int>(splits, std::max(1, f.nkb_total / 4));
+    const int EPB = f32 ? 32 : 64;
+    const size_t esz = f32 ? 4 : 2;
+    // forward: M = batch, N = out, K = spline (+ SiLU) columns
+    P.f_BN = bn_for(p.out, f32);
+    P.f_stages = stages_for(P.f_BN, f32);
+    P.f_n = (int)cdiv(p.out, P.f_BN);
+    P.f_m = (int)cdiv(p.batch, kBM);
+    P.f_nkb_main = (int)cdiv(p.Kt, BK);
+    P.f_nkb_total = P.f_nkb_main + (p.base ? (int)cdiv(p.in, BK) : 0);
+    P.f_splits = pick_splits((int64_t)P.f_n * P.f_m, sms, std::min(16, std::max(1, P.f_nkb_total / 8)));
+    P.f_kps = (int)cdiv(P.f_nkb_total, P.f_splits);
+    P.f_splits = (int)cdiv(P.f_nkb_total, P.f_kps);
+    // dcoef: M = spline columns (+ SiLU rows), N = out, K = batch
+    P.d_BN = bn_for(p.out, f32, true);
+    P.d_stages = stages_for(P.d_BN, f32);
+    P.d_n = (int)cdiv(p.out, P.d_BN);
+    P.d_nkt = (int)cdiv(p.Kt, kBM);
+    P.d_m = P.d_nkt + (p.base ? (int)cdiv(p.in, kBM) : 0);
+    P.d_nkb = (int)cdiv(p.batch, BK);
+    P.d_splits = pick_splits((int64_t)P.d_n * P.d_m, sms, std::min(16, std::max(1, P.d_nkb / 8)));
+    P.d_kps = (int)cdiv(std::max(1, P.d_nkb), P.d_splits);
+    P.d_splits = (int)cdiv(std::max(1, P.d_nkb), P.d_kps);
+    P.d_ld = p.Kt + (p.base ? p.in : 0);
+    // dx: M = batch, N = whole inputs' spline columns, K = out
+    P.x_BN = f32 ? 128 : 256;
+    P.x_stages = stages_for(P.x_BN, f32);
+    // bf16: coef is read MN-major and a tile's first column is rounded down to
+    // 16 bytes; fp32: coef^T is read K-major, any first row works
+    const int maxoff = f32 ? 0 : ((p.nb % 8 == 0) ? 0 : 7);
+    P.x_nin = std::max(1, (P.x_BN - maxoff) / p.nb);
+    P.x_n = (int)cdiv(p.in, P.x_nin);
+    P.x_m = (int)cdiv(p.batch, kBM);
+    P.x_nkb = (int)cdiv(p.out, BK);
+    // dY . w_base: M = batch, N = in, K = out
+    P.g_BN = bn_for(p.in, f32, true);
+    P.g_stages = stages_for(P.g_BN, f32);
+    P.g_n = (int)cdiv(p.in, P.g_BN);
+    P.g_m = P.x_m;
+
+    // workspace, forward
+    size_t o = 0;
+    if (f32) {
+        P.fwd.coef_hl = o;
+        o += 2 * al256((size_t)p.out * p.Kt * 4);
+        if (p.base) {
+            P.fwd.wb_hl = o;
+            o += 2 * al256((size_t)p.out * p.in * 4);
+        }
     }
-    f.kb_per_split = (int)cdiv(f.nkb_total, splits);
-    f.splits = (int)cdiv(f.nkb_total, f.kb_per_split);
-    f.ws_split_coef = f32 ? align256((size_t)p.out * p.Kt * 4) * 2 + (p.base ? align256((size_t)p.out * p.in * 4) * 2 : 0)
-                          : 0;
-    f.ws_partial = f.splits > 1 ? align256((size_t)f.splits * p.batch * p.out * 4) : 0;
-    return f;
-}
-
-int smem_bytes_for(const FwdPlan& f, bool f32)
-{
-    const int split = f32 ? 2 : 1;
-    return f.stages * (kBM * 128 + f.BN * 128) * split + 1024 + 256;
-}
-
-template <int DT>
-cudaError_t launch_fwd(const FwdPlan& f, const CUtensorMap& ch, const CUtensorMap& cl, const CUtensorMap& wh,
-                       const CUtensorMap& wl, const FwdArgs& args, cudaStream_t st)
-{
-    const int smem = smem_bytes_for(f, DT == KAN_F32);
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(f.n_tiles, f.m_tiles, f.splits);
-    fwd_kernel<DT><<<grid, kThreads, smem, st>>>(ch, cl, wh, wl, args);
-    return cudaGetLastError();
+    if (P.f_splits > 1) {
+        P.fwd.fwd_part = o;
+        o += al256((size_t)P.f_splits * p.batch * p.out * 4);
+    }
+    P.fwd.total = o;
+    // workspace, backward (fp32: coef^T, w_base^T, dY and dY^T as tf32 hi/lo)
+    o = 0;
+    P.ldb = (p.batch + 3) / 4 * 4;
+    if (f32) {
+        P.bwd.coef_hl = o;
+        o += 2 * al256((size_t)p.out * p.Kt * 4);
+        if (p.base) {
+            P.bwd.wb_hl = o;
+            o += 2 * al256((size_t)p.out * p.in * 4);
+        }
+        P.bwd.dy_hl = o;
+        o += 2 * al256((size_t)p.batch * p.out * 4);
+        P.bwd.dyt_hl = o;
+        o += 2 * al256((size_t)p.out * P.ldb * 4);
+    }
+    if (P.d_splits > 1) {
+        P.bwd.dc_part = o;
+        o += al256((size_t)P.d_splits * p.out * P.d_ld * 4);
+    }
+    if (p.base) {
+        P.bwd.gb = o;
+        o += al256((size_t)p.batch * p.in * 4);
+    }
+    P.bwd.total = o;
+    (void)esz;
+    return P;
 }
 
 inline int grid_for(int64_t n) { return (int)std::min<int64_t>(std::max<int64_t>(1, (n + 255) / 256), 148 * 8); }
+
+template <int MODE, int DT>
+cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args, cudaStream_t st)
+{
+    // the MN-major bf16 B operand arrives in whole 128-byte boxes: BN must be a multiple of 64
+    if (MODE != FWD && DT == KAN_BF16 && BN % 64 != 0) return cudaErrorInvalidConfiguration;
+    if (BN % 16 != 0 || BN < 16 || BN > 256 || (DT == KAN_F32 && BN > 128) || stages < 2)
+        return cudaErrorInvalidConfiguration;
+    const int smem = smem_bytes(BN, stages, DT == KAN_F32);
+    static int configured = 0;   // per instantiation; the attribute is per function
+    if (configured < smem) {
+        cudaError_t e = cudaFuncSetAttribute(tc_kernel<MODE, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemBudget);
+        if (e != cudaSuccess) return e;
+        configured = kSmemBudget;
+    }
+    tc_kernel<MODE, DT><<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], args);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
+                      cudaStream_t st)
+{
+    return f32 ? launch<MODE, KAN_F32>(grid, BN, stages, maps, args, st)
+               : launch<MODE, KAN_BF16>(grid, BN, stages, maps, args, st);
+}
+
+TcArgs base_args(const Problem& p)
+{
+    TcArgs a{};
+    a.status = device_status_ptr();
+    a.batch = p.batch;
+    a.in = p.in;
+    a.out_f = p.out;
+    a.G = p.G;
+    a.nb = p.nb;
+    a.lo = p.lo;
+    a.inv_h = p.inv_h;
+    a.Kt = (int)p.Kt;
+    a.seg_kb = kSegKb;
+    a.has_base = p.base;
+    return a;
+}
+
+// tf32 hi/lo copies of an fp32 array; returns the (hi, lo) pointers.
+cudaError_t split_into(const void* src, int64_t n, uint8_t* dst, const void** hi, const void** lo, cudaStream_t st)
+{
+    float* h = reinterpret_cast<float*>(dst);
+    float* l = reinterpret_cast<float*>(dst + al256((size_t)n * 4));
+    split_tf32_kernel<<<grid_for(n), 256, 0, st>>>((const float*)src, h, l, n);
+    count_launch();
+    *hi = h;
+    *lo = l;
+    return cudaGetLastError();
+}
+
+// tf32 hi/lo copies of a row-major [R, C] fp32 matrix, transposed to [C][ldo].
+cudaError_t split_t_into(const void* src, int64_t R, int64_t C, int64_t ldo, uint8_t* dst, const void** hi,
+                         const void** lo, cudaStream_t st)
+{
+    float* h = reinterpret_cast<float*>(dst);
+    float* l = reinterpret_cast<float*>(dst + al256((size_t)C * ldo * 4));
+    dim3 grid((unsigned)cdiv(C, 32), (unsigned)cdiv(R, 32));
+    split_tf32_t_kernel<<<grid, dim3(32, 8), 0, st>>>((const float*)src, R, C, h, l, ldo);
+    count_launch();
+    *hi = h;
+    *lo = l;
+    return cudaGetLastError();
+}
 
 }  // namespace
 
@@ -505,7 +948,7 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
 {
     const int esz = p.dtype == KAN_F32 ? 4 : 2;
     if ((p.Kt * esz) % 16 != 0) {
-        *why = "in*(G+3)*sizeof(dtype) is not a multiple of 16 bytes (TMA row stride)";
+        *why = "in*(G+3)*sizeof(dtype) is not a multiple of 16 bytes (TMA row stride of coef)";
         return false;
     }
     if (p.base && (p.in * esz) % 16 != 0) {
@@ -513,10 +956,14 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
         return false;
     }
     if ((p.out * esz) % 16 != 0) {
-        *why = "out*sizeof(dtype) is not a multiple of 16 bytes";
+        *why = "out*sizeof(dtype) is not a multiple of 16 bytes (TMA row stride of dY, vector stores of y)";
         return false;
     }
-    if (p.Kt > (int64_t)1 << 30 || p.batch > ((int64_t)1 << 31) - 256) {
+    if (p.nb > (p.dtype == KAN_F32 ? 125 : 249)) {
+        *why = "G too large for one dx tile (G+3 must fit the tile with its alignment offset)";
+        return false;
+    }
+    if (p.Kt + p.in > ((int64_t)1 << 30) || p.batch > ((int64_t)1 << 31) - 256 || p.out > ((int64_t)1 << 30)) {
         *why = "problem too large for 32-bit tile coordinates";
         return false;
     }
@@ -524,102 +971,181 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
     return true;
 }
 
-size_t tc_workspace_forward(const Problem& p, int num_sms)
-{
-    FwdPlan f = plan_forward(p, num_sms);
-    return f.ws_split_coef + f.ws_partial;
-}
+size_t tc_workspace_forward(const Problem& p, int num_sms) { return make_plan(p, num_sms).fwd.total; }
+size_t tc_workspace_backward(const Problem& p, int num_sms) { return make_plan(p, num_sms).bwd.total; }
 
 cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const void* w_base, void* y, void* ws,
                        int num_sms, cudaStream_t st, const char** detail)
 {
     if (p.batch == 0) return cudaSuccess;
     const bool f32 = p.dtype == KAN_F32;
-    FwdPlan f = plan_forward(p, num_sms);
-    uint8_t* wsp = reinterpret_cast<uint8_t*>(ws);
-    const void *c_hi = coef, *c_lo = coef, *w_hi = w_base ? w_base : coef, *w_lo = w_hi;
+    const int BK = f32 ? 32 : 64;
+    const Plan P = make_plan(p, num_sms);
+    uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+    const void *c_hi = coef, *c_lo = coef, *wb_hi = w_base, *wb_lo = w_base;
     cudaError_t e;
     if (f32) {
-        float* ch = reinterpret_cast<float*>(wsp);
-        float* cl = reinterpret_cast<float*>(wsp + align256((size_t)p.out * p.Kt * 4));
-        split_tf32_kernel<<<grid_for(p.out * p.Kt), 256, 0, st>>>((const float*)coef, ch, cl, p.out * p.Kt);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        c_hi = ch;
-        c_lo = cl;
-        w_hi = ch;
-        w_lo = cl;
-        if (p.base) {
-            uint8_t* wb0 = wsp + align256((size_t)p.out * p.Kt * 4) * 2;
-            float* wh = reinterpret_cast<float*>(wb0);
-            float* wl = reinterpret_cast<float*>(wb0 + align256((size_t)p.out * p.in * 4));
-            split_tf32_kernel<<<grid_for(p.out * p.in), 256, 0, st>>>((const float*)w_base, wh, wl, p.out * p.in);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            w_hi = wh;
-            w_lo = wl;
-        }
-        wsp += f.ws_split_coef;
+        if ((e = split_into(coef, p.out * p.Kt, w + P.fwd.coef_hl, &c_hi, &c_lo, st)) != cudaSuccess) return e;
+        if (p.base && (e = split_into(w_base, p.out * p.in, w + P.fwd.wb_hl, &wb_hi, &wb_lo, st)) != cudaSuccess)
+            return e;
     }
-    const int BK = f32 ? 32 : 64;
-    CUtensorMap m_ch, m_cl, m_wh, m_wl;
-    if (!make_map_2d(&m_ch, c_hi, f32, p.out, p.Kt, f.BN, BK, detail) ||
-        !make_map_2d(&m_cl, c_lo, f32, p.out, p.Kt, f.BN, BK, detail))
+    CUtensorMap maps[6];
+    if (!make_map_2d(&maps[2], c_hi, f32, p.out, p.Kt, P.f_BN, BK, detail) ||
+        !make_map_2d(&maps[3], c_lo, f32, p.out, p.Kt, P.f_BN, BK, detail))
         return cudaErrorInvalidValue;
     if (p.base) {
-        if (!make_map_2d(&m_wh, w_hi, f32, p.out, p.in, f.BN, BK, detail) ||
-            !make_map_2d(&m_wl, w_lo, f32, p.out, p.in, f.BN, BK, detail))
+        if (!make_map_2d(&maps[4], wb_hi, f32, p.out, p.in, P.f_BN, BK, detail) ||
+            !make_map_2d(&maps[5], wb_lo, f32, p.out, p.in, P.f_BN, BK, detail))
             return cudaErrorInvalidValue;
     } else {
-        m_wh = m_ch;
-        m_wl = m_cl;
+        maps[4] = maps[2];
+        maps[5] = maps[3];
     }
-    FwdArgs args{};
-    args.x = x;
-    args.y = f.splits > 1 ? (void*)wsp : y;
-    args.status = device_status_ptr();
-    args.batch = p.batch;
-    args.in = p.in;
-    args.out = p.out;
-    args.G = p.G;
-    args.nb = p.nb;
-    args.lo = p.lo;
-    args.inv_h = p.inv_h;
-    args.Kt = (int)p.Kt;
-    args.nkb_spline = f.nkb_spline;
-    args.nkb_total = f.nkb_total;
-    args.kb_per_split = f.kb_per_split;
-    args.partial = f.splits > 1;
-    args.BN = f.BN;
-    args.stages = f.stages;
-    e = f32 ? launch_fwd<KAN_F32>(f, m_ch, m_cl, m_wh, m_wl, args, st)
-            : launch_fwd<KAN_BF16>(f, m_ch, m_cl, m_wh, m_wl, args, st);
+    maps[0] = maps[2];
+    maps[1] = maps[3];
+    TcArgs a = base_args(p);
+    a.x = x;
+    a.out = P.f_splits > 1 ? (void*)(w + P.fwd.fwd_part) : y;
+    a.BN = P.f_BN;
+    a.stages = P.f_stages;
+    a.nkb_main = P.f_nkb_main;
+    a.nkb_total = P.f_nkb_total;
+    a.kb_per_split = P.f_kps;
+    a.partial = P.f_splits > 1;
+    e = launch_dt<FWD>(f32, dim3(P.f_n, P.f_m, P.f_splits), P.f_BN, P.f_stages, maps, a, st);
     if (e != cudaSuccess) return e;
-    if (f.splits > 1) {
+    if (P.f_splits > 1) {
         const int64_t n = p.batch * p.out;
-        if (f32)
-            reduce_splits_kernel<float><<<grid_for(n), 256, 0, st>>>((const float*)wsp, (float*)y, n, f.splits);
-        else
-            reduce_splits_kernel<__nv_bfloat16><<<grid_for(n), 256, 0, st>>>((const float*)wsp, (__nv_bfloat16*)y, n,
-                                                                              f.splits);
+        const float* part = reinterpret_cast<const float*>(w + P.fwd.fwd_part);
+        if (f32) {
+            reduce_splits_kernel<float><<<grid_for(n), 256, 0, st>>>(part, (float*)y, n, P.f_splits);
+            count_launch();
+        } else {
+            reduce_splits_kernel<__nv_bfloat16><<<grid_for(n), 256, 0, st>>>(part, (__nv_bfloat16*)y, n, P.f_splits);
+            count_launch();
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
-}
-
-size_t tc_workspace_backward(const Problem& p, int num_sms)
-{
-    (void)p;
-    (void)num_sms;
-    return 0;
 }
 
 cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const void* w_base, const void* dY,
                         void* dx, float* dcoef, float* dw_base, void* ws, int num_sms, cudaStream_t st,
                         const char** detail)
 {
-    (void)num_sms;
-    (void)ws;
-    (void)detail;
-    return simt_backward(p, x, coef, w_base, dY, dx, dcoef, dw_base, st);
+    const bool f32 = p.dtype == KAN_F32;
+    const int BK = f32 ? 32 : 64;
+    const int EPB = f32 ? 32 : 64;
+    const Plan P = make_plan(p, num_sms);
+    uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+    cudaError_t e;
+    if (p.batch == 0) {
+        if (dcoef && (e = zero_f32(dcoef, p.out * p.Kt, st)) != cudaSuccess) return e;
+        if (dw_base && (e = zero_f32(dw_base, p.out * p.in, st)) != cudaSuccess) return e;
+        return cudaSuccess;
+    }
+    // ---- dcoef / dw_base: A = basis^T (producers), B = dY (bf16: MN-major; fp32: dY^T K-major) ----
+    if (dcoef || dw_base) {
+        CUtensorMap maps[6];
+        if (f32) {
+            const void *th, *tl;
+            if ((e = split_t_into(dY, p.batch, p.out, P.ldb, w + P.bwd.dyt_hl, &th, &tl, st)) != cudaSuccess)
+                return e;
+            if (!make_map_2d(&maps[2], th, true, p.out, p.batch, P.d_BN, BK, detail, P.ldb) ||
+                !make_map_2d(&maps[3], tl, true, p.out, p.batch, P.d_BN, BK, detail, P.ldb))
+                return cudaErrorInvalidValue;
+        } else {
+            if (!make_map_2d(&maps[2], dY, false, p.batch, p.out, BK, EPB, detail)) return cudaErrorInvalidValue;
+            maps[3] = maps[2];
+        }
+        maps[0] = maps[1] = maps[4] = maps[5] = maps[2];
+        TcArgs a = base_args(p);
+        a.x = x;
+        float* partbuf = reinterpret_cast<float*>(w + P.bwd.dc_part);
+        a.BN = P.d_BN;
+        a.stages = P.d_stages;
+        a.nkb_main = a.nkb_total = P.d_nkb;
+        a.kb_per_split = P.d_kps;
+        a.n_kt_tiles = P.d_nkt;
+        a.part_ld = P.d_ld;
+        a.partial = P.d_splits > 1;
+        a.out = a.partial ? (void*)partbuf : (void*)dcoef;   // a skipped output is simply not stored
+        a.out2 = dw_base;
+        e = launch_dt<DCOEF>(f32, dim3(P.d_n, P.d_m, P.d_splits), P.d_BN, P.d_stages, maps, a, st);
+        if (e != cudaSuccess) return e;
+        if (a.partial) {
+            const int64_t n = p.out * P.d_ld;
+            reduce_dcoef_kernel<<<grid_for(n), 256, 0, st>>>(partbuf, dcoef, dw_base, p.out, p.Kt, p.in, P.d_ld,
+                                                              P.d_splits);
+            count_launch();
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+    }
+    // ---- dx: A = dY (K-major), B = coef (bf16: MN-major; fp32: coef^T K-major) ----
+    if (dx) {
+        const void *dy_hi = dY, *dy_lo = dY;
+        if (f32 && (e = split_into(dY, p.batch * p.out, w + P.bwd.dy_hl, &dy_hi, &dy_lo, st)) != cudaSuccess)
+            return e;
+        float* gb = nullptr;
+        if (p.base) {
+            // Gb = dY . w_base (fp32 [batch, in]) for the SiLU term of dx
+            gb = reinterpret_cast<float*>(w + P.bwd.gb);
+            CUtensorMap maps[6];
+            if (!make_map_2d(&maps[0], dy_hi, f32, p.batch, p.out, kBM, BK, detail) ||
+                !make_map_2d(&maps[1], dy_lo, f32, p.batch, p.out, kBM, BK, detail))
+                return cudaErrorInvalidValue;
+            if (f32) {
+                const void *th, *tl;
+                if ((e = split_t_into(w_base, p.out, p.in, p.out, w + P.bwd.wb_hl, &th, &tl, st)) != cudaSuccess)
+                    return e;
+                if (!make_map_2d(&maps[2], th, true, p.in, p.out, P.g_BN, BK, detail) ||
+                    !make_map_2d(&maps[3], tl, true, p.in, p.out, P.g_BN, BK, detail))
+                    return cudaErrorInvalidValue;
+            } else {
+                if (!make_map_2d(&maps[2], w_base, false, p.out, p.in, BK, EPB, detail)) return cudaErrorInvalidValue;
+                maps[3] = maps[2];
+            }
+            maps[4] = maps[2];
+            maps[5] = maps[3];
+            TcArgs a = base_args(p);
+            a.out = gb;
+            a.BN = P.g_BN;
+            a.stages = P.g_stages;
+            a.nkb_main = a.nkb_total = P.x_nkb;
+            a.kb_per_split = P.x_nkb;
+            e = launch_dt<GEMM>(f32, dim3(P.g_n, P.g_m, 1), P.g_BN, P.g_stages, maps, a, st);
+            if (e != cudaSuccess) return e;
+        }
+        CUtensorMap maps[6];
+        if (!make_map_2d(&maps[0], dy_hi, f32, p.batch, p.out, kBM, BK, detail) ||
+            !make_map_2d(&maps[1], dy_lo, f32, p.batch, p.out, kBM, BK, detail))
+            return cudaErrorInvalidValue;
+        if (f32) {
+            const void *th, *tl;
+            if ((e = split_t_into(coef, p.out, p.Kt, p.out, w + P.bwd.coef_hl, &th, &tl, st)) != cudaSuccess)
+                return e;
+            if (!make_map_2d(&maps[2], th, true, p.Kt, p.out, P.x_BN, BK, detail) ||
+                !make_map_2d(&maps[3], tl, true, p.Kt, p.out, P.x_BN, BK, detail))
+                return cudaErrorInvalidValue;
+        } else {
+            if (!make_map_2d(&maps[2], coef, false, p.out, p.Kt, BK, EPB, detail)) return cudaErrorInvalidValue;
+            maps[3] = maps[2];
+        }
+        maps[4] = maps[2];
+        maps[5] = maps[3];
+        TcArgs a = base_args(p);
+        a.x = x;
+        a.out = dx;
+        a.out2 = gb;
+        a.BN = P.x_BN;
+        a.stages = P.x_stages;
+        a.nkb_main = a.nkb_total = P.x_nkb;
+        a.kb_per_split = P.x_nkb;
+        a.n_in_tile = P.x_nin;
+        e = launch_dt<DX>(f32, dim3(P.x_n, P.x_m, 1), P.x_BN, P.x_stages, maps, a, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace kan
