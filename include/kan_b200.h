@@ -115,6 +115,29 @@ KAN_API kan_status kan_forward(const kan_shape* s, const void* x, const void* co
 KAN_API kan_status kan_backward(const kan_shape* s, const void* x, const void* coef, const void* w_base, const void* dY,
                         void* dx, float* dcoef, float* dw_base, void* workspace, size_t ws_bytes, void* stream);
 
+/* Size of the fixed device workspace used by kan_forward_fixed_scratch (32 MiB). */
+#define KAN_FIXED_SCRATCH_BYTES (32u << 20)
+
+/* kan_forward for callers that cannot allocate device memory when they run
+ * the layer (their memory comes only from a framework's own allocator, or a
+ * serving loop must not stall on cudaMalloc, or all memory is budgeted up
+ * front).  Same arguments and results as kan_forward, minus the workspace:
+ * the workspace is a fixed KAN_FIXED_SCRATCH_BYTES array in the library's
+ * device image, which every GPU that loads the library holds until the
+ * process exits.  Allocates nothing.  No counterpart on the pages this layer
+ * follows: it exists for deployment only.
+ *   - Shapes whose kan_workspace_size exceeds KAN_FIXED_SCRATCH_BYTES return
+ *     KAN_ERR_WORKSPACE (use kan_forward with your own workspace then).
+ *   - All calls share the one array: calls whose kernels overlap on the GPU
+ *     (unordered streams) race; order them on one stream or with events.
+ *   - The array keeps the last call's contents; the forward reads nothing
+ *     from it that it did not write earlier in the same call.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress with that device current); make that first call
+ *     before any stream capture begins. */
+KAN_API kan_status kan_forward_fixed_scratch(const kan_shape* s, const void* x, const void* coef, const void* w_base,
+                                             void* y, void* stream);
+
 /* The basis step alone, for inspection and tests: for each x[b,i] (batch*in
  * values) the span s (int32; the 4 non-zero functions are B_s..B_{s+3}, some
  * of which may fall outside 0..G+2 and are then absent; s = INT32_MIN when

@@ -19,7 +19,7 @@ STATUS = {0: "KAN_OK", 1: "KAN_ERR_INVALID_ARG", 2: "KAN_ERR_UNSUPPORTED", 3: "K
 
 #: every symbol the header declares
 EXPORTS = ("kan_abi_version", "kan_workspace_size", "kan_forward", "kan_backward", "kan_basis", "kan_sync_status",
-           "kan_launch_count",
+           "kan_launch_count", "kan_forward_fixed_scratch",
            "kan_selftest_wait_timeout", "kan_status_string", "kan_last_error")
 
 
@@ -69,6 +69,8 @@ def load(path: str | None = None):
     lib.kan_last_error.argtypes = []
     lib.kan_launch_count.restype = ctypes.c_uint64
     lib.kan_launch_count.argtypes = []
+    lib.kan_forward_fixed_scratch.restype = ctypes.c_int
+    lib.kan_forward_fixed_scratch.argtypes = [sp, _vp, _vp, _vp, _vp, _vp]
     if path is None:
         _lib = lib
     return lib
@@ -98,6 +100,11 @@ def kan_workspace_size(shape: kan_shape, for_backward: bool) -> int:
 
 def kan_forward(shape, x, coef, w_base, y, workspace, ws_bytes, stream):
     check(load().kan_forward(ctypes.byref(shape), x, coef, w_base, y, workspace, ws_bytes, stream), "kan_forward")
+
+
+def kan_forward_fixed_scratch(shape, x, coef, w_base, y, stream):
+    check(load().kan_forward_fixed_scratch(ctypes.byref(shape), x, coef, w_base, y, stream),
+          "kan_forward_fixed_scratch")
 
 
 def kan_backward(shape, x, coef, w_base, dY, dx, dcoef, dw_base, workspace, ws_bytes, stream):

@@ -34,8 +34,16 @@ unsigned int* device_status_ptr()
 }
 
 namespace {
-
 thread_local char g_last_error[512] = "";
+}
+
+kan_status set_last_error(kan_status st, const char* msg)
+{
+    snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+    return st;
+}
+
+namespace {
 
 kan_status fail(kan_status st, const char* fmt, const char* arg = nullptr)
 {

@@ -31,6 +31,9 @@ unsigned int* device_status_ptr();
 // Count one kernel launch (defined in kan_api.cu).
 void count_launch(int n = 1);
 
+// Record the detail string that kan_last_error() returns on this thread.
+kan_status set_last_error(kan_status st, const char* msg);
+
 // ---- CUDA-core kernels (kan_simt.cu) ----
 cudaError_t simt_basis(const Problem& p, const void* x, int32_t* span, float* w, float* dw, cudaStream_t st);
 cudaError_t simt_forward(const Problem& p, const void* x, const void* coef, const void* w_base, void* y,
