@@ -51,7 +51,10 @@ constexpr int kProducers = 256;   // warps 2-9
 constexpr int kEpi = 128;         // warps 10-13
 constexpr int kSmemBudget = 227 * 1024 - 2048;
 
-enum Mode { FWD = 0, DCOEF = 1, DX = 2, GEMM = 3 };
+// DCA (bf16): dcoef = A^T . dY with M = spline columns (then SiLU rows), N =
+// outputs, K = batch; the basis operand is written MN-major by the producers
+// (rows = batch, 64-column atoms of spline columns), dY is read MN-major.
+enum Mode { FWD = 0, DCOEF = 1, DX = 2, GEMM = 3, DCA = 4 };
 
 template <int DT> struct Cfg;
 template <> struct Cfg<KAN_BF16> {
@@ -89,6 +92,7 @@ struct TcArgs {
     int64_t part_ld;           // DCOEF partial row length (Kt + in with base)
     int n_in_tile;             // DX: inputs per N tile
     int has_base;
+    uint32_t nb_magic;         // ceil(2^32 / nb): c / nb == umulhi(c, nb_magic) for c < 2^32 / nb
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
@@ -163,7 +167,7 @@ __device__ __forceinline__ void put_a_chunk(uint32_t a_hi, uint32_t a_lo, uint32
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <int MODE, int DT>
+template <int MODE, int DT, int MAXI>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
               const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
@@ -175,8 +179,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int BK = C::BK;
     constexpr int EPB = 128 / C::ESZ;               // elements per 128-byte row
     constexpr bool F32 = DT == KAN_F32;
-    constexpr bool PRODUCE = MODE == FWD || MODE == DCOEF;
+    constexpr bool PRODUCE = MODE == FWD || MODE == DCOEF || MODE == DCA;
     constexpr bool A_BY_TMA = MODE == DX || MODE == GEMM;
+    constexpr bool A_MN = MODE == DCA;               // producer-written MN-major basis
+    static_assert(MODE != DCA || DT == KAN_BF16, "DCA is the bf16 dcoef path");
     // B stored MN-major (dY for dcoef, coef / w_base for dx) for bf16; the
     // fp32 path's split copies are transposed to K-major instead (tf32
     // MN-major operands would need the 32-byte-atom swizzle).
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
-            mbar_init(full_a(s), kProducers);
+            mbar_init(full_a(s), (MODE == FWD || MODE == DCA) ? kProducers / 2 : kProducers);
             mbar_init(full_b(s), 1);
             mbar_init(empty(s), 1);
             mbar_init(zeroed(s), kProducers);
@@ -292,9 +298,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issue ----------------
         if (lane == 0 && nk > 0) {
-            const uint32_t idesc = instr_desc(C::FMT, 0, B_MN ? 1u : 0u, kBM, BN);
+            const uint32_t idesc = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, BN);
             const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
             const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
+            const uint32_t a_lbo = A_MN ? (uint32_t)BK * 128u : 16u;
+            const uint32_t a_step = A_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
             bool ok = true;
             for (int it = 0; it < nk && ok; ++it) {
                 const int s = it % stages;
@@ -311,12 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t t_main = (g & 1) ? t_main1 : t_main0;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ad = smem_desc_sw128(A_hi(s) + ks * 32, 16, 1024);
+                    const uint64_t ad = smem_desc_sw128(A_hi(s) + ks * a_step, a_lbo, 1024);
                     const uint64_t bd = smem_desc_sw128(B_hi(s) + ks * b_step, b_lbo, 1024);
                     if constexpr (!F32) {
                         mma_bf16_ss(t_main0, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                     } else {
-                        const uint64_t adl = smem_desc_sw128(A_lo(s) + ks * 32, 16, 1024);
+                        const uint64_t adl = smem_desc_sw128(A_lo(s) + ks * a_step, a_lbo, 1024);
                         const uint64_t bdl = smem_desc_sw128(B_lo(s) + ks * b_step, b_lbo, 1024);
                         mma_tf32_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                         mma_tf32_ss(t_corr, ad, bdl, idesc, 1u);
@@ -330,68 +338,287 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < 10) {
         // ---------------- A producers ----------------
+        // Each thread fetches the x values of its next k-block into registers
+        // before it waits for and fills the current one, so the global-load
+        // latency overlaps the previous k-block's work.
         if constexpr (PRODUCE) {
             const int p = threadIdx.x - 64;
-            for (int it = 0; it < nk; ++it) {
-                const int s = it % stages;
-                const uint32_t ph = (it / stages) & 1;
-                if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
-                const int kb = kb_begin + it;
-                const uint32_t ahi = A_hi(s), alo = A_lo(s);
-                if constexpr (MODE == FWD) {
-                    // rows = batch m0..m0+127, columns = spline or SiLU columns of k-block kb
-                    constexpr int HALF = BK / 2;
-                    const uint32_t row = p & (kBM - 1);
-                    const int half = p >> 7;
-                    const int64_t b = m0 + row;
-                    const bool row_ok = b < a.batch;
-                    const T* xrow = reinterpret_cast<const T*>(a.x) + (row_ok ? b : 0) * a.in;
+            const T* X = reinterpret_cast<const T*>(a.x);
+            if constexpr (MODE == FWD) {
+                // rows = batch m0..m0+127.  Two groups of 128 threads (warps 2-5 and
+                // 6-9) take alternate k-blocks; a thread fills one whole row.  Per
+                // row and k-block at most MAXI inputs have columns in the block.
+                constexpr int EPC = 16 / C::ESZ;       // elements per 16-byte chunk
+                const uint32_t row = p & (kBM - 1);
+                const int grp = p >> 7;                // warp-uniform
+                const int64_t b = m0 + row;
+                const bool row_ok = b < a.batch;
+                const T* xrow = X + (row_ok ? b : 0) * a.in;
+                const float u0 = -a.lo * a.inv_h;      // u = x * inv_h + u0
+                const float u_hi = (float)(a.G + 3);
+                auto first_input = [&](int kb) { return (int)__umulhi((uint32_t)(kb * BK), a.nb_magic); };
+                auto last_input = [&](int kb) {
+                    const int c_end = min(kb * BK + BK, a.Kt);
+                    return (int)__umulhi((uint32_t)(c_end - 1), a.nb_magic);
+                };
+                auto fetch = [&](int kb, float (&xv)[MAXI]) {
+                    if (kb >= a.nkb_main || !row_ok) return;
+                    const int i0 = first_input(kb), n = last_input(kb) - i0 + 1;
+#pragma unroll
+                    for (int k = 0; k < MAXI; ++k) {
+                        if (k >= n) break;                  // uniform across the warp
+                        xv[k] = to_f(xrow[i0 + k]);
+                    }
+                };
+                float nxt[MAXI];
+                if (grp < nk) fetch(kb_begin + grp, nxt);
+                int uses = 0;                               // k-blocks this group has filled
+                for (int it = grp; it < nk; it += 2, ++uses) {
+                    float cur[MAXI];
+#pragma unroll
+                    for (int k = 0; k < MAXI; ++k) cur[k] = nxt[k];
+                    const int kb = kb_begin + it;
+                    if (it + 2 < nk) fetch(kb + 2, nxt);
+                    const int s = it % stages;
+                    const uint32_t ph = (it / stages) & 1;
+                    if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
+                    const uint32_t ahi = A_hi(s), alo = A_lo(s);
+                    const uint32_t rbase = row * 128u, rx = row & 7u;
                     if (kb < a.nkb_main) {
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const uint32_t off = sw128_chunk(row, half * 4 + c);
+                        for (int c = 0; c < 8; ++c) {
+                            const uint32_t off = rbase + ((c ^ rx) << 4);
                             st_shared_zero16(ahi + off);
                             if (F32) st_shared_zero16(alo + off);
                         }
-                        const int c_lo = kb * BK + half * HALF;
-                        const int c_hi = min(c_lo + HALF, a.Kt);
-                        if (row_ok && c_lo < c_hi) {
-                            const int i_first = c_lo / a.nb, i_last = (c_hi - 1) / a.nb;
-                            for (int i = i_first; i <= i_last; ++i) {
-                                const Span sp = span_of(to_f(xrow[i]), a.lo, a.inv_h, a.G);
-                                if (!sp.valid) continue;
+                        if (row_ok) {
+                            const int i0 = first_input(kb), n = last_input(kb) - i0 + 1;
+                            const int cbase = i0 * a.nb - kb * BK;   // column of input i0's B_0 in this block
+#pragma unroll
+                            for (int k = 0; k < MAXI; ++k) {
+                                if (k >= n) break;
+                                const float u = fmaf(cur[k], a.inv_h, u0);
+                                if (!(u >= -3.0f && u < u_hi)) continue;   // outside the extended knots, NaN, inf
+                                const float f = floorf(u);
+                                const int sidx = (int)f;
+                                const float t = u - f, sm = 1.0f - t;
+                                const float t2 = t * t, s2 = sm * sm;
                                 float w[4];
-                                weights(sp.t, w);
+                                w[0] = s2 * sm * (1.0f / 6.0f);
+                                w[1] = fmaf(t2, fmaf(t, 0.5f, -1.0f), 2.0f / 3.0f);
+                                w[2] = fmaf(s2, fmaf(sm, 0.5f, -1.0f), 2.0f / 3.0f);
+                                w[3] = t2 * t * (1.0f / 6.0f);
+                                const int col0 = cbase + k * a.nb + sidx;
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) {
-                                    const int m = sp.s + q;
-                                    const int col = i * a.nb + m;
-                                    if (m >= 0 && m < a.nb && col >= c_lo && col < c_hi)
-                                        put_a<DT>(ahi, alo, row, col - kb * BK, w[q]);
+                                    const int col = col0 + q;
+                                    if ((unsigned)(sidx + q) < (unsigned)a.nb && (unsigned)col < (unsigned)BK) {
+                                        const uint32_t cb = (uint32_t)col * C::ESZ;
+                                        const uint32_t off = rbase + ((((cb >> 4) ^ rx) & 7u) << 4) + (cb & 15u);
+                                        if constexpr (!F32) {
+                                            st_shared_u16(ahi + off, __bfloat16_as_ushort(__float2bfloat16_rn(w[q])));
+                                        } else {
+                                            const float hi = tf32_hi(w[q]);
+                                            st_shared_f32(ahi + off, hi);
+                                            st_shared_f32(alo + off, w[q] - hi);
+                                        }
+                                    }
                                 }
                             }
                         }
                     } else {
-                        const int i0 = (kb - a.nkb_main) * BK + half * HALF;
-                        constexpr int EPC = 16 / C::ESZ;   // elements per 16-byte chunk
+                        // SiLU columns: BK consecutive inputs, dense (in*esize % 16 == 0 with the base branch)
+                        const int i0 = (kb - a.nkb_main) * BK;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < 8; ++c) {
                             float v[EPC];
+                            const int ic = i0 + c * EPC;
+                            if (row_ok && ic + EPC <= a.in) {
+                                const uint4 q4 = *reinterpret_cast<const uint4*>(xrow + ic);
+                                const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-                            for (int e = 0; e < EPC; ++e) {
-                                const int i = i0 + c * EPC + e;
-                                v[e] = (row_ok && i < a.in) ? silu_f(to_f(xrow[i])) : 0.0f;
+                                for (int e = 0; e < EPC; ++e) {
+                                    float xv;
+                                    if constexpr (F32) {
+                                        xv = __uint_as_float(wd[e]);
+                                    } else {
+                                        xv = __uint_as_float((e & 1) ? (wd[e / 2] & 0xFFFF0000u) : (wd[e / 2] << 16));
+                                    }
+                                    v[e] = silu_f(xv);
+                                }
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < EPC; ++e) v[e] = 0.0f;
                             }
-                            put_a_chunk<DT>(ahi, alo, row, half * 4 + c, v);
+                            put_a_chunk<DT>(ahi, alo, row, (uint32_t)c, v);
                         }
                     }
-                } else {
-                    // DCOEF: rows = spline columns kt0..kt0+127 (or inputs for SiLU tiles),
-                    // columns = batch rows b0..b0+BK-1
+                    fence_async_smem();
+                    mbar_arrive(full_a(s));
+                }
+                (void)uses;
+            } else if constexpr (MODE == DCA) {
+                // A tile, MN-major: batch rows b0..b0+63 (K) by 128 columns (M) in two
+                // 64-column atoms [64 rows x 128 bytes], BK*128 bytes apart; the columns
+                // are spline columns kt0.. (or, for a SiLU tile, inputs i0..).  Two
+                // groups of 128 threads take alternate k-blocks; a thread fills one
+                // atom row: (batch row rb, atom).
+                const int grp = p >> 7;                    // warp-uniform
+                const int rb = p & (BK - 1);
+                const int atom = (p >> 6) & 1;             // warp-uniform
+                const int mt = blockIdx.y;
+                const bool silu_tile = mt >= a.n_kt_tiles;
+                const int c_lo = (silu_tile ? (mt - a.n_kt_tiles) * kBM : mt * kBM) + atom * 64;
+                const int c_end = silu_tile ? min(c_lo + 64, (int)a.in) : min(c_lo + 64, a.Kt);
+                const int i_first = (int)__umulhi((uint32_t)c_lo, a.nb_magic);
+                const int n_inp = (!silu_tile && c_lo < c_end)
+                                      ? (int)__umulhi((uint32_t)(c_end - 1), a.nb_magic) - i_first + 1 : 0;
+                const float u0 = -a.lo * a.inv_h;
+                const float u_hi = (float)(a.G + 3);
+                auto fetch = [&](int kb, float (&xv)[MAXI]) {
+                    const int64_t b = (int64_t)kb * BK + rb;
+                    if (silu_tile || b >= a.batch) return;
+                    const T* xr = X + b * a.in + i_first;
+#pragma unroll
+                    for (int k = 0; k < MAXI; ++k) {
+                        if (k >= n_inp) break;
+                        xv[k] = to_f(xr[k]);
+                    }
+                };
+                float nxt[MAXI];
+                if (grp < nk) fetch(kb_begin + grp, nxt);
+                for (int it = grp; it < nk; it += 2) {
+                    float cur[MAXI];
+#pragma unroll
+                    for (int k = 0; k < MAXI; ++k) cur[k] = nxt[k];
+                    const int kb = kb_begin + it;
+                    if (it + 2 < nk) fetch(kb + 2, nxt);
+                    const int s = it % stages;
+                    const uint32_t ph = (it / stages) & 1;
+                    if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
+                    const int64_t b = (int64_t)kb * BK + rb;
+                    const bool row_ok = b < a.batch;
+                    const uint32_t rbase = A_hi(s) + (uint32_t)atom * BK * 128u + (uint32_t)rb * 128u;
+                    const uint32_t rx = (uint32_t)rb & 7u;
+                    if (!silu_tile) {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) st_shared_zero16(rbase + ((c ^ rx) << 4));
+                        if (row_ok) {
+                            const int cbase = i_first * a.nb - c_lo;
+#pragma unroll
+                            for (int k = 0; k < MAXI; ++k) {
+                                if (k >= n_inp) break;
+                                const float u = fmaf(cur[k], a.inv_h, u0);
+                                if (!(u >= -3.0f && u < u_hi)) continue;
+                                const float f = floorf(u);
+                                const int sidx = (int)f;
+                                const float t = u - f, sm = 1.0f - t;
+                                const float t2 = t * t, s2 = sm * sm;
+                                float w[4];
+                                w[0] = s2 * sm * (1.0f / 6.0f);
+                                w[1] = fmaf(t2, fmaf(t, 0.5f, -1.0f), 2.0f / 3.0f);
+                                w[2] = fmaf(s2, fmaf(sm, 0.5f, -1.0f), 2.0f / 3.0f);
+                                w[3] = t2 * t * (1.0f / 6.0f);
+                                const int col0 = cbase + k * a.nb + sidx;
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const int col = col0 + q;
+                                    if ((unsigned)(sidx + q) < (unsigned)a.nb && (unsigned)col < 64u) {
+                                        const uint32_t cb = (uint32_t)col * 2u;
+                                        st_shared_u16(rbase + ((((cb >> 4) ^ rx) & 7u) << 4) + (cb & 15u),
+                                                      __bfloat16_as_ushort(__float2bfloat16_rn(w[q])));
+                                    }
+                                }
+                            }
+                        }
+                    } else {
+                        // SiLU columns: inputs c_lo..c_lo+63 of batch row b (in % 8 == 0 with the base branch)
+                        const T* xr = X + (row_ok ? b : 0) * a.in;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            float v[8];
+                            const int ic = c_lo + c * 8;
+                            if (row_ok && ic + 8 <= a.in) {
+                                const uint4 q4 = *reinterpret_cast<const uint4*>(xr + ic);
+                                const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    v[e] = silu_f(__uint_as_float((e & 1) ? (wd[e / 2] & 0xFFFF0000u) : (wd[e / 2] << 16)));
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+                            }
+                            st_shared_v4(rbase + ((c ^ rx) << 4), pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                         pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+                        }
+                    }
+                    fence_async_smem();
+                    mbar_arrive(full_a(s));
+                }
+            } else {
+                // DCOEF: rows = spline columns kt0..kt0+127 (or inputs of a SiLU tile),
+                // columns = batch rows b0..b0+BK-1
+                const int mt = blockIdx.y;
+                const bool silu_tile = mt >= a.n_kt_tiles;
+                constexpr int EPC = 16 / C::ESZ;
+                // spline tiles: (batch column c, input i) pairs, inputs fastest so that a
+                // warp reads consecutive x elements; the mapping is the same every k-block
+                constexpr int MAXP = (BK * (kBM / 4 + 2) + kProducers - 1) / kProducers;
+                const int kt0 = mt * kBM;
+                const int i_first = kt0 / a.nb;
+                const int i_last = min((int)a.in - 1, (kt0 + kBM - 1) / a.nb);
+                const int n_i = i_last - i_first + 1;
+                int pc[MAXP], pi[MAXP];
+#pragma unroll
+                for (int k = 0; k < MAXP; ++k) {
+                    const int e = p + k * kProducers;
+                    pc[k] = (!silu_tile && n_i > 0 && e < BK * n_i) ? e / n_i : -1;
+                    pi[k] = pc[k] >= 0 ? i_first + e % n_i : 0;
+                }
+                // SiLU tiles: input row r = p % 128 (consecutive across a warp), chunks
+                // (p / 128) * 4 .. + 3, EPC batch rows each
+                const int sr = p & (kBM - 1);
+                const int64_t si = (int64_t)(mt - a.n_kt_tiles) * kBM + sr;
+                const int sch0 = (p >> 7) * 4;
+                constexpr int NR = MAXP > 16 ? MAXP : 16;   // registers per fetch (bf16 SiLU values packed in pairs)
+                auto fetch = [&](int kb, uint32_t (&xr)[NR]) {
                     const int64_t b0 = (int64_t)kb * BK;
-                    const int mt = blockIdx.y;
-                    if (mt < a.n_kt_tiles) {
-                        const int kt0 = mt * kBM;
+                    if (!silu_tile) {
+#pragma unroll
+                        for (int k = 0; k < MAXP; ++k) {
+                            const int64_t b = b0 + pc[k];
+                            xr[k] = (pc[k] >= 0 && b < a.batch) ? __float_as_uint(to_f(X[b * a.in + pi[k]])) : 0x7FC00000u;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int e = 0; e < EPC; ++e) {
+                                const int64_t b = b0 + (sch0 + q) * EPC + e;
+                                const bool ok = si < a.in && b < a.batch;
+                                if constexpr (F32) {
+                                    xr[q * EPC + e] = ok ? __float_as_uint(X[b * a.in + si]) : 0u;
+                                } else {
+                                    const uint32_t h = ok ? (uint32_t)__bfloat16_as_ushort(X[b * a.in + si]) : 0u;
+                                    if (e & 1) xr[q * 4 + e / 2] |= h << 16;
+                                    else xr[q * 4 + e / 2] = h;
+                                }
+                            }
+                    }
+                };
+                uint32_t nxt[NR];
+                if (nk > 0) fetch(kb_begin, nxt);
+                for (int it = 0; it < nk; ++it) {
+                    uint32_t cur[NR];
+#pragma unroll
+                    for (int e = 0; e < NR; ++e) cur[e] = nxt[e];
+                    const int kb = kb_begin + it;
+                    if (it + 1 < nk) fetch(kb + 1, nxt);
+                    const int s = it % stages;
+                    const uint32_t ph = (it / stages) & 1;
+                    if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
+                    const uint32_t ahi = A_hi(s), alo = A_lo(s);
+                    if (!silu_tile) {
                         // zero the tile: 128 rows x 8 chunks, 4 chunks per thread
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
@@ -403,49 +630,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // every producer's zeros are in place before anyone scatters
                         mbar_arrive(zeroed(s));
                         if (!mbar_wait(zeroed(s), ph, a.status)) break;
-                        const int i_first = kt0 / a.nb;
-                        const int i_last = min((int)a.in - 1, (kt0 + kBM - 1) / a.nb);
-                        const int n_pairs = BK * (i_last - i_first + 1);
-                        for (int e = p; e < n_pairs; e += kProducers) {
-                            const int c = e % BK;
-                            const int i = i_first + e / BK;
-                            const int64_t b = b0 + c;
-                            if (b >= a.batch) continue;
-                            const Span sp = span_of(to_f(reinterpret_cast<const T*>(a.x)[b * a.in + i]), a.lo,
-                                                    a.inv_h, a.G);
+#pragma unroll
+                        for (int k = 0; k < MAXP; ++k) {
+                            if (pc[k] < 0) continue;
+                            // x beyond the batch was fetched as NaN: no basis, nothing stored
+                            const Span sp = span_of(__uint_as_float(cur[k]), a.lo, a.inv_h, a.G);
                             if (!sp.valid) continue;
                             float w[4];
                             weights(sp.t, w);
 #pragma unroll
                             for (int q = 0; q < 4; ++q) {
                                 const int m = sp.s + q;
-                                const int r = i * a.nb + m - kt0;
-                                if (m >= 0 && m < a.nb && r >= 0 && r < kBM) put_a<DT>(ahi, alo, (uint32_t)r, c, w[q]);
+                                const int r = pi[k] * a.nb + m - kt0;
+                                if (m >= 0 && m < a.nb && r >= 0 && r < kBM)
+                                    put_a<DT>(ahi, alo, (uint32_t)r, pc[k], w[q]);
                             }
                         }
                     } else {
-                        // SiLU rows: inputs i0..i0+127, dense
-                        const int i0 = (mt - a.n_kt_tiles) * kBM;
-                        constexpr int EPC = 16 / C::ESZ;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int e = p * 4 + c;
-                            const int r = e >> 3, ch = e & 7;
-                            const int64_t i = i0 + r;
+                        for (int q = 0; q < 4; ++q) {
                             float v[EPC];
 #pragma unroll
-                            for (int q = 0; q < EPC; ++q) {
-                                const int64_t b = b0 + ch * EPC + q;
-                                v[q] = (i < a.in && b < a.batch)
-                                           ? silu_f(to_f(reinterpret_cast<const T*>(a.x)[b * a.in + i]))
-                                           : 0.0f;
+                            for (int e = 0; e < EPC; ++e) {
+                                float xv;
+                                if constexpr (F32) {
+                                    xv = __uint_as_float(cur[q * EPC + e]);
+                                } else {
+                                    const uint32_t wd = cur[q * 4 + e / 2];
+                                    xv = __uint_as_float((e & 1) ? (wd & 0xFFFF0000u) : (wd << 16));
+                                }
+                                v[e] = si < a.in ? silu_f(xv) : 0.0f;
                             }
-                            put_a_chunk<DT>(ahi, alo, (uint32_t)r, (uint32_t)ch, v);
+                            put_a_chunk<DT>(ahi, alo, (uint32_t)sr, (uint32_t)(sch0 + q), v);
                         }
                     }
+                    fence_async_smem();
+                    mbar_arrive(full_a(s));
                 }
-                fence_async_smem();
-                mbar_arrive(full_a(s));
             }
         }
     } else {
@@ -453,6 +674,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;                       // TMEM lane quarter
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         const uint32_t r = 32 * q + lane;             // tile row of this thread
+        // DX: the x values (and dY.w_base terms) of the tile's inputs do not
+        // depend on the MMA; fetch them in chunks of XC, the first one now.
+        constexpr int XC = 16;
+        uint32_t xa[XC], ga[XC];
+        const int64_t dx_b = m0 + r;
+        const int dx_i0 = MODE == DX ? blockIdx.x * a.n_in_tile : 0;
+        const int dx_i1 = MODE == DX ? min((int)a.in, dx_i0 + a.n_in_tile) : 0;
+        auto xfetch = [&](int i_start, uint32_t (&xv)[XC], uint32_t (&gv)[XC]) {
+#pragma unroll
+            for (int k = 0; k < XC; ++k) {
+                const int i = i_start + k;
+                const bool ok = dx_b < a.batch && i < dx_i1;
+                xv[k] = ok ? __float_as_uint(to_f(reinterpret_cast<const T*>(a.x)[dx_b * a.in + i])) : 0u;
+                gv[k] = (ok && a.has_base) ? __float_as_uint(a.out2[dx_b * a.in + i]) : 0u;
+            }
+        };
+        if constexpr (MODE == DX) xfetch(dx_i0, xa, ga);
         bool go = nk > 0;
         if (F32 && go) {
             // promotion: total (+)= main[g & 1] for every segment
@@ -514,7 +752,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int e = 0; e < 16; e += 4)
                                 *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                         } else {
-                            for (int e = 0; e < 16 && j0 + e < ncols; ++e) dst[e] = v[e];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                if (j0 + e < ncols) dst[e] = v[e];
                         }
                     } else {
                         T* dst = reinterpret_cast<T*>(a.out) + bo * ncols + j0;
@@ -526,7 +766,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                                 *reinterpret_cast<uint4*>(dst + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                             } else {
-                                for (int e = 0; e < 16 && j0 + e < ncols; ++e) dst[e] = __float2bfloat16_rn(v[e]);
+#pragma unroll
+                                for (int e = 0; e < 16; ++e)
+                                    if (j0 + e < ncols) dst[e] = __float2bfloat16_rn(v[e]);
                             }
                         } else {
                             if (j0 + 16 <= ncols) {
@@ -535,12 +777,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     *reinterpret_cast<float4*>(dst + e) =
                                         make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                             } else {
-                                for (int e = 0; e < 16 && j0 + e < ncols; ++e) dst[e] = v[e];
+    #pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                if (j0 + e < ncols) dst[e] = v[e];
                             }
                         }
                     }
                 }
-            } else if constexpr (MODE == DCOEF) {
+            } else if constexpr (MODE == DCOEF || MODE == DCA) {
                 // rows are spline columns kt (or inputs of a SiLU tile); columns are outputs j
                 const int mt = blockIdx.y;
                 const bool base_tile = mt >= a.n_kt_tiles;
@@ -578,29 +822,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 16; ++e) stage[c0 + e] = v[e];
                 }
-                const int64_t b = m0 + r;
-                if (b < a.batch) {
-                    const int i0 = blockIdx.x * a.n_in_tile;
-                    const int kt_al = B_MN ? (i0 * a.nb) / (16 / C::ESZ) * (16 / C::ESZ) : i0 * a.nb;
-                    const int i1 = min((int)a.in, i0 + a.n_in_tile);
-                    const T* xr = reinterpret_cast<const T*>(a.x) + b * a.in;
-                    T* dxr = reinterpret_cast<T*>(a.out) + b * a.in;
-                    for (int i = i0; i < i1; ++i) {
-                        const float xv = to_f(xr[i]);
-                        const Span sp = span_of(xv, a.lo, a.inv_h, a.G);
-                        float acc = 0.0f;
-                        if (sp.valid) {
-                            float d[4];
-                            dweights(sp.t, a.inv_h, d);
-                            const int cb = i * a.nb - kt_al;
+                if (dx_b < a.batch) {
+                    const int kt_al = B_MN ? (dx_i0 * a.nb) / (16 / C::ESZ) * (16 / C::ESZ) : dx_i0 * a.nb;
+                    T* dxr = reinterpret_cast<T*>(a.out) + dx_b * a.in;
+                    for (int ic = dx_i0; ic < dx_i1; ic += XC) {
+                        uint32_t xc[XC], gc[XC];
 #pragma unroll
-                            for (int qq = 0; qq < 4; ++qq) {
-                                const int m = sp.s + qq;
-                                if (m >= 0 && m < a.nb) acc += stage[cb + m] * d[qq];
-                            }
+                        for (int k = 0; k < XC; ++k) {
+                            xc[k] = xa[k];
+                            gc[k] = ga[k];
                         }
-                        if (a.has_base) acc += dsilu_f(xv) * a.out2[b * a.in + i];
-                        dxr[i] = from_f<T>(acc);
+                        if (ic + XC < dx_i1) xfetch(ic + XC, xa, ga);
+#pragma unroll
+                        for (int k = 0; k < XC; ++k) {
+                            const int i = ic + k;
+                            if (i >= dx_i1) break;
+                            const float xv = __uint_as_float(xc[k]);
+                            const Span sp = span_of(xv, a.lo, a.inv_h, a.G);
+                            float acc = 0.0f;
+                            if (sp.valid) {
+                                float d[4];
+                                dweights(sp.t, a.inv_h, d);
+                                const int cb = i * a.nb - kt_al;
+#pragma unroll
+                                for (int qq = 0; qq < 4; ++qq) {
+                                    const int m = sp.s + qq;
+                                    if (m >= 0 && m < a.nb) acc += stage[cb + m] * d[qq];
+                                }
+                            }
+                            if (a.has_base) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
+                            dxr[i] = from_f<T>(acc);
+                        }
                     }
                 }
             }
@@ -787,7 +1039,6 @@ Plan make_plan(const Problem& p, int sms)
     Plan P{};
     const bool f32 = p.dtype == KAN_F32;
     const int BK = f32 ? 32 : 64;
-    const int EPB = f32 ? 32 : 64;
     const size_t esz = f32 ? 4 : 2;
     // forward: M = batch, N = out, K = spline (+ SiLU) columns
     P.f_BN = bn_for(p.out, f32);
@@ -801,10 +1052,10 @@ Plan make_plan(const Problem& p, int sms)
     P.f_splits = (int)cdiv(P.f_nkb_total, P.f_kps);
     // dcoef: M = spline columns (+ SiLU rows), N = out, K = batch
     P.d_BN = bn_for(p.out, f32, true);
-    P.d_stages = stages_for(P.d_BN, f32);
     P.d_n = (int)cdiv(p.out, P.d_BN);
     P.d_nkt = (int)cdiv(p.Kt, kBM);
     P.d_m = P.d_nkt + (p.base ? (int)cdiv(p.in, kBM) : 0);
+    P.d_stages = stages_for(P.d_BN, f32);
     P.d_nkb = (int)cdiv(p.batch, BK);
     P.d_splits = pick_splits((int64_t)P.d_n * P.d_m, sms, std::min(16, std::max(1, P.d_nkb / 8)));
     P.d_kps = (int)cdiv(std::max(1, P.d_nkb), P.d_splits);
@@ -871,7 +1122,7 @@ Plan make_plan(const Problem& p, int sms)
 
 inline int grid_for(int64_t n) { return (int)std::min<int64_t>(std::max<int64_t>(1, (n + 255) / 256), 148 * 8); }
 
-template <int MODE, int DT>
+template <int MODE, int DT, int MAXI>
 cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args, cudaStream_t st)
 {
     // the MN-major bf16 B operand arrives in whole 128-byte boxes: BN must be a multiple of 64
@@ -881,22 +1132,46 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
     const int smem = smem_bytes(BN, stages, DT == KAN_F32);
     static int configured = 0;   // per instantiation; the attribute is per function
     if (configured < smem) {
-        cudaError_t e = cudaFuncSetAttribute(tc_kernel<MODE, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(tc_kernel<MODE, DT, MAXI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kSmemBudget);
         if (e != cudaSuccess) return e;
         configured = kSmemBudget;
     }
-    tc_kernel<MODE, DT><<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], args);
+    tc_kernel<MODE, DT, MAXI><<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], args);
     count_launch();
     return cudaGetLastError();
 }
+
+// Inputs a row of one forward k-block can touch: (BK - 1) / nb + 2.
+int fwd_maxi_needed(int nb, bool f32) { return ((f32 ? 32 : 64) - 1) / nb + 2; }
 
 template <int MODE>
 cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
                       cudaStream_t st)
 {
-    return f32 ? launch<MODE, KAN_F32>(grid, BN, stages, maps, args, st)
-               : launch<MODE, KAN_BF16>(grid, BN, stages, maps, args, st);
+    if constexpr (MODE == DCA) {
+        if (f32) return cudaErrorInvalidConfiguration;
+        const int need = fwd_maxi_needed(args.nb, false);
+        if (need <= 4) return launch<MODE, KAN_BF16, 4>(grid, BN, stages, maps, args, st);
+        if (need <= 9) return launch<MODE, KAN_BF16, 9>(grid, BN, stages, maps, args, st);
+        if (need <= 17) return launch<MODE, KAN_BF16, 17>(grid, BN, stages, maps, args, st);
+        return cudaErrorInvalidConfiguration;
+    } else if constexpr (MODE == FWD) {
+        const int need = fwd_maxi_needed(args.nb, f32);
+        if (need <= 4)
+            return f32 ? launch<MODE, KAN_F32, 4>(grid, BN, stages, maps, args, st)
+                       : launch<MODE, KAN_BF16, 4>(grid, BN, stages, maps, args, st);
+        if (need <= 9)
+            return f32 ? launch<MODE, KAN_F32, 9>(grid, BN, stages, maps, args, st)
+                       : launch<MODE, KAN_BF16, 9>(grid, BN, stages, maps, args, st);
+        if (need <= 17)
+            return f32 ? launch<MODE, KAN_F32, 17>(grid, BN, stages, maps, args, st)
+                       : launch<MODE, KAN_BF16, 17>(grid, BN, stages, maps, args, st);
+        return cudaErrorInvalidConfiguration;   // G >= 1 keeps need <= 17
+    } else {
+        return f32 ? launch<MODE, KAN_F32, 1>(grid, BN, stages, maps, args, st)
+                   : launch<MODE, KAN_BF16, 1>(grid, BN, stages, maps, args, st);
+    }
 }
 
 TcArgs base_args(const Problem& p)
@@ -913,6 +1188,7 @@ TcArgs base_args(const Problem& p)
     a.Kt = (int)p.Kt;
     a.seg_kb = kSegKb;
     a.has_base = p.base;
+    a.nb_magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)p.nb - 1) / (uint64_t)p.nb);
     return a;
 }
 
@@ -963,7 +1239,8 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
         *why = "G too large for one dx tile (G+3 must fit the tile with its alignment offset)";
         return false;
     }
-    if (p.Kt + p.in > ((int64_t)1 << 30) || p.batch > ((int64_t)1 << 31) - 256 || p.out > ((int64_t)1 << 30)) {
+    if (p.Kt + p.in > ((int64_t)1 << 30) || p.Kt >= (((int64_t)1 << 32) / p.nb) || p.batch > ((int64_t)1 << 31) - 256 ||
+        p.out > ((int64_t)1 << 30)) {
         *why = "problem too large for 32-bit tile coordinates";
         return false;
     }
@@ -1054,11 +1331,12 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             if (!make_map_2d(&maps[2], th, true, p.out, p.batch, P.d_BN, BK, detail, P.ldb) ||
                 !make_map_2d(&maps[3], tl, true, p.out, p.batch, P.d_BN, BK, detail, P.ldb))
                 return cudaErrorInvalidValue;
+            maps[0] = maps[1] = maps[4] = maps[5] = maps[2];
         } else {
+            // dY as the MN-major B operand: BK-batch x 64-output boxes
             if (!make_map_2d(&maps[2], dY, false, p.batch, p.out, BK, EPB, detail)) return cudaErrorInvalidValue;
-            maps[3] = maps[2];
+            maps[0] = maps[1] = maps[3] = maps[4] = maps[5] = maps[2];
         }
-        maps[0] = maps[1] = maps[4] = maps[5] = maps[2];
         TcArgs a = base_args(p);
         a.x = x;
         float* partbuf = reinterpret_cast<float*>(w + P.bwd.dc_part);
@@ -1071,7 +1349,9 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         a.partial = P.d_splits > 1;
         a.out = a.partial ? (void*)partbuf : (void*)dcoef;   // a skipped output is simply not stored
         a.out2 = dw_base;
-        e = launch_dt<DCOEF>(f32, dim3(P.d_n, P.d_m, P.d_splits), P.d_BN, P.d_stages, maps, a, st);
+        const dim3 grid(P.d_n, P.d_m, P.d_splits);
+        e = f32 ? launch_dt<DCOEF>(true, grid, P.d_BN, P.d_stages, maps, a, st)
+                : launch_dt<DCA>(false, grid, P.d_BN, P.d_stages, maps, a, st);
         if (e != cudaSuccess) return e;
         if (a.partial) {
             const int64_t n = p.out * P.d_ld;
