@@ -867,6 +867,254 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// dx, persistent: one CTA per SM walks the (batch tile, input group) tiles.
+// Gm = dY . coef for a tile goes to one of two TMEM accumulators while the
+// epilogue warps turn the previous tile's accumulator into dx, so the B'
+// gather overlaps the next tile's MMA.  Warps: 0 TMA, 1 MMA issue + TMEM,
+// 2-5 epilogue (one per TMEM lane quarter).  fp32 keeps the tf32 correction
+// products in a second accumulator per buffer; the contraction over `out`
+// is short enough (at most 32 k-blocks) that no promotion is needed.
+// ---------------------------------------------------------------------------
+constexpr int kDxThreads = 192;
+
+struct DxArgs {
+    const void* x;
+    void* dx;
+    const float* gb;          // dY . w_base (fp32 [batch, in]) or null
+    unsigned int* status;
+    int64_t batch, in, out;
+    int G, nb;
+    float lo, inv_h;
+    int BN, stages, nkb;      // nkb: k-blocks over out
+    int n_in_tile, n_tiles_n, n_tiles;
+    int ld_stage;             // staging row stride in floats (BN + 4)
+};
+
+template <int DT>
+__global__ void __launch_bounds__(kDxThreads, 1)
+    dx_persistent_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
+                         const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
+                         const DxArgs a)
+{
+    using C = Cfg<DT>;
+    using T = typename C::T;
+    constexpr int BK = C::BK;
+    constexpr int EPB = 128 / C::ESZ;
+    constexpr bool F32 = DT == KAN_F32;
+    constexpr bool B_MN = !F32;          // bf16: coef MN-major; fp32: coef^T K-major
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+
+    const int BN = a.BN, stages = a.stages;
+    const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)BN * 128;
+    const uint32_t stage_bytes = (a_bytes + b_bytes) * C::SPLIT;
+    const uint32_t sbase = smem_addr(smem);
+    float* staging = reinterpret_cast<float*>(smem + stages * stage_bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes + 4 * 32 * a.ld_stage * 4);
+    // full[S] empty[S] acc_full[2] acc_empty[2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 4);
+    auto full = [&](int s) { return smem_addr(&bars[s]); };
+    auto empty = [&](int s) { return smem_addr(&bars[stages + s]); };
+    auto acc_full = [&](int b) { return smem_addr(&bars[2 * stages + b]); };
+    auto acc_empty = [&](int b) { return smem_addr(&bars[2 * stages + 2 + b]); };
+    auto A_hi = [&](int s) { return sbase + s * stage_bytes; };
+    auto A_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes; };
+    auto B_hi = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT; };
+    auto B_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT + b_bytes; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t acc_cols = F32 ? 2u * BN : (uint32_t)BN;   // one buffer: [main | corr] or [acc]
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(acc_full(0), 1);
+        mbar_init(acc_full(1), 1);
+        mbar_init(acc_empty(0), 128);
+        mbar_init(acc_empty(1), 128);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // tiles of this CTA: t = blockIdx.x + k * gridDim.x; (batch tile, input group) = (t / n_tiles_n, t % n_tiles_n)
+    const int my_tiles = a.n_tiles > (int)blockIdx.x ? (a.n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    auto tile_coords = [&](int lt, int64_t& m0, int& i0) {
+        const int t = (int)blockIdx.x + lt * (int)gridDim.x;
+        m0 = (int64_t)(t / a.n_tiles_n) * kBM;
+        i0 = (t % a.n_tiles_n) * a.n_in_tile;
+    };
+    auto kt_start = [&](int i0) {
+        return B_MN ? (i0 * a.nb) / (16 / C::ESZ) * (16 / C::ESZ) : i0 * a.nb;
+    };
+
+    if (warp == 0) {
+        if (lane == 0 && my_tiles > 0) {
+            prefetch_tmap(&tA_hi);
+            prefetch_tmap(&tB_hi);
+            int g = 0;   // k-block counter over all tiles (stage ring position)
+            bool ok = true;
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                int64_t m0;
+                int i0;
+                tile_coords(lt, m0, i0);
+                const int kt0 = kt_start(i0);
+                for (int kb = 0; kb < a.nkb; ++kb, ++g) {
+                    const int s = g % stages;
+                    const uint32_t ph = (g / stages) & 1;
+                    if (!mbar_wait(empty(s), ph ^ 1, a.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(full(s), (a_bytes + b_bytes) * C::SPLIT);
+                    tma_load_2d(A_hi(s), &tA_hi, full(s), kb * BK, (int)m0);
+                    if (F32) tma_load_2d(A_lo(s), &tA_lo, full(s), kb * BK, (int)m0);
+                    if (B_MN) {
+                        for (int c = 0; c < BN / EPB; ++c)
+                            tma_load_2d(B_hi(s) + (uint32_t)c * BK * 128, &tB_hi, full(s), kt0 + c * EPB, kb * BK);
+                    } else {
+                        tma_load_2d(B_hi(s), &tB_hi, full(s), kb * BK, kt0);
+                        tma_load_2d(B_lo(s), &tB_lo, full(s), kb * BK, kt0);
+                    }
+                }
+            }
+            for (int q = max(0, g - stages); q < g; ++q) mbar_wait(full(q % stages), (q / stages) & 1, a.status);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && my_tiles > 0) {
+            const uint32_t idesc = instr_desc(C::FMT, 0, B_MN ? 1u : 0u, kBM, BN);
+            const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
+            const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
+            int g = 0;
+            bool ok = true;
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                const int buf = lt & 1;
+                if (lt >= 2 && !mbar_wait(acc_empty(buf), ((lt >> 1) - 1) & 1, a.status)) break;
+                tc_fence_after();
+                const uint32_t d_main = tmem + buf * acc_cols, d_corr = d_main + BN;
+                for (int kb = 0; kb < a.nkb; ++kb, ++g) {
+                    const int s = g % stages;
+                    const uint32_t ph = (g / stages) & 1;
+                    if (!mbar_wait(full(s), ph, a.status)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = smem_desc_sw128(A_hi(s) + ks * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(B_hi(s) + ks * b_step, b_lbo, 1024);
+                        const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
+                        if constexpr (!F32) {
+                            mma_bf16_ss(d_main, ad, bd, idesc, acc);
+                        } else {
+                            const uint64_t adl = smem_desc_sw128(A_lo(s) + ks * 32, 16, 1024);
+                            const uint64_t bdl = smem_desc_sw128(B_lo(s) + ks * b_step, b_lbo, 1024);
+                            mma_tf32_ss(d_corr, adl, bd, idesc, acc);
+                            mma_tf32_ss(d_corr, ad, bdl, idesc, 1u);
+                            mma_tf32_ss(d_main, ad, bd, idesc, acc);
+                        }
+                    }
+                    mma_commit(empty(s));
+                }
+                if (ok) mma_commit(acc_full(buf));
+            }
+        }
+    } else {
+        // ---------------- epilogue: warps 2-5 ----------------
+        const int q = warp & 3;
+        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+        const int r = 32 * q + lane;
+        float* srow = staging + (size_t)(warp - 2) * 32 * a.ld_stage + (size_t)lane * a.ld_stage;
+        constexpr int XC = 16;
+        for (int lt = 0; lt < my_tiles; ++lt) {
+            int64_t m0;
+            int i0;
+            tile_coords(lt, m0, i0);
+            const int64_t b = m0 + r;
+            const int i1 = min((int)a.in, i0 + a.n_in_tile);
+            const int kt_al = kt_start(i0);
+            // x (and dY.w_base) of the first inputs, ahead of the accumulator
+            uint32_t xa[XC], ga[XC];
+            auto xfetch = [&](int i_start) {
+#pragma unroll
+                for (int k = 0; k < XC; ++k) {
+                    const int i = i_start + k;
+                    const bool okk = b < a.batch && i < i1;
+                    xa[k] = okk ? __float_as_uint(to_f(reinterpret_cast<const T*>(a.x)[b * a.in + i])) : 0u;
+                    ga[k] = (okk && a.gb) ? __float_as_uint(a.gb[b * a.in + i]) : 0u;
+                }
+            };
+            xfetch(i0);
+            const int buf = lt & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(acc_full(buf), (lt >> 1) & 1, a.status))) break;
+            tc_fence_after();
+            // stage the row: TMEM -> registers -> shared (16-byte stores; the row
+            // stride is 4 words mod 32, so a warp's stores are conflict-free)
+            const uint32_t t_main = tmem + buf * acc_cols + lane_off;
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(t_main + c0, v);
+                if constexpr (F32) {
+                    uint32_t w[16];
+                    tmem_ld16(t_main + BN + c0, w);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(w[e]));
+                } else {
+                    tmem_ld_wait();
+                }
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<uint4*>(srow + c0 + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            }
+            // the accumulator buffer is free for the tile after next
+            tc_fence_before();
+            mbar_arrive(acc_empty(buf));
+            if (b < a.batch) {
+                T* dxr = reinterpret_cast<T*>(a.dx) + b * a.in;
+                for (int ic = i0; ic < i1; ic += XC) {
+                    uint32_t xc[XC], gc[XC];
+#pragma unroll
+                    for (int k = 0; k < XC; ++k) {
+                        xc[k] = xa[k];
+                        gc[k] = ga[k];
+                    }
+                    if (ic + XC < i1) xfetch(ic + XC);
+#pragma unroll
+                    for (int k = 0; k < XC; ++k) {
+                        const int i = ic + k;
+                        if (i >= i1) break;
+                        const float xv = __uint_as_float(xc[k]);
+                        const Span sp = span_of(xv, a.lo, a.inv_h, a.G);
+                        float acc = 0.0f;
+                        if (sp.valid) {
+                            float d[4];
+                            dweights(sp.t, a.inv_h, d);
+                            const int cb = i * a.nb - kt_al;
+#pragma unroll
+                            for (int qq = 0; qq < 4; ++qq) {
+                                const int m = sp.s + qq;
+                                if (m >= 0 && m < a.nb) acc += srow[cb + m] * d[qq];
+                            }
+                        }
+                        if (a.gb) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
+                        dxr[i] = from_f<T>(acc);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 // y[e] = sum over splits z (ascending) of part[z][e].
 template <typename T>
 __global__ void reduce_splits_kernel(const float* __restrict__ part, T* __restrict__ y, int64_t n, int splits)
@@ -1029,6 +1277,9 @@ struct Plan {
     int64_t ldb;   // padded row length of dY^T (fp32)
     // dx
     int x_BN, x_stages, x_n, x_m, x_nin, x_nkb;
+    // dx, persistent kernel (used when p_ok)
+    bool p_ok;
+    int p_BN, p_stages, p_nin, p_ntn, p_tiles, p_ld, p_grid, p_smem;
     // dY . w_base
     int g_BN, g_stages, g_n, g_m;
     Layout fwd, bwd;
@@ -1071,6 +1322,23 @@ Plan make_plan(const Problem& p, int sms)
     P.x_n = (int)cdiv(p.in, P.x_nin);
     P.x_m = (int)cdiv(p.batch, kBM);
     P.x_nkb = (int)cdiv(p.out, BK);
+    // dx, persistent: BN 192 (bf16) / 128 (fp32), double-buffered TMEM, staged epilogue
+    {
+        P.p_BN = f32 ? 128 : 192;
+        const int pmaxoff = f32 ? 0 : ((p.nb % 8 == 0) ? 0 : 7);
+        P.p_nin = (P.p_BN - pmaxoff) / p.nb;
+        P.p_ld = P.p_BN + 4;
+        const int staging = 4 * 32 * P.p_ld * 4;
+        const int stage_bytes = (kBM * 128 + P.p_BN * 128) * (f32 ? 2 : 1);
+        P.p_stages = std::min(6, (232448 - 1024 - 256 - staging) / stage_bytes);
+        P.p_ok = P.p_nin >= 1 && P.p_stages >= 2 && (!f32 || P.x_nkb <= 32);
+        if (P.p_ok) {
+            P.p_ntn = (int)cdiv(p.in, P.p_nin);
+            P.p_tiles = P.p_ntn * P.x_m;
+            P.p_grid = std::max(1, std::min(P.p_tiles, sms));
+            P.p_smem = P.p_stages * stage_bytes + staging + 1024 + 256;
+        }
+    }
     // dY . w_base: M = batch, N = in, K = out
     P.g_BN = bn_for(p.in, f32, true);
     P.g_stages = stages_for(P.g_BN, f32);
@@ -1172,6 +1440,22 @@ cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap
         return f32 ? launch<MODE, KAN_F32, 1>(grid, BN, stages, maps, args, st)
                    : launch<MODE, KAN_BF16, 1>(grid, BN, stages, maps, args, st);
     }
+}
+
+template <int DT>
+cudaError_t launch_dx_persistent(const Plan& P, const CUtensorMap* maps, const DxArgs& d, cudaStream_t st)
+{
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(dx_persistent_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             232448);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    if (P.p_smem > 232448 || d.BN % 16 != 0 || d.stages < 2) return cudaErrorInvalidConfiguration;
+    dx_persistent_kernel<DT><<<P.p_grid, kDxThreads, P.p_smem, st>>>(maps[0], maps[1], maps[2], maps[3], d);
+    count_launch();
+    return cudaGetLastError();
 }
 
 TcArgs base_args(const Problem& p)
@@ -1397,6 +1681,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             if (e != cudaSuccess) return e;
         }
         CUtensorMap maps[6];
+        const int xBN = P.p_ok ? P.p_BN : P.x_BN;
         if (!make_map_2d(&maps[0], dy_hi, f32, p.batch, p.out, kBM, BK, detail) ||
             !make_map_2d(&maps[1], dy_lo, f32, p.batch, p.out, kBM, BK, detail))
             return cudaErrorInvalidValue;
@@ -1404,8 +1689,8 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             const void *th, *tl;
             if ((e = split_t_into(coef, p.out, p.Kt, p.out, w + P.bwd.coef_hl, &th, &tl, st)) != cudaSuccess)
                 return e;
-            if (!make_map_2d(&maps[2], th, true, p.Kt, p.out, P.x_BN, BK, detail) ||
-                !make_map_2d(&maps[3], tl, true, p.Kt, p.out, P.x_BN, BK, detail))
+            if (!make_map_2d(&maps[2], th, true, p.Kt, p.out, xBN, BK, detail) ||
+                !make_map_2d(&maps[3], tl, true, p.Kt, p.out, xBN, BK, detail))
                 return cudaErrorInvalidValue;
         } else {
             if (!make_map_2d(&maps[2], coef, false, p.out, p.Kt, BK, EPB, detail)) return cudaErrorInvalidValue;
@@ -1413,17 +1698,41 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         }
         maps[4] = maps[2];
         maps[5] = maps[3];
-        TcArgs a = base_args(p);
-        a.x = x;
-        a.out = dx;
-        a.out2 = gb;
-        a.BN = P.x_BN;
-        a.stages = P.x_stages;
-        a.nkb_main = a.nkb_total = P.x_nkb;
-        a.kb_per_split = P.x_nkb;
-        a.n_in_tile = P.x_nin;
-        e = launch_dt<DX>(f32, dim3(P.x_n, P.x_m, 1), P.x_BN, P.x_stages, maps, a, st);
-        if (e != cudaSuccess) return e;
+        if (P.p_ok) {
+            DxArgs d{};
+            d.x = x;
+            d.dx = dx;
+            d.gb = gb;
+            d.status = device_status_ptr();
+            d.batch = p.batch;
+            d.in = p.in;
+            d.out = p.out;
+            d.G = p.G;
+            d.nb = p.nb;
+            d.lo = p.lo;
+            d.inv_h = p.inv_h;
+            d.BN = P.p_BN;
+            d.stages = P.p_stages;
+            d.nkb = P.x_nkb;
+            d.n_in_tile = P.p_nin;
+            d.n_tiles_n = P.p_ntn;
+            d.n_tiles = P.p_tiles;
+            d.ld_stage = P.p_ld;
+            e = f32 ? launch_dx_persistent<KAN_F32>(P, maps, d, st) : launch_dx_persistent<KAN_BF16>(P, maps, d, st);
+            if (e != cudaSuccess) return e;
+        } else {
+            TcArgs a = base_args(p);
+            a.x = x;
+            a.out = dx;
+            a.out2 = gb;
+            a.BN = P.x_BN;
+            a.stages = P.x_stages;
+            a.nkb_main = a.nkb_total = P.x_nkb;
+            a.kb_per_split = P.x_nkb;
+            a.n_in_tile = P.x_nin;
+            e = launch_dt<DX>(f32, dim3(P.x_n, P.x_m, 1), P.x_BN, P.x_stages, maps, a, st);
+            if (e != cudaSuccess) return e;
+        }
     }
     return cudaSuccess;
 }
