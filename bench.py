@@ -175,7 +175,7 @@ class ClockSampler:
         q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
-        cmd = ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100"]
+        cmd = ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "50"]
         if uuid:
             cmd += ["-i", uuid]
         try:
@@ -197,12 +197,15 @@ class ClockSampler:
             f = [t.strip() for t in line.split(",")]
             if len(f) >= 8:
                 try:
-                    rows.append((float(f[0]), float(f[1]), f[3:]))
+                    rows.append((float(f[0]), float(f[1]), f[3:], float(f[2])))
                 except ValueError:
                     pass
         if not rows:
             return None
-        sm = sorted(r[0] for r in rows)
+        # "under load": samples drawing at least half the peak power seen
+        pmax = max(r[3] for r in rows)
+        loaded = [r for r in rows if r[3] >= 0.5 * pmax] or rows
+        sm = sorted(r[0] for r in loaded)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = set()
         for r in rows:
@@ -210,7 +213,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
-                "samples": len(rows)}
+                "samples": len(rows), "samples_under_load": len(loaded), "power_w_max": pmax}
 
 
 # ---------------------------------------------------------------------------
@@ -320,6 +323,7 @@ def run_ours(args, world, rank, local):
         if world > 1:
             torch.distributed.barrier()
 
+    sampler = ClockSampler(local)   # started before the warm-up so that it is sampling by the timed region
     for _ in range(args.warmup):
         flush.zero_()
         for _, c in calls:
@@ -334,7 +338,6 @@ def run_ours(args, world, rank, local):
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
           for _ in range(K)]
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    sampler = ClockSampler(local)
     barrier()
     torch.cuda.synchronize(dev)
     n0 = N.kan_launch_count()
@@ -429,8 +432,8 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=W.BENCH_DEFAULT, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")

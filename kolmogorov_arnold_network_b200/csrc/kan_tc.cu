@@ -38,6 +38,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <mutex>
 
 #include "kan_device.cuh"
@@ -93,6 +94,7 @@ struct TcArgs {
     int n_in_tile;             // DX: inputs per N tile
     int has_base;
     uint32_t nb_magic;         // ceil(2^32 / nb): c / nb == umulhi(c, nb_magic) for c < 2^32 / nb
+    int fbox;                  // FWD: rows per B box
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
@@ -164,6 +166,75 @@ __device__ __forceinline__ void put_a_chunk(uint32_t a_hi, uint32_t a_lo, uint32
     }
 }
 
+// Floor of u (|u| < 2^22) without the conversion unit: adding 1.5*2^23 with
+// round-down leaves floor(u) in the low mantissa bits.
+__device__ __forceinline__ void floor_split(float u, int& s, float& f)
+{
+    const float r = __fadd_rd(u, 12582912.0f);
+    f = r - 12582912.0f;
+    s = __float_as_int(r) - 0x4B400000;
+}
+
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v2f(uint32_t addr, float a, float b)
+{
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+
+// Byte offset of element column c inside one 128-byte swizzled row (row & 7 = rx).
+template <int ESZ>
+__device__ __forceinline__ uint32_t sw_col(int c, uint32_t rx)
+{
+    const uint32_t cb = (uint32_t)c * ESZ;
+    return ((((cb >> 4) ^ rx) & 7u) << 4) | (cb & 15u);
+}
+
+// The four weights of one input at columns col0..col0+3 of a 128-byte
+// swizzled row (basis indices sidx..sidx+3); entries whose basis index is
+// outside 0..nb-1 or whose column is outside 0..ncols-1 are skipped.  One
+// predicated store per entry keeps the warp convergent.
+template <int DT>
+__device__ __forceinline__ void scatter4(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx, int col0, int sidx, int nb,
+                                         int ncols, const float (&w)[4])
+{
+    constexpr int ESZ = DT == KAN_F32 ? 4 : 2;
+    if constexpr (DT == KAN_BF16) {
+        const __nv_bfloat162 a01 = __floats2bfloat162_rn(w[0], w[1]);
+        const __nv_bfloat162 a23 = __floats2bfloat162_rn(w[2], w[3]);
+        const uint32_t p01 = *reinterpret_cast<const uint32_t*>(&a01);
+        const uint32_t p23 = *reinterpret_cast<const uint32_t*>(&a23);
+        const uint16_t h[4] = {(uint16_t)(p01 & 0xFFFFu), (uint16_t)(p01 >> 16), (uint16_t)(p23 & 0xFFFFu),
+                               (uint16_t)(p23 >> 16)};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if ((unsigned)(sidx + q) < (unsigned)nb && (unsigned)(col0 + q) < (unsigned)ncols)
+                st_shared_u16(rb_hi + sw_col<ESZ>(col0 + q, rx), h[q]);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if ((unsigned)(sidx + q) < (unsigned)nb && (unsigned)(col0 + q) < (unsigned)ncols) {
+                const float hi = tf32_hi(w[q]);
+                st_shared_f32(rb_hi + sw_col<ESZ>(col0 + q, rx), hi);
+                st_shared_f32(rb_lo + sw_col<ESZ>(col0 + q, rx), w[q] - hi);
+            }
+    }
+}
+
+// The four local weights on the bounded coordinate t in [0,1) (see weights()).
+__device__ __forceinline__ void weights_fma(float t, float (&w)[4])
+{
+    const float sm = 1.0f - t;
+    const float t2 = t * t, s2 = sm * sm;
+    w[0] = s2 * sm * (1.0f / 6.0f);
+    w[1] = fmaf(t2, fmaf(t, 0.5f, -1.0f), 2.0f / 3.0f);
+    w[2] = fmaf(s2, fmaf(sm, 0.5f, -1.0f), 2.0f / 3.0f);
+    w[3] = t2 * t * (1.0f / 6.0f);
+}
+
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
@@ -215,7 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nk = kb_end - kb_begin;
     const int nseg = F32 ? (nk + a.seg_kb - 1) / a.seg_kb : 1;
     // TMEM columns: bf16 [acc]; fp32 [main0 | main1 | corr | total]
-    const uint32_t tmem_cols = F32 ? 512u : (BN <= 32 ? 32u : (BN <= 64 ? 64u : (BN <= 128 ? 128u : 256u)));
+    const uint32_t tmem_cols =
+        F32 ? 512u : (BN <= 32 ? 32u : (BN <= 64 ? 64u : (BN <= 128 ? 128u : (BN <= 256 ? 256u : 512u))));
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -265,13 +337,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t bytes = (b_bytes + (A_BY_TMA ? a_bytes : 0u)) * C::SPLIT;
                 mbar_arrive_expect_tx(full_b(s), bytes);
                 if (MODE == FWD) {
-                    if (kb < a.nkb_main) {
-                        tma_load_2d(B_hi(s), &tB_hi, full_b(s), kb * BK, n0);
-                        if (F32) tma_load_2d(B_lo(s), &tB_lo, full_b(s), kb * BK, n0);
-                    } else {
-                        const int kc = (kb - a.nkb_main) * BK;
-                        tma_load_2d(B_hi(s), &tB2_hi, full_b(s), kc, n0);
-                        if (F32) tma_load_2d(B_lo(s), &tB2_lo, full_b(s), kc, n0);
+                    // boxes of at most 128 rows (a.fbox): a wide tile is several of them
+                    const bool spline = kb < a.nkb_main;
+                    const int kc = spline ? kb * BK : (kb - a.nkb_main) * BK;
+                    for (int h = 0; h * a.fbox < BN; ++h) {
+                        const uint32_t off = (uint32_t)(h * a.fbox) * 128u;
+                        tma_load_2d(B_hi(s) + off, spline ? (const void*)&tB_hi : (const void*)&tB2_hi, full_b(s), kc,
+                                    n0 + h * a.fbox);
+                        if (F32)
+                            tma_load_2d(B_lo(s) + off, spline ? (const void*)&tB_lo : (const void*)&tB2_lo, full_b(s),
+                                        kc, n0 + h * a.fbox);
                     }
                 } else {
                     if (A_BY_TMA) {
@@ -298,7 +373,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issue ----------------
         if (lane == 0 && nk > 0) {
-            const uint32_t idesc = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, BN);
+            // a 384- or 512-wide bf16 tile runs as an N=256 MMA plus an N=BN-256 MMA
+            // into consecutive TMEM columns
+            const int mma_n = BN > 256 ? 256 : BN;
+            const uint32_t idesc = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, mma_n);
+            const uint32_t idesc2 = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, BN > 256 ? BN - 256 : 16);
+            // offset of B's columns 256..: 256 rows (K-major) or four 64-column atoms (MN-major)
+            const uint32_t b_half = B_MN ? 4u * BK * 128u : 256u * 128u;
             const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
             const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
             const uint32_t a_lbo = A_MN ? (uint32_t)BK * 128u : 16u;
@@ -323,6 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = smem_desc_sw128(B_hi(s) + ks * b_step, b_lbo, 1024);
                     if constexpr (!F32) {
                         mma_bf16_ss(t_main0, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+                        if (BN > 256) {
+                            const uint64_t bd2 = smem_desc_sw128(B_hi(s) + b_half + ks * b_step, b_lbo, 1024);
+                            mma_bf16_ss(t_main0 + 256u, ad, bd2, idesc2, (it > 0 || ks > 0) ? 1u : 0u);
+                        }
                     } else {
                         const uint64_t adl = smem_desc_sw128(A_lo(s) + ks * a_step, a_lbo, 1024);
                         const uint64_t bdl = smem_desc_sw128(B_lo(s) + ks * b_step, b_lbo, 1024);
@@ -399,31 +484,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if (k >= n) break;
                                 const float u = fmaf(cur[k], a.inv_h, u0);
                                 if (!(u >= -3.0f && u < u_hi)) continue;   // outside the extended knots, NaN, inf
-                                const float f = floorf(u);
-                                const int sidx = (int)f;
-                                const float t = u - f, sm = 1.0f - t;
-                                const float t2 = t * t, s2 = sm * sm;
+                                int sidx;
+                                float f;
+                                floor_split(u, sidx, f);
                                 float w[4];
-                                w[0] = s2 * sm * (1.0f / 6.0f);
-                                w[1] = fmaf(t2, fmaf(t, 0.5f, -1.0f), 2.0f / 3.0f);
-                                w[2] = fmaf(s2, fmaf(sm, 0.5f, -1.0f), 2.0f / 3.0f);
-                                w[3] = t2 * t * (1.0f / 6.0f);
-                                const int col0 = cbase + k * a.nb + sidx;
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const int col = col0 + q;
-                                    if ((unsigned)(sidx + q) < (unsigned)a.nb && (unsigned)col < (unsigned)BK) {
-                                        const uint32_t cb = (uint32_t)col * C::ESZ;
-                                        const uint32_t off = rbase + ((((cb >> 4) ^ rx) & 7u) << 4) + (cb & 15u);
-                                        if constexpr (!F32) {
-                                            st_shared_u16(ahi + off, __bfloat16_as_ushort(__float2bfloat16_rn(w[q])));
-                                        } else {
-                                            const float hi = tf32_hi(w[q]);
-                                            st_shared_f32(ahi + off, hi);
-                                            st_shared_f32(alo + off, w[q] - hi);
-                                        }
-                                    }
-                                }
+                                weights_fma(u - f, w);
+                                scatter4<DT>(ahi + rbase, alo + rbase, rx, cbase + k * a.nb + sidx, sidx, a.nb, BK, w);
                             }
                         }
                     } else {
@@ -510,25 +576,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if (k >= n_inp) break;
                                 const float u = fmaf(cur[k], a.inv_h, u0);
                                 if (!(u >= -3.0f && u < u_hi)) continue;
-                                const float f = floorf(u);
-                                const int sidx = (int)f;
-                                const float t = u - f, sm = 1.0f - t;
-                                const float t2 = t * t, s2 = sm * sm;
+                                int sidx;
+                                float f;
+                                floor_split(u, sidx, f);
                                 float w[4];
-                                w[0] = s2 * sm * (1.0f / 6.0f);
-                                w[1] = fmaf(t2, fmaf(t, 0.5f, -1.0f), 2.0f / 3.0f);
-                                w[2] = fmaf(s2, fmaf(sm, 0.5f, -1.0f), 2.0f / 3.0f);
-                                w[3] = t2 * t * (1.0f / 6.0f);
-                                const int col0 = cbase + k * a.nb + sidx;
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const int col = col0 + q;
-                                    if ((unsigned)(sidx + q) < (unsigned)a.nb && (unsigned)col < 64u) {
-                                        const uint32_t cb = (uint32_t)col * 2u;
-                                        st_shared_u16(rbase + ((((cb >> 4) ^ rx) & 7u) << 4) + (cb & 15u),
-                                                      __bfloat16_as_ushort(__float2bfloat16_rn(w[q])));
-                                    }
-                                }
+                                weights_fma(u - f, w);
+                                scatter4<KAN_BF16>(rbase, rbase, rx, cbase + k * a.nb + sidx, sidx, a.nb, 64, w);
                             }
                         }
                     } else {
@@ -910,8 +963,11 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)BN * 128;
     const uint32_t stage_bytes = (a_bytes + b_bytes) * C::SPLIT;
     const uint32_t sbase = smem_addr(smem);
-    float* staging = reinterpret_cast<float*>(smem + stages * stage_bytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes + 4 * 32 * a.ld_stage * 4);
+    // staging of the accumulator rows: fp32 for fp32 operands, bf16 for bf16
+    // operands (the dx it feeds is rounded to bf16 anyway)
+    using ST = typename std::conditional<F32, float, __nv_bfloat16>::type;
+    ST* staging = reinterpret_cast<ST*>(smem + stages * stage_bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes + 4 * 32 * a.ld_stage * (int)sizeof(ST));
     // full[S] empty[S] acc_full[2] acc_empty[2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 4);
     auto full = [&](int s) { return smem_addr(&bars[s]); };
@@ -1026,7 +1082,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         const int q = warp & 3;
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         const int r = 32 * q + lane;
-        float* srow = staging + (size_t)(warp - 2) * 32 * a.ld_stage + (size_t)lane * a.ld_stage;
+        ST* srow = staging + (size_t)(warp - 2) * 32 * a.ld_stage + (size_t)lane * a.ld_stage;
         constexpr int XC = 16;
         for (int lt = 0; lt < my_tiles; ++lt) {
             int64_t m0;
@@ -1051,7 +1107,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             if (!__all_sync(0xffffffffu, mbar_wait(acc_full(buf), (lt >> 1) & 1, a.status))) break;
             tc_fence_after();
             // stage the row: TMEM -> registers -> shared (16-byte stores; the row
-            // stride is 4 words mod 32, so a warp's stores are conflict-free)
+            // stride is 16 bytes mod 128, so a warp's stores are conflict-free)
             const uint32_t t_main = tmem + buf * acc_cols + lane_off;
             for (int c0 = 0; c0 < BN; c0 += 16) {
                 uint32_t v[16];
@@ -1065,9 +1121,17 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                 } else {
                     tmem_ld_wait();
                 }
+                if constexpr (F32) {
 #pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<uint4*>(srow + c0 + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<uint4*>(srow + c0 + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                } else {
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                    *reinterpret_cast<uint4*>(srow + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4*>(srow + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
             }
             // the accumulator buffer is free for the tile after next
             tc_fence_before();
@@ -1096,7 +1160,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 #pragma unroll
                             for (int qq = 0; qq < 4; ++qq) {
                                 const int m = sp.s + qq;
-                                if (m >= 0 && m < a.nb) acc += srow[cb + m] * d[qq];
+                                if (m >= 0 && m < a.nb) acc += to_f(srow[cb + m]) * d[qq];
                             }
                         }
                         if (a.gb) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
@@ -1249,6 +1313,25 @@ int bn_for(int64_t n, bool f32, bool mn_major = false)
     return bn;
 }
 
+// bf16 tile width over `out` columns for the kernels whose basis operand is
+// produced on chip: wider tiles reuse each produced A tile for more MMA
+// work.  Among 256, 384 and 512 the one with the least padding wins, ties
+// going to the wider; small `out` keeps the power-of-two width.
+int wide_bn(int64_t out)
+{
+    if (out <= 256) return bn_for(out, false);
+    int best = 256;
+    int64_t best_pad = cdiv(out, 256) * 256;
+    for (int bn : {384, 512}) {
+        const int64_t pad = cdiv(out, bn) * bn;
+        if (pad <= best_pad) {
+            best_pad = pad;
+            best = bn;
+        }
+    }
+    return best;
+}
+
 int stages_for(int BN, bool f32)
 {
     const int stage_bytes = (kBM * 128 + BN * 128) * (f32 ? 2 : 1);
@@ -1292,7 +1375,7 @@ Plan make_plan(const Problem& p, int sms)
     const int BK = f32 ? 32 : 64;
     const size_t esz = f32 ? 4 : 2;
     // forward: M = batch, N = out, K = spline (+ SiLU) columns
-    P.f_BN = bn_for(p.out, f32);
+    P.f_BN = f32 ? bn_for(p.out, true) : wide_bn(p.out);
     P.f_stages = stages_for(P.f_BN, f32);
     P.f_n = (int)cdiv(p.out, P.f_BN);
     P.f_m = (int)cdiv(p.batch, kBM);
@@ -1302,7 +1385,7 @@ Plan make_plan(const Problem& p, int sms)
     P.f_kps = (int)cdiv(P.f_nkb_total, P.f_splits);
     P.f_splits = (int)cdiv(P.f_nkb_total, P.f_kps);
     // dcoef: M = spline columns (+ SiLU rows), N = out, K = batch
-    P.d_BN = bn_for(p.out, f32, true);
+    P.d_BN = f32 ? bn_for(p.out, true, true) : std::max(64, wide_bn(p.out));
     P.d_n = (int)cdiv(p.out, P.d_BN);
     P.d_nkt = (int)cdiv(p.Kt, kBM);
     P.d_m = P.d_nkt + (p.base ? (int)cdiv(p.in, kBM) : 0);
@@ -1324,11 +1407,11 @@ Plan make_plan(const Problem& p, int sms)
     P.x_nkb = (int)cdiv(p.out, BK);
     // dx, persistent: BN 192 (bf16) / 128 (fp32), double-buffered TMEM, staged epilogue
     {
-        P.p_BN = f32 ? 128 : 192;
+        P.p_BN = f32 ? 128 : 256;
         const int pmaxoff = f32 ? 0 : ((p.nb % 8 == 0) ? 0 : 7);
         P.p_nin = (P.p_BN - pmaxoff) / p.nb;
-        P.p_ld = P.p_BN + 4;
-        const int staging = 4 * 32 * P.p_ld * 4;
+        P.p_ld = f32 ? P.p_BN + 4 : P.p_BN + 8;          // row stride = 16 bytes mod 128
+        const int staging = 4 * 32 * P.p_ld * (f32 ? 4 : 2);
         const int stage_bytes = (kBM * 128 + P.p_BN * 128) * (f32 ? 2 : 1);
         P.p_stages = std::min(6, (232448 - 1024 - 256 - staging) / stage_bytes);
         P.p_ok = P.p_nin >= 1 && P.p_stages >= 2 && (!f32 || P.x_nkb <= 32);
@@ -1395,7 +1478,8 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
 {
     // the MN-major bf16 B operand arrives in whole 128-byte boxes: BN must be a multiple of 64
     if (MODE != FWD && DT == KAN_BF16 && BN % 64 != 0) return cudaErrorInvalidConfiguration;
-    if (BN % 16 != 0 || BN < 16 || BN > 256 || (DT == KAN_F32 && BN > 128) || stages < 2)
+    if (BN % 16 != 0 || BN < 16 || BN > (MODE == FWD || MODE == DCA ? 512 : 256) || (BN > 256 && BN % 128 != 0) ||
+        (DT == KAN_F32 && BN > 128) || stages < 2)
         return cudaErrorInvalidConfiguration;
     const int smem = smem_bytes(BN, stages, DT == KAN_F32);
     static int configured = 0;   // per instantiation; the attribute is per function
@@ -1551,12 +1635,13 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
             return e;
     }
     CUtensorMap maps[6];
-    if (!make_map_2d(&maps[2], c_hi, f32, p.out, p.Kt, P.f_BN, BK, detail) ||
-        !make_map_2d(&maps[3], c_lo, f32, p.out, p.Kt, P.f_BN, BK, detail))
+    const int fbox = std::min(P.f_BN, 128);
+    if (!make_map_2d(&maps[2], c_hi, f32, p.out, p.Kt, fbox, BK, detail) ||
+        !make_map_2d(&maps[3], c_lo, f32, p.out, p.Kt, fbox, BK, detail))
         return cudaErrorInvalidValue;
     if (p.base) {
-        if (!make_map_2d(&maps[4], wb_hi, f32, p.out, p.in, P.f_BN, BK, detail) ||
-            !make_map_2d(&maps[5], wb_lo, f32, p.out, p.in, P.f_BN, BK, detail))
+        if (!make_map_2d(&maps[4], wb_hi, f32, p.out, p.in, fbox, BK, detail) ||
+            !make_map_2d(&maps[5], wb_lo, f32, p.out, p.in, fbox, BK, detail))
             return cudaErrorInvalidValue;
     } else {
         maps[4] = maps[2];
@@ -1569,6 +1654,7 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
     a.out = P.f_splits > 1 ? (void*)(w + P.fwd.fwd_part) : y;
     a.BN = P.f_BN;
     a.stages = P.f_stages;
+    a.fbox = fbox;
     a.nkb_main = P.f_nkb_main;
     a.nkb_total = P.f_nkb_total;
     a.kb_per_split = P.f_kps;
