@@ -47,8 +47,16 @@ namespace kan {
 namespace {
 
 constexpr int kBM = 128;          // MMA M: rows of A, TMEM lanes
-constexpr int kThreads = 448;     // 14 warps
-constexpr int kProducers = 256;   // warps 2-9
+constexpr int kProducers = 256;   // producer threads of the DCOEF (fp32) mode
+
+// Producer warps per mode: the row producers (FWD, DCA) run 4 groups of 4
+// warps that take every 4th k-block; DCOEF uses 8 warps on each k-block.
+template <int MODE> struct Warps {
+    static constexpr int kProd = (MODE == 0 || MODE == 4) ? 16 : 8;   // FWD, DCA : others
+    static constexpr int kGroups = kProd / 4;
+    static constexpr int kEpi0 = 2 + kProd;                            // first epilogue warp
+    static constexpr int kThreads = (kEpi0 + 4) * 32;
+};
 constexpr int kEpi = 128;         // warps 10-13
 constexpr int kSmemBudget = 227 * 1024 - 2048;
 
@@ -95,6 +103,7 @@ struct TcArgs {
     int has_base;
     uint32_t nb_magic;         // ceil(2^32 / nb): c / nb == umulhi(c, nb_magic) for c < 2^32 / nb
     int fbox;                  // FWD: rows per B box
+    const void* zeros;         // >= 16 KiB of zeros in global memory (the A tiles' zero fill)
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
@@ -239,7 +248,7 @@ __device__ __forceinline__ void weights_fma(float t, float (&w)[4])
 // The kernel
 // ---------------------------------------------------------------------------
 template <int MODE, int DT, int MAXI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
               const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
               const __grid_constant__ CUtensorMap tB2_hi, const __grid_constant__ CUtensorMap tB2_lo,
@@ -267,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase = smem_addr(smem);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
     // barrier block: full_a[S] full_b[S] empty[S] zeroed[S] seg_full[2] seg_empty[2] accum
+    // (zeroed[s]: the zero fill of stage s's produced tile has landed)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * stages + 5);
     auto full_a = [&](int s) { return smem_addr(&bars[s]); };
     auto full_b = [&](int s) { return smem_addr(&bars[stages + s]); };
@@ -291,10 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
-            mbar_init(full_a(s), (MODE == FWD || MODE == DCA) ? kProducers / 2 : kProducers);
+            mbar_init(full_a(s), (MODE == FWD || MODE == DCA) ? 128 : kProducers);
             mbar_init(full_b(s), 1);
             mbar_init(empty(s), 1);
-            mbar_init(zeroed(s), kProducers);
+            mbar_init(zeroed(s), 1);
         }
         mbar_init(seg_full(0), 1);
         mbar_init(seg_full(1), 1);
@@ -334,6 +344,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ph = (it / stages) & 1;
                 if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
                 const int kb = kb_begin + it;
+                if (PRODUCE) {
+                    // the produced tile starts from zeros: a bulk copy from a zero buffer
+                    // (off the load/store pipe the producers use); dense SiLU tiles skip it
+                    const bool zero_it = MODE == FWD ? kb < a.nkb_main : (int)blockIdx.y < a.n_kt_tiles;
+                    if (zero_it) {
+                        mbar_arrive_expect_tx(zeroed(s), a_bytes * C::SPLIT);
+                        bulk_copy_g2s(A_hi(s), a.zeros, a_bytes, zeroed(s));
+                        if (F32) bulk_copy_g2s(A_lo(s), a.zeros, a_bytes, zeroed(s));
+                    } else {
+                        mbar_arrive(zeroed(s));
+                    }
+                }
                 const uint32_t bytes = (b_bytes + (A_BY_TMA ? a_bytes : 0u)) * C::SPLIT;
                 mbar_arrive_expect_tx(full_b(s), bytes);
                 if (MODE == FWD) {
@@ -367,8 +389,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++issued;
             }
             // every load issued lands before the CTA can exit
-            for (int it = max(0, issued - stages); it < issued; ++it)
+            for (int it = max(0, issued - stages); it < issued; ++it) {
                 mbar_wait(full_b(it % stages), (it / stages) & 1, a.status);
+                if (PRODUCE) mbar_wait(zeroed(it % stages), (it / stages) & 1, a.status);
+            }
         }
     } else if (warp == 1) {
         // ---------------- MMA issue ----------------
@@ -421,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (ok) mma_commit(accum_bar);
         }
-    } else if (warp < 10) {
+    } else if (warp < Warps<MODE>::kEpi0) {
         // ---------------- A producers ----------------
         // Each thread fetches the x values of its next k-block into registers
         // before it waits for and fills the current one, so the global-load
@@ -430,9 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int p = threadIdx.x - 64;
             const T* X = reinterpret_cast<const T*>(a.x);
             if constexpr (MODE == FWD) {
-                // rows = batch m0..m0+127.  Two groups of 128 threads (warps 2-5 and
-                // 6-9) take alternate k-blocks; a thread fills one whole row.  Per
-                // row and k-block at most MAXI inputs have columns in the block.
+                // rows = batch m0..m0+127.  kGroups groups of 128 threads take
+                // k-blocks in turn; a thread fills one whole row.  Per row and
+                // k-block at most MAXI inputs have columns in the block.
                 constexpr int EPC = 16 / C::ESZ;       // elements per 16-byte chunk
                 const uint32_t row = p & (kBM - 1);
                 const int grp = p >> 7;                // warp-uniform
@@ -456,26 +480,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 };
                 float nxt[MAXI];
-                if (grp < nk) fetch(kb_begin + grp, nxt);
+                // At most `stages` groups: then a group's previous k-block is no older
+                // than the previous use of the stage it waits for, so neither the
+                // empty nor the zeroed barrier can be two phases behind (a parity
+                // wait on such a barrier would pass early).
+                const int NG = min(Warps<MODE>::kGroups, stages);
+                if (grp < NG && grp < nk) fetch(kb_begin + grp, nxt);
                 int uses = 0;                               // k-blocks this group has filled
-                for (int it = grp; it < nk; it += 2, ++uses) {
+                for (int it = grp; grp < NG && it < nk; it += NG, ++uses) {
                     float cur[MAXI];
 #pragma unroll
                     for (int k = 0; k < MAXI; ++k) cur[k] = nxt[k];
                     const int kb = kb_begin + it;
-                    if (it + 2 < nk) fetch(kb + 2, nxt);
+                    if (it + NG < nk) fetch(kb + NG, nxt);
                     const int s = it % stages;
                     const uint32_t ph = (it / stages) & 1;
+                    // the stage is free (its previous use consumed) and zero-filled
                     if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
+                    if (!mbar_wait(zeroed(s), ph, a.status)) break;
                     const uint32_t ahi = A_hi(s), alo = A_lo(s);
                     const uint32_t rbase = row * 128u, rx = row & 7u;
                     if (kb < a.nkb_main) {
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const uint32_t off = rbase + ((c ^ rx) << 4);
-                            st_shared_zero16(ahi + off);
-                            if (F32) st_shared_zero16(alo + off);
-                        }
                         if (row_ok) {
                             const int i0 = first_input(kb), n = last_input(kb) - i0 + 1;
                             const int cbase = i0 * a.nb - kb * BK;   // column of input i0's B_0 in this block
@@ -526,8 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if constexpr (MODE == DCA) {
                 // A tile, MN-major: batch rows b0..b0+63 (K) by 128 columns (M) in two
                 // 64-column atoms [64 rows x 128 bytes], BK*128 bytes apart; the columns
-                // are spline columns kt0.. (or, for a SiLU tile, inputs i0..).  Two
-                // groups of 128 threads take alternate k-blocks; a thread fills one
+                // are spline columns kt0.. (or, for a SiLU tile, inputs i0..).  kGroups
+                // groups of 128 threads take k-blocks in turn; a thread fills one
                 // atom row: (batch row rb, atom).
                 const int grp = p >> 7;                    // warp-uniform
                 const int rb = p & (BK - 1);
@@ -552,23 +577,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 };
                 float nxt[MAXI];
-                if (grp < nk) fetch(kb_begin + grp, nxt);
-                for (int it = grp; it < nk; it += 2) {
+                const int NG = min(Warps<MODE>::kGroups, stages);   // see the forward producer
+                if (grp < NG && grp < nk) fetch(kb_begin + grp, nxt);
+                for (int it = grp; grp < NG && it < nk; it += NG) {
                     float cur[MAXI];
 #pragma unroll
                     for (int k = 0; k < MAXI; ++k) cur[k] = nxt[k];
                     const int kb = kb_begin + it;
-                    if (it + 2 < nk) fetch(kb + 2, nxt);
+                    if (it + NG < nk) fetch(kb + NG, nxt);
                     const int s = it % stages;
                     const uint32_t ph = (it / stages) & 1;
                     if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
+                    if (!mbar_wait(zeroed(s), ph, a.status)) break;
                     const int64_t b = (int64_t)kb * BK + rb;
                     const bool row_ok = b < a.batch;
                     const uint32_t rbase = A_hi(s) + (uint32_t)atom * BK * 128u + (uint32_t)rb * 128u;
                     const uint32_t rx = (uint32_t)rb & 7u;
                     if (!silu_tile) {
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) st_shared_zero16(rbase + ((c ^ rx) << 4));
                         if (row_ok) {
                             const int cbase = i_first * a.nb - c_lo;
 #pragma unroll
@@ -670,19 +695,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int s = it % stages;
                     const uint32_t ph = (it / stages) & 1;
                     if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
+                    if (!mbar_wait(zeroed(s), ph, a.status)) break;
                     const uint32_t ahi = A_hi(s), alo = A_lo(s);
                     if (!silu_tile) {
-                        // zero the tile: 128 rows x 8 chunks, 4 chunks per thread
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int e = p * 4 + c;
-                            const uint32_t off = sw128_chunk(e >> 3, e & 7);
-                            st_shared_zero16(ahi + off);
-                            if (F32) st_shared_zero16(alo + off);
-                        }
-                        // every producer's zeros are in place before anyone scatters
-                        mbar_arrive(zeroed(s));
-                        if (!mbar_wait(zeroed(s), ph, a.status)) break;
 #pragma unroll
                         for (int k = 0; k < MAXP; ++k) {
                             if (pc[k] < 0) continue;
@@ -723,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue warps 10-13 ----------------
+        // ---------------- epilogue: the last 4 warps ----------------
         const int q = warp & 3;                       // TMEM lane quarter
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         const uint32_t r = 32 * q + lane;             // tile row of this thread
@@ -868,7 +883,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // DX: Gm row -> shared staging (the pipeline buffers are free now),
                 // then each input's 4 columns times B' (+ silu' * Gb).
                 const int ldst = BN + 1;
-                float* stage = reinterpret_cast<float*>(smem) + (size_t)(warp - 10) * 32 * ldst + (size_t)lane * ldst;
+                float* stage = reinterpret_cast<float*>(smem) + (size_t)(warp - Warps<MODE>::kEpi0) * 32 * ldst +
+                               (size_t)lane * ldst;
                 for (int c0 = 0; c0 < BN; c0 += 16) {
                     float v[16];
                     load16(c0, v);
@@ -1489,7 +1505,8 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
         if (e != cudaSuccess) return e;
         configured = kSmemBudget;
     }
-    tc_kernel<MODE, DT, MAXI><<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], args);
+    tc_kernel<MODE, DT, MAXI><<<grid, Warps<MODE>::kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                                          maps[5], args);
     count_launch();
     return cudaGetLastError();
 }
@@ -1542,6 +1559,24 @@ cudaError_t launch_dx_persistent(const Plan& P, const CUtensorMap* maps, const D
     return cudaGetLastError();
 }
 
+// 16 KiB of zeros: the source of the produced tiles' zero fill.
+static __device__ __align__(128) unsigned char g_zero_tile[16384];
+
+const void* zero_tile_ptr()
+{
+    static void* ptrs[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_zero_tile) != cudaSuccess) return nullptr;
+        ptrs[dev] = p;
+    }
+    return ptrs[dev];
+}
+
 TcArgs base_args(const Problem& p)
 {
     TcArgs a{};
@@ -1557,6 +1592,7 @@ TcArgs base_args(const Problem& p)
     a.seg_kb = kSegKb;
     a.has_base = p.base;
     a.nb_magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)p.nb - 1) / (uint64_t)p.nb);
+    a.zeros = zero_tile_ptr();
     return a;
 }
 
@@ -1623,6 +1659,10 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
                        int num_sms, cudaStream_t st, const char** detail)
 {
     if (p.batch == 0) return cudaSuccess;
+    if (!zero_tile_ptr()) {
+        *detail = "the zero tile's device address is not available";
+        return cudaErrorInvalidValue;
+    }
     const bool f32 = p.dtype == KAN_F32;
     const int BK = f32 ? 32 : 64;
     const Plan P = make_plan(p, num_sms);
@@ -1686,6 +1726,10 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
     const Plan P = make_plan(p, num_sms);
     uint8_t* w = reinterpret_cast<uint8_t*>(ws);
     cudaError_t e;
+    if (!zero_tile_ptr()) {
+        *detail = "the zero tile's device address is not available";
+        return cudaErrorInvalidValue;
+    }
     if (p.batch == 0) {
         if (dcoef && (e = zero_f32(dcoef, p.out * p.Kt, st)) != cudaSuccess) return e;
         if (dw_base && (e = zero_f32(dw_base, p.out * p.in, st)) != cudaSuccess) return e;
