@@ -290,15 +290,29 @@ __device__ __forceinline__ void named_bar_sync(int id, int count)
 // atoms (SBO = 1024, LBO unused); an MN-major tile is a set of
 // [K rows x 128 bytes] column blocks, LBO apart, whose 8-row groups are
 // SBO = 1024 apart.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes)
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint32_t layout)
 {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
     d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
+    d |= (uint64_t)(layout & 7u) << 61;
     return d;
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes)
+{
+    return smem_desc(saddr, lbo_bytes, sbo_bytes, 2u);
+}
+
+// Layout 1: 128-byte rows whose four 32-byte granules are permuted by XOR
+// with (row & 3); the atom is 4 rows (512 bytes).  This is the form an
+// MN-major tf32 operand takes: for it SBO is the stride between 4-row
+// groups along K and LBO the stride between 128-byte column blocks along MN.
+__device__ __forceinline__ uint32_t sw128b32_byte(uint32_t row, uint32_t colb)
+{
+    return row * 128u + ((((colb >> 5) ^ (row & 3u)) & 3u) << 5) + (colb & 31u);
 }
 
 // Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation:

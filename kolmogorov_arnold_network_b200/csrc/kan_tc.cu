@@ -262,7 +262,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     constexpr bool PRODUCE = MODE == FWD || MODE == DCOEF || MODE == DCA;
     constexpr bool A_BY_TMA = MODE == DX || MODE == GEMM;
     constexpr bool A_MN = MODE == DCA;               // producer-written MN-major basis
-    static_assert(MODE != DCA || DT == KAN_BF16, "DCA is the bf16 dcoef path");
+    // an MN-major tf32 operand uses the 32-byte-atom 128-byte swizzle (layout 1)
+    constexpr bool A_SW32 = A_MN && F32;
     // B stored MN-major (dY for dcoef, coef / w_base for dx) for bf16; the
     // fp32 path's split copies are transposed to K-major instead (tf32
     // MN-major operands would need the 32-byte-atom swizzle).
@@ -408,6 +409,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
             const uint32_t a_lbo = A_MN ? (uint32_t)BK * 128u : 16u;
             const uint32_t a_step = A_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
+            const uint32_t a_sbo = A_SW32 ? 512u : 1024u;
+            const uint32_t a_layout = A_SW32 ? 1u : 2u;
             bool ok = true;
             for (int it = 0; it < nk && ok; ++it) {
                 const int s = it % stages;
@@ -424,7 +427,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const uint32_t t_main = (g & 1) ? t_main1 : t_main0;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ad = smem_desc_sw128(A_hi(s) + ks * a_step, a_lbo, 1024);
+                    const uint64_t ad = smem_desc(A_hi(s) + ks * a_step, a_lbo, a_sbo, a_layout);
                     const uint64_t bd = smem_desc_sw128(B_hi(s) + ks * b_step, b_lbo, 1024);
                     if constexpr (!F32) {
                         mma_bf16_ss(t_main0, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
@@ -433,7 +436,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                             mma_bf16_ss(t_main0 + 256u, ad, bd2, idesc2, (it > 0 || ks > 0) ? 1u : 0u);
                         }
                     } else {
-                        const uint64_t adl = smem_desc_sw128(A_lo(s) + ks * a_step, a_lbo, 1024);
+                        const uint64_t adl = smem_desc(A_lo(s) + ks * a_step, a_lbo, a_sbo, a_layout);
                         const uint64_t bdl = smem_desc_sw128(B_lo(s) + ks * b_step, b_lbo, 1024);
                         mma_tf32_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                         mma_tf32_ss(t_corr, ad, bdl, idesc, 1u);
@@ -549,18 +552,20 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 }
                 (void)uses;
             } else if constexpr (MODE == DCA) {
-                // A tile, MN-major: batch rows b0..b0+63 (K) by 128 columns (M) in two
-                // 64-column atoms [64 rows x 128 bytes], BK*128 bytes apart; the columns
-                // are spline columns kt0.. (or, for a SiLU tile, inputs i0..).  kGroups
-                // groups of 128 threads take k-blocks in turn; a thread fills one
-                // atom row: (batch row rb, atom).
+                // A tile, MN-major: batch rows b0..b0+BK-1 (K) by 128 columns (M) in
+                // 128-byte atoms of EPB columns, BK*128 bytes apart (bf16: two atoms,
+                // 128-byte swizzle; fp32: four atoms, 32-byte-granule swizzle, hi and
+                // lo tiles).  The columns are spline columns kt0.. (or, for a SiLU
+                // tile, inputs i0..).  Groups of 128 threads take k-blocks in turn; a
+                // thread fills one atom row: (batch row rb, atom).
+                constexpr int NATOM = kBM / EPB;
                 const int grp = p >> 7;                    // warp-uniform
-                const int rb = p & (BK - 1);
-                const int atom = (p >> 6) & 1;             // warp-uniform
+                const int rb = p % BK;
+                const int atom = (p / BK) % NATOM;         // warp-uniform
                 const int mt = blockIdx.y;
                 const bool silu_tile = mt >= a.n_kt_tiles;
-                const int c_lo = (silu_tile ? (mt - a.n_kt_tiles) * kBM : mt * kBM) + atom * 64;
-                const int c_end = silu_tile ? min(c_lo + 64, (int)a.in) : min(c_lo + 64, a.Kt);
+                const int c_lo = (silu_tile ? (mt - a.n_kt_tiles) * kBM : mt * kBM) + atom * EPB;
+                const int c_end = silu_tile ? min(c_lo + EPB, (int)a.in) : min(c_lo + EPB, a.Kt);
                 const int i_first = (int)__umulhi((uint32_t)c_lo, a.nb_magic);
                 const int n_inp = (!silu_tile && c_lo < c_end)
                                       ? (int)__umulhi((uint32_t)(c_end - 1), a.nb_magic) - i_first + 1 : 0;
@@ -575,6 +580,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         if (k >= n_inp) break;
                         xv[k] = to_f(xr[k]);
                     }
+                };
+                // byte offset of column c (0..EPB-1) inside this thread's atom row
+                auto col_off = [&](int c) -> uint32_t {
+                    if constexpr (F32) return sw128b32_byte((uint32_t)rb, (uint32_t)c * 4u) - (uint32_t)rb * 128u;
+                    else return sw128_byte((uint32_t)rb, (uint32_t)c * 2u) - (uint32_t)rb * 128u;
                 };
                 float nxt[MAXI];
                 const int NG = min(Warps<MODE>::kGroups, stages);   // see the forward producer
@@ -591,8 +601,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     if (!mbar_wait(zeroed(s), ph, a.status)) break;
                     const int64_t b = (int64_t)kb * BK + rb;
                     const bool row_ok = b < a.batch;
-                    const uint32_t rbase = A_hi(s) + (uint32_t)atom * BK * 128u + (uint32_t)rb * 128u;
-                    const uint32_t rx = (uint32_t)rb & 7u;
+                    const uint32_t roff = (uint32_t)atom * BK * 128u + (uint32_t)rb * 128u;
+                    const uint32_t rb_hi = A_hi(s) + roff, rb_lo = A_lo(s) + roff;
                     if (!silu_tile) {
                         if (row_ok) {
                             const int cbase = i_first * a.nb - c_lo;
@@ -606,28 +616,61 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                 floor_split(u, sidx, f);
                                 float w[4];
                                 weights_fma(u - f, w);
-                                scatter4<KAN_BF16>(rbase, rbase, rx, cbase + k * a.nb + sidx, sidx, a.nb, 64, w);
+                                const int col0 = cbase + k * a.nb + sidx;
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    if ((unsigned)(sidx + q) < (unsigned)a.nb && (unsigned)(col0 + q) < (unsigned)EPB) {
+                                        const uint32_t off = col_off(col0 + q);
+                                        if constexpr (F32) {
+                                            const float hi = tf32_hi(w[q]);
+                                            st_shared_f32(rb_hi + off, hi);
+                                            st_shared_f32(rb_lo + off, w[q] - hi);
+                                        } else {
+                                            st_shared_u16(rb_hi + off, __bfloat16_as_ushort(__float2bfloat16_rn(w[q])));
+                                        }
+                                    }
+                                }
                             }
                         }
                     } else {
-                        // SiLU columns: inputs c_lo..c_lo+63 of batch row b (in % 8 == 0 with the base branch)
+                        // SiLU columns: inputs c_lo..c_lo+EPB-1 of batch row b, dense
+                        // (in * esize % 16 == 0 with the base branch)
                         const T* xr = X + (row_ok ? b : 0) * a.in;
+                        constexpr int EPC = 16 / C::ESZ;
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
-                            float v[8];
-                            const int ic = c_lo + c * 8;
-                            if (row_ok && ic + 8 <= a.in) {
+                            float v[EPC];
+                            const int ic = c_lo + c * EPC;
+                            if (row_ok && ic + EPC <= a.in) {
                                 const uint4 q4 = *reinterpret_cast<const uint4*>(xr + ic);
                                 const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-                                for (int e = 0; e < 8; ++e)
-                                    v[e] = silu_f(__uint_as_float((e & 1) ? (wd[e / 2] & 0xFFFF0000u) : (wd[e / 2] << 16)));
+                                for (int e = 0; e < EPC; ++e) {
+                                    float xv;
+                                    if constexpr (F32) xv = __uint_as_float(wd[e]);
+                                    else xv = __uint_as_float((e & 1) ? (wd[e / 2] & 0xFFFF0000u) : (wd[e / 2] << 16));
+                                    v[e] = silu_f(xv);
+                                }
                             } else {
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+                                for (int e = 0; e < EPC; ++e) v[e] = 0.0f;
                             }
-                            st_shared_v4(rbase + ((c ^ rx) << 4), pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                                         pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+                            const uint32_t off = col_off(c * EPC);   // a 16-byte chunk never straddles a granule
+                            if constexpr (F32) {
+                                float h[4], l[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    h[e] = tf32_hi(v[e]);
+                                    l[e] = v[e] - h[e];
+                                }
+                                st_shared_v4(rb_hi + off, __float_as_uint(h[0]), __float_as_uint(h[1]),
+                                             __float_as_uint(h[2]), __float_as_uint(h[3]));
+                                st_shared_v4(rb_lo + off, __float_as_uint(l[0]), __float_as_uint(l[1]),
+                                             __float_as_uint(l[2]), __float_as_uint(l[3]));
+                            } else {
+                                st_shared_v4(rb_hi + off, pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                             pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+                            }
                         }
                     }
                     fence_async_smem();
@@ -1162,10 +1205,9 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         gc[k] = ga[k];
                     }
                     if (ic + XC < i1) xfetch(ic + XC);
-#pragma unroll
-                    for (int k = 0; k < XC; ++k) {
+                    const int nkc = min(XC, i1 - ic);     // inputs in this chunk
+                    auto dx_of = [&](int k) -> float {
                         const int i = ic + k;
-                        if (i >= i1) break;
                         const float xv = __uint_as_float(xc[k]);
                         const Span sp = span_of(xv, a.lo, a.inv_h, a.G);
                         float acc = 0.0f;
@@ -1180,7 +1222,31 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                             }
                         }
                         if (a.gb) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
-                        dxr[i] = from_f<T>(acc);
+                        return acc;
+                    };
+                    if (nkc == XC && (((uintptr_t)(dxr + ic)) & 15u) == 0) {
+                        // a whole, aligned chunk: 16-byte stores
+                        float res[XC];
+#pragma unroll
+                        for (int k = 0; k < XC; ++k) res[k] = dx_of(k);
+                        constexpr int VE = 16 / (int)sizeof(T);
+#pragma unroll
+                        for (int v0 = 0; v0 < XC; v0 += VE) {
+                            if constexpr (F32) {
+                                *reinterpret_cast<float4*>(dxr + ic + v0) =
+                                    make_float4(res[v0], res[v0 + 1], res[v0 + 2], res[v0 + 3]);
+                            } else {
+                                *reinterpret_cast<uint4*>(dxr + ic + v0) =
+                                    make_uint4(pack_bf16(res[v0], res[v0 + 1]), pack_bf16(res[v0 + 2], res[v0 + 3]),
+                                               pack_bf16(res[v0 + 4], res[v0 + 5]), pack_bf16(res[v0 + 6], res[v0 + 7]));
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < XC; ++k) {
+                            if (k >= nkc) break;
+                            dxr[ic + k] = from_f<T>(dx_of(k));
+                        }
                     }
                 }
             }
@@ -1304,13 +1370,16 @@ bool make_map_2d(CUtensorMap* m, const void* base, bool f32, int64_t rows, int64
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// Split count minimising ceil(tiles*s / sms) / s (waves per unit of work), s <= cap.
+// Split-K count: only when the tiles do not fill one wave.  Then the split
+// that minimises ceil(tiles*s / sms) / s (waves per unit of work), with a small
+// price per extra split for the fp32 partial sums it writes and reduces.
 int pick_splits(int64_t tiles, int sms, int cap)
 {
+    if (tiles >= sms) return 1;
     int best = 1;
     double best_cost = 1e30;
     for (int s = 1; s <= std::max(1, cap); ++s) {
-        const double cost = (double)cdiv(tiles * s, sms) / s + 0.02 * (s - 1);  // small price per extra split
+        const double cost = (double)cdiv(tiles * s, sms) / s + 0.02 * (s - 1);
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
             best = s;
@@ -1518,14 +1587,7 @@ template <int MODE>
 cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
                       cudaStream_t st)
 {
-    if constexpr (MODE == DCA) {
-        if (f32) return cudaErrorInvalidConfiguration;
-        const int need = fwd_maxi_needed(args.nb, false);
-        if (need <= 4) return launch<MODE, KAN_BF16, 4>(grid, BN, stages, maps, args, st);
-        if (need <= 9) return launch<MODE, KAN_BF16, 9>(grid, BN, stages, maps, args, st);
-        if (need <= 17) return launch<MODE, KAN_BF16, 17>(grid, BN, stages, maps, args, st);
-        return cudaErrorInvalidConfiguration;
-    } else if constexpr (MODE == FWD) {
+    if constexpr (MODE == FWD || MODE == DCA) {
         const int need = fwd_maxi_needed(args.nb, f32);
         if (need <= 4)
             return f32 ? launch<MODE, KAN_F32, 4>(grid, BN, stages, maps, args, st)
@@ -1764,8 +1826,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         a.out = a.partial ? (void*)partbuf : (void*)dcoef;   // a skipped output is simply not stored
         a.out2 = dw_base;
         const dim3 grid(P.d_n, P.d_m, P.d_splits);
-        e = f32 ? launch_dt<DCOEF>(true, grid, P.d_BN, P.d_stages, maps, a, st)
-                : launch_dt<DCA>(false, grid, P.d_BN, P.d_stages, maps, a, st);
+        e = launch_dt<DCA>(f32, grid, P.d_BN, P.d_stages, maps, a, st);
         if (e != cudaSuccess) return e;
         if (a.partial) {
             const int64_t n = p.out * P.d_ld;
