@@ -26,7 +26,7 @@
 // keep about 21 significant bits of each product.  The tensor core's fp32
 // accumulation truncates, so long accumulations drift; the kernel therefore
 // (a) accumulates the small hi*lo + lo*hi products in their own TMEM
-// accumulator, and (b) accumulates hi*hi in short segments of `seg_kb`
+// accumulator, and (b) accumulates hi*hi in short segments of kSegKb
 // k-blocks, alternating between two TMEM buffers, which the epilogue warps add
 // into a running fp32 total (round-to-nearest) while the next segment runs.
 // bf16 operands: one kind::f16 product, fp32 accumulation in TMEM.
@@ -57,6 +57,7 @@ template <int MODE> struct Warps {
     static constexpr int kEpi0 = 2 + kProd;                            // first epilogue warp
     static constexpr int kThreads = (kEpi0 + 4) * 32;
 };
+constexpr int kSegKb = 2;         // fp32: k-blocks per promoted accumulation segment
 constexpr int kEpi = 128;         // warps 10-13
 constexpr int kSmemBudget = 227 * 1024 - 2048;
 
@@ -92,7 +93,7 @@ struct TcArgs {
     int G, nb;
     float lo, inv_h;
     int Kt;                    // in * nb
-    int BN, stages, seg_kb;
+    int BN, stages;
     int nkb_main;              // FWD: spline k-blocks; others: k-blocks over K
     int nkb_total;             // FWD: + SiLU k-blocks; others: = nkb_main
     int kb_per_split;
@@ -276,16 +277,17 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     const uint32_t stage_bytes = (a_bytes + b_bytes) * C::SPLIT;
     const uint32_t sbase = smem_addr(smem);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
-    // barrier block: full_a[S] full_b[S] empty[S] zeroed[S] seg_full[2] seg_empty[2] accum
-    // (zeroed[s]: the zero fill of stage s's produced tile has landed)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * stages + 5);
-    auto full_a = [&](int s) { return smem_addr(&bars[s]); };
-    auto full_b = [&](int s) { return smem_addr(&bars[stages + s]); };
-    auto empty = [&](int s) { return smem_addr(&bars[2 * stages + s]); };
-    auto zeroed = [&](int s) { return smem_addr(&bars[3 * stages + s]); };
-    auto seg_full = [&](int g) { return smem_addr(&bars[4 * stages + g]); };
-    auto seg_empty = [&](int g) { return smem_addr(&bars[4 * stages + 2 + g]); };
-    const uint32_t accum_bar = smem_addr(&bars[4 * stages + 4]);
+    // barrier block: full[S] empty[S] zeroed[S] seg_full[2] seg_empty[2] accum
+    // (full[s]: stage s's TMA bytes have landed and every producer thread has
+    // written its part of a produced tile -- one barrier, so the MMA thread waits
+    // once per k-block; zeroed[s]: the zero fill of stage s's produced tile has landed)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * stages + 5);
+    auto full = [&](int s) { return smem_addr(&bars[s]); };
+    auto empty = [&](int s) { return smem_addr(&bars[stages + s]); };
+    auto zeroed = [&](int s) { return smem_addr(&bars[2 * stages + s]); };
+    auto seg_full = [&](int g) { return smem_addr(&bars[3 * stages + g]); };
+    auto seg_empty = [&](int g) { return smem_addr(&bars[3 * stages + 2 + g]); };
+    const uint32_t accum_bar = smem_addr(&bars[3 * stages + 4]);
     auto A_hi = [&](int s) { return sbase + s * stage_bytes; };
     auto A_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes; };
     auto B_hi = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT; };
@@ -295,15 +297,15 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     const int kb_begin = blockIdx.z * a.kb_per_split;
     const int kb_end = min(a.nkb_total, kb_begin + a.kb_per_split);
     const int nk = kb_end - kb_begin;
-    const int nseg = F32 ? (nk + a.seg_kb - 1) / a.seg_kb : 1;
+    const int nseg = F32 ? (nk + kSegKb - 1) / kSegKb : 1;
     // TMEM columns: bf16 [acc]; fp32 [main0 | main1 | corr | total]
     const uint32_t tmem_cols =
         F32 ? 512u : (BN <= 32 ? 32u : (BN <= 64 ? 64u : (BN <= 128 ? 128u : (BN <= 256 ? 256u : 512u))));
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
-            mbar_init(full_a(s), (MODE == FWD || MODE == DCA) ? 128 : kProducers);
-            mbar_init(full_b(s), 1);
+            // the TMA thread's expect-tx arrival, plus one per producer thread
+            mbar_init(full(s), 1 + ((MODE == FWD || MODE == DCA) ? 128 : (MODE == DCOEF ? kProducers : 0)));
             mbar_init(empty(s), 1);
             mbar_init(zeroed(s), 1);
         }
@@ -340,9 +342,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 dx_kt0 = B_MN ? (i0 * a.nb) / (16 / C::ESZ) * (16 / C::ESZ) : i0 * a.nb;
             }
             int issued = 0;
-            for (int it = 0; it < nk; ++it) {
-                const int s = it % stages;
-                const uint32_t ph = (it / stages) & 1;
+            int s = 0;
+            uint32_t ph = 0;
+            for (int it = 0; it < nk; ++it, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
                 const int kb = kb_begin + it;
                 if (PRODUCE) {
@@ -358,40 +360,40 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     }
                 }
                 const uint32_t bytes = (b_bytes + (A_BY_TMA ? a_bytes : 0u)) * C::SPLIT;
-                mbar_arrive_expect_tx(full_b(s), bytes);
+                mbar_arrive_expect_tx(full(s), bytes);
                 if (MODE == FWD) {
                     // boxes of at most 128 rows (a.fbox): a wide tile is several of them
                     const bool spline = kb < a.nkb_main;
                     const int kc = spline ? kb * BK : (kb - a.nkb_main) * BK;
                     for (int h = 0; h * a.fbox < BN; ++h) {
                         const uint32_t off = (uint32_t)(h * a.fbox) * 128u;
-                        tma_load_2d(B_hi(s) + off, spline ? (const void*)&tB_hi : (const void*)&tB2_hi, full_b(s), kc,
+                        tma_load_2d(B_hi(s) + off, spline ? (const void*)&tB_hi : (const void*)&tB2_hi, full(s), kc,
                                     n0 + h * a.fbox);
                         if (F32)
-                            tma_load_2d(B_lo(s) + off, spline ? (const void*)&tB_lo : (const void*)&tB2_lo, full_b(s),
+                            tma_load_2d(B_lo(s) + off, spline ? (const void*)&tB_lo : (const void*)&tB2_lo, full(s),
                                         kc, n0 + h * a.fbox);
                     }
                 } else {
                     if (A_BY_TMA) {
-                        tma_load_2d(A_hi(s), &tA_hi, full_b(s), kb * BK, (int)m0);
-                        if (F32) tma_load_2d(A_lo(s), &tA_lo, full_b(s), kb * BK, (int)m0);
+                        tma_load_2d(A_hi(s), &tA_hi, full(s), kb * BK, (int)m0);
+                        if (F32) tma_load_2d(A_lo(s), &tA_lo, full(s), kb * BK, (int)m0);
                     }
                     const int nbase = MODE == DX ? dx_kt0 : n0;
                     if (B_MN) {
                         for (int c = 0; c < BN / EPB; ++c) {
                             const uint32_t off = (uint32_t)c * BK * 128;
-                            tma_load_2d(B_hi(s) + off, &tB_hi, full_b(s), nbase + c * EPB, kb * BK);
+                            tma_load_2d(B_hi(s) + off, &tB_hi, full(s), nbase + c * EPB, kb * BK);
                         }
                     } else {
-                        tma_load_2d(B_hi(s), &tB_hi, full_b(s), kb * BK, nbase);
-                        if (F32) tma_load_2d(B_lo(s), &tB_lo, full_b(s), kb * BK, nbase);
+                        tma_load_2d(B_hi(s), &tB_hi, full(s), kb * BK, nbase);
+                        if (F32) tma_load_2d(B_lo(s), &tB_lo, full(s), kb * BK, nbase);
                     }
                 }
                 ++issued;
             }
             // every load issued lands before the CTA can exit
             for (int it = max(0, issued - stages); it < issued; ++it) {
-                mbar_wait(full_b(it % stages), (it / stages) & 1, a.status);
+                mbar_wait(full(it % stages), (it / stages) & 1, a.status);
                 if (PRODUCE) mbar_wait(zeroed(it % stages), (it / stages) & 1, a.status);
             }
         }
@@ -412,39 +414,48 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             const uint32_t a_sbo = A_SW32 ? 512u : 1024u;
             const uint32_t a_layout = A_SW32 ? 1u : 2u;
             bool ok = true;
-            for (int it = 0; it < nk && ok; ++it) {
-                const int s = it % stages;
-                const uint32_t ph = (it / stages) & 1;
-                if (PRODUCE && !mbar_wait(full_a(s), ph, a.status)) { ok = false; break; }
-                if (!mbar_wait(full_b(s), ph, a.status)) { ok = false; break; }
-                const int g = F32 ? it / a.seg_kb : 0;
-                const bool seg_start = F32 && (it % a.seg_kb == 0);
+            int s = 0;
+            uint32_t ph = 0;
+            for (int it = 0; it < nk; ++it) {
+                if (!mbar_wait(full(s), ph, a.status)) { ok = false; break; }
+                const int g = F32 ? it / kSegKb : 0;
+                const bool seg_start = F32 && (it % kSegKb == 0);
                 if (seg_start && g >= 2 && !mbar_wait(seg_empty(g & 1), ((g >> 1) - 1) & 1, a.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t t_main = (g & 1) ? t_main1 : t_main0;
+                // descriptors of the stage's tiles; the k-steps advance the start address
+                // field (addresses stay below 2^18, so the field never carries)
+                const uint64_t ad0 = smem_desc(A_hi(s), a_lbo, a_sbo, a_layout);
+                const uint64_t bd0 = smem_desc_sw128(B_hi(s), b_lbo, 1024);
+                const uint64_t adl0 = F32 ? smem_desc(A_lo(s), a_lbo, a_sbo, a_layout) : 0;
+                const uint64_t bdl0 = F32 ? smem_desc_sw128(B_lo(s), b_lbo, 1024) : 0;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ad = smem_desc(A_hi(s) + ks * a_step, a_lbo, a_sbo, a_layout);
-                    const uint64_t bd = smem_desc_sw128(B_hi(s) + ks * b_step, b_lbo, 1024);
+                    const uint64_t ad = ad0 + (uint64_t)((ks * a_step) >> 4);
+                    const uint64_t bd = bd0 + (uint64_t)((ks * b_step) >> 4);
                     if constexpr (!F32) {
                         mma_bf16_ss(t_main0, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                         if (BN > 256) {
-                            const uint64_t bd2 = smem_desc_sw128(B_hi(s) + b_half + ks * b_step, b_lbo, 1024);
+                            const uint64_t bd2 = bd0 + (uint64_t)((b_half + ks * b_step) >> 4);
                             mma_bf16_ss(t_main0 + 256u, ad, bd2, idesc2, (it > 0 || ks > 0) ? 1u : 0u);
                         }
                     } else {
-                        const uint64_t adl = smem_desc(A_lo(s) + ks * a_step, a_lbo, a_sbo, a_layout);
-                        const uint64_t bdl = smem_desc_sw128(B_lo(s) + ks * b_step, b_lbo, 1024);
+                        const uint64_t adl = adl0 + (uint64_t)((ks * a_step) >> 4);
+                        const uint64_t bdl = bdl0 + (uint64_t)((ks * b_step) >> 4);
                         mma_tf32_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                         mma_tf32_ss(t_corr, ad, bdl, idesc, 1u);
                         mma_tf32_ss(t_main, ad, bd, idesc, (!seg_start || ks > 0) ? 1u : 0u);
                     }
                 }
                 mma_commit(empty(s));
-                if (F32 && ((it + 1) % a.seg_kb == 0 || it + 1 == nk)) mma_commit(seg_full(g & 1));
+                if (F32 && ((it + 1) % kSegKb == 0 || it + 1 == nk)) mma_commit(seg_full(g & 1));
+                if (++s == stages) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
             if (ok) mma_commit(accum_bar);
         }
@@ -548,7 +559,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                     fence_async_smem();
-                    mbar_arrive(full_a(s));
+                    mbar_arrive(full(s));
                 }
                 (void)uses;
             } else if constexpr (MODE == DCA) {
@@ -674,7 +685,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                     fence_async_smem();
-                    mbar_arrive(full_a(s));
+                    mbar_arrive(full(s));
                 }
             } else {
                 // DCOEF: rows = spline columns kt0..kt0+127 (or inputs of a SiLU tile),
@@ -776,7 +787,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                     fence_async_smem();
-                    mbar_arrive(full_a(s));
+                    mbar_arrive(full(s));
                 }
             }
         }
@@ -1074,16 +1085,16 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         if (lane == 0 && my_tiles > 0) {
             prefetch_tmap(&tA_hi);
             prefetch_tmap(&tB_hi);
-            int g = 0;   // k-block counter over all tiles (stage ring position)
+            int g = 0;   // k-block counter over all tiles
+            int s = 0;   // its stage ring position and phase
+            uint32_t ph = 0;
             bool ok = true;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
                 int64_t m0;
                 int i0;
                 tile_coords(lt, m0, i0);
                 const int kt0 = kt_start(i0);
-                for (int kb = 0; kb < a.nkb; ++kb, ++g) {
-                    const int s = g % stages;
-                    const uint32_t ph = (g / stages) & 1;
+                for (int kb = 0; kb < a.nkb; ++kb, ++g, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
                     if (!mbar_wait(empty(s), ph ^ 1, a.status)) { ok = false; break; }
                     mbar_arrive_expect_tx(full(s), (a_bytes + b_bytes) * C::SPLIT);
                     tma_load_2d(A_hi(s), &tA_hi, full(s), kb * BK, (int)m0);
@@ -1104,28 +1115,32 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             const uint32_t idesc = instr_desc(C::FMT, 0, B_MN ? 1u : 0u, kBM, BN);
             const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
             const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
-            int g = 0;
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
                 const int buf = lt & 1;
                 if (lt >= 2 && !mbar_wait(acc_empty(buf), ((lt >> 1) - 1) & 1, a.status)) break;
                 tc_fence_after();
                 const uint32_t d_main = tmem + buf * acc_cols, d_corr = d_main + BN;
-                for (int kb = 0; kb < a.nkb; ++kb, ++g) {
-                    const int s = g % stages;
-                    const uint32_t ph = (g / stages) & 1;
+                for (int kb = 0; kb < a.nkb; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
                     if (!mbar_wait(full(s), ph, a.status)) { ok = false; break; }
                     tc_fence_after();
+                    // k-steps advance the descriptors' start address field (no carry below 2^18)
+                    const uint64_t ad0 = smem_desc_sw128(A_hi(s), 16, 1024);
+                    const uint64_t bd0 = smem_desc_sw128(B_hi(s), b_lbo, 1024);
+                    const uint64_t adl0 = F32 ? smem_desc_sw128(A_lo(s), 16, 1024) : 0;
+                    const uint64_t bdl0 = F32 ? smem_desc_sw128(B_lo(s), b_lbo, 1024) : 0;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = smem_desc_sw128(A_hi(s) + ks * 32, 16, 1024);
-                        const uint64_t bd = smem_desc_sw128(B_hi(s) + ks * b_step, b_lbo, 1024);
+                        const uint64_t ad = ad0 + (uint64_t)(ks * 2);
+                        const uint64_t bd = bd0 + (uint64_t)((ks * b_step) >> 4);
                         const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
                         if constexpr (!F32) {
                             mma_bf16_ss(d_main, ad, bd, idesc, acc);
                         } else {
-                            const uint64_t adl = smem_desc_sw128(A_lo(s) + ks * 32, 16, 1024);
-                            const uint64_t bdl = smem_desc_sw128(B_lo(s) + ks * b_step, b_lbo, 1024);
+                            const uint64_t adl = adl0 + (uint64_t)(ks * 2);
+                            const uint64_t bdl = bdl0 + (uint64_t)((ks * b_step) >> 4);
                             mma_tf32_ss(d_corr, adl, bd, idesc, acc);
                             mma_tf32_ss(d_corr, ad, bdl, idesc, 1u);
                             mma_tf32_ss(d_main, ad, bd, idesc, acc);
@@ -1423,10 +1438,9 @@ int stages_for(int BN, bool f32)
     return std::min(8, (kSmemBudget - 1024 - 512) / stage_bytes);
 }
 
-// pipeline stages + 1024 alignment slack + 512 for the barrier block (4*stages+5 mbarriers) and the TMEM slot
+// pipeline stages + 1024 alignment slack + 512 for the barrier block (3*stages+5 mbarriers) and the TMEM slot
 int smem_bytes(int BN, int stages, bool f32) { return stages * (kBM * 128 + BN * 128) * (f32 ? 2 : 1) + 1024 + 512; }
 
-constexpr int kSegKb = 2;   // fp32: k-blocks per promoted accumulation segment
 
 // Workspace layout, shared by the size query and the launches.
 struct Layout {
@@ -1651,7 +1665,6 @@ TcArgs base_args(const Problem& p)
     a.lo = p.lo;
     a.inv_h = p.inv_h;
     a.Kt = (int)p.Kt;
-    a.seg_kb = kSegKb;
     a.has_base = p.base;
     a.nb_magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)p.nb - 1) / (uint64_t)p.nb);
     a.zeros = zero_tile_ptr();
