@@ -16,11 +16,19 @@
 //
 // One kernel template serves the four GEMMs:
 //   FWD    A = basis rows (producers)  B = coef / w_base, K-major (TMA)
-//   DCOEF  A = basis^T (producers)     B = dY, MN-major (TMA)
+//   DCA    A = basis^T (producers)     B = dY (TMA)
 //   DX     A = dY, K-major (TMA)       B = coef, MN-major (TMA); B'-gather epilogue
 //   GEMM   A = dY, K-major (TMA)       B = w_base, MN-major (TMA); fp32 store
-// Warp roles (14 warps): 0 TMA, 1 MMA issue + TMEM allocation, 2-9 A
-// producers, 10-13 epilogue (and, for fp32, accumulator promotion).
+// Warp roles: 0 TMA, 1 MMA issue + TMEM allocation, then the A producers
+// (FWD, DCA: 16 warps in 4 groups; the TMA-fed modes: 8 idle warps), then 4
+// epilogue warps (which also promote the fp32 accumulators).
+//
+// fp32 with the SiLU branch: silu(x_i) is one more basis function of input i,
+// with coefficient w_base[j, i].  Its column sits right after input i's G+3
+// spline columns (column stride G+4) in the tf32 copies of the coefficients
+// that the fp32 path makes anyway, so the SiLU terms ride along in every GEMM:
+// the forward sums them, dcoef's epilogue writes dw_base, and the dx epilogue
+// finds dY.w_base in its own accumulator.
 //
 // fp32 operands: three tf32 products per term, hi*hi + hi*lo + lo*hi, which
 // keep about 21 significant bits of each product.  The tensor core's fp32
@@ -47,10 +55,9 @@ namespace kan {
 namespace {
 
 constexpr int kBM = 128;          // MMA M: rows of A, TMEM lanes
-constexpr int kProducers = 256;   // producer threads of the DCOEF (fp32) mode
 
 // Producer warps per mode: the row producers (FWD, DCA) run 4 groups of 4
-// warps that take every 4th k-block; DCOEF uses 8 warps on each k-block.
+// warps that take every 4th k-block; the TMA-fed modes keep 8 idle warps.
 template <int MODE> struct Warps {
     static constexpr int kProd = (MODE == 0 || MODE == 4) ? 16 : 8;   // FWD, DCA : others
     static constexpr int kGroups = kProd / 4;
@@ -58,13 +65,13 @@ template <int MODE> struct Warps {
     static constexpr int kThreads = (kEpi0 + 4) * 32;
 };
 constexpr int kSegKb = 2;         // fp32: k-blocks per promoted accumulation segment
-constexpr int kEpi = 128;         // warps 10-13
+constexpr int kEpi = 128;         // epilogue threads (the last 4 warps)
 constexpr int kSmemBudget = 227 * 1024 - 2048;
 
 // DCA (bf16): dcoef = A^T . dY with M = spline columns (then SiLU rows), N =
 // outputs, K = batch; the basis operand is written MN-major by the producers
 // (rows = batch, 64-column atoms of spline columns), dY is read MN-major.
-enum Mode { FWD = 0, DCOEF = 1, DX = 2, GEMM = 3, DCA = 4 };
+enum Mode { FWD = 0, DX = 2, GEMM = 3, DCA = 4 };
 
 template <int DT> struct Cfg;
 template <> struct Cfg<KAN_BF16> {
@@ -85,12 +92,14 @@ template <> struct Cfg<KAN_F32> {
 };
 
 struct TcArgs {
-    const void* x;             // [batch, in] operand dtype (FWD, DCOEF, DX epilogue)
-    void* out;                 // FWD: y or partials; DCOEF: dcoef or partials; DX: dx; GEMM: fp32 [batch, in]
-    float* out2;               // DCOEF: dw_base (non-partial); DX: Gb = dY.w_base (fp32 [batch,in]) or null
+    const void* x;             // [batch, in] operand dtype (FWD, DCA, DX epilogue)
+    void* out;                 // FWD: y or partials; DCA: dcoef or partials; DX: dx; GEMM: fp32 [batch, in]
+    float* out2;               // DCA: dw_base (non-partial); DX: Gb = dY.w_base (fp32 [batch,in]) or null
     unsigned int* status;
     int64_t batch, in, out_f;
-    int G, nb;
+    int G, nb;                 // nb: columns per input (G+3, or G+4 with an interleaved SiLU column)
+    int nbs;                   // spline functions per input (G+3)
+    int ext;                   // 1: input i's SiLU column is column nbs of its group
     float lo, inv_h;
     int Kt;                    // in * nb
     int BN, stages;
@@ -98,8 +107,8 @@ struct TcArgs {
     int nkb_total;             // FWD: + SiLU k-blocks; others: = nkb_main
     int kb_per_split;
     int partial;
-    int n_kt_tiles;            // DCOEF: M tiles over spline rows (base tiles follow)
-    int64_t part_ld;           // DCOEF partial row length (Kt + in with base)
+    int n_kt_tiles;            // DCA: M tiles over spline rows (separate SiLU tiles follow)
+    int64_t part_ld;           // DCA partial row length
     int n_in_tile;             // DX: inputs per N tile
     int has_base;
     uint32_t nb_magic;         // ceil(2^32 / nb): c / nb == umulhi(c, nb_magic) for c < 2^32 / nb
@@ -234,6 +243,20 @@ __device__ __forceinline__ void scatter4(uint32_t rb_hi, uint32_t rb_lo, uint32_
     }
 }
 
+// One basis value at column `col` of a produced K-major row.
+template <int DT>
+__device__ __forceinline__ void put1(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx, int col, float v)
+{
+    constexpr int ESZ = DT == KAN_F32 ? 4 : 2;
+    if constexpr (DT == KAN_BF16) {
+        st_shared_u16(rb_hi + sw_col<ESZ>(col, rx), __bfloat16_as_ushort(__float2bfloat16_rn(v)));
+    } else {
+        const float hi = tf32_hi(v);
+        st_shared_f32(rb_hi + sw_col<ESZ>(col, rx), hi);
+        st_shared_f32(rb_lo + sw_col<ESZ>(col, rx), v - hi);
+    }
+}
+
 // The four local weights on the bounded coordinate t in [0,1) (see weights()).
 __device__ __forceinline__ void weights_fma(float t, float (&w)[4])
 {
@@ -260,7 +283,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     constexpr int BK = C::BK;
     constexpr int EPB = 128 / C::ESZ;               // elements per 128-byte row
     constexpr bool F32 = DT == KAN_F32;
-    constexpr bool PRODUCE = MODE == FWD || MODE == DCOEF || MODE == DCA;
+    constexpr bool PRODUCE = MODE == FWD || MODE == DCA;
     constexpr bool A_BY_TMA = MODE == DX || MODE == GEMM;
     constexpr bool A_MN = MODE == DCA;               // producer-written MN-major basis
     // an MN-major tf32 operand uses the 32-byte-atom 128-byte swizzle (layout 1)
@@ -305,7 +328,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             // the TMA thread's expect-tx arrival, plus one per producer thread
-            mbar_init(full(s), 1 + ((MODE == FWD || MODE == DCA) ? 128 : (MODE == DCOEF ? kProducers : 0)));
+            mbar_init(full(s), 1 + ((MODE == FWD || MODE == DCA) ? 128 : 0));
             mbar_init(empty(s), 1);
             mbar_init(zeroed(s), 1);
         }
@@ -324,11 +347,17 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_main0 = tmem, t_main1 = tmem + (uint32_t)BN, t_corr = tmem + 2u * BN, t_total = tmem + 3u * BN;
+    // fp32 with BN <= 64: B_hi and B_lo sit back to back in a stage, so one N = 2*BN
+    // product per k-step gives hi*hi and hi*lo together ([main | hi*lo] segment
+    // buffers, both promoted), and lo*hi is a second N = BN product into corr --
+    // two tensor-core instructions per k-step instead of three, and A_hi read once
+    const bool merged = F32 && BN <= 64;
+    const uint32_t wseg = merged ? 2u * BN : (uint32_t)BN;   // columns of one segment buffer
+    const uint32_t t_main0 = tmem, t_main1 = tmem + wseg, t_corr = tmem + 2u * wseg, t_total = t_corr + BN;
 
     // tile coordinates
-    const int64_t m0 = (int64_t)blockIdx.y * kBM;     // FWD/DX/GEMM: batch rows; DCOEF: see below
-    const int n0 = blockIdx.x * BN;                   // FWD/DCOEF/GEMM: output columns
+    const int64_t m0 = (int64_t)blockIdx.y * kBM;     // FWD/DX/GEMM: batch rows; DCA: see below
+    const int n0 = blockIdx.x * BN;                   // FWD/DCA/GEMM: output columns
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -405,6 +434,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             const int mma_n = BN > 256 ? 256 : BN;
             const uint32_t idesc = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, mma_n);
             const uint32_t idesc2 = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, BN > 256 ? BN - 256 : 16);
+            const uint32_t idesc_w = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, merged ? 2 * BN : 16);
             // offset of B's columns 256..: 256 rows (K-major) or four 64-column atoms (MN-major)
             const uint32_t b_half = B_MN ? 4u * BK * 128u : 256u * 128u;
             const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
@@ -442,6 +472,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                             const uint64_t bd2 = bd0 + (uint64_t)((b_half + ks * b_step) >> 4);
                             mma_bf16_ss(t_main0 + 256u, ad, bd2, idesc2, (it > 0 || ks > 0) ? 1u : 0u);
                         }
+                    } else if (merged) {
+                        const uint64_t adl = adl0 + (uint64_t)((ks * a_step) >> 4);
+                        mma_tf32_ss(t_main, ad, bd, idesc_w, (!seg_start || ks > 0) ? 1u : 0u);
+                        mma_tf32_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                     } else {
                         const uint64_t adl = adl0 + (uint64_t)((ks * a_step) >> 4);
                         const uint64_t bdl = bdl0 + (uint64_t)((ks * b_step) >> 4);
@@ -521,6 +555,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
 #pragma unroll
                             for (int k = 0; k < MAXI; ++k) {
                                 if (k >= n) break;
+                                if (F32 && a.ext) {   // input i0+k's SiLU column, when it falls in this block
+                                    const int cs = cbase + k * a.nb + a.nbs;
+                                    if ((unsigned)cs < (unsigned)BK) put1<DT>(ahi + rbase, alo + rbase, rx, cs, silu_f(cur[k]));
+                                }
                                 const float u = fmaf(cur[k], a.inv_h, u0);
                                 if (!(u >= -3.0f && u < u_hi)) continue;   // outside the extended knots, NaN, inf
                                 int sidx;
@@ -528,7 +566,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                 floor_split(u, sidx, f);
                                 float w[4];
                                 weights_fma(u - f, w);
-                                scatter4<DT>(ahi + rbase, alo + rbase, rx, cbase + k * a.nb + sidx, sidx, a.nb, BK, w);
+                                scatter4<DT>(ahi + rbase, alo + rbase, rx, cbase + k * a.nb + sidx, sidx, a.nbs, BK, w);
                             }
                         }
                     } else {
@@ -620,6 +658,20 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
 #pragma unroll
                             for (int k = 0; k < MAXI; ++k) {
                                 if (k >= n_inp) break;
+                                if (F32 && a.ext) {   // input i_first+k's SiLU column, when it falls in this atom
+                                    const int cs = cbase + k * a.nb + a.nbs;
+                                    if ((unsigned)cs < (unsigned)EPB) {
+                                        const float v = silu_f(cur[k]);
+                                        const uint32_t off = col_off(cs);
+                                        if constexpr (F32) {
+                                            const float hi = tf32_hi(v);
+                                            st_shared_f32(rb_hi + off, hi);
+                                            st_shared_f32(rb_lo + off, v - hi);
+                                        } else {
+                                            st_shared_u16(rb_hi + off, __bfloat16_as_ushort(__float2bfloat16_rn(v)));
+                                        }
+                                    }
+                                }
                                 const float u = fmaf(cur[k], a.inv_h, u0);
                                 if (!(u >= -3.0f && u < u_hi)) continue;
                                 int sidx;
@@ -630,7 +682,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                 const int col0 = cbase + k * a.nb + sidx;
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) {
-                                    if ((unsigned)(sidx + q) < (unsigned)a.nb && (unsigned)(col0 + q) < (unsigned)EPB) {
+                                    if ((unsigned)(sidx + q) < (unsigned)a.nbs && (unsigned)(col0 + q) < (unsigned)EPB) {
                                         const uint32_t off = col_off(col0 + q);
                                         if constexpr (F32) {
                                             const float hi = tf32_hi(w[q]);
@@ -687,108 +739,6 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     fence_async_smem();
                     mbar_arrive(full(s));
                 }
-            } else {
-                // DCOEF: rows = spline columns kt0..kt0+127 (or inputs of a SiLU tile),
-                // columns = batch rows b0..b0+BK-1
-                const int mt = blockIdx.y;
-                const bool silu_tile = mt >= a.n_kt_tiles;
-                constexpr int EPC = 16 / C::ESZ;
-                // spline tiles: (batch column c, input i) pairs, inputs fastest so that a
-                // warp reads consecutive x elements; the mapping is the same every k-block
-                constexpr int MAXP = (BK * (kBM / 4 + 2) + kProducers - 1) / kProducers;
-                const int kt0 = mt * kBM;
-                const int i_first = kt0 / a.nb;
-                const int i_last = min((int)a.in - 1, (kt0 + kBM - 1) / a.nb);
-                const int n_i = i_last - i_first + 1;
-                int pc[MAXP], pi[MAXP];
-#pragma unroll
-                for (int k = 0; k < MAXP; ++k) {
-                    const int e = p + k * kProducers;
-                    pc[k] = (!silu_tile && n_i > 0 && e < BK * n_i) ? e / n_i : -1;
-                    pi[k] = pc[k] >= 0 ? i_first + e % n_i : 0;
-                }
-                // SiLU tiles: input row r = p % 128 (consecutive across a warp), chunks
-                // (p / 128) * 4 .. + 3, EPC batch rows each
-                const int sr = p & (kBM - 1);
-                const int64_t si = (int64_t)(mt - a.n_kt_tiles) * kBM + sr;
-                const int sch0 = (p >> 7) * 4;
-                constexpr int NR = MAXP > 16 ? MAXP : 16;   // registers per fetch (bf16 SiLU values packed in pairs)
-                auto fetch = [&](int kb, uint32_t (&xr)[NR]) {
-                    const int64_t b0 = (int64_t)kb * BK;
-                    if (!silu_tile) {
-#pragma unroll
-                        for (int k = 0; k < MAXP; ++k) {
-                            const int64_t b = b0 + pc[k];
-                            xr[k] = (pc[k] >= 0 && b < a.batch) ? __float_as_uint(to_f(X[b * a.in + pi[k]])) : 0x7FC00000u;
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-#pragma unroll
-                            for (int e = 0; e < EPC; ++e) {
-                                const int64_t b = b0 + (sch0 + q) * EPC + e;
-                                const bool ok = si < a.in && b < a.batch;
-                                if constexpr (F32) {
-                                    xr[q * EPC + e] = ok ? __float_as_uint(X[b * a.in + si]) : 0u;
-                                } else {
-                                    const uint32_t h = ok ? (uint32_t)__bfloat16_as_ushort(X[b * a.in + si]) : 0u;
-                                    if (e & 1) xr[q * 4 + e / 2] |= h << 16;
-                                    else xr[q * 4 + e / 2] = h;
-                                }
-                            }
-                    }
-                };
-                uint32_t nxt[NR];
-                if (nk > 0) fetch(kb_begin, nxt);
-                for (int it = 0; it < nk; ++it) {
-                    uint32_t cur[NR];
-#pragma unroll
-                    for (int e = 0; e < NR; ++e) cur[e] = nxt[e];
-                    const int kb = kb_begin + it;
-                    if (it + 1 < nk) fetch(kb + 1, nxt);
-                    const int s = it % stages;
-                    const uint32_t ph = (it / stages) & 1;
-                    if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
-                    if (!mbar_wait(zeroed(s), ph, a.status)) break;
-                    const uint32_t ahi = A_hi(s), alo = A_lo(s);
-                    if (!silu_tile) {
-#pragma unroll
-                        for (int k = 0; k < MAXP; ++k) {
-                            if (pc[k] < 0) continue;
-                            // x beyond the batch was fetched as NaN: no basis, nothing stored
-                            const Span sp = span_of(__uint_as_float(cur[k]), a.lo, a.inv_h, a.G);
-                            if (!sp.valid) continue;
-                            float w[4];
-                            weights(sp.t, w);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const int m = sp.s + q;
-                                const int r = pi[k] * a.nb + m - kt0;
-                                if (m >= 0 && m < a.nb && r >= 0 && r < kBM)
-                                    put_a<DT>(ahi, alo, (uint32_t)r, pc[k], w[q]);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float v[EPC];
-#pragma unroll
-                            for (int e = 0; e < EPC; ++e) {
-                                float xv;
-                                if constexpr (F32) {
-                                    xv = __uint_as_float(cur[q * EPC + e]);
-                                } else {
-                                    const uint32_t wd = cur[q * 4 + e / 2];
-                                    xv = __uint_as_float((e & 1) ? (wd & 0xFFFF0000u) : (wd << 16));
-                                }
-                                v[e] = si < a.in ? silu_f(xv) : 0.0f;
-                            }
-                            put_a_chunk<DT>(ahi, alo, (uint32_t)sr, (uint32_t)(sch0 + q), v);
-                        }
-                    }
-                    fence_async_smem();
-                    mbar_arrive(full(s));
-                }
             }
         }
     } else {
@@ -809,7 +759,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const int i = i_start + k;
                 const bool ok = dx_b < a.batch && i < dx_i1;
                 xv[k] = ok ? __float_as_uint(to_f(reinterpret_cast<const T*>(a.x)[dx_b * a.in + i])) : 0u;
-                gv[k] = (ok && a.has_base) ? __float_as_uint(a.out2[dx_b * a.in + i]) : 0u;
+                gv[k] = (ok && a.has_base && !a.ext) ? __float_as_uint(a.out2[dx_b * a.in + i]) : 0u;
             }
         };
         if constexpr (MODE == DX) xfetch(dx_i0, xa, ga);
@@ -822,10 +772,15 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 tc_fence_after();
                 const uint32_t tm = ((g & 1) ? t_main1 : t_main0) + lane_off;
                 for (int c0 = 0; c0 < BN; c0 += 16) {
-                    uint32_t v[16], t[16];
+                    uint32_t v[16], w[16], t[16];
                     tmem_ld16(tm + c0, v);
+                    if (merged) tmem_ld16(tm + BN + c0, w);   // the segment's hi*lo half
                     if (g > 0) tmem_ld16(t_total + lane_off + c0, t);
                     tmem_ld_wait();
+                    if (merged) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(w[e]));
+                    }
                     if (g > 0) {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(t[e]));
@@ -906,7 +861,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                 }
-            } else if constexpr (MODE == DCOEF || MODE == DCA) {
+            } else if constexpr (MODE == DCA) {
                 // rows are spline columns kt (or inputs of a SiLU tile); columns are outputs j
                 const int mt = blockIdx.y;
                 const bool base_tile = mt >= a.n_kt_tiles;
@@ -918,6 +873,17 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     dst = reinterpret_cast<float*>(a.out) + (int64_t)blockIdx.z * a.out_f * a.part_ld +
                           (base_tile ? a.Kt + rowg : rowg);
                     ld = a.part_ld;
+                } else if (F32 && a.ext) {
+                    // interleaved layout: column rowg is function m of input ii
+                    const int ii = row_ok ? (int)__umulhi((uint32_t)rowg, a.nb_magic) : 0;
+                    const int m = (int)rowg - ii * a.nb;
+                    if (m < a.nbs) {
+                        dst = a.out ? reinterpret_cast<float*>(a.out) + (int64_t)ii * a.nbs + m : nullptr;
+                        ld = a.in * a.nbs;
+                    } else {
+                        dst = a.out2 ? a.out2 + ii : nullptr;
+                        ld = a.in;
+                    }
                 } else {
                     float* basep = base_tile ? a.out2 : reinterpret_cast<float*>(a.out);
                     dst = basep ? basep + rowg : nullptr;   // an output the caller skipped
@@ -970,10 +936,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
 #pragma unroll
                                 for (int qq = 0; qq < 4; ++qq) {
                                     const int m = sp.s + qq;
-                                    if (m >= 0 && m < a.nb) acc += stage[cb + m] * d[qq];
+                                    if (m >= 0 && m < a.nbs) acc += stage[cb + m] * d[qq];
                                 }
                             }
-                            if (a.has_base) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
+                            if (F32 && a.ext) acc += dsilu_f(xv) * stage[i * a.nb - kt_al + a.nbs];   // dY.w_base column
+                            else if (a.has_base) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
                             dxr[i] = from_f<T>(acc);
                         }
                     }
@@ -1004,10 +971,12 @@ constexpr int kDxThreads = 192;
 struct DxArgs {
     const void* x;
     void* dx;
-    const float* gb;          // dY . w_base (fp32 [batch, in]) or null
+    const float* gb;          // dY . w_base (fp32 [batch, in]) or null (none, or ext)
     unsigned int* status;
     int64_t batch, in, out;
-    int G, nb;
+    int G, nb;                // nb: columns per input of B (G+3, or G+4 with the SiLU column)
+    int nbs;                  // spline functions per input (G+3)
+    int ext;                  // 1: column nbs of each input group is its dY.w_base column
     float lo, inv_h;
     int BN, stages, nkb;      // nkb: k-blocks over out
     int n_in_tile, n_tiles_n, n_tiles;
@@ -1233,10 +1202,11 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 #pragma unroll
                             for (int qq = 0; qq < 4; ++qq) {
                                 const int m = sp.s + qq;
-                                if (m >= 0 && m < a.nb) acc += to_f(srow[cb + m]) * d[qq];
+                                if (m >= 0 && m < a.nbs) acc += to_f(srow[cb + m]) * d[qq];
                             }
                         }
-                        if (a.gb) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
+                        if (F32 && a.ext) acc += dsilu_f(xv) * to_f(srow[i * a.nb - kt_al + a.nbs]);   // dY.w_base, staged
+                        else if (a.gb) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
                         return acc;
                     };
                     if (nkc == XC && (((uintptr_t)(dxr + ic)) & 15u) == 0) {
@@ -1287,17 +1257,27 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, T* __restri
     }
 }
 
-// dcoef[j, kt] and dw_base[j, i] from partials [splits][out][Kt (+ in)], split order.
+// dcoef[j, kt] and dw_base[j, i] from partials [splits][out][ld], split order.
+// Columns: Kt spline columns then `in` SiLU columns, or (ext) input groups of
+// nbx columns, the last of which is the input's SiLU column.
 __global__ void reduce_dcoef_kernel(const float* __restrict__ part, float* __restrict__ dcoef,
                                     float* __restrict__ dw_base, int64_t out, int64_t Kt, int64_t in, int64_t ld,
-                                    int splits)
+                                    int splits, int nbs, int nbx, int ext)
 {
     const int64_t n = out * ld;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t j = e / ld, c = e % ld;
         float acc = 0.f;
         for (int z = 0; z < splits; ++z) acc += part[(int64_t)z * n + e];
-        if (c < Kt) {
+        if (ext) {
+            const int64_t i = c / nbx;
+            const int m = (int)(c - i * nbx);
+            if (m < nbs) {
+                if (dcoef) dcoef[j * Kt + i * nbs + m] = acc;
+            } else if (dw_base) {
+                dw_base[j * in + i] = acc;
+            }
+        } else if (c < Kt) {
             if (dcoef) dcoef[j * Kt + c] = acc;
         } else if (dw_base) {
             dw_base[j * in + (c - Kt)] = acc;
@@ -1332,6 +1312,55 @@ __global__ void split_tf32_t_kernel(const float* __restrict__ src, int64_t R, in
     for (int k = threadIdx.y; k < 32; k += blockDim.y) {
         const int64_t c = c0 + k, r = r0 + threadIdx.x;
         if (c < C && r < R) {
+            const float v = tile[threadIdx.x][k];
+            const float h = tf32_hi(v);
+            hi[c * ldo + r] = h;
+            lo[c * ldo + r] = v - h;
+        }
+    }
+}
+
+// Value of the fp32 coefficient matrix with each input's SiLU weight
+// interleaved: row j, column i*nbx + m is coef[j, i, m] for m < nbs and
+// w_base[j, i] for m == nbs.
+__device__ __forceinline__ float ext_coef(const float* __restrict__ coef, const float* __restrict__ w_base,
+                                          int64_t in, int nbs, int nbx, int64_t j, int64_t c)
+{
+    const int64_t i = c / nbx;
+    const int m = (int)(c - i * nbx);
+    return m < nbs ? coef[(j * in + i) * nbs + m] : w_base[j * in + i];
+}
+
+// tf32 hi/lo copies of the interleaved matrix, row-major [out][in*nbx].
+__global__ void split_ext_kernel(const float* __restrict__ coef, const float* __restrict__ w_base, int64_t out,
+                                 int64_t in, int nbs, int nbx, float* __restrict__ hi, float* __restrict__ lo)
+{
+    const int64_t Kx = in * nbx, n = out * Kx;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t j = e / Kx;
+        const float v = ext_coef(coef, w_base, in, nbs, nbx, j, e - j * Kx);
+        const float h = tf32_hi(v);
+        hi[e] = h;
+        lo[e] = v - h;
+    }
+}
+
+// The same, transposed: hi[c * ldo + j] (ldo >= out), through a 32x32 shared tile.
+__global__ void split_ext_t_kernel(const float* __restrict__ coef, const float* __restrict__ w_base, int64_t out,
+                                   int64_t in, int nbs, int nbx, float* __restrict__ hi, float* __restrict__ lo,
+                                   int64_t ldo)
+{
+    __shared__ float tile[32][33];
+    const int64_t Kx = in * nbx;
+    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+    for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+        const int64_t r = r0 + k, c = c0 + threadIdx.x;
+        tile[k][threadIdx.x] = (r < out && c < Kx) ? ext_coef(coef, w_base, in, nbs, nbx, r, c) : 0.0f;
+    }
+    __syncthreads();
+    for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+        const int64_t c = c0 + k, r = r0 + threadIdx.x;
+        if (c < Kx && r < out) {
             const float v = tile[threadIdx.x][k];
             const float h = tf32_hi(v);
             hi[c * ldo + r] = h;
@@ -1451,6 +1480,11 @@ struct Layout {
 };
 
 struct Plan {
+    // fp32 with the SiLU branch: interleaved coefficient copies (nbx = G+4
+    // columns per input, Kx = in * nbx); otherwise nbx = G+3 and Kx = Kt
+    bool ext;
+    int nbx;
+    int64_t Kx;
     // forward
     int f_BN, f_stages, f_n, f_m, f_splits, f_kps, f_nkb_main, f_nkb_total;
     // dcoef
@@ -1473,34 +1507,38 @@ Plan make_plan(const Problem& p, int sms)
     const bool f32 = p.dtype == KAN_F32;
     const int BK = f32 ? 32 : 64;
     const size_t esz = f32 ? 4 : 2;
+    P.ext = f32 && p.base;
+    P.nbx = p.nb + (P.ext ? 1 : 0);
+    P.Kx = p.in * P.nbx;
+    const bool sep_silu = p.base && !P.ext;   // separate SiLU k-blocks / tiles / GEMM
     // forward: M = batch, N = out, K = spline (+ SiLU) columns
     P.f_BN = f32 ? bn_for(p.out, true) : wide_bn(p.out);
     P.f_stages = stages_for(P.f_BN, f32);
     P.f_n = (int)cdiv(p.out, P.f_BN);
     P.f_m = (int)cdiv(p.batch, kBM);
-    P.f_nkb_main = (int)cdiv(p.Kt, BK);
-    P.f_nkb_total = P.f_nkb_main + (p.base ? (int)cdiv(p.in, BK) : 0);
+    P.f_nkb_main = (int)cdiv(P.Kx, BK);
+    P.f_nkb_total = P.f_nkb_main + (sep_silu ? (int)cdiv(p.in, BK) : 0);
     P.f_splits = pick_splits((int64_t)P.f_n * P.f_m, sms, std::min(16, std::max(1, P.f_nkb_total / 8)));
     P.f_kps = (int)cdiv(P.f_nkb_total, P.f_splits);
     P.f_splits = (int)cdiv(P.f_nkb_total, P.f_kps);
     // dcoef: M = spline columns (+ SiLU rows), N = out, K = batch
     P.d_BN = f32 ? bn_for(p.out, true, true) : std::max(64, wide_bn(p.out));
     P.d_n = (int)cdiv(p.out, P.d_BN);
-    P.d_nkt = (int)cdiv(p.Kt, kBM);
-    P.d_m = P.d_nkt + (p.base ? (int)cdiv(p.in, kBM) : 0);
+    P.d_nkt = (int)cdiv(P.Kx, kBM);
+    P.d_m = P.d_nkt + (sep_silu ? (int)cdiv(p.in, kBM) : 0);
     P.d_stages = stages_for(P.d_BN, f32);
     P.d_nkb = (int)cdiv(p.batch, BK);
     P.d_splits = pick_splits((int64_t)P.d_n * P.d_m, sms, std::min(16, std::max(1, P.d_nkb / 8)));
     P.d_kps = (int)cdiv(std::max(1, P.d_nkb), P.d_splits);
     P.d_splits = (int)cdiv(std::max(1, P.d_nkb), P.d_kps);
-    P.d_ld = p.Kt + (p.base ? p.in : 0);
+    P.d_ld = P.ext ? P.Kx : p.Kt + (p.base ? p.in : 0);
     // dx: M = batch, N = whole inputs' spline columns, K = out
     P.x_BN = f32 ? 128 : 256;
     P.x_stages = stages_for(P.x_BN, f32);
     // bf16: coef is read MN-major and a tile's first column is rounded down to
     // 16 bytes; fp32: coef^T is read K-major, any first row works
     const int maxoff = f32 ? 0 : ((p.nb % 8 == 0) ? 0 : 7);
-    P.x_nin = std::max(1, (P.x_BN - maxoff) / p.nb);
+    P.x_nin = std::max(1, (P.x_BN - maxoff) / P.nbx);
     P.x_n = (int)cdiv(p.in, P.x_nin);
     P.x_m = (int)cdiv(p.batch, kBM);
     P.x_nkb = (int)cdiv(p.out, BK);
@@ -1508,7 +1546,7 @@ Plan make_plan(const Problem& p, int sms)
     {
         P.p_BN = f32 ? 128 : 256;
         const int pmaxoff = f32 ? 0 : ((p.nb % 8 == 0) ? 0 : 7);
-        P.p_nin = (P.p_BN - pmaxoff) / p.nb;
+        P.p_nin = (P.p_BN - pmaxoff) / P.nbx;
         P.p_ld = f32 ? P.p_BN + 4 : P.p_BN + 8;          // row stride = 16 bytes mod 128
         const int staging = 4 * 32 * P.p_ld * (f32 ? 4 : 2);
         const int stage_bytes = (kBM * 128 + P.p_BN * 128) * (f32 ? 2 : 1);
@@ -1531,8 +1569,8 @@ Plan make_plan(const Problem& p, int sms)
     size_t o = 0;
     if (f32) {
         P.fwd.coef_hl = o;
-        o += 2 * al256((size_t)p.out * p.Kt * 4);
-        if (p.base) {
+        o += 2 * al256((size_t)p.out * P.Kx * 4);
+        if (sep_silu) {
             P.fwd.wb_hl = o;
             o += 2 * al256((size_t)p.out * p.in * 4);
         }
@@ -1547,8 +1585,8 @@ Plan make_plan(const Problem& p, int sms)
     P.ldb = (p.batch + 3) / 4 * 4;
     if (f32) {
         P.bwd.coef_hl = o;
-        o += 2 * al256((size_t)p.out * p.Kt * 4);
-        if (p.base) {
+        o += 2 * al256((size_t)p.out * P.Kx * 4);
+        if (sep_silu) {
             P.bwd.wb_hl = o;
             o += 2 * al256((size_t)p.out * p.in * 4);
         }
@@ -1561,7 +1599,7 @@ Plan make_plan(const Problem& p, int sms)
         P.bwd.dc_part = o;
         o += al256((size_t)P.d_splits * p.out * P.d_ld * 4);
     }
-    if (p.base) {
+    if (sep_silu) {
         P.bwd.gb = o;
         o += al256((size_t)p.batch * p.in * 4);
     }
@@ -1653,7 +1691,7 @@ const void* zero_tile_ptr()
     return ptrs[dev];
 }
 
-TcArgs base_args(const Problem& p)
+TcArgs base_args(const Problem& p, const Plan& P)
 {
     TcArgs a{};
     a.status = device_status_ptr();
@@ -1661,12 +1699,14 @@ TcArgs base_args(const Problem& p)
     a.in = p.in;
     a.out_f = p.out;
     a.G = p.G;
-    a.nb = p.nb;
+    a.nb = P.nbx;
+    a.nbs = p.nb;
+    a.ext = P.ext;
     a.lo = p.lo;
     a.inv_h = p.inv_h;
-    a.Kt = (int)p.Kt;
+    a.Kt = (int)P.Kx;
     a.has_base = p.base;
-    a.nb_magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)p.nb - 1) / (uint64_t)p.nb);
+    a.nb_magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)P.nbx - 1) / (uint64_t)P.nbx);
     a.zeros = zero_tile_ptr();
     return a;
 }
@@ -1697,6 +1737,27 @@ cudaError_t split_t_into(const void* src, int64_t R, int64_t C, int64_t ldo, uin
     return cudaGetLastError();
 }
 
+// tf32 hi/lo copies of coef with w_base interleaved, [out][Kx] (or transposed
+// to [Kx][ldo]); returns the (hi, lo) pointers.
+cudaError_t split_ext_into(const Problem& p, const Plan& P, const void* coef, const void* w_base, bool transposed,
+                           int64_t ldo, uint8_t* dst, const void** hi, const void** lo, cudaStream_t st)
+{
+    float* h = reinterpret_cast<float*>(dst);
+    float* l = reinterpret_cast<float*>(dst + al256((size_t)p.out * P.Kx * 4));
+    if (transposed) {
+        dim3 grid((unsigned)cdiv(P.Kx, 32), (unsigned)cdiv(p.out, 32));
+        split_ext_t_kernel<<<grid, dim3(32, 8), 0, st>>>((const float*)coef, (const float*)w_base, p.out, p.in, p.nb,
+                                                          P.nbx, h, l, ldo);
+    } else {
+        split_ext_kernel<<<grid_for(p.out * P.Kx), 256, 0, st>>>((const float*)coef, (const float*)w_base, p.out, p.in,
+                                                                 p.nb, P.nbx, h, l);
+    }
+    count_launch();
+    *hi = h;
+    *lo = l;
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool tc_supported(const Problem& p, bool backward, const char** why)
@@ -1718,7 +1779,10 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
         *why = "G too large for one dx tile (G+3 must fit the tile with its alignment offset)";
         return false;
     }
-    if (p.Kt + p.in > ((int64_t)1 << 30) || p.Kt >= (((int64_t)1 << 32) / p.nb) || p.batch > ((int64_t)1 << 31) - 256 ||
+    // (with the SiLU branch the fp32 copies have G+4 columns per input)
+    const int64_t nbx = p.nb + ((p.dtype == KAN_F32 && p.base) ? 1 : 0);
+    if (p.Kt + p.in > ((int64_t)1 << 30) || p.in * nbx >= (((int64_t)1 << 32) / nbx) ||
+        p.batch > ((int64_t)1 << 31) - 256 ||
         p.out > ((int64_t)1 << 30)) {
         *why = "problem too large for 32-bit tile coordinates";
         return false;
@@ -1744,17 +1808,20 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
     uint8_t* w = reinterpret_cast<uint8_t*>(ws);
     const void *c_hi = coef, *c_lo = coef, *wb_hi = w_base, *wb_lo = w_base;
     cudaError_t e;
-    if (f32) {
+    if (P.ext) {
+        if ((e = split_ext_into(p, P, coef, w_base, false, 0, w + P.fwd.coef_hl, &c_hi, &c_lo, st)) != cudaSuccess)
+            return e;
+    } else if (f32) {
         if ((e = split_into(coef, p.out * p.Kt, w + P.fwd.coef_hl, &c_hi, &c_lo, st)) != cudaSuccess) return e;
         if (p.base && (e = split_into(w_base, p.out * p.in, w + P.fwd.wb_hl, &wb_hi, &wb_lo, st)) != cudaSuccess)
             return e;
     }
     CUtensorMap maps[6];
     const int fbox = std::min(P.f_BN, 128);
-    if (!make_map_2d(&maps[2], c_hi, f32, p.out, p.Kt, fbox, BK, detail) ||
-        !make_map_2d(&maps[3], c_lo, f32, p.out, p.Kt, fbox, BK, detail))
+    if (!make_map_2d(&maps[2], c_hi, f32, p.out, P.Kx, fbox, BK, detail) ||
+        !make_map_2d(&maps[3], c_lo, f32, p.out, P.Kx, fbox, BK, detail))
         return cudaErrorInvalidValue;
-    if (p.base) {
+    if (p.base && !P.ext) {
         if (!make_map_2d(&maps[4], wb_hi, f32, p.out, p.in, fbox, BK, detail) ||
             !make_map_2d(&maps[5], wb_lo, f32, p.out, p.in, fbox, BK, detail))
             return cudaErrorInvalidValue;
@@ -1764,7 +1831,7 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
     }
     maps[0] = maps[2];
     maps[1] = maps[3];
-    TcArgs a = base_args(p);
+    TcArgs a = base_args(p, P);
     a.x = x;
     a.out = P.f_splits > 1 ? (void*)(w + P.fwd.fwd_part) : y;
     a.BN = P.f_BN;
@@ -1826,7 +1893,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             if (!make_map_2d(&maps[2], dY, false, p.batch, p.out, BK, EPB, detail)) return cudaErrorInvalidValue;
             maps[0] = maps[1] = maps[3] = maps[4] = maps[5] = maps[2];
         }
-        TcArgs a = base_args(p);
+        TcArgs a = base_args(p, P);
         a.x = x;
         float* partbuf = reinterpret_cast<float*>(w + P.bwd.dc_part);
         a.BN = P.d_BN;
@@ -1844,7 +1911,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         if (a.partial) {
             const int64_t n = p.out * P.d_ld;
             reduce_dcoef_kernel<<<grid_for(n), 256, 0, st>>>(partbuf, dcoef, dw_base, p.out, p.Kt, p.in, P.d_ld,
-                                                              P.d_splits);
+                                                              P.d_splits, p.nb, P.nbx, P.ext ? 1 : 0);
             count_launch();
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
@@ -1855,7 +1922,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         if (f32 && (e = split_into(dY, p.batch * p.out, w + P.bwd.dy_hl, &dy_hi, &dy_lo, st)) != cudaSuccess)
             return e;
         float* gb = nullptr;
-        if (p.base) {
+        if (p.base && !P.ext) {
             // Gb = dY . w_base (fp32 [batch, in]) for the SiLU term of dx
             gb = reinterpret_cast<float*>(w + P.bwd.gb);
             CUtensorMap maps[6];
@@ -1875,7 +1942,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             }
             maps[4] = maps[2];
             maps[5] = maps[3];
-            TcArgs a = base_args(p);
+            TcArgs a = base_args(p, P);
             a.out = gb;
             a.BN = P.g_BN;
             a.stages = P.g_stages;
@@ -1891,10 +1958,11 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             return cudaErrorInvalidValue;
         if (f32) {
             const void *th, *tl;
-            if ((e = split_t_into(coef, p.out, p.Kt, p.out, w + P.bwd.coef_hl, &th, &tl, st)) != cudaSuccess)
-                return e;
-            if (!make_map_2d(&maps[2], th, true, p.Kt, p.out, xBN, BK, detail) ||
-                !make_map_2d(&maps[3], tl, true, p.Kt, p.out, xBN, BK, detail))
+            e = P.ext ? split_ext_into(p, P, coef, w_base, true, p.out, w + P.bwd.coef_hl, &th, &tl, st)
+                      : split_t_into(coef, p.out, p.Kt, p.out, w + P.bwd.coef_hl, &th, &tl, st);
+            if (e != cudaSuccess) return e;
+            if (!make_map_2d(&maps[2], th, true, P.Kx, p.out, xBN, BK, detail) ||
+                !make_map_2d(&maps[3], tl, true, P.Kx, p.out, xBN, BK, detail))
                 return cudaErrorInvalidValue;
         } else {
             if (!make_map_2d(&maps[2], coef, false, p.out, p.Kt, BK, EPB, detail)) return cudaErrorInvalidValue;
@@ -1912,7 +1980,9 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             d.in = p.in;
             d.out = p.out;
             d.G = p.G;
-            d.nb = p.nb;
+            d.nb = P.nbx;
+            d.nbs = p.nb;
+            d.ext = P.ext ? 1 : 0;
             d.lo = p.lo;
             d.inv_h = p.inv_h;
             d.BN = P.p_BN;
@@ -1925,7 +1995,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             e = f32 ? launch_dx_persistent<KAN_F32>(P, maps, d, st) : launch_dx_persistent<KAN_BF16>(P, maps, d, st);
             if (e != cudaSuccess) return e;
         } else {
-            TcArgs a = base_args(p);
+            TcArgs a = base_args(p, P);
             a.x = x;
             a.out = dx;
             a.out2 = gb;
