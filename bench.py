@@ -78,6 +78,33 @@ def aggregate_rate(units_per_rank_step: float, steps: int, world: int, t_max_ms:
     return world * units_per_rank_step * steps / (t_max_ms / 1000.0)
 
 
+def csrc_hash() -> str:
+    """Hash of the kernel sources (names and bytes), to match ncu figures to the kernels they were taken on."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "kolmogorov_arnold_network_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, call: str):
+    """DRAM bytes per launch of a call's main kernel from the committed ncu capture
+    (profiles/traffic.json), or None when there is none or the kernels changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("csrc_hash") != csrc_hash():
+        return None
+    e = d.get("workloads", {}).get(workload, {}).get(call)
+    return None if e is None else e.get("dram_bytes")
+
+
 # ---------------------------------------------------------------------------
 # FLOP / byte accounting (per call, algorithmic)
 def layer_dense_flops(batch, L):
@@ -147,6 +174,8 @@ class Runner:
                 N.kan_forward(l["s"], P(l["x"]), P(l["coef"]), P(l["wb"]), P(l["y"]), P(l["ws_f"]),
                               0 if l["ws_f"] is None else l["ws_f"].numel(), st)
             out.append((f"fwd{li}", fwd))
+        if self.w.mode == "fwd":
+            return out
         for li in reversed(range(len(self.layers))):
             l = self.layers[li]
             dy = self.dY if li == len(self.layers) - 1 else self.layers[li + 1]["dx"]
@@ -164,13 +193,17 @@ class Runner:
 
     def h2d(self):
         self.x.copy_(self.h_x, non_blocking=True)
-        self.dY.copy_(self.h_dY, non_blocking=True)
-        return self.h_x.numel() * self.h_x.element_size() + self.h_dY.numel() * self.h_dY.element_size()
+        n = self.h_x.numel() * self.h_x.element_size()
+        if self.w.mode != "fwd":
+            self.dY.copy_(self.h_dY, non_blocking=True)
+            n += self.h_dY.numel() * self.h_dY.element_size()
+        return n
 
     def d2h(self):
         n = 0
+        keys = ("y",) if self.w.mode == "fwd" else ("y", "dx", "dcoef", "dwb")
         for l, h in zip(self.layers, self.h_out):
-            for k in ("y", "dx", "dcoef", "dwb"):
+            for k in keys:
                 if h[k] is not None:
                     h[k].copy_(l[k], non_blocking=True)
                     n += h[k].numel() * h[k].element_size()
@@ -248,7 +281,7 @@ def cpu_baseline(w: W.Workload, target_s=12.0):
             acts.append(act)
             act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], nthreads=cores)
         g = dY
-        for li in reversed(range(len(w.layers))):
+        for li in (reversed(range(len(w.layers))) if w.mode != "fwd" else ()):
             L = w.layers[li]
             gx, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"],
                                   nthreads=cores)
@@ -270,7 +303,7 @@ def cpu_baseline(w: W.Workload, target_s=12.0):
     edges = passes * sum(rows * L.inp * L.out for L in w.layers)
     return {"value": edges / t, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{passes} pass(es) over {rows} of {w.batch} rows of {w.name}, fp64 Cox-de Boor "
-                      f"forward+backward, {t:.1f} s"}
+                      f"{'forward' if w.mode == 'fwd' else 'forward+backward'}, {t:.1f} s"}
 
 
 def run_reference(args, world, rank):
@@ -290,7 +323,7 @@ def run_reference(args, world, rank):
             acts.append(act)
             act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], nthreads=cores)
         g = d["dY"][:rows]
-        for li in reversed(range(len(w.layers))):
+        for li in (reversed(range(len(w.layers))) if w.mode != "fwd" else ()):
             L = w.layers[li]
             g, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"],
                                  nthreads=cores)
@@ -323,7 +356,7 @@ def run_reference(args, world, rank):
 def config_of(w: W.Workload):
     L0 = w.layers[0]
     c = {"workload": w.name, "batch": w.batch, "layers": [[L.inp, L.out] for L in w.layers], "G": L0.G,
-         "grid": [L0.lo, L0.hi], "silu_base": L0.base, "mode": "fwd+bwd", "l2": "256 MiB flush between steps",
+         "grid": [L0.lo, L0.hi], "silu_base": L0.base, "mode": w.mode, "l2": "256 MiB flush between steps",
          "note": w.note}
     if w.dtype == "f32":
         c["compute"] = "fp32 operands as 3 tf32 tensor-core products, fp32 accumulation"
@@ -403,7 +436,7 @@ def run_ours(args, world, rank, local):
         peak_note = f"tf32 dense = {pk['src']} bf16 burst x nominal tf32/bf16 ratio {TF32_PER_BF16:.3f}"
     achieved = flops / avg_s / 1e12
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": None, "kernel": f"{kind} call of layer {li}", "peak_note": peak_note,
+            "traffic": measured_traffic(w.name, kind), "kernel": f"{kind} call of layer {li}", "peak_note": peak_note,
             "algorithmic_flops_per_launch": flops,
             "algorithmic_bytes_per_launch": layer_bytes(w.batch, L, 4 if w.dtype == "f32" else 2, kind),
             "call_ms": {k: v / K for k, v in per_call.items()}}
