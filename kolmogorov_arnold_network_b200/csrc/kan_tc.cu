@@ -102,7 +102,8 @@ struct TcArgs {
     int ext;                   // 1: input i's SiLU column is column nbs of its group
     float lo, inv_h;
     int Kt;                    // in * nb
-    int BN, stages;
+    int BN, stages;            // stages: pipeline depth of B (and of A when A also arrives by TMA)
+    int stages_a;              // FWD, DCA: depth of the produced-A ring (its own barriers)
     int nkb_main;              // FWD: spline k-blocks; others: k-blocks over K
     int nkb_total;             // FWD: + SiLU k-blocks; others: = nkb_main
     int kb_per_split;
@@ -111,9 +112,9 @@ struct TcArgs {
     int64_t part_ld;           // DCA partial row length
     int n_in_tile;             // DX: inputs per N tile
     int has_base;
+    int x_vec;                 // 1: rows of x are 16-byte aligned (in * sizeof(T) % 16 == 0), vector loads allowed
     uint32_t nb_magic;         // ceil(2^32 / nb): c / nb == umulhi(c, nb_magic) for c < 2^32 / nb
     int fbox;                  // FWD: rows per B box
-    const void* zeros;         // >= 16 KiB of zeros in global memory (the A tiles' zero fill)
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
@@ -212,34 +213,104 @@ __device__ __forceinline__ uint32_t sw_col(int c, uint32_t rx)
     return ((((cb >> 4) ^ rx) & 7u) << 4) | (cb & 15u);
 }
 
-// The four weights of one input at columns col0..col0+3 of a 128-byte
-// swizzled row (basis indices sidx..sidx+3); entries whose basis index is
-// outside 0..nb-1 or whose column is outside 0..ncols-1 are skipped.  One
-// predicated store per entry keeps the warp convergent.
+// The four weights of one input whose B_0 sits at column `base` of a 128-byte
+// swizzled row: entry q (basis index s+q) goes to column base+s+q when
+// mlo <= s+q < mhi (the caller's range keeps the column inside the row and the
+// basis index inside 0..nb-1; an empty range stores nothing).  One predicated
+// store per entry keeps the warp convergent.
 template <int DT>
-__device__ __forceinline__ void scatter4(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx, int col0, int sidx, int nb,
-                                         int ncols, const float (&w)[4])
+__device__ __forceinline__ void scatter_win(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx, int base, int s, int mlo,
+                                            int mhi, const float (&w)[4])
 {
     constexpr int ESZ = DT == KAN_F32 ? 4 : 2;
+    const uint32_t width = (uint32_t)(mhi - mlo);
     if constexpr (DT == KAN_BF16) {
-        const __nv_bfloat162 a01 = __floats2bfloat162_rn(w[0], w[1]);
-        const __nv_bfloat162 a23 = __floats2bfloat162_rn(w[2], w[3]);
-        const uint32_t p01 = *reinterpret_cast<const uint32_t*>(&a01);
-        const uint32_t p23 = *reinterpret_cast<const uint32_t*>(&a23);
+        const uint32_t p01 = pack_bf16(w[0], w[1]), p23 = pack_bf16(w[2], w[3]);
         const uint16_t h[4] = {(uint16_t)(p01 & 0xFFFFu), (uint16_t)(p01 >> 16), (uint16_t)(p23 & 0xFFFFu),
                                (uint16_t)(p23 >> 16)};
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            if ((unsigned)(sidx + q) < (unsigned)nb && (unsigned)(col0 + q) < (unsigned)ncols)
-                st_shared_u16(rb_hi + sw_col<ESZ>(col0 + q, rx), h[q]);
+            if ((uint32_t)(s + q - mlo) < width) st_shared_u16(rb_hi + sw_col<ESZ>(base + s + q, rx), h[q]);
     } else {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            if ((unsigned)(sidx + q) < (unsigned)nb && (unsigned)(col0 + q) < (unsigned)ncols) {
+            if ((uint32_t)(s + q - mlo) < width) {
+                const uint32_t off = sw_col<ESZ>(base + s + q, rx);
                 const float hi = tf32_hi(w[q]);
-                st_shared_f32(rb_hi + sw_col<ESZ>(col0 + q, rx), hi);
-                st_shared_f32(rb_lo + sw_col<ESZ>(col0 + q, rx), w[q] - hi);
+                st_shared_f32(rb_hi + off, hi);
+                st_shared_f32(rb_lo + off, w[q] - hi);
             }
+    }
+}
+
+// Zero one 128-byte row of a produced tile (and of its lo copy for fp32).
+// Store c writes 16-byte chunk c ^ rx (rx = row & 7), so the 8 consecutive
+// rows of a quarter-warp hit 8 different chunks: no bank conflicts.
+template <int DT>
+__device__ __forceinline__ void zero_row(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx)
+{
+#pragma unroll
+    for (uint32_t c = 0; c < 8; ++c) {
+        st_shared_zero16(rb_hi + 16u * (c ^ rx));
+        if constexpr (DT == KAN_F32) st_shared_zero16(rb_lo + 16u * (c ^ rx));
+    }
+}
+
+// xv[k] = x[i0 + k] for k < MAXI from one row of x (values at or past `in`
+// read as 0; only the first n, n <= MAXI warp-uniform, are used by the caller).  With vec, the row is read as 16-byte vectors starting at the
+// aligned element below i0: a warp's lanes each read their own row, so every
+// load instruction costs one L1 sector lookup per lane, and one vector replaces
+// up to 8 (bf16) or 4 (fp32) scalar loads.  The window is then shifted into
+// place by the warp-uniform offset o = i0 mod (16 / sizeof(T)) through a small
+// select / funnel-shift network (no dynamically indexed registers).
+template <typename T, int MAXI>
+__device__ __forceinline__ void load_x_window(const T* __restrict__ row, int i0, int n, int in, bool vec,
+                                              float (&xv)[MAXI])
+{
+    constexpr int EPV = 16 / (int)sizeof(T);              // elements per 16-byte vector
+    constexpr int NV = (EPV - 1 + MAXI + EPV - 1) / EPV;  // vectors covering any window
+    if (!vec) {
+#pragma unroll
+        for (int k = 0; k < MAXI; ++k) xv[k] = (k < n && i0 + k < in) ? to_f(row[i0 + k]) : 0.0f;
+        return;
+    }
+    const int ia = i0 & ~(EPV - 1);
+    const int o = i0 - ia;                                  // 0 .. EPV-1, uniform across the warp
+    uint32_t raw[4 * NV + 4];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        // (a vector holding none of the n values is skipped; in % EPV == 0)
+        if (v * EPV < o + n && ia + v * EPV < in) q = *reinterpret_cast<const uint4*>(row + ia + v * EPV);
+        raw[4 * v] = q.x;
+        raw[4 * v + 1] = q.y;
+        raw[4 * v + 2] = q.z;
+        raw[4 * v + 3] = q.w;
+    }
+#pragma unroll
+    for (int j = 4 * NV; j < 4 * NV + 4; ++j) raw[j] = 0u;
+    if constexpr (sizeof(T) == 4) {
+        // shift by o words: two select levels
+        uint32_t t[4 * NV + 2];
+#pragma unroll
+        for (int j = 0; j < 4 * NV + 2; ++j) t[j] = (o & 1) ? raw[j + 1] : raw[j];
+#pragma unroll
+        for (int k = 0; k < MAXI; ++k) xv[k] = __uint_as_float((o & 2) ? t[k + 2] : t[k]);
+    } else {
+        // shift by o halves: o >> 1 words by two select levels, then o & 1 halves by a funnel shift
+        const int r = o >> 1;
+        uint32_t t[4 * NV + 3], u[4 * NV + 1];
+#pragma unroll
+        for (int j = 0; j < 4 * NV + 3; ++j) t[j] = (r & 1) ? raw[j + 1] : raw[j];
+#pragma unroll
+        for (int j = 0; j < 4 * NV + 1; ++j) u[j] = (r & 2) ? t[j + 2] : t[j];
+        const uint32_t sh = (uint32_t)(o & 1) * 16u;
+#pragma unroll
+        for (int k = 0; k < MAXI; k += 2) {
+            const uint32_t w = __funnelshift_r(u[k / 2], u[k / 2 + 1], sh);
+            xv[k] = __uint_as_float(w << 16);
+            if (k + 1 < MAXI) xv[k + 1] = __uint_as_float(w & 0xFFFF0000u);
+        }
     }
 }
 
@@ -295,26 +366,33 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
 
+    // Two rings of pipeline stages: B (TMA) with `stages` slots, and A with
+    // `sa_n` slots.  A produced tile (FWD, DCA) is small next to a wide B tile,
+    // so its ring is deeper: the producer groups fill A tiles several k-blocks
+    // ahead of the MMA while the B ring only has to cover the TMA latency.  When
+    // A arrives by TMA too (DX, GEMM) the two rings advance together (sa_n = stages).
     const int BN = a.BN, stages = a.stages;
+    const int sa_n = PRODUCE ? a.stages_a : a.stages;
     const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)BN * 128;
-    const uint32_t stage_bytes = (a_bytes + b_bytes) * C::SPLIT;
+    const uint32_t a_stage = a_bytes * C::SPLIT, b_stage = b_bytes * C::SPLIT;
     const uint32_t sbase = smem_addr(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
-    // barrier block: full[S] empty[S] zeroed[S] seg_full[2] seg_empty[2] accum
-    // (full[s]: stage s's TMA bytes have landed and every producer thread has
-    // written its part of a produced tile -- one barrier, so the MMA thread waits
-    // once per k-block; zeroed[s]: the zero fill of stage s's produced tile has landed)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * stages + 5);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sa_n * a_stage + stages * b_stage);
+    // barrier block: full[S] empty[S] afull[SA] aempty[SA] seg_full[2] seg_empty[2] accum
+    // (full[s]: B slot s (and, TMA-fed, A slot s) has landed; afull[s]: every
+    // producer thread of a group has written its row of A slot s)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 2 * sa_n + 5);
     auto full = [&](int s) { return smem_addr(&bars[s]); };
     auto empty = [&](int s) { return smem_addr(&bars[stages + s]); };
-    auto zeroed = [&](int s) { return smem_addr(&bars[2 * stages + s]); };
-    auto seg_full = [&](int g) { return smem_addr(&bars[3 * stages + g]); };
-    auto seg_empty = [&](int g) { return smem_addr(&bars[3 * stages + 2 + g]); };
-    const uint32_t accum_bar = smem_addr(&bars[3 * stages + 4]);
-    auto A_hi = [&](int s) { return sbase + s * stage_bytes; };
-    auto A_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes; };
-    auto B_hi = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT; };
-    auto B_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT + b_bytes; };
+    auto afull = [&](int s) { return smem_addr(&bars[2 * stages + s]); };
+    auto aempty = [&](int s) { return smem_addr(&bars[2 * stages + sa_n + s]); };
+    const int sb0 = 2 * stages + 2 * sa_n;
+    auto seg_full = [&](int g) { return smem_addr(&bars[sb0 + g]); };
+    auto seg_empty = [&](int g) { return smem_addr(&bars[sb0 + 2 + g]); };
+    const uint32_t accum_bar = smem_addr(&bars[sb0 + 4]);
+    auto A_hi = [&](int s) { return sbase + s * a_stage; };
+    auto A_lo = [&](int s) { return sbase + s * a_stage + a_bytes; };
+    auto B_hi = [&](int s) { return sbase + sa_n * a_stage + s * b_stage; };
+    auto B_lo = [&](int s) { return sbase + sa_n * a_stage + s * b_stage + b_bytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kb_begin = blockIdx.z * a.kb_per_split;
@@ -327,10 +405,12 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
-            // the TMA thread's expect-tx arrival, plus one per producer thread
-            mbar_init(full(s), 1 + ((MODE == FWD || MODE == DCA) ? 128 : 0));
-            mbar_init(empty(s), 1);
-            mbar_init(zeroed(s), 1);
+            mbar_init(full(s), 1);          // the TMA thread's expect-tx arrival
+            mbar_init(empty(s), 1);         // the MMA thread's commit
+        }
+        for (int s = 0; s < sa_n; ++s) {
+            mbar_init(afull(s), 128);       // every thread of one producer group
+            mbar_init(aempty(s), 1);        // the MMA thread's commit
         }
         mbar_init(seg_full(0), 1);
         mbar_init(seg_full(1), 1);
@@ -376,18 +456,6 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             for (int it = 0; it < nk; ++it, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
                 const int kb = kb_begin + it;
-                if (PRODUCE) {
-                    // the produced tile starts from zeros: a bulk copy from a zero buffer
-                    // (off the load/store pipe the producers use); dense SiLU tiles skip it
-                    const bool zero_it = MODE == FWD ? kb < a.nkb_main : (int)blockIdx.y < a.n_kt_tiles;
-                    if (zero_it) {
-                        mbar_arrive_expect_tx(zeroed(s), a_bytes * C::SPLIT);
-                        bulk_copy_g2s(A_hi(s), a.zeros, a_bytes, zeroed(s));
-                        if (F32) bulk_copy_g2s(A_lo(s), a.zeros, a_bytes, zeroed(s));
-                    } else {
-                        mbar_arrive(zeroed(s));
-                    }
-                }
                 const uint32_t bytes = (b_bytes + (A_BY_TMA ? a_bytes : 0u)) * C::SPLIT;
                 mbar_arrive_expect_tx(full(s), bytes);
                 if (MODE == FWD) {
@@ -421,10 +489,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 ++issued;
             }
             // every load issued lands before the CTA can exit
-            for (int it = max(0, issued - stages); it < issued; ++it) {
+            for (int it = max(0, issued - stages); it < issued; ++it)
                 mbar_wait(full(it % stages), (it / stages) & 1, a.status);
-                if (PRODUCE) mbar_wait(zeroed(it % stages), (it / stages) & 1, a.status);
-            }
         }
     } else if (warp == 1) {
         // ---------------- MMA issue ----------------
@@ -444,10 +510,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             const uint32_t a_sbo = A_SW32 ? 512u : 1024u;
             const uint32_t a_layout = A_SW32 ? 1u : 2u;
             bool ok = true;
-            int s = 0;
-            uint32_t ph = 0;
+            int s = 0, sa = 0;            // B and A ring positions (equal when A arrives by TMA)
+            uint32_t ph = 0, pha = 0;
             for (int it = 0; it < nk; ++it) {
                 if (!mbar_wait(full(s), ph, a.status)) { ok = false; break; }
+                if (PRODUCE && !mbar_wait(afull(sa), pha, a.status)) { ok = false; break; }
                 const int g = F32 ? it / kSegKb : 0;
                 const bool seg_start = F32 && (it % kSegKb == 0);
                 if (seg_start && g >= 2 && !mbar_wait(seg_empty(g & 1), ((g >> 1) - 1) & 1, a.status)) {
@@ -458,9 +525,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const uint32_t t_main = (g & 1) ? t_main1 : t_main0;
                 // descriptors of the stage's tiles; the k-steps advance the start address
                 // field (addresses stay below 2^18, so the field never carries)
-                const uint64_t ad0 = smem_desc(A_hi(s), a_lbo, a_sbo, a_layout);
+                const int sA = PRODUCE ? sa : s;
+                const uint64_t ad0 = smem_desc(A_hi(sA), a_lbo, a_sbo, a_layout);
                 const uint64_t bd0 = smem_desc_sw128(B_hi(s), b_lbo, 1024);
-                const uint64_t adl0 = F32 ? smem_desc(A_lo(s), a_lbo, a_sbo, a_layout) : 0;
+                const uint64_t adl0 = F32 ? smem_desc(A_lo(sA), a_lbo, a_sbo, a_layout) : 0;
                 const uint64_t bdl0 = F32 ? smem_desc_sw128(B_lo(s), b_lbo, 1024) : 0;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
@@ -485,10 +553,15 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     }
                 }
                 mma_commit(empty(s));
+                if (PRODUCE) mma_commit(aempty(sa));
                 if (F32 && ((it + 1) % kSegKb == 0 || it + 1 == nk)) mma_commit(seg_full(g & 1));
                 if (++s == stages) {
                     s = 0;
                     ph ^= 1;
+                }
+                if (PRODUCE && ++sa == sa_n) {
+                    sa = 0;
+                    pha ^= 1;
                 }
             }
             if (ok) mma_commit(accum_bar);
@@ -501,6 +574,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         if constexpr (PRODUCE) {
             const int p = threadIdx.x - 64;
             const T* X = reinterpret_cast<const T*>(a.x);
+            // Take A slot sa for a k-block: wait until the MMA has consumed its
+            // previous contents.  Each thread then zeroes the one 128-byte row it
+            // fills (16-byte stores, conflict-free under the swizzle) before it
+            // writes the row's non-zero basis values: no zero traffic from L2.
+            auto acquire = [&](int sa, uint32_t pha) -> bool { return mbar_wait(aempty(sa), pha ^ 1, a.status); };
             if constexpr (MODE == FWD) {
                 // rows = batch m0..m0+127.  kGroups groups of 128 threads take
                 // k-blocks in turn; a thread fills one whole row.  Per row and
@@ -520,19 +598,17 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 };
                 auto fetch = [&](int kb, float (&xv)[MAXI]) {
                     if (kb >= a.nkb_main || !row_ok) return;
-                    const int i0 = first_input(kb), n = last_input(kb) - i0 + 1;
-#pragma unroll
-                    for (int k = 0; k < MAXI; ++k) {
-                        if (k >= n) break;                  // uniform across the warp
-                        xv[k] = to_f(xrow[i0 + k]);
-                    }
+                    const int i0 = first_input(kb);
+                    load_x_window<T, MAXI>(xrow, i0, last_input(kb) - i0 + 1, (int)a.in, a.x_vec != 0, xv);
                 };
                 float nxt[MAXI];
-                // At most `stages` groups: then a group's previous k-block is no older
-                // than the previous use of the stage it waits for, so neither the
-                // empty nor the zeroed barrier can be two phases behind (a parity
+#pragma unroll
+                for (int k = 0; k < MAXI; ++k) nxt[k] = 0.0f;
+                // At most sa_n groups: then a group's previous k-block is no older
+                // than the previous use of the A slot it waits for, so neither the
+                // aempty barrier nor any other can be two phases behind (a parity
                 // wait on such a barrier would pass early).
-                const int NG = min(Warps<MODE>::kGroups, stages);
+                const int NG = min(Warps<MODE>::kGroups, sa_n);
                 if (grp < NG && grp < nk) fetch(kb_begin + grp, nxt);
                 int uses = 0;                               // k-blocks this group has filled
                 for (int it = grp; grp < NG && it < nk; it += NG, ++uses) {
@@ -541,32 +617,41 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     for (int k = 0; k < MAXI; ++k) cur[k] = nxt[k];
                     const int kb = kb_begin + it;
                     if (it + NG < nk) fetch(kb + NG, nxt);
-                    const int s = it % stages;
-                    const uint32_t ph = (it / stages) & 1;
-                    // the stage is free (its previous use consumed) and zero-filled
-                    if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
-                    if (!mbar_wait(zeroed(s), ph, a.status)) break;
+                    const int s = it % sa_n;
+                    const uint32_t ph = (it / sa_n) & 1;
+                    // the slot is free (its previous use consumed)
+                    if (!acquire(s, ph)) break;
                     const uint32_t ahi = A_hi(s), alo = A_lo(s);
                     const uint32_t rbase = row * 128u, rx = row & 7u;
                     if (kb < a.nkb_main) {
+                        zero_row<DT>(ahi + rbase, alo + rbase, rx);
                         if (row_ok) {
                             const int i0 = first_input(kb), n = last_input(kb) - i0 + 1;
                             const int cbase = i0 * a.nb - kb * BK;   // column of input i0's B_0 in this block
+                            // Straight-line over the MAXI input slots (the slots past n
+                            // store nothing), so the inputs' arithmetic can interleave.
 #pragma unroll
                             for (int k = 0; k < MAXI; ++k) {
-                                if (k >= n) break;
+                                const int base = cbase + k * a.nb;   // column of this input's B_0 (uniform)
+                                const bool act = k < n;
                                 if (F32 && a.ext) {   // input i0+k's SiLU column, when it falls in this block
-                                    const int cs = cbase + k * a.nb + a.nbs;
-                                    if ((unsigned)cs < (unsigned)BK) put1<DT>(ahi + rbase, alo + rbase, rx, cs, silu_f(cur[k]));
+                                    const int cs = base + a.nbs;
+                                    if (act && (unsigned)cs < (unsigned)BK)
+                                        put1<DT>(ahi + rbase, alo + rbase, rx, cs, silu_f(cur[k]));
                                 }
-                                const float u = fmaf(cur[k], a.inv_h, u0);
-                                if (!(u >= -3.0f && u < u_hi)) continue;   // outside the extended knots, NaN, inf
+                                float u = fmaf(cur[k], a.inv_h, u0);
+                                // outside the extended knots, NaN, inf: no stores
+                                const bool ok = act && u >= -3.0f && u < u_hi;
+                                u = ok ? u : 0.0f;
                                 int sidx;
                                 float f;
                                 floor_split(u, sidx, f);
                                 float w[4];
                                 weights_fma(u - f, w);
-                                scatter4<DT>(ahi + rbase, alo + rbase, rx, cbase + k * a.nb + sidx, sidx, a.nbs, BK, w);
+                                // basis indices whose columns lie in this block
+                                const int mlo = ok ? max(0, -base) : 0;
+                                const int mhi = ok ? min(a.nbs, BK - base) : 0;
+                                scatter_win<DT>(ahi + rbase, alo + rbase, rx, base, sidx, mlo, mhi, w);
                             }
                         }
                     } else {
@@ -597,7 +682,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                     fence_async_smem();
-                    mbar_arrive(full(s));
+                    mbar_arrive(afull(s));
                 }
                 (void)uses;
             } else if constexpr (MODE == DCA) {
@@ -623,12 +708,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 auto fetch = [&](int kb, float (&xv)[MAXI]) {
                     const int64_t b = (int64_t)kb * BK + rb;
                     if (silu_tile || b >= a.batch) return;
-                    const T* xr = X + b * a.in + i_first;
-#pragma unroll
-                    for (int k = 0; k < MAXI; ++k) {
-                        if (k >= n_inp) break;
-                        xv[k] = to_f(xr[k]);
-                    }
+                    load_x_window<T, MAXI>(X + b * a.in, i_first, n_inp, (int)a.in, a.x_vec != 0, xv);
                 };
                 // byte offset of column c (0..EPB-1) inside this thread's atom row
                 auto col_off = [&](int c) -> uint32_t {
@@ -636,7 +716,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     else return sw128_byte((uint32_t)rb, (uint32_t)c * 2u) - (uint32_t)rb * 128u;
                 };
                 float nxt[MAXI];
-                const int NG = min(Warps<MODE>::kGroups, stages);   // see the forward producer
+#pragma unroll
+                for (int k = 0; k < MAXI; ++k) nxt[k] = 0.0f;
+                const int NG = min(Warps<MODE>::kGroups, sa_n);   // see the forward producer
                 if (grp < NG && grp < nk) fetch(kb_begin + grp, nxt);
                 for (int it = grp; grp < NG && it < nk; it += NG) {
                     float cur[MAXI];
@@ -644,23 +726,25 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     for (int k = 0; k < MAXI; ++k) cur[k] = nxt[k];
                     const int kb = kb_begin + it;
                     if (it + NG < nk) fetch(kb + NG, nxt);
-                    const int s = it % stages;
-                    const uint32_t ph = (it / stages) & 1;
-                    if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
-                    if (!mbar_wait(zeroed(s), ph, a.status)) break;
+                    const int s = it % sa_n;
+                    const uint32_t ph = (it / sa_n) & 1;
+                    if (!acquire(s, ph)) break;
                     const int64_t b = (int64_t)kb * BK + rb;
                     const bool row_ok = b < a.batch;
                     const uint32_t roff = (uint32_t)atom * BK * 128u + (uint32_t)rb * 128u;
                     const uint32_t rb_hi = A_hi(s) + roff, rb_lo = A_lo(s) + roff;
                     if (!silu_tile) {
+                        // this thread's atom row starts from zeros (rows past the batch stay zero)
+                        zero_row<DT>(rb_hi, rb_lo, (uint32_t)rb & 7u);
                         if (row_ok) {
                             const int cbase = i_first * a.nb - c_lo;
+                            // straight-line over the MAXI input slots (see the forward producer)
 #pragma unroll
                             for (int k = 0; k < MAXI; ++k) {
-                                if (k >= n_inp) break;
+                                const bool act = k < n_inp;
                                 if (F32 && a.ext) {   // input i_first+k's SiLU column, when it falls in this atom
                                     const int cs = cbase + k * a.nb + a.nbs;
-                                    if ((unsigned)cs < (unsigned)EPB) {
+                                    if (act && (unsigned)cs < (unsigned)EPB) {
                                         const float v = silu_f(cur[k]);
                                         const uint32_t off = col_off(cs);
                                         if constexpr (F32) {
@@ -672,17 +756,22 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                         }
                                     }
                                 }
-                                const float u = fmaf(cur[k], a.inv_h, u0);
-                                if (!(u >= -3.0f && u < u_hi)) continue;
+                                float u = fmaf(cur[k], a.inv_h, u0);
+                                const bool ok = act && u >= -3.0f && u < u_hi;   // NaN, inf fail
+                                u = ok ? u : 0.0f;
                                 int sidx;
                                 float f;
                                 floor_split(u, sidx, f);
                                 float w[4];
                                 weights_fma(u - f, w);
-                                const int col0 = cbase + k * a.nb + sidx;
+                                const int base = cbase + k * a.nb;
+                                // basis indices whose columns lie in this atom (empty when !ok)
+                                const int mlo = ok ? max(0, -base) : 0;
+                                const uint32_t width = ok ? (uint32_t)(min(a.nbs, EPB - base) - mlo) : 0u;
+                                const int col0 = base + sidx;
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) {
-                                    if ((unsigned)(sidx + q) < (unsigned)a.nbs && (unsigned)(col0 + q) < (unsigned)EPB) {
+                                    if ((uint32_t)(sidx + q - mlo) < width) {
                                         const uint32_t off = col_off(col0 + q);
                                         if constexpr (F32) {
                                             const float hi = tf32_hi(w[q]);
@@ -737,7 +826,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                     fence_async_smem();
-                    mbar_arrive(full(s));
+                    mbar_arrive(afull(s));
                 }
             }
         }
@@ -1467,8 +1556,25 @@ int stages_for(int BN, bool f32)
     return std::min(8, (kSmemBudget - 1024 - 512) / stage_bytes);
 }
 
-// pipeline stages + 1024 alignment slack + 512 for the barrier block (3*stages+5 mbarriers) and the TMEM slot
-int smem_bytes(int BN, int stages, bool f32) { return stages * (kBM * 128 + BN * 128) * (f32 ? 2 : 1) + 1024 + 512; }
+// Kernels with a produced A tile: as many B slots as fit (at most 4) while
+// the A ring keeps at least 4 slots (3 for fp32), then the rest of the shared
+// memory to the A ring (at most 8 slots).  A wide B tile (64 KiB for 512
+// bf16 columns) leaves room for only 2 B slots.
+void stages_ab(int BN, bool f32, int& sb, int& sa)
+{
+    const int a_stage = kBM * 128 * (f32 ? 2 : 1), b_stage = BN * 128 * (f32 ? 2 : 1);
+    const int avail = kSmemBudget - 1024 - 512;
+    const int sa_min = f32 ? 3 : 4;
+    sb = 4;
+    while (sb > 2 && (avail - sb * b_stage) / a_stage < sa_min) --sb;
+    sa = std::min(8, (avail - sb * b_stage) / a_stage);
+}
+
+// pipeline slots + 1024 alignment slack + 512 for the barrier block (2*stages + 2*stages_a + 5 mbarriers) and the TMEM slot
+int smem_bytes(int BN, int stages, int stages_a, bool f32)
+{
+    return (stages * BN * 128 + stages_a * kBM * 128) * (f32 ? 2 : 1) + 1024 + 512;
+}
 
 
 // Workspace layout, shared by the size query and the launches.
@@ -1486,9 +1592,9 @@ struct Plan {
     int nbx;
     int64_t Kx;
     // forward
-    int f_BN, f_stages, f_n, f_m, f_splits, f_kps, f_nkb_main, f_nkb_total;
+    int f_BN, f_stages, f_stages_a, f_n, f_m, f_splits, f_kps, f_nkb_main, f_nkb_total;
     // dcoef
-    int d_BN, d_stages, d_n, d_m, d_nkt, d_splits, d_kps, d_nkb;
+    int d_BN, d_stages, d_stages_a, d_n, d_m, d_nkt, d_splits, d_kps, d_nkb;
     int64_t d_ld;
     int64_t ldb;   // padded row length of dY^T (fp32)
     // dx
@@ -1513,7 +1619,7 @@ Plan make_plan(const Problem& p, int sms)
     const bool sep_silu = p.base && !P.ext;   // separate SiLU k-blocks / tiles / GEMM
     // forward: M = batch, N = out, K = spline (+ SiLU) columns
     P.f_BN = f32 ? bn_for(p.out, true) : wide_bn(p.out);
-    P.f_stages = stages_for(P.f_BN, f32);
+    stages_ab(P.f_BN, f32, P.f_stages, P.f_stages_a);
     P.f_n = (int)cdiv(p.out, P.f_BN);
     P.f_m = (int)cdiv(p.batch, kBM);
     P.f_nkb_main = (int)cdiv(P.Kx, BK);
@@ -1526,7 +1632,7 @@ Plan make_plan(const Problem& p, int sms)
     P.d_n = (int)cdiv(p.out, P.d_BN);
     P.d_nkt = (int)cdiv(P.Kx, kBM);
     P.d_m = P.d_nkt + (sep_silu ? (int)cdiv(p.in, kBM) : 0);
-    P.d_stages = stages_for(P.d_BN, f32);
+    stages_ab(P.d_BN, f32, P.d_stages, P.d_stages_a);
     P.d_nkb = (int)cdiv(p.batch, BK);
     P.d_splits = pick_splits((int64_t)P.d_n * P.d_m, sms, std::min(16, std::max(1, P.d_nkb / 8)));
     P.d_kps = (int)cdiv(std::max(1, P.d_nkb), P.d_splits);
@@ -1613,12 +1719,16 @@ inline int grid_for(int64_t n) { return (int)std::min<int64_t>(std::max<int64_t>
 template <int MODE, int DT, int MAXI>
 cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args, cudaStream_t st)
 {
+    constexpr bool produce = MODE == FWD || MODE == DCA;
+    const int stages_a = produce ? args.stages_a : stages;
     // the MN-major bf16 B operand arrives in whole 128-byte boxes: BN must be a multiple of 64
     if (MODE != FWD && DT == KAN_BF16 && BN % 64 != 0) return cudaErrorInvalidConfiguration;
     if (BN % 16 != 0 || BN < 16 || BN > (MODE == FWD || MODE == DCA ? 512 : 256) || (BN > 256 && BN % 128 != 0) ||
-        (DT == KAN_F32 && BN > 128) || stages < 2)
+        (DT == KAN_F32 && BN > 128) || stages < 2 || stages_a < 2 || stages + stages_a > 24 ||
+        (!produce && stages_a != stages))
         return cudaErrorInvalidConfiguration;
-    const int smem = smem_bytes(BN, stages, DT == KAN_F32);
+    const int smem = smem_bytes(BN, stages, stages_a, DT == KAN_F32);
+    if (smem > kSmemBudget) return cudaErrorInvalidConfiguration;
     static int configured = 0;   // per instantiation; the attribute is per function
     if (configured < smem) {
         cudaError_t e = cudaFuncSetAttribute(tc_kernel<MODE, DT, MAXI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1673,24 +1783,6 @@ cudaError_t launch_dx_persistent(const Plan& P, const CUtensorMap* maps, const D
     return cudaGetLastError();
 }
 
-// 16 KiB of zeros: the source of the produced tiles' zero fill.
-static __device__ __align__(128) unsigned char g_zero_tile[16384];
-
-const void* zero_tile_ptr()
-{
-    static void* ptrs[64] = {nullptr};
-    static std::mutex mu;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!ptrs[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_zero_tile) != cudaSuccess) return nullptr;
-        ptrs[dev] = p;
-    }
-    return ptrs[dev];
-}
-
 TcArgs base_args(const Problem& p, const Plan& P)
 {
     TcArgs a{};
@@ -1706,8 +1798,8 @@ TcArgs base_args(const Problem& p, const Plan& P)
     a.inv_h = p.inv_h;
     a.Kt = (int)P.Kx;
     a.has_base = p.base;
+    a.x_vec = (p.in * (p.dtype == KAN_F32 ? 4 : 2)) % 16 == 0;
     a.nb_magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)P.nbx - 1) / (uint64_t)P.nbx);
-    a.zeros = zero_tile_ptr();
     return a;
 }
 
@@ -1798,10 +1890,6 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
                        int num_sms, cudaStream_t st, const char** detail)
 {
     if (p.batch == 0) return cudaSuccess;
-    if (!zero_tile_ptr()) {
-        *detail = "the zero tile's device address is not available";
-        return cudaErrorInvalidValue;
-    }
     const bool f32 = p.dtype == KAN_F32;
     const int BK = f32 ? 32 : 64;
     const Plan P = make_plan(p, num_sms);
@@ -1836,6 +1924,7 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
     a.out = P.f_splits > 1 ? (void*)(w + P.fwd.fwd_part) : y;
     a.BN = P.f_BN;
     a.stages = P.f_stages;
+    a.stages_a = P.f_stages_a;
     a.fbox = fbox;
     a.nkb_main = P.f_nkb_main;
     a.nkb_total = P.f_nkb_total;
@@ -1868,10 +1957,6 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
     const Plan P = make_plan(p, num_sms);
     uint8_t* w = reinterpret_cast<uint8_t*>(ws);
     cudaError_t e;
-    if (!zero_tile_ptr()) {
-        *detail = "the zero tile's device address is not available";
-        return cudaErrorInvalidValue;
-    }
     if (p.batch == 0) {
         if (dcoef && (e = zero_f32(dcoef, p.out * p.Kt, st)) != cudaSuccess) return e;
         if (dw_base && (e = zero_f32(dw_base, p.out * p.in, st)) != cudaSuccess) return e;
@@ -1898,6 +1983,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         float* partbuf = reinterpret_cast<float*>(w + P.bwd.dc_part);
         a.BN = P.d_BN;
         a.stages = P.d_stages;
+        a.stages_a = P.d_stages_a;
         a.nkb_main = a.nkb_total = P.d_nkb;
         a.kb_per_split = P.d_kps;
         a.n_kt_tiles = P.d_nkt;
