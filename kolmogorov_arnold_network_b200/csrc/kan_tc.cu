@@ -1051,11 +1051,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
 // Gm = dY . coef for a tile goes to one of two TMEM accumulators while the
 // epilogue warps turn the previous tile's accumulator into dx, so the B'
 // gather overlaps the next tile's MMA.  Warps: 0 TMA, 1 MMA issue + TMEM,
-// 2-5 epilogue (one per TMEM lane quarter).  fp32 keeps the tf32 correction
+// 2-9 epilogue (two per TMEM lane quarter).  fp32 keeps the tf32 correction
 // products in a second accumulator per buffer; the contraction over `out`
 // is short enough (at most 32 k-blocks) that no promotion is needed.
 // ---------------------------------------------------------------------------
-constexpr int kDxThreads = 192;
+constexpr int kDxThreads = 320;   // warps: 0 TMA, 1 MMA, 2-9 epilogue
 
 struct DxArgs {
     const void* x;
@@ -1098,6 +1098,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes + 4 * 32 * a.ld_stage * (int)sizeof(ST));
     // full[S] empty[S] acc_full[2] acc_empty[2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 4);
+    volatile int* pair_ok = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [4 quarters][2 warps]
     auto full = [&](int s) { return smem_addr(&bars[s]); };
     auto empty = [&](int s) { return smem_addr(&bars[stages + s]); };
     auto acc_full = [&](int b) { return smem_addr(&bars[2 * stages + b]); };
@@ -1116,8 +1117,8 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         }
         mbar_init(acc_full(0), 1);
         mbar_init(acc_full(1), 1);
-        mbar_init(acc_empty(0), 128);
-        mbar_init(acc_empty(1), 128);
+        mbar_init(acc_empty(0), 256);   // every epilogue thread
+        mbar_init(acc_empty(1), 256);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -1210,38 +1211,59 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue: warps 2-5 ----------------
+        // ---------------- epilogue: warps 2-9 ----------------
+        // Two warps per TMEM lane quarter (q = warp & 3; h = which of the two):
+        // each stages half of the accumulator row's columns into the quarter's
+        // shared staging rows, the pair meets at a named barrier, and then each
+        // turns half of the tile's inputs into dx.
         const int q = warp & 3;
+        const int h = (warp - 2) >> 2;
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         const int r = 32 * q + lane;
-        ST* srow = staging + (size_t)(warp - 2) * 32 * a.ld_stage + (size_t)lane * a.ld_stage;
+        ST* srow = staging + (size_t)q * 32 * a.ld_stage + (size_t)lane * a.ld_stage;
+        const int half_cols = BN / 2;                 // a multiple of 16
         constexpr int XC = 16;
+        const bool x_vec = (a.in * (int64_t)sizeof(T)) % 16 == 0;
+        const bool g_vec = (a.in * 4) % 16 == 0;
         for (int lt = 0; lt < my_tiles; ++lt) {
             int64_t m0;
             int i0;
             tile_coords(lt, m0, i0);
             const int64_t b = m0 + r;
+            const bool b_ok = b < a.batch;
             const int i1 = min((int)a.in, i0 + a.n_in_tile);
             const int kt_al = kt_start(i0);
+            // this warp's inputs: the first or second half of the tile's
+            const int im = i0 + (i1 - i0 + 1) / 2;
+            const int ia = h ? im : i0, ib = h ? i1 : im;
+            const T* xrow = reinterpret_cast<const T*>(a.x) + (b_ok ? b : 0) * a.in;
+            const float* grow = a.gb ? a.gb + (b_ok ? b : 0) * a.in : nullptr;
             // x (and dY.w_base) of the first inputs, ahead of the accumulator
-            uint32_t xa[XC], ga[XC];
+            float xa[XC], ga[XC];
             auto xfetch = [&](int i_start) {
-#pragma unroll
-                for (int k = 0; k < XC; ++k) {
-                    const int i = i_start + k;
-                    const bool okk = b < a.batch && i < i1;
-                    xa[k] = okk ? __float_as_uint(to_f(reinterpret_cast<const T*>(a.x)[b * a.in + i])) : 0u;
-                    ga[k] = (okk && a.gb) ? __float_as_uint(a.gb[b * a.in + i]) : 0u;
+                const int n = min(XC, ib - i_start);
+                if (b_ok && n > 0) {
+                    load_x_window<T, XC>(xrow, i_start, n, (int)a.in, x_vec, xa);
+                    if (grow) load_x_window<float, XC>(grow, i_start, n, (int)a.in, g_vec, ga);
                 }
             };
-            xfetch(i0);
+#pragma unroll
+            for (int k = 0; k < XC; ++k) xa[k] = ga[k] = 0.0f;
+            xfetch(ia);
             const int buf = lt & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(acc_full(buf), (lt >> 1) & 1, a.status))) break;
+            // The pair agrees on the bounded wait's outcome (so that both leave the
+            // loop together, never one of them waiting at a named barrier for the
+            // other); the barrier also tells each that its partner has finished
+            // reading the previous tile's staged row.
+            const bool got = __all_sync(0xffffffffu, mbar_wait(acc_full(buf), (lt >> 1) & 1, a.status));
+            if (lane == 0) pair_ok[2 * q + h] = got ? 1 : 0;
+            named_bar_sync(1 + q, 64);
+            if (!(pair_ok[2 * q] && pair_ok[2 * q + 1])) break;
             tc_fence_after();
-            // stage the row: TMEM -> registers -> shared (16-byte stores; the row
-            // stride is 16 bytes mod 128, so a warp's stores are conflict-free)
+            // stage this warp's half of the row: TMEM -> registers -> shared (16-byte
+            // stores; the row stride is 16 bytes mod 128, so a warp's stores are conflict-free)
             const uint32_t t_main = tmem + buf * acc_cols + lane_off;
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = h * half_cols; c0 < (h + 1) * half_cols; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld16(t_main + c0, v);
                 if constexpr (F32) {
@@ -1268,20 +1290,22 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             // the accumulator buffer is free for the tile after next
             tc_fence_before();
             mbar_arrive(acc_empty(buf));
-            if (b < a.batch) {
+            // both halves of the row are staged
+            named_bar_sync(1 + q, 64);
+            if (b_ok) {
                 T* dxr = reinterpret_cast<T*>(a.dx) + b * a.in;
-                for (int ic = i0; ic < i1; ic += XC) {
-                    uint32_t xc[XC], gc[XC];
+                for (int ic = ia; ic < ib; ic += XC) {
+                    float xc[XC], gc[XC];
 #pragma unroll
                     for (int k = 0; k < XC; ++k) {
                         xc[k] = xa[k];
                         gc[k] = ga[k];
                     }
-                    if (ic + XC < i1) xfetch(ic + XC);
-                    const int nkc = min(XC, i1 - ic);     // inputs in this chunk
+                    if (ic + XC < ib) xfetch(ic + XC);
+                    const int nkc = min(XC, ib - ic);     // inputs in this chunk
                     auto dx_of = [&](int k) -> float {
                         const int i = ic + k;
-                        const float xv = __uint_as_float(xc[k]);
+                        const float xv = xc[k];
                         const Span sp = span_of(xv, a.lo, a.inv_h, a.G);
                         float acc = 0.0f;
                         if (sp.valid) {
@@ -1295,7 +1319,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                             }
                         }
                         if (F32 && a.ext) acc += dsilu_f(xv) * to_f(srow[i * a.nb - kt_al + a.nbs]);   // dY.w_base, staged
-                        else if (a.gb) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
+                        else if (a.gb) acc += dsilu_f(xv) * gc[k];
                         return acc;
                     };
                     if (nkc == XC && (((uintptr_t)(dxr + ic)) & 15u) == 0) {
