@@ -201,7 +201,8 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 operands, fp32 accumulation.
+// D[tmem] (+)= A[smem] * B[smem]^T, 16-bit operands (bf16 or fp16, per the
+// instruction descriptor), fp32 accumulation.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate)
 {
@@ -209,18 +210,6 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uin
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Same with tf32 operands (32-bit containers; the unit reads the tf32 part).
-__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -297,18 +286,9 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return smem_desc(saddr, lbo_bytes, sbo_bytes, 2u);
 }
 
-// Layout 1: 128-byte rows whose four 32-byte granules are permuted by XOR
-// with (row & 3); the atom is 4 rows (512 bytes).  This is the form an
-// MN-major tf32 operand takes: for it SBO is the stride between 4-row
-// groups along K and LBO the stride between 128-byte column blocks along MN.
-__device__ __forceinline__ uint32_t sw128b32_byte(uint32_t row, uint32_t colb)
-{
-    return row * 128u + ((((colb >> 5) ^ (row & 3u)) & 3u) << 5) + (colb & 31u);
-}
-
-// Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation:
+// Instruction descriptor for kind::f16 with fp32 accumulation:
 //   bits 4-5 D format (1 = f32), bits 7-9 A format, bits 10-12 B format
-//   (bf16 = 1, tf32 = 2), bit 15 A major, bit 16 B major (0 = K, 1 = MN),
+//   (fp16 = 0, bf16 = 1), bit 15 A major, bit 16 B major (0 = K, 1 = MN),
 //   bits 17-22 N >> 3, bits 24-28 M >> 4.
 __host__ __device__ constexpr uint32_t instr_desc(uint32_t ab_format, uint32_t a_mn_major, uint32_t b_mn_major,
                                                   uint32_t M, uint32_t N)
@@ -328,17 +308,6 @@ __device__ __forceinline__ uint32_t sw128_chunk(uint32_t row, uint32_t chunk)
 __device__ __forceinline__ uint32_t sw128_byte(uint32_t row, uint32_t colb)
 {
     return sw128_chunk(row, colb >> 4) | (colb & 15u);
-}
-
-// tf32 split: hi keeps the 10 explicit mantissa bits of x rounded to
-// nearest (cvt.rna.tf32.f32), lo = x - hi is exact in fp32 and is itself
-// read by the unit at tf32 precision; hi*hi' + hi*lo' + lo*hi' then carries
-// about 21 bits of each product.
-__device__ __forceinline__ float tf32_hi(float x)
-{
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
 }
 
 }  // namespace kan

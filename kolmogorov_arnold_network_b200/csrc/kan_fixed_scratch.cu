@@ -6,7 +6,7 @@
 // (cudaMalloc can synchronise the device and take driver locks), and hosts
 // that budget all device memory up front.  kan_forward needs caller-provided
 // workspace on the tensor-core path (split-K partial sums, and for fp32 the
-// tf32 hi/lo copies of the coefficients).  kan_forward_fixed_scratch runs the
+// fp16 hi/lo copies of the coefficients).  kan_forward_fixed_scratch runs the
 // same forward with that workspace taken from a fixed array that lives in this
 // library's device image instead.
 //

@@ -25,18 +25,23 @@
 //
 // fp32 with the SiLU branch: silu(x_i) is one more basis function of input i,
 // with coefficient w_base[j, i].  Its column sits right after input i's G+3
-// spline columns (column stride G+4) in the tf32 copies of the coefficients
+// spline columns (column stride G+4) in the fp16 copies of the coefficients
 // that the fp32 path makes anyway, so the SiLU terms ride along in every GEMM:
 // the forward sums them, dcoef's epilogue writes dw_base, and the dx epilogue
 // finds dY.w_base in its own accumulator.
 //
-// fp32 operands: three tf32 products per term, hi*hi + hi*lo + lo*hi, which
-// keep about 21 significant bits of each product.  The tensor core's fp32
-// accumulation truncates, so long accumulations drift; the kernel therefore
-// (a) accumulates the small hi*lo + lo*hi products in their own TMEM
-// accumulator, and (b) accumulates hi*hi in short segments of kSegKb
-// k-blocks, alternating between two TMEM buffers, which the epilogue warps add
-// into a running fp32 total (round-to-nearest) while the next segment runs.
+// fp32 operands: every operand value v (times a per-call power-of-two scale
+// taken from the operands' absolute maxima, so that it sits well inside the
+// fp16 range) is split into two fp16 parts, hi = fp16(v) and lo =
+// fp16((v - hi) * 2^11), which together carry about 22 significant bits.
+// Three fp16 tensor-core products per term, hi*hi + (hi*lo + lo*hi) * 2^-11,
+// keep about 21 bits of each product; the basis values need no scale (they
+// lie in [0, 2/3]).  The tensor core's fp32 accumulation truncates, so long
+// accumulations drift; the kernel therefore (a) accumulates the small hi*lo +
+// lo*hi products in their own TMEM accumulator, and (b) accumulates hi*hi in
+// short segments of kSegKb k-blocks, alternating between two TMEM buffers,
+// which the epilogue warps add into a running fp32 total (round-to-nearest)
+// while the next segment runs.
 // bf16 operands: one kind::f16 product, fp32 accumulation in TMEM.
 //
 // Deterministic by construction: every output element is reduced by one CTA
@@ -48,6 +53,8 @@
 #include <algorithm>
 #include <type_traits>
 #include <mutex>
+
+#include <cuda_fp16.h>
 
 #include "kan_device.cuh"
 
@@ -82,14 +89,59 @@ template <> struct Cfg<KAN_BF16> {
     static constexpr int UMMA_K = 16;
     static constexpr uint32_t FMT = 1;     // bf16
 };
+// fp32 operands: each value v (times a power-of-two scale) as two fp16
+// parts, hi = fp16(v) and lo = fp16((v - hi) * 2^11); the tensor core sums
+// hi*hi and, in a separate accumulator, hi*lo + lo*hi (scaled back by 2^-11).
 template <> struct Cfg<KAN_F32> {
-    using T = float;
-    static constexpr int BK = 32;
-    static constexpr int ESZ = 4;
-    static constexpr int SPLIT = 2;        // hi and lo tf32 parts
-    static constexpr int UMMA_K = 8;
-    static constexpr uint32_t FMT = 2;     // tf32
+    using T = float;                       // x, y, dx element
+    static constexpr int BK = 64;          // K elements per 128-byte operand row
+    static constexpr int ESZ = 2;          // operand element size (fp16)
+    static constexpr int SPLIT = 2;        // hi and lo fp16 parts
+    static constexpr int UMMA_K = 16;
+    static constexpr uint32_t FMT = 0;     // f16
 };
+
+// Scale of the lo part of a split operand, and its inverse.
+constexpr float kLoScale = 2048.0f;
+constexpr float kLoInv = 1.0f / 2048.0f;
+
+// v -> (hi, lo) fp16 bit patterns with v ~= hi + lo * 2^-11 (about 22
+// significant bits; v - hi is exact in fp32).
+__device__ __forceinline__ void split_f16(float v, uint16_t& hi, uint16_t& lo)
+{
+    const __half h = __float2half_rn(v);
+    const __half l = __float2half_rn((v - __half2float(h)) * kLoScale);
+    hi = __half_as_ushort(h);
+    lo = __half_as_ushort(l);
+}
+
+// Power-of-two scale s with m * s in [2^12, 2^13) (1 when m is 0, NaN or inf):
+// scaled values stay well inside the fp16 range, and their lo parts too.
+__host__ __device__ __forceinline__ float pow2_scale(float m)
+{
+    if (!(m > 0.0f) || !(m <= 3.0e38f)) return 1.0f;
+    int ex;
+    (void)frexpf(m, &ex);                  // m = f * 2^ex, f in [0.5, 1)
+    const int e = min(100, max(-100, 13 - ex));
+    return ldexpf(1.0f, e);
+}
+
+// Per-call operand scales of the fp32 path, from the absolute maxima that
+// absmax_kernel leaves in the workspace: amax[0] coef, [1] w_base, [2] x, [3] dY.
+//   x: silu(x) values (|silu(x)| <= |x|)
+//   c: coef, and w_base times c / x (so that silu * w_base carries the same scale c)
+//   d: dY
+struct Scales {
+    float c, x, d;
+};
+__device__ __forceinline__ Scales scales_of(const unsigned int* amax)
+{
+    Scales sc;
+    sc.x = pow2_scale(__uint_as_float(amax[2]));
+    sc.c = pow2_scale(fmaxf(__uint_as_float(amax[0]), __uint_as_float(amax[1]) / sc.x));
+    sc.d = pow2_scale(__uint_as_float(amax[3]));
+    return sc;
+}
 
 struct TcArgs {
     const void* x;             // [batch, in] operand dtype (FWD, DCA, DX epilogue)
@@ -113,6 +165,7 @@ struct TcArgs {
     int n_in_tile;             // DX: inputs per N tile
     int has_base;
     int x_vec;                 // 1: rows of x are 16-byte aligned (in * sizeof(T) % 16 == 0), vector loads allowed
+    const unsigned int* amax;  // fp32: absolute maxima of the operands (scales_of)
     uint32_t nb_magic;         // ceil(2^32 / nb): c / nb == umulhi(c, nb_magic) for c < 2^32 / nb
     int fbox;                  // FWD: rows per B box
 };
@@ -138,10 +191,6 @@ __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v)
     asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
-__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v)
-{
-    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
@@ -149,22 +198,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// One A element at (row, col) of a K-major swizzled tile: bf16, or the tf32 hi/lo pair.
-template <int DT>
-__device__ __forceinline__ void put_a(uint32_t a_hi, uint32_t a_lo, uint32_t row, int col, float v)
-{
-    const uint32_t off = sw128_byte(row, (uint32_t)col * Cfg<DT>::ESZ);
-    if constexpr (DT == KAN_BF16) {
-        __nv_bfloat16 h = __float2bfloat16_rn(v);
-        st_shared_u16(a_hi + off, *reinterpret_cast<uint16_t*>(&h));
-    } else {
-        const float hi = tf32_hi(v);
-        st_shared_f32(a_hi + off, hi);
-        st_shared_f32(a_lo + off, v - hi);
-    }
-}
-
-// 16 bytes of dense A values (8 bf16 or 4 fp32) at 16-byte chunk `chunk` of `row`.
+// 16 bytes of dense A values (8 operand elements) at 16-byte chunk `chunk` of `row`.
 template <int DT>
 __device__ __forceinline__ void put_a_chunk(uint32_t a_hi, uint32_t a_lo, uint32_t row, uint32_t chunk, const float* v)
 {
@@ -173,16 +207,17 @@ __device__ __forceinline__ void put_a_chunk(uint32_t a_hi, uint32_t a_lo, uint32
         st_shared_v4(a_hi + off, pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
                      pack_bf16(v[6], v[7]));
     } else {
-        float h[4], l[4];
+        uint32_t h[4], l[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            h[e] = tf32_hi(v[e]);
-            l[e] = v[e] - h[e];
+            uint16_t h0, l0, h1, l1;
+            split_f16(v[2 * e], h0, l0);
+            split_f16(v[2 * e + 1], h1, l1);
+            h[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+            l[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
         }
-        st_shared_v4(a_hi + off, __float_as_uint(h[0]), __float_as_uint(h[1]), __float_as_uint(h[2]),
-                     __float_as_uint(h[3]));
-        st_shared_v4(a_lo + off, __float_as_uint(l[0]), __float_as_uint(l[1]), __float_as_uint(l[2]),
-                     __float_as_uint(l[3]));
+        st_shared_v4(a_hi + off, h[0], h[1], h[2], h[3]);
+        st_shared_v4(a_lo + off, l[0], l[1], l[2], l[3]);
     }
 }
 
@@ -222,7 +257,7 @@ template <int DT>
 __device__ __forceinline__ void scatter_win(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx, int base, int s, int mlo,
                                             int mhi, const float (&w)[4])
 {
-    constexpr int ESZ = DT == KAN_F32 ? 4 : 2;
+    constexpr int ESZ = 2;   // operand element size, both dtypes
     const uint32_t width = (uint32_t)(mhi - mlo);
     if constexpr (DT == KAN_BF16) {
         const uint32_t p01 = pack_bf16(w[0], w[1]), p23 = pack_bf16(w[2], w[3]);
@@ -236,9 +271,10 @@ __device__ __forceinline__ void scatter_win(uint32_t rb_hi, uint32_t rb_lo, uint
         for (int q = 0; q < 4; ++q)
             if ((uint32_t)(s + q - mlo) < width) {
                 const uint32_t off = sw_col<ESZ>(base + s + q, rx);
-                const float hi = tf32_hi(w[q]);
-                st_shared_f32(rb_hi + off, hi);
-                st_shared_f32(rb_lo + off, w[q] - hi);
+                uint16_t h, l;
+                split_f16(w[q], h, l);
+                st_shared_u16(rb_hi + off, h);
+                st_shared_u16(rb_lo + off, l);
             }
     }
 }
@@ -318,13 +354,14 @@ __device__ __forceinline__ void load_x_window(const T* __restrict__ row, int i0,
 template <int DT>
 __device__ __forceinline__ void put1(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx, int col, float v)
 {
-    constexpr int ESZ = DT == KAN_F32 ? 4 : 2;
+    constexpr int ESZ = 2;
     if constexpr (DT == KAN_BF16) {
         st_shared_u16(rb_hi + sw_col<ESZ>(col, rx), __bfloat16_as_ushort(__float2bfloat16_rn(v)));
     } else {
-        const float hi = tf32_hi(v);
-        st_shared_f32(rb_hi + sw_col<ESZ>(col, rx), hi);
-        st_shared_f32(rb_lo + sw_col<ESZ>(col, rx), v - hi);
+        uint16_t h, l;
+        split_f16(v, h, l);
+        st_shared_u16(rb_hi + sw_col<ESZ>(col, rx), h);
+        st_shared_u16(rb_lo + sw_col<ESZ>(col, rx), l);
     }
 }
 
@@ -357,12 +394,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     constexpr bool PRODUCE = MODE == FWD || MODE == DCA;
     constexpr bool A_BY_TMA = MODE == DX || MODE == GEMM;
     constexpr bool A_MN = MODE == DCA;               // producer-written MN-major basis
-    // an MN-major tf32 operand uses the 32-byte-atom 128-byte swizzle (layout 1)
-    constexpr bool A_SW32 = A_MN && F32;
-    // B stored MN-major (dY for dcoef, coef / w_base for dx) for bf16; the
-    // fp32 path's split copies are transposed to K-major instead (tf32
-    // MN-major operands would need the 32-byte-atom swizzle).
-    constexpr bool B_MN = MODE != FWD && !F32;
+    constexpr bool A_SW32 = false;                   // (2-byte operands: the plain 128-byte swizzle)
+    // B stored MN-major (dY for dcoef, coef / w_base for dx), for both dtypes
+    // (the fp32 path's fp16 split copies keep the source layout)
+    constexpr bool B_MN = MODE != FWD;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
 
@@ -480,6 +515,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         for (int c = 0; c < BN / EPB; ++c) {
                             const uint32_t off = (uint32_t)c * BK * 128;
                             tma_load_2d(B_hi(s) + off, &tB_hi, full(s), nbase + c * EPB, kb * BK);
+                            if (F32) tma_load_2d(B_lo(s) + off, &tB_lo, full(s), nbase + c * EPB, kb * BK);
                         }
                     } else {
                         tma_load_2d(B_hi(s), &tB_hi, full(s), kb * BK, nbase);
@@ -542,14 +578,14 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     } else if (merged) {
                         const uint64_t adl = adl0 + (uint64_t)((ks * a_step) >> 4);
-                        mma_tf32_ss(t_main, ad, bd, idesc_w, (!seg_start || ks > 0) ? 1u : 0u);
-                        mma_tf32_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+                        mma_bf16_ss(t_main, ad, bd, idesc_w, (!seg_start || ks > 0) ? 1u : 0u);
+                        mma_bf16_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                     } else {
                         const uint64_t adl = adl0 + (uint64_t)((ks * a_step) >> 4);
                         const uint64_t bdl = bdl0 + (uint64_t)((ks * b_step) >> 4);
-                        mma_tf32_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
-                        mma_tf32_ss(t_corr, ad, bdl, idesc, 1u);
-                        mma_tf32_ss(t_main, ad, bd, idesc, (!seg_start || ks > 0) ? 1u : 0u);
+                        mma_bf16_ss(t_corr, adl, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+                        mma_bf16_ss(t_corr, ad, bdl, idesc, 1u);
+                        mma_bf16_ss(t_main, ad, bd, idesc, (!seg_start || ks > 0) ? 1u : 0u);
                     }
                 }
                 mma_commit(empty(s));
@@ -574,6 +610,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         if constexpr (PRODUCE) {
             const int p = threadIdx.x - 64;
             const T* X = reinterpret_cast<const T*>(a.x);
+            const float sx = F32 ? scales_of(a.amax).x : 1.0f;   // scale of the SiLU values (fp32)
             // Take A slot sa for a k-block: wait until the MMA has consumed its
             // previous contents.  Each thread then zeroes the one 128-byte row it
             // fills (16-byte stores, conflict-free under the swizzle) before it
@@ -583,7 +620,6 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 // rows = batch m0..m0+127.  kGroups groups of 128 threads take
                 // k-blocks in turn; a thread fills one whole row.  Per row and
                 // k-block at most MAXI inputs have columns in the block.
-                constexpr int EPC = 16 / C::ESZ;       // elements per 16-byte chunk
                 const uint32_t row = p & (kBM - 1);
                 const int grp = p >> 7;                // warp-uniform
                 const int64_t b = m0 + row;
@@ -637,7 +673,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                 if (F32 && a.ext) {   // input i0+k's SiLU column, when it falls in this block
                                     const int cs = base + a.nbs;
                                     if (act && (unsigned)cs < (unsigned)BK)
-                                        put1<DT>(ahi + rbase, alo + rbase, rx, cs, silu_f(cur[k]));
+                                        put1<DT>(ahi + rbase, alo + rbase, rx, cs, silu_f(cur[k]) * sx);
                                 }
                                 float u = fmaf(cur[k], a.inv_h, u0);
                                 // outside the extended knots, NaN, inf: no stores
@@ -655,30 +691,29 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                             }
                         }
                     } else {
-                        // SiLU columns: BK consecutive inputs, dense (in*esize % 16 == 0 with the base branch)
-                        const int i0 = (kb - a.nkb_main) * BK;
+                        // SiLU columns: BK consecutive inputs, dense (bf16 only: the fp32
+                        // path carries silu(x) as one more column per input; in * 2 % 16 == 0
+                        // with the base branch)
+                        if constexpr (!F32) {
+                            const int i0 = (kb - a.nkb_main) * BK;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            float v[EPC];
-                            const int ic = i0 + c * EPC;
-                            if (row_ok && ic + EPC <= a.in) {
-                                const uint4 q4 = *reinterpret_cast<const uint4*>(xrow + ic);
-                                const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
+                            for (int c = 0; c < 8; ++c) {
+                                float v[8];
+                                const int ic = i0 + c * 8;
+                                if (row_ok && ic + 8 <= a.in) {
+                                    const uint4 q4 = *reinterpret_cast<const uint4*>(xrow + ic);
+                                    const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-                                for (int e = 0; e < EPC; ++e) {
-                                    float xv;
-                                    if constexpr (F32) {
-                                        xv = __uint_as_float(wd[e]);
-                                    } else {
-                                        xv = __uint_as_float((e & 1) ? (wd[e / 2] & 0xFFFF0000u) : (wd[e / 2] << 16));
-                                    }
-                                    v[e] = silu_f(xv);
+                                    for (int e = 0; e < 8; ++e)
+                                        v[e] = silu_f(__uint_as_float((e & 1) ? (wd[e / 2] & 0xFFFF0000u) : (wd[e / 2] << 16)));
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) v[e] = 0.0f;
                                 }
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < EPC; ++e) v[e] = 0.0f;
+                                put_a_chunk<DT>(ahi, alo, row, (uint32_t)c, v);
                             }
-                            put_a_chunk<DT>(ahi, alo, row, (uint32_t)c, v);
+                        } else {
+                            record_status(a.status, KAN_ERR_DEVICE_CHECK);   // never planned for fp32
                         }
                     }
                     fence_async_smem();
@@ -687,9 +722,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 (void)uses;
             } else if constexpr (MODE == DCA) {
                 // A tile, MN-major: batch rows b0..b0+BK-1 (K) by 128 columns (M) in
-                // 128-byte atoms of EPB columns, BK*128 bytes apart (bf16: two atoms,
-                // 128-byte swizzle; fp32: four atoms, 32-byte-granule swizzle, hi and
-                // lo tiles).  The columns are spline columns kt0.. (or, for a SiLU
+                // two 128-byte atoms of EPB = 64 columns, BK*128 bytes apart, 128-byte
+                // swizzle (fp32: hi and lo tiles).  The columns are spline columns kt0.. (or, for a SiLU
                 // tile, inputs i0..).  Groups of 128 threads take k-blocks in turn; a
                 // thread fills one atom row: (batch row rb, atom).
                 constexpr int NATOM = kBM / EPB;
@@ -712,8 +746,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 };
                 // byte offset of column c (0..EPB-1) inside this thread's atom row
                 auto col_off = [&](int c) -> uint32_t {
-                    if constexpr (F32) return sw128b32_byte((uint32_t)rb, (uint32_t)c * 4u) - (uint32_t)rb * 128u;
-                    else return sw128_byte((uint32_t)rb, (uint32_t)c * 2u) - (uint32_t)rb * 128u;
+                    return sw128_byte((uint32_t)rb, (uint32_t)c * 2u) - (uint32_t)rb * 128u;
                 };
                 float nxt[MAXI];
 #pragma unroll
@@ -745,12 +778,13 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                 if (F32 && a.ext) {   // input i_first+k's SiLU column, when it falls in this atom
                                     const int cs = cbase + k * a.nb + a.nbs;
                                     if (act && (unsigned)cs < (unsigned)EPB) {
-                                        const float v = silu_f(cur[k]);
+                                        const float v = silu_f(cur[k]) * sx;
                                         const uint32_t off = col_off(cs);
                                         if constexpr (F32) {
-                                            const float hi = tf32_hi(v);
-                                            st_shared_f32(rb_hi + off, hi);
-                                            st_shared_f32(rb_lo + off, v - hi);
+                                            uint16_t h, l;
+                                            split_f16(v, h, l);
+                                            st_shared_u16(rb_hi + off, h);
+                                            st_shared_u16(rb_lo + off, l);
                                         } else {
                                             st_shared_u16(rb_hi + off, __bfloat16_as_ushort(__float2bfloat16_rn(v)));
                                         }
@@ -774,9 +808,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                     if ((uint32_t)(sidx + q - mlo) < width) {
                                         const uint32_t off = col_off(col0 + q);
                                         if constexpr (F32) {
-                                            const float hi = tf32_hi(w[q]);
-                                            st_shared_f32(rb_hi + off, hi);
-                                            st_shared_f32(rb_lo + off, w[q] - hi);
+                                            uint16_t h, l;
+                                            split_f16(w[q], h, l);
+                                            st_shared_u16(rb_hi + off, h);
+                                            st_shared_u16(rb_lo + off, l);
                                         } else {
                                             st_shared_u16(rb_hi + off, __bfloat16_as_ushort(__float2bfloat16_rn(w[q])));
                                         }
@@ -786,43 +821,29 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     } else {
                         // SiLU columns: inputs c_lo..c_lo+EPB-1 of batch row b, dense
-                        // (in * esize % 16 == 0 with the base branch)
-                        const T* xr = X + (row_ok ? b : 0) * a.in;
-                        constexpr int EPC = 16 / C::ESZ;
+                        // (bf16 only: the fp32 path carries silu(x) as one more
+                        // column per input; in * 2 % 16 == 0 with the base branch)
+                        if constexpr (!F32) {
+                            const T* xr = X + (row_ok ? b : 0) * a.in;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            float v[EPC];
-                            const int ic = c_lo + c * EPC;
-                            if (row_ok && ic + EPC <= a.in) {
-                                const uint4 q4 = *reinterpret_cast<const uint4*>(xr + ic);
-                                const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
+                            for (int c = 0; c < 8; ++c) {
+                                float v[8];
+                                const int ic = c_lo + c * 8;
+                                if (row_ok && ic + 8 <= a.in) {
+                                    const uint4 q4 = *reinterpret_cast<const uint4*>(xr + ic);
+                                    const uint32_t wd[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-                                for (int e = 0; e < EPC; ++e) {
-                                    float xv;
-                                    if constexpr (F32) xv = __uint_as_float(wd[e]);
-                                    else xv = __uint_as_float((e & 1) ? (wd[e / 2] & 0xFFFF0000u) : (wd[e / 2] << 16));
-                                    v[e] = silu_f(xv);
+                                    for (int e = 0; e < 8; ++e)
+                                        v[e] = silu_f(__uint_as_float((e & 1) ? (wd[e / 2] & 0xFFFF0000u) : (wd[e / 2] << 16)));
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) v[e] = 0.0f;
                                 }
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < EPC; ++e) v[e] = 0.0f;
-                            }
-                            const uint32_t off = col_off(c * EPC);   // a 16-byte chunk never straddles a granule
-                            if constexpr (F32) {
-                                float h[4], l[4];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    h[e] = tf32_hi(v[e]);
-                                    l[e] = v[e] - h[e];
-                                }
-                                st_shared_v4(rb_hi + off, __float_as_uint(h[0]), __float_as_uint(h[1]),
-                                             __float_as_uint(h[2]), __float_as_uint(h[3]));
-                                st_shared_v4(rb_lo + off, __float_as_uint(l[0]), __float_as_uint(l[1]),
-                                             __float_as_uint(l[2]), __float_as_uint(l[3]));
-                            } else {
-                                st_shared_v4(rb_hi + off, pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                st_shared_v4(rb_hi + col_off(c * 8), pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
                                              pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
                             }
+                        } else {
+                            record_status(a.status, KAN_ERR_DEVICE_CHECK);   // never planned for fp32
                         }
                     }
                     fence_async_smem();
@@ -866,9 +887,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     if (merged) tmem_ld16(tm + BN + c0, w);   // the segment's hi*lo half
                     if (g > 0) tmem_ld16(t_total + lane_off + c0, t);
                     tmem_ld_wait();
-                    if (merged) {
+                    if (merged) {   // (the hi*lo half carries the lo parts' 2^11)
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(w[e]));
+                        for (int e = 0; e < 16; ++e)
+                            v[e] = __float_as_uint(fmaf(__uint_as_float(w[e]), kLoInv, __uint_as_float(v[e])));
                     }
                     if (g > 0) {
 #pragma unroll
@@ -884,8 +906,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         if (go) go = __all_sync(0xffffffffu, mbar_wait(accum_bar, 0, a.status));
         if (go) {
             tc_fence_after();
-            // value of accumulator column c0..c0+15 of this thread's row
-            auto load16 = [&](int c0, float (&out)[16]) {
+            // value of accumulator column c0..c0+15 of this thread's row (fp32:
+            // total + corr * 2^-11, times `mul`, the inverse of the operand scales)
+            auto load16 = [&](int c0, float (&out)[16], float mul) {
                 uint32_t v[16];
                 if constexpr (F32) {
                     uint32_t w[16];
@@ -893,8 +916,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     tmem_ld16(t_corr + lane_off + c0, w);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) out[e] = __uint_as_float(v[e]) + __uint_as_float(w[e]);
+                    for (int e = 0; e < 16; ++e)
+                        out[e] = fmaf(__uint_as_float(w[e]), kLoInv, __uint_as_float(v[e])) * mul;
                 } else {
+                    (void)mul;
                     tmem_ld16(t_main0 + lane_off + c0, v);
                     tmem_ld_wait();
 #pragma unroll
@@ -905,9 +930,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             if constexpr (MODE == FWD || MODE == GEMM) {
                 const int64_t bo = m0 + r;
                 const int64_t ncols = MODE == FWD ? a.out_f : a.in;
+                const float mul = F32 ? 1.0f / scales_of(a.amax).c : 1.0f;   // y = acc / s_c
                 for (int c0 = 0; c0 < BN; c0 += 16) {
                     float v[16];
-                    load16(c0, v);
+                    load16(c0, v, mul);
                     if (bo >= a.batch) continue;
                     const int64_t j0 = n0 + c0;
                     if (MODE == GEMM || a.partial) {
@@ -978,9 +1004,19 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     dst = basep ? basep + rowg : nullptr;   // an output the caller skipped
                     ld = base_tile ? a.in : a.Kt;
                 }
+                // fp32: dcoef = acc / s_d, dw_base (the SiLU rows) = acc / (s_d s_x)
+                float mul = 1.0f;
+                if constexpr (F32) {
+                    const Scales sc = scales_of(a.amax);
+                    mul = 1.0f / sc.d;
+                    if (a.ext && row_ok) {
+                        const int ii = (int)__umulhi((uint32_t)rowg, a.nb_magic);
+                        if ((int)rowg - ii * a.nb >= a.nbs) mul /= sc.x;
+                    }
+                }
                 for (int c0 = 0; c0 < BN; c0 += 16) {
                     float v[16];
-                    load16(c0, v);
+                    load16(c0, v, mul);
                     if (!row_ok || !dst) continue;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -996,9 +1032,16 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                (size_t)lane * ldst;
                 for (int c0 = 0; c0 < BN; c0 += 16) {
                     float v[16];
-                    load16(c0, v);
+                    load16(c0, v, 1.0f);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) stage[c0 + e] = v[e];
+                }
+                // fp32: the staged columns are scaled by s_d s_c (spline) and s_d s_c / s_x (SiLU)
+                float inv_dc = 1.0f, ext_mul = 1.0f;
+                if constexpr (F32) {
+                    const Scales sc = scales_of(a.amax);
+                    inv_dc = 1.0f / (sc.d * sc.c);
+                    ext_mul = inv_dc * sc.x;
                 }
                 if (dx_b < a.batch) {
                     const int kt_al = B_MN ? (dx_i0 * a.nb) / (16 / C::ESZ) * (16 / C::ESZ) : dx_i0 * a.nb;
@@ -1028,7 +1071,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                     if (m >= 0 && m < a.nbs) acc += stage[cb + m] * d[qq];
                                 }
                             }
-                            if (F32 && a.ext) acc += dsilu_f(xv) * stage[i * a.nb - kt_al + a.nbs];   // dY.w_base column
+                            acc *= inv_dc;
+                            if (F32 && a.ext) acc += dsilu_f(xv) * stage[i * a.nb - kt_al + a.nbs] * ext_mul;   // dY.w_base
                             else if (a.has_base) acc += dsilu_f(xv) * __uint_as_float(gc[k]);
                             dxr[i] = from_f<T>(acc);
                         }
@@ -1051,7 +1095,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
 // Gm = dY . coef for a tile goes to one of two TMEM accumulators while the
 // epilogue warps turn the previous tile's accumulator into dx, so the B'
 // gather overlaps the next tile's MMA.  Warps: 0 TMA, 1 MMA issue + TMEM,
-// 2-9 epilogue (two per TMEM lane quarter).  fp32 keeps the tf32 correction
+// 2-9 epilogue (two per TMEM lane quarter).  fp32 keeps the fp16 correction
 // products in a second accumulator per buffer; the contraction over `out`
 // is short enough (at most 32 k-blocks) that no promotion is needed.
 // ---------------------------------------------------------------------------
@@ -1069,7 +1113,8 @@ struct DxArgs {
     float lo, inv_h;
     int BN, stages, nkb;      // nkb: k-blocks over out
     int n_in_tile, n_tiles_n, n_tiles;
-    int ld_stage;             // staging row stride in floats (BN + 4)
+    int ld_stage;             // staging row stride in elements
+    const unsigned int* amax; // fp32: absolute maxima of the operands (scales_of)
 };
 
 template <int DT>
@@ -1083,7 +1128,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     constexpr int BK = C::BK;
     constexpr int EPB = 128 / C::ESZ;
     constexpr bool F32 = DT == KAN_F32;
-    constexpr bool B_MN = !F32;          // bf16: coef MN-major; fp32: coef^T K-major
+    constexpr bool B_MN = true;          // coef (its fp16 hi/lo copies for fp32) MN-major
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
 
@@ -1159,8 +1204,11 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     tma_load_2d(A_hi(s), &tA_hi, full(s), kb * BK, (int)m0);
                     if (F32) tma_load_2d(A_lo(s), &tA_lo, full(s), kb * BK, (int)m0);
                     if (B_MN) {
-                        for (int c = 0; c < BN / EPB; ++c)
+                        for (int c = 0; c < BN / EPB; ++c) {
                             tma_load_2d(B_hi(s) + (uint32_t)c * BK * 128, &tB_hi, full(s), kt0 + c * EPB, kb * BK);
+                            if (F32)
+                                tma_load_2d(B_lo(s) + (uint32_t)c * BK * 128, &tB_lo, full(s), kt0 + c * EPB, kb * BK);
+                        }
                     } else {
                         tma_load_2d(B_hi(s), &tB_hi, full(s), kb * BK, kt0);
                         tma_load_2d(B_lo(s), &tB_lo, full(s), kb * BK, kt0);
@@ -1200,9 +1248,9 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         } else {
                             const uint64_t adl = adl0 + (uint64_t)(ks * 2);
                             const uint64_t bdl = bdl0 + (uint64_t)((ks * b_step) >> 4);
-                            mma_tf32_ss(d_corr, adl, bd, idesc, acc);
-                            mma_tf32_ss(d_corr, ad, bdl, idesc, 1u);
-                            mma_tf32_ss(d_main, ad, bd, idesc, acc);
+                            mma_bf16_ss(d_corr, adl, bd, idesc, acc);
+                            mma_bf16_ss(d_corr, ad, bdl, idesc, 1u);
+                            mma_bf16_ss(d_main, ad, bd, idesc, acc);
                         }
                     }
                     mma_commit(empty(s));
@@ -1225,6 +1273,13 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         constexpr int XC = 16;
         const bool x_vec = (a.in * (int64_t)sizeof(T)) % 16 == 0;
         const bool g_vec = (a.in * 4) % 16 == 0;
+        // fp32: the staged columns carry s_d s_c (spline) and s_d s_c / s_x (SiLU)
+        float inv_dc = 1.0f, ext_mul = 1.0f;
+        if constexpr (F32) {
+            const Scales sc = scales_of(a.amax);
+            inv_dc = 1.0f / (sc.d * sc.c);
+            ext_mul = inv_dc * sc.x;
+        }
         for (int lt = 0; lt < my_tiles; ++lt) {
             int64_t m0;
             int i0;
@@ -1266,12 +1321,13 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             for (int c0 = h * half_cols; c0 < (h + 1) * half_cols; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld16(t_main + c0, v);
-                if constexpr (F32) {
+                if constexpr (F32) {   // main + corr * 2^-11
                     uint32_t w[16];
                     tmem_ld16(t_main + BN + c0, w);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(w[e]));
+                    for (int e = 0; e < 16; ++e)
+                        v[e] = __float_as_uint(fmaf(__uint_as_float(w[e]), kLoInv, __uint_as_float(v[e])));
                 } else {
                     tmem_ld_wait();
                 }
@@ -1318,7 +1374,8 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                                 if (m >= 0 && m < a.nbs) acc += to_f(srow[cb + m]) * d[qq];
                             }
                         }
-                        if (F32 && a.ext) acc += dsilu_f(xv) * to_f(srow[i * a.nb - kt_al + a.nbs]);   // dY.w_base, staged
+                        acc *= inv_dc;
+                        if (F32 && a.ext) acc += dsilu_f(xv) * to_f(srow[i * a.nb - kt_al + a.nbs]) * ext_mul;   // dY.w_base, staged
                         else if (a.gb) acc += dsilu_f(xv) * gc[k];
                         return acc;
                     };
@@ -1398,87 +1455,58 @@ __global__ void reduce_dcoef_kernel(const float* __restrict__ part, float* __res
     }
 }
 
-// hi/lo tf32 split of an fp32 array.
-__global__ void split_tf32_kernel(const float* __restrict__ src, float* __restrict__ hi, float* __restrict__ lo,
-                                  int64_t n)
+// Absolute maxima of up to four fp32 arrays (amax[k] over src[k][0..n[k]),
+// NaN ignored) as the bit patterns of non-negative floats, combined with
+// atomicMax: the maximum does not depend on the order, so the result is
+// deterministic.  amax must start at 0.
+struct AmaxArgs {
+    const float* src[4];
+    int64_t n[4];
+};
+__global__ void absmax_kernel(AmaxArgs a, unsigned int* __restrict__ amax)
 {
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        const float v = src[e];
-        const float h = tf32_hi(v);
-        hi[e] = h;
-        lo[e] = v - h;
-    }
-}
-
-// hi/lo tf32 split of a row-major fp32 [R, C] matrix, written transposed:
-// hi[c * ldo + r], lo[c * ldo + r] (ldo >= R), through a 32x32 shared tile.
-__global__ void split_tf32_t_kernel(const float* __restrict__ src, int64_t R, int64_t C, float* __restrict__ hi,
-                                    float* __restrict__ lo, int64_t ldo)
-{
-    __shared__ float tile[32][33];
-    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
-    for (int k = threadIdx.y; k < 32; k += blockDim.y) {
-        const int64_t r = r0 + k, c = c0 + threadIdx.x;
-        tile[k][threadIdx.x] = (r < R && c < C) ? src[r * C + c] : 0.0f;
+    __shared__ unsigned int red[4];
+    if (threadIdx.x < 4) red[threadIdx.x] = 0u;
+    __syncthreads();
+    for (int k = 0; k < 4; ++k) {
+        if (!a.src[k]) continue;
+        float m = 0.0f;
+        const int64_t n = a.n[k];
+        const float* __restrict__ src = a.src[k];
+        for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+            m = fmaxf(m, fabsf(src[e]));
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((threadIdx.x & 31) == 0) atomicMax(&red[k], __float_as_uint(m));
     }
     __syncthreads();
-    for (int k = threadIdx.y; k < 32; k += blockDim.y) {
-        const int64_t c = c0 + k, r = r0 + threadIdx.x;
-        if (c < C && r < R) {
-            const float v = tile[threadIdx.x][k];
-            const float h = tf32_hi(v);
-            hi[c * ldo + r] = h;
-            lo[c * ldo + r] = v - h;
-        }
-    }
+    if (threadIdx.x < 4 && a.src[threadIdx.x]) atomicMax(&amax[threadIdx.x], red[threadIdx.x]);
 }
 
-// Value of the fp32 coefficient matrix with each input's SiLU weight
-// interleaved: row j, column i*nbx + m is coef[j, i, m] for m < nbs and
-// w_base[j, i] for m == nbs.
-__device__ __forceinline__ float ext_coef(const float* __restrict__ coef, const float* __restrict__ w_base,
-                                          int64_t in, int nbs, int nbx, int64_t j, int64_t c)
+// fp16 hi/lo split of an fp32 array, times the dY scale (amax slot 3).
+__global__ void split_f16_kernel(const float* __restrict__ src, uint16_t* __restrict__ hi, uint16_t* __restrict__ lo,
+                                 int64_t n, const unsigned int* __restrict__ amax)
 {
-    const int64_t i = c / nbx;
-    const int m = (int)(c - i * nbx);
-    return m < nbs ? coef[(j * in + i) * nbs + m] : w_base[j * in + i];
+    const float sc = scales_of(amax).d;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+        split_f16(src[e] * sc, hi[e], lo[e]);
 }
 
-// tf32 hi/lo copies of the interleaved matrix, row-major [out][in*nbx].
-__global__ void split_ext_kernel(const float* __restrict__ coef, const float* __restrict__ w_base, int64_t out,
-                                 int64_t in, int nbs, int nbx, float* __restrict__ hi, float* __restrict__ lo)
+// fp16 hi/lo split of the coefficient matrix, row-major [out][in*nbx]:
+// column i*nbx + m is coef[j, i, m] * s_c for m < nbs, and (with the SiLU
+// branch, nbx = nbs + 1) w_base[j, i] * s_c / s_x for m == nbs.
+__global__ void split_coef_f16_kernel(const float* __restrict__ coef, const float* __restrict__ w_base, int64_t out,
+                                      int64_t in, int nbs, int nbx, uint16_t* __restrict__ hi, uint16_t* __restrict__ lo,
+                                      const unsigned int* __restrict__ amax)
 {
+    const Scales sc = scales_of(amax);
+    const float sw = sc.c / sc.x;
     const int64_t Kx = in * nbx, n = out * Kx;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t j = e / Kx;
-        const float v = ext_coef(coef, w_base, in, nbs, nbx, j, e - j * Kx);
-        const float h = tf32_hi(v);
-        hi[e] = h;
-        lo[e] = v - h;
-    }
-}
-
-// The same, transposed: hi[c * ldo + j] (ldo >= out), through a 32x32 shared tile.
-__global__ void split_ext_t_kernel(const float* __restrict__ coef, const float* __restrict__ w_base, int64_t out,
-                                   int64_t in, int nbs, int nbx, float* __restrict__ hi, float* __restrict__ lo,
-                                   int64_t ldo)
-{
-    __shared__ float tile[32][33];
-    const int64_t Kx = in * nbx;
-    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
-    for (int k = threadIdx.y; k < 32; k += blockDim.y) {
-        const int64_t r = r0 + k, c = c0 + threadIdx.x;
-        tile[k][threadIdx.x] = (r < out && c < Kx) ? ext_coef(coef, w_base, in, nbs, nbx, r, c) : 0.0f;
-    }
-    __syncthreads();
-    for (int k = threadIdx.y; k < 32; k += blockDim.y) {
-        const int64_t c = c0 + k, r = r0 + threadIdx.x;
-        if (c < Kx && r < out) {
-            const float v = tile[threadIdx.x][k];
-            const float h = tf32_hi(v);
-            hi[c * ldo + r] = h;
-            lo[c * ldo + r] = v - h;
-        }
+        const int64_t j = e / Kx, c = e - j * Kx;
+        const int64_t i = c / nbx;
+        const int m = (int)(c - i * nbx);
+        const float v = m < nbs ? coef[(j * in + i) * nbs + m] * sc.c : w_base[j * in + i] * sw;
+        split_f16(v, hi[e], lo[e]);
     }
 }
 
@@ -1499,9 +1527,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
     return fn;
 }
 
-// 2-D tiled map over a row-major [rows, cols] matrix; box = [box_rows, box_cols]
-// with box_cols * esize = 128 bytes, 128-byte swizzle, zero fill out of bounds.
-bool make_map_2d(CUtensorMap* m, const void* base, bool f32, int64_t rows, int64_t cols, int box_rows, int box_cols,
+// 2-D tiled map over a row-major [rows, cols] matrix of 2-byte operand
+// elements (bf16, or the fp16 split copies of the fp32 path); box =
+// [box_rows, box_cols] with box_cols * 2 = 128 bytes, 128-byte swizzle, zero
+// fill out of bounds.
+bool make_map_2d(CUtensorMap* m, const void* base, bool f16, int64_t rows, int64_t cols, int box_rows, int box_cols,
                  const char** detail, int64_t ld = -1)
 {
     auto enc = get_encoder();
@@ -1509,12 +1539,12 @@ bool make_map_2d(CUtensorMap* m, const void* base, bool f32, int64_t rows, int64
         *detail = "cuTensorMapEncodeTiled is not available from the driver";
         return false;
     }
-    const int esz = f32 ? 4 : 2;
+    const int esz = 2;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)((ld > 0 ? ld : cols) * esz)};
     cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+    CUresult r = enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -1527,30 +1557,46 @@ bool make_map_2d(CUtensorMap* m, const void* base, bool f32, int64_t rows, int64
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// Split-K count: only when the tiles do not fill one wave.  Then the split
-// that minimises ceil(tiles*s / sms) / s (waves per unit of work), with a small
-// price per extra split for the fp32 partial sums it writes and reduces.
-int pick_splits(int64_t tiles, int sms, int cap)
+// Split-K count s (1..cap) minimising the estimated time
+//   waves(s) / s * t_tile  +  waves(s) * t_wave  +  (s > 1 ? 2 (s + 1) t_part : 0),
+// waves(s) = ceil(tiles * s / sms); t_tile: one whole output tile's contraction
+// on one SM; t_wave: the fixed cost of a wave of CTAs (set-up, pipeline fill,
+// epilogue); t_part: writing one set of fp32 partials for every tile (the
+// reduction reads them back and launches once more, hence the factor 2).
+// Splitting evens out a ragged last wave; it is taken only when the estimate
+// improves on the unsplit one by at least 10%.
+int pick_splits(int64_t tiles, int sms, int cap, double t_tile, double t_part)
 {
-    if (tiles >= sms) return 1;
+    constexpr double t_wave = 4.0e-6;
+    auto cost = [&](int s) {
+        const double waves = (double)cdiv(tiles * s, sms);
+        return waves / s * t_tile + waves * t_wave + (s > 1 ? 2.0 * (s + 1) * t_part : 0.0);
+    };
+    const double c1 = cost(1);
     int best = 1;
-    double best_cost = 1e30;
-    for (int s = 1; s <= std::max(1, cap); ++s) {
-        const double cost = (double)cdiv(tiles * s, sms) / s + 0.02 * (s - 1);
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
+    double best_cost = c1;
+    for (int s = 2; s <= std::max(1, cap); ++s) {
+        const double c = cost(s);
+        if (c < best_cost * (1.0 - 1e-9) && c < 0.9 * c1) {
+            best_cost = c;
             best = s;
         }
     }
     return best;
 }
 
+// Seconds for one tile of BN output columns over K contraction elements on one
+// SM (dense tensor rate; fp32 runs 3 fp16 products), and for writing one set of
+// fp32 partials of `tiles` such tiles at HBM rate.
+double tile_seconds(int BN, int64_t K, bool f32) { return 2.0 * kBM * BN * (double)K * (f32 ? 3 : 1) / 9.0e12; }
+double partial_seconds(int64_t tiles, int BN) { return (double)tiles * kBM * BN * 4.0 / 5.0e12; }
+
 // Tile width over n output columns.  An MN-major bf16 B operand is loaded in
 // 64-column (128-byte) boxes, so its tile is at least one box wide.
 int bn_for(int64_t n, bool f32, bool mn_major = false)
 {
     const int cap = f32 ? 128 : 256;
-    int bn = (mn_major && !f32) ? 64 : 32;
+    int bn = mn_major ? 64 : 32;
     while (bn < n && bn < cap) bn *= 2;
     return bn;
 }
@@ -1603,8 +1649,8 @@ int smem_bytes(int BN, int stages, int stages_a, bool f32)
 
 // Workspace layout, shared by the size query and the launches.
 struct Layout {
-    size_t coef_hl = 0, wb_hl = 0, dy_hl = 0;   // tf32 hi/lo copies (fp32 only)
-    size_t dyt_hl = 0;                           // tf32 hi/lo of dY^T [out][ldb] (fp32 backward)
+    size_t amax = 0;                             // fp32: 4 absolute maxima (the operand scales)
+    size_t coef_hl = 0, dy_hl = 0;               // fp32: fp16 hi/lo copies of coef (w_base interleaved), dY
     size_t fwd_part = 0, dc_part = 0, gb = 0;   // split partials and dY.w_base
     size_t total = 0;
 };
@@ -1620,7 +1666,6 @@ struct Plan {
     // dcoef
     int d_BN, d_stages, d_stages_a, d_n, d_m, d_nkt, d_splits, d_kps, d_nkb;
     int64_t d_ld;
-    int64_t ldb;   // padded row length of dY^T (fp32)
     // dx
     int x_BN, x_stages, x_n, x_m, x_nin, x_nkb;
     // dx, persistent kernel (used when p_ok)
@@ -1635,8 +1680,7 @@ Plan make_plan(const Problem& p, int sms)
 {
     Plan P{};
     const bool f32 = p.dtype == KAN_F32;
-    const int BK = f32 ? 32 : 64;
-    const size_t esz = f32 ? 4 : 2;
+    const int BK = 64;   // K elements per 128-byte operand row (2-byte operands, both dtypes)
     P.ext = f32 && p.base;
     P.nbx = p.nb + (P.ext ? 1 : 0);
     P.Kx = p.in * P.nbx;
@@ -1648,7 +1692,11 @@ Plan make_plan(const Problem& p, int sms)
     P.f_m = (int)cdiv(p.batch, kBM);
     P.f_nkb_main = (int)cdiv(P.Kx, BK);
     P.f_nkb_total = P.f_nkb_main + (sep_silu ? (int)cdiv(p.in, BK) : 0);
-    P.f_splits = pick_splits((int64_t)P.f_n * P.f_m, sms, std::min(16, std::max(1, P.f_nkb_total / 8)));
+    {
+        const int64_t tiles = (int64_t)P.f_n * P.f_m;
+        P.f_splits = pick_splits(tiles, sms, std::min(16, std::max(1, P.f_nkb_total / 8)),
+                                 tile_seconds(P.f_BN, (int64_t)P.f_nkb_total * BK, f32), partial_seconds(tiles, P.f_BN));
+    }
     P.f_kps = (int)cdiv(P.f_nkb_total, P.f_splits);
     P.f_splits = (int)cdiv(P.f_nkb_total, P.f_kps);
     // dcoef: M = spline columns (+ SiLU rows), N = out, K = batch
@@ -1658,30 +1706,33 @@ Plan make_plan(const Problem& p, int sms)
     P.d_m = P.d_nkt + (sep_silu ? (int)cdiv(p.in, kBM) : 0);
     stages_ab(P.d_BN, f32, P.d_stages, P.d_stages_a);
     P.d_nkb = (int)cdiv(p.batch, BK);
-    P.d_splits = pick_splits((int64_t)P.d_n * P.d_m, sms, std::min(16, std::max(1, P.d_nkb / 8)));
+    {
+        const int64_t tiles = (int64_t)P.d_n * P.d_m;
+        P.d_splits = pick_splits(tiles, sms, std::min(16, std::max(1, P.d_nkb / 8)),
+                                 tile_seconds(P.d_BN, (int64_t)P.d_nkb * BK, f32), partial_seconds(tiles, P.d_BN));
+    }
     P.d_kps = (int)cdiv(std::max(1, P.d_nkb), P.d_splits);
     P.d_splits = (int)cdiv(std::max(1, P.d_nkb), P.d_kps);
     P.d_ld = P.ext ? P.Kx : p.Kt + (p.base ? p.in : 0);
-    // dx: M = batch, N = whole inputs' spline columns, K = out
+    // dx: M = batch, N = whole inputs' columns, K = out; coef (or its fp16
+    // copies) is read MN-major and a tile's first column is rounded down to 16 bytes
     P.x_BN = f32 ? 128 : 256;
     P.x_stages = stages_for(P.x_BN, f32);
-    // bf16: coef is read MN-major and a tile's first column is rounded down to
-    // 16 bytes; fp32: coef^T is read K-major, any first row works
-    const int maxoff = f32 ? 0 : ((p.nb % 8 == 0) ? 0 : 7);
+    const int maxoff = (P.nbx % 8 == 0) ? 0 : 7;
     P.x_nin = std::max(1, (P.x_BN - maxoff) / P.nbx);
     P.x_n = (int)cdiv(p.in, P.x_nin);
     P.x_m = (int)cdiv(p.batch, kBM);
     P.x_nkb = (int)cdiv(p.out, BK);
-    // dx, persistent: BN 192 (bf16) / 128 (fp32), double-buffered TMEM, staged epilogue
+    // dx, persistent: BN 256 (bf16) / 128 (fp32), double-buffered TMEM, staged epilogue;
+    // fp32 accumulates over `out` without promotion, so at most 1024 terms
     {
         P.p_BN = f32 ? 128 : 256;
-        const int pmaxoff = f32 ? 0 : ((p.nb % 8 == 0) ? 0 : 7);
-        P.p_nin = (P.p_BN - pmaxoff) / P.nbx;
+        P.p_nin = (P.p_BN - maxoff) / P.nbx;
         P.p_ld = f32 ? P.p_BN + 4 : P.p_BN + 8;          // row stride = 16 bytes mod 128
         const int staging = 4 * 32 * P.p_ld * (f32 ? 4 : 2);
         const int stage_bytes = (kBM * 128 + P.p_BN * 128) * (f32 ? 2 : 1);
         P.p_stages = std::min(6, (232448 - 1024 - 256 - staging) / stage_bytes);
-        P.p_ok = P.p_nin >= 1 && P.p_stages >= 2 && (!f32 || P.x_nkb <= 32);
+        P.p_ok = P.p_nin >= 1 && P.p_stages >= 2 && (!f32 || p.out <= 1024);
         if (P.p_ok) {
             P.p_ntn = (int)cdiv(p.in, P.p_nin);
             P.p_tiles = P.p_ntn * P.x_m;
@@ -1689,41 +1740,34 @@ Plan make_plan(const Problem& p, int sms)
             P.p_smem = P.p_stages * stage_bytes + staging + 1024 + 256;
         }
     }
-    // dY . w_base: M = batch, N = in, K = out
+    // dY . w_base (bf16 with the SiLU branch): M = batch, N = in, K = out
     P.g_BN = bn_for(p.in, f32, true);
     P.g_stages = stages_for(P.g_BN, f32);
     P.g_n = (int)cdiv(p.in, P.g_BN);
     P.g_m = P.x_m;
 
-    // workspace, forward
+    // workspace, forward (fp32: maxima, fp16 hi/lo copy of coef with w_base interleaved)
     size_t o = 0;
     if (f32) {
+        P.fwd.amax = o;
+        o += 256;
         P.fwd.coef_hl = o;
-        o += 2 * al256((size_t)p.out * P.Kx * 4);
-        if (sep_silu) {
-            P.fwd.wb_hl = o;
-            o += 2 * al256((size_t)p.out * p.in * 4);
-        }
+        o += 2 * al256((size_t)p.out * P.Kx * 2);
     }
     if (P.f_splits > 1) {
         P.fwd.fwd_part = o;
         o += al256((size_t)P.f_splits * p.batch * p.out * 4);
     }
     P.fwd.total = o;
-    // workspace, backward (fp32: coef^T, w_base^T, dY and dY^T as tf32 hi/lo)
+    // workspace, backward (fp32: maxima, fp16 hi/lo copies of dY and of coef)
     o = 0;
-    P.ldb = (p.batch + 3) / 4 * 4;
     if (f32) {
+        P.bwd.amax = o;
+        o += 256;
         P.bwd.coef_hl = o;
-        o += 2 * al256((size_t)p.out * P.Kx * 4);
-        if (sep_silu) {
-            P.bwd.wb_hl = o;
-            o += 2 * al256((size_t)p.out * p.in * 4);
-        }
+        o += 2 * al256((size_t)p.out * P.Kx * 2);
         P.bwd.dy_hl = o;
-        o += 2 * al256((size_t)p.batch * p.out * 4);
-        P.bwd.dyt_hl = o;
-        o += 2 * al256((size_t)p.out * P.ldb * 4);
+        o += 2 * al256((size_t)p.batch * p.out * 2);
     }
     if (P.d_splits > 1) {
         P.bwd.dc_part = o;
@@ -1734,7 +1778,6 @@ Plan make_plan(const Problem& p, int sms)
         o += al256((size_t)p.batch * p.in * 4);
     }
     P.bwd.total = o;
-    (void)esz;
     return P;
 }
 
@@ -1746,7 +1789,7 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
     constexpr bool produce = MODE == FWD || MODE == DCA;
     const int stages_a = produce ? args.stages_a : stages;
     // the MN-major bf16 B operand arrives in whole 128-byte boxes: BN must be a multiple of 64
-    if (MODE != FWD && DT == KAN_BF16 && BN % 64 != 0) return cudaErrorInvalidConfiguration;
+    if (MODE != FWD && BN % 64 != 0) return cudaErrorInvalidConfiguration;
     if (BN % 16 != 0 || BN < 16 || BN > (MODE == FWD || MODE == DCA ? 512 : 256) || (BN > 256 && BN % 128 != 0) ||
         (DT == KAN_F32 && BN > 128) || stages < 2 || stages_a < 2 || stages + stages_a > 24 ||
         (!produce && stages_a != stages))
@@ -1767,7 +1810,7 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
 }
 
 // Inputs a row of one forward k-block can touch: (BK - 1) / nb + 2.
-int fwd_maxi_needed(int nb, bool f32) { return ((f32 ? 32 : 64) - 1) / nb + 2; }
+int fwd_maxi_needed(int nb, bool f32) { return (64 - 1) / nb + 2; (void)f32; }
 
 template <int MODE>
 cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
@@ -1827,47 +1870,52 @@ TcArgs base_args(const Problem& p, const Plan& P)
     return a;
 }
 
-// tf32 hi/lo copies of an fp32 array; returns the (hi, lo) pointers.
-cudaError_t split_into(const void* src, int64_t n, uint8_t* dst, const void** hi, const void** lo, cudaStream_t st)
+// fp32 path: the absolute maxima of coef, w_base, x (with the SiLU branch) and
+// dY (any may be null) into amax[0..3], the source of the operand scales.
+cudaError_t amax_into(const Problem& p, const void* coef, const void* w_base, const void* x, const void* dY,
+                      unsigned int* amax, cudaStream_t st)
 {
-    float* h = reinterpret_cast<float*>(dst);
-    float* l = reinterpret_cast<float*>(dst + al256((size_t)n * 4));
-    split_tf32_kernel<<<grid_for(n), 256, 0, st>>>((const float*)src, h, l, n);
+    cudaError_t e = cudaMemsetAsync(amax, 0, 4 * sizeof(unsigned int), st);
+    if (e != cudaSuccess) return e;
+    AmaxArgs a{};
+    a.src[0] = (const float*)coef;
+    a.n[0] = p.out * p.Kt;
+    a.src[1] = p.base ? (const float*)w_base : nullptr;
+    a.n[1] = p.out * p.in;
+    a.src[2] = p.base ? (const float*)x : nullptr;
+    a.n[2] = p.batch * p.in;
+    a.src[3] = (const float*)dY;
+    a.n[3] = p.batch * p.out;
+    int64_t nmax = 0;
+    for (int k = 0; k < 4; ++k)
+        if (a.src[k]) nmax = std::max(nmax, a.n[k]);
+    absmax_kernel<<<grid_for(nmax), 256, 0, st>>>(a, amax);
+    count_launch();
+    return cudaGetLastError();
+}
+
+// fp16 hi/lo copies of coef (w_base interleaved), [out][Kx]; returns the (hi, lo) pointers.
+cudaError_t split_coef_into(const Problem& p, const Plan& P, const void* coef, const void* w_base, uint8_t* dst,
+                            const unsigned int* amax, const void** hi, const void** lo, cudaStream_t st)
+{
+    uint16_t* h = reinterpret_cast<uint16_t*>(dst);
+    uint16_t* l = reinterpret_cast<uint16_t*>(dst + al256((size_t)p.out * P.Kx * 2));
+    split_coef_f16_kernel<<<grid_for(p.out * P.Kx), 256, 0, st>>>((const float*)coef, (const float*)w_base, p.out,
+                                                                 p.in, p.nb, P.nbx, h, l, amax);
     count_launch();
     *hi = h;
     *lo = l;
     return cudaGetLastError();
 }
 
-// tf32 hi/lo copies of a row-major [R, C] fp32 matrix, transposed to [C][ldo].
-cudaError_t split_t_into(const void* src, int64_t R, int64_t C, int64_t ldo, uint8_t* dst, const void** hi,
-                         const void** lo, cudaStream_t st)
+// fp16 hi/lo copies of dY, [batch][out]; returns the (hi, lo) pointers.
+cudaError_t split_dy_into(const Problem& p, const void* dY, uint8_t* dst, const unsigned int* amax, const void** hi,
+                          const void** lo, cudaStream_t st)
 {
-    float* h = reinterpret_cast<float*>(dst);
-    float* l = reinterpret_cast<float*>(dst + al256((size_t)C * ldo * 4));
-    dim3 grid((unsigned)cdiv(C, 32), (unsigned)cdiv(R, 32));
-    split_tf32_t_kernel<<<grid, dim3(32, 8), 0, st>>>((const float*)src, R, C, h, l, ldo);
-    count_launch();
-    *hi = h;
-    *lo = l;
-    return cudaGetLastError();
-}
-
-// tf32 hi/lo copies of coef with w_base interleaved, [out][Kx] (or transposed
-// to [Kx][ldo]); returns the (hi, lo) pointers.
-cudaError_t split_ext_into(const Problem& p, const Plan& P, const void* coef, const void* w_base, bool transposed,
-                           int64_t ldo, uint8_t* dst, const void** hi, const void** lo, cudaStream_t st)
-{
-    float* h = reinterpret_cast<float*>(dst);
-    float* l = reinterpret_cast<float*>(dst + al256((size_t)p.out * P.Kx * 4));
-    if (transposed) {
-        dim3 grid((unsigned)cdiv(P.Kx, 32), (unsigned)cdiv(p.out, 32));
-        split_ext_t_kernel<<<grid, dim3(32, 8), 0, st>>>((const float*)coef, (const float*)w_base, p.out, p.in, p.nb,
-                                                          P.nbx, h, l, ldo);
-    } else {
-        split_ext_kernel<<<grid_for(p.out * P.Kx), 256, 0, st>>>((const float*)coef, (const float*)w_base, p.out, p.in,
-                                                                 p.nb, P.nbx, h, l);
-    }
+    const int64_t n = p.batch * p.out;
+    uint16_t* h = reinterpret_cast<uint16_t*>(dst);
+    uint16_t* l = reinterpret_cast<uint16_t*>(dst + al256((size_t)n * 2));
+    split_f16_kernel<<<grid_for(n), 256, 0, st>>>((const float*)dY, h, l, n, amax);
     count_launch();
     *hi = h;
     *lo = l;
@@ -1878,25 +1926,28 @@ cudaError_t split_ext_into(const Problem& p, const Plan& P, const void* coef, co
 
 bool tc_supported(const Problem& p, bool backward, const char** why)
 {
-    const int esz = p.dtype == KAN_F32 ? 4 : 2;
-    if ((p.Kt * esz) % 16 != 0) {
-        *why = "in*(G+3)*sizeof(dtype) is not a multiple of 16 bytes (TMA row stride of coef)";
+    // Every tensor-core operand is 2 bytes wide: bf16 data as it is, or the fp16
+    // hi/lo copies of fp32 data (coef with w_base interleaved: G+4 columns per input).
+    const bool f32 = p.dtype == KAN_F32;
+    const int64_t nbx = p.nb + ((f32 && p.base) ? 1 : 0);
+    if ((p.in * nbx * 2) % 16 != 0) {
+        *why = f32 ? "in*(G+3) (in*(G+4) with the SiLU branch) is not a multiple of 8 (TMA row stride of the "
+                     "coefficient operand)"
+                   : "in*(G+3)*2 is not a multiple of 16 bytes (TMA row stride of coef)";
         return false;
     }
-    if (p.base && (p.in * esz) % 16 != 0) {
-        *why = "in*sizeof(dtype) is not a multiple of 16 bytes (TMA row stride of w_base)";
+    if (!f32 && p.base && (p.in * 2) % 16 != 0) {
+        *why = "in*2 is not a multiple of 16 bytes (TMA row stride of w_base)";
         return false;
     }
-    if ((p.out * esz) % 16 != 0) {
-        *why = "out*sizeof(dtype) is not a multiple of 16 bytes (TMA row stride of dY, vector stores of y)";
+    if ((p.out * 2) % 16 != 0) {
+        *why = "out is not a multiple of 8 (TMA row stride of the dY operand, vector stores of y)";
         return false;
     }
-    if (p.nb > (p.dtype == KAN_F32 ? 125 : 249)) {
-        *why = "G too large for one dx tile (G+3 must fit the tile with its alignment offset)";
+    if (nbx > 121 && (f32 || nbx > 249)) {
+        *why = "G too large for one dx tile (the input's columns must fit the tile with its alignment offset)";
         return false;
     }
-    // (with the SiLU branch the fp32 copies have G+4 columns per input)
-    const int64_t nbx = p.nb + ((p.dtype == KAN_F32 && p.base) ? 1 : 0);
     if (p.Kt + p.in > ((int64_t)1 << 30) || p.in * nbx >= (((int64_t)1 << 32) / nbx) ||
         p.batch > ((int64_t)1 << 31) - 256 ||
         p.out > ((int64_t)1 << 30)) {
@@ -1915,17 +1966,16 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
 {
     if (p.batch == 0) return cudaSuccess;
     const bool f32 = p.dtype == KAN_F32;
-    const int BK = f32 ? 32 : 64;
+    const int BK = 64;
     const Plan P = make_plan(p, num_sms);
     uint8_t* w = reinterpret_cast<uint8_t*>(ws);
     const void *c_hi = coef, *c_lo = coef, *wb_hi = w_base, *wb_lo = w_base;
+    unsigned int* amax = f32 ? reinterpret_cast<unsigned int*>(w + P.fwd.amax) : nullptr;
     cudaError_t e;
-    if (P.ext) {
-        if ((e = split_ext_into(p, P, coef, w_base, false, 0, w + P.fwd.coef_hl, &c_hi, &c_lo, st)) != cudaSuccess)
-            return e;
-    } else if (f32) {
-        if ((e = split_into(coef, p.out * p.Kt, w + P.fwd.coef_hl, &c_hi, &c_lo, st)) != cudaSuccess) return e;
-        if (p.base && (e = split_into(w_base, p.out * p.in, w + P.fwd.wb_hl, &wb_hi, &wb_lo, st)) != cudaSuccess)
+    if (f32) {
+        // operand scales, then the fp16 hi/lo copy of coef (w_base interleaved)
+        if ((e = amax_into(p, coef, w_base, x, nullptr, amax, st)) != cudaSuccess) return e;
+        if ((e = split_coef_into(p, P, coef, w_base, w + P.fwd.coef_hl, amax, &c_hi, &c_lo, st)) != cudaSuccess)
             return e;
     }
     CUtensorMap maps[6];
@@ -1945,6 +1995,7 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
     maps[1] = maps[3];
     TcArgs a = base_args(p, P);
     a.x = x;
+    a.amax = amax;
     a.out = P.f_splits > 1 ? (void*)(w + P.fwd.fwd_part) : y;
     a.BN = P.f_BN;
     a.stages = P.f_stages;
@@ -1976,8 +2027,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
                         const char** detail)
 {
     const bool f32 = p.dtype == KAN_F32;
-    const int BK = f32 ? 32 : 64;
-    const int EPB = f32 ? 32 : 64;
+    const int BK = 64, EPB = 64;
     const Plan P = make_plan(p, num_sms);
     uint8_t* w = reinterpret_cast<uint8_t*>(ws);
     cudaError_t e;
@@ -1986,24 +2036,28 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         if (dw_base && (e = zero_f32(dw_base, p.out * p.in, st)) != cudaSuccess) return e;
         return cudaSuccess;
     }
-    // ---- dcoef / dw_base: A = basis^T (producers), B = dY (bf16: MN-major; fp32: dY^T K-major) ----
+    unsigned int* amax = f32 ? reinterpret_cast<unsigned int*>(w + P.bwd.amax) : nullptr;
+    const void *dy_hi = dY, *dy_lo = dY;
+    if (f32) {
+        // operand scales (coef and w_base for dx's coefficient copy, x for the
+        // SiLU values, dY), then dY's fp16 hi/lo copy, shared by dcoef and dx
+        if ((e = amax_into(p, coef, w_base, x, dY, amax, st)) != cudaSuccess) return e;
+        if ((e = split_dy_into(p, dY, w + P.bwd.dy_hl, amax, &dy_hi, &dy_lo, st)) != cudaSuccess) return e;
+    }
+    // ---- dcoef / dw_base: A = basis^T (producers), B = dY MN-major (BK-batch x 64-output boxes) ----
     if (dcoef || dw_base) {
         CUtensorMap maps[6];
+        if (!make_map_2d(&maps[2], dy_hi, f32, p.batch, p.out, BK, EPB, detail)) return cudaErrorInvalidValue;
         if (f32) {
-            const void *th, *tl;
-            if ((e = split_t_into(dY, p.batch, p.out, P.ldb, w + P.bwd.dyt_hl, &th, &tl, st)) != cudaSuccess)
-                return e;
-            if (!make_map_2d(&maps[2], th, true, p.out, p.batch, P.d_BN, BK, detail, P.ldb) ||
-                !make_map_2d(&maps[3], tl, true, p.out, p.batch, P.d_BN, BK, detail, P.ldb))
-                return cudaErrorInvalidValue;
-            maps[0] = maps[1] = maps[4] = maps[5] = maps[2];
+            if (!make_map_2d(&maps[3], dy_lo, true, p.batch, p.out, BK, EPB, detail)) return cudaErrorInvalidValue;
         } else {
-            // dY as the MN-major B operand: BK-batch x 64-output boxes
-            if (!make_map_2d(&maps[2], dY, false, p.batch, p.out, BK, EPB, detail)) return cudaErrorInvalidValue;
-            maps[0] = maps[1] = maps[3] = maps[4] = maps[5] = maps[2];
+            maps[3] = maps[2];
         }
+        maps[0] = maps[4] = maps[2];
+        maps[1] = maps[5] = maps[3];
         TcArgs a = base_args(p, P);
         a.x = x;
+        a.amax = amax;
         float* partbuf = reinterpret_cast<float*>(w + P.bwd.dc_part);
         a.BN = P.d_BN;
         a.stages = P.d_stages;
@@ -2026,32 +2080,18 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
     }
-    // ---- dx: A = dY (K-major), B = coef (bf16: MN-major; fp32: coef^T K-major) ----
+    // ---- dx: A = dY K-major, B = coef MN-major (fp32: their fp16 hi/lo copies) ----
     if (dx) {
-        const void *dy_hi = dY, *dy_lo = dY;
-        if (f32 && (e = split_into(dY, p.batch * p.out, w + P.bwd.dy_hl, &dy_hi, &dy_lo, st)) != cudaSuccess)
-            return e;
         float* gb = nullptr;
         if (p.base && !P.ext) {
-            // Gb = dY . w_base (fp32 [batch, in]) for the SiLU term of dx
+            // bf16: Gb = dY . w_base (fp32 [batch, in]) for the SiLU term of dx
             gb = reinterpret_cast<float*>(w + P.bwd.gb);
             CUtensorMap maps[6];
-            if (!make_map_2d(&maps[0], dy_hi, f32, p.batch, p.out, kBM, BK, detail) ||
-                !make_map_2d(&maps[1], dy_lo, f32, p.batch, p.out, kBM, BK, detail))
+            if (!make_map_2d(&maps[0], dY, false, p.batch, p.out, kBM, BK, detail) ||
+                !make_map_2d(&maps[2], w_base, false, p.out, p.in, BK, EPB, detail))
                 return cudaErrorInvalidValue;
-            if (f32) {
-                const void *th, *tl;
-                if ((e = split_t_into(w_base, p.out, p.in, p.out, w + P.bwd.wb_hl, &th, &tl, st)) != cudaSuccess)
-                    return e;
-                if (!make_map_2d(&maps[2], th, true, p.in, p.out, P.g_BN, BK, detail) ||
-                    !make_map_2d(&maps[3], tl, true, p.in, p.out, P.g_BN, BK, detail))
-                    return cudaErrorInvalidValue;
-            } else {
-                if (!make_map_2d(&maps[2], w_base, false, p.out, p.in, BK, EPB, detail)) return cudaErrorInvalidValue;
-                maps[3] = maps[2];
-            }
-            maps[4] = maps[2];
-            maps[5] = maps[3];
+            maps[1] = maps[0];
+            maps[3] = maps[4] = maps[5] = maps[2];
             TcArgs a = base_args(p, P);
             a.out = gb;
             a.BN = P.g_BN;
@@ -2062,19 +2102,17 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             if (e != cudaSuccess) return e;
         }
         CUtensorMap maps[6];
-        const int xBN = P.p_ok ? P.p_BN : P.x_BN;
-        if (!make_map_2d(&maps[0], dy_hi, f32, p.batch, p.out, kBM, BK, detail) ||
-            !make_map_2d(&maps[1], dy_lo, f32, p.batch, p.out, kBM, BK, detail))
-            return cudaErrorInvalidValue;
+        if (!make_map_2d(&maps[0], dy_hi, f32, p.batch, p.out, kBM, BK, detail)) return cudaErrorInvalidValue;
         if (f32) {
-            const void *th, *tl;
-            e = P.ext ? split_ext_into(p, P, coef, w_base, true, p.out, w + P.bwd.coef_hl, &th, &tl, st)
-                      : split_t_into(coef, p.out, p.Kt, p.out, w + P.bwd.coef_hl, &th, &tl, st);
-            if (e != cudaSuccess) return e;
-            if (!make_map_2d(&maps[2], th, true, P.Kx, p.out, xBN, BK, detail) ||
-                !make_map_2d(&maps[3], tl, true, P.Kx, p.out, xBN, BK, detail))
+            if (!make_map_2d(&maps[1], dy_lo, true, p.batch, p.out, kBM, BK, detail)) return cudaErrorInvalidValue;
+            const void *c_hi, *c_lo;
+            if ((e = split_coef_into(p, P, coef, w_base, w + P.bwd.coef_hl, amax, &c_hi, &c_lo, st)) != cudaSuccess)
+                return e;
+            if (!make_map_2d(&maps[2], c_hi, true, p.out, P.Kx, BK, EPB, detail) ||
+                !make_map_2d(&maps[3], c_lo, true, p.out, P.Kx, BK, EPB, detail))
                 return cudaErrorInvalidValue;
         } else {
+            maps[1] = maps[0];
             if (!make_map_2d(&maps[2], coef, false, p.out, p.Kt, BK, EPB, detail)) return cudaErrorInvalidValue;
             maps[3] = maps[2];
         }
@@ -2086,6 +2124,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             d.dx = dx;
             d.gb = gb;
             d.status = device_status_ptr();
+            d.amax = amax;
             d.batch = p.batch;
             d.in = p.in;
             d.out = p.out;
@@ -2107,6 +2146,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         } else {
             TcArgs a = base_args(p, P);
             a.x = x;
+            a.amax = amax;
             a.out = dx;
             a.out2 = gb;
             a.BN = P.x_BN;

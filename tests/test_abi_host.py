@@ -108,7 +108,7 @@ def test_forced_tensor_path_unsupported_stride(lib):
 
 
 def test_workspace_too_small(lib):
-    # fp32 on the tensor path needs the tf32 hi/lo copies of coef
+    # fp32 on the tensor path needs the fp16 hi/lo copies of coef (and the operand maxima)
     s = shp(batch=4096, n_in=64, n_out=256, path=N.KAN_PATH_TENSOR)
     need = ctypes.c_size_t(0)
     assert lib.kan_workspace_size(ctypes.byref(s), 0, ctypes.byref(need)) == 0

@@ -7,7 +7,7 @@ the caller.
 Checked here, through the C ABI: two calls in a row give the same result as
 kan_forward with a caller-allocated workspace (within the parity tolerance of
 the other tests), on shapes that do use workspace (split-K partial sums, and
-the tf32 hi/lo copies for fp32), and a shape whose workspace exceeds the
+the fp16 hi/lo copies for fp32), and a shape whose workspace exceeds the
 fixed size is refused with KAN_ERR_WORKSPACE.  This file is named to be
 collected last, and passes alone in a fresh process as well.
 """
@@ -57,7 +57,7 @@ def test_fixed_scratch_matches_caller_workspace(dt):
 
 
 def test_fixed_scratch_refuses_oversized_workspace():
-    # fp32, 512 x 2048 -> 512, G = 50: the tf32 copies of coef alone exceed 32 MiB
+    # fp32, 512 x 2048 -> 512, G = 50: the fp16 hi/lo copies of coef alone exceed 32 MiB
     s = N.make_shape(4096, 2048, 512, 50, -1.0, 1.0, N.KAN_F32, False, N.KAN_PATH_TENSOR)
     assert N.kan_workspace_size(s, False) > 32 * 1024 * 1024
     lib = N.load()
