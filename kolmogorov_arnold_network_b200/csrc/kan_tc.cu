@@ -1429,21 +1429,23 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, T* __restri
 
 // dcoef[j, kt] and dw_base[j, i] from partials [splits][out][ld], split order.
 // Columns: Kt spline columns then `in` SiLU columns, or (ext) input groups of
-// nbx columns, the last of which is the input's SiLU column.
+// nbx columns, the last of which is the input's SiLU column.  Rows j step
+// by gridDim.y; column c / nbx through a multiply-high (nbx_magic = ceil(2^32 / nbx)).
 __global__ void reduce_dcoef_kernel(const float* __restrict__ part, float* __restrict__ dcoef,
                                     float* __restrict__ dw_base, int64_t out, int64_t Kt, int64_t in, int64_t ld,
-                                    int splits, int nbs, int nbx, int ext)
+                                    int splits, int nbs, int nbx, int ext, uint32_t nbx_magic)
 {
     const int64_t n = out * ld;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t j = e / ld, c = e % ld;
+    for (int64_t j = blockIdx.y; j < out; j += gridDim.y)
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < (int)ld; c += gridDim.x * blockDim.x) {
+        const int64_t e = j * ld + c;
         float acc = 0.f;
         for (int z = 0; z < splits; ++z) acc += part[(int64_t)z * n + e];
         if (ext) {
-            const int64_t i = c / nbx;
-            const int m = (int)(c - i * nbx);
+            const int i = (int)__umulhi((uint32_t)c, nbx_magic);
+            const int m = c - i * nbx;
             if (m < nbs) {
-                if (dcoef) dcoef[j * Kt + i * nbs + m] = acc;
+                if (dcoef) dcoef[j * Kt + (int64_t)i * nbs + m] = acc;
             } else if (dw_base) {
                 dw_base[j * in + i] = acc;
             }
@@ -1458,7 +1460,8 @@ __global__ void reduce_dcoef_kernel(const float* __restrict__ part, float* __res
 // Absolute maxima of up to four fp32 arrays (amax[k] over src[k][0..n[k]),
 // NaN ignored) as the bit patterns of non-negative floats, combined with
 // atomicMax: the maximum does not depend on the order, so the result is
-// deterministic.  amax must start at 0.
+// deterministic.  amax must start at 0.  Arrays are 16-byte aligned and read
+// as float4 (a scalar tail when n is not a multiple of 4).
 struct AmaxArgs {
     const float* src[4];
     int64_t n[4];
@@ -1468,13 +1471,18 @@ __global__ void absmax_kernel(AmaxArgs a, unsigned int* __restrict__ amax)
     __shared__ unsigned int red[4];
     if (threadIdx.x < 4) red[threadIdx.x] = 0u;
     __syncthreads();
+    const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, nth = (int64_t)gridDim.x * blockDim.x;
+#pragma unroll
     for (int k = 0; k < 4; ++k) {
         if (!a.src[k]) continue;
         float m = 0.0f;
-        const int64_t n = a.n[k];
-        const float* __restrict__ src = a.src[k];
-        for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
-            m = fmaxf(m, fabsf(src[e]));
+        const int64_t n = a.n[k], n4 = n / 4;
+        const float4* __restrict__ v4 = reinterpret_cast<const float4*>(a.src[k]);
+        for (int64_t e = tid; e < n4; e += nth) {
+            const float4 q = v4[e];
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+        }
+        for (int64_t e = 4 * n4 + tid; e < n; e += nth) m = fmaxf(m, fabsf(a.src[k][e]));
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((threadIdx.x & 31) == 0) atomicMax(&red[k], __float_as_uint(m));
     }
@@ -1482,31 +1490,44 @@ __global__ void absmax_kernel(AmaxArgs a, unsigned int* __restrict__ amax)
     if (threadIdx.x < 4 && a.src[threadIdx.x]) atomicMax(&amax[threadIdx.x], red[threadIdx.x]);
 }
 
-// fp16 hi/lo split of an fp32 array, times the dY scale (amax slot 3).
+// fp16 hi/lo split of an fp32 array, times the dY scale (amax slot 3); four
+// values per thread step (n % 4 == 0: n is batch * out with out % 8 == 0).
 __global__ void split_f16_kernel(const float* __restrict__ src, uint16_t* __restrict__ hi, uint16_t* __restrict__ lo,
                                  int64_t n, const unsigned int* __restrict__ amax)
 {
     const float sc = scales_of(amax).d;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
-        split_f16(src[e] * sc, hi[e], lo[e]);
+    const int64_t n4 = n / 4;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
+        const float4 q = reinterpret_cast<const float4*>(src)[e];
+        uint16_t h[4], l[4];
+        split_f16(q.x * sc, h[0], l[0]);
+        split_f16(q.y * sc, h[1], l[1]);
+        split_f16(q.z * sc, h[2], l[2]);
+        split_f16(q.w * sc, h[3], l[3]);
+        reinterpret_cast<uint2*>(hi)[e] = make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
+        reinterpret_cast<uint2*>(lo)[e] = make_uint2(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16));
+    }
 }
 
 // fp16 hi/lo split of the coefficient matrix, row-major [out][in*nbx]:
 // column i*nbx + m is coef[j, i, m] * s_c for m < nbs, and (with the SiLU
-// branch, nbx = nbs + 1) w_base[j, i] * s_c / s_x for m == nbs.
+// branch, nbx = nbs + 1) w_base[j, i] * s_c / s_x for m == nbs.  Rows j step
+// by gridDim.y, one column per thread (coalesced writes; the reads are
+// consecutive apart from the SiLU columns); c / nbx through a multiply-high.
 __global__ void split_coef_f16_kernel(const float* __restrict__ coef, const float* __restrict__ w_base, int64_t out,
                                       int64_t in, int nbs, int nbx, uint16_t* __restrict__ hi, uint16_t* __restrict__ lo,
-                                      const unsigned int* __restrict__ amax)
+                                      const unsigned int* __restrict__ amax, uint32_t nbx_magic)
 {
     const Scales sc = scales_of(amax);
     const float sw = sc.c / sc.x;
-    const int64_t Kx = in * nbx, n = out * Kx;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t j = e / Kx, c = e - j * Kx;
-        const int64_t i = c / nbx;
-        const int m = (int)(c - i * nbx);
-        const float v = m < nbs ? coef[(j * in + i) * nbs + m] * sc.c : w_base[j * in + i] * sw;
-        split_f16(v, hi[e], lo[e]);
+    const int Kx = (int)(in * nbx);
+    for (int64_t j = blockIdx.y; j < out; j += gridDim.y)
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < Kx; c += gridDim.x * blockDim.x) {
+        const float* __restrict__ crow = coef + j * in * nbs;
+        const int i = (int)__umulhi((uint32_t)c, nbx_magic);
+        const int m = c - i * nbx;
+        const float v = m < nbs ? crow[i * nbs + m] * sc.c : w_base[j * in + i] * sw;
+        split_f16(v, hi[j * Kx + c], lo[j * Kx + c]);
     }
 }
 
@@ -1821,6 +1842,9 @@ cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap
         if (need <= 4)
             return f32 ? launch<MODE, KAN_F32, 4>(grid, BN, stages, maps, args, st)
                        : launch<MODE, KAN_BF16, 4>(grid, BN, stages, maps, args, st);
+        if (need <= 7)
+            return f32 ? launch<MODE, KAN_F32, 7>(grid, BN, stages, maps, args, st)
+                       : launch<MODE, KAN_BF16, 7>(grid, BN, stages, maps, args, st);
         if (need <= 9)
             return f32 ? launch<MODE, KAN_F32, 9>(grid, BN, stages, maps, args, st)
                        : launch<MODE, KAN_BF16, 9>(grid, BN, stages, maps, args, st);
@@ -1889,7 +1913,7 @@ cudaError_t amax_into(const Problem& p, const void* coef, const void* w_base, co
     int64_t nmax = 0;
     for (int k = 0; k < 4; ++k)
         if (a.src[k]) nmax = std::max(nmax, a.n[k]);
-    absmax_kernel<<<grid_for(nmax), 256, 0, st>>>(a, amax);
+    absmax_kernel<<<std::min(grid_for(nmax / 4), 148 * 4), 256, 0, st>>>(a, amax);
     count_launch();
     return cudaGetLastError();
 }
@@ -1900,8 +1924,10 @@ cudaError_t split_coef_into(const Problem& p, const Plan& P, const void* coef, c
 {
     uint16_t* h = reinterpret_cast<uint16_t*>(dst);
     uint16_t* l = reinterpret_cast<uint16_t*>(dst + al256((size_t)p.out * P.Kx * 2));
-    split_coef_f16_kernel<<<grid_for(p.out * P.Kx), 256, 0, st>>>((const float*)coef, (const float*)w_base, p.out,
-                                                                 p.in, p.nb, P.nbx, h, l, amax);
+    const dim3 grid((unsigned)std::min<int64_t>(cdiv(P.Kx, 256), 64), (unsigned)std::min<int64_t>(p.out, 65535));
+    const uint32_t magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)P.nbx - 1) / (uint64_t)P.nbx);
+    split_coef_f16_kernel<<<grid, 256, 0, st>>>((const float*)coef, (const float*)w_base, p.out, p.in, p.nb, P.nbx, h,
+                                                l, amax, magic);
     count_launch();
     *hi = h;
     *lo = l;
@@ -1915,7 +1941,7 @@ cudaError_t split_dy_into(const Problem& p, const void* dY, uint8_t* dst, const 
     const int64_t n = p.batch * p.out;
     uint16_t* h = reinterpret_cast<uint16_t*>(dst);
     uint16_t* l = reinterpret_cast<uint16_t*>(dst + al256((size_t)n * 2));
-    split_f16_kernel<<<grid_for(n), 256, 0, st>>>((const float*)dY, h, l, n, amax);
+    split_f16_kernel<<<grid_for(n / 4), 256, 0, st>>>((const float*)dY, h, l, n, amax);
     count_launch();
     *hi = h;
     *lo = l;
@@ -2041,7 +2067,8 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
     if (f32) {
         // operand scales (coef and w_base for dx's coefficient copy, x for the
         // SiLU values, dY), then dY's fp16 hi/lo copy, shared by dcoef and dx
-        if ((e = amax_into(p, coef, w_base, x, dY, amax, st)) != cudaSuccess) return e;
+        // (coef and w_base scale only dx's coefficient copy)
+        if ((e = amax_into(p, dx ? coef : nullptr, dx ? w_base : nullptr, x, dY, amax, st)) != cudaSuccess) return e;
         if ((e = split_dy_into(p, dY, w + P.bwd.dy_hl, amax, &dy_hi, &dy_lo, st)) != cudaSuccess) return e;
     }
     // ---- dcoef / dw_base: A = basis^T (producers), B = dY MN-major (BK-batch x 64-output boxes) ----
@@ -2074,8 +2101,10 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         if (e != cudaSuccess) return e;
         if (a.partial) {
             const int64_t n = p.out * P.d_ld;
-            reduce_dcoef_kernel<<<grid_for(n), 256, 0, st>>>(partbuf, dcoef, dw_base, p.out, p.Kt, p.in, P.d_ld,
-                                                              P.d_splits, p.nb, P.nbx, P.ext ? 1 : 0);
+            const dim3 rgrid((unsigned)std::min<int64_t>(cdiv(P.d_ld, 256), 64),
+                             (unsigned)std::min<int64_t>(p.out, 65535));
+            reduce_dcoef_kernel<<<rgrid, 256, 0, st>>>(partbuf, dcoef, dw_base, p.out, p.Kt, p.in, P.d_ld, P.d_splits,
+                                                       p.nb, P.nbx, P.ext ? 1 : 0, a.nb_magic);
             count_launch();
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
