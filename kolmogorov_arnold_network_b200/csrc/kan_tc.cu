@@ -908,22 +908,31 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             tc_fence_after();
             // value of accumulator column c0..c0+15 of this thread's row (fp32:
             // total + corr * 2^-11, times `mul`, the inverse of the operand scales)
-            auto load16 = [&](int c0, float (&out)[16], float mul) {
-                uint32_t v[16];
+            // (columns c0..c0+31: both halves' loads in flight together; BN % 32 == 0)
+            auto load32 = [&](int c0, float (&out)[32], float mul) {
+                uint32_t v[2][16];
                 if constexpr (F32) {
-                    uint32_t w[16];
-                    tmem_ld16(t_total + lane_off + c0, v);
-                    tmem_ld16(t_corr + lane_off + c0, w);
+                    uint32_t w[2][16];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        tmem_ld16(t_total + lane_off + c0 + 16 * j, v[j]);
+                        tmem_ld16(t_corr + lane_off + c0 + 16 * j, w[j]);
+                    }
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        out[e] = fmaf(__uint_as_float(w[e]), kLoInv, __uint_as_float(v[e])) * mul;
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            out[16 * j + e] = fmaf(__uint_as_float(w[j][e]), kLoInv, __uint_as_float(v[j][e])) * mul;
                 } else {
                     (void)mul;
-                    tmem_ld16(t_main0 + lane_off + c0, v);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) tmem_ld16(t_main0 + lane_off + c0 + 16 * j, v[j]);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) out[e] = __uint_as_float(v[e]);
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) out[16 * j + e] = __uint_as_float(v[j][e]);
                 }
             };
 
@@ -931,9 +940,15 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const int64_t bo = m0 + r;
                 const int64_t ncols = MODE == FWD ? a.out_f : a.in;
                 const float mul = F32 ? 1.0f / scales_of(a.amax).c : 1.0f;   // y = acc / s_c
-                for (int c0 = 0; c0 < BN; c0 += 16) {
+                for (int c1 = 0; c1 < BN; c1 += 32) {
+                  float v32[32];
+                  load32(c1, v32, mul);
+#pragma unroll
+                  for (int jh = 0; jh < 2; ++jh) {
+                    const int c0 = c1 + 16 * jh;
                     float v[16];
-                    load16(c0, v, mul);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = v32[16 * jh + e];
                     if (bo >= a.batch) continue;
                     const int64_t j0 = n0 + c0;
                     if (MODE == GEMM || a.partial) {
@@ -976,6 +991,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                 }
+                }
             } else if constexpr (MODE == DCA) {
                 // rows are spline columns kt (or inputs of a SiLU tile); columns are outputs j
                 const int mt = blockIdx.y;
@@ -1014,14 +1030,14 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         if ((int)rowg - ii * a.nb >= a.nbs) mul /= sc.x;
                     }
                 }
-                for (int c0 = 0; c0 < BN; c0 += 16) {
-                    float v[16];
-                    load16(c0, v, mul);
+                for (int c1 = 0; c1 < BN; c1 += 32) {
+                    float v32[32];
+                    load32(c1, v32, mul);
                     if (!row_ok || !dst) continue;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int64_t j = n0 + c0 + e;
-                        if (j < a.out_f) dst[j * ld] = v[e];
+                    for (int e = 0; e < 32; ++e) {
+                        const int64_t j = n0 + c1 + e;
+                        if (j < a.out_f) dst[j * ld] = v32[e];
                     }
                 }
             } else {
@@ -1030,11 +1046,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const int ldst = BN + 1;
                 float* stage = reinterpret_cast<float*>(smem) + (size_t)(warp - Warps<MODE>::kEpi0) * 32 * ldst +
                                (size_t)lane * ldst;
-                for (int c0 = 0; c0 < BN; c0 += 16) {
-                    float v[16];
-                    load16(c0, v, 1.0f);
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    load32(c0, v, 1.0f);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) stage[c0 + e] = v[e];
+                    for (int e = 0; e < 32; ++e) stage[c0 + e] = v[e];
                 }
                 // fp32: the staged columns are scaled by s_d s_c (spline) and s_d s_c / s_x (SiLU)
                 float inv_dc = 1.0f, ext_mul = 1.0f;
@@ -1115,6 +1131,8 @@ struct DxArgs {
     int n_in_tile, n_tiles_n, n_tiles;
     int ld_stage;             // staging row stride in elements
     const unsigned int* amax; // fp32: absolute maxima of the operands (scales_of)
+    int a_res;                // 1: short contraction (nkb k-blocks of dY fit beside the B ring): each
+                              // CTA walks a contiguous run of tiles and keeps the dY rows resident
 };
 
 template <int DT>
@@ -1133,25 +1151,32 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     uint8_t* smem = align1024(smem_raw);
 
     const int BN = a.BN, stages = a.stages;
+    const bool ares = a.a_res != 0;
     const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)BN * 128;
-    const uint32_t stage_bytes = (a_bytes + b_bytes) * C::SPLIT;
+    const uint32_t a_stage = a_bytes * C::SPLIT, b_stage = b_bytes * C::SPLIT;
+    const uint32_t stage_bytes = a_stage + b_stage;
     const uint32_t sbase = smem_addr(smem);
+    // Slots: a ring of `stages` (A, B) pairs; or, with the dY rows resident,
+    // nkb A blocks followed by a ring of `stages` B slots.
+    const uint32_t ring_bytes = ares ? a.nkb * a_stage + stages * b_stage : stages * stage_bytes;
     // staging of the accumulator rows: fp32 for fp32 operands, bf16 for bf16
     // operands (the dx it feeds is rounded to bf16 anyway)
     using ST = typename std::conditional<F32, float, __nv_bfloat16>::type;
-    ST* staging = reinterpret_cast<ST*>(smem + stages * stage_bytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes + 4 * 32 * a.ld_stage * (int)sizeof(ST));
-    // full[S] empty[S] acc_full[2] acc_empty[2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 4);
+    ST* staging = reinterpret_cast<ST*>(smem + ring_bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ring_bytes + 4 * 32 * a.ld_stage * (int)sizeof(ST));
+    // full[S] empty[S] acc_full[2] acc_empty[2] a_full a_empty
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 6);
     volatile int* pair_ok = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [4 quarters][2 warps]
     auto full = [&](int s) { return smem_addr(&bars[s]); };
     auto empty = [&](int s) { return smem_addr(&bars[stages + s]); };
     auto acc_full = [&](int b) { return smem_addr(&bars[2 * stages + b]); };
     auto acc_empty = [&](int b) { return smem_addr(&bars[2 * stages + 2 + b]); };
-    auto A_hi = [&](int s) { return sbase + s * stage_bytes; };
-    auto A_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes; };
-    auto B_hi = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT; };
-    auto B_lo = [&](int s) { return sbase + s * stage_bytes + a_bytes * C::SPLIT + b_bytes; };
+    const uint32_t a_full = smem_addr(&bars[2 * stages + 4]), a_empty = smem_addr(&bars[2 * stages + 5]);
+    // A of ring slot s (or, resident, of k-block s)
+    auto A_hi = [&](int s) { return sbase + s * (ares ? a_stage : stage_bytes); };
+    auto A_lo = [&](int s) { return A_hi(s) + a_bytes; };
+    auto B_hi = [&](int s) { return ares ? sbase + a.nkb * a_stage + s * b_stage : sbase + s * stage_bytes + a_stage; };
+    auto B_lo = [&](int s) { return B_hi(s) + b_bytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t acc_cols = F32 ? 2u * BN : (uint32_t)BN;   // one buffer: [main | corr] or [acc]
@@ -1164,6 +1189,8 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         mbar_init(acc_full(1), 1);
         mbar_init(acc_empty(0), 256);   // every epilogue thread
         mbar_init(acc_empty(1), 256);
+        mbar_init(a_full, 1);           // resident dY rows landed (TMA bytes)
+        mbar_init(a_empty, 1);          // the MMA is done with them (commit)
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -1174,10 +1201,15 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // tiles of this CTA: t = blockIdx.x + k * gridDim.x; (batch tile, input group) = (t / n_tiles_n, t % n_tiles_n)
-    const int my_tiles = a.n_tiles > (int)blockIdx.x ? (a.n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    // tiles of this CTA: t = blockIdx.x + k * gridDim.x, or (resident dY) the
+    // contiguous run [t_begin, t_end); (batch tile, input group) = (t / n_tiles_n, t % n_tiles_n)
+    const int t_begin = (int)((int64_t)a.n_tiles * blockIdx.x / gridDim.x);
+    const int t_end = (int)((int64_t)a.n_tiles * (blockIdx.x + 1) / gridDim.x);
+    const int my_tiles = ares ? t_end - t_begin
+                              : (a.n_tiles > (int)blockIdx.x ? (a.n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0);
+    auto tile_of = [&](int lt) { return ares ? t_begin + lt : (int)blockIdx.x + lt * (int)gridDim.x; };
     auto tile_coords = [&](int lt, int64_t& m0, int& i0) {
-        const int t = (int)blockIdx.x + lt * (int)gridDim.x;
+        const int t = tile_of(lt);
         m0 = (int64_t)(t / a.n_tiles_n) * kBM;
         i0 = (t % a.n_tiles_n) * a.n_in_tile;
     };
@@ -1193,16 +1225,31 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             int s = 0;   // its stage ring position and phase
             uint32_t ph = 0;
             bool ok = true;
+            int a_loads = 0;          // resident dY loads issued
+            int64_t a_m = -1;         // their batch tile
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
                 int64_t m0;
                 int i0;
                 tile_coords(lt, m0, i0);
                 const int kt0 = kt_start(i0);
+                if (ares && m0 != a_m) {
+                    // new batch tile: once the MMA is done with the previous rows, load these
+                    if (a_loads > 0 && !mbar_wait(a_empty, (a_loads - 1) & 1, a.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(a_full, a.nkb * a_stage);
+                    for (int kb = 0; kb < a.nkb; ++kb) {
+                        tma_load_2d(A_hi(kb), &tA_hi, a_full, kb * BK, (int)m0);
+                        if (F32) tma_load_2d(A_lo(kb), &tA_lo, a_full, kb * BK, (int)m0);
+                    }
+                    ++a_loads;
+                    a_m = m0;
+                }
                 for (int kb = 0; kb < a.nkb; ++kb, ++g, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
                     if (!mbar_wait(empty(s), ph ^ 1, a.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(full(s), (a_bytes + b_bytes) * C::SPLIT);
-                    tma_load_2d(A_hi(s), &tA_hi, full(s), kb * BK, (int)m0);
-                    if (F32) tma_load_2d(A_lo(s), &tA_lo, full(s), kb * BK, (int)m0);
+                    mbar_arrive_expect_tx(full(s), ares ? b_stage : stage_bytes);
+                    if (!ares) {
+                        tma_load_2d(A_hi(s), &tA_hi, full(s), kb * BK, (int)m0);
+                        if (F32) tma_load_2d(A_lo(s), &tA_lo, full(s), kb * BK, (int)m0);
+                    }
                     if (B_MN) {
                         for (int c = 0; c < BN / EPB; ++c) {
                             tma_load_2d(B_hi(s) + (uint32_t)c * BK * 128, &tB_hi, full(s), kt0 + c * EPB, kb * BK);
@@ -1216,6 +1263,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                 }
             }
             for (int q = max(0, g - stages); q < g; ++q) mbar_wait(full(q % stages), (q / stages) & 1, a.status);
+            if (a_loads > 0) mbar_wait(a_full, (a_loads - 1) & 1, a.status);
         }
     } else if (warp == 1) {
         if (lane == 0 && my_tiles > 0) {
@@ -1225,8 +1273,18 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
+            int a_uses = 0;           // resident dY loads consumed
+            int64_t a_m = -1;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
                 const int buf = lt & 1;
+                int64_t m0;
+                int i0;
+                tile_coords(lt, m0, i0);
+                if (ares && m0 != a_m) {
+                    if (!mbar_wait(a_full, a_uses & 1, a.status)) break;
+                    ++a_uses;
+                    a_m = m0;
+                }
                 if (lt >= 2 && !mbar_wait(acc_empty(buf), ((lt >> 1) - 1) & 1, a.status)) break;
                 tc_fence_after();
                 const uint32_t d_main = tmem + buf * acc_cols, d_corr = d_main + BN;
@@ -1234,9 +1292,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     if (!mbar_wait(full(s), ph, a.status)) { ok = false; break; }
                     tc_fence_after();
                     // k-steps advance the descriptors' start address field (no carry below 2^18)
-                    const uint64_t ad0 = smem_desc_sw128(A_hi(s), 16, 1024);
+                    const int sa = ares ? kb : s;
+                    const uint64_t ad0 = smem_desc_sw128(A_hi(sa), 16, 1024);
                     const uint64_t bd0 = smem_desc_sw128(B_hi(s), b_lbo, 1024);
-                    const uint64_t adl0 = F32 ? smem_desc_sw128(A_lo(s), 16, 1024) : 0;
+                    const uint64_t adl0 = F32 ? smem_desc_sw128(A_lo(sa), 16, 1024) : 0;
                     const uint64_t bdl0 = F32 ? smem_desc_sw128(B_lo(s), b_lbo, 1024) : 0;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
@@ -1255,7 +1314,15 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     }
                     mma_commit(empty(s));
                 }
-                if (ok) mma_commit(acc_full(buf));
+                if (!ok) break;
+                mma_commit(acc_full(buf));
+                // the last tile of this batch tile's run: release the resident rows
+                if (ares && lt + 1 < my_tiles) {
+                    int64_t mn;
+                    int in_;
+                    tile_coords(lt + 1, mn, in_);
+                    if (mn != m0) mma_commit(a_empty);
+                }
             }
         }
     } else {
@@ -1318,29 +1385,41 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             // stage this warp's half of the row: TMEM -> registers -> shared (16-byte
             // stores; the row stride is 16 bytes mod 128, so a warp's stores are conflict-free)
             const uint32_t t_main = tmem + buf * acc_cols + lane_off;
-            for (int c0 = h * half_cols; c0 < (h + 1) * half_cols; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(t_main + c0, v);
+            // 64 columns per round: all of the round's TMEM loads are in flight
+            // together and one wait covers them
+            for (int c1 = h * half_cols; c1 < (h + 1) * half_cols; c1 += 64) {
+                uint32_t v[4][16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tmem_ld16(t_main + c1 + 16 * j, v[j]);
                 if constexpr (F32) {   // main + corr * 2^-11
-                    uint32_t w[16];
-                    tmem_ld16(t_main + BN + c0, w);
+                    uint32_t w[4][16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) tmem_ld16(t_main + BN + c1 + 16 * j, w[j]);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        v[e] = __float_as_uint(fmaf(__uint_as_float(w[e]), kLoInv, __uint_as_float(v[e])));
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            v[j][e] = __float_as_uint(fmaf(__uint_as_float(w[j][e]), kLoInv, __uint_as_float(v[j][e])));
                 } else {
                     tmem_ld_wait();
                 }
-                if constexpr (F32) {
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        *reinterpret_cast<uint4*>(srow + c0 + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                } else {
-                    uint32_t pk[8];
+                for (int j = 0; j < 4; ++j) {
+                    const int c0 = c1 + 16 * j;
+                    if constexpr (F32) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                    *reinterpret_cast<uint4*>(srow + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4*>(srow + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        for (int e = 0; e < 16; e += 4)
+                            *reinterpret_cast<uint4*>(srow + c0 + e) =
+                                make_uint4(v[j][e], v[j][e + 1], v[j][e + 2], v[j][e + 3]);
+                    } else {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            pk[e] = pack_bf16(__uint_as_float(v[j][2 * e]), __uint_as_float(v[j][2 * e + 1]));
+                        *reinterpret_cast<uint4*>(srow + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4*>(srow + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
                 }
             }
             // the accumulator buffer is free for the tile after next
@@ -1690,7 +1769,7 @@ struct Plan {
     // dx
     int x_BN, x_stages, x_n, x_m, x_nin, x_nkb;
     // dx, persistent kernel (used when p_ok)
-    bool p_ok;
+    bool p_ok, p_ares;
     int p_BN, p_stages, p_nin, p_ntn, p_tiles, p_ld, p_grid, p_smem;
     // dY . w_base
     int g_BN, g_stages, g_n, g_m;
@@ -1751,14 +1830,27 @@ Plan make_plan(const Problem& p, int sms)
         P.p_nin = (P.p_BN - maxoff) / P.nbx;
         P.p_ld = f32 ? P.p_BN + 4 : P.p_BN + 8;          // row stride = 16 bytes mod 128
         const int staging = 4 * 32 * P.p_ld * (f32 ? 4 : 2);
-        const int stage_bytes = (kBM * 128 + P.p_BN * 128) * (f32 ? 2 : 1);
-        P.p_stages = std::min(6, (232448 - 1024 - 256 - staging) / stage_bytes);
+        const int a_stage = kBM * 128 * (f32 ? 2 : 1), b_stage = P.p_BN * 128 * (f32 ? 2 : 1);
+        const int stage_bytes = a_stage + b_stage;
+        const int avail = 232448 - 1024 - 256 - staging;
+        P.p_stages = std::min(6, avail / stage_bytes);
+        // A short contraction (at most 2 k-blocks over `out`): keep the dY rows
+        // resident per batch tile when that leaves more B slots than the (A, B) ring
+        P.p_ares = false;
+        if (P.x_nkb <= 2) {
+            const int sb = std::min(6, (avail - P.x_nkb * a_stage) / b_stage);
+            if (sb >= 3 && sb > P.p_stages) {
+                P.p_ares = true;
+                P.p_stages = sb;
+            }
+        }
         P.p_ok = P.p_nin >= 1 && P.p_stages >= 2 && (!f32 || p.out <= 1024);
         if (P.p_ok) {
             P.p_ntn = (int)cdiv(p.in, P.p_nin);
             P.p_tiles = P.p_ntn * P.x_m;
             P.p_grid = std::max(1, std::min(P.p_tiles, sms));
-            P.p_smem = P.p_stages * stage_bytes + staging + 1024 + 256;
+            P.p_smem = (P.p_ares ? P.x_nkb * a_stage + P.p_stages * b_stage : P.p_stages * stage_bytes) + staging +
+                       1024 + 256;
         }
     }
     // dY . w_base (bf16 with the SiLU branch): M = batch, N = in, K = out
@@ -2170,6 +2262,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             d.n_tiles_n = P.p_ntn;
             d.n_tiles = P.p_tiles;
             d.ld_stage = P.p_ld;
+            d.a_res = P.p_ares ? 1 : 0;
             e = f32 ? launch_dx_persistent<KAN_F32>(P, maps, d, st) : launch_dx_persistent<KAN_BF16>(P, maps, d, st);
             if (e != cudaSuccess) return e;
         } else {
