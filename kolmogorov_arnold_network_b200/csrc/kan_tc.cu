@@ -1427,8 +1427,22 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             mbar_arrive(acc_empty(buf));
             // both halves of the row are staged
             named_bar_sync(1 + q, 64);
+            // dx of this warp's inputs [ia, ib): each lane computes its row's values
+            // and parks them in slots slot_base + 0.. of its own staging row, which
+            // lie below every column still to be read (input ia + k reads columns at
+            // or above (ia + k) * nb - kt_al > slot_base + k - 1) and inside this
+            // warp's own column range; the warp then writes its 32 x n block with
+            // contiguous row segments instead of 32 scattered rows per store.
+            const int slot_base = ia * a.nb - kt_al;
+            const int n_mine = ib - ia;
+            // Whole aligned chunks of XC inputs go out directly as 16-byte vectors (a
+            // lane writes 32 or 64 contiguous bytes); otherwise bf16 values take the
+            // block write below (2-byte scattered stores would cost an L2 sector
+            // each), fp32 values are stored directly.
+            const bool vec_out = n_mine % XC == 0 && (ia * (int)sizeof(T)) % 16 == 0 && (a.in * (int64_t)sizeof(T)) % 16 == 0;
+            const bool block_out = !vec_out && !F32;
+            T* dxr = reinterpret_cast<T*>(a.dx) + (b_ok ? b : 0) * a.in;
             if (b_ok) {
-                T* dxr = reinterpret_cast<T*>(a.dx) + b * a.in;
                 for (int ic = ia; ic < ib; ic += XC) {
                     float xc[XC], gc[XC];
 #pragma unroll
@@ -1458,8 +1472,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         else if (a.gb) acc += dsilu_f(xv) * gc[k];
                         return acc;
                     };
-                    if (nkc == XC && (((uintptr_t)(dxr + ic)) & 15u) == 0) {
-                        // a whole, aligned chunk: 16-byte stores
+                    if (vec_out) {
                         float res[XC];
 #pragma unroll
                         for (int k = 0; k < XC; ++k) res[k] = dx_of(k);
@@ -1479,8 +1492,28 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 #pragma unroll
                         for (int k = 0; k < XC; ++k) {
                             if (k >= nkc) break;
-                            dxr[ic + k] = from_f<T>(dx_of(k));
+                            const float r = dx_of(k);
+                            if (block_out) srow[slot_base + (ic - ia) + k] = from_f<ST>(r);
+                            else dxr[ic + k] = from_f<T>(r);
                         }
+                    }
+                }
+            }
+            __syncwarp();
+            if (block_out && n_mine > 0) {
+                // element e of the warp's block is (row e / n_mine, input e % n_mine); a
+                // store instruction covers 32 consecutive elements
+                const ST* sq = staging + (size_t)q * 32 * a.ld_stage;
+                T* dxq = reinterpret_cast<T*>(a.dx) + (m0 + 32 * q) * a.in + ia;
+                const int q32 = 32 / n_mine, r32 = 32 - q32 * n_mine;
+                int rr = lane / n_mine, cc = lane - (lane / n_mine) * n_mine;
+                for (int e = lane; e < 32 * n_mine; e += 32) {
+                    if (m0 + 32 * q + rr < a.batch) dxq[(int64_t)rr * a.in + cc] = sq[(size_t)rr * a.ld_stage + slot_base + cc];
+                    rr += q32;
+                    cc += r32;
+                    if (cc >= n_mine) {
+                        cc -= n_mine;
+                        ++rr;
                     }
                 }
             }
