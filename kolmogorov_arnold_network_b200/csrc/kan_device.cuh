@@ -69,11 +69,16 @@ __device__ __forceinline__ void dweights(float t, float inv_h, float d[4])
     d[3] = 0.5f * t * t * inv_h;
 }
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// silu(x) = x sigma(x) and silu'(x) = sigma(x) (1 + x (1 - sigma(x))), with
+// sigma(x) = 1 / (1 + e^-x) through the correctly rounded reciprocal (no
+// division sequence); sigma -> 0 as e^-x -> inf, and x = -inf gives 0.
+__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.0f + __expf(-x)); }
+
+__device__ __forceinline__ float silu_f(float x) { return x * sigmoid_f(x); }
 
 __device__ __forceinline__ float dsilu_f(float x)
 {
-    float sg = 1.0f / (1.0f + __expf(-x));
+    const float sg = sigmoid_f(x);
     return sg * (1.0f + x * (1.0f - sg));
 }
 

@@ -292,63 +292,81 @@ __device__ __forceinline__ void zero_row(uint32_t rb_hi, uint32_t rb_lo, uint32_
     }
 }
 
-// xv[k] = x[i0 + k] for k < MAXI from one row of x (values at or past `in`
-// read as 0; only the first n, n <= MAXI warp-uniform, are used by the caller).  With vec, the row is read as 16-byte vectors starting at the
-// aligned element below i0: a warp's lanes each read their own row, so every
-// load instruction costs one L1 sector lookup per lane, and one vector replaces
-// up to 8 (bf16) or 4 (fp32) scalar loads.  The window is then shifted into
-// place by the warp-uniform offset o = i0 mod (16 / sizeof(T)) through a small
-// select / funnel-shift network (no dynamically indexed registers).
+// A window of x[i0 .. i0 + MAXI) from one row of x, fetched in two steps so
+// that the load latency can hide behind other work: issue() starts the loads
+// into raw registers, values() shifts them into place (values at or past `in`
+// read as 0; only the first n, n <= MAXI warp-uniform, are used by the caller).
+// With vec, the row is read as 16-byte vectors starting at the aligned element
+// below i0: a warp's lanes each read their own row, so every load instruction
+// costs one L1 sector lookup per lane, and one vector replaces up to 8 (bf16)
+// or 4 (fp32) scalar loads.  The window is shifted into place by the
+// warp-uniform offset o = i0 mod (16 / sizeof(T)) through a small select /
+// funnel-shift network (no dynamically indexed registers).
 template <typename T, int MAXI>
-__device__ __forceinline__ void load_x_window(const T* __restrict__ row, int i0, int n, int in, bool vec,
-                                              float (&xv)[MAXI])
-{
-    constexpr int EPV = 16 / (int)sizeof(T);              // elements per 16-byte vector
-    constexpr int NV = (EPV - 1 + MAXI + EPV - 1) / EPV;  // vectors covering any window
-    if (!vec) {
+struct XWindow {
+    static constexpr int EPV = 16 / (int)sizeof(T);              // elements per 16-byte vector
+    static constexpr int NV = (EPV - 1 + MAXI + EPV - 1) / EPV;  // vectors covering any window
+    static constexpr int NR = 4 * NV + 4;
+    uint32_t raw[NR];
+    int o;                                                       // -1: raw already holds the values
+
+    __device__ __forceinline__ void issue(const T* __restrict__ row, int i0, int n, int in, bool vec)
+    {
+        if (!vec) {
+            o = -1;
 #pragma unroll
-        for (int k = 0; k < MAXI; ++k) xv[k] = (k < n && i0 + k < in) ? to_f(row[i0 + k]) : 0.0f;
-        return;
+            for (int k = 0; k < MAXI; ++k)
+                raw[k] = __float_as_uint((k < n && i0 + k < in) ? to_f(row[i0 + k]) : 0.0f);
+            return;
+        }
+        const int ia = i0 & ~(EPV - 1);
+        o = i0 - ia;                                             // 0 .. EPV-1, uniform across the warp
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            uint4 q = make_uint4(0u, 0u, 0u, 0u);
+            // (a vector holding none of the n values is skipped; in % EPV == 0)
+            if (v * EPV < o + n && ia + v * EPV < in) q = *reinterpret_cast<const uint4*>(row + ia + v * EPV);
+            raw[4 * v] = q.x;
+            raw[4 * v + 1] = q.y;
+            raw[4 * v + 2] = q.z;
+            raw[4 * v + 3] = q.w;
+        }
+#pragma unroll
+        for (int j = 4 * NV; j < NR; ++j) raw[j] = 0u;
     }
-    const int ia = i0 & ~(EPV - 1);
-    const int o = i0 - ia;                                  // 0 .. EPV-1, uniform across the warp
-    uint32_t raw[4 * NV + 4];
+
+    __device__ __forceinline__ void values(float (&xv)[MAXI]) const
+    {
+        if (o < 0) {
 #pragma unroll
-    for (int v = 0; v < NV; ++v) {
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        // (a vector holding none of the n values is skipped; in % EPV == 0)
-        if (v * EPV < o + n && ia + v * EPV < in) q = *reinterpret_cast<const uint4*>(row + ia + v * EPV);
-        raw[4 * v] = q.x;
-        raw[4 * v + 1] = q.y;
-        raw[4 * v + 2] = q.z;
-        raw[4 * v + 3] = q.w;
-    }
+            for (int k = 0; k < MAXI; ++k) xv[k] = __uint_as_float(raw[k]);
+            return;
+        }
+        if constexpr (sizeof(T) == 4) {
+            // shift by o words: two select levels
+            uint32_t t[NR - 2];
 #pragma unroll
-    for (int j = 4 * NV; j < 4 * NV + 4; ++j) raw[j] = 0u;
-    if constexpr (sizeof(T) == 4) {
-        // shift by o words: two select levels
-        uint32_t t[4 * NV + 2];
+            for (int j = 0; j < NR - 2; ++j) t[j] = (o & 1) ? raw[j + 1] : raw[j];
 #pragma unroll
-        for (int j = 0; j < 4 * NV + 2; ++j) t[j] = (o & 1) ? raw[j + 1] : raw[j];
+            for (int k = 0; k < MAXI; ++k) xv[k] = __uint_as_float((o & 2) ? t[k + 2] : t[k]);
+        } else {
+            // shift by o halves: o >> 1 words by two select levels, then o & 1 halves by a funnel shift
+            const int r = o >> 1;
+            uint32_t t[NR - 1], u[NR - 3];
 #pragma unroll
-        for (int k = 0; k < MAXI; ++k) xv[k] = __uint_as_float((o & 2) ? t[k + 2] : t[k]);
-    } else {
-        // shift by o halves: o >> 1 words by two select levels, then o & 1 halves by a funnel shift
-        const int r = o >> 1;
-        uint32_t t[4 * NV + 3], u[4 * NV + 1];
+            for (int j = 0; j < NR - 1; ++j) t[j] = (r & 1) ? raw[j + 1] : raw[j];
 #pragma unroll
-        for (int j = 0; j < 4 * NV + 3; ++j) t[j] = (r & 1) ? raw[j + 1] : raw[j];
+            for (int j = 0; j < NR - 3; ++j) u[j] = (r & 2) ? t[j + 2] : t[j];
+            const uint32_t sh = (uint32_t)(o & 1) * 16u;
 #pragma unroll
-        for (int j = 0; j < 4 * NV + 1; ++j) u[j] = (r & 2) ? t[j + 2] : t[j];
-        const uint32_t sh = (uint32_t)(o & 1) * 16u;
-#pragma unroll
-        for (int k = 0; k < MAXI; k += 2) {
-            const uint32_t w = __funnelshift_r(u[k / 2], u[k / 2 + 1], sh);
-            xv[k] = __uint_as_float(w << 16);
-            if (k + 1 < MAXI) xv[k + 1] = __uint_as_float(w & 0xFFFF0000u);
+            for (int k = 0; k < MAXI; k += 2) {
+                const uint32_t w = __funnelshift_r(u[k / 2], u[k / 2 + 1], sh);
+                xv[k] = __uint_as_float(w << 16);
+                if (k + 1 < MAXI) xv[k + 1] = __uint_as_float(w & 0xFFFF0000u);
+            }
         }
     }
-}
+};
 
 // One basis value at column `col` of a produced K-major row.
 template <int DT>
@@ -632,27 +650,29 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     const int c_end = min(kb * BK + BK, a.Kt);
                     return (int)__umulhi((uint32_t)(c_end - 1), a.nb_magic);
                 };
-                auto fetch = [&](int kb, float (&xv)[MAXI]) {
+                // the x window of the group's next k-block: loads issued one
+                // iteration ahead, shifted into place when that k-block starts
+                XWindow<T, MAXI> nxw;
+                nxw.o = -1;
+#pragma unroll
+                for (int j = 0; j < XWindow<T, MAXI>::NR; ++j) nxw.raw[j] = 0u;
+                auto fetch = [&](int kb) {
                     if (kb >= a.nkb_main || !row_ok) return;
                     const int i0 = first_input(kb);
-                    load_x_window<T, MAXI>(xrow, i0, last_input(kb) - i0 + 1, (int)a.in, a.x_vec != 0, xv);
+                    nxw.issue(xrow, i0, last_input(kb) - i0 + 1, (int)a.in, a.x_vec != 0);
                 };
-                float nxt[MAXI];
-#pragma unroll
-                for (int k = 0; k < MAXI; ++k) nxt[k] = 0.0f;
                 // At most sa_n groups: then a group's previous k-block is no older
                 // than the previous use of the A slot it waits for, so neither the
                 // aempty barrier nor any other can be two phases behind (a parity
                 // wait on such a barrier would pass early).
                 const int NG = min(Warps<MODE>::kGroups, sa_n);
-                if (grp < NG && grp < nk) fetch(kb_begin + grp, nxt);
+                if (grp < NG && grp < nk) fetch(kb_begin + grp);
                 int uses = 0;                               // k-blocks this group has filled
                 for (int it = grp; grp < NG && it < nk; it += NG, ++uses) {
                     float cur[MAXI];
-#pragma unroll
-                    for (int k = 0; k < MAXI; ++k) cur[k] = nxt[k];
+                    nxw.values(cur);
                     const int kb = kb_begin + it;
-                    if (it + NG < nk) fetch(kb + NG, nxt);
+                    if (it + NG < nk) fetch(kb + NG);
                     const int s = it % sa_n;
                     const uint32_t ph = (it / sa_n) & 1;
                     // the slot is free (its previous use consumed)
@@ -739,26 +759,26 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                       ? (int)__umulhi((uint32_t)(c_end - 1), a.nb_magic) - i_first + 1 : 0;
                 const float u0 = -a.lo * a.inv_h;
                 const float u_hi = (float)(a.G + 3);
-                auto fetch = [&](int kb, float (&xv)[MAXI]) {
+                XWindow<T, MAXI> nxw;   // (see the forward producer)
+                nxw.o = -1;
+#pragma unroll
+                for (int j = 0; j < XWindow<T, MAXI>::NR; ++j) nxw.raw[j] = 0u;
+                auto fetch = [&](int kb) {
                     const int64_t b = (int64_t)kb * BK + rb;
                     if (silu_tile || b >= a.batch) return;
-                    load_x_window<T, MAXI>(X + b * a.in, i_first, n_inp, (int)a.in, a.x_vec != 0, xv);
+                    nxw.issue(X + b * a.in, i_first, n_inp, (int)a.in, a.x_vec != 0);
                 };
                 // byte offset of column c (0..EPB-1) inside this thread's atom row
                 auto col_off = [&](int c) -> uint32_t {
                     return sw128_byte((uint32_t)rb, (uint32_t)c * 2u) - (uint32_t)rb * 128u;
                 };
-                float nxt[MAXI];
-#pragma unroll
-                for (int k = 0; k < MAXI; ++k) nxt[k] = 0.0f;
                 const int NG = min(Warps<MODE>::kGroups, sa_n);   // see the forward producer
-                if (grp < NG && grp < nk) fetch(kb_begin + grp, nxt);
+                if (grp < NG && grp < nk) fetch(kb_begin + grp);
                 for (int it = grp; grp < NG && it < nk; it += NG) {
                     float cur[MAXI];
-#pragma unroll
-                    for (int k = 0; k < MAXI; ++k) cur[k] = nxt[k];
+                    nxw.values(cur);
                     const int kb = kb_begin + it;
-                    if (it + NG < nk) fetch(kb + NG, nxt);
+                    if (it + NG < nk) fetch(kb + NG);
                     const int s = it % sa_n;
                     const uint32_t ph = (it / sa_n) & 1;
                     if (!acquire(s, ph)) break;
@@ -1347,31 +1367,54 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             inv_dc = 1.0f / (sc.d * sc.c);
             ext_mul = inv_dc * sc.x;
         }
-        for (int lt = 0; lt < my_tiles; ++lt) {
-            int64_t m0;
-            int i0;
+        // this lane's row and this warp's half of a tile's inputs
+        auto tile_part = [&](int lt, int64_t& m0, int& i0, int64_t& b, int& ia, int& ib) {
             tile_coords(lt, m0, i0);
-            const int64_t b = m0 + r;
-            const bool b_ok = b < a.batch;
+            b = m0 + r;
             const int i1 = min((int)a.in, i0 + a.n_in_tile);
-            const int kt_al = kt_start(i0);
-            // this warp's inputs: the first or second half of the tile's
             const int im = i0 + (i1 - i0 + 1) / 2;
-            const int ia = h ? im : i0, ib = h ? i1 : im;
-            const T* xrow = reinterpret_cast<const T*>(a.x) + (b_ok ? b : 0) * a.in;
-            const float* grow = a.gb ? a.gb + (b_ok ? b : 0) * a.in : nullptr;
-            // x (and dY.w_base) of the first inputs, ahead of the accumulator
-            float xa[XC], ga[XC];
-            auto xfetch = [&](int i_start) {
-                const int n = min(XC, ib - i_start);
-                if (b_ok && n > 0) {
-                    load_x_window<T, XC>(xrow, i_start, n, (int)a.in, x_vec, xa);
-                    if (grow) load_x_window<float, XC>(grow, i_start, n, (int)a.in, g_vec, ga);
-                }
-            };
+            ia = h ? im : i0;
+            ib = h ? i1 : im;
+        };
+        // x (and dY.w_base) windows: their loads are issued a chunk (across tiles,
+        // a tile) ahead and shifted into place when the chunk starts
+        XWindow<T, XC> xw;
+        XWindow<float, XC> gw;
+        xw.o = gw.o = -1;
 #pragma unroll
-            for (int k = 0; k < XC; ++k) xa[k] = ga[k] = 0.0f;
-            xfetch(ia);
+        for (int j = 0; j < XWindow<T, XC>::NR; ++j) xw.raw[j] = 0u;
+#pragma unroll
+        for (int j = 0; j < XWindow<float, XC>::NR; ++j) gw.raw[j] = 0u;
+        auto xfetch = [&](int64_t bq, int i_start, int i_end) {
+            const int n = min(XC, i_end - i_start);
+            if (bq < a.batch && n > 0) {
+                xw.issue(reinterpret_cast<const T*>(a.x) + bq * a.in, i_start, n, (int)a.in, x_vec);
+                if (a.gb) gw.issue(a.gb + bq * a.in, i_start, n, (int)a.in, g_vec);
+            }
+        };
+        if (my_tiles > 0) {
+            int64_t m0, b;
+            int i0, ia, ib;
+            tile_part(0, m0, i0, b, ia, ib);
+            xfetch(b, ia, ib);
+        }
+        for (int lt = 0; lt < my_tiles; ++lt) {
+            int64_t m0, b;
+            int i0, ia, ib;
+            tile_part(lt, m0, i0, b, ia, ib);
+            const bool b_ok = b < a.batch;
+            const int kt_al = kt_start(i0);
+            // the next tile's first window, issued when this tile's last chunk starts
+            // (exactly once per tile, also when this warp has no inputs in it)
+            bool prefetched = false;
+            auto prefetch_next = [&]() {
+                prefetched = true;
+                if (lt + 1 >= my_tiles) return;
+                int64_t m0n, bn;
+                int i0n, ian, ibn;
+                tile_part(lt + 1, m0n, i0n, bn, ian, ibn);
+                xfetch(bn, ian, ibn);
+            };
             const int buf = lt & 1;
             // The pair agrees on the bounded wait's outcome (so that both leave the
             // loop together, never one of them waiting at a named barrier for the
@@ -1445,12 +1488,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             if (b_ok) {
                 for (int ic = ia; ic < ib; ic += XC) {
                     float xc[XC], gc[XC];
-#pragma unroll
-                    for (int k = 0; k < XC; ++k) {
-                        xc[k] = xa[k];
-                        gc[k] = ga[k];
-                    }
-                    if (ic + XC < ib) xfetch(ic + XC);
+                    xw.values(xc);
+                    gw.values(gc);
+                    if (ic + XC < ib) xfetch(b, ic + XC, ib);
+                    else prefetch_next();
                     const int nkc = min(XC, ib - ic);     // inputs in this chunk
                     auto dx_of = [&](int k) -> float {
                         const int i = ic + k;
@@ -1499,6 +1540,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     }
                 }
             }
+            if (!prefetched) prefetch_next();
             __syncwarp();
             if (block_out && n_mine > 0) {
                 // element e of the warp's block is (row e / n_mine, input e % n_mine); a
