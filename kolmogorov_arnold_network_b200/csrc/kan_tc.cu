@@ -168,6 +168,8 @@ struct TcArgs {
     const unsigned int* amax;  // fp32: absolute maxima of the operands (scales_of)
     uint32_t nb_magic;         // ceil(2^32 / nb): c / nb == umulhi(c, nb_magic) for c < 2^32 / nb
     int fbox;                  // FWD: rows per B box
+    int pair;                  // FWD, DCA (bf16): CTA pairs sharing cta_group::2 MMAs
+    int m_tiles;               // FWD, DCA: M tiles holding work (a pair grid may have one more)
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
@@ -397,7 +399,12 @@ __device__ __forceinline__ void weights_fma(float t, float (&w)[4])
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <int MODE, int DT, int MAXI>
+// PAIR: two CTAs (a cluster of 2 x 1, adjacent M tiles along x) share each MMA
+// (tcgen05 cta_group::2, M = 256): each keeps its own 128 produced A rows and
+// holds half of the B tile, so each SM streams half the B bytes.  The leader
+// (rank 0) issues the MMAs; the follower's B loads complete on the leader's
+// barriers and its producers arrive there remotely; commits reach both CTAs.
+template <int MODE, int DT, int MAXI, bool PAIR = false>
 __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
               const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
@@ -411,6 +418,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     constexpr bool F32 = DT == KAN_F32;
     constexpr bool PRODUCE = MODE == FWD || MODE == DCA;
     constexpr bool A_BY_TMA = MODE == DX || MODE == GEMM;
+    static_assert(!PAIR || (PRODUCE && DT == KAN_BF16), "CTA pairs: bf16 forward and dcoef only");
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
     constexpr bool A_MN = MODE == DCA;               // producer-written MN-major basis
     constexpr bool A_SW32 = false;                   // (2-byte operands: the plain 128-byte swizzle)
     // B stored MN-major (dY for dcoef, coef / w_base for dx), for both dtypes
@@ -426,7 +436,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     // A arrives by TMA too (DX, GEMM) the two rings advance together (sa_n = stages).
     const int BN = a.BN, stages = a.stages;
     const int sa_n = PRODUCE ? a.stages_a : a.stages;
-    const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)BN * 128;
+    // (a CTA of a pair holds half of each N = 256 MMA's B rows)
+    const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)(PAIR ? BN / 2 : BN) * 128;
     const uint32_t a_stage = a_bytes * C::SPLIT, b_stage = b_bytes * C::SPLIT;
     const uint32_t sbase = smem_addr(smem);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sa_n * a_stage + stages * b_stage);
@@ -462,8 +473,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             mbar_init(empty(s), 1);         // the MMA thread's commit
         }
         for (int s = 0; s < sa_n; ++s) {
-            mbar_init(afull(s), 128);       // every thread of one producer group
-            mbar_init(aempty(s), 1);        // the MMA thread's commit
+            mbar_init(afull(s), PAIR ? 256 : 128);   // every thread of one producer group (of both CTAs)
+            mbar_init(aempty(s), 1);                 // the MMA thread's commit
         }
         mbar_init(seg_full(0), 1);
         mbar_init(seg_full(1), 1);
@@ -473,11 +484,17 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), tmem_cols);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_addr(tmem_slot), tmem_cols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_addr(tmem_slot), tmem_cols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // fp32 with BN <= 64: B_hi and B_lo sit back to back in a stage, so one N = 2*BN
@@ -489,8 +506,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     const uint32_t t_main0 = tmem, t_main1 = tmem + wseg, t_corr = tmem + 2u * wseg, t_total = t_corr + BN;
 
     // tile coordinates
-    const int64_t m0 = (int64_t)blockIdx.y * kBM;     // FWD/DX/GEMM: batch rows; DCA: see below
-    const int n0 = blockIdx.x * BN;                   // FWD/DCA/GEMM: output columns
+    // (a pair grid runs the M tiles along x: its clusters are 2 x 1)
+    const int tile_m = PAIR ? (int)blockIdx.x : (int)blockIdx.y;
+    const int tile_n = PAIR ? (int)blockIdx.y : (int)blockIdx.x;
+    const int64_t m0 = (int64_t)tile_m * kBM;         // FWD/DX/GEMM: batch rows; DCA: see below
+    const int n0 = tile_n * BN;                       // FWD/DCA/GEMM: output columns
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -509,6 +529,27 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             for (int it = 0; it < nk; ++it, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
                 if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
                 const int kb = kb_begin + it;
+                if constexpr (PAIR) {
+                    // this CTA's half of the B rows of each N = 256 MMA, landing on the
+                    // leader's full barrier (which expects both halves)
+                    const uint32_t fl = mapa_shared(full(s), 0);
+                    if (leader) mbar_arrive_expect_tx(full(s), 2u * b_bytes);
+                    const bool spline = kb < a.nkb_main;   // (FWD: then the SiLU k-blocks, w_base)
+                    for (int h = 0; 256 * h < BN; ++h) {
+                        if (MODE == FWD) {
+                            tma_load_2d_pair(B_hi(s) + (uint32_t)h * 128u * 128u,
+                                             spline ? (const void*)&tB_hi : (const void*)&tB2_hi, fl,
+                                             spline ? kb * BK : (kb - a.nkb_main) * BK, n0 + 256 * h + 128 * (int)rank);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 2; ++c)
+                                tma_load_2d_pair(B_hi(s) + (uint32_t)(2 * h + c) * BK * 128u, &tB_hi, fl,
+                                                 n0 + 256 * h + 128 * (int)rank + 64 * c, kb * BK);
+                        }
+                    }
+                    ++issued;
+                    continue;
+                }
                 const uint32_t bytes = (b_bytes + (A_BY_TMA ? a_bytes : 0u)) * C::SPLIT;
                 mbar_arrive_expect_tx(full(s), bytes);
                 if (MODE == FWD) {
@@ -542,21 +583,26 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 }
                 ++issued;
             }
-            // every load issued lands before the CTA can exit
-            for (int it = max(0, issued - stages); it < issued; ++it)
-                mbar_wait(full(it % stages), (it / stages) & 1, a.status);
+            // every load issued lands before the CTA can exit (a pair's follower
+            // sees that through its slots being released after the MMA used them)
+            for (int it = max(0, issued - stages); it < issued; ++it) {
+                if (PAIR && !leader) mbar_wait(empty(it % stages), (it / stages) & 1, a.status);
+                else mbar_wait(full(it % stages), (it / stages) & 1, a.status);
+            }
         }
     } else if (warp == 1) {
         // ---------------- MMA issue ----------------
-        if (lane == 0 && nk > 0) {
+        if (lane == 0 && nk > 0 && leader) {
             // a 384- or 512-wide bf16 tile runs as an N=256 MMA plus an N=BN-256 MMA
             // into consecutive TMEM columns
             const int mma_n = BN > 256 ? 256 : BN;
             const uint32_t idesc = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, mma_n);
             const uint32_t idesc2 = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, BN > 256 ? BN - 256 : 16);
             const uint32_t idesc_w = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, merged ? 2 * BN : 16);
-            // offset of B's columns 256..: 256 rows (K-major) or four 64-column atoms (MN-major)
-            const uint32_t b_half = B_MN ? 4u * BK * 128u : 256u * 128u;
+            // offset of B's columns 256..: 256 rows (K-major) or four 64-column atoms (MN-major);
+            // a pair's CTA holds half of each: 128 rows or two atoms
+            const uint32_t b_half = B_MN ? (PAIR ? 2u : 4u) * BK * 128u : (PAIR ? 128u : 256u) * 128u;
+            const uint32_t idesc_p = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, 2 * kBM, 256);
             const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
             const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
             const uint32_t a_lbo = A_MN ? (uint32_t)BK * 128u : 16u;
@@ -567,8 +613,14 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             int s = 0, sa = 0;            // B and A ring positions (equal when A arrives by TMA)
             uint32_t ph = 0, pha = 0;
             for (int it = 0; it < nk; ++it) {
-                if (!mbar_wait(full(s), ph, a.status)) { ok = false; break; }
-                if (PRODUCE && !mbar_wait(afull(sa), pha, a.status)) { ok = false; break; }
+                if (PAIR) {
+                    // (the follower's bytes and producer arrivals land here from the other CTA)
+                    if (!mbar_wait_cluster(full(s), ph, a.status)) { ok = false; break; }
+                    if (!mbar_wait_cluster(afull(sa), pha, a.status)) { ok = false; break; }
+                } else {
+                    if (!mbar_wait(full(s), ph, a.status)) { ok = false; break; }
+                    if (PRODUCE && !mbar_wait(afull(sa), pha, a.status)) { ok = false; break; }
+                }
                 const int g = F32 ? it / kSegKb : 0;
                 const bool seg_start = F32 && (it % kSegKb == 0);
                 if (seg_start && g >= 2 && !mbar_wait(seg_empty(g & 1), ((g >> 1) - 1) & 1, a.status)) {
@@ -588,7 +640,13 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t ad = ad0 + (uint64_t)((ks * a_step) >> 4);
                     const uint64_t bd = bd0 + (uint64_t)((ks * b_step) >> 4);
-                    if constexpr (!F32) {
+                    if constexpr (PAIR) {
+                        mma_f16_ss_pair(t_main0, ad, bd, idesc_p, (it > 0 || ks > 0) ? 1u : 0u);
+                        if (BN > 256) {
+                            const uint64_t bd2 = bd0 + (uint64_t)((b_half + ks * b_step) >> 4);
+                            mma_f16_ss_pair(t_main0 + 256u, ad, bd2, idesc_p, (it > 0 || ks > 0) ? 1u : 0u);
+                        }
+                    } else if constexpr (!F32) {
                         mma_bf16_ss(t_main0, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
                         if (BN > 256) {
                             const uint64_t bd2 = bd0 + (uint64_t)((b_half + ks * b_step) >> 4);
@@ -606,8 +664,13 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         mma_bf16_ss(t_main, ad, bd, idesc, (!seg_start || ks > 0) ? 1u : 0u);
                     }
                 }
-                mma_commit(empty(s));
-                if (PRODUCE) mma_commit(aempty(sa));
+                if constexpr (PAIR) {
+                    mma_commit_pair(empty(s));
+                    mma_commit_pair(aempty(sa));
+                } else {
+                    mma_commit(empty(s));
+                    if (PRODUCE) mma_commit(aempty(sa));
+                }
                 if (F32 && ((it + 1) % kSegKb == 0 || it + 1 == nk)) mma_commit(seg_full(g & 1));
                 if (++s == stages) {
                     s = 0;
@@ -618,7 +681,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     pha ^= 1;
                 }
             }
-            if (ok) mma_commit(accum_bar);
+            if (ok) {
+                if constexpr (PAIR) mma_commit_pair(accum_bar);
+                else mma_commit(accum_bar);
+            }
         }
     } else if (warp < Warps<MODE>::kEpi0) {
         // ---------------- A producers ----------------
@@ -737,7 +803,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                     fence_async_smem();
-                    mbar_arrive(afull(s));
+                    if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(afull(s), 0));
+                    else mbar_arrive(afull(s));
                 }
                 (void)uses;
             } else if constexpr (MODE == DCA) {
@@ -750,8 +817,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const int grp = p >> 7;                    // warp-uniform
                 const int rb = p % BK;
                 const int atom = (p / BK) % NATOM;         // warp-uniform
-                const int mt = blockIdx.y;
-                const bool silu_tile = mt >= a.n_kt_tiles;
+                const int mt = tile_m;
+                // (the padding tile of a pair grid: all spline columns past Kt, so zero)
+                const bool silu_tile = mt >= a.n_kt_tiles && mt < a.m_tiles;
                 const int c_lo = (silu_tile ? (mt - a.n_kt_tiles) * kBM : mt * kBM) + atom * EPB;
                 const int c_end = silu_tile ? min(c_lo + EPB, (int)a.in) : min(c_lo + EPB, a.Kt);
                 const int i_first = (int)__umulhi((uint32_t)c_lo, a.nb_magic);
@@ -867,7 +935,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                     fence_async_smem();
-                    mbar_arrive(afull(s));
+                    if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(afull(s), 0));
+                    else mbar_arrive(afull(s));
                 }
             }
         }
@@ -1014,10 +1083,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 }
             } else if constexpr (MODE == DCA) {
                 // rows are spline columns kt (or inputs of a SiLU tile); columns are outputs j
-                const int mt = blockIdx.y;
+                const int mt = tile_m;
                 const bool base_tile = mt >= a.n_kt_tiles;
                 const int64_t rowg = base_tile ? (int64_t)(mt - a.n_kt_tiles) * kBM + r : (int64_t)mt * kBM + r;
-                const bool row_ok = base_tile ? rowg < a.in : rowg < a.Kt;
+                const bool row_ok = mt < a.m_tiles && (base_tile ? rowg < a.in : rowg < a.Kt);
                 float* dst;
                 int64_t ld;
                 if (a.partial) {
@@ -1120,9 +1189,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // neither CTA leaves while the pair's MMAs or arrivals may touch it
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, tmem_cols);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem, tmem_cols);
+        else tmem_dealloc(tmem, tmem_cols);
     }
 }
 
@@ -1838,6 +1909,8 @@ struct Plan {
     int64_t Kx;
     // forward
     int f_BN, f_stages, f_stages_a, f_n, f_m, f_splits, f_kps, f_nkb_main, f_nkb_total;
+    bool f_pair, d_pair;   // bf16 tiles of 256 or 512 columns: CTA pairs (f_my / d_my M tiles, even, along x)
+    int f_my, d_my;
     // dcoef
     int d_BN, d_stages, d_stages_a, d_n, d_m, d_nkt, d_splits, d_kps, d_nkb;
     int64_t d_ld;
@@ -1862,9 +1935,11 @@ Plan make_plan(const Problem& p, int sms)
     const bool sep_silu = p.base && !P.ext;   // separate SiLU k-blocks / tiles / GEMM
     // forward: M = batch, N = out, K = spline (+ SiLU) columns
     P.f_BN = f32 ? bn_for(p.out, true) : wide_bn(p.out);
-    stages_ab(P.f_BN, f32, P.f_stages, P.f_stages_a);
+    P.f_pair = !f32 && (P.f_BN == 256 || P.f_BN == 512);
+    stages_ab(P.f_pair ? P.f_BN / 2 : P.f_BN, f32, P.f_stages, P.f_stages_a);
     P.f_n = (int)cdiv(p.out, P.f_BN);
     P.f_m = (int)cdiv(p.batch, kBM);
+    P.f_my = P.f_pair ? (P.f_m + 1) / 2 * 2 : P.f_m;
     P.f_nkb_main = (int)cdiv(P.Kx, BK);
     P.f_nkb_total = P.f_nkb_main + (sep_silu ? (int)cdiv(p.in, BK) : 0);
     {
@@ -1876,10 +1951,12 @@ Plan make_plan(const Problem& p, int sms)
     P.f_splits = (int)cdiv(P.f_nkb_total, P.f_kps);
     // dcoef: M = spline columns (+ SiLU rows), N = out, K = batch
     P.d_BN = f32 ? bn_for(p.out, true, true) : std::max(64, wide_bn(p.out));
+    P.d_pair = !f32 && (P.d_BN == 256 || P.d_BN == 512);
     P.d_n = (int)cdiv(p.out, P.d_BN);
     P.d_nkt = (int)cdiv(P.Kx, kBM);
     P.d_m = P.d_nkt + (sep_silu ? (int)cdiv(p.in, kBM) : 0);
-    stages_ab(P.d_BN, f32, P.d_stages, P.d_stages_a);
+    P.d_my = P.d_pair ? (P.d_m + 1) / 2 * 2 : P.d_m;
+    stages_ab(P.d_pair ? P.d_BN / 2 : P.d_BN, f32, P.d_stages, P.d_stages_a);
     P.d_nkb = (int)cdiv(p.batch, BK);
     {
         const int64_t tiles = (int64_t)P.d_n * P.d_m;
@@ -1971,7 +2048,7 @@ Plan make_plan(const Problem& p, int sms)
 
 inline int grid_for(int64_t n) { return (int)std::min<int64_t>(std::max<int64_t>(1, (n + 255) / 256), 148 * 8); }
 
-template <int MODE, int DT, int MAXI>
+template <int MODE, int DT, int MAXI, bool PAIR>
 cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args, cudaStream_t st)
 {
     constexpr bool produce = MODE == FWD || MODE == DCA;
@@ -1982,23 +2059,55 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
         (DT == KAN_F32 && BN > 128) || stages < 2 || stages_a < 2 || stages + stages_a > 24 ||
         (!produce && stages_a != stages))
         return cudaErrorInvalidConfiguration;
-    const int smem = smem_bytes(BN, stages, stages_a, DT == KAN_F32);
+    // a pair's CTAs hold half of each N = 256 MMA's B rows; the grid is (M tiles, N tiles, splits)
+    if (PAIR && ((BN != 256 && BN != 512) || grid.x % 2 != 0)) return cudaErrorInvalidConfiguration;
+    const int smem = smem_bytes(PAIR ? BN / 2 : BN, stages, stages_a, DT == KAN_F32);
     if (smem > kSmemBudget) return cudaErrorInvalidConfiguration;
     static int configured = 0;   // per instantiation; the attribute is per function
     if (configured < smem) {
-        cudaError_t e = cudaFuncSetAttribute(tc_kernel<MODE, DT, MAXI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemBudget);
+        cudaError_t e = cudaFuncSetAttribute(tc_kernel<MODE, DT, MAXI, PAIR>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
         if (e != cudaSuccess) return e;
         configured = kSmemBudget;
     }
-    tc_kernel<MODE, DT, MAXI><<<grid, Warps<MODE>::kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                                          maps[5], args);
-    count_launch();
+    if constexpr (PAIR) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(Warps<MODE>::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, tc_kernel<MODE, DT, MAXI, true>, maps[0], maps[1], maps[2], maps[3],
+                                           maps[4], maps[5], args);
+        count_launch();
+        if (e != cudaSuccess) return e;
+    } else {
+        tc_kernel<MODE, DT, MAXI, false><<<grid, Warps<MODE>::kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3],
+                                                                                    maps[4], maps[5], args);
+        count_launch();
+    }
     return cudaGetLastError();
 }
 
 // Inputs a row of one forward k-block can touch: (BK - 1) / nb + 2.
 int fwd_maxi_needed(int nb, bool f32) { return (64 - 1) / nb + 2; (void)f32; }
+
+template <int MODE, int MAXI>
+cudaError_t launch_m(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
+                     cudaStream_t st)
+{
+    if (f32) return launch<MODE, KAN_F32, MAXI, false>(grid, BN, stages, maps, args, st);
+    if constexpr (MODE == FWD || MODE == DCA) {
+        if (args.pair) return launch<MODE, KAN_BF16, MAXI, true>(grid, BN, stages, maps, args, st);
+    }
+    return launch<MODE, KAN_BF16, MAXI, false>(grid, BN, stages, maps, args, st);
+}
 
 template <int MODE>
 cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
@@ -2006,22 +2115,13 @@ cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap
 {
     if constexpr (MODE == FWD || MODE == DCA) {
         const int need = fwd_maxi_needed(args.nb, f32);
-        if (need <= 4)
-            return f32 ? launch<MODE, KAN_F32, 4>(grid, BN, stages, maps, args, st)
-                       : launch<MODE, KAN_BF16, 4>(grid, BN, stages, maps, args, st);
-        if (need <= 7)
-            return f32 ? launch<MODE, KAN_F32, 7>(grid, BN, stages, maps, args, st)
-                       : launch<MODE, KAN_BF16, 7>(grid, BN, stages, maps, args, st);
-        if (need <= 9)
-            return f32 ? launch<MODE, KAN_F32, 9>(grid, BN, stages, maps, args, st)
-                       : launch<MODE, KAN_BF16, 9>(grid, BN, stages, maps, args, st);
-        if (need <= 17)
-            return f32 ? launch<MODE, KAN_F32, 17>(grid, BN, stages, maps, args, st)
-                       : launch<MODE, KAN_BF16, 17>(grid, BN, stages, maps, args, st);
+        if (need <= 4) return launch_m<MODE, 4>(f32, grid, BN, stages, maps, args, st);
+        if (need <= 7) return launch_m<MODE, 7>(f32, grid, BN, stages, maps, args, st);
+        if (need <= 9) return launch_m<MODE, 9>(f32, grid, BN, stages, maps, args, st);
+        if (need <= 17) return launch_m<MODE, 17>(f32, grid, BN, stages, maps, args, st);
         return cudaErrorInvalidConfiguration;   // G >= 1 keeps need <= 17
     } else {
-        return f32 ? launch<MODE, KAN_F32, 1>(grid, BN, stages, maps, args, st)
-                   : launch<MODE, KAN_BF16, 1>(grid, BN, stages, maps, args, st);
+        return launch_m<MODE, 1>(f32, grid, BN, stages, maps, args, st);
     }
 }
 
@@ -2198,7 +2298,10 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
     a.nkb_total = P.f_nkb_total;
     a.kb_per_split = P.f_kps;
     a.partial = P.f_splits > 1;
-    e = launch_dt<FWD>(f32, dim3(P.f_n, P.f_m, P.f_splits), P.f_BN, P.f_stages, maps, a, st);
+    a.pair = P.f_pair ? 1 : 0;
+    a.m_tiles = P.f_m;
+    const dim3 fgrid = P.f_pair ? dim3(P.f_my, P.f_n, P.f_splits) : dim3(P.f_n, P.f_m, P.f_splits);
+    e = launch_dt<FWD>(f32, fgrid, P.f_BN, P.f_stages, maps, a, st);
     if (e != cudaSuccess) return e;
     if (P.f_splits > 1) {
         const int64_t n = p.batch * p.out;
@@ -2263,7 +2366,9 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         a.partial = P.d_splits > 1;
         a.out = a.partial ? (void*)partbuf : (void*)dcoef;   // a skipped output is simply not stored
         a.out2 = dw_base;
-        const dim3 grid(P.d_n, P.d_m, P.d_splits);
+        a.pair = P.d_pair ? 1 : 0;
+        a.m_tiles = P.d_m;
+        const dim3 grid = P.d_pair ? dim3(P.d_my, P.d_n, P.d_splits) : dim3(P.d_n, P.d_m, P.d_splits);
         e = launch_dt<DCA>(f32, grid, P.d_BN, P.d_stages, maps, a, st);
         if (e != cudaSuccess) return e;
         if (a.partial) {

@@ -99,6 +99,9 @@ SMALL = [
     (130, 16, 48, 50, -1.0, 1.0, False),
     (200, 32, 520, 5, -3.0, 3.0, True),
     (129, 8, 16, 8, -1.0, 1.0, True),
+    # wide bf16 tiles run as CTA pairs: odd M-tile counts (a padding tile), ragged N
+    (300, 32, 1000, 8, -1.0, 1.0, False),
+    (300, 16, 256, 8, -1.0, 1.0, True),
 ]
 
 
