@@ -530,22 +530,23 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 if (!mbar_wait(empty(s), ph ^ 1, a.status)) break;
                 const int kb = kb_begin + it;
                 if constexpr (PAIR) {
-                    // this CTA's half of the B rows of each N = 256 MMA, landing on the
-                    // leader's full barrier (which expects both halves)
+                    // this CTA's half of the B columns of each MMA (N = 256, then N = BN - 256),
+                    // landing on the leader's full barrier (which expects both halves): local
+                    // column lc < 128 is tile column 128 * rank + lc, the rest 256 + h2 * rank + lc - 128
                     const uint32_t fl = mapa_shared(full(s), 0);
                     if (leader) mbar_arrive_expect_tx(full(s), 2u * b_bytes);
-                    const bool spline = kb < a.nkb_main;   // (FWD: then the SiLU k-blocks, w_base)
-                    for (int h = 0; 256 * h < BN; ++h) {
-                        if (MODE == FWD) {
-                            tma_load_2d_pair(B_hi(s) + (uint32_t)h * 128u * 128u,
+                    const int h2 = (BN - 256) / 2;
+                    auto tile_col = [&](int lc) { return lc < 128 ? 128 * (int)rank + lc : 256 + h2 * (int)rank + lc - 128; };
+                    if (MODE == FWD) {
+                        const bool spline = kb < a.nkb_main;   // (then the SiLU k-blocks, w_base)
+                        for (int lc = 0; lc < BN / 2; lc += a.fbox)
+                            tma_load_2d_pair(B_hi(s) + (uint32_t)lc * 128u,
                                              spline ? (const void*)&tB_hi : (const void*)&tB2_hi, fl,
-                                             spline ? kb * BK : (kb - a.nkb_main) * BK, n0 + 256 * h + 128 * (int)rank);
-                        } else {
-#pragma unroll
-                            for (int c = 0; c < 2; ++c)
-                                tma_load_2d_pair(B_hi(s) + (uint32_t)(2 * h + c) * BK * 128u, &tB_hi, fl,
-                                                 n0 + 256 * h + 128 * (int)rank + 64 * c, kb * BK);
-                        }
+                                             spline ? kb * BK : (kb - a.nkb_main) * BK, n0 + tile_col(lc));
+                    } else {
+                        for (int lc = 0; lc < BN / 2; lc += EPB)   // 64-column atoms
+                            tma_load_2d_pair(B_hi(s) + (uint32_t)(lc / EPB) * BK * 128u, &tB_hi, fl, n0 + tile_col(lc),
+                                             kb * BK);
                     }
                     ++issued;
                     continue;
@@ -600,9 +601,10 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
             const uint32_t idesc2 = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, BN > 256 ? BN - 256 : 16);
             const uint32_t idesc_w = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, kBM, merged ? 2 * BN : 16);
             // offset of B's columns 256..: 256 rows (K-major) or four 64-column atoms (MN-major);
-            // a pair's CTA holds half of each: 128 rows or two atoms
+            // a pair's CTA holds 128 of the first 256: 128 rows or two atoms
             const uint32_t b_half = B_MN ? (PAIR ? 2u : 4u) * BK * 128u : (PAIR ? 128u : 256u) * 128u;
             const uint32_t idesc_p = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, 2 * kBM, 256);
+            const uint32_t idesc_p2 = instr_desc(C::FMT, A_MN ? 1u : 0u, B_MN ? 1u : 0u, 2 * kBM, BN > 256 ? BN - 256 : 16);
             const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
             const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
             const uint32_t a_lbo = A_MN ? (uint32_t)BK * 128u : 16u;
@@ -644,7 +646,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         mma_f16_ss_pair(t_main0, ad, bd, idesc_p, (it > 0 || ks > 0) ? 1u : 0u);
                         if (BN > 256) {
                             const uint64_t bd2 = bd0 + (uint64_t)((b_half + ks * b_step) >> 4);
-                            mma_f16_ss_pair(t_main0 + 256u, ad, bd2, idesc_p, (it > 0 || ks > 0) ? 1u : 0u);
+                            mma_f16_ss_pair(t_main0 + 256u, ad, bd2, idesc_p2, (it > 0 || ks > 0) ? 1u : 0u);
                         }
                     } else if constexpr (!F32) {
                         mma_bf16_ss(t_main0, ad, bd, idesc, (it > 0 || ks > 0) ? 1u : 0u);
@@ -1909,7 +1911,7 @@ struct Plan {
     int64_t Kx;
     // forward
     int f_BN, f_stages, f_stages_a, f_n, f_m, f_splits, f_kps, f_nkb_main, f_nkb_total;
-    bool f_pair, d_pair;   // bf16 tiles of 256 or 512 columns: CTA pairs (f_my / d_my M tiles, even, along x)
+    bool f_pair, d_pair;   // bf16 tiles of 256, 384 or 512 columns: CTA pairs (f_my / d_my M tiles, even, along x)
     int f_my, d_my;
     // dcoef
     int d_BN, d_stages, d_stages_a, d_n, d_m, d_nkt, d_splits, d_kps, d_nkb;
@@ -1935,7 +1937,7 @@ Plan make_plan(const Problem& p, int sms)
     const bool sep_silu = p.base && !P.ext;   // separate SiLU k-blocks / tiles / GEMM
     // forward: M = batch, N = out, K = spline (+ SiLU) columns
     P.f_BN = f32 ? bn_for(p.out, true) : wide_bn(p.out);
-    P.f_pair = !f32 && (P.f_BN == 256 || P.f_BN == 512);
+    P.f_pair = !f32 && P.f_BN >= 256;
     stages_ab(P.f_pair ? P.f_BN / 2 : P.f_BN, f32, P.f_stages, P.f_stages_a);
     P.f_n = (int)cdiv(p.out, P.f_BN);
     P.f_m = (int)cdiv(p.batch, kBM);
@@ -1951,7 +1953,7 @@ Plan make_plan(const Problem& p, int sms)
     P.f_splits = (int)cdiv(P.f_nkb_total, P.f_kps);
     // dcoef: M = spline columns (+ SiLU rows), N = out, K = batch
     P.d_BN = f32 ? bn_for(p.out, true, true) : std::max(64, wide_bn(p.out));
-    P.d_pair = !f32 && (P.d_BN == 256 || P.d_BN == 512);
+    P.d_pair = !f32 && P.d_BN >= 256;
     P.d_n = (int)cdiv(p.out, P.d_BN);
     P.d_nkt = (int)cdiv(P.Kx, kBM);
     P.d_m = P.d_nkt + (sep_silu ? (int)cdiv(p.in, kBM) : 0);
@@ -2060,7 +2062,9 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
         (!produce && stages_a != stages))
         return cudaErrorInvalidConfiguration;
     // a pair's CTAs hold half of each N = 256 MMA's B rows; the grid is (M tiles, N tiles, splits)
-    if (PAIR && ((BN != 256 && BN != 512) || grid.x % 2 != 0)) return cudaErrorInvalidConfiguration;
+    if (PAIR && (BN < 256 || BN % 128 != 0 || (MODE == FWD && args.fbox != (BN == 384 ? 64 : 128)) ||
+                 grid.x % 2 != 0))
+        return cudaErrorInvalidConfiguration;
     const int smem = smem_bytes(PAIR ? BN / 2 : BN, stages, stages_a, DT == KAN_F32);
     if (smem > kSmemBudget) return cudaErrorInvalidConfiguration;
     static int configured = 0;   // per instantiation; the attribute is per function
@@ -2272,7 +2276,8 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
             return e;
     }
     CUtensorMap maps[6];
-    const int fbox = std::min(P.f_BN, 128);
+    // (a pair's CTA loads 128 + (BN - 256) / 2 rows of each B tile: boxes of 64 rows for BN = 384)
+    const int fbox = P.f_pair && P.f_BN == 384 ? 64 : std::min(P.f_BN, 128);
     if (!make_map_2d(&maps[2], c_hi, f32, p.out, P.Kx, fbox, BK, detail) ||
         !make_map_2d(&maps[3], c_lo, f32, p.out, P.Kx, fbox, BK, detail))
         return cudaErrorInvalidValue;

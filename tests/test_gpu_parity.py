@@ -102,6 +102,7 @@ SMALL = [
     # wide bf16 tiles run as CTA pairs: odd M-tile counts (a padding tile), ragged N
     (300, 32, 1000, 8, -1.0, 1.0, False),
     (300, 16, 256, 8, -1.0, 1.0, True),
+    (300, 8, 696, 20, -1.0, 1.0, True),
 ]
 
 
