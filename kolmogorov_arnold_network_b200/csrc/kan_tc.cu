@@ -1207,6 +1207,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
 // 2-9 epilogue (two per TMEM lane quarter).  fp32 keeps the fp16 correction
 // products in a second accumulator per buffer; the contraction over `out`
 // is short enough (at most 32 k-blocks) that no promotion is needed.
+// PAIR (bf16): clusters of two CTAs walk the same tiles of 256 batch rows; the
+// leader issues cta_group::2 MMAs (M = 256) over both CTAs' dY rows and the two
+// halves of the B columns, one held by each CTA, so each SM streams half of B;
+// commits reach both CTAs and both CTAs' epilogues release the leader's
+// accumulator buffers.
 // ---------------------------------------------------------------------------
 constexpr int kDxThreads = 320;   // warps: 0 TMA, 1 MMA, 2-9 epilogue
 
@@ -1226,9 +1231,10 @@ struct DxArgs {
     const unsigned int* amax; // fp32: absolute maxima of the operands (scales_of)
     int a_res;                // 1: short contraction (nkb k-blocks of dY fit beside the B ring): each
                               // CTA walks a contiguous run of tiles and keeps the dY rows resident
+    int pair;                 // (informational) tiles of 2 x 128 batch rows run by CTA pairs
 };
 
-template <int DT>
+template <int DT, bool PAIR>
 __global__ void __launch_bounds__(kDxThreads, 1)
     dx_persistent_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
                          const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
@@ -1240,12 +1246,19 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     constexpr int EPB = 128 / C::ESZ;
     constexpr bool F32 = DT == KAN_F32;
     constexpr bool B_MN = true;          // coef (its fp16 hi/lo copies for fp32) MN-major
+    static_assert(!PAIR || DT == KAN_BF16, "CTA pairs: bf16 only");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    // the walk's units: clusters (PAIR) or CTAs
+    const int unit = PAIR ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
+    const int n_units = PAIR ? (int)gridDim.x >> 1 : (int)gridDim.x;
 
     const int BN = a.BN, stages = a.stages;
     const bool ares = a.a_res != 0;
-    const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)BN * 128;
+    // (a pair's CTA holds half of the B columns: BN / 2, whole 64-column atoms)
+    const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)(PAIR ? BN / 2 : BN) * 128;
     const uint32_t a_stage = a_bytes * C::SPLIT, b_stage = b_bytes * C::SPLIT;
     const uint32_t stage_bytes = a_stage + b_stage;
     const uint32_t sbase = smem_addr(smem);
@@ -1280,30 +1293,36 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         }
         mbar_init(acc_full(0), 1);
         mbar_init(acc_full(1), 1);
-        mbar_init(acc_empty(0), 256);   // every epilogue thread
-        mbar_init(acc_empty(1), 256);
+        mbar_init(acc_empty(0), PAIR ? 16 : 8);   // every epilogue warp (of both CTAs)
+        mbar_init(acc_empty(1), PAIR ? 16 : 8);
         mbar_init(a_full, 1);           // resident dY rows landed (TMA bytes)
         mbar_init(a_empty, 1);          // the MMA is done with them (commit)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_slot), 512);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_addr(tmem_slot), 512);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_addr(tmem_slot), 512);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // tiles of this CTA: t = blockIdx.x + k * gridDim.x, or (resident dY) the
-    // contiguous run [t_begin, t_end); (batch tile, input group) = (t / n_tiles_n, t % n_tiles_n)
-    const int t_begin = (int)((int64_t)a.n_tiles * blockIdx.x / gridDim.x);
-    const int t_end = (int)((int64_t)a.n_tiles * (blockIdx.x + 1) / gridDim.x);
-    const int my_tiles = ares ? t_end - t_begin
-                              : (a.n_tiles > (int)blockIdx.x ? (a.n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0);
-    auto tile_of = [&](int lt) { return ares ? t_begin + lt : (int)blockIdx.x + lt * (int)gridDim.x; };
+    // tiles of this unit: t = unit + k * n_units, or (resident dY) the contiguous
+    // run [t_begin, t_end); (batch tile, input group) = (t / n_tiles_n, t % n_tiles_n),
+    // a batch tile being 128 rows, or 256 for a pair (rows 128 * rank.. of it here)
+    const int t_begin = (int)((int64_t)a.n_tiles * unit / n_units);
+    const int t_end = (int)((int64_t)a.n_tiles * (unit + 1) / n_units);
+    const int my_tiles = ares ? t_end - t_begin : (a.n_tiles > unit ? (a.n_tiles - 1 - unit) / n_units + 1 : 0);
+    auto tile_of = [&](int lt) { return ares ? t_begin + lt : unit + lt * n_units; };
     auto tile_coords = [&](int lt, int64_t& m0, int& i0) {
         const int t = tile_of(lt);
-        m0 = (int64_t)(t / a.n_tiles_n) * kBM;
+        m0 = (int64_t)(t / a.n_tiles_n) * (PAIR ? 2 * kBM : kBM) + (int64_t)kBM * rank;
         i0 = (t % a.n_tiles_n) * a.n_in_tile;
     };
     auto kt_start = [&](int i0) {
@@ -1328,16 +1347,34 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                 if (ares && m0 != a_m) {
                     // new batch tile: once the MMA is done with the previous rows, load these
                     if (a_loads > 0 && !mbar_wait(a_empty, (a_loads - 1) & 1, a.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(a_full, a.nkb * a_stage);
-                    for (int kb = 0; kb < a.nkb; ++kb) {
-                        tma_load_2d(A_hi(kb), &tA_hi, a_full, kb * BK, (int)m0);
-                        if (F32) tma_load_2d(A_lo(kb), &tA_lo, a_full, kb * BK, (int)m0);
+                    if constexpr (PAIR) {
+                        // both CTAs' rows complete on the leader's barrier
+                        const uint32_t af = mapa_shared(a_full, 0);
+                        if (leader) mbar_arrive_expect_tx(a_full, 2u * a.nkb * a_stage);
+                        for (int kb = 0; kb < a.nkb; ++kb) tma_load_2d_pair(A_hi(kb), &tA_hi, af, kb * BK, (int)m0);
+                    } else {
+                        mbar_arrive_expect_tx(a_full, a.nkb * a_stage);
+                        for (int kb = 0; kb < a.nkb; ++kb) {
+                            tma_load_2d(A_hi(kb), &tA_hi, a_full, kb * BK, (int)m0);
+                            if (F32) tma_load_2d(A_lo(kb), &tA_lo, a_full, kb * BK, (int)m0);
+                        }
                     }
                     ++a_loads;
                     a_m = m0;
                 }
                 for (int kb = 0; kb < a.nkb; ++kb, ++g, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
                     if (!mbar_wait(empty(s), ph ^ 1, a.status)) { ok = false; break; }
+                    if constexpr (PAIR) {
+                        // this CTA's rows of dY and its half of the B columns (BN / 2 * rank..),
+                        // landing on the leader's full barrier, which expects both CTAs' bytes
+                        const uint32_t fl = mapa_shared(full(s), 0);
+                        if (leader) mbar_arrive_expect_tx(full(s), 2u * (ares ? b_stage : stage_bytes));
+                        if (!ares) tma_load_2d_pair(A_hi(s), &tA_hi, fl, kb * BK, (int)m0);
+                        for (int c = 0; c < BN / 2 / EPB; ++c)
+                            tma_load_2d_pair(B_hi(s) + (uint32_t)c * BK * 128, &tB_hi, fl,
+                                             kt0 + BN / 2 * (int)rank + c * EPB, kb * BK);
+                        continue;
+                    }
                     mbar_arrive_expect_tx(full(s), ares ? b_stage : stage_bytes);
                     if (!ares) {
                         tma_load_2d(A_hi(s), &tA_hi, full(s), kb * BK, (int)m0);
@@ -1355,12 +1392,27 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     }
                 }
             }
-            for (int q = max(0, g - stages); q < g; ++q) mbar_wait(full(q % stages), (q / stages) & 1, a.status);
-            if (a_loads > 0) mbar_wait(a_full, (a_loads - 1) & 1, a.status);
+            // every load issued lands before the CTA can exit (a pair's follower sees
+            // that through the MMA's releases of its slots and of its resident rows)
+            if (PAIR && !leader) {
+                for (int q = max(0, g - stages); q < g; ++q) mbar_wait(empty(q % stages), (q / stages) & 1, a.status);
+                if (a_loads > 0) mbar_wait(a_empty, (a_loads - 1) & 1, a.status);
+            } else {
+                for (int q = max(0, g - stages); q < g; ++q) mbar_wait(full(q % stages), (q / stages) & 1, a.status);
+                if (a_loads > 0) mbar_wait(a_full, (a_loads - 1) & 1, a.status);
+            }
         }
     } else if (warp == 1) {
-        if (lane == 0 && my_tiles > 0) {
-            const uint32_t idesc = instr_desc(C::FMT, 0, B_MN ? 1u : 0u, kBM, BN);
+        if (lane == 0 && my_tiles > 0 && leader) {
+            const uint32_t idesc = instr_desc(C::FMT, 0, B_MN ? 1u : 0u, PAIR ? 2 * kBM : kBM, BN);
+            // (a pair's waits see the other CTA's bytes and arrivals: cluster scope)
+            auto wait = [&](uint32_t bar, uint32_t parity) {
+                return PAIR ? mbar_wait_cluster(bar, parity, a.status) : mbar_wait(bar, parity, a.status);
+            };
+            auto commit = [&](uint32_t bar) {
+                if constexpr (PAIR) mma_commit_pair(bar);
+                else mma_commit(bar);
+            };
             const uint32_t b_lbo = B_MN ? (uint32_t)BK * 128u : 16u;
             const uint32_t b_step = B_MN ? (uint32_t)C::UMMA_K * 128u : 32u;
             int s = 0;
@@ -1374,15 +1426,15 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                 int i0;
                 tile_coords(lt, m0, i0);
                 if (ares && m0 != a_m) {
-                    if (!mbar_wait(a_full, a_uses & 1, a.status)) break;
+                    if (!wait(a_full, a_uses & 1)) break;
                     ++a_uses;
                     a_m = m0;
                 }
-                if (lt >= 2 && !mbar_wait(acc_empty(buf), ((lt >> 1) - 1) & 1, a.status)) break;
+                if (lt >= 2 && !wait(acc_empty(buf), ((lt >> 1) - 1) & 1)) break;
                 tc_fence_after();
                 const uint32_t d_main = tmem + buf * acc_cols, d_corr = d_main + BN;
                 for (int kb = 0; kb < a.nkb; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
-                    if (!mbar_wait(full(s), ph, a.status)) { ok = false; break; }
+                    if (!wait(full(s), ph)) { ok = false; break; }
                     tc_fence_after();
                     // k-steps advance the descriptors' start address field (no carry below 2^18)
                     const int sa = ares ? kb : s;
@@ -1395,7 +1447,9 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         const uint64_t ad = ad0 + (uint64_t)(ks * 2);
                         const uint64_t bd = bd0 + (uint64_t)((ks * b_step) >> 4);
                         const uint32_t acc = (kb > 0 || ks > 0) ? 1u : 0u;
-                        if constexpr (!F32) {
+                        if constexpr (PAIR) {
+                            mma_f16_ss_pair(d_main, ad, bd, idesc, acc);
+                        } else if constexpr (!F32) {
                             mma_bf16_ss(d_main, ad, bd, idesc, acc);
                         } else {
                             const uint64_t adl = adl0 + (uint64_t)(ks * 2);
@@ -1405,16 +1459,17 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                             mma_bf16_ss(d_main, ad, bd, idesc, acc);
                         }
                     }
-                    mma_commit(empty(s));
+                    commit(empty(s));
                 }
                 if (!ok) break;
-                mma_commit(acc_full(buf));
+                commit(acc_full(buf));
                 // the last tile of this batch tile's run: release the resident rows
-                if (ares && lt + 1 < my_tiles) {
-                    int64_t mn;
+                // (a pair: after the last run too, which the follower waits for before it exits)
+                if (ares) {
+                    int64_t mn = -1;
                     int in_;
-                    tile_coords(lt + 1, mn, in_);
-                    if (mn != m0) mma_commit(a_empty);
+                    if (lt + 1 < my_tiles) tile_coords(lt + 1, mn, in_);
+                    if (lt + 1 < my_tiles ? mn != m0 : PAIR) commit(a_empty);
                 }
             }
         }
@@ -1538,9 +1593,14 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     }
                 }
             }
-            // the accumulator buffer is free for the tile after next
+            // the accumulator buffer is free for the tile after next (one arrival per
+            // warp, on the leader's barrier for a pair)
             tc_fence_before();
-            mbar_arrive(acc_empty(buf));
+            __syncwarp();
+            if (lane == 0) {
+                if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(acc_empty(buf), 0));
+                else mbar_arrive(acc_empty(buf));
+            }
             // both halves of the row are staged
             named_bar_sync(1 + q, 64);
             // dx of this warp's inputs [ia, ib): each lane computes its row's values
@@ -1637,9 +1697,11 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // neither CTA leaves while the pair's MMAs or arrivals may touch it
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem, 512);
+        else tmem_dealloc(tmem, 512);
     }
 }
 
@@ -1919,7 +1981,7 @@ struct Plan {
     // dx
     int x_BN, x_stages, x_n, x_m, x_nin, x_nkb;
     // dx, persistent kernel (used when p_ok)
-    bool p_ok, p_ares;
+    bool p_ok, p_ares, p_pair;
     int p_BN, p_stages, p_nin, p_ntn, p_tiles, p_ld, p_grid, p_smem;
     // dY . w_base
     int g_BN, g_stages, g_n, g_m;
@@ -1981,10 +2043,13 @@ Plan make_plan(const Problem& p, int sms)
     // fp32 accumulates over `out` without promotion, so at most 1024 terms
     {
         P.p_BN = f32 ? 128 : 256;
+        // bf16 with at least 4 batch tiles: CTA pairs over 256-row tiles, each CTA
+        // holding half of the B columns
+        P.p_pair = !f32 && P.x_m >= 4;
         P.p_nin = (P.p_BN - maxoff) / P.nbx;
         P.p_ld = f32 ? P.p_BN + 4 : P.p_BN + 8;          // row stride = 16 bytes mod 128
         const int staging = 4 * 32 * P.p_ld * (f32 ? 4 : 2);
-        const int a_stage = kBM * 128 * (f32 ? 2 : 1), b_stage = P.p_BN * 128 * (f32 ? 2 : 1);
+        const int a_stage = kBM * 128 * (f32 ? 2 : 1), b_stage = (P.p_pair ? P.p_BN / 2 : P.p_BN) * 128 * (f32 ? 2 : 1);
         const int stage_bytes = a_stage + b_stage;
         const int avail = 232448 - 1024 - 256 - staging;
         P.p_stages = std::min(6, avail / stage_bytes);
@@ -2001,8 +2066,8 @@ Plan make_plan(const Problem& p, int sms)
         P.p_ok = P.p_nin >= 1 && P.p_stages >= 2 && (!f32 || p.out <= 1024);
         if (P.p_ok) {
             P.p_ntn = (int)cdiv(p.in, P.p_nin);
-            P.p_tiles = P.p_ntn * P.x_m;
-            P.p_grid = std::max(1, std::min(P.p_tiles, sms));
+            P.p_tiles = P.p_ntn * (P.p_pair ? (P.x_m + 1) / 2 : P.x_m);
+            P.p_grid = P.p_pair ? std::max(2, std::min(2 * P.p_tiles, sms) / 2 * 2) : std::max(1, std::min(P.p_tiles, sms));
             P.p_smem = (P.p_ares ? P.x_nkb * a_stage + P.p_stages * b_stage : P.p_stages * stage_bytes) + staging +
                        1024 + 256;
         }
@@ -2129,19 +2194,39 @@ cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap
     }
 }
 
-template <int DT>
+template <int DT, bool PAIR>
 cudaError_t launch_dx_persistent(const Plan& P, const CUtensorMap* maps, const DxArgs& d, cudaStream_t st)
 {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(dx_persistent_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(dx_persistent_kernel<DT, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              232448);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     if (P.p_smem > 232448 || d.BN % 16 != 0 || d.stages < 2) return cudaErrorInvalidConfiguration;
-    dx_persistent_kernel<DT><<<P.p_grid, kDxThreads, P.p_smem, st>>>(maps[0], maps[1], maps[2], maps[3], d);
-    count_launch();
+    // a pair's CTA loads BN / 2 columns of B in 64-column atoms; the grid is whole clusters
+    if (PAIR && (d.BN % 128 != 0 || P.p_grid % 2 != 0)) return cudaErrorInvalidConfiguration;
+    if constexpr (PAIR) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(P.p_grid, 1, 1);
+        cfg.blockDim = dim3(kDxThreads, 1, 1);
+        cfg.dynamicSmemBytes = (size_t)P.p_smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, dx_persistent_kernel<DT, true>, maps[0], maps[1], maps[2], maps[3], d);
+        count_launch();
+        if (e != cudaSuccess) return e;
+    } else {
+        dx_persistent_kernel<DT, false><<<P.p_grid, kDxThreads, P.p_smem, st>>>(maps[0], maps[1], maps[2], maps[3], d);
+        count_launch();
+    }
     return cudaGetLastError();
 }
 
@@ -2448,7 +2533,10 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             d.n_tiles = P.p_tiles;
             d.ld_stage = P.p_ld;
             d.a_res = P.p_ares ? 1 : 0;
-            e = f32 ? launch_dx_persistent<KAN_F32>(P, maps, d, st) : launch_dx_persistent<KAN_BF16>(P, maps, d, st);
+            d.pair = P.p_pair ? 1 : 0;
+            e = f32 ? launch_dx_persistent<KAN_F32, false>(P, maps, d, st)
+                    : (P.p_pair ? launch_dx_persistent<KAN_BF16, true>(P, maps, d, st)
+                                : launch_dx_persistent<KAN_BF16, false>(P, maps, d, st));
             if (e != cudaSuccess) return e;
         } else {
             TcArgs a = base_args(p, P);

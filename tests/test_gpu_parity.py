@@ -103,6 +103,9 @@ SMALL = [
     (300, 32, 1000, 8, -1.0, 1.0, False),
     (300, 16, 256, 8, -1.0, 1.0, True),
     (300, 8, 696, 20, -1.0, 1.0, True),
+    # dx as CTA pairs over 256-row tiles: an odd batch-tile count, dY resident or streamed
+    (800, 32, 64, 8, -1.0, 1.0, True),
+    (800, 24, 296, 20, -1.0, 1.0, False),
 ]
 
 
