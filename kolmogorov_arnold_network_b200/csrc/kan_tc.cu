@@ -172,9 +172,13 @@ struct TcArgs {
     int m_tiles;               // FWD, DCA: M tiles holding work (a pair grid may have one more)
 };
 
+// (offset arithmetic on the shared array itself, not an integer round trip, so
+// that accesses through the result stay shared-memory loads and stores rather
+// than generic ones)
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
 {
-    return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+    const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
 __device__ __forceinline__ void st_shared_zero16(uint32_t addr)

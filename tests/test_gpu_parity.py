@@ -106,6 +106,8 @@ SMALL = [
     # dx as CTA pairs over 256-row tiles: an odd batch-tile count, dY resident or streamed
     (800, 32, 64, 8, -1.0, 1.0, True),
     (800, 24, 296, 20, -1.0, 1.0, False),
+    # G = 5: a ragged last k-block, x rows not 16-byte aligned
+    (300, 20, 256, 5, -3.0, 3.0, False),
 ]
 
 
