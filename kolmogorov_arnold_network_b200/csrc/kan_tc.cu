@@ -1771,9 +1771,14 @@ __global__ void absmax_kernel(AmaxArgs a, unsigned int* __restrict__ amax)
         float m = 0.0f;
         const int64_t n = a.n[k], n4 = n / 4;
         const float4* __restrict__ v4 = reinterpret_cast<const float4*>(a.src[k]);
-        for (int64_t e = tid; e < n4; e += nth) {
-            const float4 q = v4[e];
-            m = fmaxf(m, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+        // four independent 16-byte loads in flight per thread and step
+        for (int64_t e = tid; e < n4; e += 4 * nth) {
+            float4 q[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) q[u] = e + u * nth < n4 ? v4[e + u * nth] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(q[u].x), fabsf(q[u].y)), fmaxf(fabsf(q[u].z), fabsf(q[u].w))));
         }
         for (int64_t e = 4 * n4 + tid; e < n; e += nth) m = fmaxf(m, fabsf(a.src[k][e]));
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -1805,8 +1810,9 @@ __global__ void split_f16_kernel(const float* __restrict__ src, uint16_t* __rest
 // fp16 hi/lo split of the coefficient matrix, row-major [out][in*nbx]:
 // column i*nbx + m is coef[j, i, m] * s_c for m < nbs, and (with the SiLU
 // branch, nbx = nbs + 1) w_base[j, i] * s_c / s_x for m == nbs.  Rows j step
-// by gridDim.y, one column per thread (coalesced writes; the reads are
-// consecutive apart from the SiLU columns); c / nbx through a multiply-high.
+// by gridDim.y, four consecutive columns per thread (8-byte writes; Kx % 4 == 0;
+// the reads are consecutive apart from the SiLU columns); c / nbx through a
+// multiply-high.
 __global__ void split_coef_f16_kernel(const float* __restrict__ coef, const float* __restrict__ w_base, int64_t out,
                                       int64_t in, int nbs, int nbx, uint16_t* __restrict__ hi, uint16_t* __restrict__ lo,
                                       const unsigned int* __restrict__ amax, uint32_t nbx_magic)
@@ -1815,12 +1821,19 @@ __global__ void split_coef_f16_kernel(const float* __restrict__ coef, const floa
     const float sw = sc.c / sc.x;
     const int Kx = (int)(in * nbx);
     for (int64_t j = blockIdx.y; j < out; j += gridDim.y)
-    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < Kx; c += gridDim.x * blockDim.x) {
+    for (int c4 = 4 * (blockIdx.x * blockDim.x + threadIdx.x); c4 < Kx; c4 += 4 * gridDim.x * blockDim.x) {
         const float* __restrict__ crow = coef + j * in * nbs;
-        const int i = (int)__umulhi((uint32_t)c, nbx_magic);
-        const int m = c - i * nbx;
-        const float v = m < nbs ? crow[i * nbs + m] * sc.c : w_base[j * in + i] * sw;
-        split_f16(v, hi[j * Kx + c], lo[j * Kx + c]);
+        uint16_t h[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int c = c4 + e;
+            const int i = (int)__umulhi((uint32_t)c, nbx_magic);
+            const int m = c - i * nbx;
+            const float v = m < nbs ? crow[i * nbs + m] * sc.c : w_base[j * in + i] * sw;
+            split_f16(v, h[e], l[e]);
+        }
+        *reinterpret_cast<uint2*>(hi + j * Kx + c4) = make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
+        *reinterpret_cast<uint2*>(lo + j * Kx + c4) = make_uint2(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16));
     }
 }
 
@@ -2284,7 +2297,7 @@ cudaError_t split_coef_into(const Problem& p, const Plan& P, const void* coef, c
 {
     uint16_t* h = reinterpret_cast<uint16_t*>(dst);
     uint16_t* l = reinterpret_cast<uint16_t*>(dst + al256((size_t)p.out * P.Kx * 2));
-    const dim3 grid((unsigned)std::min<int64_t>(cdiv(P.Kx, 256), 64), (unsigned)std::min<int64_t>(p.out, 65535));
+    const dim3 grid((unsigned)std::min<int64_t>(cdiv(P.Kx, 4 * 256), 64), (unsigned)std::min<int64_t>(p.out, 65535));
     const uint32_t magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)P.nbx - 1) / (uint64_t)P.nbx);
     split_coef_f16_kernel<<<grid, 256, 0, st>>>((const float*)coef, (const float*)w_base, p.out, p.in, p.nb, P.nbx, h,
                                                 l, amax, magic);
