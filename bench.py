@@ -225,8 +225,12 @@ class ClockSampler:
         cmd = ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "50"]
         if uuid:
             cmd += ["-i", uuid]
+        self.first = ""
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            # wait for the first sample, so that even a timed region shorter than
+            # nvidia-smi's start-up is covered by the stream that follows
+            self.first = self.proc.stdout.readline()
         except Exception:
             self.proc = None
 
@@ -240,7 +244,7 @@ class ClockSampler:
             self.proc.kill()
             out, _ = self.proc.communicate()
         rows = []
-        for line in out.strip().splitlines():
+        for line in (self.first + out).strip().splitlines():
             f = [t.strip() for t in line.split(",")]
             if len(f) >= 8:
                 try:
@@ -259,8 +263,11 @@ class ClockSampler:
             for nm, v in zip(names, r[2][1:]):
                 if v.lower() == "active":
                     reasons.add(nm)
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
-                "samples": len(rows), "samples_under_load": len(loaded), "power_w_max": pmax}
+        res = {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
+               "samples": len(rows), "samples_under_load": len(loaded), "power_w_max": pmax}
+        if len(rows) < 3:
+            res["note"] = "timed region about as short as the 50 ms sampling interval: few samples"
+        return res
 
 
 # ---------------------------------------------------------------------------
