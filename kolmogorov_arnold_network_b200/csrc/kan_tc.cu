@@ -236,16 +236,6 @@ __device__ __forceinline__ void floor_split(float u, int& s, float& f)
     s = __float_as_int(r) - 0x4B400000;
 }
 
-__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v)
-{
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void st_shared_v2f(uint32_t addr, float a, float b)
-{
-    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
-}
-
 // Byte offset of element column c inside one 128-byte swizzled row (row & 7 = rx).
 template <int ESZ>
 __device__ __forceinline__ uint32_t sw_col(int c, uint32_t rx)
@@ -2479,7 +2469,6 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         e = launch_dt<DCA>(f32, grid, P.d_BN, P.d_stages, maps, a, st);
         if (e != cudaSuccess) return e;
         if (a.partial) {
-            const int64_t n = p.out * P.d_ld;
             const dim3 rgrid((unsigned)std::min<int64_t>(cdiv(P.d_ld, 256), 64),
                              (unsigned)std::min<int64_t>(p.out, 65535));
             reduce_dcoef_kernel<<<rgrid, 256, 0, st>>>(partbuf, dcoef, dw_base, p.out, p.Kt, p.in, P.d_ld, P.d_splits,
