@@ -2,19 +2,31 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+Default workload: the KAN FFN block (8192 tokens, 768 -> 3072 -> 768, G = 5 on
+[-3, 3], bf16 operands with fp32 accumulation), the largest single-GPU
+workload of the method's measurement plan by edge evaluations per step.
+
 A step is one pass of the whole hot path over one batch of synthetic input:
-the forward (y), then the backward (dx, and dcoef / dw_base), through the C ABI
-of libkan_b200.so.  Edge evaluations per step = batch * in * out (summed over
-the layers of the FFN block).  One JSON line is printed by rank 0.
+kan_forward of every layer, then one kan_backward per layer (last layer first)
+returning dx, dcoef and dw_base together, all through the C ABI of
+libkan_b200.so.  Edge evaluations per step = batch * in * out (summed over the
+layers of the FFN block).  One JSON line is printed by rank 0.
 
 Timing: W untimed steps, then K timed steps between a barrier and a device
 synchronize on both sides.  Each step is bracketed by CUDA events on the
 launching stream; a 256 MiB buffer (larger than the 126 MB L2) is rewritten
-between steps, outside the events.  Each C-ABI call inside the step carries
-its own events too, which give the dominant kernel's launch time for the
-roofline.  With N > 1 (torchrun), every rank runs an independent replica of
-the workload (weak scaling, no collective on the data path) and the time is
-the maximum over ranks.
+between steps, outside the events.  Each call carries its own events, and the
+library records two more inside it (kan_set_timing_marks) at the boundaries
+of its kernel groups, so that every call splits into operand preparation,
+dcoef and dx time: the dominant one gives the roofline.  With N > 1
+(torchrun), every rank runs an independent replica of the workload (weak
+scaling, no collective on the data path) and the time is the maximum over
+ranks.
+
+Also in the line: the measured fp32 FMA peak (the library's calibration
+kernel), the whole step against its bound, the bilinear adjoint identity per
+layer as a parity check that needs no reference, and (one GPU) the same
+figures for the other large workloads of the plan ("other_workloads").
 
 --impl reference times the fp64 CPU oracle on the host cores instead (the
 only reference this build has), each step a bounded row sample of the same
@@ -90,27 +102,17 @@ def csrc_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload: str, call: str):
-    """DRAM bytes per launch of a call's main kernel from the committed ncu capture
-    (profiles/traffic.json), or None when there is none or the kernels changed since."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    try:
-        with open(path) as f:
-            d = json.load(f)
-    except (OSError, ValueError):
-        return None
-    if d.get("csrc_hash") != csrc_hash():
-        return None
-    e = d.get("workloads", {}).get(workload, {}).get(call)
-    return None if e is None else e.get("dram_bytes")
-
-
 # ---------------------------------------------------------------------------
 # FLOP / byte accounting (per call, algorithmic)
 def layer_dense_flops(batch, L):
     """Dense-expanded FLOPs of one layer GEMM: 2 * batch * out * (in*(G+3) [+ in for SiLU])."""
     k = L.inp * (L.G + 3) + (L.inp if L.base else 0)
     return 2.0 * batch * L.out * k
+
+
+def layer_alg_flops(batch, L):
+    """Algorithmic FLOPs of one layer GEMM: 4 FMAs per edge (+1 with SiLU), 2 FLOPs each."""
+    return (8.0 + (2.0 if L.base else 0.0)) * batch * L.inp * L.out
 
 
 def layer_bytes(batch, L, esz, call):
@@ -125,9 +127,33 @@ def layer_bytes(batch, L, esz, call):
     return x + dy + coef + batch * L.inp * esz          # dx
 
 
+def measured_counters(workload: str, call: str):
+    """The committed ncu figures of a call's main kernel (profiles/traffic.json): DRAM bytes per launch
+    and tensor-pipe activity, or None when there are none or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("csrc_hash") != csrc_hash():
+        return None
+    return d.get("workloads", {}).get(workload, {}).get(call)
+
+
+def measured_traffic(workload: str, call: str):
+    """DRAM bytes per launch of a call's main kernel from the committed ncu capture, or None."""
+    e = measured_counters(workload, call)
+    return None if e is None else e.get("dram_bytes")
+
+
 # ---------------------------------------------------------------------------
 class Runner:
-    """Pre-allocated buffers and the step's C-ABI calls for one workload."""
+    """Pre-allocated buffers and the step's C-ABI calls for one workload.
+
+    A step is the forward of every layer, then one kan_backward per layer (last
+    layer first) that returns dx, dcoef and dw_base together: the call pattern
+    of training through the library."""
 
     def __init__(self, w: W.Workload, dev):
         from kolmogorov_arnold_network_b200 import _native as N
@@ -153,9 +179,12 @@ class Runner:
             self.layers.append(dict(L=L, s=s, x=act, coef=coef, wb=wb, y=y, dx=dx, dcoef=dcoef, dwb=dwb,
                                     ws_f=ws_f, ws_b=ws_b))
             act = y
-        # pinned host mirrors for the end-to-end variant
-        self.h_x = d["x"].pin_memory()
-        self.h_dY = d["dY"].pin_memory()
+        self.h_x = self.h_dY = None
+
+    def pin_host(self):
+        """Pinned host mirrors of the inputs and outputs (the end-to-end variant)."""
+        self.h_x = self.host["x"].pin_memory()
+        self.h_dY = self.host["dY"].pin_memory()
         self.h_out = []
         for l in self.layers:
             self.h_out.append(dict(y=torch.empty_like(l["y"], device="cpu").pin_memory(),
@@ -164,31 +193,38 @@ class Runner:
                                    dwb=None if l["dwb"] is None else
                                    torch.empty_like(l["dwb"], device="cpu").pin_memory()))
 
+    def dy_of(self, li):
+        return self.dY if li == len(self.layers) - 1 else self.layers[li + 1]["dx"]
+
     def calls(self):
-        """The step as a list of (name, callable), in launch order."""
+        """The step as a list of (name, kind, callable(marks)), in launch order; kind is "fwd" or "bwd".
+        marks = (after_prep, after_dcoef) event handles or None, set for the duration of the call."""
         N, P = self.N, lambda t: None if t is None else t.data_ptr()
         st = torch.cuda.current_stream(self.dev).cuda_stream
         out = []
         for li, l in enumerate(self.layers):
-            def fwd(l=l):
+            def fwd(marks=None, l=l):
+                if marks is not None:
+                    N.kan_set_timing_marks(marks[0], None)
                 N.kan_forward(l["s"], P(l["x"]), P(l["coef"]), P(l["wb"]), P(l["y"]), P(l["ws_f"]),
                               0 if l["ws_f"] is None else l["ws_f"].numel(), st)
-            out.append((f"fwd{li}", fwd))
+                if marks is not None:
+                    N.kan_set_timing_marks(None, None)
+            out.append((f"fwd{li}", "fwd", fwd))
         if self.w.mode == "fwd":
             return out
         for li in reversed(range(len(self.layers))):
             l = self.layers[li]
-            dy = self.dY if li == len(self.layers) - 1 else self.layers[li + 1]["dx"]
+            dy = self.dy_of(li)
 
-            def dcoef(l=l, dy=dy):
-                N.kan_backward(l["s"], P(l["x"]), P(l["coef"]), P(l["wb"]), P(dy), None, P(l["dcoef"]),
+            def bwd(marks=None, l=l, dy=dy):
+                if marks is not None:
+                    N.kan_set_timing_marks(marks[0], marks[1])
+                N.kan_backward(l["s"], P(l["x"]), P(l["coef"]), P(l["wb"]), P(dy), P(l["dx"]), P(l["dcoef"]),
                                P(l["dwb"]), P(l["ws_b"]), 0 if l["ws_b"] is None else l["ws_b"].numel(), st)
-
-            def dx(l=l, dy=dy):
-                N.kan_backward(l["s"], P(l["x"]), P(l["coef"]), P(l["wb"]), P(dy), P(l["dx"]), None, None,
-                               P(l["ws_b"]), 0 if l["ws_b"] is None else l["ws_b"].numel(), st)
-            out.append((f"dcoef{li}", dcoef))
-            out.append((f"dx{li}", dx))
+                if marks is not None:
+                    N.kan_set_timing_marks(None, None)
+            out.append((f"bwd{li}", "bwd", bwd))
         return out
 
     def h2d(self):
@@ -208,6 +244,154 @@ class Runner:
                     h[k].copy_(l[k], non_blocking=True)
                     n += h[k].numel() * h[k].element_size()
         return n
+
+    def adjoint_errors(self):
+        """Bilinear adjoint identity per layer (y is linear in coef and w_base):
+        <dY, y> = <dcoef, coef> + <dw_base, w_base>, relative to sum |dY * y|.  Holds at any size,
+        needs no reference implementation."""
+        out = {}
+        for li, l in enumerate(self.layers):
+            dy = self.dy_of(li).double()
+            y = l["y"].double()
+            lhs = (dy * y).sum().item()
+            rhs = (l["dcoef"].double() * l["coef"].double()).sum().item()
+            if l["wb"] is not None:
+                rhs += (l["dwb"].double() * l["wb"].double()).sum().item()
+            scale = (dy * y).abs().sum().item()
+            out[f"layer{li}"] = abs(lhs - rhs) / scale if scale > 0 else abs(lhs - rhs)
+        return out
+
+
+def _ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def time_steps(R: Runner, K: int, warmup: int, flush, barrier=lambda: None):
+    """W untimed steps, then K steps each bracketed by events on the launching stream, with the L2 flush
+    buffer rewritten between steps (outside the events).  Every call records its own events and the
+    library's timing marks, which split it into segments: "prep<li>" (fp32 operand preparation),
+    "fwd<li>", "dcoef<li>", "dx<li>".  Returns (total ms, {segment: total ms}, launches)."""
+    N = R.N
+    calls = R.calls()
+    stream = torch.cuda.current_stream(R.dev)
+    for _ in range(warmup):
+        flush.zero_()
+        for _, _, c in calls:
+            c()
+    torch.cuda.synchronize(R.dev)
+    st = N.kan_sync_status(None)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {N.STATUS.get(st, st)}")
+    # per call: start, after_prep, after_dcoef (backward only), end
+    evs = [[dict(start=_ev(), prep=_ev(), mid=_ev() if kind == "bwd" else None, end=_ev())
+            for _, kind, _ in calls] for _ in range(K)]
+    step_ev = [(_ev(), _ev()) for _ in range(K)]
+    # torch creates an event's CUDA handle at its first record: record every mark event once now, so that
+    # the handles passed to the library exist
+    for row in evs:
+        for e in row:
+            for v in e.values():
+                if v is not None:
+                    v.record(stream)
+    barrier()
+    torch.cuda.synchronize(R.dev)
+    n0 = N.kan_launch_count()
+    for k in range(K):
+        flush.zero_()
+        step_ev[k][0].record(stream)
+        for e, (_, kind, c) in zip(evs[k], calls):
+            e["start"].record(stream)
+            c((e["prep"].cuda_event, None if e["mid"] is None else e["mid"].cuda_event))
+            e["end"].record(stream)
+        step_ev[k][1].record(stream)
+    torch.cuda.synchronize(R.dev)
+    barrier()
+    launches = N.kan_launch_count() - n0
+    total = sum(a.elapsed_time(b) for a, b in step_ev)
+    seg = {}
+    for k in range(K):
+        for e, (nm, kind, _) in zip(evs[k], calls):
+            li = nm[3:]
+            parts = [(f"prep{li}", e["start"], e["prep"])]
+            if kind == "fwd":
+                parts.append((f"fwd{li}", e["prep"], e["end"]))
+            else:
+                parts += [(f"dcoef{li}", e["prep"], e["mid"]), (f"dx{li}", e["mid"], e["end"])]
+            for key, e0, e1 in parts:
+                seg[key] = seg.get(key, 0.0) + e0.elapsed_time(e1)
+    return total, seg, launches
+
+
+def ffma_peak(dev, sms):
+    """The fp32 FMA rate of this GPU, measured with the library's calibration kernel (best of 3 launches
+    of about 50 ms each), in TFLOP/s."""
+    from kolmogorov_arnold_network_b200 import _native as N
+    blocks = sms * 4
+    sink = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+    st = torch.cuda.current_stream(dev)
+    iters = 2000
+    N.kan_ffma_probe(blocks, iters, sink.data_ptr(), st.cuda_stream)      # warm-up
+    torch.cuda.synchronize(dev)
+    best = 0.0
+    for _ in range(3):
+        a, b = _ev(), _ev()
+        a.record(st)
+        fl = N.kan_ffma_probe(blocks, iters * 25, sink.data_ptr(), st.cuda_stream)
+        b.record(st)
+        torch.cuda.synchronize(dev)
+        best = max(best, fl / (a.elapsed_time(b) / 1000.0) / 1e12)
+    return best
+
+
+def step_roofline(w: W.Workload, ms_per_step: float, pk: dict, ffma_tflops: float):
+    """The whole step against its bound: bf16, dense-expanded FLOPs of every GEMM at the bf16 tensor
+    peak; fp32, algorithmic FLOPs at the fp32 FMA peak (3 GEMMs per layer for forward + backward)."""
+    gemms = 1 if w.mode == "fwd" else 3
+    if w.dtype == "bf16":
+        fl = gemms * sum(layer_dense_flops(w.batch, L) for L in w.layers)
+        t = fl / (pk["bf16"] * 1e12)
+    else:
+        fl = gemms * sum(layer_alg_flops(w.batch, L) for L in w.layers)
+        t = fl / (ffma_tflops * 1e12)
+    return {"t_roof_ms": t * 1000.0, "frac": t * 1000.0 / ms_per_step,
+            "bound": "bf16 tensor, dense-expanded" if w.dtype == "bf16" else "fp32 FMA, algorithmic"}
+
+
+def roofline_of(w: W.Workload, seg: dict, K: int, pk: dict, ffma_tflops: float):
+    """Roofline of the dominant kernel segment (fwd, dcoef or dx of one layer).
+
+    bf16: dense-expanded FLOPs of the GEMM at the measured bf16 tensor peak.  fp32: the fp32 bound of
+    the method's measurement plan, algorithmic FLOPs (4 FMAs per edge, +1 with SiLU) at the measured
+    fp32 FMA peak; the dense-expanded fraction at the fp16 tensor peak is reported beside it."""
+    gemm = {k: v for k, v in seg.items() if not k.startswith("prep")}
+    dom = max(gemm, key=gemm.get)
+    kind, li = dom.rstrip("0123456789"), int(dom[len(dom.rstrip("0123456789")):])
+    L = w.layers[li]
+    avg_s = gemm[dom] / K / 1000.0
+    dense = layer_dense_flops(w.batch, L)
+    counters = measured_counters(w.name, kind) or {}
+    if w.dtype == "bf16":
+        achieved = dense / avg_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16"], "peak_note": f"bf16 dense, {pk['src']} burst (of {pk['src']})",
+                "frac_of_sustained": achieved / pk["bf16_sus"] if pk.get("bf16_sus") else None,
+                "flops_per_launch": dense, "flops_kind": "dense-expanded"}
+    else:
+        alg = layer_alg_flops(w.batch, L)
+        achieved = alg / avg_s / 1e12
+        tens = dense / avg_s / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": ffma_tflops, "unit": "TFLOP/s",
+                "frac": achieved / ffma_tflops,
+                "peak_note": "fp32 FMA peak measured in this run by the library's calibration kernel",
+                "flops_per_launch": alg, "flops_kind": "algorithmic (4 FMA per edge, +1 with SiLU)",
+                "tensor_dense_achieved": tens, "tensor_dense_frac": tens / (pk["bf16"] * F16_PER_BF16),
+                "note": ("the kernel runs on fp16 tensor cores (3 products of hi/lo splits); tensor_dense_frac is "
+                         "its dense-expanded FLOPs at the fp16 tensor peak, at most 1/3 by construction")}
+    roof.update({"traffic": counters.get("dram_bytes"), "tensor_pipe_active": counters.get("tensor_pipe_active"),
+                 "kernel": f"{kind} of layer {li}", "launch_ms": avg_s * 1000.0,
+                 "algorithmic_bytes_per_launch": layer_bytes(w.batch, L, 4 if w.dtype == "f32" else 2, kind),
+                 "segment_ms": {k: v / K for k, v in seg.items()}})
+    return roof
 
 
 class ClockSampler:
@@ -373,13 +557,16 @@ def config_of(w: W.Workload):
     return c
 
 
+#: workloads timed beside the headline one (each in the same JSON line, with the adjoint-identity check)
+EXTRA_WORKLOADS = ["layer784x64_silu", "layer1024_g20_bf16"] + \
+    [f"sweep512_g{G}_{dt}_fwdbwd" for G in (8, 20, 50) for dt in ("bf16", "f32")]
+
+
 def run_ours(args, world, rank, local):
-    from kolmogorov_arnold_network_b200 import _native as N
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = W.WORKLOADS[args.workload]
-    R = Runner(w, dev)
-    calls = R.calls()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -387,75 +574,27 @@ def run_ours(args, world, rank, local):
         if world > 1:
             torch.distributed.barrier()
 
+    R = Runner(w, dev)
     sampler = ClockSampler(local)   # started before the warm-up so that it is sampling by the timed region
-    for _ in range(args.warmup):
-        flush.zero_()
-        for _, c in calls:
-            c()
-    torch.cuda.synchronize(dev)
-    st = N.kan_sync_status(None)
-    if st != 0:
-        raise RuntimeError(f"device status after warm-up: {N.STATUS.get(st, st)}")
-
-    # ---- device-resident timed region ----
-    K = args.steps
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
-          for _ in range(K)]
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    barrier()
-    torch.cuda.synchronize(dev)
-    n0 = N.kan_launch_count()
     wall0 = time.perf_counter()
-    for k in range(K):
-        flush.zero_()
-        step_ev[k][0].record(stream)
-        for (a, b), (_, c) in zip(ev[k], calls):
-            a.record(stream)
-            c()
-            b.record(stream)
-        step_ev[k][1].record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
+    K = args.steps
+    total, seg, launches = time_steps(R, K, args.warmup, flush, barrier)
     wall = time.perf_counter() - wall0
-    launches = N.kan_launch_count() - n0
     clocks = sampler.stop()
-    step_ms = sum(s.elapsed_time(e) for s, e in step_ev)
-    per_call = {}
-    for k in range(K):
-        for (a, b), (nm, _) in zip(ev[k], calls):
-            per_call[nm] = per_call.get(nm, 0.0) + a.elapsed_time(b)
-    t_max = max_over_ranks(step_ms, world, dev)
-    edges = w.edges
-    value = aggregate_rate(edges, K, world, t_max)
-
-    # ---- roofline of the dominant call ----
+    t_max = max_over_ranks(total, world, dev)
+    value = aggregate_rate(w.edges, K, world, t_max)
+    adj = R.adjoint_errors()
+    tol = 1e-5 if w.dtype == "f32" else 2e-2
+    ffma = ffma_peak(dev, sms)
     pk = peaks()
-    dom = max(per_call, key=per_call.get)
-    li = int(dom[-1])
-    L = w.layers[li]
-    kind = dom[:-1]
-    flops = layer_dense_flops(w.batch, L)
-    avg_s = per_call[dom] / K / 1000.0
-    if w.dtype == "bf16":
-        peak = pk["bf16"]
-        peak_note = f"bf16 dense, {pk['src']} burst"
-    else:
-        peak = pk["bf16"] * F16_PER_BF16
-        peak_note = f"fp16 dense = {pk['src']} bf16 burst x nominal fp16/bf16 ratio {F16_PER_BF16:.1f}"
-    achieved = flops / avg_s / 1e12
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": measured_traffic(w.name, kind), "kernel": f"{kind} call of layer {li}", "peak_note": peak_note,
-            "algorithmic_flops_per_launch": flops,
-            "algorithmic_bytes_per_launch": layer_bytes(w.batch, L, 4 if w.dtype == "f32" else 2, kind),
-            "call_ms": {k: v / K for k, v in per_call.items()}}
-    if w.dtype == "f32":
-        roof["note"] = ("3 fp16 products per term: the executed tensor FLOPs are 3x the algorithmic ones, so "
-                        "frac <= 1/3 by construction")
+    roof = roofline_of(w, seg, K, pk, ffma)
 
     # ---- end to end: pinned host inputs in, results out, every step ----
     e2e = None
     if not args.no_e2e:
-        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        R.pin_host()
+        calls = R.calls()
+        e2e_ev = [(_ev(), _ev()) for _ in range(K)]
         hb = db = 0
         barrier()
         torch.cuda.synchronize(dev)
@@ -463,34 +602,72 @@ def run_ours(args, world, rank, local):
             flush.zero_()
             e2e_ev[k][0].record(stream)
             hb = R.h2d()
-            for _, c in calls:
+            for _, _, c in calls:
                 c()
             db = R.d2h()
             e2e_ev[k][1].record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in e2e_ev), world, dev)
-        e2e = {"value": aggregate_rate(edges, K, world, e_ms), "unit": UNIT, "h2d_bytes_per_step": hb,
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, dev)
+        e2e = {"value": aggregate_rate(w.edges, K, world, e_ms), "unit": UNIT, "h2d_bytes_per_step": hb,
                "d2h_bytes_per_step": db}
+    del R
 
-    st = N.kan_sync_status(None)
+    # ---- the other workloads of the method's measurement plan, one GPU only ----
+    others = {}
+    if world == 1 and not args.no_extras:
+        for nm in EXTRA_WORKLOADS:
+            if nm == w.name:
+                continue
+            wx = W.WORKLOADS[nm]
+            Rx = Runner(wx, dev)
+            kx = min(K, args.extra_steps)
+            tx, segx, _ = time_steps(Rx, kx, 3, flush)
+            msx = tx / kx
+            rx = roofline_of(wx, segx, kx, pk, ffma)
+            ax = Rx.adjoint_errors()
+            tolx = 1e-5 if wx.dtype == "f32" else 2e-2
+            others[nm] = {"ms_per_step": msx, "value": wx.edges / (msx / 1000.0), "unit": UNIT, "steps": kx,
+                          "dtype": wx.dtype, "dominant": rx["kernel"], "bound": rx["bound"], "frac": rx["frac"],
+                          "tensor_dense_frac": rx.get("tensor_dense_frac"),
+                          "segment_ms": rx["segment_ms"], "step_roofline": step_roofline(wx, msx, pk, ffma),
+                          "adjoint_rel_err": ax, "adjoint_ok": all(v <= tolx for v in ax.values())}
+            del Rx
+            torch.cuda.empty_cache()
+
+    st = R_status()
     if st != 0:
-        raise RuntimeError(f"device status after timing: {N.STATUS.get(st, st)}")
+        raise RuntimeError(f"device status after timing: {st}")
     if rank == 0:
+        ms = t_max / K
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-                "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": w.dtype, "data": "synthetic", "config": config_of(w), "roofline": roof,
-                "e2e": e2e, "gpu_launches": launches, "clocks": clocks, "wall_s": wall}
+                "step_roofline": step_roofline(w, ms, pk, ffma),
+                "parity": {"check": "adjoint identity <dY,y> = <dcoef,coef> (+<dw_base,w_base>) per layer, "
+                                    "relative to sum|dY*y|", "rel_err": adj, "tol": tol,
+                           "ok": all(v <= tol for v in adj.values())},
+                "e2e": e2e, "gpu_launches": launches, "clocks": clocks, "wall_s": wall,
+                "ffma_peak_tflops": ffma, "peaks": pk}
+        if others:
+            line["other_workloads"] = others
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
 
 
+def R_status():
+    from kolmogorov_arnold_network_b200 import _native as N
+    return N.kan_sync_status(None)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--extra-steps", type=int, default=30)
+    ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--workload", default=W.BENCH_DEFAULT, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")

@@ -38,7 +38,12 @@
  * Pointers must be 16-byte aligned.
  *
  * Ownership: the caller owns every buffer, the workspace included.  The
- * library keeps no allocation across calls; it allocates nothing itself.
+ * library allocates no memory per call.  It holds two fixed device arrays in
+ * its own image, which every GPU that loads it keeps until the process exits:
+ * a 4-byte status word, and the KAN_FIXED_SCRATCH_BYTES workspace used only by
+ * kan_forward_fixed_scratch.  Their device addresses are looked up once per
+ * device and kept: do not use the library across a cudaDeviceReset (or any
+ * other teardown of the device's primary context) in the same process.
  *
  * Streams: every compute call is asynchronous on `stream` (a cudaStream_t
  * passed as void*, NULL = legacy default stream).  Errors found on the host
@@ -80,7 +85,7 @@ typedef enum {
 } kan_status;
 
 /* Kernel family selection (kan_shape.path). */
-#define KAN_PATH_AUTO 0    /* tensor-core kernels when the shape allows them, else CUDA-core kernels */
+#define KAN_PATH_AUTO 0    /* tensor-core kernels when TMA can address the shape's rows, else CUDA-core kernels */
 #define KAN_PATH_TENSOR 1  /* tcgen05/TMEM GEMM kernels with TMA-staged operands; KAN_ERR_UNSUPPORTED if not possible */
 #define KAN_PATH_SIMT 2    /* CUDA-core kernels (any shape) */
 
@@ -159,6 +164,31 @@ KAN_API kan_status kan_selftest_wait_timeout(int64_t limit_ns, void* stream);
 /* Number of kernels this library has launched in this process (all entry
  * points, all devices), for accounting of the launches inside a timed region. */
 KAN_API uint64_t kan_launch_count(void);
+
+/* Optional timing marks for benchmarks.  While set, the kan_forward and
+ * kan_backward calls made on this host thread record the given CUDA events
+ * (cudaEvent_t passed as void*, created and owned by the caller) on their
+ * stream at the boundaries between their kernel groups:
+ *   after_prep  : after the operand preparation (fp32: operand maxima and the
+ *                 fp16 hi/lo copies; bf16: nothing precedes it), before the
+ *                 first GEMM kernel (forward and backward);
+ *   after_dcoef : kan_backward only, after the dcoef / dw_base kernels and
+ *                 before the dx kernels.
+ * An event recorded before and one after the call then split the call into
+ * preparation, dcoef and dx time.  NULL arguments record nothing; call with
+ * (NULL, NULL) to turn the marks off.  No counterpart on the pages: a
+ * measurement aid.  Always KAN_OK. */
+KAN_API kan_status kan_set_timing_marks(void* after_prep, void* after_dcoef);
+
+/* Calibration kernel for the CUDA-core fp32 roofline (the bound of the fp32
+ * path counts algorithmic FMAs): launches `blocks` blocks of 256 threads, each
+ * thread running 8 independent fp32 FMA chains for iters * 32 steps, and
+ * writes one float per thread to `sink` (device memory, blocks * 256 floats,
+ * so that the work is not optimised away).  *flops receives the FLOPs the
+ * launch executes (2 per FMA).  Asynchronous on `stream`; time it with events.
+ * No counterpart on the pages: a measurement aid.  KAN_ERR_INVALID_ARG for
+ * blocks < 1, iters < 1 or a null pointer. */
+KAN_API kan_status kan_ffma_probe(int32_t blocks, int64_t iters, float* sink, double* flops, void* stream);
 
 /* Static description of a status code. */
 KAN_API const char* kan_status_string(kan_status st);

@@ -19,7 +19,7 @@ STATUS = {0: "KAN_OK", 1: "KAN_ERR_INVALID_ARG", 2: "KAN_ERR_UNSUPPORTED", 3: "K
 
 #: every symbol the header declares
 EXPORTS = ("kan_abi_version", "kan_workspace_size", "kan_forward", "kan_backward", "kan_basis", "kan_sync_status",
-           "kan_launch_count", "kan_forward_fixed_scratch",
+           "kan_launch_count", "kan_forward_fixed_scratch", "kan_set_timing_marks", "kan_ffma_probe",
            "kan_selftest_wait_timeout", "kan_status_string", "kan_last_error")
 
 
@@ -71,6 +71,10 @@ def load(path: str | None = None):
     lib.kan_launch_count.argtypes = []
     lib.kan_forward_fixed_scratch.restype = ctypes.c_int
     lib.kan_forward_fixed_scratch.argtypes = [sp, _vp, _vp, _vp, _vp, _vp]
+    lib.kan_set_timing_marks.restype = ctypes.c_int
+    lib.kan_set_timing_marks.argtypes = [_vp, _vp]
+    lib.kan_ffma_probe.restype = ctypes.c_int
+    lib.kan_ffma_probe.argtypes = [ctypes.c_int32, ctypes.c_int64, _vp, ctypes.POINTER(ctypes.c_double), _vp]
     if path is None:
         _lib = lib
     return lib
@@ -114,6 +118,18 @@ def kan_backward(shape, x, coef, w_base, dY, dx, dcoef, dw_base, workspace, ws_b
 
 def kan_basis(shape, x, span, w, dw, stream):
     check(load().kan_basis(ctypes.byref(shape), x, span, w, dw, stream), "kan_basis")
+
+
+def kan_set_timing_marks(after_prep, after_dcoef):
+    """Events (cudaEvent_t handles as ints, or None) recorded inside later calls on this thread."""
+    check(load().kan_set_timing_marks(after_prep, after_dcoef), "kan_set_timing_marks")
+
+
+def kan_ffma_probe(blocks, iters, sink, stream) -> float:
+    """Launch the fp32 FMA calibration kernel; returns the FLOPs it executes."""
+    f = ctypes.c_double(0.0)
+    check(load().kan_ffma_probe(int(blocks), int(iters), sink, ctypes.byref(f), stream), "kan_ffma_probe")
+    return f.value
 
 
 def kan_sync_status(stream) -> int:

@@ -35,6 +35,15 @@ unsigned int* device_status_ptr()
 
 namespace {
 thread_local char g_last_error[512] = "";
+thread_local TimingMarks g_marks;
+}
+
+const TimingMarks& timing_marks() { return g_marks; }
+
+void set_timing_marks(void* after_prep, void* after_dcoef)
+{
+    g_marks.after_prep = reinterpret_cast<cudaEvent_t>(after_prep);
+    g_marks.after_dcoef = reinterpret_cast<cudaEvent_t>(after_dcoef);
 }
 
 kan_status set_last_error(kan_status st, const char* msg)
@@ -113,10 +122,9 @@ kan_status choose(const Problem& p, bool backward, bool* use_tc)
         *use_tc = true;
         return KAN_OK;
     }
-    // automatic: tiny problems are launch-bound either way; the CUDA-core
-    // kernels cover them (and every shape TMA cannot address)
-    const bool tiny = p.batch * p.in * p.out < ((int64_t)1 << 16);
-    *use_tc = ok && !tiny;
+    // automatic: the tensor-core kernels for every shape whose strides TMA can
+    // address; the CUDA-core kernels only for the others
+    *use_tc = ok;
     return KAN_OK;
 }
 
@@ -242,6 +250,12 @@ kan_status kan_selftest_wait_timeout(int64_t limit_ns, void* stream)
     if (!dp) return fail(KAN_ERR_CUDA, "device status word not available");
     cudaError_t e = simt_wait_selftest(limit_ns, dp, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kan_selftest_wait_timeout");
+    return KAN_OK;
+}
+
+kan_status kan_set_timing_marks(void* after_prep, void* after_dcoef)
+{
+    set_timing_marks(after_prep, after_dcoef);
     return KAN_OK;
 }
 

@@ -34,6 +34,16 @@ void count_launch(int n = 1);
 // Record the detail string that kan_last_error() returns on this thread.
 kan_status set_last_error(kan_status st, const char* msg);
 
+// Caller-provided timing marks (kan_set_timing_marks), per host thread:
+// events recorded on the call's stream after the operand preparation and, in
+// the backward, after the dcoef kernels.  Null members record nothing.
+struct TimingMarks {
+    cudaEvent_t after_prep = nullptr;
+    cudaEvent_t after_dcoef = nullptr;
+};
+const TimingMarks& timing_marks();
+inline cudaError_t record_mark(cudaEvent_t ev, cudaStream_t st) { return ev ? cudaEventRecord(ev, st) : cudaSuccess; }
+
 // ---- CUDA-core kernels (kan_simt.cu) ----
 cudaError_t simt_basis(const Problem& p, const void* x, int32_t* span, float* w, float* dw, cudaStream_t st);
 cudaError_t simt_forward(const Problem& p, const void* x, const void* coef, const void* w_base, void* y,

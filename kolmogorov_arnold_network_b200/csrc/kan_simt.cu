@@ -10,7 +10,6 @@ namespace {
 
 constexpr int kFwdRows = 4;       // batch rows per forward block
 constexpr int kFwdChunk = 512;    // inputs staged per pass in the forward block
-constexpr int kMaxNb = KAN_MAX_G + 3;
 
 template <typename T>
 __global__ void basis_kernel(const T* __restrict__ x, int64_t n, float lo, float inv_h, int G, int32_t* span,
@@ -96,7 +95,9 @@ __global__ void forward_kernel(const T* __restrict__ x, const T* __restrict__ co
     }
 }
 
-// dcoef[j, i, :], dw_base[j, i]: one thread per (j, i), batch summed in order.
+// dcoef[j, i, m] (m < nb) and dw_base[j, i] (m == nb): one thread per
+// (j, i, m), batch summed in order; each thread keeps one accumulator and adds
+// the weight of its own basis function when the input's span covers it.
 template <typename T>
 __global__ void dcoef_kernel(const T* __restrict__ x, const T* __restrict__ dY, float* __restrict__ dcoef,
                              float* __restrict__ dw_base, int64_t batch, int64_t in, int64_t out, int G, float lo,
@@ -104,29 +105,29 @@ __global__ void dcoef_kernel(const T* __restrict__ x, const T* __restrict__ dY, 
 {
     const int nb = G + 3;
     const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (e >= in * out) return;
-    const int64_t j = e / in, i = e % in;
-    float acc[kMaxNb];
-    for (int m = 0; m < nb; ++m) acc[m] = 0.f;
-    float accb = 0.f;
+    if (e >= in * out * (nb + 1)) return;
+    const int m = (int)(e % (nb + 1));
+    const int64_t ji = e / (nb + 1);
+    const int64_t j = ji / in, i = ji % in;
+    if (m == nb ? !dw_base : !dcoef) return;
+    float acc = 0.f;
     for (int64_t b = 0; b < batch; ++b) {
-        float xv = to_f(x[b * in + i]);
-        float g = to_f(dY[b * out + j]);
-        Span sp = span_of(xv, lo, inv_h, G);
-        if (sp.valid) {
+        const float xv = to_f(x[b * in + i]);
+        const float g = to_f(dY[b * out + j]);
+        if (m == nb) {
+            acc += silu_f(xv) * g;
+            continue;
+        }
+        const Span sp = span_of(xv, lo, inv_h, G);
+        const int q = m - sp.s;
+        if (sp.valid && q >= 0 && q < 4) {
             float wv[4];
             weights(sp.t, wv);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                int m = sp.s + q;
-                if (m >= 0 && m < nb) acc[m] += wv[q] * g;
-            }
+            acc += (q == 0 ? wv[0] : q == 1 ? wv[1] : q == 2 ? wv[2] : wv[3]) * g;   // (no indexed registers)
         }
-        if (dw_base) accb += silu_f(xv) * g;
     }
-    if (dcoef)
-        for (int m = 0; m < nb; ++m) dcoef[e * nb + m] = acc[m];
-    if (dw_base) dw_base[e] = accb;
+    if (m == nb) dw_base[ji] = acc;
+    else dcoef[ji * nb + m] = acc;
 }
 
 // dx[b, i]: one thread per (b, i), j summed in order.
@@ -207,6 +208,8 @@ cudaError_t simt_forward(const Problem& p, const void* x, const void* coef, cons
                          cudaStream_t st)
 {
     if (p.batch == 0) return cudaSuccess;
+    cudaError_t e = record_mark(timing_marks().after_prep, st);
+    if (e != cudaSuccess) return e;
     const int blocks = (int)((p.batch + kFwdRows - 1) / kFwdRows);
     const int threads = p.out >= 128 ? 128 : (int)((p.out + 31) / 32 * 32);
     if (p.dtype == KAN_F32) {
@@ -231,8 +234,9 @@ cudaError_t simt_backward(const Problem& p, const void* x, const void* coef, con
         if (dw_base && (e = zero_f32(dw_base, p.out * p.in, st)) != cudaSuccess) return e;
         return cudaSuccess;
     }
+    if ((e = record_mark(timing_marks().after_prep, st)) != cudaSuccess) return e;
     if (dcoef || dw_base) {
-        const int64_t n = p.in * p.out;
+        const int64_t n = p.in * p.out * (p.nb + 1);
         if (p.dtype == KAN_F32) {
             dcoef_kernel<float><<<blocks_for(n, 128), 128, 0, st>>>((const float*)x, (const float*)dY, dcoef, dw_base,
                                                                      p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
@@ -245,6 +249,7 @@ cudaError_t simt_backward(const Problem& p, const void* x, const void* coef, con
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if ((e = record_mark(timing_marks().after_dcoef, st)) != cudaSuccess) return e;
     if (dx) {
         const int64_t n = p.batch * p.in;
         if (p.dtype == KAN_F32) {

@@ -1063,7 +1063,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                     if (j0 + e < ncols) dst[e] = __float2bfloat16_rn(v[e]);
                             }
                         } else {
-                            if (j0 + 16 <= ncols) {
+                            if (j0 + 16 <= ncols && (ncols & 3) == 0) {
 #pragma unroll
                                 for (int e = 0; e < 16; e += 4)
                                     *reinterpret_cast<float4*>(dst + e) =
@@ -1797,6 +1797,24 @@ __global__ void split_f16_kernel(const float* __restrict__ src, uint16_t* __rest
     }
 }
 
+// The same split for a [rows, cols] matrix whose copy has rows of ld >= cols
+// elements (ld % 8 == 0, so that the copy's rows are 16-byte aligned for TMA);
+// the padding columns are written as 0.  One element per thread step.
+__global__ void split_f16_rows_kernel(const float* __restrict__ src, uint16_t* __restrict__ hi,
+                                      uint16_t* __restrict__ lo, int64_t rows, int64_t cols, int64_t ld,
+                                      const unsigned int* __restrict__ amax)
+{
+    const float sc = scales_of(amax).d;
+    const int64_t n = rows * ld;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = e / ld, c = e - r * ld;
+        uint16_t h = 0, l = 0;
+        if (c < cols) split_f16(src[r * cols + c] * sc, h, l);
+        hi[e] = h;
+        lo[e] = l;
+    }
+}
+
 // fp16 hi/lo split of the coefficient matrix, row-major [out][in*nbx]:
 // column i*nbx + m is coef[j, i, m] * s_c for m < nbs, and (with the SiLU
 // branch, nbx = nbs + 1) w_base[j, i] * s_c / s_x for m == nbs.  Rows j step
@@ -1973,6 +1991,8 @@ struct Layout {
 };
 
 struct Plan {
+    // row length of the fp16 copies of dY (fp32: out rounded up to 8, so that TMA can address them)
+    int64_t ldo;
     // fp32 with the SiLU branch: interleaved coefficient copies (nbx = G+4
     // columns per input, Kx = in * nbx); otherwise nbx = G+3 and Kx = Kt
     bool ext;
@@ -2001,6 +2021,7 @@ Plan make_plan(const Problem& p, int sms)
     const bool f32 = p.dtype == KAN_F32;
     const int BK = 64;   // K elements per 128-byte operand row (2-byte operands, both dtypes)
     P.ext = f32 && p.base;
+    P.ldo = f32 ? (p.out + 7) / 8 * 8 : p.out;
     P.nbx = p.nb + (P.ext ? 1 : 0);
     P.Kx = p.in * P.nbx;
     const bool sep_silu = p.base && !P.ext;   // separate SiLU k-blocks / tiles / GEMM
@@ -2106,7 +2127,7 @@ Plan make_plan(const Problem& p, int sms)
         P.bwd.coef_hl = o;
         o += 2 * al256((size_t)p.out * P.Kx * 2);
         P.bwd.dy_hl = o;
-        o += 2 * al256((size_t)p.batch * p.out * 2);
+        o += 2 * al256((size_t)p.batch * P.ldo * 2);
     }
     if (P.d_splits > 1) {
         P.bwd.dc_part = o;
@@ -2297,14 +2318,17 @@ cudaError_t split_coef_into(const Problem& p, const Plan& P, const void* coef, c
     return cudaGetLastError();
 }
 
-// fp16 hi/lo copies of dY, [batch][out]; returns the (hi, lo) pointers.
-cudaError_t split_dy_into(const Problem& p, const void* dY, uint8_t* dst, const unsigned int* amax, const void** hi,
-                          const void** lo, cudaStream_t st)
+// fp16 hi/lo copies of dY, [batch][ldo] (ldo = out rounded up to 8); returns the (hi, lo) pointers.
+cudaError_t split_dy_into(const Problem& p, int64_t ldo, const void* dY, uint8_t* dst, const unsigned int* amax,
+                          const void** hi, const void** lo, cudaStream_t st)
 {
-    const int64_t n = p.batch * p.out;
+    const int64_t n = p.batch * ldo;
     uint16_t* h = reinterpret_cast<uint16_t*>(dst);
     uint16_t* l = reinterpret_cast<uint16_t*>(dst + al256((size_t)n * 2));
-    split_f16_kernel<<<grid_for(n / 4), 256, 0, st>>>((const float*)dY, h, l, n, amax);
+    if (ldo == p.out)
+        split_f16_kernel<<<grid_for(n / 4), 256, 0, st>>>((const float*)dY, h, l, n, amax);
+    else
+        split_f16_rows_kernel<<<grid_for(n), 256, 0, st>>>((const float*)dY, h, l, p.batch, p.out, ldo, amax);
     count_launch();
     *hi = h;
     *lo = l;
@@ -2329,8 +2353,9 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
         *why = "in*2 is not a multiple of 16 bytes (TMA row stride of w_base)";
         return false;
     }
-    if ((p.out * 2) % 16 != 0) {
-        *why = "out is not a multiple of 8 (TMA row stride of the dY operand, vector stores of y)";
+    if (!f32 && (p.out * 2) % 16 != 0) {
+        // (fp32 reads dY through its fp16 copies, whose rows are padded to 8 elements)
+        *why = "bf16 with out not a multiple of 8 (TMA row stride of dY)";
         return false;
     }
     if (nbx > 121 && (f32 || nbx > 249)) {
@@ -2367,6 +2392,7 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
         if ((e = split_coef_into(p, P, coef, w_base, w + P.fwd.coef_hl, amax, &c_hi, &c_lo, st)) != cudaSuccess)
             return e;
     }
+    if ((e = record_mark(timing_marks().after_prep, st)) != cudaSuccess) return e;
     CUtensorMap maps[6];
     // (a pair's CTA loads 128 + (BN - 256) / 2 rows of each B tile: boxes of 64 rows for BN = 384)
     const int fbox = P.f_pair && P.f_BN == 384 ? 64 : std::min(P.f_BN, 128);
@@ -2430,20 +2456,24 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         return cudaSuccess;
     }
     unsigned int* amax = f32 ? reinterpret_cast<unsigned int*>(w + P.bwd.amax) : nullptr;
-    const void *dy_hi = dY, *dy_lo = dY;
+    const void *dy_hi = dY, *dy_lo = dY, *c_hi = coef, *c_lo = coef;
     if (f32) {
         // operand scales (coef and w_base for dx's coefficient copy, x for the
-        // SiLU values, dY), then dY's fp16 hi/lo copy, shared by dcoef and dx
-        // (coef and w_base scale only dx's coefficient copy)
+        // SiLU values, dY), then dY's fp16 hi/lo copy, shared by dcoef and dx,
+        // and (for dx) the coefficients' copy
         if ((e = amax_into(p, dx ? coef : nullptr, dx ? w_base : nullptr, x, dY, amax, st)) != cudaSuccess) return e;
-        if ((e = split_dy_into(p, dY, w + P.bwd.dy_hl, amax, &dy_hi, &dy_lo, st)) != cudaSuccess) return e;
+        if ((e = split_dy_into(p, P.ldo, dY, w + P.bwd.dy_hl, amax, &dy_hi, &dy_lo, st)) != cudaSuccess) return e;
+        if (dx && (e = split_coef_into(p, P, coef, w_base, w + P.bwd.coef_hl, amax, &c_hi, &c_lo, st)) != cudaSuccess)
+            return e;
     }
+    if ((e = record_mark(timing_marks().after_prep, st)) != cudaSuccess) return e;
     // ---- dcoef / dw_base: A = basis^T (producers), B = dY MN-major (BK-batch x 64-output boxes) ----
     if (dcoef || dw_base) {
         CUtensorMap maps[6];
-        if (!make_map_2d(&maps[2], dy_hi, f32, p.batch, p.out, BK, EPB, detail)) return cudaErrorInvalidValue;
+        if (!make_map_2d(&maps[2], dy_hi, f32, p.batch, p.out, BK, EPB, detail, P.ldo)) return cudaErrorInvalidValue;
         if (f32) {
-            if (!make_map_2d(&maps[3], dy_lo, true, p.batch, p.out, BK, EPB, detail)) return cudaErrorInvalidValue;
+            if (!make_map_2d(&maps[3], dy_lo, true, p.batch, p.out, BK, EPB, detail, P.ldo))
+                return cudaErrorInvalidValue;
         } else {
             maps[3] = maps[2];
         }
@@ -2477,6 +2507,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
     }
+    if ((e = record_mark(timing_marks().after_dcoef, st)) != cudaSuccess) return e;
     // ---- dx: A = dY K-major, B = coef MN-major (fp32: their fp16 hi/lo copies) ----
     if (dx) {
         float* gb = nullptr;
@@ -2499,12 +2530,10 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             if (e != cudaSuccess) return e;
         }
         CUtensorMap maps[6];
-        if (!make_map_2d(&maps[0], dy_hi, f32, p.batch, p.out, kBM, BK, detail)) return cudaErrorInvalidValue;
+        if (!make_map_2d(&maps[0], dy_hi, f32, p.batch, p.out, kBM, BK, detail, P.ldo)) return cudaErrorInvalidValue;
         if (f32) {
-            if (!make_map_2d(&maps[1], dy_lo, true, p.batch, p.out, kBM, BK, detail)) return cudaErrorInvalidValue;
-            const void *c_hi, *c_lo;
-            if ((e = split_coef_into(p, P, coef, w_base, w + P.bwd.coef_hl, amax, &c_hi, &c_lo, st)) != cudaSuccess)
-                return e;
+            if (!make_map_2d(&maps[1], dy_lo, true, p.batch, p.out, kBM, BK, detail, P.ldo))
+                return cudaErrorInvalidValue;
             if (!make_map_2d(&maps[2], c_hi, true, p.out, P.Kx, BK, EPB, detail) ||
                 !make_map_2d(&maps[3], c_lo, true, p.out, P.Kx, BK, EPB, detail))
                 return cudaErrorInvalidValue;

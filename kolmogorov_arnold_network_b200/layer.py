@@ -47,7 +47,12 @@ def _stream(t):
 
 
 def workspace(shape: N.kan_shape, for_backward: bool, device) -> torch.Tensor | None:
-    n = N.kan_workspace_size(shape, for_backward)
+    device = torch.device(device)
+    if device.type == "cuda":
+        with torch.cuda.device(device):
+            n = N.kan_workspace_size(shape, for_backward)
+    else:
+        n = N.kan_workspace_size(shape, for_backward)
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
@@ -64,7 +69,9 @@ def forward(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, y=None, ws=No
     _check(y, "y", x.dtype, (batch, n_out))
     if ws is None:
         ws = workspace(s, False, x.device)
-    N.kan_forward(s, _p(x), _p(coef), _p(w_base), _p(y), _p(ws), 0 if ws is None else ws.numel(), _stream(x))
+    # the library works on the current device: make it x's
+    with torch.cuda.device(x.device):
+        N.kan_forward(s, _p(x), _p(coef), _p(w_base), _p(y), _p(ws), 0 if ws is None else ws.numel(), _stream(x))
     return y
 
 
@@ -87,8 +94,9 @@ def backward(x, coef, dY, G, lo, hi, w_base=None, need_dx=True, need_dcoef=True,
                if (need_dw_base and w_base is not None) else None)
     if ws is None:
         ws = workspace(s, True, x.device)
-    N.kan_backward(s, _p(x), _p(coef), _p(w_base), _p(dY), _p(dx), _p(dcoef), _p(dwb), _p(ws),
-                   0 if ws is None else ws.numel(), _stream(x))
+    with torch.cuda.device(x.device):
+        N.kan_backward(s, _p(x), _p(coef), _p(w_base), _p(dY), _p(dx), _p(dcoef), _p(dwb), _p(ws),
+                       0 if ws is None else ws.numel(), _stream(x))
     return dx, dcoef, dwb
 
 
@@ -100,7 +108,8 @@ def basis(x, G, lo, hi):
     span = torch.empty((batch, n_in), dtype=torch.int32, device=x.device)
     w = torch.empty((batch, n_in, 4), dtype=torch.float32, device=x.device)
     dw = torch.empty((batch, n_in, 4), dtype=torch.float32, device=x.device)
-    N.kan_basis(s, _p(x), _p(span), _p(w), _p(dw), _stream(x))
+    with torch.cuda.device(x.device):
+        N.kan_basis(s, _p(x), _p(span), _p(w), _p(dw), _stream(x))
     return span, w, dw
 
 

@@ -78,8 +78,8 @@ WORKLOADS = {
                                  ("normal", 1.0), 0.05, note="KAN FFN block 768->3072->768, 8192 tokens"),
 }
 
-#: the workload the benchmark times by default
-BENCH_DEFAULT = "layer784x64_silu"
+#: the workload the benchmark times by default: the largest single-GPU one by edge evaluations per step
+BENCH_DEFAULT = "ffn768_3072_bf16"
 
 
 def _gen(family: int, tensor_id: int) -> torch.Generator:

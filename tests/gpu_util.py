@@ -43,6 +43,22 @@ def sample_cols(n, k=12, seed=1):
     return np.array(sorted(c))
 
 
+def tile_rows(batch, tile=128):
+    """Every row of the first two batch tiles (a whole CTA pair of the paired kernels) and of the last
+    batch tile (ragged or not)."""
+    first = np.arange(min(batch, 2 * tile))
+    last = np.arange(((batch - 1) // tile) * tile, batch)
+    return np.unique(np.concatenate([first, last]))
+
+
+def tile_inputs(n_in, nb, tile=128):
+    """The inputs whose basis columns (nb per input) fall in the first two 128-column M tiles of the
+    dcoef GEMM (a whole CTA pair) or in its last M tile."""
+    kt = n_in * nb
+    cols = np.concatenate([np.arange(min(kt, 2 * tile)), np.arange(((kt - 1) // tile) * tile, kt)])
+    return np.unique(cols // nb)
+
+
 def gpu_layer(x, coef, w_base, dY, G, lo, hi, path=0, want_bwd=True):
     """Run forward (+ backward) through the C ABI on CUDA tensors; returns CUDA tensors."""
     y = L.forward(x, coef, G, lo, hi, w_base, path=path)

@@ -13,9 +13,10 @@ Sources of the facts:
   P3  non-negativity (InKAN landing page, "Numerically Stable"), local
       support over 4 knot intervals (InKAN landing page, "What is a KAN?").
   P4  exact local weights of the uniform cubic B-spline
-      (tests/golden/cubic_bspline_local_weights.txt).
-  P5  Marsden's identity, cubic polynomial reproduction (textbook), through
-      the layer forward and dx.
+      (tests/golden/cubic_bspline_local_weights.txt); for degrees 1-5, the
+      weights at a knot (Eulerian numbers over k!, textbook).
+  P5  Marsden's identity, degree-k polynomial reproduction (textbook),
+      through the layer forward and dx.
   P6  finite differences of <dY, y(x)> against dx.
   P7  dcoef and dw_base entries equal <dY, y(one-hot parameter)>.
   P8  bilinear adjoint identity <dY, y> = <dcoef, coef> + <dw_base, w_base>.
@@ -93,7 +94,10 @@ def pin_partition_of_unity(o, grids=((8, -1.0, 1.0), (20, -1.0, 1.0), (5, -3.0, 
         B, dB = o.basis(inside, G, lo, hi, k=k)
         if np.max(np.abs(B.sum(1) - 1.0)) > 1e-14:
             return f"P2 G={G}: sum B != 1 inside [lo,hi]"
-        if np.max(np.abs(dB.sum(1))) * h > 1e-13:
+        # (degree 1 is not differentiable at the knots; with half-open intervals its derivative at
+        # x = hi is the right-hand one, taken in the extended interval, so hi itself is left out)
+        dsum = dB.sum(1) if k > 1 else dB[:-1].sum(1)
+        if np.max(np.abs(dsum)) * h > 1e-13:
             return f"P2 G={G}: sum B' != 0 inside [lo,hi]"
         ext = np.concatenate([np.linspace(lo - k * h, lo, 200, endpoint=False)[1:],
                               np.linspace(hi, hi + k * h, 200, endpoint=False)[1:]])
@@ -101,7 +105,7 @@ def pin_partition_of_unity(o, grids=((8, -1.0, 1.0), (20, -1.0, 1.0), (5, -3.0, 
         s = Be.sum(1)
         if not (np.all(s < 1.0 - 1e-15) and np.all(s > 0.0)):
             return f"P2 G={G}: sum B not in (0,1) in the extended intervals"
-        beyond = np.array([lo - k * h - 1e-9, lo - k * h - 0.5, hi + k * h, hi + k * h + 0.3, -np.inf, np.inf])
+        beyond = np.array([lo - k * h - 1e-9, lo - k * h - 0.5, hi + k * h + 1e-9, hi + k * h + 0.3, -np.inf, np.inf])
         Bb, dBb = o.basis(beyond, G, lo, hi, k=k)
         if np.any(Bb != 0.0) or np.any(dBb != 0.0):
             return f"P2 G={G}: basis not zero beyond the extended knots"
@@ -109,11 +113,13 @@ def pin_partition_of_unity(o, grids=((8, -1.0, 1.0), (20, -1.0, 1.0), (5, -3.0, 
 
 
 def pin_nonneg_local(o, grids=((8, -1.0, 1.0), (20, -1.0, 1.0), (5, -3.0, 3.0)), k=3):
+    # the cubic B-spline peaks at 2/3 (its value at the middle knot); any degree stays within [0, 1]
+    top = 2.0 / 3.0 if k == 3 else 1.0
     for G, lo, hi in grids:
         x = _sweep(G, lo, hi, k)
         B, _ = o.basis(x, G, lo, hi, k=k)
-        if np.any(B < 0.0) or np.any(B > 2.0 / 3.0 + 1e-15):
-            return f"P3 G={G}: basis outside [0, 2/3]"
+        if np.any(B < 0.0) or np.any(B > top + 1e-15):
+            return f"P3 k={k} G={G}: basis outside [0, {top}]"
         if np.max((B != 0.0).sum(1)) > k + 1:
             return f"P3 G={G}: more than k+1 non-zero basis values"
         t = knots_np(G, lo, hi, k)
@@ -156,61 +162,89 @@ def pin_exact_values(o):
     return None
 
 
-def marsden_coef(targets, G, lo, hi):
-    """coef[j,i,m] = psi_m(y_ji) = (y-t_{m+1})(y-t_{m+2})(y-t_{m+3}) for y = targets[j,i]."""
-    t = knots_np(G, lo, hi)
+def marsden_coef(targets, G, lo, hi, k=3):
+    """coef[j,i,m] = psi_m(y_ji) = prod_{l=1..k} (y - t_{m+l}) for y = targets[j,i] (Marsden's identity:
+    sum_m psi_m(y) B_m(x) = (y - x)^k for x in [lo, hi], degree-k B-splines)."""
+    t = knots_np(G, lo, hi, k)
     y = np.asarray(targets, dtype=np.float64)[..., None]
-    m = np.arange(G + 3)
-    return (y - t[m + 1]) * (y - t[m + 2]) * (y - t[m + 3])
+    m = np.arange(G + k)
+    out = np.ones(y.shape[:-1] + (G + k,))
+    for l in range(1, k + 1):
+        out = out * (y - t[m + l])
+    return out
 
 
-def pin_marsden(o, rng=None):
+def pin_marsden(o, rng=None, k=3):
     rng = rng or np.random.default_rng(11)
     for G, lo, hi in ((8, -1.0, 1.0), (5, -3.0, 3.0), (20, -1.0, 1.0)):
         batch, n_in, n_out = 37, 6, 3
         x = rng.uniform(lo, hi, size=(batch, n_in))
         x[0, 0], x[1, 1] = lo, hi - 1e-12
         yt = rng.uniform(-2, 2, size=(n_out, n_in))
-        coef = marsden_coef(yt, G, lo, hi)
-        y = o.forward(x, coef, G, lo, hi)
-        ref = ((yt[None, :, :] - x[:, None, :]) ** 3).sum(2)
+        coef = marsden_coef(yt, G, lo, hi, k)
+        y = o.forward(x, coef, G, lo, hi, k=k)
+        ref = ((yt[None, :, :] - x[:, None, :]) ** k).sum(2)
         if np.max(np.abs(y - ref)) > 1e-12 * max(1.0, np.max(np.abs(ref))):
-            return f"P5 G={G}: forward != sum_i (y_ji - x_bi)^3"
+            return f"P5 k={k} G={G}: forward != sum_i (y_ji - x_bi)^k"
         dY = rng.normal(size=(batch, n_out))
-        dx, _, _ = o.backward(x, coef, dY, G, lo, hi)
-        dref = np.einsum("bj,bji->bi", dY, -3.0 * (yt[None, :, :] - x[:, None, :]) ** 2)
+        dx, _, _ = o.backward(x, coef, dY, G, lo, hi, k=k)
+        dref = np.einsum("bj,bji->bi", dY, -k * (yt[None, :, :] - x[:, None, :]) ** (k - 1))
         if np.max(np.abs(dx - dref)) > 1e-11 * max(1.0, np.max(np.abs(dref))):
-            return f"P5 G={G}: dx != -3 sum_j dY_bj (y_ji - x_bi)^2"
+            return f"P5 k={k} G={G}: dx != -k sum_j dY_bj (y_ji - x_bi)^(k-1)"
     return None
 
 
-def _small_problem(rng, G, lo, hi, base, batch=32, n_in=8, n_out=4):
+def pin_knot_values_eulerian(o, degrees=(1, 2, 3, 4, 5)):
+    """At a knot, the k+1 local weights of the uniform degree-k B-spline are the Eulerian numbers
+    A(k, 0..k-1) over k! followed by 0 (textbook: the cardinal B-spline at the integers)."""
+    euler = {1: (1,), 2: (1, 1), 3: (1, 4, 1), 4: (1, 11, 11, 1), 5: (1, 26, 66, 26, 1)}
+    G, lo, hi = 8, -1.0, 1.0
+    h = (hi - lo) / G
+    for k in degrees:
+        want = [a / math.factorial(k) for a in euler[k]] + [0.0]
+        for s in (-k, 0, 3, G - 1):
+            x = lo + s * h
+            B, _ = o.basis([x], G, lo, hi, k=k)
+            for r in range(k + 1):
+                m = s + r
+                if 0 <= m < G + k and abs(B[0, m] - want[r]) > 1e-14:
+                    return f"P4 k={k} s={s}: B_{m} at the knot = {B[0, m]!r} != {want[r]}"
+    return None
+
+
+def _small_problem(rng, G, lo, hi, base, batch=32, n_in=8, n_out=4, k=3):
     h = (hi - lo) / G
     x = rng.uniform(lo - 2 * h, hi + 2 * h, size=(batch, n_in))
-    coef = rng.normal(0, 0.1, size=(n_out, n_in, G + 3))
+    coef = rng.normal(0, 0.1, size=(n_out, n_in, G + k))
     wb = rng.normal(0, 0.3, size=(n_out, n_in)) if base else None
     dY = rng.normal(size=(batch, n_out))
     return x, coef, wb, dY
 
 
-def pin_finite_difference(o, rng=None):
+def pin_finite_difference(o, rng=None, k=3):
     rng = rng or np.random.default_rng(12)
     G, lo, hi = 8, -1.0, 1.0
     for base in (False, True):
-        x, coef, wb, dY = _small_problem(rng, G, lo, hi, base)
-        dx, _, _ = o.backward(x, coef, dY, G, lo, hi, w_base=wb)
+        x, coef, wb, dY = _small_problem(rng, G, lo, hi, base, k=k)
+        dx, _, _ = o.backward(x, coef, dY, G, lo, hi, w_base=wb, k=k)
         eps = 1e-6
         fd = np.zeros_like(x)
         for b in range(x.shape[0]):
             for i in range(x.shape[1]):
                 xp = x.copy(); xp[b, i] += eps
                 xm = x.copy(); xm[b, i] -= eps
-                yp = o.forward(xp[b:b + 1], coef, G, lo, hi, w_base=wb)
-                ym = o.forward(xm[b:b + 1], coef, G, lo, hi, w_base=wb)
+                yp = o.forward(xp[b:b + 1], coef, G, lo, hi, w_base=wb, k=k)
+                ym = o.forward(xm[b:b + 1], coef, G, lo, hi, w_base=wb, k=k)
                 fd[b, i] = float(((yp - ym) * dY[b:b + 1]).sum()) / (2 * eps)
-        err = np.max(np.abs(fd - dx)) / np.max(np.abs(dx))
+        # degree 1 has kinks at the knots: leave out inputs within eps of one
+        if k == 1:
+            u = (x - lo) / ((hi - lo) / G)
+            far = np.abs(u - np.round(u)) > 1e-4
+        else:
+            far = np.ones_like(x, dtype=bool)
+        err = np.max(np.abs(fd - dx)[far]) / np.max(np.abs(dx))
         if not err <= 1e-7:
-            return f"P6 base={base}: dx vs central differences rel err {err:.2e}"
+            return f"P6 k={k} base={base}: dx vs central differences rel err {err:.2e}"
     return None
 
 
@@ -293,7 +327,8 @@ def pin_one_hot(o, rng=None):
 
 
 ALL_PINS = [pin_truncated_power, pin_partition_of_unity, pin_nonneg_local, pin_exact_values, pin_marsden,
-            pin_finite_difference, pin_param_gradients, pin_adjoint, pin_library_matmul, pin_one_hot]
+            pin_finite_difference, pin_param_gradients, pin_adjoint, pin_library_matmul, pin_one_hot,
+            pin_knot_values_eulerian]
 
 
 def run_all(o):

@@ -16,7 +16,7 @@ from kolmogorov_arnold_network_b200 import workloads as W
 
 import pins
 from gpu_util import (TOL, check_layer_against_oracle, cuda, f64, gpu_layer, rel_err, sample_cols, sample_rows,
-                      workload_inputs)
+                      tile_inputs, tile_rows, workload_inputs)
 
 pytestmark = pytest.mark.gpu
 
@@ -143,14 +143,30 @@ def test_workload_parity(oracle, name):
     torch.cuda.synchronize()
     assert N.kan_sync_status(None) == 0
     small = w.batch * Ly.inp * Ly.out <= 4096 * 784 * 64
-    rows = None if small else sample_rows(w.batch)
-    ci = None if small else sample_cols(Ly.inp)
-    co = None if small else sample_cols(Ly.out)
+    # large workloads: every row of whole batch tiles (the first CTA pair and the last, ragged tile) plus a
+    # random sample; dcoef for every output of the inputs of whole M tiles (the first pair, the last tile)
+    rows = None if small else np.union1d(tile_rows(w.batch), sample_rows(w.batch))
+    ci = None if small else tile_inputs(Ly.inp, Ly.G + 3)
+    co = None if small else np.arange(Ly.out)
     errs = check_layer_against_oracle(oracle, x, coef, wb, dY, Ly.G, Ly.lo, Ly.hi, y.cpu(), dx.cpu(), dc.cpu(),
                                       None if dwb is None else dwb.cpu(), w.dtype, rows=rows, cols_in=ci,
                                       cols_out=co)
     bad = {k: v for k, v in errs.items() if not v <= TOL[w.dtype]}
     assert not bad, f"{errs}"
+
+
+def test_tiny_layer_on_the_tensor_path(oracle):
+    # KANLayer(8, 4) (out = 4, fp32): the fp16 copies of dY are padded to 8 columns for TMA
+    w = W.WORKLOADS["layer8x4"]
+    Ly = w.layers[0]
+    x, coef, wb, dY = workload_inputs(w)
+    y, dx, dc, dwb = gpu_layer(cuda(x), cuda(coef), cuda(wb), cuda(dY), Ly.G, Ly.lo, Ly.hi,
+                               path=N.KAN_PATH_TENSOR)
+    torch.cuda.synchronize()
+    assert N.kan_sync_status(None) == 0
+    errs = check_layer_against_oracle(oracle, x, coef, wb, dY, Ly.G, Ly.lo, Ly.hi, y.cpu(), dx.cpu(), dc.cpu(),
+                                      None, w.dtype)
+    assert all(v <= TOL[w.dtype] for v in errs.values()), errs
 
 
 def test_ffn_block_parity(oracle):
@@ -165,13 +181,16 @@ def test_ffn_block_parity(oracle):
     dx, dc1, _ = L.backward(xg, c1g, dh, L1.G, L1.lo, L1.hi)
     torch.cuda.synchronize()
     assert N.kan_sync_status(None) == 0
-    rows = sample_rows(w.batch, 16)
+    rows = np.union1d(tile_rows(w.batch), sample_rows(w.batch, 16))
     tol = TOL["bf16"]
-    # per layer, each fed the GPU's own bf16 inputs
+    # per layer, each fed the GPU's own bf16 inputs; whole batch tiles, and dcoef for every output of the
+    # inputs of whole M tiles
     e1 = check_layer_against_oracle(oracle, x, c1, None, dh.cpu(), L1.G, L1.lo, L1.hi, h.cpu(), dx.cpu(), dc1.cpu(),
-                                    None, "bf16", rows=rows, cols_in=sample_cols(L1.inp), cols_out=sample_cols(L1.out))
+                                    None, "bf16", rows=rows, cols_in=tile_inputs(L1.inp, L1.G + 3),
+                                    cols_out=np.arange(L1.out))
     e2 = check_layer_against_oracle(oracle, h.cpu(), c2, None, dY, L2.G, L2.lo, L2.hi, y.cpu(), dh.cpu(), dc2.cpu(),
-                                    None, "bf16", rows=rows, cols_in=sample_cols(L2.inp), cols_out=sample_cols(L2.out))
+                                    None, "bf16", rows=rows, cols_in=tile_inputs(L2.inp, L2.G + 3),
+                                    cols_out=np.arange(L2.out))
     # end to end, the oracle's h in fp64 (not re-rounded)
     h_ref = oracle.forward(x[rows], c1, L1.G, L1.lo, L1.hi)
     y_ref = oracle.forward(h_ref, c2, L2.G, L2.lo, L2.hi)
@@ -268,7 +287,7 @@ def test_deterministic(name):
     Ly = w.layers[0]
     x, coef, wb, dY = [cuda(t) for t in workload_inputs(w)]
     first = gpu_layer(x, coef, wb, dY, Ly.G, Ly.lo, Ly.hi)
-    for _ in range(3):
+    for _ in range(10):
         again = gpu_layer(x, coef, wb, dY, Ly.G, Ly.lo, Ly.hi)
         for a, b in zip(first, again):
             if a is not None:

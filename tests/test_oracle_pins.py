@@ -22,6 +22,17 @@ def test_truncated_power_general_degree(oracle):
     assert pins.pin_truncated_power(oracle, grids=((8, -1.0, 1.0), (5, -3.0, 3.0)), degrees=(1, 2, 4, 5)) is None
 
 
+@pytest.mark.parametrize("k", [1, 2, 4, 5])
+def test_general_degree_pins(oracle, k):
+    # Spline degree k (the FlashKAN abstract: "k sequential passes for degree-k splines", normalised
+    # coordinate clamped to [0, k+1]): partition of unity, non-negativity and k+1 non-zeros,
+    # degree-k polynomial reproduction through forward and dx, and finite differences.
+    assert pins.pin_partition_of_unity(oracle, k=k) is None
+    assert pins.pin_nonneg_local(oracle, k=k) is None
+    assert pins.pin_marsden(oracle, k=k) is None
+    assert pins.pin_finite_difference(oracle, k=k) is None
+
+
 def test_golden_rows_sum(oracle):
     # the fixture itself: weights sum to 1, derivatives to 0 (exact rationals)
     for row in pins.read_golden():
