@@ -105,25 +105,25 @@ def csrc_hash() -> str:
 # ---------------------------------------------------------------------------
 # FLOP / byte accounting (per call, algorithmic)
 def layer_dense_flops(batch, L):
-    """Dense-expanded FLOPs of one layer GEMM: 2 * batch * out * (in*(G+3) [+ in for SiLU])."""
-    k = L.inp * (L.G + 3) + (L.inp if L.base else 0)
+    """Dense-expanded FLOPs of one layer GEMM: 2 * batch * out * (in*(G+k) [+ in for SiLU])."""
+    k = L.inp * L.nb + (L.inp if L.base else 0)
     return 2.0 * batch * L.out * k
 
 
 def layer_alg_flops(batch, L):
-    """Algorithmic FLOPs of one layer GEMM: 4 FMAs per edge (+1 with SiLU), 2 FLOPs each."""
-    return (8.0 + (2.0 if L.base else 0.0)) * batch * L.inp * L.out
+    """Algorithmic FLOPs of one layer GEMM: k+1 FMAs per edge (4 for cubic splines; +1 with SiLU), 2 FLOPs each."""
+    return (2.0 * (L.degree + 1) + (2.0 if L.base else 0.0)) * batch * L.inp * L.out
 
 
 def layer_bytes(batch, L, esz, call):
     """Algorithmic HBM bytes of one call: operands read once, outputs written once."""
     x = batch * L.inp * esz
     dy = batch * L.out * esz
-    coef = L.out * L.inp * (L.G + 3) * esz + (L.out * L.inp * esz if L.base else 0)
+    coef = L.out * L.inp * L.nb * esz + (L.out * L.inp * esz if L.base else 0)
     if call == "fwd":
         return x + coef + batch * L.out * esz
     if call == "dcoef":
-        return x + dy + (L.out * L.inp * (L.G + 3) + (L.out * L.inp if L.base else 0)) * 4
+        return x + dy + (L.out * L.inp * L.nb + (L.out * L.inp if L.base else 0)) * 4
     return x + dy + coef + batch * L.inp * esz          # dx
 
 
@@ -169,7 +169,7 @@ class Runner:
         for li, L in enumerate(w.layers):
             coef = d[f"coef{li}"].to(dev)
             wb = None if d[f"w_base{li}"] is None else d[f"w_base{li}"].to(dev)
-            s = LY.shape_of(act, coef, L.G, L.lo, L.hi, wb)
+            s = LY.shape_of(act, coef, L.G, L.lo, L.hi, wb, degree=L.degree)
             ws_f = LY.workspace(s, False, dev)
             ws_b = LY.workspace(s, True, dev)
             y = torch.empty((w.batch, L.out), dtype=dt, device=dev)
@@ -470,11 +470,12 @@ def cpu_baseline(w: W.Workload, target_s=12.0):
         acts = []
         for li, L in enumerate(w.layers):
             acts.append(act)
-            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], nthreads=cores)
+            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
+                            nthreads=cores)
         g = dY
         for li in (reversed(range(len(w.layers))) if w.mode != "fwd" else ()):
             L = w.layers[li]
-            gx, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"],
+            gx, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
                                   nthreads=cores)
             g = gx
         return time.perf_counter() - t0
@@ -512,11 +513,12 @@ def run_reference(args, world, rank):
         acts = []
         for li, L in enumerate(w.layers):
             acts.append(act)
-            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], nthreads=cores)
+            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
+                            nthreads=cores)
         g = d["dY"][:rows]
         for li in (reversed(range(len(w.layers))) if w.mode != "fwd" else ()):
             L = w.layers[li]
-            g, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"],
+            g, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
                                  nthreads=cores)
 
     # size the per-step sample so that warmup + steps end within ~2 minutes
@@ -547,7 +549,8 @@ def run_reference(args, world, rank):
 def config_of(w: W.Workload):
     L0 = w.layers[0]
     c = {"workload": w.name, "batch": w.batch, "layers": [[L.inp, L.out] for L in w.layers], "G": L0.G,
-         "grid": [L0.lo, L0.hi], "silu_base": L0.base, "mode": w.mode, "l2": "256 MiB flush between steps",
+         "degree": L0.degree, "grid": [L0.lo, L0.hi], "silu_base": L0.base, "mode": w.mode,
+         "l2": "256 MiB flush between steps",
          "note": w.note}
     if w.dtype == "f32":
         c["compute"] = ("fp32 operands as fp16 hi/lo splits (power-of-two scaled), 3 fp16 tensor-core products, "
@@ -559,7 +562,8 @@ def config_of(w: W.Workload):
 
 #: workloads timed beside the headline one (each in the same JSON line, with the adjoint-identity check)
 EXTRA_WORKLOADS = ["layer784x64_silu", "layer1024_g20_bf16"] + \
-    [f"sweep512_g{G}_{dt}_fwdbwd" for G in (8, 20, 50) for dt in ("bf16", "f32")]
+    [f"sweep512_g{G}_{dt}_fwdbwd" for G in (8, 20, 50) for dt in ("bf16", "f32")] + \
+    [f"degree512_k{k}_g20_bf16_fwdbwd" for k in (1, 2, 4, 5)]
 
 
 def run_ours(args, world, rank, local):

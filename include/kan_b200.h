@@ -4,18 +4,22 @@
  *
  * The operation (sources):
  *   y[b,j] = sum_i phi_ji(x[b,i])                  InKAN landing page, "What is a KAN?"
- *   phi_ji(x) = sum_m coef[j,i,m] B_m(x)            cubic B-spline with local support
+ *   phi_ji(x) = sum_m coef[j,i,m] B_m(x)            B-spline with local support
  *                                                   (same page and section)
  *             (+ w_base[j,i] silu(x) when has_base) optional SiLU base branch
- *   B_m: uniform cubic B-splines on G intervals of [lo,hi], the grid extended
- *   by 3 knots on each side, m = 0..G+2 ("predefined, bounded grids": UKAN
- *   abstract, "Want to train KANS at scale? Now UKAN!").  Knots
- *   t_k = lo + (k-3)(hi-lo)/G, k = 0..G+6; supp B_m = [t_m, t_{m+4}).
- *   An input outside [t_0, t_{G+6}) (and any NaN or inf) has all B_m = 0.
- *   Each input touches only 4 basis functions ("local 4-basis lookup":
- *   InKAN landing page, "Why InKAN?"), which are evaluated in the stable
- *   piecewise form with non-negative output (same page, "Numerically
- *   Stable"); no Cox-de Boor recursion runs on the device.
+ *   B_m: uniform B-splines of degree k (kan_shape.degree, 1..5; cubic, k = 3,
+ *   is the InKAN page's layer) on G intervals of [lo,hi], the grid extended
+ *   by k knots on each side, m = 0..G+k-1 ("predefined, bounded grids": UKAN
+ *   abstract, "Want to train KANS at scale? Now UKAN!"; degree-k splines and
+ *   the normalised coordinate bounded to [0, k+1]: FlashKAN abstract, mlsift
+ *   "GPU kernel" listing).  Knots t_j = lo + (j-k)(hi-lo)/G, j = 0..G+2k;
+ *   supp B_m = [t_m, t_{m+k+1}).  An input outside [t_0, t_{G+2k}) (and any
+ *   NaN or inf) has all B_m = 0.  Each input touches only k+1 basis
+ *   functions (for k = 3 the "local 4-basis lookup": InKAN landing page,
+ *   "Why InKAN?"), evaluated on the bounded local coordinate with
+ *   non-negative arithmetic only (same page, "Numerically Stable"): the cubic
+ *   pieces in closed form, other degrees by k passes of the recursion over
+ *   those k+1 values alone.
  *
  * Gradients (backward):
  *   dcoef[j,i,m]  = sum_b B_m(x[b,i]) dY[b,j]
@@ -27,12 +31,12 @@
  *
  * Layouts: every tensor is dense row-major (C order) in device memory.
  *   x       [batch, in]          operand dtype
- *   coef    [out, in, G+3]       operand dtype
+ *   coef    [out, in, G+k]       operand dtype (k = degree)
  *   w_base  [out, in]            operand dtype (only when has_base)
  *   y       [batch, out]         operand dtype
  *   dY      [batch, out]         operand dtype
  *   dx      [batch, in]          operand dtype
- *   dcoef   [out, in, G+3]       float32, overwritten
+ *   dcoef   [out, in, G+k]       float32, overwritten
  *   dw_base [out, in]            float32, overwritten
  * The operand dtype is float32 or bfloat16; accumulation is always fp32.
  * Pointers must be 16-byte aligned.
@@ -70,13 +74,13 @@
 extern "C" {
 #endif
 
-#define KAN_ABI_VERSION 1
+#define KAN_ABI_VERSION 2
 
 typedef enum { KAN_F32 = 0, KAN_BF16 = 1 } kan_dtype;
 
 typedef enum {
     KAN_OK = 0,
-    KAN_ERR_INVALID_ARG = 1,   /* a null pointer, a non-positive size, G < 1, hi <= lo, ... */
+    KAN_ERR_INVALID_ARG = 1,   /* a null pointer, a non-positive size, G < 1, hi <= lo, degree not 1..5, ... */
     KAN_ERR_UNSUPPORTED = 2,   /* valid but not handled: misaligned pointer, G > 250, forced path not possible */
     KAN_ERR_WORKSPACE = 3,     /* workspace smaller than kan_workspace_size() */
     KAN_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed (detail in kan_last_error) */
@@ -98,6 +102,7 @@ typedef struct {
     int32_t dtype;     /* kan_dtype of x, coef, w_base, y, dY, dx */
     int32_t has_base;  /* 1: add the SiLU base branch w_base[j,i] silu(x[b,i]) */
     int32_t path;      /* KAN_PATH_* */
+    int32_t degree;    /* spline degree k, 1..5 (3: cubic) */
 } kan_shape;
 
 /* ABI version of the loaded library (KAN_ABI_VERSION it was built with). */
@@ -144,10 +149,11 @@ KAN_API kan_status kan_forward_fixed_scratch(const kan_shape* s, const void* x, 
                                              void* y, void* stream);
 
 /* The basis step alone, for inspection and tests: for each x[b,i] (batch*in
- * values) the span s (int32; the 4 non-zero functions are B_s..B_{s+3}, some
- * of which may fall outside 0..G+2 and are then absent; s = INT32_MIN when
- * the input is outside the extended knots), the 4 weights w[.,4] = B_{s+r}(x)
- * and the 4 derivatives dw[.,4] = B'_{s+r}(x).  Any output may be NULL. */
+ * values) the span s (int32; the k+1 non-zero functions are B_s..B_{s+k},
+ * some of which may fall outside 0..G+k-1 and are then absent; s = INT32_MIN
+ * when the input is outside the extended knots), the k+1 weights
+ * w[., k+1] = B_{s+r}(x) and the k+1 derivatives dw[., k+1] = B'_{s+r}(x)
+ * (k = s->degree).  Any output may be NULL. */
 KAN_API kan_status kan_basis(const kan_shape* s, const void* x, int32_t* span, float* w, float* dw, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word that

@@ -83,13 +83,15 @@ kan_status validate(const kan_shape* s, Problem* p)
     if (s->dtype != KAN_F32 && s->dtype != KAN_BF16) return fail(KAN_ERR_INVALID_ARG, "unknown dtype");
     if (s->has_base != 0 && s->has_base != 1) return fail(KAN_ERR_INVALID_ARG, "has_base must be 0 or 1");
     if (s->path < KAN_PATH_AUTO || s->path > KAN_PATH_SIMT) return fail(KAN_ERR_INVALID_ARG, "unknown path");
-    const int64_t nb = s->G + 3;
+    if (s->degree < 1 || s->degree > 5) return fail(KAN_ERR_INVALID_ARG, "degree must be 1..5");
+    const int64_t nb = s->G + s->degree;
     if (s->in > ((int64_t)1 << 40) / nb || s->out > ((int64_t)1 << 40) || s->batch > ((int64_t)1 << 40))
         return fail(KAN_ERR_UNSUPPORTED, "sizes too large");
     p->batch = s->batch;
     p->in = s->in;
     p->out = s->out;
     p->G = s->G;
+    p->k = s->degree;
     p->nb = (int)nb;
     p->Kt = s->in * nb;
     p->lo = s->lo;

@@ -15,35 +15,48 @@ namespace kan {
 // ---------------------------------------------------------------------------
 // Span and local weights (steps S1, S2)
 //
-// For the uniform grid t_k = lo + (k-3)h, h = (hi-lo)/G, an input x lies in
-// knot interval floor(u)+3 with u = (x-lo)/h.  With s = floor(u) and the
-// local coordinate t = u - s in [0,1), exactly B_s..B_{s+3} can be non-zero
-// (the "local 4-basis lookup" of the InKAN landing page, "Why InKAN?"), and
-// those with index outside 0..G+2 do not exist.  The input is inside the
-// extended knots iff -3 <= u < G+3; NaN and +-inf fail that test, so they
-// contribute nothing and never reach an index computation.
+// For the uniform grid t_j = lo + (j-k)h of degree k, h = (hi-lo)/G, an input
+// x lies in knot interval floor(u)+k with u = (x-lo)/h.  With s = floor(u)
+// and the local coordinate t = u - s in [0,1), exactly B_s..B_{s+k} can be
+// non-zero (the "local 4-basis lookup" of the InKAN landing page, "Why
+// InKAN?", for k = 3), and those with index outside 0..G+k-1 do not exist.
+// The input is inside the extended knots iff -k <= u < G+k; NaN and +-inf
+// fail that test, so they contribute nothing and never reach an index
+// computation (the FlashKAN abstract's clamp of the normalised coordinate to
+// [0, k+1] gives the same zeros).
 //
-// The weights are the four pieces of the uniform cubic B-spline written in a
+// Cubic weights: the four pieces of the uniform cubic B-spline written in a
 // form without cancellation on the bounded coordinate t in [0,1) (the
 // "stable piecewise polynomial evaluation" with non-negative output of the
-// InKAN page, "Numerically Stable"; the clamp to a bounded coordinate is the
-// FlashKAN abstract's stabilisation):
+// InKAN page, "Numerically Stable"):
 //   w0 = (1-t)^3/6            w3 = t^3/6
 //   w1 = 2/3 - t^2 (2-t)/2    w2 = 2/3 - (1-t)^2 (1+t)/2     (w2(t) = w1(1-t))
 // and their derivatives with respect to x (factor 1/h):
 //   w0' = -(1-t)^2/2   w1' = (3t^2-4t)/2   w2' = -(3(1-t)^2-4(1-t))/2   w3' = t^2/2
+//
+// Any degree k (1..5): the k+1 weights are built in k passes of the local
+// triangle on the unit-spaced knots (the FlashKAN abstract's "k sequential
+// passes for degree-k splines", done on k+1 registers instead of the whole
+// knot vector):
+//   b^0 = (1);  b^d_r = ((t + d - r) b^{d-1}_{r-1} + (r + 1 - t) b^{d-1}_r) / d,  r = 0..d
+// (b^{d-1}_{-1} = b^{d-1}_d = 0).  Every factor is non-negative for t in
+// [0,1), so no cancellation occurs.  The derivatives come from the degree
+// k-1 weights: w'_r = (b^{k-1}_{r-1} - b^{k-1}_r) / h.
 // ---------------------------------------------------------------------------
+constexpr int KAN_MAX_DEGREE = 5;
+constexpr int KAN_MAX_NW = KAN_MAX_DEGREE + 1;   // local weights of the highest degree
+
 struct Span {
-    int s;       // first of the 4 basis indices
+    int s;       // first of the k+1 basis indices
     float t;     // local coordinate in [0,1)
     bool valid;  // inside the extended knots
 };
 
-__device__ __forceinline__ Span span_of(float x, float lo, float inv_h, int G)
+__device__ __forceinline__ Span span_of(float x, float lo, float inv_h, int G, int k)
 {
     Span r;
     float u = (x - lo) * inv_h;
-    r.valid = (u >= -3.0f) && (u < (float)(G + 3));
+    r.valid = (u >= -(float)k) && (u < (float)(G + k));
     float f = floorf(r.valid ? u : 0.0f);
     r.s = (int)f;
     r.t = r.valid ? (u - f) : 0.0f;
@@ -67,6 +80,38 @@ __device__ __forceinline__ void dweights(float t, float inv_h, float d[4])
     d[1] = (1.5f * t - 2.0f) * t * inv_h;
     d[2] = -(1.5f * s - 2.0f) * s * inv_h;
     d[3] = 0.5f * t * t * inv_h;
+}
+
+// Degree-k weights b[0..k] (entries past k are 0) by the local triangle; with
+// DERIV, also the derivatives d[0..k] (times inv_h).  k is warp-uniform in
+// every caller, so the early exit does not diverge.
+template <bool DERIV>
+__device__ __forceinline__ void weights_k(float t, int k, float inv_h, float (&b)[KAN_MAX_NW], float (&d)[KAN_MAX_NW])
+{
+#pragma unroll
+    for (int r = 0; r < KAN_MAX_NW; ++r) b[r] = r == 0 ? 1.0f : 0.0f;
+#pragma unroll
+    for (int dg = 1; dg <= KAN_MAX_DEGREE; ++dg) {
+        if (dg > k) break;
+        if (DERIV && dg == k) {
+            // degree k-1 values are in b[0..k-1]: w'_r = (b_{r-1} - b_r) / h
+#pragma unroll
+            for (int r = 0; r < KAN_MAX_NW; ++r) {
+                const float left = r > 0 ? b[r - 1] : 0.0f;
+                const float right = r < dg ? b[r] : 0.0f;
+                d[r] = r <= dg ? (left - right) * inv_h : 0.0f;
+            }
+        }
+        const float inv_d = 1.0f / (float)dg;
+        // in place, from the top: b[r] still holds degree dg-1 when it is read
+#pragma unroll
+        for (int r = KAN_MAX_NW - 1; r >= 0; --r) {
+            if (r > dg) continue;
+            const float left = r > 0 ? (t + (float)(dg - r)) * b[r - 1] : 0.0f;
+            const float right = r < dg ? ((float)(r + 1) - t) * b[r] : 0.0f;
+            b[r] = (left + right) * inv_d;
+        }
+    }
 }
 
 // silu(x) = x sigma(x) and silu'(x) = sigma(x) (1 + x (1 - sigma(x))), with

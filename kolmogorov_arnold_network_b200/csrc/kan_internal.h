@@ -17,7 +17,8 @@ namespace kan {
 struct Problem {
     int64_t batch, in, out;
     int G;
-    int nb;          // G + 3 basis functions per edge
+    int k;           // spline degree (1..5)
+    int nb;          // G + k basis functions per edge
     int64_t Kt;      // in * nb (spline columns of the dense expansion)
     float lo, hi, inv_h;
     int dtype;       // KAN_F32 / KAN_BF16

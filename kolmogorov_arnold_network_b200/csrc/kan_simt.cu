@@ -9,27 +9,43 @@ namespace kan {
 namespace {
 
 constexpr int kFwdRows = 4;       // batch rows per forward block
-constexpr int kFwdChunk = 512;    // inputs staged per pass in the forward block
+constexpr int kFwdChunk = 256;    // inputs staged per pass in the forward block
+
+// Weights (and derivatives) of an input on its local coordinate: the cubic
+// closed form for k = 3, the local triangle otherwise (entries past k are 0).
+__device__ __forceinline__ void local_weights(float t, int k, float inv_h, float (&w)[KAN_MAX_NW],
+                                              float (&d)[KAN_MAX_NW], bool want_d)
+{
+    if (k == 3) {
+        float w4[4], d4[4];
+        weights(t, w4);
+        if (want_d) dweights(t, inv_h, d4);
+#pragma unroll
+        for (int r = 0; r < KAN_MAX_NW; ++r) {
+            w[r] = r < 4 ? w4[r] : 0.0f;
+            d[r] = (want_d && r < 4) ? d4[r] : 0.0f;
+        }
+    } else if (want_d) {
+        weights_k<true>(t, k, inv_h, w, d);
+    } else {
+        weights_k<false>(t, k, inv_h, w, d);
+    }
+}
 
 template <typename T>
-__global__ void basis_kernel(const T* __restrict__ x, int64_t n, float lo, float inv_h, int G, int32_t* span,
+__global__ void basis_kernel(const T* __restrict__ x, int64_t n, float lo, float inv_h, int G, int k, int32_t* span,
                              float* w, float* dw)
 {
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        Span sp = span_of(to_f(x[e]), lo, inv_h, G);
-        float wv[4] = {0.f, 0.f, 0.f, 0.f}, dv[4] = {0.f, 0.f, 0.f, 0.f};
-        if (sp.valid) {
-            weights(sp.t, wv);
-            dweights(sp.t, inv_h, dv);
-        }
+        Span sp = span_of(to_f(x[e]), lo, inv_h, G, k);
+        float wv[KAN_MAX_NW], dv[KAN_MAX_NW];
+        local_weights(sp.t, k, inv_h, wv, dv, true);
         if (span) span[e] = sp.valid ? sp.s : INT32_MIN;
-        if (w) {
 #pragma unroll
-            for (int r = 0; r < 4; ++r) w[e * 4 + r] = wv[r];
-        }
-        if (dw) {
-#pragma unroll
-            for (int r = 0; r < 4; ++r) dw[e * 4 + r] = dv[r];
+        for (int r = 0; r < KAN_MAX_NW; ++r) {
+            if (r > k) break;
+            if (w) w[e * (k + 1) + r] = sp.valid ? wv[r] : 0.0f;
+            if (dw) dw[e * (k + 1) + r] = sp.valid ? dv[r] : 0.0f;
         }
     }
 }
@@ -38,13 +54,13 @@ __global__ void basis_kernel(const T* __restrict__ x, int64_t n, float lo, float
 // and weights for a chunk of inputs are staged in shared memory.
 template <typename T>
 __global__ void forward_kernel(const T* __restrict__ x, const T* __restrict__ coef, const T* __restrict__ w_base,
-                               T* __restrict__ y, int64_t batch, int64_t in, int64_t out, int G, float lo,
+                               T* __restrict__ y, int64_t batch, int64_t in, int64_t out, int G, int k, float lo,
                                float inv_h)
 {
     __shared__ int s_span[kFwdRows][kFwdChunk];
-    __shared__ float s_w[kFwdRows][kFwdChunk][4];
+    __shared__ float s_w[kFwdRows][kFwdChunk][KAN_MAX_NW];
     __shared__ float s_silu[kFwdRows][kFwdChunk];
-    const int nb = G + 3;
+    const int nb = G + k;
     const int64_t b0 = (int64_t)blockIdx.x * kFwdRows;
     const int nrows = (int)(batch - b0 < kFwdRows ? batch - b0 : kFwdRows);
 
@@ -60,12 +76,13 @@ __global__ void forward_kernel(const T* __restrict__ x, const T* __restrict__ co
             for (int e = threadIdx.x; e < kFwdRows * ni; e += blockDim.x) {
                 int r = e / ni, ii = e % ni;
                 float xv = r < nrows ? to_f(x[(b0 + r) * in + i0 + ii]) : 0.f;
-                Span sp = span_of(xv, lo, inv_h, G);
-                float wv[4] = {0.f, 0.f, 0.f, 0.f};
-                if (sp.valid && r < nrows) weights(sp.t, wv);
-                s_span[r][ii] = (sp.valid && r < nrows) ? sp.s : -1000;
+                Span sp = span_of(xv, lo, inv_h, G, k);
+                float wv[KAN_MAX_NW], dv[KAN_MAX_NW];
+                local_weights(sp.t, k, inv_h, wv, dv, false);
+                const bool use = sp.valid && r < nrows;
+                s_span[r][ii] = use ? sp.s : -1000;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) s_w[r][ii][q] = wv[q];
+                for (int q = 0; q < KAN_MAX_NW; ++q) s_w[r][ii][q] = use ? wv[q] : 0.f;
                 s_silu[r][ii] = (w_base && r < nrows) ? silu_f(xv) : 0.f;
             }
             __syncthreads();
@@ -77,9 +94,9 @@ __global__ void forward_kernel(const T* __restrict__ x, const T* __restrict__ co
                     for (int r = 0; r < kFwdRows; ++r) {
                         int s = s_span[r][ii];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
+                        for (int q = 0; q < KAN_MAX_NW; ++q) {
                             int m = s + q;
-                            if (m >= 0 && m < nb) acc[r] += to_f(cji[m]) * s_w[r][ii][q];
+                            if (q <= k && m >= 0 && m < nb) acc[r] += to_f(cji[m]) * s_w[r][ii][q];
                         }
                     }
                     if (w_base) {
@@ -100,10 +117,10 @@ __global__ void forward_kernel(const T* __restrict__ x, const T* __restrict__ co
 // the weight of its own basis function when the input's span covers it.
 template <typename T>
 __global__ void dcoef_kernel(const T* __restrict__ x, const T* __restrict__ dY, float* __restrict__ dcoef,
-                             float* __restrict__ dw_base, int64_t batch, int64_t in, int64_t out, int G, float lo,
-                             float inv_h)
+                             float* __restrict__ dw_base, int64_t batch, int64_t in, int64_t out, int G, int k,
+                             float lo, float inv_h)
 {
-    const int nb = G + 3;
+    const int nb = G + k;
     const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (e >= in * out * (nb + 1)) return;
     const int m = (int)(e % (nb + 1));
@@ -118,12 +135,15 @@ __global__ void dcoef_kernel(const T* __restrict__ x, const T* __restrict__ dY, 
             acc += silu_f(xv) * g;
             continue;
         }
-        const Span sp = span_of(xv, lo, inv_h, G);
+        const Span sp = span_of(xv, lo, inv_h, G, k);
         const int q = m - sp.s;
-        if (sp.valid && q >= 0 && q < 4) {
-            float wv[4];
-            weights(sp.t, wv);
-            acc += (q == 0 ? wv[0] : q == 1 ? wv[1] : q == 2 ? wv[2] : wv[3]) * g;   // (no indexed registers)
+        if (sp.valid && q >= 0 && q <= k) {
+            float wv[KAN_MAX_NW], dv[KAN_MAX_NW];
+            local_weights(sp.t, k, inv_h, wv, dv, false);
+            float wq = 0.0f;   // (selected without indexing registers)
+#pragma unroll
+            for (int r = 0; r < KAN_MAX_NW; ++r) wq = r == q ? wv[r] : wq;
+            acc += wq * g;
         }
     }
     if (m == nb) dw_base[ji] = acc;
@@ -134,16 +154,16 @@ __global__ void dcoef_kernel(const T* __restrict__ x, const T* __restrict__ dY, 
 template <typename T>
 __global__ void dx_kernel(const T* __restrict__ x, const T* __restrict__ coef, const T* __restrict__ w_base,
                           const T* __restrict__ dY, T* __restrict__ dx, int64_t batch, int64_t in, int64_t out,
-                          int G, float lo, float inv_h)
+                          int G, int k, float lo, float inv_h)
 {
-    const int nb = G + 3;
+    const int nb = G + k;
     const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (e >= batch * in) return;
     const int64_t b = e / in, i = e % in;
     float xv = to_f(x[e]);
-    Span sp = span_of(xv, lo, inv_h, G);
-    float dv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (sp.valid) dweights(sp.t, inv_h, dv);
+    Span sp = span_of(xv, lo, inv_h, G, k);
+    float wv[KAN_MAX_NW], dv[KAN_MAX_NW];
+    local_weights(sp.t, k, inv_h, wv, dv, true);
     const float ds = w_base ? dsilu_f(xv) : 0.f;
     float acc = 0.f;
     for (int64_t j = 0; j < out; ++j) {
@@ -151,9 +171,9 @@ __global__ void dx_kernel(const T* __restrict__ x, const T* __restrict__ coef, c
         float d = 0.f;
         if (sp.valid) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < KAN_MAX_NW; ++q) {
                 int m = sp.s + q;
-                if (m >= 0 && m < nb) d += to_f(cji[m]) * dv[q];
+                if (q <= k && m >= 0 && m < nb) d += to_f(cji[m]) * dv[q];
             }
         }
         if (w_base) d += to_f(w_base[j * in + i]) * ds;
@@ -194,11 +214,11 @@ cudaError_t simt_basis(const Problem& p, const void* x, int32_t* span, float* w,
     const int64_t n = p.batch * p.in;
     if (n == 0) return cudaSuccess;
     if (p.dtype == KAN_F32) {
-        basis_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>((const float*)x, n, p.lo, p.inv_h, p.G, span, w, dw);
+        basis_kernel<float><<<blocks_for(n, 256), 256, 0, st>>>((const float*)x, n, p.lo, p.inv_h, p.G, p.k, span, w, dw);
         count_launch();
     } else {
         basis_kernel<__nv_bfloat16><<<blocks_for(n, 256), 256, 0, st>>>((const __nv_bfloat16*)x, n, p.lo, p.inv_h,
-                                                                         p.G, span, w, dw);
+                                                                         p.G, p.k, span, w, dw);
         count_launch();
     }
     return cudaGetLastError();
@@ -214,12 +234,12 @@ cudaError_t simt_forward(const Problem& p, const void* x, const void* coef, cons
     const int threads = p.out >= 128 ? 128 : (int)((p.out + 31) / 32 * 32);
     if (p.dtype == KAN_F32) {
         forward_kernel<float><<<blocks, threads, 0, st>>>((const float*)x, (const float*)coef, (const float*)w_base,
-                                                          (float*)y, p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+                                                          (float*)y, p.batch, p.in, p.out, p.G, p.k, p.lo, p.inv_h);
         count_launch();
     } else {
         forward_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
             (const __nv_bfloat16*)x, (const __nv_bfloat16*)coef, (const __nv_bfloat16*)w_base, (__nv_bfloat16*)y,
-            p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+            p.batch, p.in, p.out, p.G, p.k, p.lo, p.inv_h);
         count_launch();
     }
     return cudaGetLastError();
@@ -239,12 +259,12 @@ cudaError_t simt_backward(const Problem& p, const void* x, const void* coef, con
         const int64_t n = p.in * p.out * (p.nb + 1);
         if (p.dtype == KAN_F32) {
             dcoef_kernel<float><<<blocks_for(n, 128), 128, 0, st>>>((const float*)x, (const float*)dY, dcoef, dw_base,
-                                                                     p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+                                                                     p.batch, p.in, p.out, p.G, p.k, p.lo, p.inv_h);
             count_launch();
         } else {
             dcoef_kernel<__nv_bfloat16><<<blocks_for(n, 128), 128, 0, st>>>(
-                (const __nv_bfloat16*)x, (const __nv_bfloat16*)dY, dcoef, dw_base, p.batch, p.in, p.out, p.G, p.lo,
-                p.inv_h);
+                (const __nv_bfloat16*)x, (const __nv_bfloat16*)dY, dcoef, dw_base, p.batch, p.in, p.out, p.G, p.k,
+                p.lo, p.inv_h);
             count_launch();
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -255,12 +275,12 @@ cudaError_t simt_backward(const Problem& p, const void* x, const void* coef, con
         if (p.dtype == KAN_F32) {
             dx_kernel<float><<<blocks_for(n, 128), 128, 0, st>>>((const float*)x, (const float*)coef,
                                                                   (const float*)w_base, (const float*)dY, (float*)dx,
-                                                                  p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+                                                                  p.batch, p.in, p.out, p.G, p.k, p.lo, p.inv_h);
             count_launch();
         } else {
             dx_kernel<__nv_bfloat16><<<blocks_for(n, 128), 128, 0, st>>>(
                 (const __nv_bfloat16*)x, (const __nv_bfloat16*)coef, (const __nv_bfloat16*)w_base,
-                (const __nv_bfloat16*)dY, (__nv_bfloat16*)dx, p.batch, p.in, p.out, p.G, p.lo, p.inv_h);
+                (const __nv_bfloat16*)dY, (__nv_bfloat16*)dx, p.batch, p.in, p.out, p.G, p.k, p.lo, p.inv_h);
             count_launch();
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -1,18 +1,18 @@
 // kan_tc.cu -- tensor-core (tcgen05 / TMEM / TMA) kernels of the KAN layer.
 //
 // The layer is a contraction over the dense basis expansion
-//   A[b, i*(G+3)+m] = B_m(x[b,i])            (at most 4 non-zeros per (b,i))
-// with coef viewed as a [out, in*(G+3)] matrix:
+//   A[b, i*(G+k)+m] = B_m(x[b,i])            (at most k+1 non-zeros per (b,i))
+// with coef viewed as a [out, in*(G+k)] matrix (k: spline degree, 3 = cubic):
 //   forward  y     = A . coef^T        (+ silu(x) . w_base^T)
 //   dcoef          = dY^T . A          (dw_base = dY^T . silu(x))
-//   dx             = sum over each input's 4 columns of (dY . coef) times B'
+//   dx             = sum over each input's k+1 columns of (dY . coef) times B'
 //                    (+ silu'(x) * (dY . w_base))
 // A never exists in global memory: producer warps evaluate each input's span
-// and four weights (the InKAN page's "local 4-basis lookup" in its stable
-// piecewise form) and write the dense, mostly-zero A tile (or its transpose)
-// straight into shared memory in the 128-byte-swizzled layout the tensor core
-// reads.  The dense expansion costs little on tensor cores, and the per-input
-// work stays O(4) whatever G is.
+// and k+1 weights (the InKAN page's "local 4-basis lookup" in its stable
+// piecewise form, for cubic splines) and write the dense, mostly-zero A tile
+// (or its transpose) straight into shared memory in the 128-byte-swizzled
+// layout the tensor core reads.  The dense expansion costs little on tensor
+// cores, and the per-input work stays O(k+1) whatever G is.
 //
 // One kernel template serves the four GEMMs:
 //   FWD    A = basis rows (producers)  B = coef / w_base, K-major (TMA)
@@ -24,7 +24,7 @@
 // epilogue warps (which also promote the fp32 accumulators).
 //
 // fp32 with the SiLU branch: silu(x_i) is one more basis function of input i,
-// with coefficient w_base[j, i].  Its column sits right after input i's G+3
+// with coefficient w_base[j, i].  Its column sits right after input i's G+k
 // spline columns (column stride G+4) in the fp16 copies of the coefficients
 // that the fp32 path makes anyway, so the SiLU terms ride along in every GEMM:
 // the forward sums them, dcoef's epilogue writes dw_base, and the dx epilogue
@@ -149,8 +149,9 @@ struct TcArgs {
     float* out2;               // DCA: dw_base (non-partial); DX: Gb = dY.w_base (fp32 [batch,in]) or null
     unsigned int* status;
     int64_t batch, in, out_f;
-    int G, nb;                 // nb: columns per input (G+3, or G+4 with an interleaved SiLU column)
-    int nbs;                   // spline functions per input (G+3)
+    int G, nb;                 // nb: columns per input (G+k, or G+k+1 with an interleaved SiLU column)
+    int nbs;                   // spline functions per input (G+k)
+    int k;                     // spline degree
     int ext;                   // 1: input i's SiLU column is column nbs of its group
     float lo, inv_h;
     int Kt;                    // in * nb
@@ -244,28 +245,33 @@ __device__ __forceinline__ uint32_t sw_col(int c, uint32_t rx)
     return ((((cb >> 4) ^ rx) & 7u) << 4) | (cb & 15u);
 }
 
-// The four weights of one input whose B_0 sits at column `base` of a 128-byte
-// swizzled row: entry q (basis index s+q) goes to column base+s+q when
-// mlo <= s+q < mhi (the caller's range keeps the column inside the row and the
-// basis index inside 0..nb-1; an empty range stores nothing).  One predicated
-// store per entry keeps the warp convergent.
-template <int DT>
+// The local weights of one input whose B_0 sits at column `base` of a
+// 128-byte swizzled row: entry q (basis index s+q, q <= kq) goes to column
+// base+s+q when mlo <= s+q < mhi (the caller's range keeps the column inside
+// the row and the basis index inside 0..nb-1; an empty range stores nothing).
+// One predicated store per entry keeps the warp convergent.  NW = 4 with
+// kq = 3 for cubic splines; NW = KAN_MAX_NW with the runtime degree otherwise.
+template <int DT, int NW>
 __device__ __forceinline__ void scatter_win(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx, int base, int s, int mlo,
-                                            int mhi, const float (&w)[4])
+                                            int mhi, const float (&w)[NW], int kq)
 {
     constexpr int ESZ = 2;   // operand element size, both dtypes
     const uint32_t width = (uint32_t)(mhi - mlo);
     if constexpr (DT == KAN_BF16) {
-        const uint32_t p01 = pack_bf16(w[0], w[1]), p23 = pack_bf16(w[2], w[3]);
-        const uint16_t h[4] = {(uint16_t)(p01 & 0xFFFFu), (uint16_t)(p01 >> 16), (uint16_t)(p23 & 0xFFFFu),
-                               (uint16_t)(p23 >> 16)};
+        uint16_t h[NW];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            if ((uint32_t)(s + q - mlo) < width) st_shared_u16(rb_hi + sw_col<ESZ>(base + s + q, rx), h[q]);
+        for (int q = 0; q < NW; q += 2) {
+            const uint32_t p = pack_bf16(w[q], q + 1 < NW ? w[q + 1] : 0.0f);
+            h[q] = (uint16_t)(p & 0xFFFFu);
+            if (q + 1 < NW) h[q + 1] = (uint16_t)(p >> 16);
+        }
+#pragma unroll
+        for (int q = 0; q < NW; ++q)
+            if (q <= kq && (uint32_t)(s + q - mlo) < width) st_shared_u16(rb_hi + sw_col<ESZ>(base + s + q, rx), h[q]);
     } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            if ((uint32_t)(s + q - mlo) < width) {
+        for (int q = 0; q < NW; ++q)
+            if (q <= kq && (uint32_t)(s + q - mlo) < width) {
                 const uint32_t off = sw_col<ESZ>(base + s + q, rx);
                 uint16_t h, l;
                 split_f16(w[q], h, l);
@@ -398,7 +404,9 @@ __device__ __forceinline__ void weights_fma(float t, float (&w)[4])
 // holds half of the B tile, so each SM streams half the B bytes.  The leader
 // (rank 0) issues the MMAs; the follower's B loads complete on the leader's
 // barriers and its producers arrive there remotely; commits reach both CTAs.
-template <int MODE, int DT, int MAXI, bool PAIR = false>
+// KD: 3 for cubic splines (closed-form weights, 4 per input), 0 for any
+// other degree (the runtime degree a.k; weights by the local triangle).
+template <int MODE, int DT, int MAXI, bool PAIR = false, int KD = 3>
 __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
               const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
@@ -706,7 +714,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const bool row_ok = b < a.batch;
                 const T* xrow = X + (row_ok ? b : 0) * a.in;
                 const float u0 = -a.lo * a.inv_h;      // u = x * inv_h + u0
-                const float u_hi = (float)(a.G + 3);
+                const float u_lo = -(float)a.k, u_hi = (float)(a.G + a.k);
                 auto first_input = [&](int kb) { return (int)__umulhi((uint32_t)(kb * BK), a.nb_magic); };
                 auto last_input = [&](int kb) {
                     const int c_end = min(kb * BK + BK, a.Kt);
@@ -759,17 +767,24 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                 }
                                 float u = fmaf(cur[k], a.inv_h, u0);
                                 // outside the extended knots, NaN, inf: no stores
-                                const bool ok = act && u >= -3.0f && u < u_hi;
+                                const bool ok = act && u >= u_lo && u < u_hi;
                                 u = ok ? u : 0.0f;
                                 int sidx;
                                 float f;
                                 floor_split(u, sidx, f);
-                                float w[4];
-                                weights_fma(u - f, w);
                                 // basis indices whose columns lie in this block
                                 const int mlo = ok ? max(0, -base) : 0;
                                 const int mhi = ok ? min(a.nbs, BK - base) : 0;
-                                scatter_win<DT>(ahi + rbase, alo + rbase, rx, base, sidx, mlo, mhi, w);
+                                if constexpr (KD == 3) {
+                                    float w[4];
+                                    weights_fma(u - f, w);
+                                    scatter_win<DT, 4>(ahi + rbase, alo + rbase, rx, base, sidx, mlo, mhi, w, 3);
+                                } else {
+                                    float w[KAN_MAX_NW], dd[KAN_MAX_NW];
+                                    weights_k<false>(u - f, a.k, 0.0f, w, dd);
+                                    scatter_win<DT, KAN_MAX_NW>(ahi + rbase, alo + rbase, rx, base, sidx, mlo, mhi, w,
+                                                                a.k);
+                                }
                             }
                         }
                     } else {
@@ -822,7 +837,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const int n_inp = (!silu_tile && c_lo < c_end)
                                       ? (int)__umulhi((uint32_t)(c_end - 1), a.nb_magic) - i_first + 1 : 0;
                 const float u0 = -a.lo * a.inv_h;
-                const float u_hi = (float)(a.G + 3);
+                const float u_lo = -(float)a.k, u_hi = (float)(a.G + a.k);
                 XWindow<T, MAXI> nxw;   // (see the forward producer)
                 nxw.o = -1;
 #pragma unroll
@@ -875,21 +890,28 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                     }
                                 }
                                 float u = fmaf(cur[k], a.inv_h, u0);
-                                const bool ok = act && u >= -3.0f && u < u_hi;   // NaN, inf fail
+                                const bool ok = act && u >= u_lo && u < u_hi;   // NaN, inf fail
                                 u = ok ? u : 0.0f;
                                 int sidx;
                                 float f;
                                 floor_split(u, sidx, f);
-                                float w[4];
-                                weights_fma(u - f, w);
+                                constexpr int NW = KD == 3 ? 4 : KAN_MAX_NW;
+                                float w[NW];
+                                if constexpr (KD == 3) {
+                                    weights_fma(u - f, w);
+                                } else {
+                                    float dd[KAN_MAX_NW];
+                                    weights_k<false>(u - f, a.k, 0.0f, w, dd);
+                                }
+                                const int kq = KD == 3 ? 3 : a.k;
                                 const int base = cbase + k * a.nb;
                                 // basis indices whose columns lie in this atom (empty when !ok)
                                 const int mlo = ok ? max(0, -base) : 0;
                                 const uint32_t width = ok ? (uint32_t)(min(a.nbs, EPB - base) - mlo) : 0u;
                                 const int col0 = base + sidx;
 #pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    if ((uint32_t)(sidx + q - mlo) < width) {
+                                for (int q = 0; q < NW; ++q) {
+                                    if (q <= kq && (uint32_t)(sidx + q - mlo) < width) {
                                         const uint32_t off = col_off(col0 + q);
                                         if constexpr (F32) {
                                             uint16_t h, l;
@@ -1160,16 +1182,22 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                             const int i = ic + k;
                             if (i >= dx_i1) break;
                             const float xv = __uint_as_float(xc[k]);
-                            const Span sp = span_of(xv, a.lo, a.inv_h, a.G);
+                            const Span sp = span_of(xv, a.lo, a.inv_h, a.G, a.k);
                             float acc = 0.0f;
                             if (sp.valid) {
-                                float d[4];
-                                dweights(sp.t, a.inv_h, d);
+                                constexpr int NW = KD == 3 ? 4 : KAN_MAX_NW;
+                                float d[NW];
+                                if constexpr (KD == 3) {
+                                    dweights(sp.t, a.inv_h, d);
+                                } else {
+                                    float ww[KAN_MAX_NW];
+                                    weights_k<true>(sp.t, a.k, a.inv_h, ww, d);
+                                }
                                 const int cb = i * a.nb - kt_al;
 #pragma unroll
-                                for (int qq = 0; qq < 4; ++qq) {
+                                for (int qq = 0; qq < NW; ++qq) {
                                     const int m = sp.s + qq;
-                                    if (m >= 0 && m < a.nbs) acc += stage[cb + m] * d[qq];
+                                    if (qq <= a.k && m >= 0 && m < a.nbs) acc += stage[cb + m] * d[qq];
                                 }
                             }
                             acc *= inv_dc;
@@ -1215,8 +1243,9 @@ struct DxArgs {
     const float* gb;          // dY . w_base (fp32 [batch, in]) or null (none, or ext)
     unsigned int* status;
     int64_t batch, in, out;
-    int G, nb;                // nb: columns per input of B (G+3, or G+4 with the SiLU column)
-    int nbs;                  // spline functions per input (G+3)
+    int G, nb;                // nb: columns per input of B (G+k, or G+k+1 with the SiLU column)
+    int nbs;                  // spline functions per input (G+k)
+    int k;                    // spline degree
     int ext;                  // 1: column nbs of each input group is its dY.w_base column
     float lo, inv_h;
     int BN, stages, nkb;      // nkb: k-blocks over out
@@ -1228,7 +1257,7 @@ struct DxArgs {
     int pair;                 // (informational) tiles of 2 x 128 batch rows run by CTA pairs
 };
 
-template <int DT, bool PAIR>
+template <int DT, bool PAIR, int KD = 3>
 __global__ void __launch_bounds__(kDxThreads, 1)
     dx_persistent_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
                          const __grid_constant__ CUtensorMap tB_hi, const __grid_constant__ CUtensorMap tB_lo,
@@ -1623,16 +1652,22 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     auto dx_of = [&](int k) -> float {
                         const int i = ic + k;
                         const float xv = xc[k];
-                        const Span sp = span_of(xv, a.lo, a.inv_h, a.G);
+                        const Span sp = span_of(xv, a.lo, a.inv_h, a.G, a.k);
                         float acc = 0.0f;
                         if (sp.valid) {
-                            float d[4];
-                            dweights(sp.t, a.inv_h, d);
+                            constexpr int NW = KD == 3 ? 4 : KAN_MAX_NW;
+                            float d[NW];
+                            if constexpr (KD == 3) {
+                                dweights(sp.t, a.inv_h, d);
+                            } else {
+                                float ww[KAN_MAX_NW];
+                                weights_k<true>(sp.t, a.k, a.inv_h, ww, d);
+                            }
                             const int cb = i * a.nb - kt_al;
 #pragma unroll
-                            for (int qq = 0; qq < 4; ++qq) {
+                            for (int qq = 0; qq < NW; ++qq) {
                                 const int m = sp.s + qq;
-                                if (m >= 0 && m < a.nbs) acc += to_f(srow[cb + m]) * d[qq];
+                                if (qq <= a.k && m >= 0 && m < a.nbs) acc += to_f(srow[cb + m]) * d[qq];
                             }
                         }
                         acc *= inv_dc;
@@ -1994,7 +2029,7 @@ struct Plan {
     // row length of the fp16 copies of dY (fp32: out rounded up to 8, so that TMA can address them)
     int64_t ldo;
     // fp32 with the SiLU branch: interleaved coefficient copies (nbx = G+4
-    // columns per input, Kx = in * nbx); otherwise nbx = G+3 and Kx = Kt
+    // columns per input, Kx = in * nbx); otherwise nbx = G+k and Kx = Kt
     bool ext;
     int nbx;
     int64_t Kx;
@@ -2143,7 +2178,7 @@ Plan make_plan(const Problem& p, int sms)
 
 inline int grid_for(int64_t n) { return (int)std::min<int64_t>(std::max<int64_t>(1, (n + 255) / 256), 148 * 8); }
 
-template <int MODE, int DT, int MAXI, bool PAIR>
+template <int MODE, int DT, int MAXI, bool PAIR, int KD>
 cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args, cudaStream_t st)
 {
     constexpr bool produce = MODE == FWD || MODE == DCA;
@@ -2162,7 +2197,7 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
     if (smem > kSmemBudget) return cudaErrorInvalidConfiguration;
     static int configured = 0;   // per instantiation; the attribute is per function
     if (configured < smem) {
-        cudaError_t e = cudaFuncSetAttribute(tc_kernel<MODE, DT, MAXI, PAIR>,
+        cudaError_t e = cudaFuncSetAttribute(tc_kernel<MODE, DT, MAXI, PAIR, KD>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
         if (e != cudaSuccess) return e;
         configured = kSmemBudget;
@@ -2180,13 +2215,13 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, tc_kernel<MODE, DT, MAXI, true>, maps[0], maps[1], maps[2], maps[3],
-                                           maps[4], maps[5], args);
+        cudaError_t e = cudaLaunchKernelEx(&cfg, tc_kernel<MODE, DT, MAXI, true, KD>, maps[0], maps[1], maps[2],
+                                           maps[3], maps[4], maps[5], args);
         count_launch();
         if (e != cudaSuccess) return e;
     } else {
-        tc_kernel<MODE, DT, MAXI, false><<<grid, Warps<MODE>::kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3],
-                                                                                    maps[4], maps[5], args);
+        tc_kernel<MODE, DT, MAXI, false, KD><<<grid, Warps<MODE>::kThreads, smem, st>>>(maps[0], maps[1], maps[2],
+                                                                                        maps[3], maps[4], maps[5], args);
         count_launch();
     }
     return cudaGetLastError();
@@ -2195,40 +2230,51 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
 // Inputs a row of one forward k-block can touch: (BK - 1) / nb + 2.
 int fwd_maxi_needed(int nb, bool f32) { return (64 - 1) / nb + 2; (void)f32; }
 
-template <int MODE, int MAXI>
+template <int MODE, int MAXI, int KD>
 cudaError_t launch_m(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
                      cudaStream_t st)
 {
-    if (f32) return launch<MODE, KAN_F32, MAXI, false>(grid, BN, stages, maps, args, st);
+    if (f32) return launch<MODE, KAN_F32, MAXI, false, KD>(grid, BN, stages, maps, args, st);
     if constexpr (MODE == FWD || MODE == DCA) {
-        if (args.pair) return launch<MODE, KAN_BF16, MAXI, true>(grid, BN, stages, maps, args, st);
+        if (args.pair) return launch<MODE, KAN_BF16, MAXI, true, KD>(grid, BN, stages, maps, args, st);
     }
-    return launch<MODE, KAN_BF16, MAXI, false>(grid, BN, stages, maps, args, st);
+    return launch<MODE, KAN_BF16, MAXI, false, KD>(grid, BN, stages, maps, args, st);
 }
 
+template <int MODE, int KD>
+cudaError_t launch_k(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
+                     cudaStream_t st)
+{
+    if constexpr (MODE == FWD || MODE == DCA) {
+        const int need = fwd_maxi_needed(args.nb, f32);
+        if (need <= 4) return launch_m<MODE, 4, KD>(f32, grid, BN, stages, maps, args, st);
+        if (need <= 7) return launch_m<MODE, 7, KD>(f32, grid, BN, stages, maps, args, st);
+        if (need <= 9) return launch_m<MODE, 9, KD>(f32, grid, BN, stages, maps, args, st);
+        if (need <= 17) return launch_m<MODE, 17, KD>(f32, grid, BN, stages, maps, args, st);
+        return cudaErrorInvalidConfiguration;   // nb >= 4 keeps need <= 17
+    } else {
+        return launch_m<MODE, 1, KD>(f32, grid, BN, stages, maps, args, st);
+    }
+}
+
+// cubic splines run the closed-form instantiation; other degrees the general
+// one (the GEMM of dY . w_base involves no basis)
 template <int MODE>
 cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
                       cudaStream_t st)
 {
-    if constexpr (MODE == FWD || MODE == DCA) {
-        const int need = fwd_maxi_needed(args.nb, f32);
-        if (need <= 4) return launch_m<MODE, 4>(f32, grid, BN, stages, maps, args, st);
-        if (need <= 7) return launch_m<MODE, 7>(f32, grid, BN, stages, maps, args, st);
-        if (need <= 9) return launch_m<MODE, 9>(f32, grid, BN, stages, maps, args, st);
-        if (need <= 17) return launch_m<MODE, 17>(f32, grid, BN, stages, maps, args, st);
-        return cudaErrorInvalidConfiguration;   // G >= 1 keeps need <= 17
-    } else {
-        return launch_m<MODE, 1>(f32, grid, BN, stages, maps, args, st);
-    }
+    if (MODE == GEMM || args.k == 3) return launch_k<MODE, 3>(f32, grid, BN, stages, maps, args, st);
+    if constexpr (MODE != GEMM) return launch_k<MODE, 0>(f32, grid, BN, stages, maps, args, st);
+    return cudaErrorInvalidConfiguration;
 }
 
-template <int DT, bool PAIR>
+template <int DT, bool PAIR, int KD>
 cudaError_t launch_dx_persistent(const Plan& P, const CUtensorMap* maps, const DxArgs& d, cudaStream_t st)
 {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(dx_persistent_kernel<DT, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             232448);
+        cudaError_t e = cudaFuncSetAttribute(dx_persistent_kernel<DT, PAIR, KD>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -2248,11 +2294,13 @@ cudaError_t launch_dx_persistent(const Plan& P, const CUtensorMap* maps, const D
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, dx_persistent_kernel<DT, true>, maps[0], maps[1], maps[2], maps[3], d);
+        cudaError_t e =
+            cudaLaunchKernelEx(&cfg, dx_persistent_kernel<DT, true, KD>, maps[0], maps[1], maps[2], maps[3], d);
         count_launch();
         if (e != cudaSuccess) return e;
     } else {
-        dx_persistent_kernel<DT, false><<<P.p_grid, kDxThreads, P.p_smem, st>>>(maps[0], maps[1], maps[2], maps[3], d);
+        dx_persistent_kernel<DT, false, KD><<<P.p_grid, kDxThreads, P.p_smem, st>>>(maps[0], maps[1], maps[2],
+                                                                                     maps[3], d);
         count_launch();
     }
     return cudaGetLastError();
@@ -2266,6 +2314,7 @@ TcArgs base_args(const Problem& p, const Plan& P)
     a.in = p.in;
     a.out_f = p.out;
     a.G = p.G;
+    a.k = p.k;
     a.nb = P.nbx;
     a.nbs = p.nb;
     a.ext = P.ext;
@@ -2344,9 +2393,9 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
     const bool f32 = p.dtype == KAN_F32;
     const int64_t nbx = p.nb + ((f32 && p.base) ? 1 : 0);
     if ((p.in * nbx * 2) % 16 != 0) {
-        *why = f32 ? "in*(G+3) (in*(G+4) with the SiLU branch) is not a multiple of 8 (TMA row stride of the "
+        *why = f32 ? "in*(G+k) (in*(G+k+1) with the SiLU branch) is not a multiple of 8 (TMA row stride of the "
                      "coefficient operand)"
-                   : "in*(G+3)*2 is not a multiple of 16 bytes (TMA row stride of coef)";
+                   : "in*(G+k)*2 is not a multiple of 16 bytes (TMA row stride of coef)";
         return false;
     }
     if (!f32 && p.base && (p.in * 2) % 16 != 0) {
@@ -2356,6 +2405,10 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
     if (!f32 && (p.out * 2) % 16 != 0) {
         // (fp32 reads dY through its fp16 copies, whose rows are padded to 8 elements)
         *why = "bf16 with out not a multiple of 8 (TMA row stride of dY)";
+        return false;
+    }
+    if (p.nb < 4) {
+        *why = "fewer than 4 basis functions per input (G + degree < 4): too many inputs per k-block row";
         return false;
     }
     if (nbx > 121 && (f32 || nbx > 249)) {
@@ -2555,6 +2608,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             d.in = p.in;
             d.out = p.out;
             d.G = p.G;
+            d.k = p.k;
             d.nb = P.nbx;
             d.nbs = p.nb;
             d.ext = P.ext ? 1 : 0;
@@ -2569,9 +2623,14 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             d.ld_stage = P.p_ld;
             d.a_res = P.p_ares ? 1 : 0;
             d.pair = P.p_pair ? 1 : 0;
-            e = f32 ? launch_dx_persistent<KAN_F32, false>(P, maps, d, st)
-                    : (P.p_pair ? launch_dx_persistent<KAN_BF16, true>(P, maps, d, st)
-                                : launch_dx_persistent<KAN_BF16, false>(P, maps, d, st));
+            if (p.k == 3)
+                e = f32 ? launch_dx_persistent<KAN_F32, false, 3>(P, maps, d, st)
+                        : (P.p_pair ? launch_dx_persistent<KAN_BF16, true, 3>(P, maps, d, st)
+                                    : launch_dx_persistent<KAN_BF16, false, 3>(P, maps, d, st));
+            else
+                e = f32 ? launch_dx_persistent<KAN_F32, false, 0>(P, maps, d, st)
+                        : (P.p_pair ? launch_dx_persistent<KAN_BF16, true, 0>(P, maps, d, st)
+                                    : launch_dx_persistent<KAN_BF16, false, 0>(P, maps, d, st));
             if (e != cudaSuccess) return e;
         } else {
             TcArgs a = base_args(p, P);

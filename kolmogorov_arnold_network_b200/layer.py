@@ -37,9 +37,9 @@ def _check(t, name, dtype=None, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def shape_of(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO) -> N.kan_shape:
+def shape_of(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, degree=3) -> N.kan_shape:
     batch, n_in = x.shape
-    return N.make_shape(batch, n_in, coef.shape[0], G, lo, hi, _code(x), w_base is not None, path)
+    return N.make_shape(batch, n_in, coef.shape[0], G, lo, hi, _code(x), w_base is not None, path, degree)
 
 
 def _stream(t):
@@ -56,14 +56,14 @@ def workspace(shape: N.kan_shape, for_backward: bool, device) -> torch.Tensor | 
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
-def forward(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, y=None, ws=None):
-    """y[b,j] = sum_i sum_m coef[j,i,m] B_m(x[b,i]) (+ sum_i w_base[j,i] silu(x[b,i]))."""
+def forward(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, y=None, ws=None, degree=3):
+    """y[b,j] = sum_i sum_m coef[j,i,m] B_m(x[b,i]) (+ sum_i w_base[j,i] silu(x[b,i])), degree-k B-splines."""
     batch, n_in = x.shape
     n_out = coef.shape[0]
     _check(x, "x", None)
-    _check(coef, "coef", x.dtype, (n_out, n_in, G + 3))
+    _check(coef, "coef", x.dtype, (n_out, n_in, G + degree))
     _check(w_base, "w_base", x.dtype, (n_out, n_in))
-    s = shape_of(x, coef, G, lo, hi, w_base, path)
+    s = shape_of(x, coef, G, lo, hi, w_base, path, degree)
     if y is None:
         y = torch.empty((batch, n_out), dtype=x.dtype, device=x.device)
     _check(y, "y", x.dtype, (batch, n_out))
@@ -76,15 +76,15 @@ def forward(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, y=None, ws=No
 
 
 def backward(x, coef, dY, G, lo, hi, w_base=None, need_dx=True, need_dcoef=True, need_dw_base=True,
-             path=N.KAN_PATH_AUTO, out=None, ws=None):
+             path=N.KAN_PATH_AUTO, out=None, ws=None, degree=3):
     """(dx, dcoef, dw_base) of the layer for upstream gradient dY; dcoef/dw_base are float32."""
     batch, n_in = x.shape
     n_out = coef.shape[0]
     _check(x, "x", None)
-    _check(coef, "coef", x.dtype, (n_out, n_in, G + 3))
+    _check(coef, "coef", x.dtype, (n_out, n_in, G + degree))
     _check(w_base, "w_base", x.dtype, (n_out, n_in))
     _check(dY, "dY", x.dtype, (batch, n_out))
-    s = shape_of(x, coef, G, lo, hi, w_base, path)
+    s = shape_of(x, coef, G, lo, hi, w_base, path, degree)
     if out is not None:
         dx, dcoef, dwb = out
     else:
@@ -100,14 +100,14 @@ def backward(x, coef, dY, G, lo, hi, w_base=None, need_dx=True, need_dcoef=True,
     return dx, dcoef, dwb
 
 
-def basis(x, G, lo, hi):
-    """(span int32 [.., in], w [.., in, 4], dw [.., in, 4]) of the basis step alone."""
+def basis(x, G, lo, hi, degree=3):
+    """(span int32 [.., in], w [.., in, k+1], dw [.., in, k+1]) of the basis step alone."""
     _check(x, "x", None)
     batch, n_in = x.shape
-    s = N.make_shape(batch, n_in, 1, G, lo, hi, _code(x), False)
+    s = N.make_shape(batch, n_in, 1, G, lo, hi, _code(x), False, degree=degree)
     span = torch.empty((batch, n_in), dtype=torch.int32, device=x.device)
-    w = torch.empty((batch, n_in, 4), dtype=torch.float32, device=x.device)
-    dw = torch.empty((batch, n_in, 4), dtype=torch.float32, device=x.device)
+    w = torch.empty((batch, n_in, degree + 1), dtype=torch.float32, device=x.device)
+    dw = torch.empty((batch, n_in, degree + 1), dtype=torch.float32, device=x.device)
     with torch.cuda.device(x.device):
         N.kan_basis(s, _p(x), _p(span), _p(w), _p(dw), _stream(x))
     return span, w, dw
@@ -115,44 +115,46 @@ def basis(x, G, lo, hi):
 
 class _KANFunction(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, x, coef, w_base, G, lo, hi):
+    def forward(ctx, x, coef, w_base, G, lo, hi, degree):
         x = x.contiguous()
-        y = forward(x, coef, G, lo, hi, w_base)
+        y = forward(x, coef, G, lo, hi, w_base, degree=degree)
         ctx.save_for_backward(x, coef, w_base)
-        ctx.grid = (G, lo, hi)
+        ctx.grid = (G, lo, hi, degree)
         return y
 
     @staticmethod
     def backward(ctx, dY):
         x, coef, w_base = ctx.saved_tensors
-        G, lo, hi = ctx.grid
+        G, lo, hi, degree = ctx.grid
         dx, dcoef, dwb = backward(x, coef, dY.contiguous().to(x.dtype), G, lo, hi, w_base,
                                   need_dx=ctx.needs_input_grad[0], need_dcoef=ctx.needs_input_grad[1],
-                                  need_dw_base=w_base is not None and ctx.needs_input_grad[2])
+                                  need_dw_base=w_base is not None and ctx.needs_input_grad[2], degree=degree)
         return (dx, None if dcoef is None else dcoef.to(coef.dtype), None if dwb is None else dwb.to(w_base.dtype),
-                None, None, None)
+                None, None, None, None)
 
 
 class KANLayer(torch.nn.Module):
-    """Cubic B-spline KAN layer, a drop-in for ``nn.Linear(in, out)``.
+    """B-spline KAN layer (cubic by default), a drop-in for ``nn.Linear(in, out)``.
 
-    Parameters: ``coef`` [out, in, G+3] and, with ``base=True``, ``w_base``
+    Parameters: ``coef`` [out, in, G+degree] and, with ``base=True``, ``w_base``
     [out, in] for the SiLU base branch.
     """
 
     def __init__(self, in_features, out_features, G=8, lo=-1.0, hi=1.0, base=False, coef_std=0.1,
-                 dtype=torch.float32, device=None):
+                 dtype=torch.float32, device=None, degree=3):
         super().__init__()
         self.in_features, self.out_features = in_features, out_features
-        self.G, self.lo, self.hi = int(G), float(lo), float(hi)
+        self.G, self.lo, self.hi, self.degree = int(G), float(lo), float(hi), int(degree)
         self.coef = torch.nn.Parameter(
-            torch.randn(out_features, in_features, G + 3, dtype=torch.float32, device=device).mul_(coef_std).to(dtype))
+            torch.randn(out_features, in_features, G + degree, dtype=torch.float32, device=device)
+            .mul_(coef_std).to(dtype))
         self.w_base = (torch.nn.Parameter(torch.randn(out_features, in_features, dtype=torch.float32, device=device)
                                           .mul_(in_features ** -0.5).to(dtype)) if base else None)
 
     def forward(self, x):
         lead = x.shape[:-1]
-        y = _KANFunction.apply(x.reshape(-1, self.in_features), self.coef, self.w_base, self.G, self.lo, self.hi)
+        y = _KANFunction.apply(x.reshape(-1, self.in_features), self.coef, self.w_base, self.G, self.lo, self.hi,
+                               self.degree)
         return y.reshape(*lead, self.out_features)
 
 

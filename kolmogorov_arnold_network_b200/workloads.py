@@ -20,13 +20,19 @@ import torch
 
 @dataclass(frozen=True)
 class Layer:
-    """One KAN layer's hyper-parameters (cubic B-splines on a uniform grid)."""
+    """One KAN layer's hyper-parameters (B-splines of degree `degree` on a uniform grid)."""
     inp: int
     out: int
     G: int
     lo: float
     hi: float
     base: bool = False
+    degree: int = 3
+
+    @property
+    def nb(self) -> int:
+        """Basis functions per edge: G + degree."""
+        return self.G + self.degree
 
 
 @dataclass(frozen=True)
@@ -63,6 +69,15 @@ def _grid_sweep():
     return out
 
 
+def _degree_sweep():
+    out = {}
+    for k in (1, 2, 4, 5):
+        nm = f"degree512_k{k}_g20_bf16_fwdbwd"
+        out[nm] = Workload(nm, 6, 65536, (Layer(512, 512, 20, -1.0, 1.0, degree=k),), "bf16", ("uniform", -1.0, 1.0),
+                           0.1, note=f"spline degree {k}: 512x512, batch 65536, G=20")
+    return out
+
+
 WORKLOADS = {
     "layer8x4": Workload("layer8x4", 1, 32, (Layer(8, 4, 8, -1.0, 1.0),), "f32", ("uniform", -1.0, 1.0), 0.1,
                          note="KANLayer(8,4) on a [32,8] batch, G=8 on [-1,1]"),
@@ -76,6 +91,7 @@ WORKLOADS = {
     "ffn768_3072_bf16": Workload("ffn768_3072_bf16", 5, 8192,
                                  (Layer(768, 3072, 5, -3.0, 3.0), Layer(3072, 768, 5, -3.0, 3.0)), "bf16",
                                  ("normal", 1.0), 0.05, note="KAN FFN block 768->3072->768, 8192 tokens"),
+    **_degree_sweep(),
 }
 
 #: the workload the benchmark times by default: the largest single-GPU one by edge evaluations per step
@@ -103,7 +119,7 @@ def draw_x(w: Workload, rows: int | None = None) -> torch.Tensor:
 def draw_coef(w: Workload, layer: int = 0) -> torch.Tensor:
     L = w.layers[layer]
     g = _gen(w.family, 1 if layer == 0 else 4)
-    c = torch.randn((L.out, L.inp, L.G + 3), generator=g, dtype=torch.float32) * w.coef_std
+    c = torch.randn((L.out, L.inp, L.nb), generator=g, dtype=torch.float32) * w.coef_std
     return c.to(w.torch_dtype)
 
 
@@ -131,9 +147,11 @@ def draw_all(w: Workload, rows: int | None = None) -> dict:
     return d
 
 
-def custom(batch, inp, out, G, lo, hi, dtype="f32", base=False, x_range=None, coef_std=0.1, family=90):
+def custom(batch, inp, out, G, lo, hi, dtype="f32", base=False, x_range=None, coef_std=0.1, family=90, degree=3):
     """An ad-hoc single-layer workload (tests of ragged and edge shapes)."""
     h = (hi - lo) / G
-    xr = x_range or (lo - 2 * h, hi + 2 * h)
-    return Workload(f"custom_{batch}x{inp}x{out}_g{G}_{dtype}", family, batch, (Layer(inp, out, G, lo, hi, base),),
-                    dtype, ("uniform", xr[0], xr[1]), coef_std)
+    # reach into the extended intervals (and, for degrees other than 3, a little beyond them)
+    ext = 2.0 if degree == 3 else degree - 0.5
+    xr = x_range or (lo - ext * h, hi + ext * h)
+    return Workload(f"custom_{batch}x{inp}x{out}_g{G}_k{degree}_{dtype}", family, batch,
+                    (Layer(inp, out, G, lo, hi, base, degree),), dtype, ("uniform", xr[0], xr[1]), coef_std)

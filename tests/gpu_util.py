@@ -59,31 +59,32 @@ def tile_inputs(n_in, nb, tile=128):
     return np.unique(cols // nb)
 
 
-def gpu_layer(x, coef, w_base, dY, G, lo, hi, path=0, want_bwd=True):
+def gpu_layer(x, coef, w_base, dY, G, lo, hi, path=0, want_bwd=True, degree=3):
     """Run forward (+ backward) through the C ABI on CUDA tensors; returns CUDA tensors."""
-    y = L.forward(x, coef, G, lo, hi, w_base, path=path)
+    y = L.forward(x, coef, G, lo, hi, w_base, path=path, degree=degree)
     if not want_bwd:
         return y, None, None, None
-    dx, dcoef, dwb = L.backward(x, coef, dY, G, lo, hi, w_base, path=path)
+    dx, dcoef, dwb = L.backward(x, coef, dY, G, lo, hi, w_base, path=path, degree=degree)
     return y, dx, dcoef, dwb
 
 
 def check_layer_against_oracle(o, x, coef, w_base, dY, G, lo, hi, y, dx, dcoef, dwb, dtype, rows=None,
-                               cols_in=None, cols_out=None):
+                               cols_in=None, cols_out=None, k=3):
     """Compare GPU outputs (CPU tensors) with the oracle, on sampled rows / (j, i) slices if given.
 
     Returns a dict of errors."""
     errs = {}
     xr = x if rows is None else x[rows]
     dYr = dY if rows is None else dY[rows]
-    y_ref = o.forward(xr, coef, G, lo, hi, w_base=w_base)
+    y_ref = o.forward(xr, coef, G, lo, hi, w_base=w_base, k=k)
     errs["y"] = rel_err(f64(y if rows is None else y[rows]), y_ref)
     if dx is not None:
-        dx_ref, _, _ = o.backward(xr, coef, dYr, G, lo, hi, w_base=w_base, want_dcoef=False, want_dw_base=False)
+        dx_ref, _, _ = o.backward(xr, coef, dYr, G, lo, hi, w_base=w_base, want_dcoef=False, want_dw_base=False,
+                                  k=k)
         errs["dx"] = rel_err(f64(dx if rows is None else dx[rows]), dx_ref)
     if dcoef is not None:
         if cols_in is None:
-            _, dc_ref, dwb_ref = o.backward(x, coef, dY, G, lo, hi, w_base=w_base, want_dx=False)
+            _, dc_ref, dwb_ref = o.backward(x, coef, dY, G, lo, hi, w_base=w_base, want_dx=False, k=k)
             errs["dcoef"] = rel_err(f64(dcoef), dc_ref)
             if dwb is not None:
                 errs["dw_base"] = rel_err(f64(dwb), dwb_ref)
@@ -92,7 +93,7 @@ def check_layer_against_oracle(o, x, coef, w_base, dY, G, lo, hi, y, dx, dcoef, 
             dYs = dY[:, cols_out]
             cs = coef[cols_out][:, cols_in]
             wbs = None if w_base is None else w_base[cols_out][:, cols_in]
-            _, dc_ref, dwb_ref = o.backward(xs, cs, dYs, G, lo, hi, w_base=wbs, want_dx=False)
+            _, dc_ref, dwb_ref = o.backward(xs, cs, dYs, G, lo, hi, w_base=wbs, want_dx=False, k=k)
             errs["dcoef"] = rel_err(f64(dcoef[cols_out][:, cols_in]), dc_ref)
             if dwb is not None:
                 errs["dw_base"] = rel_err(f64(dwb[cols_out][:, cols_in]), dwb_ref)

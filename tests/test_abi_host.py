@@ -39,12 +39,12 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version(lib):
-    assert N.kan_abi_version() == 1
+    assert N.kan_abi_version() == 2
 
 
 def test_shape_struct_layout():
-    assert ctypes.sizeof(N.kan_shape) == 48
-    assert N.kan_shape.G.offset == 24 and N.kan_shape.path.offset == 44
+    assert ctypes.sizeof(N.kan_shape) == 56
+    assert N.kan_shape.G.offset == 24 and N.kan_shape.path.offset == 44 and N.kan_shape.degree.offset == 48
 
 
 def st(code):
@@ -72,7 +72,7 @@ def shp(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(G=0), 1), (dict(G=-2), 1), (dict(G=251), 2), (dict(hi=-1.0), 1), (dict(lo=float("nan")), 1),
     (dict(hi=float("inf")), 1), (dict(n_in=0), 1), (dict(n_out=0), 1), (dict(batch=-1), 1), (dict(dtype=3), 1),
-    (dict(path=7), 1),
+    (dict(path=7), 1), (dict(degree=0), 1), (dict(degree=6), 1),
 ])
 def test_bad_shapes(lib, kw, code):
     assert fwd(shp(**kw)) == code

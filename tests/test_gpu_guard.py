@@ -58,24 +58,31 @@ class Guarded:
             assert not np.any(bits[self.g:self.g + self.n] == pat), f"{name}: elements left unwritten"
 
 
+CASES = [c + (3,) for c in SMALL] + [
+    # other spline degrees: k+1 weights per input in the producers and the dx gather
+    (300, 16, 256, 8, -1.0, 1.0, True, 1), (800, 24, 296, 20, -1.0, 1.0, False, 5),
+    (300, 40, 296, 8, -1.0, 1.0, False, 2), (257, 24, 64, 20, -1.0, 1.0, True, 4)]
+
+
 @pytest.mark.parametrize("path", [N.KAN_PATH_TENSOR, N.KAN_PATH_SIMT], ids=["tensor", "simt"])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
-@pytest.mark.parametrize("case", SMALL, ids=lambda c: "b{}_i{}_o{}_g{}{}".format(c[0], c[1], c[2], c[3],
-                                                                                    "_silu" if c[6] else ""))
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "b{}_i{}_o{}_g{}{}_k{}".format(c[0], c[1], c[2], c[3],
+                                                                                         "_silu" if c[6] else "", c[7]))
 def test_no_store_outside_the_outputs(path, dt, case):
-    batch, n_in, n_out, G, lo, hi, base = case
-    w = W.custom(batch, n_in, n_out, G, lo, hi, dtype=dt, base=base)
+    batch, n_in, n_out, G, lo, hi, base, k = case
+    w = W.custom(batch, n_in, n_out, G, lo, hi, dtype=dt, base=base, degree=k)
     x, coef, wb, dY = (None if t is None else t.cuda() for t in workload_inputs(w))
     tdt = x.dtype
-    s = L.shape_of(x, coef, G, lo, hi, wb, path)
+    s = L.shape_of(x, coef, G, lo, hi, wb, path, degree=k)
     y = Guarded((batch, n_out), tdt)
     dx = Guarded((batch, n_in), tdt)
     dc = Guarded(tuple(coef.shape), torch.float32)
     dwb = Guarded(tuple(wb.shape), torch.float32) if wb is not None else None
     wsf = Guarded((max(1, N.kan_workspace_size(s, False)),), torch.uint8)
     wsb = Guarded((max(1, N.kan_workspace_size(s, True)),), torch.uint8)
-    L.forward(x, coef, G, lo, hi, wb, path=path, y=y.t, ws=wsf.t)
-    L.backward(x, coef, dY, G, lo, hi, wb, path=path, out=(dx.t, dc.t, None if dwb is None else dwb.t), ws=wsb.t)
+    L.forward(x, coef, G, lo, hi, wb, path=path, y=y.t, ws=wsf.t, degree=k)
+    L.backward(x, coef, dY, G, lo, hi, wb, path=path, out=(dx.t, dc.t, None if dwb is None else dwb.t), ws=wsb.t,
+               degree=k)
     torch.cuda.synchronize()
     assert N.kan_sync_status(None) == 0
     y.check("y")

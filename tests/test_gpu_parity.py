@@ -33,14 +33,14 @@ def _gpu():
 
 # ---------------------------------------------------------------------------
 # basis step (S1, S2)
-def dense_from_basis(span, w, nb):
+def dense_from_basis(span, w, nb, k=3):
     span = span.cpu().numpy().reshape(-1)
-    w = w.cpu().double().numpy().reshape(-1, 4)
+    w = w.cpu().double().numpy().reshape(-1, k + 1)
     out = np.zeros((span.size, nb))
     for e in range(span.size):
         if span[e] == np.iinfo(np.int32).min:
             continue
-        for r in range(4):
+        for r in range(k + 1):
             m = span[e] + r
             if 0 <= m < nb:
                 out[e, m] = w[e, r]
@@ -126,6 +126,98 @@ def test_small_parity(oracle, path, dt, case):
                                       None if dwb is None else dwb.cpu(), dt)
     bad = {k: v for k, v in errs.items() if not v <= TOL[dt]}
     assert not bad, f"{errs}"
+
+
+# ---------------------------------------------------------------------------
+# spline degree k = 1..5 (FlashKAN abstract: degree-k splines, coordinate bounded to [0, k+1])
+DEGREES = [1, 2, 4, 5]
+DEG_SMALL = [
+    (300, 40, 296, 8, -1.0, 1.0, False),
+    (257, 24, 64, 20, -1.0, 1.0, True),
+    # CTA pairs (forward, dcoef), dx pairs over 256-row tiles
+    (300, 16, 256, 8, -1.0, 1.0, True),
+    (800, 24, 296, 20, -1.0, 1.0, False),
+    # x rows not 16-byte aligned (bf16), G + k = 8
+    (300, 20, 256, None, -3.0, 3.0, False),
+]
+
+
+@pytest.mark.parametrize("k", DEGREES)
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("G,lo,hi", [(8, -1.0, 1.0), (50, -1.0, 1.0), (5, -3.0, 3.0)])
+def test_basis_degree_vs_oracle(oracle, k, dt, G, lo, hi):
+    h = (hi - lo) / G
+    g = torch.Generator().manual_seed(100 + k)
+    x = (torch.rand(4096, generator=g) * (hi - lo + 2 * (k + 1) * h) + lo - (k + 1) * h)
+    x = torch.cat([x, torch.tensor([lo, hi, lo - k * h, hi + k * h, float("inf"), -float("inf"),
+                                    float("nan")])]).to(DT[dt])
+    span, w, dw = L.basis(x.reshape(-1, 1).to("cuda"), G, lo, hi, degree=k)
+    B_ref, dB_ref = oracle.basis(f64(x), G, lo, hi, k=k)
+    B = dense_from_basis(span, w, G + k, k)
+    dB = dense_from_basis(span, dw, G + k, k)
+    u = np.abs((f64(x) - lo) / h)
+    u = np.where(np.isfinite(u), u, 0.0)
+    tol = 2.0 ** -21 * (1.0 + u)[:, None]
+    assert np.all(np.abs(B - B_ref) <= tol)
+    # degree 1 is not differentiable at the knots: within the fp32 rounding of u = (x - lo)/h of a knot,
+    # the derivative of either side is correct, so those inputs are left out of the derivative check
+    near_knot = np.abs(u - np.round(u)) < 2.0 ** -20 * (1.0 + u) if k == 1 else np.zeros_like(u, dtype=bool)
+    assert np.all((np.abs(dB - dB_ref) * h <= 4 * tol) | near_knot[:, None])
+    assert np.all(B >= 0.0)
+    assert np.max((B != 0).sum(1)) <= k + 1
+
+
+@pytest.mark.parametrize("k", DEGREES)
+@pytest.mark.parametrize("path", ["tensor", "simt"])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("case", DEG_SMALL, ids=lambda c: "b{}_i{}_o{}_g{}{}".format(c[0], c[1], c[2], c[3],
+                                                                                        "_silu" if c[6] else ""))
+def test_degree_parity(oracle, k, path, dt, case):
+    batch, n_in, n_out, G, lo, hi, base = case
+    G = G if G is not None else 8 - k
+    w = W.custom(batch, n_in, n_out, G, lo, hi, dtype=dt, base=base, degree=k)
+    x, coef, wb, dY = workload_inputs(w)
+    y, dx, dc, dwb = gpu_layer(cuda(x), cuda(coef), cuda(wb), cuda(dY), G, lo, hi, path=PATHS[path], degree=k)
+    torch.cuda.synchronize()
+    assert N.kan_sync_status(None) == 0
+    errs = check_layer_against_oracle(oracle, x, coef, wb, dY, G, lo, hi, y.cpu(), dx.cpu(), dc.cpu(),
+                                      None if dwb is None else dwb.cpu(), dt, k=k)
+    bad = {kk: v for kk, v in errs.items() if not v <= TOL[dt]}
+    assert not bad, f"{errs}"
+
+
+@pytest.mark.parametrize("k", DEGREES)
+def test_marsden_degree_closed_form(k):
+    # coef[j,i,m] = prod_{l=1..k} (y_ji - t_{m+l}) reproduces y[b,j] = sum_i (y_ji - x_bi)^k and
+    # dx = -k sum_j dY (y_ji - x_bi)^(k-1) for x in [lo, hi] (Marsden's identity), at any batch size
+    G, lo, hi = 8, -1.0, 1.0
+    batch, n_in, n_out = 16384, 32, 96
+    g = torch.Generator().manual_seed(50 + k)
+    x = torch.rand(batch, n_in, generator=g) * 2 - 1
+    yt = (torch.rand(n_out, n_in, generator=g) * 0.5 - 0.25).double().numpy()
+    coef = torch.from_numpy(pins.marsden_coef(yt, G, lo, hi, k)).float()
+    dY = torch.randn(batch, n_out, generator=g)
+    y, dx, _, _ = gpu_layer(cuda(x), cuda(coef), None, cuda(dY), G, lo, hi, path=N.KAN_PATH_TENSOR, degree=k)
+    xd = f64(x)
+    ref = ((yt[None, :, :] - xd[:, None, :]) ** k).sum(2)
+    dref = np.einsum("bj,bji->bi", f64(dY), -k * (yt[None, :, :] - xd[:, None, :]) ** (k - 1))
+    assert rel_err(f64(y.cpu()), ref) <= TOL["f32"]
+    assert rel_err(f64(dx.cpu()), dref) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("name", [f"degree512_k{k}_g20_bf16_fwdbwd" for k in DEGREES])
+def test_degree_workload_parity(oracle, name):
+    w = W.WORKLOADS[name]
+    Ly = w.layers[0]
+    x, coef, wb, dY = workload_inputs(w)
+    y, dx, dc, dwb = gpu_layer(cuda(x), cuda(coef), cuda(wb), cuda(dY), Ly.G, Ly.lo, Ly.hi, degree=Ly.degree)
+    torch.cuda.synchronize()
+    assert N.kan_sync_status(None) == 0
+    rows = np.union1d(tile_rows(w.batch), sample_rows(w.batch))
+    errs = check_layer_against_oracle(oracle, x, coef, wb, dY, Ly.G, Ly.lo, Ly.hi, y.cpu(), dx.cpu(), dc.cpu(), None,
+                                      w.dtype, rows=rows, cols_in=tile_inputs(Ly.inp, Ly.nb),
+                                      cols_out=np.arange(Ly.out), k=Ly.degree)
+    assert all(v <= TOL[w.dtype] for v in errs.values()), errs
 
 
 # ---------------------------------------------------------------------------
