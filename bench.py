@@ -560,6 +560,81 @@ def config_of(w: W.Workload):
     return c
 
 
+class GrRunner:
+    """Buffers and the two C-ABI calls of one GR-KAN workload: the forward (y) and one backward that
+    returns dx, da and db."""
+
+    def __init__(self, w: W.GrWorkload, dev):
+        from kolmogorov_arnold_network_b200 import _native as N
+        self.N, self.w, self.dev = N, w, dev
+        d = W.draw_grkan(w)
+        self.x, self.dY = d["x"].to(dev), d["dY"].to(dev)
+        self.a, self.b = d["a"].to(dev), d["b"].to(dev)
+        self.y = torch.empty_like(self.x)
+        self.dx = torch.empty_like(self.x)
+        self.da = torch.empty_like(self.a)
+        self.db = torch.empty_like(self.b)
+        code = N.KAN_F32 if w.dtype == "f32" else N.KAN_BF16
+        self.s = N.make_grkan_shape(w.rows, w.channels, w.groups, w.m, w.n, code)
+        self.ws = torch.empty(max(16, N.kan_grkan_workspace_size(self.s)), dtype=torch.uint8, device=dev)
+
+    def calls(self):
+        N, st = self.N, torch.cuda.current_stream(self.dev).cuda_stream
+
+        def fwd():
+            N.kan_grkan_forward(self.s, self.x.data_ptr(), self.a.data_ptr(), self.b.data_ptr(), self.y.data_ptr(), st)
+
+        def bwd():
+            N.kan_grkan_backward(self.s, self.x.data_ptr(), self.a.data_ptr(), self.b.data_ptr(), self.dY.data_ptr(),
+                                 self.dx.data_ptr(), self.da.data_ptr(), self.db.data_ptr(), self.ws.data_ptr(),
+                                 self.ws.numel(), st)
+        return [("fwd", fwd), ("bwd", bwd)]
+
+
+def time_grkan(w: W.GrWorkload, dev, K, flush, pk):
+    """GR-KAN forward + backward: K steps, events around each call, L2 flushed between steps; the
+    backward (the larger call) against the HBM roofline."""
+    R = GrRunner(w, dev)
+    calls = R.calls()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        flush.zero_()
+        for _, c in calls:
+            c()
+    torch.cuda.synchronize(dev)
+    ev = [[(_ev(), _ev()) for _ in calls] for _ in range(K)]
+    for k in range(K):
+        flush.zero_()
+        for (a, b), (_, c) in zip(ev[k], calls):
+            a.record(stream)
+            c()
+            b.record(stream)
+    torch.cuda.synchronize(dev)
+    seg = {nm: sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(K)) / K for i, (nm, _) in enumerate(calls)}
+    esz = 4 if w.dtype == "f32" else 2
+    n = w.elements
+    bytes_ = {"fwd": 2.0 * n * esz, "bwd": 3.0 * n * esz}      # fwd: x in, y out; bwd: x, dY in, dx out
+    gbs = {k: bytes_[k] / (seg[k] / 1000.0) / 1e9 for k in seg}
+    ms = seg["fwd"] + seg["bwd"]
+    out = {"ms_per_step": ms, "value": n / (ms / 1000.0), "unit": "elements/s", "steps": K, "dtype": w.dtype,
+           "dominant": "bwd", "bound": "hbm", "achieved": gbs["bwd"], "peak": pk["hbm"], "peak_unit": "GB/s",
+           "frac": gbs["bwd"] / pk["hbm"], "fwd_frac": gbs["fwd"] / pk["hbm"], "segment_ms": seg,
+           "algorithmic_bytes_per_launch": bytes_,
+           "step_roofline": {"t_roof_ms": (bytes_["fwd"] + bytes_["bwd"]) / (pk["hbm"] * 1e9) * 1000.0,
+                             "frac": (bytes_["fwd"] + bytes_["bwd"]) / (pk["hbm"] * 1e9) * 1000.0 / ms,
+                             "bound": "HBM, algorithmic bytes"},
+           "config": {"rows": w.rows, "channels": w.channels, "groups": w.groups, "m": w.m, "n": w.n,
+                      "note": w.note}}
+    # bitwise reproducibility of the atomic-free gradient reduction
+    d1 = (R.da.clone(), R.db.clone())
+    calls[1][1]()
+    torch.cuda.synchronize(dev)
+    out["deterministic"] = bool(torch.equal(d1[0], R.da) and torch.equal(d1[1], R.db))
+    del R
+    torch.cuda.empty_cache()
+    return out
+
+
 #: workloads timed beside the headline one (each in the same JSON line, with the adjoint-identity check)
 EXTRA_WORKLOADS = ["layer784x64_silu", "layer1024_g20_bf16"] + \
     [f"sweep512_g{G}_{dt}_fwdbwd" for G in (8, 20, 50) for dt in ("bf16", "f32")] + \
@@ -638,6 +713,8 @@ def run_ours(args, world, rank, local):
                           "adjoint_rel_err": ax, "adjoint_ok": all(v <= tolx for v in ax.values())}
             del Rx
             torch.cuda.empty_cache()
+        for nm, wg in W.GR_WORKLOADS.items():
+            others[nm] = time_grkan(wg, dev, min(K, args.extra_steps), flush, pk)
 
     st = R_status()
     if st != 0:

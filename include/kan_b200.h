@@ -196,6 +196,53 @@ KAN_API kan_status kan_set_timing_marks(void* after_prep, void* after_dcoef);
  * blocks < 1, iters < 1 or a null pointer. */
 KAN_API kan_status kan_ffma_probe(int32_t blocks, int64_t iters, float* sink, double* flops, void* stream);
 
+/* ------------------------------------------------------------------------
+ * GR-KAN: the group-rational activation of the Kolmogorov-Arnold Transformer.
+ *
+ * The FlashKAT abstract ("FlashKAT: Understanding and Addressing Performance
+ * Bottlenecks in the Kolmogorov-Arnold Transformer", Abstract) traces the slow
+ * training of GR-KAN to the gradient accumulation of its backward pass (memory
+ * stalls, atomic adds) and fixes it by keeping the accumulation on chip.  The
+ * rational function is the Pade activation unit of that page's reference list,
+ * in the form whose denominator cannot vanish:
+ *   y[r,c] = phi_g(x[r,c]),  phi_g(x) = P_g(x) / (1 + |S_g(x)|),
+ *   P_g(x) = sum_{p=0..m} a[g,p] x^p,  S_g(x) = sum_{q=1..n} b[g,q-1] x^q,
+ *   g = c / (channels / groups)   (contiguous, equal channel groups).
+ * Backward for upstream gradient dY (sign(0) = 0):
+ *   dx[r,c]  = dY (P' - phi sign(S) S') / (1 + |S|)
+ *   da[g,p]  = sum over the group's elements of dY x^p / (1 + |S|)
+ *   db[g,q-1]= sum over the group's elements of -dY phi sign(S) x^q / (1 + |S|)
+ * The sums are reduced without atomics in a fixed order (per-block partials
+ * in the caller's workspace, then one pass in fp64): bitwise reproducible.
+ *
+ * Layouts (row-major): x, y, dY, dx [rows, channels] in the operand dtype
+ * (KAN_F32 or KAN_BF16); a [groups, m+1], b [groups, n], da, db float32
+ * (da, db overwritten).  Pointers 16-byte aligned; channels / groups times the
+ * element size must be a multiple of 16 bytes (else KAN_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int64_t rows;        /* tokens, >= 0 */
+    int64_t channels;    /* >= 1, a multiple of groups */
+    int32_t groups;      /* >= 1 */
+    int32_t num_degree;  /* m, 1..7: P has m+1 coefficients */
+    int32_t den_degree;  /* n, 1..8: S has n coefficients (no constant term) */
+    int32_t dtype;       /* kan_dtype of x, y, dY, dx */
+} kan_grkan_shape;
+
+/* Bytes of workspace kan_grkan_backward needs for da / db on the current device. */
+KAN_API kan_status kan_grkan_workspace_size(const kan_grkan_shape* s, size_t* bytes);
+
+/* y = phi(x).  Asynchronous on stream; host errors return before any launch. */
+KAN_API kan_status kan_grkan_forward(const kan_grkan_shape* s, const void* x, const float* a, const float* b, void* y,
+                                     void* stream);
+
+/* dx, da, db for upstream gradient dY; any of the three may be NULL to skip
+ * it.  The workspace (kan_grkan_workspace_size bytes) is needed only when da
+ * or db is requested.  KAN_ERR_WORKSPACE if it is too small. */
+KAN_API kan_status kan_grkan_backward(const kan_grkan_shape* s, const void* x, const float* a, const float* b,
+                                      const void* dY, void* dx, float* da, float* db, void* workspace,
+                                      size_t ws_bytes, void* stream);
+
 /* Static description of a status code. */
 KAN_API const char* kan_status_string(kan_status st);
 

@@ -20,6 +20,7 @@ STATUS = {0: "KAN_OK", 1: "KAN_ERR_INVALID_ARG", 2: "KAN_ERR_UNSUPPORTED", 3: "K
 #: every symbol the header declares
 EXPORTS = ("kan_abi_version", "kan_workspace_size", "kan_forward", "kan_backward", "kan_basis", "kan_sync_status",
            "kan_launch_count", "kan_forward_fixed_scratch", "kan_set_timing_marks", "kan_ffma_probe",
+           "kan_grkan_workspace_size", "kan_grkan_forward", "kan_grkan_backward",
            "kan_selftest_wait_timeout", "kan_status_string", "kan_last_error")
 
 
@@ -28,6 +29,11 @@ class kan_shape(ctypes.Structure):
                 ("G", ctypes.c_int32), ("lo", ctypes.c_float), ("hi", ctypes.c_float),
                 ("dtype", ctypes.c_int32), ("has_base", ctypes.c_int32), ("path", ctypes.c_int32),
                 ("degree", ctypes.c_int32)]
+
+
+class kan_grkan_shape(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("channels", ctypes.c_int64), ("groups", ctypes.c_int32),
+                ("num_degree", ctypes.c_int32), ("den_degree", ctypes.c_int32), ("dtype", ctypes.c_int32)]
 
 
 class KanError(RuntimeError):
@@ -72,6 +78,13 @@ def load(path: str | None = None):
     lib.kan_launch_count.argtypes = []
     lib.kan_forward_fixed_scratch.restype = ctypes.c_int
     lib.kan_forward_fixed_scratch.argtypes = [sp, _vp, _vp, _vp, _vp, _vp]
+    gp = ctypes.POINTER(kan_grkan_shape)
+    lib.kan_grkan_workspace_size.restype = ctypes.c_int
+    lib.kan_grkan_workspace_size.argtypes = [gp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kan_grkan_forward.restype = ctypes.c_int
+    lib.kan_grkan_forward.argtypes = [gp, _vp, _vp, _vp, _vp, _vp]
+    lib.kan_grkan_backward.restype = ctypes.c_int
+    lib.kan_grkan_backward.argtypes = [gp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
     lib.kan_set_timing_marks.restype = ctypes.c_int
     lib.kan_set_timing_marks.argtypes = [_vp, _vp]
     lib.kan_ffma_probe.restype = ctypes.c_int
@@ -119,6 +132,25 @@ def kan_backward(shape, x, coef, w_base, dY, dx, dcoef, dw_base, workspace, ws_b
 
 def kan_basis(shape, x, span, w, dw, stream):
     check(load().kan_basis(ctypes.byref(shape), x, span, w, dw, stream), "kan_basis")
+
+
+def make_grkan_shape(rows, channels, groups, num_degree, den_degree, dtype) -> kan_grkan_shape:
+    return kan_grkan_shape(int(rows), int(channels), int(groups), int(num_degree), int(den_degree), int(dtype))
+
+
+def kan_grkan_workspace_size(shape: kan_grkan_shape) -> int:
+    n = ctypes.c_size_t(0)
+    check(load().kan_grkan_workspace_size(ctypes.byref(shape), ctypes.byref(n)), "kan_grkan_workspace_size")
+    return n.value
+
+
+def kan_grkan_forward(shape, x, a, b, y, stream):
+    check(load().kan_grkan_forward(ctypes.byref(shape), x, a, b, y, stream), "kan_grkan_forward")
+
+
+def kan_grkan_backward(shape, x, a, b, dY, dx, da, db, workspace, ws_bytes, stream):
+    check(load().kan_grkan_backward(ctypes.byref(shape), x, a, b, dY, dx, da, db, workspace, ws_bytes, stream),
+          "kan_grkan_backward")
 
 
 def kan_set_timing_marks(after_prep, after_dcoef):

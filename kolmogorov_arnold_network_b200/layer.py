@@ -158,6 +158,83 @@ class KANLayer(torch.nn.Module):
         return y.reshape(*lead, self.out_features)
 
 
+# ---------------------------------------------------------------------------
+# GR-KAN: the group-rational activation (safe Pade form per channel group)
+def grkan_shape(x, a, b, groups):
+    rows, C = x.shape
+    return N.make_grkan_shape(rows, C, groups, a.shape[1] - 1, b.shape[1], _code(x))
+
+
+def grkan_forward(x, a, b, groups, y=None):
+    """y = P_g(x) / (1 + |S_g(x)|) per channel, g = channel // (C / groups); a [G, m+1], b [G, n] float32."""
+    _check(x, "x", None)
+    _check(a, "a", torch.float32)
+    _check(b, "b", torch.float32)
+    s = grkan_shape(x, a, b, groups)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(y, "y", x.dtype, tuple(x.shape))
+    with torch.cuda.device(x.device):
+        N.kan_grkan_forward(s, _p(x), _p(a), _p(b), _p(y), _stream(x))
+    return y
+
+
+def grkan_backward(x, a, b, dY, groups, need_dx=True, need_da=True, need_db=True, out=None, ws=None):
+    """(dx, da, db) for upstream gradient dY; da, db are float32, reduced without atomics."""
+    _check(x, "x", None)
+    _check(dY, "dY", x.dtype, tuple(x.shape))
+    s = grkan_shape(x, a, b, groups)
+    if out is not None:
+        dx, da, db = out
+    else:
+        dx = torch.empty_like(x) if need_dx else None
+        da = torch.empty(a.shape, dtype=torch.float32, device=x.device) if need_da else None
+        db = torch.empty(b.shape, dtype=torch.float32, device=x.device) if need_db else None
+    if ws is None and (da is not None or db is not None):
+        with torch.cuda.device(x.device):
+            n = N.kan_grkan_workspace_size(s)
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device=x.device)
+    with torch.cuda.device(x.device):
+        N.kan_grkan_backward(s, _p(x), _p(a), _p(b), _p(dY), _p(dx), _p(da), _p(db), _p(ws),
+                             0 if ws is None else ws.numel(), _stream(x))
+    return dx, da, db
+
+
+class _GRKANFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, a, b, groups):
+        x = x.contiguous()
+        ctx.save_for_backward(x, a, b)
+        ctx.groups = groups
+        return grkan_forward(x, a, b, groups)
+
+    @staticmethod
+    def backward(ctx, dY):
+        x, a, b = ctx.saved_tensors
+        dx, da, db = grkan_backward(x, a, b, dY.contiguous().to(x.dtype), ctx.groups,
+                                    need_dx=ctx.needs_input_grad[0], need_da=ctx.needs_input_grad[1],
+                                    need_db=ctx.needs_input_grad[2])
+        return dx, da, db, None
+
+
+class GRKAN(torch.nn.Module):
+    """Group-rational activation over the last dimension (channels): ``groups`` coefficient sets of a
+    degree-(m, n) safe Pade function, initialised to the identity-like phi(x) = x."""
+
+    def __init__(self, channels, groups=8, num_degree=5, den_degree=4, device=None):
+        super().__init__()
+        self.channels, self.groups = channels, groups
+        a = torch.zeros(groups, num_degree + 1, dtype=torch.float32, device=device)
+        a[:, 1] = 1.0
+        self.a = torch.nn.Parameter(a)
+        self.b = torch.nn.Parameter(torch.zeros(groups, den_degree, dtype=torch.float32, device=device))
+
+    def forward(self, x):
+        lead = x.shape[:-1]
+        y = _GRKANFunction.apply(x.reshape(-1, self.channels), self.a, self.b, self.groups)
+        return y.reshape(*lead, self.channels)
+
+
 class KANNetwork(torch.nn.Module):
     """Stack of KANLayer: ``KANNetwork([784, 64, 10])``."""
 

@@ -98,6 +98,41 @@ WORKLOADS = {
 BENCH_DEFAULT = "ffn768_3072_bf16"
 
 
+@dataclass(frozen=True)
+class GrWorkload:
+    """A GR-KAN (group-rational activation) workload: x [rows, channels] in `groups` channel groups,
+    numerator degree m, denominator degree n."""
+    name: str
+    family: int
+    rows: int
+    channels: int
+    groups: int
+    m: int
+    n: int
+    dtype: str
+    note: str = ""
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def elements(self) -> int:
+        return self.rows * self.channels
+
+
+def _grkan():
+    out = {}
+    for dt in ("bf16", "f32"):
+        nm = f"grkan_vitb_{dt}"
+        out[nm] = GrWorkload(nm, 7, 128 * 197, 3072, 8, 5, 4, dt,
+                             note="GR-KAN on the 3072-wide hidden activation of a ViT-B MLP, 128 images x 197 tokens")
+    return out
+
+
+GR_WORKLOADS = _grkan()
+
+
 def _gen(family: int, tensor_id: int) -> torch.Generator:
     g = torch.Generator(device="cpu")
     g.manual_seed(1000 * family + tensor_id)
@@ -145,6 +180,22 @@ def draw_all(w: Workload, rows: int | None = None) -> dict:
         d[f"coef{li}"] = draw_coef(w, li)
         d[f"w_base{li}"] = draw_w_base(w, li)
     return d
+
+
+def draw_grkan(w: GrWorkload, rows: int | None = None) -> dict:
+    """x ~ N(0, 1), dY ~ N(0, 1) in the operand dtype; a ~ N(0, 0.5), b ~ N(0, 0.5) float32 (ids 0, 3, 1, 2)."""
+    rows = w.rows if rows is None else rows
+    x = torch.randn((rows, w.channels), generator=_gen(w.family, 0), dtype=torch.float32).to(w.torch_dtype)
+    dY = torch.randn((rows, w.channels), generator=_gen(w.family, 3), dtype=torch.float32).to(w.torch_dtype)
+    a = torch.randn((w.groups, w.m + 1), generator=_gen(w.family, 1), dtype=torch.float32) * 0.5
+    b = torch.randn((w.groups, w.n), generator=_gen(w.family, 2), dtype=torch.float32) * 0.5
+    return {"x": x, "dY": dY, "a": a, "b": b}
+
+
+def custom_grkan(rows, channels, groups, m=5, n=4, dtype="f32", family=91):
+    """An ad-hoc GR-KAN workload (tests of ragged and edge shapes)."""
+    return GrWorkload(f"grkan_custom_{rows}x{channels}_g{groups}_{m}{n}_{dtype}", family, rows, channels, groups, m, n,
+                      dtype)
 
 
 def custom(batch, inp, out, G, lo, hi, dtype="f32", base=False, x_range=None, coef_std=0.1, family=90, degree=3):
