@@ -105,25 +105,26 @@ def csrc_hash() -> str:
 # ---------------------------------------------------------------------------
 # FLOP / byte accounting (per call, algorithmic)
 def layer_dense_flops(batch, L):
-    """Dense-expanded FLOPs of one layer GEMM: 2 * batch * out * (in*(G+k) [+ in for SiLU])."""
-    k = L.inp * L.nb + (L.inp if L.base else 0)
+    """Dense-expanded FLOPs of one layer GEMM: 2 * batch * out * (units * columns per unit [+ in for SiLU])."""
+    k = L.units * L.cols + (L.inp if L.base else 0)
     return 2.0 * batch * L.out * k
 
 
 def layer_alg_flops(batch, L):
-    """Algorithmic FLOPs of one layer GEMM: k+1 FMAs per edge (4 for cubic splines; +1 with SiLU), 2 FLOPs each."""
-    return (2.0 * (L.degree + 1) + (2.0 if L.base else 0.0)) * batch * L.inp * L.out
+    """Algorithmic FLOPs of one layer GEMM: (k+1)^dims FMAs per edge (4 for cubic splines, 16 for cubic
+    surfaces; +1 with SiLU), 2 FLOPs each."""
+    return (2.0 * (L.degree + 1) ** L.dims + (2.0 if L.base else 0.0)) * batch * L.units * L.out
 
 
 def layer_bytes(batch, L, esz, call):
     """Algorithmic HBM bytes of one call: operands read once, outputs written once."""
     x = batch * L.inp * esz
     dy = batch * L.out * esz
-    coef = L.out * L.inp * L.nb * esz + (L.out * L.inp * esz if L.base else 0)
+    coef = L.out * L.units * L.cols * esz + (L.out * L.inp * esz if L.base else 0)
     if call == "fwd":
         return x + coef + batch * L.out * esz
     if call == "dcoef":
-        return x + dy + (L.out * L.inp * L.nb + (L.out * L.inp if L.base else 0)) * 4
+        return x + dy + (L.out * L.units * L.cols + (L.out * L.inp if L.base else 0)) * 4
     return x + dy + coef + batch * L.inp * esz          # dx
 
 
@@ -169,7 +170,7 @@ class Runner:
         for li, L in enumerate(w.layers):
             coef = d[f"coef{li}"].to(dev)
             wb = None if d[f"w_base{li}"] is None else d[f"w_base{li}"].to(dev)
-            s = LY.shape_of(act, coef, L.G, L.lo, L.hi, wb, degree=L.degree)
+            s = LY.shape_of(act, coef, L.G, L.lo, L.hi, wb, degree=L.degree, dims=L.dims)
             ws_f = LY.workspace(s, False, dev)
             ws_b = LY.workspace(s, True, dev)
             y = torch.empty((w.batch, L.out), dtype=dt, device=dev)
@@ -455,6 +456,29 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+def _oracle_step(o, d, w: W.Workload, rows: int, cores: int):
+    """The whole hot path of the workload on the first `rows` rows, by the fp64 oracle (forward through
+    every layer, then the backward of every layer, last first)."""
+    from oracle import kan2d
+    act = d["x"][:rows]
+    acts = []
+    for li, L in enumerate(w.layers):
+        acts.append(act)
+        if L.dims == 2:
+            act = kan2d.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, k=L.degree, o=o)
+        else:
+            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
+                            nthreads=cores)
+    g = d["dY"][:rows]
+    for li in (reversed(range(len(w.layers))) if w.mode != "fwd" else ()):
+        L = w.layers[li]
+        if L.dims == 2:
+            g, _ = kan2d.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, k=L.degree, o=o)
+        else:
+            g, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
+                                 nthreads=cores)
+
+
 def cpu_baseline(w: W.Workload, target_s=12.0):
     """The fp64 oracle, as it stands, on a row sample of the workload (host cores)."""
     import oracle
@@ -463,21 +487,8 @@ def cpu_baseline(w: W.Workload, target_s=12.0):
     d = W.draw_all(w)
 
     def run(rows):
-        x = d["x"][:rows]
-        dY = d["dY"][:rows]
         t0 = time.perf_counter()
-        act = x
-        acts = []
-        for li, L in enumerate(w.layers):
-            acts.append(act)
-            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
-                            nthreads=cores)
-        g = dY
-        for li in (reversed(range(len(w.layers))) if w.mode != "fwd" else ()):
-            L = w.layers[li]
-            gx, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
-                                  nthreads=cores)
-            g = gx
+        _oracle_step(o, d, w, rows, cores)
         return time.perf_counter() - t0
 
     probe = max(cores, 8)
@@ -492,7 +503,7 @@ def cpu_baseline(w: W.Workload, target_s=12.0):
         passes += 1
         if t >= 0.8 * target_s or passes >= 100:
             break
-    edges = passes * sum(rows * L.inp * L.out for L in w.layers)
+    edges = passes * sum(rows * L.units * L.out for L in w.layers)
     return {"value": edges / t, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{passes} pass(es) over {rows} of {w.batch} rows of {w.name}, fp64 Cox-de Boor "
                       f"{'forward' if w.mode == 'fwd' else 'forward+backward'}, {t:.1f} s"}
@@ -508,18 +519,7 @@ def run_reference(args, world, rank):
     d = W.draw_all(w)
 
     def step(rows):
-        x = d["x"][:rows]
-        act = x
-        acts = []
-        for li, L in enumerate(w.layers):
-            acts.append(act)
-            act = o.forward(act, d[f"coef{li}"], L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
-                            nthreads=cores)
-        g = d["dY"][:rows]
-        for li in (reversed(range(len(w.layers))) if w.mode != "fwd" else ()):
-            L = w.layers[li]
-            g, _, _ = o.backward(acts[li], d[f"coef{li}"], g, L.G, L.lo, L.hi, w_base=d[f"w_base{li}"], k=L.degree,
-                                 nthreads=cores)
+        _oracle_step(o, d, w, rows, cores)
 
     # size the per-step sample so that warmup + steps end within ~2 minutes
     probe = max(cores, 8)
@@ -534,7 +534,7 @@ def run_reference(args, world, rank):
     for _ in range(args.steps):
         step(rows)
     dt = time.perf_counter() - t0
-    edges = sum(rows * L.inp * L.out for L in w.layers) * args.steps
+    edges = sum(rows * L.units * L.out for L in w.layers) * args.steps
     value = edges / dt
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
@@ -549,7 +549,7 @@ def run_reference(args, world, rank):
 def config_of(w: W.Workload):
     L0 = w.layers[0]
     c = {"workload": w.name, "batch": w.batch, "layers": [[L.inp, L.out] for L in w.layers], "G": L0.G,
-         "degree": L0.degree, "grid": [L0.lo, L0.hi], "silu_base": L0.base, "mode": w.mode,
+         "degree": L0.degree, "dims": L0.dims, "grid": [L0.lo, L0.hi], "silu_base": L0.base, "mode": w.mode,
          "l2": "256 MiB flush between steps",
          "note": w.note}
     if w.dtype == "f32":
@@ -638,7 +638,8 @@ def time_grkan(w: W.GrWorkload, dev, K, flush, pk):
 #: workloads timed beside the headline one (each in the same JSON line, with the adjoint-identity check)
 EXTRA_WORKLOADS = ["layer784x64_silu", "layer1024_g20_bf16"] + \
     [f"sweep512_g{G}_{dt}_fwdbwd" for G in (8, 20, 50) for dt in ("bf16", "f32")] + \
-    [f"degree512_k{k}_g20_bf16_fwdbwd" for k in (1, 2, 4, 5)]
+    [f"degree512_k{k}_g20_bf16_fwdbwd" for k in (1, 2, 4, 5)] + \
+    [f"surface512_g8_{dt}_fwdbwd" for dt in ("bf16", "f32")]
 
 
 def run_ours(args, world, rank, local):

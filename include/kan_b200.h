@@ -41,6 +41,19 @@
  * The operand dtype is float32 or bfloat16; accumulation is always fp32.
  * Pointers must be 16-byte aligned.
  *
+ * 2-D surfaces (kan_shape.dims = 2): "tensor-product B-spline surfaces for
+ * joint function approximation" (InKAN landing page, "Why InKAN?", item "1D
+ * and 2D Splines").  The inputs are taken in consecutive pairs (u, v) =
+ * (x[b,2p], x[b,2p+1]) and each edge (j, p) carries a surface on the same
+ * knot grid in both coordinates:
+ *   y[b,j] = sum_p sum_{m1,m2} coef[j,p,m1,m2] B_m1(u) B_m2(v)
+ *   dcoef[j,p,m1,m2] = sum_b dY[b,j] B_m1(u) B_m2(v)
+ *   dx[b,2p]   = sum_j dY[b,j] sum coef[j,p,m1,m2] B'_m1(u) B_m2(v)
+ *   dx[b,2p+1] = sum_j dY[b,j] sum coef[j,p,m1,m2] B_m1(u) B'_m2(v)
+ * with coef and dcoef [out, in/2, G+k, G+k].  Requires in even, no SiLU
+ * branch, cubic splines (degree 3), and the tensor-core path: (G+3)^2 at most
+ * 249 columns per pair for bf16 and 121 for fp32 (KAN_ERR_UNSUPPORTED else).
+ *
  * Ownership: the caller owns every buffer, the workspace included.  The
  * library allocates no memory per call.  It holds two fixed device arrays in
  * its own image, which every GPU that loads it keeps until the process exits:
@@ -103,6 +116,7 @@ typedef struct {
     int32_t has_base;  /* 1: add the SiLU base branch w_base[j,i] silu(x[b,i]) */
     int32_t path;      /* KAN_PATH_* */
     int32_t degree;    /* spline degree k, 1..5 (3: cubic) */
+    int32_t dims;      /* 1: univariate splines; 2: tensor-product surfaces over input pairs (below) */
 } kan_shape;
 
 /* ABI version of the loaded library (KAN_ABI_VERSION it was built with). */

@@ -28,7 +28,7 @@ class kan_shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("in_", ctypes.c_int64), ("out", ctypes.c_int64),
                 ("G", ctypes.c_int32), ("lo", ctypes.c_float), ("hi", ctypes.c_float),
                 ("dtype", ctypes.c_int32), ("has_base", ctypes.c_int32), ("path", ctypes.c_int32),
-                ("degree", ctypes.c_int32)]
+                ("degree", ctypes.c_int32), ("dims", ctypes.c_int32)]
 
 
 class kan_grkan_shape(ctypes.Structure):
@@ -99,9 +99,9 @@ def check(status: int, where: str):
         raise KanError(status, where, load().kan_last_error().decode())
 
 
-def make_shape(batch, n_in, n_out, G, lo, hi, dtype, has_base, path=KAN_PATH_AUTO, degree=3) -> kan_shape:
+def make_shape(batch, n_in, n_out, G, lo, hi, dtype, has_base, path=KAN_PATH_AUTO, degree=3, dims=1) -> kan_shape:
     return kan_shape(int(batch), int(n_in), int(n_out), int(G), float(lo), float(hi), int(dtype), int(bool(has_base)),
-                     int(path), int(degree))
+                     int(path), int(degree), int(dims))
 
 
 # ---- the C-ABI calls, same names, raw pointers (ints) and sizes ----

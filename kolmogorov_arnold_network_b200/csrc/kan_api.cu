@@ -84,16 +84,28 @@ kan_status validate(const kan_shape* s, Problem* p)
     if (s->has_base != 0 && s->has_base != 1) return fail(KAN_ERR_INVALID_ARG, "has_base must be 0 or 1");
     if (s->path < KAN_PATH_AUTO || s->path > KAN_PATH_SIMT) return fail(KAN_ERR_INVALID_ARG, "unknown path");
     if (s->degree < 1 || s->degree > 5) return fail(KAN_ERR_INVALID_ARG, "degree must be 1..5");
-    const int64_t nb = s->G + s->degree;
-    if (s->in > ((int64_t)1 << 40) / nb || s->out > ((int64_t)1 << 40) || s->batch > ((int64_t)1 << 40))
+    if (s->dims != 1 && s->dims != 2) return fail(KAN_ERR_INVALID_ARG, "dims must be 1 or 2");
+    if (s->dims == 2) {
+        if (s->in % 2 != 0) return fail(KAN_ERR_INVALID_ARG, "2-D surfaces need an even input count");
+        if (s->has_base) return fail(KAN_ERR_INVALID_ARG, "2-D surfaces have no SiLU branch");
+        if (s->degree != 3) return fail(KAN_ERR_UNSUPPORTED, "2-D surfaces are cubic (degree 3) only");
+        if (s->path == KAN_PATH_SIMT) return fail(KAN_ERR_UNSUPPORTED, "2-D surfaces run on the tensor-core path only");
+    }
+    const int64_t nb1 = s->G + s->degree;
+    const int64_t nb = s->dims == 2 ? nb1 * nb1 : nb1;
+    const int64_t units = s->dims == 2 ? s->in / 2 : s->in;
+    if (units > ((int64_t)1 << 40) / nb || s->out > ((int64_t)1 << 40) || s->batch > ((int64_t)1 << 40))
         return fail(KAN_ERR_UNSUPPORTED, "sizes too large");
     p->batch = s->batch;
-    p->in = s->in;
+    p->in = units;
+    p->x_ld = s->in;
     p->out = s->out;
     p->G = s->G;
     p->k = s->degree;
+    p->dims = s->dims;
+    p->nb1 = (int)nb1;
     p->nb = (int)nb;
-    p->Kt = s->in * nb;
+    p->Kt = units * nb;
     p->lo = s->lo;
     p->hi = s->hi;
     p->inv_h = (float)((double)s->G / ((double)s->hi - (double)s->lo));
@@ -125,7 +137,8 @@ kan_status choose(const Problem& p, bool backward, bool* use_tc)
         return KAN_OK;
     }
     // automatic: the tensor-core kernels for every shape whose strides TMA can
-    // address; the CUDA-core kernels only for the others
+    // address; the CUDA-core kernels only for the others (1-D layers)
+    if (!ok && p.dims == 2) return fail(KAN_ERR_UNSUPPORTED, "2-D surfaces: tensor-core path not possible: %s", why);
     *use_tc = ok;
     return KAN_OK;
 }

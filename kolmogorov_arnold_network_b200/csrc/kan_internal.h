@@ -18,8 +18,11 @@ struct Problem {
     int64_t batch, in, out;
     int G;
     int k;           // spline degree (1..5)
-    int nb;          // G + k basis functions per edge
-    int64_t Kt;      // in * nb (spline columns of the dense expansion)
+    int dims;        // 1: univariate; 2: tensor-product surfaces over consecutive input pairs
+    int nb1;         // G + k univariate basis functions
+    int nb;          // columns of the dense expansion per unit: nb1 (1-D) or nb1^2 (2-D, one unit = one pair)
+    int64_t x_ld;    // row length of x and dx (the layer's input count)
+    int64_t Kt;      // in * nb (spline columns of the dense expansion); `in` counts units (pairs for 2-D)
     float lo, hi, inv_h;
     int dtype;       // KAN_F32 / KAN_BF16
     bool base;

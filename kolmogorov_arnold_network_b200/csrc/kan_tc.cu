@@ -152,6 +152,9 @@ struct TcArgs {
     int G, nb;                 // nb: columns per input (G+k, or G+k+1 with an interleaved SiLU column)
     int nbs;                   // spline functions per input (G+k)
     int k;                     // spline degree
+    int nb1;                   // univariate basis functions (G+k); 2-D: nb = nbs = nb1^2
+    int64_t x_ld;              // row length of x and dx (2 * in for 2-D surfaces, whose units are input pairs)
+    int twod;                  // 1: 2-D surfaces
     int ext;                   // 1: input i's SiLU column is column nbs of its group
     float lo, inv_h;
     int Kt;                    // in * nb
@@ -281,6 +284,30 @@ __device__ __forceinline__ void scatter_win(uint32_t rb_hi, uint32_t rb_lo, uint
     }
 }
 
+// The 16 products w1[r1] w2[r2] of one input pair's surface, whose B_{0,0}
+// sits at column `base` of a 128-byte swizzled row: entry (r1, r2) goes to
+// column base + (s1+r1) nb1 + s2 + r2 when both basis indices lie in 0..nb1-1
+// and the column in [0, width).  Four runs of four consecutive columns, one
+// scatter_win each; an empty range stores nothing.
+template <int DT>
+__device__ __forceinline__ void scatter_surface(uint32_t rb_hi, uint32_t rb_lo, uint32_t rx, int base, int s1, int s2,
+                                                int nb1, int width, bool ok, const float (&w1)[4],
+                                                const float (&w2)[4])
+{
+#pragma unroll
+    for (int r1 = 0; r1 < 4; ++r1) {
+        const int m1 = s1 + r1;
+        const bool v = ok && m1 >= 0 && m1 < nb1;
+        const int b1 = base + m1 * nb1;
+        const int mlo = v ? max(0, -b1) : 0;
+        const int mhi = v ? max(mlo, min(nb1, width - b1)) : 0;
+        float wr[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) wr[q] = w1[r1] * w2[q];
+        scatter_win<DT, 4>(rb_hi, rb_lo, rx, b1, s2, mlo, mhi, wr, 3);
+    }
+}
+
 // Zero one 128-byte row of a produced tile (and of its lo copy for fp32).
 // Store c writes 16-byte chunk c ^ rx (rx = row & 7), so the 8 consecutive
 // rows of a quarter-warp hit 8 different chunks: no bank conflicts.
@@ -405,7 +432,9 @@ __device__ __forceinline__ void weights_fma(float t, float (&w)[4])
 // (rank 0) issues the MMAs; the follower's B loads complete on the leader's
 // barriers and its producers arrive there remotely; commits reach both CTAs.
 // KD: 3 for cubic splines (closed-form weights, 4 per input), 0 for any
-// other degree (the runtime degree a.k; weights by the local triangle).
+// other degree (the runtime degree a.k; weights by the local triangle), 32
+// for cubic 2-D surfaces (a unit is an input pair with nb1^2 columns; MAXI
+// then counts x values, two per unit).
 template <int MODE, int DT, int MAXI, bool PAIR = false, int KD = 3>
 __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap tA_hi, const __grid_constant__ CUtensorMap tA_lo,
@@ -419,6 +448,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     constexpr int EPB = 128 / C::ESZ;               // elements per 128-byte row
     constexpr bool F32 = DT == KAN_F32;
     constexpr bool PRODUCE = MODE == FWD || MODE == DCA;
+    constexpr bool TWOD = KD == 32;
+    static_assert(!TWOD || PRODUCE, "2-D surfaces: produced-A kernels only");
     constexpr bool A_BY_TMA = MODE == DX || MODE == GEMM;
     static_assert(!PAIR || (PRODUCE && DT == KAN_BF16), "CTA pairs: bf16 forward and dcoef only");
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -712,7 +743,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 const int grp = p >> 7;                // warp-uniform
                 const int64_t b = m0 + row;
                 const bool row_ok = b < a.batch;
-                const T* xrow = X + (row_ok ? b : 0) * a.in;
+                const T* xrow = X + (row_ok ? b : 0) * a.x_ld;
                 const float u0 = -a.lo * a.inv_h;      // u = x * inv_h + u0
                 const float u_lo = -(float)a.k, u_hi = (float)(a.G + a.k);
                 auto first_input = [&](int kb) { return (int)__umulhi((uint32_t)(kb * BK), a.nb_magic); };
@@ -729,7 +760,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 auto fetch = [&](int kb) {
                     if (kb >= a.nkb_main || !row_ok) return;
                     const int i0 = first_input(kb);
-                    nxw.issue(xrow, i0, last_input(kb) - i0 + 1, (int)a.in, a.x_vec != 0);
+                    // (2-D: a unit's two x values; MAXI counts values)
+                    if constexpr (TWOD) nxw.issue(xrow, 2 * i0, 2 * (last_input(kb) - i0 + 1), (int)a.x_ld, a.x_vec != 0);
+                    else nxw.issue(xrow, i0, last_input(kb) - i0 + 1, (int)a.in, a.x_vec != 0);
                 };
                 // At most sa_n groups: then a group's previous k-block is no older
                 // than the previous use of the A slot it waits for, so neither the
@@ -754,6 +787,25 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         if (row_ok) {
                             const int i0 = first_input(kb), n = last_input(kb) - i0 + 1;
                             const int cbase = i0 * a.nb - kb * BK;   // column of input i0's B_0 in this block
+                            if constexpr (TWOD) {
+                                // surfaces: MAXI / 2 pair slots, 16 products each
+#pragma unroll
+                                for (int k = 0; k < MAXI / 2; ++k) {
+                                    const int base = cbase + k * a.nb;
+                                    float uu = fmaf(cur[2 * k], a.inv_h, u0), uv = fmaf(cur[2 * k + 1], a.inv_h, u0);
+                                    const bool ok = k < n && uu >= u_lo && uu < u_hi && uv >= u_lo && uv < u_hi;
+                                    uu = ok ? uu : 0.0f;
+                                    uv = ok ? uv : 0.0f;
+                                    int s1, s2;
+                                    float f1, f2, w1[4], w2[4];
+                                    floor_split(uu, s1, f1);
+                                    floor_split(uv, s2, f2);
+                                    weights_fma(uu - f1, w1);
+                                    weights_fma(uv - f2, w2);
+                                    scatter_surface<DT>(ahi + rbase, alo + rbase, rx, base, s1, s2, a.nb1, BK, ok, w1,
+                                                        w2);
+                                }
+                            } else {
                             // Straight-line over the MAXI input slots (the slots past n
                             // store nothing), so the inputs' arithmetic can interleave.
 #pragma unroll
@@ -785,6 +837,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                                     scatter_win<DT, KAN_MAX_NW>(ahi + rbase, alo + rbase, rx, base, sidx, mlo, mhi, w,
                                                                 a.k);
                                 }
+                            }
                             }
                         }
                     } else {
@@ -845,7 +898,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 auto fetch = [&](int kb) {
                     const int64_t b = (int64_t)kb * BK + rb;
                     if (silu_tile || b >= a.batch) return;
-                    nxw.issue(X + b * a.in, i_first, n_inp, (int)a.in, a.x_vec != 0);
+                    if constexpr (TWOD) nxw.issue(X + b * a.x_ld, 2 * i_first, 2 * n_inp, (int)a.x_ld, a.x_vec != 0);
+                    else nxw.issue(X + b * a.in, i_first, n_inp, (int)a.in, a.x_vec != 0);
                 };
                 // byte offset of column c (0..EPB-1) inside this thread's atom row
                 auto col_off = [&](int c) -> uint32_t {
@@ -868,7 +922,47 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     if (!silu_tile) {
                         // this thread's atom row starts from zeros (rows past the batch stay zero)
                         zero_row<DT>(rb_hi, rb_lo, (uint32_t)rb & 7u);
-                        if (row_ok) {
+                        if (row_ok && TWOD) {
+                            const int cbase = i_first * a.nb - c_lo;
+                            // surfaces: MAXI / 2 pair slots, 16 products each, in four runs of four columns
+#pragma unroll
+                            for (int k = 0; k < MAXI / 2; ++k) {
+                                const int base = cbase + k * a.nb;
+                                float uu = fmaf(cur[2 * k], a.inv_h, u0), uv = fmaf(cur[2 * k + 1], a.inv_h, u0);
+                                const bool ok = k < n_inp && uu >= u_lo && uu < u_hi && uv >= u_lo && uv < u_hi;
+                                uu = ok ? uu : 0.0f;
+                                uv = ok ? uv : 0.0f;
+                                int s1, s2;
+                                float f1, f2, w1[4], w2[4];
+                                floor_split(uu, s1, f1);
+                                floor_split(uv, s2, f2);
+                                weights_fma(uu - f1, w1);
+                                weights_fma(uv - f2, w2);
+#pragma unroll
+                                for (int r1 = 0; r1 < 4; ++r1) {
+                                    const int m1 = s1 + r1;
+                                    const bool v = ok && m1 >= 0 && m1 < a.nb1;
+                                    const int b1 = base + m1 * a.nb1;
+                                    const int mlo = v ? max(0, -b1) : 0;
+                                    const uint32_t width = v ? (uint32_t)(max(mlo, min(a.nb1, EPB - b1)) - mlo) : 0u;
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) {
+                                        if ((uint32_t)(s2 + q - mlo) < width) {
+                                            const uint32_t off = col_off(b1 + s2 + q);
+                                            const float wv = w1[r1] * w2[q];
+                                            if constexpr (F32) {
+                                                uint16_t h, l;
+                                                split_f16(wv, h, l);
+                                                st_shared_u16(rb_hi + off, h);
+                                                st_shared_u16(rb_lo + off, l);
+                                            } else {
+                                                st_shared_u16(rb_hi + off, __bfloat16_as_ushort(__float2bfloat16_rn(wv)));
+                                            }
+                                        }
+                                    }
+                                }
+                            }
+                        } else if (row_ok) {
                             const int cbase = i_first * a.nb - c_lo;
                             // straight-line over the MAXI input slots (see the forward producer)
 #pragma unroll
@@ -1246,6 +1340,8 @@ struct DxArgs {
     int G, nb;                // nb: columns per input of B (G+k, or G+k+1 with the SiLU column)
     int nbs;                  // spline functions per input (G+k)
     int k;                    // spline degree
+    int nb1;                  // univariate basis functions (G+k); 2-D: nb = nbs = nb1^2
+    int64_t x_ld;             // row length of x and dx
     int ext;                  // 1: column nbs of each input group is its dY.w_base column
     float lo, inv_h;
     int BN, stages, nkb;      // nkb: k-blocks over out
@@ -1268,6 +1364,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     constexpr int BK = C::BK;
     constexpr int EPB = 128 / C::ESZ;
     constexpr bool F32 = DT == KAN_F32;
+    constexpr bool TWOD = KD == 32;      // units are input pairs with nb1^2 columns (cubic surfaces)
     constexpr bool B_MN = true;          // coef (its fp16 hi/lo copies for fp32) MN-major
     static_assert(!PAIR || DT == KAN_BF16, "CTA pairs: bf16 only");
     extern __shared__ uint8_t smem_raw[];
@@ -1543,7 +1640,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                 if (a.gb) gw.issue(a.gb + bq * a.in, i_start, n, (int)a.in, g_vec);
             }
         };
-        if (my_tiles > 0) {
+        if (!TWOD && my_tiles > 0) {
             int64_t m0, b;
             int i0, ia, ib;
             tile_part(0, m0, i0, b, ia, ib);
@@ -1626,6 +1723,49 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             }
             // both halves of the row are staged
             named_bar_sync(1 + q, 64);
+            if constexpr (TWOD) {
+                // surfaces: for each pair (u, v) of this warp's units, the 16 staged columns
+                // times B'(u) B(v) and B(u) B'(v); the pair's two dx values go out together
+                if (b_ok) {
+                    const T* xr = reinterpret_cast<const T*>(a.x) + b * a.x_ld;
+                    T* dxr2 = reinterpret_cast<T*>(a.dx) + b * a.x_ld;
+                    for (int i = ia; i < ib; ++i) {
+                        const float xu = to_f(xr[2 * i]), xv = to_f(xr[2 * i + 1]);
+                        const Span su = span_of(xu, a.lo, a.inv_h, a.G, 3), sv = span_of(xv, a.lo, a.inv_h, a.G, 3);
+                        float du = 0.0f, dv = 0.0f;
+                        if (su.valid && sv.valid) {
+                            float wu[4], wv[4], gu[4], gv[4];
+                            weights(su.t, wu);
+                            weights(sv.t, wv);
+                            dweights(su.t, a.inv_h, gu);
+                            dweights(sv.t, a.inv_h, gv);
+                            const int cb = i * a.nb - kt_al;
+#pragma unroll
+                            for (int r1 = 0; r1 < 4; ++r1) {
+                                const int m1 = su.s + r1;
+                                if (m1 < 0 || m1 >= a.nb1) continue;
+#pragma unroll
+                                for (int r2 = 0; r2 < 4; ++r2) {
+                                    const int m2 = sv.s + r2;
+                                    if (m2 < 0 || m2 >= a.nb1) continue;
+                                    const float g = to_f(srow[cb + m1 * a.nb1 + m2]);
+                                    du = fmaf(g, gu[r1] * wv[r2], du);
+                                    dv = fmaf(g, wu[r1] * gv[r2], dv);
+                                }
+                            }
+                            du *= inv_dc;
+                            dv *= inv_dc;
+                        }
+                        if constexpr (F32) {
+                            *reinterpret_cast<float2*>(dxr2 + 2 * i) = make_float2(du, dv);
+                        } else {
+                            *reinterpret_cast<uint32_t*>(dxr2 + 2 * i) = pack_bf16(du, dv);
+                        }
+                    }
+                }
+                __syncwarp();
+                continue;
+            }
             // dx of this warp's inputs [ia, ib): each lane computes its row's values
             // and parks them in slots slot_base + 0.. of its own staging row, which
             // lie below every column still to be read (input ia + k reads columns at
@@ -2227,8 +2367,9 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
     return cudaGetLastError();
 }
 
-// Inputs a row of one forward k-block can touch: (BK - 1) / nb + 2.
-int fwd_maxi_needed(int nb, bool f32) { return (64 - 1) / nb + 2; (void)f32; }
+// x values a row of one produced k-block can touch: (BK - 1) / nb + 2 units,
+// one x value each (two for the input pairs of 2-D surfaces).
+int fwd_maxi_needed(int nb, bool twod) { return ((64 - 1) / nb + 2) * (twod ? 2 : 1); }
 
 template <int MODE, int MAXI, int KD>
 cudaError_t launch_m(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
@@ -2246,7 +2387,7 @@ cudaError_t launch_k(bool f32, dim3 grid, int BN, int stages, const CUtensorMap*
                      cudaStream_t st)
 {
     if constexpr (MODE == FWD || MODE == DCA) {
-        const int need = fwd_maxi_needed(args.nb, f32);
+        const int need = fwd_maxi_needed(args.nb, KD == 32);
         if (need <= 4) return launch_m<MODE, 4, KD>(f32, grid, BN, stages, maps, args, st);
         if (need <= 7) return launch_m<MODE, 7, KD>(f32, grid, BN, stages, maps, args, st);
         if (need <= 9) return launch_m<MODE, 9, KD>(f32, grid, BN, stages, maps, args, st);
@@ -2263,6 +2404,10 @@ template <int MODE>
 cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
                       cudaStream_t st)
 {
+    if (args.twod) {   // 2-D surfaces: produced-A kernels only (dx runs persistent)
+        if constexpr (MODE == FWD || MODE == DCA) return launch_k<MODE, 32>(f32, grid, BN, stages, maps, args, st);
+        return cudaErrorInvalidConfiguration;
+    }
     if (MODE == GEMM || args.k == 3) return launch_k<MODE, 3>(f32, grid, BN, stages, maps, args, st);
     if constexpr (MODE != GEMM) return launch_k<MODE, 0>(f32, grid, BN, stages, maps, args, st);
     return cudaErrorInvalidConfiguration;
@@ -2315,6 +2460,9 @@ TcArgs base_args(const Problem& p, const Plan& P)
     a.out_f = p.out;
     a.G = p.G;
     a.k = p.k;
+    a.nb1 = p.nb1;
+    a.x_ld = p.x_ld;
+    a.twod = p.dims == 2;
     a.nb = P.nbx;
     a.nbs = p.nb;
     a.ext = P.ext;
@@ -2322,7 +2470,7 @@ TcArgs base_args(const Problem& p, const Plan& P)
     a.inv_h = p.inv_h;
     a.Kt = (int)P.Kx;
     a.has_base = p.base;
-    a.x_vec = (p.in * (p.dtype == KAN_F32 ? 4 : 2)) % 16 == 0;
+    a.x_vec = (p.x_ld * (p.dtype == KAN_F32 ? 4 : 2)) % 16 == 0;
     a.nb_magic = (uint32_t)((((uint64_t)1 << 32) + (uint64_t)P.nbx - 1) / (uint64_t)P.nbx);
     return a;
 }
@@ -2411,6 +2559,11 @@ bool tc_supported(const Problem& p, bool backward, const char** why)
         *why = "fewer than 4 basis functions per input (G + degree < 4): too many inputs per k-block row";
         return false;
     }
+    if (p.dims == 2 && f32 && p.out > 1024) {
+        *why = "2-D surfaces in fp32 with more than 1024 outputs (the persistent dx kernel's limit)";
+        return false;
+    }
+
     if (nbx > 121 && (f32 || nbx > 249)) {
         *why = "G too large for one dx tile (the input's columns must fit the tile with its alignment offset)";
         return false;
@@ -2609,6 +2762,8 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             d.out = p.out;
             d.G = p.G;
             d.k = p.k;
+            d.nb1 = p.nb1;
+            d.x_ld = p.x_ld;
             d.nb = P.nbx;
             d.nbs = p.nb;
             d.ext = P.ext ? 1 : 0;
@@ -2623,7 +2778,11 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
             d.ld_stage = P.p_ld;
             d.a_res = P.p_ares ? 1 : 0;
             d.pair = P.p_pair ? 1 : 0;
-            if (p.k == 3)
+            if (p.dims == 2)
+                e = f32 ? launch_dx_persistent<KAN_F32, false, 32>(P, maps, d, st)
+                        : (P.p_pair ? launch_dx_persistent<KAN_BF16, true, 32>(P, maps, d, st)
+                                    : launch_dx_persistent<KAN_BF16, false, 32>(P, maps, d, st));
+            else if (p.k == 3)
                 e = f32 ? launch_dx_persistent<KAN_F32, false, 3>(P, maps, d, st)
                         : (P.p_pair ? launch_dx_persistent<KAN_BF16, true, 3>(P, maps, d, st)
                                     : launch_dx_persistent<KAN_BF16, false, 3>(P, maps, d, st));
@@ -2633,6 +2792,7 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
                                     : launch_dx_persistent<KAN_BF16, false, 0>(P, maps, d, st));
             if (e != cudaSuccess) return e;
         } else {
+            if (p.dims == 2) return cudaErrorInvalidConfiguration;   // (tc_supported rules it out)
             TcArgs a = base_args(p, P);
             a.x = x;
             a.amax = amax;

@@ -37,9 +37,14 @@ def _check(t, name, dtype=None, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def shape_of(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, degree=3) -> N.kan_shape:
+def shape_of(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, degree=3, dims=1) -> N.kan_shape:
     batch, n_in = x.shape
-    return N.make_shape(batch, n_in, coef.shape[0], G, lo, hi, _code(x), w_base is not None, path, degree)
+    return N.make_shape(batch, n_in, coef.shape[0], G, lo, hi, _code(x), w_base is not None, path, degree, dims)
+
+
+def _coef_shape(n_out, n_in, G, degree, dims):
+    nb = G + degree
+    return (n_out, n_in, nb) if dims == 1 else (n_out, n_in // 2, nb, nb)
 
 
 def _stream(t):
@@ -56,14 +61,15 @@ def workspace(shape: N.kan_shape, for_backward: bool, device) -> torch.Tensor | 
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
-def forward(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, y=None, ws=None, degree=3):
-    """y[b,j] = sum_i sum_m coef[j,i,m] B_m(x[b,i]) (+ sum_i w_base[j,i] silu(x[b,i])), degree-k B-splines."""
+def forward(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, y=None, ws=None, degree=3, dims=1):
+    """y[b,j] = sum_i sum_m coef[j,i,m] B_m(x[b,i]) (+ sum_i w_base[j,i] silu(x[b,i])), degree-k B-splines;
+    dims=2: sum_p sum_{m1,m2} coef[j,p,m1,m2] B_m1(x[b,2p]) B_m2(x[b,2p+1]) (tensor-product surfaces)."""
     batch, n_in = x.shape
     n_out = coef.shape[0]
     _check(x, "x", None)
-    _check(coef, "coef", x.dtype, (n_out, n_in, G + degree))
+    _check(coef, "coef", x.dtype, _coef_shape(n_out, n_in, G, degree, dims))
     _check(w_base, "w_base", x.dtype, (n_out, n_in))
-    s = shape_of(x, coef, G, lo, hi, w_base, path, degree)
+    s = shape_of(x, coef, G, lo, hi, w_base, path, degree, dims)
     if y is None:
         y = torch.empty((batch, n_out), dtype=x.dtype, device=x.device)
     _check(y, "y", x.dtype, (batch, n_out))
@@ -76,15 +82,15 @@ def forward(x, coef, G, lo, hi, w_base=None, path=N.KAN_PATH_AUTO, y=None, ws=No
 
 
 def backward(x, coef, dY, G, lo, hi, w_base=None, need_dx=True, need_dcoef=True, need_dw_base=True,
-             path=N.KAN_PATH_AUTO, out=None, ws=None, degree=3):
+             path=N.KAN_PATH_AUTO, out=None, ws=None, degree=3, dims=1):
     """(dx, dcoef, dw_base) of the layer for upstream gradient dY; dcoef/dw_base are float32."""
     batch, n_in = x.shape
     n_out = coef.shape[0]
     _check(x, "x", None)
-    _check(coef, "coef", x.dtype, (n_out, n_in, G + degree))
+    _check(coef, "coef", x.dtype, _coef_shape(n_out, n_in, G, degree, dims))
     _check(w_base, "w_base", x.dtype, (n_out, n_in))
     _check(dY, "dY", x.dtype, (batch, n_out))
-    s = shape_of(x, coef, G, lo, hi, w_base, path, degree)
+    s = shape_of(x, coef, G, lo, hi, w_base, path, degree, dims)
     if out is not None:
         dx, dcoef, dwb = out
     else:
@@ -233,6 +239,44 @@ class GRKAN(torch.nn.Module):
         lead = x.shape[:-1]
         y = _GRKANFunction.apply(x.reshape(-1, self.channels), self.a, self.b, self.groups)
         return y.reshape(*lead, self.channels)
+
+
+class _KAN2DFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, coef, G, lo, hi):
+        x = x.contiguous()
+        ctx.save_for_backward(x, coef)
+        ctx.grid = (G, lo, hi)
+        return forward(x, coef, G, lo, hi, dims=2)
+
+    @staticmethod
+    def backward(ctx, dY):
+        x, coef = ctx.saved_tensors
+        G, lo, hi = ctx.grid
+        dx, dcoef, _ = backward(x, coef, dY.contiguous().to(x.dtype), G, lo, hi, need_dx=ctx.needs_input_grad[0],
+                                need_dcoef=ctx.needs_input_grad[1], dims=2)
+        return dx, None if dcoef is None else dcoef.to(coef.dtype), None, None, None
+
+
+class KANLayer2D(torch.nn.Module):
+    """Layer of cubic tensor-product B-spline surfaces over consecutive input pairs:
+    ``coef`` [out, in/2, G+3, G+3]; ``in_features`` must be even."""
+
+    def __init__(self, in_features, out_features, G=8, lo=-1.0, hi=1.0, coef_std=0.1, dtype=torch.float32,
+                 device=None):
+        super().__init__()
+        if in_features % 2:
+            raise ValueError("in_features must be even (inputs are taken in pairs)")
+        self.in_features, self.out_features = in_features, out_features
+        self.G, self.lo, self.hi = int(G), float(lo), float(hi)
+        self.coef = torch.nn.Parameter(
+            torch.randn(out_features, in_features // 2, G + 3, G + 3, dtype=torch.float32, device=device)
+            .mul_(coef_std).to(dtype))
+
+    def forward(self, x):
+        lead = x.shape[:-1]
+        y = _KAN2DFunction.apply(x.reshape(-1, self.in_features), self.coef, self.G, self.lo, self.hi)
+        return y.reshape(*lead, self.out_features)
 
 
 class KANNetwork(torch.nn.Module):

@@ -28,11 +28,22 @@ class Layer:
     hi: float
     base: bool = False
     degree: int = 3
+    dims: int = 1                # 2: tensor-product surfaces over consecutive input pairs
 
     @property
     def nb(self) -> int:
-        """Basis functions per edge: G + degree."""
+        """Basis functions per coordinate: G + degree."""
         return self.G + self.degree
+
+    @property
+    def units(self) -> int:
+        """Edge functions per output: inputs (1-D) or input pairs (2-D)."""
+        return self.inp if self.dims == 1 else self.inp // 2
+
+    @property
+    def cols(self) -> int:
+        """Columns of the dense basis expansion per unit: nb (1-D) or nb^2 (2-D)."""
+        return self.nb if self.dims == 1 else self.nb * self.nb
 
 
 @dataclass(frozen=True)
@@ -54,8 +65,9 @@ class Workload:
 
     @property
     def edges(self) -> int:
-        """Edge evaluations per step: batch * in * out summed over layers."""
-        return sum(self.batch * L.inp * L.out for L in self.layers)
+        """Edge evaluations per step: batch * in * out summed over layers (a 2-D surface edge takes an
+        input pair: batch * in/2 * out)."""
+        return sum(self.batch * L.units * L.out for L in self.layers)
 
 
 def _grid_sweep():
@@ -78,6 +90,15 @@ def _degree_sweep():
     return out
 
 
+def _surfaces():
+    out = {}
+    for dt, batch in (("bf16", 65536), ("f32", 16384)):
+        nm = f"surface512_g8_{dt}_fwdbwd"
+        out[nm] = Workload(nm, 8, batch, (Layer(512, 512, 8, -1.0, 1.0, dims=2),), dt, ("uniform", -1.0, 1.0), 0.1,
+                           note=f"2-D tensor-product surfaces: 512 inputs in 256 pairs -> 512, batch {batch}, G=8")
+    return out
+
+
 WORKLOADS = {
     "layer8x4": Workload("layer8x4", 1, 32, (Layer(8, 4, 8, -1.0, 1.0),), "f32", ("uniform", -1.0, 1.0), 0.1,
                          note="KANLayer(8,4) on a [32,8] batch, G=8 on [-1,1]"),
@@ -92,6 +113,7 @@ WORKLOADS = {
                                  (Layer(768, 3072, 5, -3.0, 3.0), Layer(3072, 768, 5, -3.0, 3.0)), "bf16",
                                  ("normal", 1.0), 0.05, note="KAN FFN block 768->3072->768, 8192 tokens"),
     **_degree_sweep(),
+    **_surfaces(),
 }
 
 #: the workload the benchmark times by default: the largest single-GPU one by edge evaluations per step
@@ -154,7 +176,8 @@ def draw_x(w: Workload, rows: int | None = None) -> torch.Tensor:
 def draw_coef(w: Workload, layer: int = 0) -> torch.Tensor:
     L = w.layers[layer]
     g = _gen(w.family, 1 if layer == 0 else 4)
-    c = torch.randn((L.out, L.inp, L.nb), generator=g, dtype=torch.float32) * w.coef_std
+    shape = (L.out, L.inp, L.nb) if L.dims == 1 else (L.out, L.inp // 2, L.nb, L.nb)
+    c = torch.randn(shape, generator=g, dtype=torch.float32) * w.coef_std
     return c.to(w.torch_dtype)
 
 
@@ -198,11 +221,12 @@ def custom_grkan(rows, channels, groups, m=5, n=4, dtype="f32", family=91):
                       dtype)
 
 
-def custom(batch, inp, out, G, lo, hi, dtype="f32", base=False, x_range=None, coef_std=0.1, family=90, degree=3):
+def custom(batch, inp, out, G, lo, hi, dtype="f32", base=False, x_range=None, coef_std=0.1, family=90, degree=3,
+           dims=1):
     """An ad-hoc single-layer workload (tests of ragged and edge shapes)."""
     h = (hi - lo) / G
     # reach into the extended intervals (and, for degrees other than 3, a little beyond them)
     ext = 2.0 if degree == 3 else degree - 0.5
     xr = x_range or (lo - ext * h, hi + ext * h)
-    return Workload(f"custom_{batch}x{inp}x{out}_g{G}_k{degree}_{dtype}", family, batch,
-                    (Layer(inp, out, G, lo, hi, base, degree),), dtype, ("uniform", xr[0], xr[1]), coef_std)
+    return Workload(f"custom_{batch}x{inp}x{out}_g{G}_k{degree}_d{dims}_{dtype}", family, batch,
+                    (Layer(inp, out, G, lo, hi, base, degree, dims),), dtype, ("uniform", xr[0], xr[1]), coef_std)
