@@ -283,9 +283,9 @@ def time_steps(R: Runner, K: int, warmup: int, flush, barrier=lambda: None):
     st = N.kan_sync_status(None)
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {N.STATUS.get(st, st)}")
-    # per call: start, after_prep, after_dcoef (backward only), end
-    evs = [[dict(start=_ev(), prep=_ev(), mid=_ev() if kind == "bwd" else None, end=_ev())
-            for _, kind, _ in calls] for _ in range(K)]
+    # per call: start, after_prep (layer calls), after_dcoef (backward only), end
+    evs = [[dict(start=_ev(), prep=_ev() if kind in ("fwd", "bwd") else None, mid=_ev() if kind == "bwd" else None,
+                 end=_ev()) for _, kind, _ in calls] for _ in range(K)]
     step_ev = [(_ev(), _ev()) for _ in range(K)]
     # torch creates an event's CUDA handle at its first record: record every mark event once now, so that
     # the handles passed to the library exist
@@ -302,7 +302,10 @@ def time_steps(R: Runner, K: int, warmup: int, flush, barrier=lambda: None):
         step_ev[k][0].record(stream)
         for e, (_, kind, c) in zip(evs[k], calls):
             e["start"].record(stream)
-            c((e["prep"].cuda_event, None if e["mid"] is None else e["mid"].cuda_event))
+            if e["prep"] is None:
+                c()
+            else:
+                c((e["prep"].cuda_event, None if e["mid"] is None else e["mid"].cuda_event))
             e["end"].record(stream)
         step_ev[k][1].record(stream)
     torch.cuda.synchronize(R.dev)
@@ -312,6 +315,9 @@ def time_steps(R: Runner, K: int, warmup: int, flush, barrier=lambda: None):
     seg = {}
     for k in range(K):
         for e, (nm, kind, _) in zip(evs[k], calls):
+            if kind not in ("fwd", "bwd"):
+                seg[nm] = seg.get(nm, 0.0) + e["start"].elapsed_time(e["end"])
+                continue
             li = nm[3:]
             parts = [(f"prep{li}", e["start"], e["prep"])]
             if kind == "fwd":
@@ -364,7 +370,7 @@ def roofline_of(w: W.Workload, seg: dict, K: int, pk: dict, ffma_tflops: float):
     bf16: dense-expanded FLOPs of the GEMM at the measured bf16 tensor peak.  fp32: the fp32 bound of
     the method's measurement plan, algorithmic FLOPs (4 FMAs per edge, +1 with SiLU) at the measured
     fp32 FMA peak; the dense-expanded fraction at the fp16 tensor peak is reported beside it."""
-    gemm = {k: v for k, v in seg.items() if not k.startswith("prep")}
+    gemm = {k: v for k, v in seg.items() if k.rstrip("0123456789") in ("fwd", "dcoef", "dx")}
     dom = max(gemm, key=gemm.get)
     kind, li = dom.rstrip("0123456789"), int(dom[len(dom.rstrip("0123456789")):])
     L = w.layers[li]
@@ -560,6 +566,64 @@ def config_of(w: W.Workload):
     return c
 
 
+class UkRunner(Runner):
+    """A UKAN layer step: the generator's window, the layer's forward and backward on it, and the
+    generator's backward.  The window (the groups the fixed synthetic batch reaches) is sized once, before
+    the timed steps, from the inputs' device-side range."""
+
+    def __init__(self, w: W.UkWorkload, dev):
+        from kolmogorov_arnold_network_b200 import _native as N
+        from kolmogorov_arnold_network_b200 import layer as LY
+        self.N, self.LY, self.uk, self.dev = N, LY, w, dev
+        d = W.draw_ukan(w)
+        self.host = d
+        self.x, self.dY = d["x"].to(dev), d["dY"].to(dev)
+        self.W1, self.b1, self.W2, self.b2 = (d[k].to(dev) for k in ("W1", "b1", "W2", "b2"))
+        self.q0, self.nq = LY.ukan_window(self.x, w.h, w.group)
+        self.us = LY.ukan_shape(w.inp, w.out, w.group, self.W1, self.q0, self.nq, w.torch_dtype)
+        self.ks = N.kan_ukan_layer_shape(self.us, w.batch, w.h)
+        self.coef = torch.empty((w.out, w.inp, self.nq * w.group), dtype=w.torch_dtype, device=dev)
+        self.pre = torch.empty((self.nq, w.hidden), dtype=torch.float32, device=dev)
+        self.y = torch.empty((w.batch, w.out), dtype=w.torch_dtype, device=dev)
+        self.dx = torch.empty_like(self.x)
+        self.dcoef = torch.empty(self.coef.shape, dtype=torch.float32, device=dev)
+        self.g = [torch.empty_like(t) for t in (self.W1, self.b1, self.W2, self.b2)]
+        self.ws_f = LY.workspace(self.ks, False, dev)
+        self.ws_b = LY.workspace(self.ks, True, dev)
+        self.ws_g = torch.empty(max(16, N.kan_ukan_workspace_size(self.us)), dtype=torch.uint8, device=dev)
+        self.w = W.Workload(w.name, w.family, w.batch, (W.Layer(w.inp, w.out, self.ks.G, self.ks.lo, self.ks.hi),),
+                            w.dtype, ("normal", w.x_std), 0.0, note=w.note)
+
+    def calls(self):
+        N, P = self.N, lambda t: None if t is None else t.data_ptr()
+        st = torch.cuda.current_stream(self.dev).cuda_stream
+        ks, us = self.ks, self.us
+
+        def gen():
+            N.kan_ukan_generate(us, P(self.W1), P(self.b1), P(self.W2), P(self.b2), P(self.coef), P(self.pre), st)
+
+        def fwd(marks=None):
+            if marks is not None:
+                N.kan_set_timing_marks(marks[0], None)
+            N.kan_forward(ks, P(self.x), P(self.coef), None, P(self.y), P(self.ws_f),
+                          0 if self.ws_f is None else self.ws_f.numel(), st)
+            if marks is not None:
+                N.kan_set_timing_marks(None, None)
+
+        def bwd(marks=None):
+            if marks is not None:
+                N.kan_set_timing_marks(marks[0], marks[1])
+            N.kan_backward(ks, P(self.x), P(self.coef), None, P(self.dY), P(self.dx), P(self.dcoef), None,
+                           P(self.ws_b), 0 if self.ws_b is None else self.ws_b.numel(), st)
+            if marks is not None:
+                N.kan_set_timing_marks(None, None)
+
+        def gen_bwd():
+            N.kan_ukan_generate_backward(us, P(self.W1), P(self.W2), P(self.pre), P(self.dcoef), *(P(t) for t in self.g),
+                                         P(self.ws_g), self.ws_g.numel(), st)
+        return [("gen0", "gen", gen), ("fwd0", "fwd", fwd), ("bwd0", "bwd", bwd), ("genbwd0", "gen", gen_bwd)]
+
+
 class GrRunner:
     """Buffers and the two C-ABI calls of one GR-KAN workload: the forward (y) and one backward that
     returns dx, da and db."""
@@ -716,6 +780,20 @@ def run_ours(args, world, rank, local):
             torch.cuda.empty_cache()
         for nm, wg in W.GR_WORKLOADS.items():
             others[nm] = time_grkan(wg, dev, min(K, args.extra_steps), flush, pk)
+        for nm, wu in W.UK_WORKLOADS.items():
+            Ru = UkRunner(wu, dev)
+            ku = min(K, args.extra_steps)
+            tu, segu, _ = time_steps(Ru, ku, 3, flush)
+            msu = tu / ku
+            ru = roofline_of(Ru.w, segu, ku, pk, ffma)
+            others[nm] = {"ms_per_step": msu, "value": wu.edges / (msu / 1000.0), "unit": UNIT, "steps": ku,
+                          "dtype": wu.dtype, "dominant": ru["kernel"], "bound": ru["bound"], "frac": ru["frac"],
+                          "segment_ms": ru["segment_ms"], "step_roofline": step_roofline(Ru.w, msu, pk, ffma),
+                          "window": {"q0": Ru.q0, "nq": Ru.nq, "G": Ru.ks.G, "basis_per_input": Ru.nq * wu.group},
+                          "note": "generator window sized once before the timed steps; step = generate + layer "
+                                  "forward + layer backward + generator backward"}
+            del Ru
+            torch.cuda.empty_cache()
 
     st = R_status()
     if st != 0:

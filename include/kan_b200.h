@@ -257,6 +257,69 @@ KAN_API kan_status kan_grkan_backward(const kan_grkan_shape* s, const void* x, c
                                       const void* dY, void* dx, float* da, float* db, void* workspace,
                                       size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * UKAN: KAN layers on an unbounded grid with generated coefficients.
+ *
+ * "Want to train KANS at scale? Now UKAN!" (Abstract): a coefficient-generator
+ * (CG) model produces, on the fly, only the B-spline coefficients required
+ * locally on an unbounded symmetric grid, fed with the positional encoding of
+ * grid groups.  Reading taken here: knots j h for every integer j, cubic
+ * B-splines B_m(x) = N(x/h - m); group q holds the basis indices
+ * q*group .. q*group + group - 1; PE(q)[2l] = sin(q w_l), PE(q)[2l+1] =
+ * cos(q w_l), w_l = 10000^(-2l/pe_dim) (the sinusoidal encoding of the page's
+ * "Attention Is All You Need" reference); the generator is
+ *   hid(q) = silu(W1 PE(q) + b1),  c(q) = W2 hid(q) + b2,
+ *   coef[j, i, m] = c(q)[(j*in + i)*group + (m - q*group)],  q = floor(m / group),
+ * with W1 [hidden, pe_dim], b1 [hidden], W2 [out*in*group, hidden],
+ * b2 [out*in*group], all float32.
+ *
+ * A step: kan_input_range gives the batch's min / max (device), from which
+ * the caller picks the groups q0 .. q0+nq-1 that its inputs reach (basis
+ * floor(x/h) - 3 .. floor(x/h)); kan_ukan_generate writes those groups'
+ * coefficients as the window coef [out, in, nq*group] (operand dtype); the
+ * layer runs through kan_forward / kan_backward with the kan_shape that
+ * kan_ukan_layer_shape returns (G = nq*group - 3, lo = (q0*group + 3) h: the
+ * window's basis 0 is the unbounded basis q0*group; inputs outside the window
+ * see no basis); kan_ukan_generate_backward takes the layer's dcoef back
+ * through the generator.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int64_t in, out;     /* layer inputs and outputs, >= 1 */
+    int32_t group;       /* basis functions per grid group, >= 1 */
+    int32_t pe_dim;      /* encoding width, even, 2..256 */
+    int32_t hidden;      /* generator hidden width, 1..256 */
+    int32_t q0, nq;      /* first group of the window and number of groups (nq*group >= 4, nq*hidden <= 12288) */
+    int32_t dtype;       /* kan_dtype of the generated window (the layer's operand dtype) */
+} kan_ukan_shape;
+
+/* The kan_shape of the layer on the window (host only; h > 0 the knot spacing). */
+KAN_API kan_status kan_ukan_layer_shape(const kan_ukan_shape* s, int64_t batch, float h, kan_shape* out);
+
+/* coef [out, in, nq*group] (operand dtype) from the generator; pre [nq, hidden]
+ * float32 receives the hidden pre-activations W1 PE(q) + b1 (kept for the
+ * backward).  Asynchronous on stream. */
+KAN_API kan_status kan_ukan_generate(const kan_ukan_shape* s, const float* W1, const float* b1, const float* W2,
+                                     const float* b2, void* coef, float* pre, void* stream);
+
+/* Bytes of workspace kan_ukan_generate_backward needs for dW1 / db1. */
+KAN_API kan_status kan_ukan_workspace_size(const kan_ukan_shape* s, size_t* bytes);
+
+/* Gradients of the generator's parameters from the window's dcoef [out, in,
+ * nq*group] float32 (kan_backward's output) and the pre-activations of
+ * kan_ukan_generate: dW2, db2 row by row, dW1, db1 through a fixed-order
+ * reduction (block partials in the workspace, no atomics).  Any output may be
+ * NULL; the workspace is needed only for dW1 / db1.  Outputs overwritten. */
+KAN_API kan_status kan_ukan_generate_backward(const kan_ukan_shape* s, const float* W1, const float* W2,
+                                              const float* pre, const float* dcoef, float* dW1, float* db1,
+                                              float* dW2, float* db2, void* workspace, size_t ws_bytes, void* stream);
+
+/* minmax[0..1] (device float32) = min and max of the n values x (KAN_F32 or
+ * KAN_BF16), through block partials in the workspace (at least 2368 bytes).
+ * Asynchronous on stream.  No counterpart on the pages: it sizes the UKAN
+ * window. */
+KAN_API kan_status kan_input_range(int64_t n, const void* x, int32_t dtype, float* minmax, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
 /* Static description of a status code. */
 KAN_API const char* kan_status_string(kan_status st);
 

@@ -21,6 +21,8 @@ STATUS = {0: "KAN_OK", 1: "KAN_ERR_INVALID_ARG", 2: "KAN_ERR_UNSUPPORTED", 3: "K
 EXPORTS = ("kan_abi_version", "kan_workspace_size", "kan_forward", "kan_backward", "kan_basis", "kan_sync_status",
            "kan_launch_count", "kan_forward_fixed_scratch", "kan_set_timing_marks", "kan_ffma_probe",
            "kan_grkan_workspace_size", "kan_grkan_forward", "kan_grkan_backward",
+           "kan_ukan_layer_shape", "kan_ukan_generate", "kan_ukan_workspace_size", "kan_ukan_generate_backward",
+           "kan_input_range",
            "kan_selftest_wait_timeout", "kan_status_string", "kan_last_error")
 
 
@@ -34,6 +36,12 @@ class kan_shape(ctypes.Structure):
 class kan_grkan_shape(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("channels", ctypes.c_int64), ("groups", ctypes.c_int32),
                 ("num_degree", ctypes.c_int32), ("den_degree", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class kan_ukan_shape(ctypes.Structure):
+    _fields_ = [("in_", ctypes.c_int64), ("out", ctypes.c_int64), ("group", ctypes.c_int32),
+                ("pe_dim", ctypes.c_int32), ("hidden", ctypes.c_int32), ("q0", ctypes.c_int32), ("nq", ctypes.c_int32),
+                ("dtype", ctypes.c_int32)]
 
 
 class KanError(RuntimeError):
@@ -85,6 +93,17 @@ def load(path: str | None = None):
     lib.kan_grkan_forward.argtypes = [gp, _vp, _vp, _vp, _vp, _vp]
     lib.kan_grkan_backward.restype = ctypes.c_int
     lib.kan_grkan_backward.argtypes = [gp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    up = ctypes.POINTER(kan_ukan_shape)
+    lib.kan_ukan_layer_shape.restype = ctypes.c_int
+    lib.kan_ukan_layer_shape.argtypes = [up, ctypes.c_int64, ctypes.c_float, sp]
+    lib.kan_ukan_generate.restype = ctypes.c_int
+    lib.kan_ukan_generate.argtypes = [up, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.kan_ukan_workspace_size.restype = ctypes.c_int
+    lib.kan_ukan_workspace_size.argtypes = [up, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kan_ukan_generate_backward.restype = ctypes.c_int
+    lib.kan_ukan_generate_backward.argtypes = [up, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.kan_input_range.restype = ctypes.c_int
+    lib.kan_input_range.argtypes = [ctypes.c_int64, _vp, ctypes.c_int32, _vp, _vp, ctypes.c_size_t, _vp]
     lib.kan_set_timing_marks.restype = ctypes.c_int
     lib.kan_set_timing_marks.argtypes = [_vp, _vp]
     lib.kan_ffma_probe.restype = ctypes.c_int
@@ -151,6 +170,36 @@ def kan_grkan_forward(shape, x, a, b, y, stream):
 def kan_grkan_backward(shape, x, a, b, dY, dx, da, db, workspace, ws_bytes, stream):
     check(load().kan_grkan_backward(ctypes.byref(shape), x, a, b, dY, dx, da, db, workspace, ws_bytes, stream),
           "kan_grkan_backward")
+
+
+def make_ukan_shape(n_in, n_out, group, pe_dim, hidden, q0, nq, dtype) -> kan_ukan_shape:
+    return kan_ukan_shape(int(n_in), int(n_out), int(group), int(pe_dim), int(hidden), int(q0), int(nq), int(dtype))
+
+
+def kan_ukan_layer_shape(shape: kan_ukan_shape, batch, h) -> kan_shape:
+    out = kan_shape()
+    check(load().kan_ukan_layer_shape(ctypes.byref(shape), int(batch), float(h), ctypes.byref(out)),
+          "kan_ukan_layer_shape")
+    return out
+
+
+def kan_ukan_generate(shape, W1, b1, W2, b2, coef, pre, stream):
+    check(load().kan_ukan_generate(ctypes.byref(shape), W1, b1, W2, b2, coef, pre, stream), "kan_ukan_generate")
+
+
+def kan_ukan_workspace_size(shape: kan_ukan_shape) -> int:
+    n = ctypes.c_size_t(0)
+    check(load().kan_ukan_workspace_size(ctypes.byref(shape), ctypes.byref(n)), "kan_ukan_workspace_size")
+    return n.value
+
+
+def kan_ukan_generate_backward(shape, W1, W2, pre, dcoef, dW1, db1, dW2, db2, workspace, ws_bytes, stream):
+    check(load().kan_ukan_generate_backward(ctypes.byref(shape), W1, W2, pre, dcoef, dW1, db1, dW2, db2, workspace,
+                                            ws_bytes, stream), "kan_ukan_generate_backward")
+
+
+def kan_input_range(n, x, dtype, minmax, workspace, ws_bytes, stream):
+    check(load().kan_input_range(int(n), x, int(dtype), minmax, workspace, ws_bytes, stream), "kan_input_range")
 
 
 def kan_set_timing_marks(after_prep, after_dcoef):

@@ -279,6 +279,104 @@ class KANLayer2D(torch.nn.Module):
         return y.reshape(*lead, self.out_features)
 
 
+# ---------------------------------------------------------------------------
+# UKAN: unbounded grid, coefficients from a generator of grid-group encodings
+_RANGE_WS = 2368
+
+
+def ukan_window(x, h, group):
+    """(q0, nq): the grid groups whose basis functions the inputs reach (basis floor(x/h) - 3 .. floor(x/h)),
+    from the inputs' device-side minimum and maximum (one small read-back)."""
+    import math
+    ws = torch.empty(_RANGE_WS, dtype=torch.uint8, device=x.device)
+    mm = torch.empty(2, dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        N.kan_input_range(x.numel(), _p(x), _code(x), _p(mm), _p(ws), _RANGE_WS, _stream(x))
+    lo, hi = mm.tolist()
+    if not (math.isfinite(lo) and math.isfinite(hi)):
+        raise ValueError("UKAN layers need finite inputs (the window of generated groups is sized from them)")
+    s_lo, s_hi = math.floor(lo / h), math.floor(hi / h)
+    q0 = math.floor((s_lo - 3) / group)
+    nq = math.floor(s_hi / group) - q0 + 1
+    while nq * group < 4:
+        nq += 1
+    return q0, nq
+
+
+def ukan_shape(n_in, n_out, group, W1, q0, nq, dtype):
+    return N.make_ukan_shape(n_in, n_out, group, W1.shape[1], W1.shape[0], q0, nq,
+                             N.KAN_F32 if dtype == torch.float32 else N.KAN_BF16)
+
+
+def ukan_generate(W1, b1, W2, b2, n_in, n_out, group, q0, nq, dtype=torch.float32):
+    """(coef [out, in, nq*group] in dtype, pre [nq, hidden] float32): the generator's window."""
+    for t, nm in ((W1, "W1"), (b1, "b1"), (W2, "W2"), (b2, "b2")):
+        _check(t, nm, torch.float32)
+    s = ukan_shape(n_in, n_out, group, W1, q0, nq, dtype)
+    coef = torch.empty((n_out, n_in, nq * group), dtype=dtype, device=W1.device)
+    pre = torch.empty((nq, W1.shape[0]), dtype=torch.float32, device=W1.device)
+    with torch.cuda.device(W1.device):
+        N.kan_ukan_generate(s, _p(W1), _p(b1), _p(W2), _p(b2), _p(coef), _p(pre), _stream(W1))
+    return coef, pre
+
+
+def ukan_generate_backward(W1, W2, pre, dcoef, n_in, n_out, group, q0, nq, dtype=torch.float32):
+    """(dW1, db1, dW2, db2) from the window's dcoef [out, in, nq*group] (float32)."""
+    s = ukan_shape(n_in, n_out, group, W1, q0, nq, dtype)
+    dW1, dW2 = torch.empty_like(W1), torch.empty_like(W2)
+    db1 = torch.empty(W1.shape[0], dtype=torch.float32, device=W1.device)
+    db2 = torch.empty(W2.shape[0], dtype=torch.float32, device=W1.device)
+    with torch.cuda.device(W1.device):
+        n = N.kan_ukan_workspace_size(s)
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device=W1.device)
+        N.kan_ukan_generate_backward(s, _p(W1), _p(W2), _p(pre), _p(dcoef), _p(dW1), _p(db1), _p(dW2), _p(db2),
+                                     _p(ws), ws.numel(), _stream(W1))
+    return dW1, db1, dW2, db2
+
+
+class _UKANFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, W1, b1, W2, b2, h, group, n_out):
+        x = x.contiguous()
+        batch, n_in = x.shape
+        q0, nq = ukan_window(x, h, group)
+        coef, pre = ukan_generate(W1, b1, W2, b2, n_in, n_out, group, q0, nq, x.dtype)
+        ks = N.kan_ukan_layer_shape(ukan_shape(n_in, n_out, group, W1, q0, nq, x.dtype), batch, h)
+        y = forward(x, coef, ks.G, ks.lo, ks.hi)
+        ctx.save_for_backward(x, W1, W2, coef, pre)
+        ctx.meta = (h, group, n_out, q0, nq, ks.G, ks.lo, ks.hi)
+        return y
+
+    @staticmethod
+    def backward(ctx, dY):
+        x, W1, W2, coef, pre = ctx.saved_tensors
+        h, group, n_out, q0, nq, G, lo, hi = ctx.meta
+        dx, dcoef, _ = backward(x, coef, dY.contiguous().to(x.dtype), G, lo, hi, need_dx=ctx.needs_input_grad[0])
+        dW1, db1, dW2, db2 = ukan_generate_backward(W1, W2, pre, dcoef, x.shape[1], n_out, group, q0, nq, x.dtype)
+        return dx, dW1, db1, dW2, db2, None, None, None
+
+
+class UKANLayer(torch.nn.Module):
+    """KAN layer on an unbounded grid (spacing h) whose cubic B-spline coefficients come from a generator:
+    an MLP of the sinusoidal encodings of grid groups (``group`` basis functions each).  Only the groups that
+    the batch's inputs reach are generated; the inputs need no normalisation."""
+
+    def __init__(self, in_features, out_features, h=0.25, group=4, pe_dim=16, hidden=32, device=None):
+        super().__init__()
+        self.in_features, self.out_features, self.h, self.group = in_features, out_features, float(h), int(group)
+        kw = dict(dtype=torch.float32, device=device)
+        self.W1 = torch.nn.Parameter(torch.randn(hidden, pe_dim, **kw) * pe_dim ** -0.5)
+        self.b1 = torch.nn.Parameter(torch.zeros(hidden, **kw))
+        self.W2 = torch.nn.Parameter(torch.randn(out_features * in_features * group, hidden, **kw) * 0.1 * hidden ** -0.5)
+        self.b2 = torch.nn.Parameter(torch.zeros(out_features * in_features * group, **kw))
+
+    def forward(self, x):
+        lead = x.shape[:-1]
+        y = _UKANFunction.apply(x.reshape(-1, self.in_features), self.W1, self.b1, self.W2, self.b2, self.h,
+                                self.group, self.out_features)
+        return y.reshape(*lead, self.out_features)
+
+
 class KANNetwork(torch.nn.Module):
     """Stack of KANLayer: ``KANNetwork([784, 64, 10])``."""
 

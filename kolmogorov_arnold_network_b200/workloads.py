@@ -155,6 +155,40 @@ def _grkan():
 GR_WORKLOADS = _grkan()
 
 
+@dataclass(frozen=True)
+class UkWorkload:
+    """A UKAN layer workload: x ~ N(0, x_std) [batch, in] (no normalisation to a grid range), knot spacing h,
+    `group` basis functions per grid group, generator with pe_dim-wide encodings and `hidden` units."""
+    name: str
+    family: int
+    batch: int
+    inp: int
+    out: int
+    h: float
+    group: int
+    pe_dim: int
+    hidden: int
+    dtype: str
+    x_std: float
+    note: str = ""
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def edges(self) -> int:
+        return self.batch * self.inp * self.out
+
+
+UK_WORKLOADS = {
+    "ukan512_bf16": UkWorkload("ukan512_bf16", 9, 65536, 512, 512, 0.25, 4, 16, 32, "bf16", 1.0,
+                               note="UKAN layer 512->512, batch 65536, unbounded grid h=0.25, groups of 4"),
+    "ukan512_f32": UkWorkload("ukan512_f32", 9, 16384, 512, 512, 0.25, 4, 16, 32, "f32", 1.0,
+                              note="UKAN layer 512->512, batch 16384, unbounded grid h=0.25, groups of 4"),
+}
+
+
 def _gen(family: int, tensor_id: int) -> torch.Generator:
     g = torch.Generator(device="cpu")
     g.manual_seed(1000 * family + tensor_id)
@@ -213,6 +247,26 @@ def draw_grkan(w: GrWorkload, rows: int | None = None) -> dict:
     a = torch.randn((w.groups, w.m + 1), generator=_gen(w.family, 1), dtype=torch.float32) * 0.5
     b = torch.randn((w.groups, w.n), generator=_gen(w.family, 2), dtype=torch.float32) * 0.5
     return {"x": x, "dY": dY, "a": a, "b": b}
+
+
+def draw_ukan(w: UkWorkload, rows: int | None = None) -> dict:
+    """x ~ N(0, x_std), dY ~ N(0, 1) in the operand dtype; generator parameters float32:
+    W1 ~ N(0, 1/pe_dim), b1 ~ N(0, 0.1^2), W2 ~ N(0, 0.1^2 / hidden), b2 ~ N(0, 0.1^2) (ids 0, 3, 1, 2, 4, 5)."""
+    rows = w.batch if rows is None else rows
+    f32 = torch.float32
+    x = (torch.randn((rows, w.inp), generator=_gen(w.family, 0), dtype=f32) * w.x_std).to(w.torch_dtype)
+    dY = torch.randn((rows, w.out), generator=_gen(w.family, 3), dtype=f32).to(w.torch_dtype)
+    E = w.out * w.inp * w.group
+    return {"x": x, "dY": dY,
+            "W1": torch.randn((w.hidden, w.pe_dim), generator=_gen(w.family, 1), dtype=f32) * w.pe_dim ** -0.5,
+            "b1": torch.randn(w.hidden, generator=_gen(w.family, 2), dtype=f32) * 0.1,
+            "W2": torch.randn((E, w.hidden), generator=_gen(w.family, 4), dtype=f32) * 0.1 * w.hidden ** -0.5,
+            "b2": torch.randn(E, generator=_gen(w.family, 5), dtype=f32) * 0.1}
+
+
+def custom_ukan(batch, inp, out, h=0.25, group=4, pe_dim=16, hidden=32, dtype="f32", x_std=1.0, family=92):
+    return UkWorkload(f"ukan_custom_{batch}x{inp}x{out}_{dtype}", family, batch, inp, out, h, group, pe_dim, hidden,
+                      dtype, x_std)
 
 
 def custom_grkan(rows, channels, groups, m=5, n=4, dtype="f32", family=91):

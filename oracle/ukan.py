@@ -124,13 +124,22 @@ def backward(x, W1, b1, W2, b2, dY, n_out, h, g, q0=None, nq=None):
         B, dB = basis(x, m0 + m_loc, h)
         dx += dB * (dY @ coef[:, :, m_loc])                # sum_j dY[b,j] coef[j,i,m] B'_m(x[b,i])
         dcoef[:, :, m_loc] = dY.T @ B                      # sum_b dY[b,j] B_m(x[b,i])
-    # back through the generator: dc(q) from dcoef, then the MLP
+    dW1, db1, dW2, db2 = generator_backward(W1, b1, W2, dcoef, q0, nq)
+    return dx, dW1, db1, dW2, db2, dcoef
+
+
+def generator_backward(W1, b1, W2, dcoef, q0, nq):
+    """(dW1, db1, dW2, db2) from the window's dcoef [out, in, nq * g]: back through the generator."""
+    W1, b1, W2, dcoef = _f64(W1), _f64(b1), _f64(W2), _f64(dcoef)
+    n_out, n_in, ng = dcoef.shape
+    g = ng // nq
+    pe = posenc(np.arange(q0, q0 + nq), W1.shape[1])
+    pre = pe @ W1.T + b1                                   # [nq, H]
     dc = dcoef.reshape(n_out, n_in, nq, g).transpose(2, 0, 1, 3).reshape(nq, -1)   # [nq, out*in*g]
     hid = silu(pre)
     dW2 = dc.T @ hid                                       # [out*in*g, H]
     db2 = dc.sum(0)
     dpre = (dc @ W2) * dsilu(pre)                          # [nq, H]
-    pe = posenc(np.arange(q0, q0 + nq), W1.shape[1])
     dW1 = dpre.T @ pe                                      # [H, d]
     db1 = dpre.sum(0)
-    return dx, dW1, db1, dW2, db2, dcoef
+    return dW1, db1, dW2, db2
