@@ -287,7 +287,7 @@ typedef struct {
     int64_t in, out;     /* layer inputs and outputs, >= 1 */
     int32_t group;       /* basis functions per grid group, >= 1 */
     int32_t pe_dim;      /* encoding width, even, 2..256 */
-    int32_t hidden;      /* generator hidden width, 1..256 */
+    int32_t hidden;      /* generator hidden width, a multiple of 4 in 4..256 */
     int32_t q0, nq;      /* first group of the window and number of groups (nq*group >= 4, nq*hidden <= 12288) */
     int32_t dtype;       /* kan_dtype of the generated window (the layer's operand dtype) */
 } kan_ukan_shape;

@@ -60,11 +60,15 @@ template <typename T> __device__ __forceinline__ T cvt_out(float v);
 template <> __device__ __forceinline__ float cvt_out<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 cvt_out<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
 
-// Chunks of CE edges per block iteration: the chunk's W2 rows (CE * g rows of
-// H floats, contiguous in W2) are staged in shared memory by coalesced loads,
-// then every thread computes four window entries (one W2 row, four groups)
-// from shared memory and writes them into the edges' contiguous window rows.
+// Chunks of kCE edges per block iteration: the chunk's W2 rows (kCE * g rows
+// of H floats, contiguous in W2) are staged in shared memory by coalesced
+// loads (rows padded to H + 4 floats: 16-byte aligned, conflict-free 16-byte
+// reads across rows), then every thread computes four window entries (one W2
+// row, four groups) with 16-byte shared loads and writes them into the edges'
+// contiguous window rows.  H is a multiple of 4.
 constexpr int kCE = 32;
+
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
 template <typename T>
 __global__ void __launch_bounds__(kUkThreads) ukan_generate_kernel(const float* __restrict__ W1,
@@ -74,34 +78,31 @@ __global__ void __launch_bounds__(kUkThreads) ukan_generate_kernel(const float* 
                                                                     float* __restrict__ pre_out, int64_t edges, int g,
                                                                     int d, int H, int q0, int nq)
 {
-    extern __shared__ float sh[];
-    const int hp = H + 1;                        // padded row stride (no bank conflicts across rows)
-    float* hid = sh;                             // [nq][hp]
-    float* sw = sh + nq * hp;                    // [kCE * g][hp]
-    for (int t = threadIdx.x; t < nq * H; t += blockDim.x) {
-        const int ql = t / H, h = t - ql * H;
-        hid[ql * hp + h] = 0.0f;
-    }
-    __syncthreads();
+    extern __shared__ __align__(16) float sh[];
+    const int hp = H + 4;
+    const int nqp = (nq + 3) / 4 * 4;           // hidden rows padded to whole blocks of four groups
+    float* hid = sh;                             // [nqp][hp] (rows past nq are zero)
+    float* sw = sh + nqp * hp;                   // [kCE * g][hp]
     {
-        // pre-activations (block 0 also stores them for the backward), then silu
         float* pre = sw;                         // scratch: [nq * H] fits in the W2 staging area
         hidden_pre(W1, b1, q0, nq, d, H, pre);
         __syncthreads();
-        for (int t = threadIdx.x; t < nq * H; t += blockDim.x) {
-            if (blockIdx.x == 0) pre_out[t] = pre[t];
+        for (int t = threadIdx.x; t < nqp * H; t += blockDim.x) {
             const int ql = t / H, h = t - ql * H;
-            hid[ql * hp + h] = silu_pre(pre[t]);
+            const float v = ql < nq ? pre[t] : 0.0f;
+            if (blockIdx.x == 0 && ql < nq) pre_out[t] = v;
+            hid[ql * hp + h] = ql < nq ? silu_pre(v) : 0.0f;
         }
         __syncthreads();
     }
-    const int nqb = (nq + 3) / 4;
+    const int nqb = nqp / 4;
     for (int64_t c0 = (int64_t)blockIdx.x * kCE; c0 < edges; c0 += (int64_t)gridDim.x * kCE) {
         const int ne = (int)(edges - c0 < kCE ? edges - c0 : kCE);
         __syncthreads();
-        for (int t = threadIdx.x; t < ne * g * H; t += blockDim.x) {
-            const int row = t / H, h = t - row * H;
-            sw[row * hp + h] = W2[c0 * g * H + t];
+        for (int t = threadIdx.x; t < ne * g * (H / 4); t += blockDim.x) {
+            const int row = t / (H / 4), h4 = t - row * (H / 4);
+            *reinterpret_cast<float4*>(sw + row * hp + 4 * h4) =
+                *reinterpret_cast<const float4*>(W2 + (c0 * g + row) * H + 4 * h4);
         }
         __syncthreads();
         // work items: (edge, group block, row r) with r fastest
@@ -109,14 +110,15 @@ __global__ void __launch_bounds__(kUkThreads) ukan_generate_kernel(const float* 
             const int r = it % g, rest = it / g;
             const int qb = rest % nqb, e = rest / nqb;
             const float* w = sw + (e * g + r) * hp;
+            const float* hq = hid + (qb * 4) * hp;
             const float bias = b2[(c0 + e) * g + r];
             float acc[4] = {bias, bias, bias, bias};
-            for (int h = 0; h < H; ++h) {
-                const float wv = w[h];
+            for (int h = 0; h < H; h += 4) {
+                const float4 wv = lds4(w + h);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int ql = min(qb * 4 + u, nq - 1);
-                    acc[u] = fmaf(wv, hid[ql * hp + h], acc[u]);
+                    const float4 hv = lds4(hq + u * hp + h);
+                    acc[u] = fmaf(wv.x, hv.x, fmaf(wv.y, hv.y, fmaf(wv.z, hv.z, fmaf(wv.w, hv.w, acc[u]))));
                 }
             }
             T* crow = coef + (c0 + e) * (int64_t)nq * g;
@@ -131,18 +133,18 @@ __global__ void __launch_bounds__(kUkThreads) ukan_generate_kernel(const float* 
 
 // dW2[e, :] = sum_q dc(q)[e] hid(q), db2[e] = sum_q dc(q)[e]: chunks of kCE edges
 // (their dcoef window rows staged in shared memory), each thread four hidden
-// units of one W2 row, written contiguously.
+// units of one W2 row (16-byte loads and stores).
 __global__ void __launch_bounds__(kUkThreads) ukan_dw2_kernel(const float* __restrict__ pre,
                                                                const float* __restrict__ dcoef,
                                                                float* __restrict__ dW2, float* __restrict__ db2,
                                                                int64_t edges, int g, int H, int nq)
 {
-    extern __shared__ float sh[];
+    extern __shared__ __align__(16) float sh[];
     float* hid = sh;                             // [nq][H]
     float* sd = sh + nq * H;                     // [kCE][nq * g]
     for (int t = threadIdx.x; t < nq * H; t += blockDim.x) hid[t] = silu_pre(pre[t]);
     const int nw = nq * g;
-    const int hb_n = (H + 3) / 4;
+    const int hb_n = H / 4;
     for (int64_t c0 = (int64_t)blockIdx.x * kCE; c0 < edges; c0 += (int64_t)gridDim.x * kCE) {
         const int ne = (int)(edges - c0 < kCE ? edges - c0 : kCE);
         __syncthreads();
@@ -160,38 +162,43 @@ __global__ void __launch_bounds__(kUkThreads) ukan_dw2_kernel(const float* __res
         for (int it = threadIdx.x; it < ne * g * hb_n; it += blockDim.x) {
             const int hb = it % hb_n, row = it / hb_n;
             const int e = row / g, r = row - e * g;
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             for (int ql = 0; ql < nq; ++ql) {
                 const float dv = sd[e * nw + ql * g + r];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) acc[u] = fmaf(dv, hid[ql * H + min(hb * 4 + u, H - 1)], acc[u]);
+                const float4 hv = lds4(hid + ql * H + 4 * hb);
+                acc.x = fmaf(dv, hv.x, acc.x);
+                acc.y = fmaf(dv, hv.y, acc.y);
+                acc.z = fmaf(dv, hv.z, acc.z);
+                acc.w = fmaf(dv, hv.w, acc.w);
             }
-            float* w = dW2 + ((c0 + e) * g + r) * H;
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (hb * 4 + u < H) w[hb * 4 + u] = acc[u];
+            *reinterpret_cast<float4*>(dW2 + ((c0 + e) * g + r) * H + 4 * hb) = acc;
         }
     }
 }
 
 // Block partials of dhid[ql, h] = sum_e dc(ql)[e] W2[e, h] over a contiguous
 // range of edges: chunks of 64 edges (64 g rows of W2 and the matching dcoef
-// values) staged in shared memory, each thread accumulating a 4 x 4 tile of
-// (group, hidden unit) pairs in registers; one partial row per block.
+// values) staged in shared memory; a thread accumulates a 4 x 4 tile of
+// (group, hidden unit) pairs over one of RG interleaved subsets of the rows,
+// and the RG partial tiles are added in subset order at the end; one partial
+// row per block.
 __global__ void __launch_bounds__(kUkThreads) ukan_dhid_kernel(const float* __restrict__ W2,
                                                                 const float* __restrict__ dcoef,
                                                                 float* __restrict__ part, int64_t edges, int g, int H,
                                                                 int nq, int64_t edges_per_block)
 {
     constexpr int CE = 64;                                    // edges per chunk
-    extern __shared__ float sh[];
+    extern __shared__ __align__(16) float sh[];
     const int rows = CE * g;                                  // W2 rows per chunk
-    float* sw = sh;                                           // [rows][H]
-    float* sd = sh + rows * H;                                // [nq][rows]
-    const int tq_n = (nq + kTq - 1) / kTq, th_n = (H + kTh - 1) / kTh;
+    const int hp = H + 4;
+    float* sw = sh;                                           // [rows][hp]
+    float* sd = sh + rows * hp;                               // [nq][rows]
+    const int tq_n = (nq + kTq - 1) / kTq, th_n = H / kTh;
+    const int tiles = tq_n * th_n;
+    const int RG = tiles >= kUkThreads ? 1 : kUkThreads / tiles;   // row subsets
+    const int rg = threadIdx.x / tiles;                       // (>= RG: idle; tiles > 256: see the s loop)
     const int64_t e_begin = (int64_t)blockIdx.x * edges_per_block;
     const int64_t e_end = min(edges, e_begin + edges_per_block);
-    // this thread's tiles (a thread may own several when nq * H is large)
     float acc[4][kTq][kTh];
 #pragma unroll
     for (int s = 0; s < 4; ++s)
@@ -202,49 +209,113 @@ __global__ void __launch_bounds__(kUkThreads) ukan_dhid_kernel(const float* __re
     for (int64_t c0 = e_begin; c0 < e_end; c0 += CE) {
         const int ne = (int)(e_end - c0 < CE ? e_end - c0 : CE);
         __syncthreads();
-        for (int t = threadIdx.x; t < ne * g * H; t += blockDim.x) sw[t] = W2[(c0 * g) * H + t];
+        for (int t = threadIdx.x; t < ne * g * (H / 4); t += blockDim.x) {
+            const int row = t / (H / 4), h4 = t - row * (H / 4);
+            *reinterpret_cast<float4*>(sw + row * hp + 4 * h4) =
+                *reinterpret_cast<const float4*>(W2 + (c0 * g + row) * H + 4 * h4);
+        }
         for (int t = threadIdx.x; t < nq * ne * g; t += blockDim.x) {
             const int ql = t / (ne * g), rr = t - ql * (ne * g);
             const int e = rr / g, r = rr - e * g;
             sd[ql * rows + rr] = dcoef[(c0 + e) * (int64_t)nq * g + ql * g + r];
         }
         __syncthreads();
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int tile = threadIdx.x + s * blockDim.x;
-            if (tile >= tq_n * th_n) break;
+        if (RG > 1) {
+            if (rg >= RG) continue;
+            const int tile = threadIdx.x - rg * tiles;
             const int tq = tile / th_n, th = tile - tq * th_n;
-            for (int rr = 0; rr < ne * g; ++rr) {
-                float dv[kTq], wv[kTh];
+            for (int rr = rg; rr < ne * g; rr += RG) {
+                float dv[kTq];
 #pragma unroll
                 for (int a = 0; a < kTq; ++a) dv[a] = tq * kTq + a < nq ? sd[(tq * kTq + a) * rows + rr] : 0.0f;
+                const float4 wv = lds4(sw + rr * hp + th * kTh);
 #pragma unroll
-                for (int b = 0; b < kTh; ++b) wv[b] = th * kTh + b < H ? sw[rr * H + th * kTh + b] : 0.0f;
+                for (int a = 0; a < kTq; ++a) {
+                    acc[0][a][0] = fmaf(dv[a], wv.x, acc[0][a][0]);
+                    acc[0][a][1] = fmaf(dv[a], wv.y, acc[0][a][1]);
+                    acc[0][a][2] = fmaf(dv[a], wv.z, acc[0][a][2]);
+                    acc[0][a][3] = fmaf(dv[a], wv.w, acc[0][a][3]);
+                }
+            }
+        } else {
 #pragma unroll
-                for (int a = 0; a < kTq; ++a)
+            for (int s = 0; s < 4; ++s) {
+                const int tile = threadIdx.x + s * blockDim.x;
+                if (tile >= tiles) break;
+                const int tq = tile / th_n, th = tile - tq * th_n;
+                for (int rr = 0; rr < ne * g; ++rr) {
+                    float dv[kTq];
 #pragma unroll
-                    for (int b = 0; b < kTh; ++b) acc[s][a][b] = fmaf(dv[a], wv[b], acc[s][a][b]);
+                    for (int a = 0; a < kTq; ++a) dv[a] = tq * kTq + a < nq ? sd[(tq * kTq + a) * rows + rr] : 0.0f;
+                    const float4 wv = lds4(sw + rr * hp + th * kTh);
+#pragma unroll
+                    for (int a = 0; a < kTq; ++a) {
+                        acc[s][a][0] = fmaf(dv[a], wv.x, acc[s][a][0]);
+                        acc[s][a][1] = fmaf(dv[a], wv.y, acc[s][a][1]);
+                        acc[s][a][2] = fmaf(dv[a], wv.z, acc[s][a][2]);
+                        acc[s][a][3] = fmaf(dv[a], wv.w, acc[s][a][3]);
+                    }
+                }
             }
         }
+    }
+    if (RG > 1) {
+        // the RG subsets' tiles, added in subset order
+        __syncthreads();
+        float* red = sh;                                      // [RG][tiles][16]
+        if (rg < RG) {
+            const int tile = threadIdx.x - rg * tiles;
+#pragma unroll
+            for (int a = 0; a < kTq; ++a)
+#pragma unroll
+                for (int b = 0; b < kTh; ++b) red[(rg * tiles + tile) * 16 + a * kTh + b] = acc[0][a][b];
+        }
+        __syncthreads();
+        for (int t = threadIdx.x; t < tiles * 16; t += blockDim.x) {
+            const int tile = t / 16, ab = t - tile * 16, a = ab / kTh, b = ab - a * kTh;
+            float v = 0.0f;
+            for (int q = 0; q < RG; ++q) v += red[(q * tiles + tile) * 16 + ab];
+            const int tq = tile / th_n, th = tile - tq * th_n;
+            const int ql = tq * kTq + a, h = th * kTh + b;
+            if (ql < nq) part[(int64_t)blockIdx.x * nq * H + ql * H + h] = v;
+        }
+        return;
     }
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
         const int tile = threadIdx.x + s * blockDim.x;
-        if (tile >= tq_n * th_n) break;
+        if (tile >= tiles) break;
         const int tq = tile / th_n, th = tile - tq * th_n;
 #pragma unroll
         for (int a = 0; a < kTq; ++a)
 #pragma unroll
             for (int b = 0; b < kTh; ++b) {
                 const int ql = tq * kTq + a, h = th * kTh + b;
-                if (ql < nq && h < H) part[(int64_t)blockIdx.x * nq * H + ql * H + h] = acc[s][a][b];
+                if (ql < nq) part[(int64_t)blockIdx.x * nq * H + ql * H + h] = acc[s][a][b];
             }
     }
 }
 
-// dhid from the block partials (fixed order, fp64), then dpre = dhid silu'(pre),
+// Sums of the block partials for every (group, hidden unit), split into kSub
+// contiguous runs of blocks summed in parallel, the runs then added in order
+// (fp64 throughout): dhid.
+constexpr int kSub = 8;
+
+__global__ void __launch_bounds__(kUkThreads) ukan_dhid_sum_kernel(const float* __restrict__ part, int nblocks,
+                                                                    int n, double* __restrict__ sub)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n * kSub) return;
+    const int o = t / kSub, k = t - o * kSub;
+    const int per = (nblocks + kSub - 1) / kSub;
+    double v = 0.0;
+    for (int b = k * per; b < min(nblocks, (k + 1) * per); ++b) v += (double)part[(int64_t)b * n + o];
+    sub[t] = v;
+}
+
+// dhid from the run sums (added in run order), then dpre = dhid silu'(pre),
 // dW1[h, :] = sum_q dpre[q, h] PE(q), db1[h] = sum_q dpre[q, h].  One block.
-__global__ void __launch_bounds__(kUkThreads) ukan_dw1_kernel(const float* __restrict__ part, int nblocks,
+__global__ void __launch_bounds__(kUkThreads) ukan_dw1_kernel(const double* __restrict__ sub,
                                                                const float* __restrict__ pre, int q0, int nq, int d,
                                                                int H, float* __restrict__ dW1, float* __restrict__ db1)
 {
@@ -252,7 +323,7 @@ __global__ void __launch_bounds__(kUkThreads) ukan_dw1_kernel(const float* __res
     float* dpre = sh;                                         // [nq][H]
     for (int t = threadIdx.x; t < nq * H; t += blockDim.x) {
         double s = 0.0;
-        for (int b = 0; b < nblocks; ++b) s += (double)part[(int64_t)b * nq * H + t];
+        for (int k = 0; k < kSub; ++k) s += sub[t * kSub + k];
         const float z = pre[t];
         const float sg = __frcp_rn(1.0f + __expf(-z));
         dpre[t] = (float)s * (sg * (1.0f + z * (1.0f - sg)));
@@ -329,7 +400,8 @@ kan_status validate(const kan_ukan_shape* s)
     if (!s) return uk_fail(KAN_ERR_INVALID_ARG, "shape is NULL");
     if (s->in < 1 || s->out < 1 || s->group < 1) return uk_fail(KAN_ERR_INVALID_ARG, "in, out, group must be >= 1");
     if (s->pe_dim < 2 || s->pe_dim % 2 || s->pe_dim > 256) return uk_fail(KAN_ERR_INVALID_ARG, "pe_dim must be even, 2..256");
-    if (s->hidden < 1 || s->hidden > kMaxHidden) return uk_fail(KAN_ERR_INVALID_ARG, "hidden must be 1..256");
+    if (s->hidden < 4 || s->hidden > kMaxHidden || s->hidden % 4)
+        return uk_fail(KAN_ERR_INVALID_ARG, "hidden must be a multiple of 4 in 4..256");
     if (s->nq < 1 || (int64_t)s->nq * s->group < 4) return uk_fail(KAN_ERR_INVALID_ARG, "nq * group must be >= 4");
     if ((int64_t)s->nq * s->hidden > kMaxHidTerms) return uk_fail(KAN_ERR_UNSUPPORTED, "nq * hidden > 12288");
     if (s->dtype != KAN_F32 && s->dtype != KAN_BF16) return uk_fail(KAN_ERR_INVALID_ARG, "unknown dtype");
@@ -353,13 +425,25 @@ int chunk_blocks(int64_t edges)
 
 size_t gen_smem(const kan_ukan_shape& s)
 {
-    const int hp = s.hidden + 1;
-    return (size_t)(s.nq * hp + std::max(kCE * s.group * hp, s.nq * s.hidden)) * sizeof(float);
+    const int hp = s.hidden + 4, nqp = (s.nq + 3) / 4 * 4;
+    return (size_t)(nqp * hp + std::max(kCE * s.group * hp, s.nq * s.hidden)) * sizeof(float);
 }
 
 size_t dw2_smem(const kan_ukan_shape& s) { return (size_t)(s.nq * s.hidden + kCE * s.nq * s.group) * sizeof(float); }
 
-size_t dhid_smem(const kan_ukan_shape& s) { return (size_t)(64 * s.group * s.hidden + s.nq * 64 * s.group) * sizeof(float); }
+// workspace: the dhid block partials (float), then the run sums (double)
+size_t part_bytes(const kan_ukan_shape& s)
+{
+    return ((size_t)dhid_blocks(s.in * s.out) * s.nq * s.hidden * sizeof(float) + 255) & ~(size_t)255;
+}
+size_t ukan_ws_bytes(const kan_ukan_shape& s) { return part_bytes(s) + (size_t)s.nq * s.hidden * kSub * sizeof(double); }
+
+size_t dhid_smem(const kan_ukan_shape& s)
+{
+    // staging, or the final combine of the row subsets ([RG][tiles][16] <= 256 * 16 floats)
+    const size_t stage = (size_t)(64 * s.group * (s.hidden + 4) + s.nq * 64 * s.group);
+    return std::max<size_t>(stage, 256 * 16) * sizeof(float);
+}
 
 }  // namespace
 }  // namespace kan
@@ -425,7 +509,7 @@ kan_status kan_ukan_workspace_size(const kan_ukan_shape* s, size_t* bytes)
     kan_status st = validate(s);
     if (st != KAN_OK) return st;
     if (!bytes) return uk_fail(KAN_ERR_INVALID_ARG, "bytes is NULL");
-    *bytes = (size_t)dhid_blocks(s->in * s->out) * s->nq * s->hidden * sizeof(float);
+    *bytes = ukan_ws_bytes(*s);
     return KAN_OK;
 }
 
@@ -454,26 +538,31 @@ kan_status kan_ukan_generate_backward(const kan_ukan_shape* s, const float* W1, 
     }
     if (e == cudaSuccess && (dW1 || db1)) {
         const int nb = dhid_blocks(edges);
-        const size_t need = (size_t)nb * s->nq * s->hidden * sizeof(float);
+        const size_t need = ukan_ws_bytes(*s);
         if (ws_bytes < need || !workspace) return uk_fail(KAN_ERR_WORKSPACE, "workspace too small");
-        const int tiles = ((s->nq + kTq - 1) / kTq) * ((s->hidden + kTh - 1) / kTh);
-        if (tiles > 4 * kUkThreads) return uk_fail(KAN_ERR_UNSUPPORTED, "nq * hidden too large for the dhid tiles");
-        const size_t smem = dhid_smem(*s);
-        if (smem > 227 * 1024) return uk_fail(KAN_ERR_UNSUPPORTED, "group * hidden too large for the dhid stage");
-        static size_t configured = 0;
-        if (smem > 48 * 1024 && configured < smem) {
-            cudaFuncSetAttribute(ukan_dhid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-            configured = 227 * 1024;
-        }
         const int64_t per = (edges + nb - 1) / nb;
         float* part = reinterpret_cast<float*>(workspace);
-        ukan_dhid_kernel<<<nb, kUkThreads, smem, cs>>>(W2, dcoef, part, edges, s->group, s->hidden, s->nq, per);
+        double* sub = reinterpret_cast<double*>(reinterpret_cast<char*>(workspace) + part_bytes(*s));
+        {
+            const int tiles = ((s->nq + kTq - 1) / kTq) * ((s->hidden + kTh - 1) / kTh);
+            if (tiles > 4 * kUkThreads) return uk_fail(KAN_ERR_UNSUPPORTED, "nq * hidden too large for the dhid tiles");
+            const size_t smem = dhid_smem(*s);
+            if (smem > 227 * 1024) return uk_fail(KAN_ERR_UNSUPPORTED, "group * hidden too large for the dhid stage");
+            static size_t configured = 0;
+            if (smem > 48 * 1024 && configured < smem) {
+                cudaFuncSetAttribute(ukan_dhid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+                configured = 227 * 1024;
+            }
+            ukan_dhid_kernel<<<nb, kUkThreads, smem, cs>>>(W2, dcoef, part, edges, s->group, s->hidden, s->nq, per);
+        }
         count_launch();
         e = cudaGetLastError();
         if (e == cudaSuccess) {
-            ukan_dw1_kernel<<<1, kUkThreads, (size_t)s->nq * s->hidden * sizeof(float), cs>>>(
-                part, nb, pre, s->q0, s->nq, s->pe_dim, s->hidden, dW1, db1);
-            count_launch();
+            const int n = s->nq * s->hidden;
+            ukan_dhid_sum_kernel<<<(n * kSub + kUkThreads - 1) / kUkThreads, kUkThreads, 0, cs>>>(part, nb, n, sub);
+            ukan_dw1_kernel<<<1, kUkThreads, (size_t)n * sizeof(float), cs>>>(sub, pre, s->q0, s->nq, s->pe_dim,
+                                                                            s->hidden, dW1, db1);
+            count_launch(2);
             e = cudaGetLastError();
         }
     }
