@@ -423,6 +423,79 @@ __device__ __forceinline__ void weights_fma(float t, float (&w)[4])
     w[3] = t2 * t * (1.0f / 6.0f);
 }
 
+// 64-bit shifts whose amounts past 63 (including negative amounts read as
+// unsigned) give 0, as the PTX shift instructions clamp them.
+__device__ __forceinline__ uint64_t shl64(uint64_t v, int n)
+{
+    uint64_t r;
+    asm("shl.b64 %0, %1, %2;" : "=l"(r) : "l"(v), "r"(n));
+    return r;
+}
+__device__ __forceinline__ uint64_t shr64(uint64_t v, int n)
+{
+    uint64_t r;
+    asm("shr.b64 %0, %1, %2;" : "=l"(r) : "l"(v), "r"(n));
+    return r;
+}
+
+// One input's eight basis columns as a 16-byte chunk (G + 3 = 8, so that the
+// columns of input i are exactly chunk i of the operand row): the four packed
+// 16-bit weights P (w0 in the low bits) placed at columns s..s+3, the columns
+// outside 0..7 dropped.  Branch-free for s in -3..7 (P = 0 stores zeros).
+__device__ __forceinline__ uint4 chunk8(uint64_t P, int s)
+{
+    const int b = 16 * s;
+    const uint64_t lo = shl64(P, b) | shr64(P, -b);
+    const uint64_t hi = shl64(P, b - 64) | shr64(P, 64 - b);
+    return make_uint4((uint32_t)lo, (uint32_t)(lo >> 32), (uint32_t)hi, (uint32_t)(hi >> 32));
+}
+
+// The packed weights of one input for chunk8 (bf16, or the fp16 hi / lo parts
+// of the fp32 path): span s and, when the input is outside the extended knots
+// (or not a real input), P = 0.
+template <int DT>
+__device__ __forceinline__ void input_chunk(float x, bool act, float inv_h, float u0, float u_hi, int& s,
+                                            uint64_t& P_hi, uint64_t& P_lo)
+{
+    float u = fmaf(x, inv_h, u0);
+    const bool ok = act && u >= -3.0f && u < u_hi;
+    u = ok ? u : 0.0f;
+    float f;
+    floor_split(u, s, f);
+    float w[4];
+    weights_fma(u - f, w);
+    if constexpr (DT == KAN_BF16) {
+        const uint64_t p = (uint64_t)pack_bf16(w[0], w[1]) | ((uint64_t)pack_bf16(w[2], w[3]) << 32);
+        P_hi = ok ? p : 0ull;
+        P_lo = 0ull;
+    } else {
+        uint16_t h[4], l[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) split_f16(w[q], h[q], l[q]);
+        const uint64_t ph = (uint64_t)h[0] | ((uint64_t)h[1] << 16) | ((uint64_t)h[2] << 32) | ((uint64_t)h[3] << 48);
+        const uint64_t pl = (uint64_t)l[0] | ((uint64_t)l[1] << 16) | ((uint64_t)l[2] << 32) | ((uint64_t)l[3] << 48);
+        P_hi = ok ? ph : 0ull;
+        P_lo = ok ? pl : 0ull;
+    }
+}
+
+// The eight x values of a window that starts on a 16-byte boundary, straight
+// from the raw registers of an XWindow (no shift needed).
+template <typename T, int MAXI>
+__device__ __forceinline__ void aligned8(const XWindow<T, MAXI>& w, float (&xv)[8])
+{
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            xv[2 * e] = __uint_as_float(w.raw[e] << 16);
+            xv[2 * e + 1] = __uint_as_float(w.raw[e] & 0xFFFF0000u);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xv[e] = __uint_as_float(w.raw[e]);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
@@ -773,7 +846,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 int uses = 0;                               // k-blocks this group has filled
                 for (int it = grp; grp < NG && it < nk; it += NG, ++uses) {
                     float cur[MAXI];
-                    nxw.values(cur);
+                    const XWindow<T, MAXI> cur_raw = nxw;   // this k-block's window (the next one is fetched below)
                     const int kb = kb_begin + it;
                     if (it + NG < nk) fetch(kb + NG);
                     const int s = it % sa_n;
@@ -782,7 +855,30 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     if (!acquire(s, ph)) break;
                     const uint32_t ahi = A_hi(s), alo = A_lo(s);
                     const uint32_t rbase = row * 128u, rx = row & 7u;
-                    if (kb < a.nkb_main) {
+                    // G + 3 = 8 (bf16 or fp32, no SiLU column, x rows 16-byte aligned): every
+                    // input of the k-block owns one whole 16-byte chunk of the row, built in
+                    // registers and stored at once (no zeroing pass, no scattered stores)
+                    bool chunked = false;
+                    if constexpr (MAXI == 9 && KD == 3) chunked = a.nb == 8 && !a.ext && a.x_vec && kb < a.nkb_main;
+                    if (chunked) {
+                        float xv[8];
+                        aligned8(cur_raw, xv);
+                        const int n8 = row_ok ? min(8, (int)a.in - first_input(kb)) : 0;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            int sidx;
+                            uint64_t Ph, Pl;
+                            input_chunk<DT>(xv[c], c < n8, a.inv_h, u0, u_hi, sidx, Ph, Pl);
+                            const uint32_t off = sw128_chunk(row, (uint32_t)c);
+                            const uint4 vh = chunk8(Ph, sidx);
+                            st_shared_v4(ahi + off, vh.x, vh.y, vh.z, vh.w);
+                            if constexpr (F32) {
+                                const uint4 vl = chunk8(Pl, sidx);
+                                st_shared_v4(alo + off, vl.x, vl.y, vl.z, vl.w);
+                            }
+                        }
+                    } else if (kb < a.nkb_main) {
+                        cur_raw.values(cur);
                         zero_row<DT>(ahi + rbase, alo + rbase, rx);
                         if (row_ok) {
                             const int i0 = first_input(kb), n = last_input(kb) - i0 + 1;
@@ -909,7 +1005,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 if (grp < NG && grp < nk) fetch(kb_begin + grp);
                 for (int it = grp; grp < NG && it < nk; it += NG) {
                     float cur[MAXI];
-                    nxw.values(cur);
+                    const XWindow<T, MAXI> cur_raw = nxw;   // this k-block's window (the next one is fetched below)
                     const int kb = kb_begin + it;
                     if (it + NG < nk) fetch(kb + NG);
                     const int s = it % sa_n;
@@ -919,7 +1015,29 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     const bool row_ok = b < a.batch;
                     const uint32_t roff = (uint32_t)atom * BK * 128u + (uint32_t)rb * 128u;
                     const uint32_t rb_hi = A_hi(s) + roff, rb_lo = A_lo(s) + roff;
-                    if (!silu_tile) {
+                    // G + 3 = 8: each input of the atom row owns one whole 16-byte chunk (see
+                    // the forward producer)
+                    bool chunked = false;
+                    if constexpr (MAXI == 9 && KD == 3) chunked = !silu_tile && a.nb == 8 && !a.ext && a.x_vec;
+                    if (chunked) {
+                        float xv[8];
+                        aligned8(cur_raw, xv);
+                        const int n8 = row_ok ? n_inp : 0;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            int sidx;
+                            uint64_t Ph, Pl;
+                            input_chunk<DT>(xv[c], c < n8, a.inv_h, u0, u_hi, sidx, Ph, Pl);
+                            const uint32_t off = (((uint32_t)c ^ ((uint32_t)rb & 7u)) << 4);
+                            const uint4 vh = chunk8(Ph, sidx);
+                            st_shared_v4(rb_hi + off, vh.x, vh.y, vh.z, vh.w);
+                            if constexpr (F32) {
+                                const uint4 vl = chunk8(Pl, sidx);
+                                st_shared_v4(rb_lo + off, vl.x, vl.y, vl.z, vl.w);
+                            }
+                        }
+                    } else if (!silu_tile) {
+                        cur_raw.values(cur);
                         // this thread's atom row starts from zeros (rows past the batch stay zero)
                         zero_row<DT>(rb_hi, rb_lo, (uint32_t)rb & 7u);
                         if (row_ok && TWOD) {
