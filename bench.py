@@ -1,6 +1,7 @@
 """Benchmark: KAN layer forward+backward edge evaluations per second on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py --only NAME [--steps K]      # one workload by itself, its own JSON line
 
 Default workload: the KAN FFN block (8192 tokens, 768 -> 3072 -> 768, G = 5 on
 [-3, 3], bf16 operands with fp32 accumulation), the largest single-GPU
@@ -706,6 +707,56 @@ EXTRA_WORKLOADS = ["layer784x64_silu", "layer1024_g20_bf16"] + \
     [f"surface512_g8_{dt}_fwdbwd" for dt in ("bf16", "f32")]
 
 
+def time_other(nm: str, dev, K: int, flush, pk: dict, ffma: float) -> dict:
+    """One workload beside the headline one: K steps after 3 warm-up steps, L2 flushed between steps."""
+    if nm in W.GR_WORKLOADS:
+        return time_grkan(W.GR_WORKLOADS[nm], dev, K, flush, pk)
+    if nm in W.UK_WORKLOADS:
+        wu = W.UK_WORKLOADS[nm]
+        Ru = UkRunner(wu, dev)
+        tu, segu, _ = time_steps(Ru, K, 3, flush)
+        msu = tu / K
+        ru = roofline_of(Ru.w, segu, K, pk, ffma)
+        out = {"ms_per_step": msu, "value": wu.edges / (msu / 1000.0), "unit": UNIT, "steps": K,
+               "dtype": wu.dtype, "dominant": ru["kernel"], "bound": ru["bound"], "frac": ru["frac"],
+               "segment_ms": ru["segment_ms"], "step_roofline": step_roofline(Ru.w, msu, pk, ffma),
+               "window": {"q0": Ru.q0, "nq": Ru.nq, "G": Ru.ks.G, "basis_per_input": Ru.nq * wu.group},
+               "note": "generator window sized once before the timed steps; step = generate + layer "
+                       "forward + layer backward + generator backward"}
+        del Ru
+        torch.cuda.empty_cache()
+        return out
+    wx = W.WORKLOADS[nm]
+    Rx = Runner(wx, dev)
+    tx, segx, _ = time_steps(Rx, K, 3, flush)
+    msx = tx / K
+    rx = roofline_of(wx, segx, K, pk, ffma)
+    ax = Rx.adjoint_errors()
+    tolx = 1e-5 if wx.dtype == "f32" else 2e-2
+    out = {"ms_per_step": msx, "value": wx.edges / (msx / 1000.0), "unit": UNIT, "steps": K,
+           "dtype": wx.dtype, "dominant": rx["kernel"], "bound": rx["bound"], "frac": rx["frac"],
+           "tensor_dense_frac": rx.get("tensor_dense_frac"),
+           "segment_ms": rx["segment_ms"], "step_roofline": step_roofline(wx, msx, pk, ffma),
+           "adjoint_rel_err": ax, "adjoint_ok": all(v <= tolx for v in ax.values())}
+    del Rx
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_only(args, local):
+    """``--only NAME``: one workload of the measurement plan by itself (one GPU, no headline line); used to
+    profile a kernel that the headline workload does not run."""
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    res = time_other(args.only, dev, args.steps, flush, peaks(), ffma_peak(dev, sms))
+    st = R_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {st}")
+    print(json.dumps({"workload": args.only, **res}), flush=True)
+
+
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -760,40 +811,9 @@ def run_ours(args, world, rank, local):
     # ---- the other workloads of the method's measurement plan, one GPU only ----
     others = {}
     if world == 1 and not args.no_extras:
-        for nm in EXTRA_WORKLOADS:
-            if nm == w.name:
-                continue
-            wx = W.WORKLOADS[nm]
-            Rx = Runner(wx, dev)
-            kx = min(K, args.extra_steps)
-            tx, segx, _ = time_steps(Rx, kx, 3, flush)
-            msx = tx / kx
-            rx = roofline_of(wx, segx, kx, pk, ffma)
-            ax = Rx.adjoint_errors()
-            tolx = 1e-5 if wx.dtype == "f32" else 2e-2
-            others[nm] = {"ms_per_step": msx, "value": wx.edges / (msx / 1000.0), "unit": UNIT, "steps": kx,
-                          "dtype": wx.dtype, "dominant": rx["kernel"], "bound": rx["bound"], "frac": rx["frac"],
-                          "tensor_dense_frac": rx.get("tensor_dense_frac"),
-                          "segment_ms": rx["segment_ms"], "step_roofline": step_roofline(wx, msx, pk, ffma),
-                          "adjoint_rel_err": ax, "adjoint_ok": all(v <= tolx for v in ax.values())}
-            del Rx
-            torch.cuda.empty_cache()
-        for nm, wg in W.GR_WORKLOADS.items():
-            others[nm] = time_grkan(wg, dev, min(K, args.extra_steps), flush, pk)
-        for nm, wu in W.UK_WORKLOADS.items():
-            Ru = UkRunner(wu, dev)
-            ku = min(K, args.extra_steps)
-            tu, segu, _ = time_steps(Ru, ku, 3, flush)
-            msu = tu / ku
-            ru = roofline_of(Ru.w, segu, ku, pk, ffma)
-            others[nm] = {"ms_per_step": msu, "value": wu.edges / (msu / 1000.0), "unit": UNIT, "steps": ku,
-                          "dtype": wu.dtype, "dominant": ru["kernel"], "bound": ru["bound"], "frac": ru["frac"],
-                          "segment_ms": ru["segment_ms"], "step_roofline": step_roofline(Ru.w, msu, pk, ffma),
-                          "window": {"q0": Ru.q0, "nq": Ru.nq, "G": Ru.ks.G, "basis_per_input": Ru.nq * wu.group},
-                          "note": "generator window sized once before the timed steps; step = generate + layer "
-                                  "forward + layer backward + generator backward"}
-            del Ru
-            torch.cuda.empty_cache()
+        for nm in EXTRA_WORKLOADS + sorted(W.GR_WORKLOADS) + sorted(W.UK_WORKLOADS):
+            if nm != w.name:
+                others[nm] = time_other(nm, dev, min(K, args.extra_steps), flush, pk, ffma)
 
     st = R_status()
     if st != 0:
@@ -832,6 +852,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None,
+                    choices=sorted(set(W.WORKLOADS) | set(W.GR_WORKLOADS) | set(W.UK_WORKLOADS)),
+                    help="time one workload by itself (one GPU) and print its own JSON line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -840,6 +863,10 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.only:
+            if world > 1:
+                raise SystemExit("--only runs on one GPU")
+            run_only(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

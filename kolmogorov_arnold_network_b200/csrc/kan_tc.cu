@@ -14,9 +14,12 @@
 // layout the tensor core reads.  The dense expansion costs little on tensor
 // cores, and the per-input work stays O(k+1) whatever G is.
 //
-// One kernel template serves the four GEMMs:
+// One kernel template serves five GEMMs:
 //   FWD    A = basis rows (producers)  B = coef / w_base, K-major (TMA)
 //   DCA    A = basis^T (producers)     B = dY (TMA)
+//   DCB    A = dY^T, MN-major (TMA)    B = basis^T (producers): dcoef with
+//          the outputs on M and the spline columns on N (bf16, no SiLU
+//          branch), for `out` that wide N tiles would pad or split unevenly
 //   DX     A = dY, K-major (TMA)       B = coef, MN-major (TMA); B'-gather epilogue
 //   GEMM   A = dY, K-major (TMA)       B = w_base, MN-major (TMA); fp32 store
 // Warp roles: 0 TMA, 1 MMA issue + TMEM allocation, then the A producers
@@ -66,7 +69,7 @@ constexpr int kBM = 128;          // MMA M: rows of A, TMEM lanes
 // Producer warps per mode: the row producers (FWD, DCA) run 4 groups of 4
 // warps that take every 4th k-block; the TMA-fed modes keep 8 idle warps.
 template <int MODE> struct Warps {
-    static constexpr int kProd = (MODE == 0 || MODE == 4) ? 16 : 8;   // FWD, DCA : others
+    static constexpr int kProd = (MODE == 0 || MODE == 4 || MODE == 5) ? 16 : 8;   // FWD, DCA, DCB : others
     static constexpr int kGroups = kProd / 4;
     static constexpr int kEpi0 = 2 + kProd;                            // first epilogue warp
     static constexpr int kThreads = (kEpi0 + 4) * 32;
@@ -78,7 +81,7 @@ constexpr int kSmemBudget = 227 * 1024 - 2048;
 // DCA (bf16): dcoef = A^T . dY with M = spline columns (then SiLU rows), N =
 // outputs, K = batch; the basis operand is written MN-major by the producers
 // (rows = batch, 64-column atoms of spline columns), dY is read MN-major.
-enum Mode { FWD = 0, DX = 2, GEMM = 3, DCA = 4 };
+enum Mode { FWD = 0, DX = 2, GEMM = 3, DCA = 4, DCB = 5 };
 
 template <int DT> struct Cfg;
 template <> struct Cfg<KAN_BF16> {
@@ -174,6 +177,8 @@ struct TcArgs {
     int fbox;                  // FWD: rows per B box
     int pair;                  // FWD, DCA (bf16): CTA pairs sharing cta_group::2 MMAs
     int m_tiles;               // FWD, DCA: M tiles holding work (a pair grid may have one more)
+    int store_tma;             // FWD (unsplit), DCB: the output tile leaves through TMA stores of
+                               // 128-row x 128-byte boxes (tensor map tA_hi over y or dcoef)
 };
 
 // (offset arithmetic on the shared array itself, not an integer round trip, so
@@ -450,6 +455,56 @@ __device__ __forceinline__ uint4 chunk8(uint64_t P, int s)
     return make_uint4((uint32_t)lo, (uint32_t)(lo >> 32), (uint32_t)hi, (uint32_t)(hi >> 32));
 }
 
+// bf16 placement by byte permutes: the packed weights of an input sit in two
+// words (w0, w1 | w2, w3), and each 32-bit word of the input's 16-byte chunk
+// is one prmt of those two words under a selector that depends on the span s
+// alone.  The selectors of span s are entry s + 3 (s in -3..7) of a 12-entry
+// table in shared memory; entry 11 stores zeros (an input outside the
+// extended knots).  A selector nibble with its top bit set copies the sign
+// bit of the byte it names into the whole byte, and nibble 9 names the high
+// byte of w0, whose sign is clear (the weights are nonnegative): a zero byte.
+constexpr int kSelEntries = 12;
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Selector of output word e (columns 2e, 2e+1) for table entry t.
+__device__ __forceinline__ uint32_t sel_word(int t, int e)
+{
+    if (t >= kSelEntries - 1) return 0x9999u;
+    const int s = t - 3;
+    uint32_t sel = 0;
+    for (int h = 0; h < 2; ++h) {
+        const int q = 2 * e + h - s;   // weight index landing in column 2e + h
+        const bool in = q >= 0 && q <= 3;
+        const uint32_t lo = in ? 2u * q : 9u, hi = in ? 2u * q + 1u : 9u;
+        sel |= (lo | (hi << 4)) << (8 * h);
+    }
+    return sel;
+}
+
+// bf16 weights of one input as two packed words and its selector-table entry
+// (kSelEntries - 1 when the input is outside the extended knots or not real).
+__device__ __forceinline__ void input_prmt(float x, bool act, float inv_h, float u0, float u_hi, uint32_t& entry,
+                                           uint32_t& p0, uint32_t& p1)
+{
+    float u = fmaf(x, inv_h, u0);
+    const bool ok = act && u >= -3.0f && u < u_hi;
+    u = ok ? u : 0.0f;   // (keeps w0 nonnegative, whose sign byte the zero selectors read)
+    int s;
+    float f;
+    floor_split(u, s, f);
+    float w[4];
+    weights_fma(u - f, w);
+    p0 = pack_bf16(w[0], w[1]);
+    p1 = pack_bf16(w[2], w[3]);
+    entry = ok ? (uint32_t)(s + 3) : (uint32_t)(kSelEntries - 1);
+}
+
 // The packed weights of one input for chunk8 (bf16, or the fp16 hi / lo parts
 // of the fp32 path): span s and, when the input is outside the extended knots
 // (or not a real input), P = 0.
@@ -520,20 +575,24 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     constexpr int BK = C::BK;
     constexpr int EPB = 128 / C::ESZ;               // elements per 128-byte row
     constexpr bool F32 = DT == KAN_F32;
-    constexpr bool PRODUCE = MODE == FWD || MODE == DCA;
+    constexpr bool PRODUCE = MODE == FWD || MODE == DCA || MODE == DCB;
+    // DCB: the produced ring holds the B operand and the TMA ring the A operand
+    constexpr bool SWAP = MODE == DCB;
+    static_assert(!SWAP || (PAIR && DT == KAN_BF16 && KD == 3), "DCB: bf16 cubic 1-D, CTA pairs");
     constexpr bool TWOD = KD == 32;
     static_assert(!TWOD || PRODUCE, "2-D surfaces: produced-A kernels only");
     constexpr bool A_BY_TMA = MODE == DX || MODE == GEMM;
     static_assert(!PAIR || (PRODUCE && DT == KAN_BF16), "CTA pairs: bf16 forward and dcoef only");
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
-    constexpr bool A_MN = MODE == DCA;               // producer-written MN-major basis
+    constexpr bool A_MN = MODE == DCA || MODE == DCB;   // producer-written basis^T, or dY^T (DCB)
     constexpr bool A_SW32 = false;                   // (2-byte operands: the plain 128-byte swizzle)
     // B stored MN-major (dY for dcoef, coef / w_base for dx), for both dtypes
     // (the fp32 path's fp16 split copies keep the source layout)
     constexpr bool B_MN = MODE != FWD;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
+    __shared__ uint4 sel_tab[kSelEntries];   // bf16 chunk placement (see input_prmt)
 
     // Two rings of pipeline stages: B (TMA) with `stages` slots, and A with
     // `sa_n` slots.  A produced tile (FWD, DCA) is small next to a wide B tile,
@@ -543,7 +602,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
     const int BN = a.BN, stages = a.stages;
     const int sa_n = PRODUCE ? a.stages_a : a.stages;
     // (a CTA of a pair holds half of each N = 256 MMA's B rows)
-    const uint32_t a_bytes = kBM * 128, b_bytes = (uint32_t)(PAIR ? BN / 2 : BN) * 128;
+    // (DCB: the produced A ring carries the B operand, bn_cta columns, and the TMA ring dY^T, kBM rows)
+    const uint32_t bn_cta = (uint32_t)(PAIR ? BN / 2 : BN) * 128;
+    const uint32_t a_bytes = SWAP ? bn_cta : kBM * 128, b_bytes = SWAP ? kBM * 128 : bn_cta;
     const uint32_t a_stage = a_bytes * C::SPLIT, b_stage = b_bytes * C::SPLIT;
     const uint32_t sbase = smem_addr(smem);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sa_n * a_stage + stages * b_stage);
@@ -574,6 +635,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         F32 ? 512u : (BN <= 32 ? 32u : (BN <= 64 ? 64u : (BN <= 128 ? 128u : (BN <= 256 ? 256u : 512u))));
 
     if (threadIdx.x == 0) {
+        if constexpr (PRODUCE && !F32)
+            for (int t = 0; t < kSelEntries; ++t)
+                sel_tab[t] = make_uint4(sel_word(t, 0), sel_word(t, 1), sel_word(t, 2), sel_word(t, 3));
         for (int s = 0; s < stages; ++s) {
             mbar_init(full(s), 1);          // the TMA thread's expect-tx arrival
             mbar_init(empty(s), 1);         // the MMA thread's commit
@@ -643,7 +707,11 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     if (leader) mbar_arrive_expect_tx(full(s), 2u * b_bytes);
                     const int h2 = (BN - 256) / 2;
                     auto tile_col = [&](int lc) { return lc < 128 ? 128 * (int)rank + lc : 256 + h2 * (int)rank + lc - 128; };
-                    if (MODE == FWD) {
+                    if (SWAP) {
+                        // this CTA's 128 rows of dY^T: two 64-output atoms of BK batch rows
+                        for (int c = 0; c < kBM / EPB; ++c)
+                            tma_load_2d_pair(B_hi(s) + (uint32_t)c * BK * 128u, &tB_hi, fl, (int)m0 + c * EPB, kb * BK);
+                    } else if (MODE == FWD) {
                         const bool spline = kb < a.nkb_main;   // (then the SiLU k-blocks, w_base)
                         for (int lc = 0; lc < BN / 2; lc += a.fbox)
                             tma_load_2d_pair(B_hi(s) + (uint32_t)lc * 128u,
@@ -740,8 +808,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 // descriptors of the stage's tiles; the k-steps advance the start address
                 // field (addresses stay below 2^18, so the field never carries)
                 const int sA = PRODUCE ? sa : s;
-                const uint64_t ad0 = smem_desc(A_hi(sA), a_lbo, a_sbo, a_layout);
-                const uint64_t bd0 = smem_desc_sw128(B_hi(s), b_lbo, 1024);
+                const uint64_t ad0 = smem_desc(SWAP ? B_hi(s) : A_hi(sA), a_lbo, a_sbo, a_layout);
+                const uint64_t bd0 = smem_desc_sw128(SWAP ? A_hi(sa) : B_hi(s), b_lbo, 1024);
                 const uint64_t adl0 = F32 ? smem_desc(A_lo(sA), a_lbo, a_sbo, a_layout) : 0;
                 const uint64_t bdl0 = F32 ? smem_desc_sw128(B_lo(s), b_lbo, 1024) : 0;
 #pragma unroll
@@ -794,12 +862,17 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 else mma_commit(accum_bar);
             }
         }
-    } else if (warp < Warps<MODE>::kEpi0) {
+    } else {
         // ---------------- A producers ----------------
+        // Warps 2 .. kEpi0-1 in groups of four and, with bf16 operands, the
+        // epilogue warps as one more group until the last k-block is filled
+        // (they have nothing else to do before the accumulator is complete; the
+        // fp32 epilogue promotes accumulator segments meanwhile).
         // Each thread fetches the x values of its next k-block into registers
         // before it waits for and fills the current one, so the global-load
         // latency overlaps the previous k-block's work.
-        if constexpr (PRODUCE) {
+        const bool producer_warp = warp < Warps<MODE>::kEpi0;
+        if constexpr (PRODUCE) if (producer_warp || !F32) {
             const int p = threadIdx.x - 64;
             const T* X = reinterpret_cast<const T*>(a.x);
             const float sx = F32 ? scales_of(a.amax).x : 1.0f;   // scale of the SiLU values (fp32)
@@ -841,7 +914,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 // than the previous use of the A slot it waits for, so neither the
                 // aempty barrier nor any other can be two phases behind (a parity
                 // wait on such a barrier would pass early).
-                const int NG = min(Warps<MODE>::kGroups, sa_n);
+                const int NG = min(Warps<MODE>::kGroups + (F32 ? 0 : 1), sa_n);
                 if (grp < NG && grp < nk) fetch(kb_begin + grp);
                 int uses = 0;                               // k-blocks this group has filled
                 for (int it = grp; grp < NG && it < nk; it += NG, ++uses) {
@@ -866,15 +939,20 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         const int n8 = row_ok ? min(8, (int)a.in - first_input(kb)) : 0;
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
-                            int sidx;
-                            uint64_t Ph, Pl;
-                            input_chunk<DT>(xv[c], c < n8, a.inv_h, u0, u_hi, sidx, Ph, Pl);
                             const uint32_t off = sw128_chunk(row, (uint32_t)c);
-                            const uint4 vh = chunk8(Ph, sidx);
-                            st_shared_v4(ahi + off, vh.x, vh.y, vh.z, vh.w);
                             if constexpr (F32) {
-                                const uint4 vl = chunk8(Pl, sidx);
+                                int sidx;
+                                uint64_t Ph, Pl;
+                                input_chunk<DT>(xv[c], c < n8, a.inv_h, u0, u_hi, sidx, Ph, Pl);
+                                const uint4 vh = chunk8(Ph, sidx), vl = chunk8(Pl, sidx);
+                                st_shared_v4(ahi + off, vh.x, vh.y, vh.z, vh.w);
                                 st_shared_v4(alo + off, vl.x, vl.y, vl.z, vl.w);
+                            } else {
+                                uint32_t t, p0, p1;
+                                input_prmt(xv[c], c < n8, a.inv_h, u0, u_hi, t, p0, p1);
+                                const uint4 sel = sel_tab[t];
+                                st_shared_v4(ahi + off, prmt(p0, p1, sel.x), prmt(p0, p1, sel.y), prmt(p0, p1, sel.z),
+                                             prmt(p0, p1, sel.w));
                             }
                         }
                     } else if (kb < a.nkb_main) {
@@ -1001,7 +1079,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 auto col_off = [&](int c) -> uint32_t {
                     return sw128_byte((uint32_t)rb, (uint32_t)c * 2u) - (uint32_t)rb * 128u;
                 };
-                const int NG = min(Warps<MODE>::kGroups, sa_n);   // see the forward producer
+                const int NG = min(Warps<MODE>::kGroups + (F32 ? 0 : 1), sa_n);   // see the forward producer
                 if (grp < NG && grp < nk) fetch(kb_begin + grp);
                 for (int it = grp; grp < NG && it < nk; it += NG) {
                     float cur[MAXI];
@@ -1025,15 +1103,20 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         const int n8 = row_ok ? n_inp : 0;
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
-                            int sidx;
-                            uint64_t Ph, Pl;
-                            input_chunk<DT>(xv[c], c < n8, a.inv_h, u0, u_hi, sidx, Ph, Pl);
                             const uint32_t off = (((uint32_t)c ^ ((uint32_t)rb & 7u)) << 4);
-                            const uint4 vh = chunk8(Ph, sidx);
-                            st_shared_v4(rb_hi + off, vh.x, vh.y, vh.z, vh.w);
                             if constexpr (F32) {
-                                const uint4 vl = chunk8(Pl, sidx);
+                                int sidx;
+                                uint64_t Ph, Pl;
+                                input_chunk<DT>(xv[c], c < n8, a.inv_h, u0, u_hi, sidx, Ph, Pl);
+                                const uint4 vh = chunk8(Ph, sidx), vl = chunk8(Pl, sidx);
+                                st_shared_v4(rb_hi + off, vh.x, vh.y, vh.z, vh.w);
                                 st_shared_v4(rb_lo + off, vl.x, vl.y, vl.z, vl.w);
+                            } else {
+                                uint32_t t, p0, p1;
+                                input_prmt(xv[c], c < n8, a.inv_h, u0, u_hi, t, p0, p1);
+                                const uint4 sel = sel_tab[t];
+                                st_shared_v4(rb_hi + off, prmt(p0, p1, sel.x), prmt(p0, p1, sel.y),
+                                             prmt(p0, p1, sel.z), prmt(p0, p1, sel.w));
                             }
                         }
                     } else if (!silu_tile) {
@@ -1168,9 +1251,106 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(afull(s), 0));
                     else mbar_arrive(afull(s));
                 }
+            } else if constexpr (MODE == DCB) {
+                // B tile, MN-major: batch rows b0..b0+BK-1 (K) by this CTA's bn_cta spline
+                // columns (N) in atoms of EPB = 64 columns, BK*128 bytes apart; a pair's CTA
+                // holds tile columns 128*rank + [0, 128) and 256 + h2*rank + [0, BN/2 - 128)
+                // (the halves of each N = 256 MMA).  Groups of 128 threads take k-blocks in
+                // turn; a thread fills the rows of batch row rb in atoms a0 and a0 + 2.
+                const int NAT = (PAIR ? BN / 2 : BN) / EPB;
+                const int grp = p >> 7;                    // warp-uniform
+                const int rb = p % BK;
+                const int a0 = (p / BK) & 1;               // warp-uniform
+                const int h2 = (BN - 256) / 2;
+                const float u0 = -a.lo * a.inv_h;
+                const float u_lo = -3.0f, u_hi = (float)(a.G + 3);
+                int c_lo[2], n_inp[2], i_first[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int at = a0 + 2 * e;
+                    const int lc = at * EPB;
+                    c_lo[e] = n0 + (lc < 128 ? 128 * (int)rank + lc : 256 + h2 * (int)rank + lc - 128);
+                    const int c_end = min(c_lo[e] + EPB, a.Kt);
+                    i_first[e] = (int)__umulhi((uint32_t)c_lo[e], a.nb_magic);
+                    n_inp[e] = (at < NAT && c_lo[e] < c_end)
+                                   ? (int)__umulhi((uint32_t)(c_end - 1), a.nb_magic) - i_first[e] + 1 : 0;
+                }
+                XWindow<T, MAXI> nxw[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    nxw[e].o = -1;
+#pragma unroll
+                    for (int j = 0; j < XWindow<T, MAXI>::NR; ++j) nxw[e].raw[j] = 0u;
+                }
+                auto fetch = [&](int kb) {
+                    const int64_t b = (int64_t)kb * BK + rb;
+                    if (b >= a.batch) return;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        if (n_inp[e] > 0) nxw[e].issue(X + b * a.in, i_first[e], n_inp[e], (int)a.in, a.x_vec != 0);
+                };
+                const bool chunked = MAXI == 9 && a.nb == 8 && a.x_vec;
+                const int NG = min(Warps<MODE>::kGroups + (F32 ? 0 : 1), sa_n);   // see the forward producer
+                if (grp < NG && grp < nk) fetch(kb_begin + grp);
+                for (int it = grp; grp < NG && it < nk; it += NG) {
+                    const XWindow<T, MAXI> cur_raw[2] = {nxw[0], nxw[1]};
+                    const int kb = kb_begin + it;
+                    if (it + NG < nk) fetch(kb + NG);
+                    const int s = it % sa_n;
+                    const uint32_t ph = (it / sa_n) & 1;
+                    if (!acquire(s, ph)) break;
+                    const int64_t b = (int64_t)kb * BK + rb;
+                    const bool row_ok = b < a.batch;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int at = a0 + 2 * e;
+                        if (at >= NAT) continue;
+                        const uint32_t rbase = A_hi(s) + (uint32_t)at * BK * 128u + (uint32_t)rb * 128u;
+                        const int n8 = row_ok ? n_inp[e] : 0;
+                        if (chunked) {
+                            float xv[8];
+                            aligned8(cur_raw[e], xv);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                uint32_t t, p0, p1;
+                                input_prmt(xv[c], c < n8, a.inv_h, u0, u_hi, t, p0, p1);
+                                const uint4 sel = sel_tab[t];
+                                st_shared_v4(rbase + (((uint32_t)c ^ ((uint32_t)rb & 7u)) << 4), prmt(p0, p1, sel.x),
+                                             prmt(p0, p1, sel.y), prmt(p0, p1, sel.z), prmt(p0, p1, sel.w));
+                            }
+                        } else {
+                            float cur[MAXI];
+                            cur_raw[e].values(cur);
+                            zero_row<DT>(rbase, rbase, (uint32_t)rb & 7u);
+                            const int cbase = i_first[e] * a.nb - c_lo[e];
+#pragma unroll
+                            for (int k = 0; k < MAXI; ++k) {
+                                float u = fmaf(cur[k], a.inv_h, u0);
+                                const bool ok = k < n8 && u >= u_lo && u < u_hi;   // NaN, inf fail
+                                u = ok ? u : 0.0f;
+                                int sidx;
+                                float f, w[4];
+                                floor_split(u, sidx, f);
+                                weights_fma(u - f, w);
+                                const int base = cbase + k * a.nb;
+                                const int mlo = ok ? max(0, -base) : 0;
+                                const uint32_t width = ok ? (uint32_t)(min(a.nbs, EPB - base) - mlo) : 0u;
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    if ((uint32_t)(sidx + q - mlo) < width)
+                                        st_shared_u16(rbase + (uint32_t)(sw128_byte((uint32_t)rb, (uint32_t)(base + sidx + q) * 2u) -
+                                                                         (uint32_t)rb * 128u),
+                                                      __bfloat16_as_ushort(__float2bfloat16_rn(w[q])));
+                            }
+                        }
+                    }
+                    fence_async_smem();
+                    if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(afull(s), 0));
+                    else mbar_arrive(afull(s));
+                }
             }
         }
-    } else {
+        if (!producer_warp) {
         // ---------------- epilogue: the last 4 warps ----------------
         const int q = warp & 3;                       // TMEM lane quarter
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
@@ -1255,7 +1435,61 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 }
             };
 
-            if constexpr (MODE == FWD || MODE == GEMM) {
+            // The output tile through shared memory and TMA stores: boxes of 128 rows x
+            // 128 bytes (32 fp32 or 64 bf16 columns) in a ring of 8 slots at the start of
+            // the pipeline buffers (idle once the accumulator is complete), written in
+            // the 128-byte swizzle (conflict-free), stored by one thread; whole lines
+            // leave the SM instead of one 16-byte piece per row and store.
+            auto store_tile = [&](bool bf16_out, float mul) {
+                const int cpb = bf16_out ? 64 : 32;
+                const bool issuer = warp == Warps<MODE>::kEpi0 && lane == 0;
+                const int nslot = min(8, (int)((sa_n * a_stage + stages * b_stage) >> 14));   // 16 KB slots
+                int box = 0;
+                for (int c1 = 0; c1 < BN; c1 += cpb, ++box) {
+                    const uint32_t slot = sbase + (uint32_t)(box % nslot) * 16384u;
+                    if (box >= nslot) {   // the store that used this slot has read it
+                        if (issuer) {
+                            if (nslot == 8) bulk_wait_read<7>();
+                            else bulk_wait_read<0>();
+                        }
+                        named_bar_sync(1, kEpi);
+                    }
+                    uint32_t wv[32];
+                    if (bf16_out) {
+                        float va[32], vb[32];
+                        load32(c1, va, mul);
+                        load32(c1 + 32, vb, mul);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            wv[e] = pack_bf16(va[2 * e], va[2 * e + 1]);
+                            wv[16 + e] = pack_bf16(vb[2 * e], vb[2 * e + 1]);
+                        }
+                    } else {
+                        float v[32];
+                        load32(c1, v, mul);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) wv[e] = __float_as_uint(v[e]);
+                    }
+                    const uint32_t rowp = slot + r * 128u;
+#pragma unroll
+                    for (uint32_t c = 0; c < 8; ++c)
+                        st_shared_v4(rowp + ((c ^ (r & 7u)) << 4), wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+                    fence_async_smem();
+                    named_bar_sync(1, kEpi);
+                    if (issuer) {
+                        // (a box wholly past the last row or column, e.g. a pair grid's padding
+                        // tile, is not stored; its group stays empty)
+                        if (m0 < (MODE == DCB ? a.out_f : a.batch) && n0 + c1 < (MODE == DCB ? (int64_t)a.Kt : a.out_f))
+                            tma_store_2d(&tA_hi, slot, n0 + c1, (int)m0);
+                        bulk_commit();
+                    }
+                }
+                if (issuer) bulk_wait_read<0>();   // the boxes are read before the CTA may exit
+            };
+
+            if (MODE == FWD && a.store_tma && !a.partial) {
+                store_tile(!F32, F32 ? 1.0f / scales_of(a.amax).c : 1.0f);
+            } else if constexpr (MODE == FWD || MODE == GEMM) {
                 const int64_t bo = m0 + r;
                 const int64_t ncols = MODE == FWD ? a.out_f : a.in;
                 const float mul = F32 ? 1.0f / scales_of(a.amax).c : 1.0f;   // y = acc / s_c
@@ -1310,6 +1544,31 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                         }
                     }
                 }
+                }
+            } else if constexpr (MODE == DCB) {
+                // rows are outputs j, columns spline columns kt: dcoef[j, n0 + c]
+                if (a.store_tma) {
+                    store_tile(false, 1.0f);
+                } else {
+                    const int64_t j = m0 + r;
+                    float* dst = reinterpret_cast<float*>(a.out) + (j < a.out_f ? j : 0) * a.Kt;
+                    const bool vec = (a.Kt & 3) == 0;
+                    for (int c1 = 0; c1 < BN; c1 += 32) {
+                        float v32[32];
+                        load32(c1, v32, 1.0f);
+                        if (j >= a.out_f || !a.out) continue;
+                        const int64_t k0 = n0 + c1;
+                        if (vec && k0 + 32 <= a.Kt) {
+#pragma unroll
+                            for (int e = 0; e < 32; e += 4)
+                                *reinterpret_cast<float4*>(dst + k0 + e) =
+                                    make_float4(v32[e], v32[e + 1], v32[e + 2], v32[e + 3]);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (k0 + e < a.Kt) dst[k0 + e] = v32[e];
+                        }
+                    }
                 }
             } else if constexpr (MODE == DCA) {
                 // rows are spline columns kt (or inputs of a SiLU tile); columns are outputs j
@@ -1420,6 +1679,7 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     }
                 }
             }
+        }
         }
     }
 
@@ -2185,6 +2445,25 @@ bool make_map_2d(CUtensorMap* m, const void* base, bool f16, int64_t rows, int64
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
+// Tensor map for the TMA-store epilogue: an output matrix [rows, cols] (fp32, or
+// bf16 for y) in boxes of 128 rows x 128 bytes, 128-byte swizzle.  False (and
+// the caller stores directly) when TMA cannot address it: a row length that is
+// not a multiple of 16 bytes or a base that is not 16-byte aligned.
+bool make_store_map(CUtensorMap* m, void* base, bool f32, int64_t rows, int64_t cols)
+{
+    const int esz = f32 ? 4 : 2;
+    if (!base || (cols * esz) % 16 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
+    auto enc = get_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * esz)};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)kBM};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Split-K count s (1..cap) minimising the estimated time
 //   waves(s) / s * t_tile  +  waves(s) * t_wave  +  (s > 1 ? 2 (s + 1) t_part : 0),
 // waves(s) = ceil(tiles * s / sms); t_tile: one whole output tile's contraction
@@ -2218,6 +2497,19 @@ int pick_splits(int64_t tiles, int sms, int cap, double t_tile, double t_part)
 // fp32 partials of `tiles` such tiles at HBM rate.
 double tile_seconds(int BN, int64_t K, bool f32) { return 2.0 * kBM * BN * (double)K * (f32 ? 3 : 1) / 9.0e12; }
 double partial_seconds(int64_t tiles, int BN) { return (double)tiles * kBM * BN * 4.0 / 5.0e12; }
+
+// Tensor-core cycles per SM of one k-block (four K = 16 steps) of a CTA-pair tile
+// BN columns wide, issued as instructions of N <= 256: about 161 cycles for
+// N = 256 and about 97 for any N <= 128 (in between by interpolation).
+double kblock_cycles(int BN)
+{
+    double c = 0.0;
+    for (int n = BN; n > 0; n -= 256) {
+        const int m = std::min(n, 256);
+        c += m > 128 ? 97.0 + (m - 128) * 0.5 : 97.0;
+    }
+    return 4.0 * c;
+}
 
 // Tile width over n output columns.  An MN-major bf16 B operand is loaded in
 // 64-column (128-byte) boxes, so its tile is at least one box wide.
@@ -2274,6 +2566,13 @@ int smem_bytes(int BN, int stages, int stages_a, bool f32)
     return (stages * BN * 128 + stages_a * kBM * 128) * (f32 ? 2 : 1) + 1024 + 512;
 }
 
+// DCB (bf16 pairs): `stages` TMA slots of kBM dY^T rows and `stages_a` produced
+// slots of bn_cta basis columns (64-column atoms of BK batch rows)
+int smem_bytes_dcb(int bn_cta, int stages, int stages_a)
+{
+    return stages * kBM * 128 + stages_a * bn_cta * 128 + 1024 + 512;
+}
+
 
 // Workspace layout, shared by the size query and the launches.
 struct Layout {
@@ -2298,6 +2597,9 @@ struct Plan {
     // dcoef
     int d_BN, d_stages, d_stages_a, d_n, d_m, d_nkt, d_splits, d_kps, d_nkb;
     int64_t d_ld;
+    // dcoef as DCB (outputs on M, spline columns on N), when that runs fewer tensor-core cycles
+    bool dcb;
+    int b_BN, b_stages, b_stages_a, b_m, b_my, b_n;
     // dx
     int x_BN, x_stages, x_n, x_m, x_nin, x_nkb;
     // dx, persistent kernel (used when p_ok)
@@ -2351,6 +2653,31 @@ Plan make_plan(const Problem& p, int sms)
     P.d_kps = (int)cdiv(std::max(1, P.d_nkb), P.d_splits);
     P.d_splits = (int)cdiv(std::max(1, P.d_nkb), P.d_kps);
     P.d_ld = P.ext ? P.Kx : p.Kt + (p.base ? p.in : 0);
+    // DCB (bf16 cubic 1-D without the SiLU branch, G >= 5): M = outputs, N = spline columns in
+    // 512-column pair tiles, K = batch, no split; taken when its waves of pair tiles
+    // times the tile's k-block cycles undercut the DCA plan's by 5% (an `out` that
+    // 512-column tiles would pad, e.g. 768 as two 384-column tiles)
+    P.dcb = false;
+    if (!f32 && !p.base && p.k == 3 && p.dims == 1 && P.nbx >= 8) {
+        const int64_t slots = std::max(1, sms / 2);
+        const int bBN = 512;
+        const int b_m = (int)cdiv(p.out, kBM);
+        const int b_my = (b_m + 1) / 2 * 2;
+        const int b_n = (int)cdiv(p.Kt, bBN);
+        const int64_t dca_ctas = (P.d_pair ? (int64_t)P.d_my : (int64_t)P.d_m) * P.d_n * P.d_splits;
+        const double c_dca = (double)cdiv(P.d_pair ? dca_ctas / 2 : dca_ctas, P.d_pair ? slots : 2 * slots) *
+                             (double)P.d_kps * kblock_cycles(P.d_BN);
+        const double c_dcb = (double)cdiv((int64_t)b_my / 2 * b_n, slots) * (double)P.d_nkb * kblock_cycles(bBN);
+        if (c_dcb < 0.95 * c_dca) {
+            P.dcb = true;
+            P.b_BN = bBN;
+            P.b_m = b_m;
+            P.b_my = b_my;
+            P.b_n = b_n;
+            P.b_stages = 3;
+            P.b_stages_a = std::min(8, (kSmemBudget - 1024 - 512 - P.b_stages * kBM * 128) / (bBN / 2 * 128));
+        }
+    }
     // dx: M = batch, N = whole inputs' columns, K = out; coef (or its fp16
     // copies) is read MN-major and a tile's first column is rounded down to 16 bytes
     P.x_BN = f32 ? 128 : 256;
@@ -2422,7 +2749,7 @@ Plan make_plan(const Problem& p, int sms)
         P.bwd.dy_hl = o;
         o += 2 * al256((size_t)p.batch * P.ldo * 2);
     }
-    if (P.d_splits > 1) {
+    if (P.d_splits > 1 && !P.dcb) {
         P.bwd.dc_part = o;
         o += al256((size_t)P.d_splits * p.out * P.d_ld * 4);
     }
@@ -2439,11 +2766,11 @@ inline int grid_for(int64_t n) { return (int)std::min<int64_t>(std::max<int64_t>
 template <int MODE, int DT, int MAXI, bool PAIR, int KD>
 cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args, cudaStream_t st)
 {
-    constexpr bool produce = MODE == FWD || MODE == DCA;
+    constexpr bool produce = MODE == FWD || MODE == DCA || MODE == DCB;
     const int stages_a = produce ? args.stages_a : stages;
     // the MN-major bf16 B operand arrives in whole 128-byte boxes: BN must be a multiple of 64
     if (MODE != FWD && BN % 64 != 0) return cudaErrorInvalidConfiguration;
-    if (BN % 16 != 0 || BN < 16 || BN > (MODE == FWD || MODE == DCA ? 512 : 256) || (BN > 256 && BN % 128 != 0) ||
+    if (BN % 16 != 0 || BN < 16 || BN > (produce ? 512 : 256) || (BN > 256 && BN % 128 != 0) ||
         (DT == KAN_F32 && BN > 128) || stages < 2 || stages_a < 2 || stages + stages_a > 24 ||
         (!produce && stages_a != stages))
         return cudaErrorInvalidConfiguration;
@@ -2451,7 +2778,9 @@ cudaError_t launch(dim3 grid, int BN, int stages, const CUtensorMap* maps, const
     if (PAIR && (BN < 256 || BN % 128 != 0 || (MODE == FWD && args.fbox != (BN == 384 ? 64 : 128)) ||
                  grid.x % 2 != 0))
         return cudaErrorInvalidConfiguration;
-    const int smem = smem_bytes(PAIR ? BN / 2 : BN, stages, stages_a, DT == KAN_F32);
+    // (DCB: the TMA ring holds kBM-row dY^T tiles and the produced ring the B columns)
+    const int smem = MODE == DCB ? smem_bytes_dcb(BN / 2, stages, stages_a)
+                                 : smem_bytes(PAIR ? BN / 2 : BN, stages, stages_a, DT == KAN_F32);
     if (smem > kSmemBudget) return cudaErrorInvalidConfiguration;
     static int configured = 0;   // per instantiation; the attribute is per function
     if (configured < smem) {
@@ -2493,23 +2822,30 @@ template <int MODE, int MAXI, int KD>
 cudaError_t launch_m(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
                      cudaStream_t st)
 {
-    if (f32) return launch<MODE, KAN_F32, MAXI, false, KD>(grid, BN, stages, maps, args, st);
-    if constexpr (MODE == FWD || MODE == DCA) {
-        if (args.pair) return launch<MODE, KAN_BF16, MAXI, true, KD>(grid, BN, stages, maps, args, st);
+    if constexpr (MODE == DCB) {   // bf16 CTA pairs only
+        if (f32 || !args.pair) return cudaErrorInvalidConfiguration;
+        return launch<DCB, KAN_BF16, MAXI, true, KD>(grid, BN, stages, maps, args, st);
+    } else {
+        if (f32) return launch<MODE, KAN_F32, MAXI, false, KD>(grid, BN, stages, maps, args, st);
+        if constexpr (MODE == FWD || MODE == DCA) {
+            if (args.pair) return launch<MODE, KAN_BF16, MAXI, true, KD>(grid, BN, stages, maps, args, st);
+        }
+        return launch<MODE, KAN_BF16, MAXI, false, KD>(grid, BN, stages, maps, args, st);
     }
-    return launch<MODE, KAN_BF16, MAXI, false, KD>(grid, BN, stages, maps, args, st);
 }
 
 template <int MODE, int KD>
 cudaError_t launch_k(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
                      cudaStream_t st)
 {
-    if constexpr (MODE == FWD || MODE == DCA) {
+    if constexpr (MODE == FWD || MODE == DCA || MODE == DCB) {
         const int need = fwd_maxi_needed(args.nb, KD == 32);
         if (need <= 4) return launch_m<MODE, 4, KD>(f32, grid, BN, stages, maps, args, st);
         if (need <= 7) return launch_m<MODE, 7, KD>(f32, grid, BN, stages, maps, args, st);
         if (need <= 9) return launch_m<MODE, 9, KD>(f32, grid, BN, stages, maps, args, st);
-        if (need <= 17) return launch_m<MODE, 17, KD>(f32, grid, BN, stages, maps, args, st);
+        // (DCB keeps two x windows per thread: planned for nb >= 8 only)
+        if constexpr (MODE != DCB)
+            if (need <= 17) return launch_m<MODE, 17, KD>(f32, grid, BN, stages, maps, args, st);
         return cudaErrorInvalidConfiguration;   // nb >= 4 keeps need <= 17
     } else {
         return launch_m<MODE, 1, KD>(f32, grid, BN, stages, maps, args, st);
@@ -2522,13 +2858,18 @@ template <int MODE>
 cudaError_t launch_dt(bool f32, dim3 grid, int BN, int stages, const CUtensorMap* maps, const TcArgs& args,
                       cudaStream_t st)
 {
-    if (args.twod) {   // 2-D surfaces: produced-A kernels only (dx runs persistent)
-        if constexpr (MODE == FWD || MODE == DCA) return launch_k<MODE, 32>(f32, grid, BN, stages, maps, args, st);
+    if constexpr (MODE == DCB) {   // cubic 1-D only
+        if (args.twod || args.k != 3) return cudaErrorInvalidConfiguration;
+        return launch_k<DCB, 3>(f32, grid, BN, stages, maps, args, st);
+    } else {
+        if (args.twod) {   // 2-D surfaces: produced-A kernels only (dx runs persistent)
+            if constexpr (MODE == FWD || MODE == DCA) return launch_k<MODE, 32>(f32, grid, BN, stages, maps, args, st);
+            return cudaErrorInvalidConfiguration;
+        }
+        if (MODE == GEMM || args.k == 3) return launch_k<MODE, 3>(f32, grid, BN, stages, maps, args, st);
+        if constexpr (MODE != GEMM) return launch_k<MODE, 0>(f32, grid, BN, stages, maps, args, st);
         return cudaErrorInvalidConfiguration;
     }
-    if (MODE == GEMM || args.k == 3) return launch_k<MODE, 3>(f32, grid, BN, stages, maps, args, st);
-    if constexpr (MODE != GEMM) return launch_k<MODE, 0>(f32, grid, BN, stages, maps, args, st);
-    return cudaErrorInvalidConfiguration;
 }
 
 template <int DT, bool PAIR, int KD>
@@ -2747,6 +3088,8 @@ cudaError_t tc_forward(const Problem& p, const void* x, const void* coef, const 
     a.partial = P.f_splits > 1;
     a.pair = P.f_pair ? 1 : 0;
     a.m_tiles = P.f_m;
+    // unsplit: y leaves through TMA stores when the tile is whole boxes wide and TMA can address y
+    a.store_tma = !a.partial && P.f_BN % (f32 ? 32 : 64) == 0 && make_store_map(&maps[0], y, f32, p.batch, p.out);
     const dim3 fgrid = P.f_pair ? dim3(P.f_my, P.f_n, P.f_splits) : dim3(P.f_n, P.f_m, P.f_splits);
     e = launch_dt<FWD>(f32, fgrid, P.f_BN, P.f_stages, maps, a, st);
     if (e != cudaSuccess) return e;
@@ -2819,10 +3162,24 @@ cudaError_t tc_backward(const Problem& p, const void* x, const void* coef, const
         a.out2 = dw_base;
         a.pair = P.d_pair ? 1 : 0;
         a.m_tiles = P.d_m;
-        const dim3 grid = P.d_pair ? dim3(P.d_my, P.d_n, P.d_splits) : dim3(P.d_n, P.d_m, P.d_splits);
-        e = launch_dt<DCA>(f32, grid, P.d_BN, P.d_stages, maps, a, st);
+        if (P.dcb) {
+            // outputs on M (dY^T by TMA through the same boxes), spline columns on N
+            a.BN = P.b_BN;
+            a.stages = P.b_stages;
+            a.stages_a = P.b_stages_a;
+            a.kb_per_split = P.d_nkb;
+            a.partial = 0;
+            a.out = dcoef;
+            a.pair = 1;
+            a.m_tiles = P.b_m;
+            a.store_tma = make_store_map(&maps[0], dcoef, true, p.out, p.Kt);
+            e = launch_dt<DCB>(false, dim3(P.b_my, P.b_n, 1), P.b_BN, P.b_stages, maps, a, st);
+        } else {
+            const dim3 grid = P.d_pair ? dim3(P.d_my, P.d_n, P.d_splits) : dim3(P.d_n, P.d_m, P.d_splits);
+            e = launch_dt<DCA>(f32, grid, P.d_BN, P.d_stages, maps, a, st);
+        }
         if (e != cudaSuccess) return e;
-        if (a.partial) {
+        if (a.partial && !P.dcb) {
             const dim3 rgrid((unsigned)std::min<int64_t>(cdiv(P.d_ld, 256), 64),
                              (unsigned)std::min<int64_t>(p.out, 65535));
             reduce_dcoef_kernel<<<rgrid, 256, 0, st>>>(partbuf, dcoef, dw_base, p.out, p.Kt, p.in, P.d_ld, P.d_splits,

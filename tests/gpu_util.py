@@ -52,10 +52,11 @@ def tile_rows(batch, tile=128):
 
 
 def tile_inputs(n_in, nb, tile=128):
-    """The inputs whose basis columns (nb per input) fall in the first two 128-column M tiles of the
-    dcoef GEMM (a whole CTA pair) or in its last M tile."""
+    """The inputs whose basis columns (nb per input) fall in the first four 128-column tiles of the
+    dcoef GEMM (a whole CTA pair of 128-column M tiles, and a whole 512-column N tile when the spline
+    columns run along N) or in its last 128-column tile."""
     kt = n_in * nb
-    cols = np.concatenate([np.arange(min(kt, 2 * tile)), np.arange(((kt - 1) // tile) * tile, kt)])
+    cols = np.concatenate([np.arange(min(kt, 4 * tile)), np.arange(((kt - 1) // tile) * tile, kt)])
     return np.unique(cols // nb)
 
 

@@ -292,6 +292,43 @@ def test_ffn_block_parity(oracle):
     assert e_end <= tol, e_end
 
 
+# dcoef with the outputs on M and the spline columns on N (the plan takes it for bf16 layers whose `out`
+# 512-column tiles would pad, when its waves of 512-column pair tiles are fewer): a ragged batch (last
+# k-block), a ragged last M tile (out = 648), a ragged last N tile (in * (G+3) not a multiple of 512),
+# rows of x not 16-byte aligned (the general producer) and G = 8 (11 columns per input)
+DCB_CASES = [
+    # batch, in, out, G, lo, hi
+    (300, 1536, 648, 5, -3.0, 3.0),
+    (257, 1532, 768, 5, -3.0, 3.0),
+    (300, 1024, 768, 8, -1.0, 1.0),
+]
+
+
+@pytest.mark.parametrize("case", DCB_CASES, ids=lambda c: "b{}_i{}_o{}_g{}".format(*c[:4]))
+def test_dcoef_outputs_on_m(oracle, case):
+    batch, n_in, n_out, G, lo, hi = case
+    w = W.custom(batch, n_in, n_out, G, lo, hi, dtype="bf16")
+    x, coef, _, dY = workload_inputs(w)
+    y, dx, dc, _ = gpu_layer(cuda(x), cuda(coef), None, cuda(dY), G, lo, hi)
+    torch.cuda.synchronize()
+    assert N.kan_sync_status(None) == 0
+    nb = G + 3
+    kt = n_in * nb
+    # the inputs of the first 512-column tile (both CTAs' halves), of one in the middle and of the last
+    # (ragged) one; every output, the padded M rows included
+    mid = (kt // 2) // 512 * 512
+    cols = np.concatenate([np.arange(512), np.arange(mid, mid + 512), np.arange((kt - 1) // 512 * 512, kt)])
+    ci = np.unique(cols // nb)
+    rows = np.union1d(tile_rows(batch), sample_rows(batch))
+    errs = check_layer_against_oracle(oracle, x, coef, None, dY, G, lo, hi, y.cpu(), dx.cpu(), dc.cpu(), None,
+                                      "bf16", rows=rows, cols_in=ci, cols_out=np.arange(n_out))
+    assert all(v <= TOL["bf16"] for v in errs.values()), errs
+    # bitwise repeatable
+    _, _, dc2, _ = gpu_layer(cuda(x), cuda(coef), None, cuda(dY), G, lo, hi)
+    torch.cuda.synchronize()
+    assert torch.equal(dc, dc2)
+
+
 # ---------------------------------------------------------------------------
 # properties that hold at any size
 @pytest.mark.parametrize("path", ["tensor", "simt"])
