@@ -24,7 +24,9 @@
 // the block reduces them with warp shuffles and one shared-memory pass in a
 // fixed order and writes one partial per block; a second kernel adds the
 // partials of every group in row-chunk order in fp64.  No atomics, and the
-// result is the same bit for bit on every run.  Every pass over HBM is a
+// result is the same bit for bit on every run.  Two elements of a vector
+// share their group's coefficients, so the arithmetic runs on element pairs
+// with the packed f32x2 instructions (half the FMA-pipe instructions).  Every pass over HBM is a
 // streaming read or write of whole 16-byte vectors: the kernels are bound by
 // HBM bandwidth.
 #include <cuda_bf16.h>
@@ -98,20 +100,46 @@ template <> struct Vec<__nv_bfloat16> {
 
 __device__ __forceinline__ uint4 ld_vec(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
+// Two fp32 lanes in one 64-bit register pair, operated on by the packed
+// f32x2 instructions of sm_100 (one instruction, two independent
+// round-to-nearest results): two elements of the same group share their
+// coefficients, so their arithmetic runs pairwise.
+using f2 = uint64_t;
+__device__ __forceinline__ f2 pk2(float a, float b)
+{
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void unpk2(f2 v, float& a, float& b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v)); }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c)
+{
+    f2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b)
+{
+    f2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 // Value and derivative of sum_i c_i x^i (i = 0..deg) by Horner's rule (the
-// better-conditioned order for the wide range of x^i); DMAX bounds the
-// unrolled loop, every index is a compile-time constant (c stays in registers).
+// better-conditioned order for the wide range of x^i), for two elements at
+// once; DMAX bounds the unrolled loop, every index is a compile-time constant
+// (c stays in registers).
 template <int DMAX, int NCO>
-__device__ __forceinline__ void horner_d(const float (&c)[NCO], int deg, float x, float& v, float& d)
+__device__ __forceinline__ void horner_d2(const f2 (&c)[NCO], int deg, f2 x, f2& v, f2& d)
 {
     static_assert(DMAX < NCO, "coefficient array too short");
-    v = 0.0f;
-    d = 0.0f;
+    v = 0ull;
+    d = 0ull;
 #pragma unroll
     for (int i = DMAX; i >= 0; --i) {
         if (i <= deg) {
-            d = fmaf(d, x, v);
-            v = fmaf(v, x, c[i]);
+            d = fma2(d, x, v);
+            v = fma2(v, x, c[i]);
         }
     }
 }
@@ -122,10 +150,12 @@ __device__ __forceinline__ void horner_d(const float (&c)[NCO], int deg, float x
 // vectors are loaded (and kept packed) before this step's arithmetic, so the
 // loads' latency hides behind it.
 template <typename T, bool BWD, int M1, int N>
-__global__ void __launch_bounds__(kThreads, BWD ? 3 : 4) grkan_kernel(const GrArgs a)
+__global__ void __launch_bounds__(kThreads, BWD ? (M1 ? 3 : 2) : 4) grkan_kernel(const GrArgs a)
 {
     constexpr int VEC = Vec<T>::N;
-    constexpr int RIF = BWD ? 1 : 2;                 // rows per step and thread
+    // rows per step and thread (the backward's fp32 rows, with half the elements per vector, take two
+    // rows per step to keep enough bytes in flight; measured faster than one on B200)
+    constexpr int RIF = BWD ? (sizeof(T) == 4 ? 2 : 1) : 2;
     const int m1 = M1 ? M1 : a.m1, n = N ? N : a.n;
     constexpr int MC = M1 ? M1 : kMaxNum;            // numerator coefficients, unroll bound
     constexpr int NC = N ? N : kMaxDen;              // denominator coefficients, unroll bound
@@ -141,15 +171,16 @@ __global__ void __launch_bounds__(kThreads, BWD ? 3 : 4) grkan_kernel(const GrAr
     if (tid < kMaxNum) sa[tid] = tid < m1 ? a.a[g * m1 + tid] : 0.0f;
     if (tid <= kMaxDen) sb[tid] = (tid >= 1 && tid <= n) ? a.b[g * n + tid - 1] : 0.0f;
     __syncthreads();
-    float ca[MC], cb[NC + 1];
+    f2 ca[MC], cb[NC + 1];
 #pragma unroll
-    for (int i = 0; i < MC; ++i) ca[i] = sa[i];
+    for (int i = 0; i < MC; ++i) ca[i] = pk2(sa[i], sa[i]);
 #pragma unroll
-    for (int i = 0; i <= NC; ++i) cb[i] = sb[i];
+    for (int i = 0; i <= NC; ++i) cb[i] = pk2(sb[i], sb[i]);
 
-    float acc[MC + NC];
+    // gradient terms, per lane of the element pairs (summed in a fixed order at the end)
+    f2 acc2[MC + NC];
 #pragma unroll
-    for (int i = 0; i < MC + NC; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < MC + NC; ++i) acc2[i] = 0ull;
 
     const int64_t r_begin = (int64_t)blockIdx.y * a.rows_per_chunk;
     const int64_t r_end = min(a.rows, r_begin + a.rows_per_chunk);
@@ -185,28 +216,33 @@ __global__ void __launch_bounds__(kThreads, BWD ? 3 : 4) grkan_kernel(const GrAr
                 if (rh >= r_end) break;
                 float ov[VEC];
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    const float x = xv[h][e];
-                    float P, dP, S, dS;
-                    horner_d<MC - 1>(ca, m1 - 1, x, P, dP);
-                    horner_d<NC>(cb, n, x, S, dS);
-                    const float iQ = __fdividef(1.0f, 1.0f + fabsf(S));
-                    const float phi = P * iQ;
+                for (int e = 0; e < VEC; e += 2) {
+                    const f2 x = pk2(xv[h][e], xv[h][e + 1]);
+                    f2 P, dP, S, dS;
+                    horner_d2<MC - 1>(ca, m1 - 1, x, P, dP);
+                    horner_d2<NC>(cb, n, x, S, dS);
+                    float s0, s1;
+                    unpk2(S, s0, s1);
+                    const f2 iQ = pk2(__fdividef(1.0f, 1.0f + fabsf(s0)), __fdividef(1.0f, 1.0f + fabsf(s1)));
+                    const f2 phi = mul2(P, iQ);
                     if (!BWD) {
-                        ov[e] = phi;
+                        unpk2(phi, ov[e], ov[e + 1]);
                         continue;
                     }
-                    const float sg = S > 0.0f ? 1.0f : (S < 0.0f ? -1.0f : 0.0f);
-                    const float ga = gv[h][e] * iQ;           // d phi / d a_p = x^p / Q
-                    ov[e] = ga * (dP - phi * sg * dS);
+                    // nps = -phi sign(S)
+                    float p0, p1;
+                    unpk2(phi, p0, p1);
+                    const f2 nps = pk2(s0 > 0.0f ? -p0 : (s0 < 0.0f ? p0 : 0.0f), s1 > 0.0f ? -p1 : (s1 < 0.0f ? p1 : 0.0f));
+                    const f2 ga = mul2(pk2(gv[h][e], gv[h][e + 1]), iQ);   // d phi / d a_p = x^p / Q
+                    unpk2(mul2(ga, fma2(nps, dS, dP)), ov[e], ov[e + 1]);
                     if (a.part) {
-                        const float gb = -ga * phi * sg;      // d phi / d b_q = -phi sign(S) x^q / Q
-                        float xp = 1.0f;
+                        const f2 gb = mul2(ga, nps);                     // d phi / d b_q = -phi sign(S) x^q / Q
+                        f2 xp = pk2(1.0f, 1.0f);
 #pragma unroll
                         for (int i = 0; i <= PW; ++i) {
-                            if (i < MC) acc[i] = fmaf(ga, xp, acc[i]);
-                            if (i >= 1 && i <= NC) acc[MC + i - 1] = fmaf(gb, xp, acc[MC + i - 1]);
-                            if (i < PW) xp *= x;
+                            if (i < MC) acc2[i] = fma2(ga, xp, acc2[i]);
+                            if (i >= 1 && i <= NC) acc2[MC + i - 1] = fma2(gb, xp, acc2[MC + i - 1]);
+                            if (i < PW) xp = mul2(xp, x);
                         }
                     }
                 }
@@ -215,6 +251,13 @@ __global__ void __launch_bounds__(kThreads, BWD ? 3 : 4) grkan_kernel(const GrAr
         }
     }
     if (!BWD || !a.part) return;
+    float acc[MC + NC];
+#pragma unroll
+    for (int i = 0; i < MC + NC; ++i) {
+        float lo, hi;
+        unpk2(acc2[i], lo, hi);
+        acc[i] = lo + hi;
+    }
     // block reduction in a fixed order: lanes by shuffles (inactive lanes hold zeros), then the
     // warps' sums in warp order; entries past the runtime counts are zero
     __shared__ float wsum[kThreads / 32][kAcc];
