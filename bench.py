@@ -130,8 +130,9 @@ def layer_bytes(batch, L, esz, call):
 
 
 def measured_counters(workload: str, call: str):
-    """The committed ncu figures of a call's main kernel (profiles/traffic.json): DRAM bytes per launch
-    and tensor-pipe activity, or None when there are none or the kernel sources changed since."""
+    """The committed ncu figures of a call's main kernel (profiles/traffic.json, keyed by segment: "fwd1",
+    "dcoef1", "dx1" for layer index 1, "bwd" for GR-KAN): DRAM bytes per launch and tensor-pipe activity,
+    or None when there are none or the kernel sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -377,7 +378,7 @@ def roofline_of(w: W.Workload, seg: dict, K: int, pk: dict, ffma_tflops: float):
     L = w.layers[li]
     avg_s = gemm[dom] / K / 1000.0
     dense = layer_dense_flops(w.batch, L)
-    counters = measured_counters(w.name, kind) or {}
+    counters = measured_counters(w.name, dom) or {}
     if w.dtype == "bf16":
         achieved = dense / avg_s / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
@@ -684,6 +685,7 @@ def time_grkan(w: W.GrWorkload, dev, K, flush, pk):
     out = {"ms_per_step": ms, "value": n / (ms / 1000.0), "unit": "elements/s", "steps": K, "dtype": w.dtype,
            "dominant": "bwd", "bound": "hbm", "achieved": gbs["bwd"], "peak": pk["hbm"], "peak_unit": "GB/s",
            "frac": gbs["bwd"] / pk["hbm"], "fwd_frac": gbs["fwd"] / pk["hbm"], "segment_ms": seg,
+           "traffic": (measured_counters(w.name, "bwd") or {}).get("dram_bytes"),
            "algorithmic_bytes_per_launch": bytes_,
            "step_roofline": {"t_roof_ms": (bytes_["fwd"] + bytes_["bwd"]) / (pk["hbm"] * 1e9) * 1000.0,
                              "frac": (bytes_["fwd"] + bytes_["bwd"]) / (pk["hbm"] * 1e9) * 1000.0 / ms,
