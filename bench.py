@@ -185,16 +185,27 @@ class Runner:
         self.h_x = self.h_dY = None
 
     def pin_host(self):
-        """Pinned host mirrors of the inputs and outputs (the end-to-end variant)."""
+        """Pinned host mirrors of the inputs and of the step's results (the end-to-end variant): the last
+        layer's y, the first layer's dx and every layer's dcoef (and dw_base); the activations and
+        gradients between the layers stay on the device."""
         self.h_x = self.host["x"].pin_memory()
         self.h_dY = self.host["dY"].pin_memory()
+        pin = lambda t: None if t is None else torch.empty_like(t, device="cpu").pin_memory()
+        last = len(self.layers) - 1
         self.h_out = []
-        for l in self.layers:
-            self.h_out.append(dict(y=torch.empty_like(l["y"], device="cpu").pin_memory(),
-                                   dx=torch.empty_like(l["dx"], device="cpu").pin_memory(),
-                                   dcoef=torch.empty_like(l["dcoef"], device="cpu").pin_memory(),
-                                   dwb=None if l["dwb"] is None else
-                                   torch.empty_like(l["dwb"], device="cpu").pin_memory()))
+        for li, l in enumerate(self.layers):
+            fwd_only = self.w.mode == "fwd"
+            self.h_out.append(dict(y=pin(l["y"]) if li == last else None,
+                                   dx=pin(l["dx"]) if li == 0 and not fwd_only else None,
+                                   dcoef=None if fwd_only else pin(l["dcoef"]),
+                                   dwb=None if fwd_only else pin(l["dwb"])))
+
+    def results_of(self, name):
+        """(host, device) pairs of the step's results that call `name` completes."""
+        kind, li = name.rstrip("0123456789"), int(name[len(name.rstrip("0123456789")):])
+        l, h = self.layers[li], self.h_out[li]
+        keys = ("y",) if kind == "fwd" else ("dx", "dcoef", "dwb")
+        return [(h[k], l[k]) for k in keys if h[k] is not None]
 
     def dy_of(self, li):
         return self.dY if li == len(self.layers) - 1 else self.layers[li + 1]["dx"]
@@ -238,14 +249,17 @@ class Runner:
             n += self.h_dY.numel() * self.h_dY.element_size()
         return n
 
-    def d2h(self):
+    def d2h_after(self, name, stream, copy_stream):
+        """Copy the results of call `name` to pinned host memory on the copy stream, once `stream` has
+        produced them (they leave while the next calls compute); returns the bytes copied."""
         n = 0
-        keys = ("y",) if self.w.mode == "fwd" else ("y", "dx", "dcoef", "dwb")
-        for l, h in zip(self.layers, self.h_out):
-            for k in keys:
-                if h[k] is not None:
-                    h[k].copy_(l[k], non_blocking=True)
-                    n += h[k].numel() * h[k].element_size()
+        pairs = self.results_of(name)
+        if pairs:
+            copy_stream.wait_stream(stream)
+            with torch.cuda.stream(copy_stream):
+                for h, d in pairs:
+                    h.copy_(d, non_blocking=True)
+                    n += h.numel() * h.element_size()
         return n
 
     def adjoint_errors(self):
@@ -793,15 +807,18 @@ def run_ours(args, world, rank, local):
         calls = R.calls()
         e2e_ev = [(_ev(), _ev()) for _ in range(K)]
         hb = db = 0
+        copy_stream = torch.cuda.Stream(dev)
         barrier()
         torch.cuda.synchronize(dev)
         for k in range(K):
             flush.zero_()
             e2e_ev[k][0].record(stream)
             hb = R.h2d()
-            for _, _, c in calls:
+            db = 0
+            for nm, _, c in calls:
                 c()
-            db = R.d2h()
+                db += R.d2h_after(nm, stream, copy_stream)
+            stream.wait_stream(copy_stream)   # the step ends when its results are on the host
             e2e_ev[k][1].record(stream)
         torch.cuda.synchronize(dev)
         barrier()
