@@ -151,6 +151,15 @@ def measured_traffic(workload: str, call: str):
 
 
 # ---------------------------------------------------------------------------
+def result_keys(li: int, n_layers: int, mode: str):
+    """The step's results among layer li's tensors (what the end-to-end variant copies to the host): the
+    last layer's y, the first layer's dx and every layer's dcoef and dw_base (without a backward, y only)."""
+    keys = ["y"] if li == n_layers - 1 else []
+    if mode != "fwd":
+        keys += (["dx"] if li == 0 else []) + ["dcoef", "dwb"]
+    return keys
+
+
 class Runner:
     """Pre-allocated buffers and the step's C-ABI calls for one workload.
 
@@ -191,14 +200,10 @@ class Runner:
         self.h_x = self.host["x"].pin_memory()
         self.h_dY = self.host["dY"].pin_memory()
         pin = lambda t: None if t is None else torch.empty_like(t, device="cpu").pin_memory()
-        last = len(self.layers) - 1
         self.h_out = []
         for li, l in enumerate(self.layers):
-            fwd_only = self.w.mode == "fwd"
-            self.h_out.append(dict(y=pin(l["y"]) if li == last else None,
-                                   dx=pin(l["dx"]) if li == 0 and not fwd_only else None,
-                                   dcoef=None if fwd_only else pin(l["dcoef"]),
-                                   dwb=None if fwd_only else pin(l["dwb"])))
+            keys = result_keys(li, len(self.layers), self.w.mode)
+            self.h_out.append({k: pin(l[k]) if k in keys else None for k in ("y", "dx", "dcoef", "dwb")})
 
     def results_of(self, name):
         """(host, device) pairs of the step's results that call `name` completes."""

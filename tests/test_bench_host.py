@@ -71,3 +71,12 @@ def test_traffic_lookup_follows_the_source_hash(tmp_path, monkeypatch):
     assert bench.measured_traffic("w", "fwd") is None
     os.remove(prof / "traffic.json")
     assert bench.measured_traffic("w", "fwd") is None
+
+
+def test_end_to_end_copies_only_the_steps_results():
+    # a two-layer block: y of the last layer, dx of the first, every layer's dcoef / dw_base
+    assert bench.result_keys(0, 2, "fwdbwd") == ["dx", "dcoef", "dwb"]
+    assert bench.result_keys(1, 2, "fwdbwd") == ["y", "dcoef", "dwb"]
+    assert bench.result_keys(0, 1, "fwdbwd") == ["y", "dx", "dcoef", "dwb"]
+    assert bench.result_keys(0, 1, "fwd") == ["y"]
+    assert bench.result_keys(0, 2, "fwd") == []
