@@ -347,6 +347,21 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Arrivals without release semantics, for signals that publish no memory data:
+// "this warp has read the accumulator into registers" (its tcgen05 loads have
+// completed, tcgen05.wait::ld, and tcgen05.fence::before_thread_sync precedes
+// the arrival).  A release at cluster scope would first wait for every earlier
+// global store of the thread to complete (measured ~0.9 us per arrival after
+// a tile's dx stores, on the critical path of the pair's epilogue).
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // try_wait with acquire at cluster scope (for barriers that CTAs of the pair arrive on).
 __device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity)
 {

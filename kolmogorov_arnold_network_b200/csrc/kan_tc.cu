@@ -869,8 +869,8 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
         // (they have nothing else to do before the accumulator is complete; the
         // fp32 epilogue promotes accumulator segments meanwhile).
         // Each thread fetches the x values of its next k-block into registers
-        // before it waits for and fills the current one, so the global-load
-        // latency overlaps the previous k-block's work.
+        // right after it has handed over the current one, so the global-load
+        // latency overlaps the other groups' k-blocks.
         const bool producer_warp = warp < Warps<MODE>::kEpi0;
         if constexpr (PRODUCE) if (producer_warp || !F32) {
             const int p = threadIdx.x - 64;
@@ -921,7 +921,6 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     float cur[MAXI];
                     const XWindow<T, MAXI> cur_raw = nxw;   // this k-block's window (the next one is fetched below)
                     const int kb = kb_begin + it;
-                    if (it + NG < nk) fetch(kb + NG);
                     const int s = it % sa_n;
                     const uint32_t ph = (it / sa_n) & 1;
                     // the slot is free (its previous use consumed)
@@ -1043,6 +1042,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     fence_async_smem();
                     if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(afull(s), 0));
                     else mbar_arrive(afull(s));
+                    // the group's next window, issued only now: a release arrival waits for
+                    // every earlier load of the thread, so loads in flight would delay it
+                    if (it + NG < nk) fetch(kb + NG);
                 }
                 (void)uses;
             } else if constexpr (MODE == DCA) {
@@ -1085,7 +1087,6 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     float cur[MAXI];
                     const XWindow<T, MAXI> cur_raw = nxw;   // this k-block's window (the next one is fetched below)
                     const int kb = kb_begin + it;
-                    if (it + NG < nk) fetch(kb + NG);
                     const int s = it % sa_n;
                     const uint32_t ph = (it / sa_n) & 1;
                     if (!acquire(s, ph)) break;
@@ -1250,6 +1251,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     fence_async_smem();
                     if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(afull(s), 0));
                     else mbar_arrive(afull(s));
+                    // the group's next window, issued only now: a release arrival waits for
+                    // every earlier load of the thread, so loads in flight would delay it
+                    if (it + NG < nk) fetch(kb + NG);
                 }
             } else if constexpr (MODE == DCB) {
                 // B tile, MN-major: batch rows b0..b0+BK-1 (K) by this CTA's bn_cta spline
@@ -1295,7 +1299,6 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                 for (int it = grp; grp < NG && it < nk; it += NG) {
                     const XWindow<T, MAXI> cur_raw[2] = {nxw[0], nxw[1]};
                     const int kb = kb_begin + it;
-                    if (it + NG < nk) fetch(kb + NG);
                     const int s = it % sa_n;
                     const uint32_t ph = (it / sa_n) & 1;
                     if (!acquire(s, ph)) break;
@@ -1347,6 +1350,9 @@ __global__ void __launch_bounds__(Warps<MODE>::kThreads, 1)
                     fence_async_smem();
                     if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(afull(s), 0));
                     else mbar_arrive(afull(s));
+                    // the group's next window, issued only now: a release arrival waits for
+                    // every earlier load of the thread, so loads in flight would delay it
+                    if (it + NG < nk) fetch(kb + NG);
                 }
             }
         }
@@ -2092,12 +2098,13 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                 }
             }
             // the accumulator buffer is free for the tile after next (one arrival per
-            // warp, on the leader's barrier for a pair)
+            // warp, on the leader's barrier for a pair; relaxed: it publishes no data, and
+            // a release would first wait for this warp's previous dx stores)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if (PAIR && !leader) mbar_arrive_cluster(mapa_shared(acc_empty(buf), 0));
-                else mbar_arrive(acc_empty(buf));
+                if (PAIR && !leader) mbar_arrive_cluster_relaxed(mapa_shared(acc_empty(buf), 0));
+                else mbar_arrive_relaxed(acc_empty(buf));
             }
             // both halves of the row are staged
             named_bar_sync(1 + q, 64);
