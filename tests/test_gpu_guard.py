@@ -61,7 +61,10 @@ class Guarded:
 CASES = [c + (3,) for c in SMALL] + [
     # other spline degrees: k+1 weights per input in the producers and the dx gather
     (300, 16, 256, 8, -1.0, 1.0, True, 1), (800, 24, 296, 20, -1.0, 1.0, False, 5),
-    (300, 40, 296, 8, -1.0, 1.0, False, 2), (257, 24, 64, 20, -1.0, 1.0, True, 4)]
+    (300, 40, 296, 8, -1.0, 1.0, False, 2), (257, 24, 64, 20, -1.0, 1.0, True, 4),
+    # bf16: dcoef with the outputs on M (DCB, TMA-stored), a ragged last M tile / a ragged last N tile and
+    # rows of x that are not 16-byte aligned
+    (300, 1536, 648, 5, -3.0, 3.0, False, 3), (257, 1532, 768, 5, -3.0, 3.0, False, 3)]
 
 
 @pytest.mark.parametrize("path", [N.KAN_PATH_TENSOR, N.KAN_PATH_SIMT], ids=["tensor", "simt"])
